@@ -1,0 +1,160 @@
+/*
+ * tam.h - C ABI of the B200 attention-mass top-k library (libtam.so).
+ *
+ * The method (arXiv 2606.07703, "How Much Dense Attention is Necessary?
+ * Oracle-Guided Sparse Prefill for Full/GQA Layers in Hybrid Long-Context
+ * Models"): for each query position of a causal GQA prefill layer, compute
+ * dense attention, average the per-head probabilities over all query heads
+ * into one token-mass row, keep the top-k tokens of that row (per query, or
+ * once for a block of consecutive queries), and recompute attention for every
+ * head only on that support, with the softmax renormalised over it
+ * (Abstract; gist.science technical report §2.1 "Der Attention-Mass Top-k
+ * Oracle").  A head-collapsed indexer picks the support from one shared
+ * low-dimensional score instead (report §2.2).
+ *
+ * Notation.  N query/key positions (batch 1, causal: query i sees keys j <= i),
+ * Hq query heads, Hkv KV heads (Hq % Hkv == 0), head dim d, G = Hq / Hkv.
+ * Query head h reads KV head g(h) = h / G (consecutive heads share a KV head).
+ * scale = 1/sqrt(d).
+ *
+ * Layouts (all row-major, contiguous, device memory unless stated):
+ *   q   [N, Hq, d]    element (i,h,c) at (i*Hq + h)*d + c
+ *   k,v [N, Hkv, d]   element (j,g,c) at (j*Hkv + g)*d + c
+ *   out [N, Hq, d]    same dtype as q
+ *   lse [Hq, N] fp32  natural-log sum of exp(scale * q.k) over the keys used
+ *   sup_idx  [n_sel, budget_k] int32, each row ascending, padded with -1
+ *   sup_len  [n_sel] int32,   sup_mass / sup_score [n_sel, budget_k] fp32 (0 in the padding)
+ *   n_sel = N for per-query support (block_q == 1), ceil(N / block_q) otherwise.
+ *
+ * dtype: TAM_BF16 (bf16 storage, fp32 accumulation; tensor cores) or TAM_F32
+ * (fp32 storage and arithmetic on CUDA cores).
+ *
+ * Ownership.  The caller allocates and frees every buffer, including the
+ * workspace; the library never allocates device memory.  Every launch goes to
+ * `stream` (a cudaStream_t; NULL = the legacy default stream) and the calls
+ * return right after enqueueing.
+ *
+ * Errors.  Argument errors are detected on the host before anything is
+ * enqueued and returned directly: TAM_ERR_INVALID_ARG (null pointer, bad
+ * shape, pointer not 16-byte aligned, k < 1, block_q < 1), TAM_ERR_UNSUPPORTED
+ * (d not 64/128, k > 4096, N*k >= 2^31, combination not built), TAM_ERR_WORKSPACE
+ * (ws_bytes below the size query).  A failed launch returns TAM_ERR_CUDA.
+ * Errors found on the device (a bounded wait that gave up, a candidate
+ * buffer that overflowed) are recorded in a status block at the start of the
+ * workspace and are read by tam_check_status.  No call traps and no call prints.
+ */
+#ifndef TAM_H
+#define TAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TAM_OK = 0,
+    TAM_ERR_INVALID_ARG = 1,
+    TAM_ERR_UNSUPPORTED = 2,
+    TAM_ERR_WORKSPACE = 3,
+    TAM_ERR_CUDA = 4,
+    TAM_ERR_TIMEOUT = 5,
+    TAM_ERR_OVERFLOW = 6
+} tam_status;
+
+typedef enum { TAM_BF16 = 0, TAM_F32 = 1 } tam_dtype;
+
+/* Library version as 10000*major + 100*minor + patch. */
+int tam_version(void);
+
+/* Human-readable name of a status code (static string; never NULL). */
+const char* tam_status_string(int status);
+
+/*
+ * Workspace bytes tam_mass_oracle_prefill needs for this problem (always a
+ * multiple of 256).  Returns 0 for arguments that the call would reject.
+ */
+size_t tam_mass_oracle_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
+                                 int block_q);
+
+/*
+ * The attention-mass top-k oracle for one causal GQA prefill layer
+ * (Abstract; technical report §2.1):
+ *   pass 1  lse[h,i]  = log sum_{j<=i} exp(scale * q[i,h].k[j,g(h)])
+ *   pass 2  P_i[j]    = (1/Hq) sum_h exp(scale * q[i,h].k[j,g(h)] - lse[h,i]),   j <= i
+ *           block_q == 1: S_i = top-min(k, i+1) of P_i                     (n_sel = N)
+ *           block_q  > 1: M_b[j] = sum_{i in block b, i >= j} P_i[j] for j <= e_b,
+ *                         e_b = min(N, (b+1)*block_q) - 1, S_b = top-min(k, e_b+1) of M_b
+ *           ranking: larger value first, equal values -> smaller index first;
+ *           sup_idx rows are written ascending, sup_mass holds P_i[j] (or M_b[j]).
+ *   pass 3  (only if out != NULL) for every head h of query i,
+ *           out[i,h] = sum_{j in T_i} softmax_{T_i}(scale * q[i,h].k[j,g(h)]) v[j,g(h)],
+ *           T_i = S_i (per query) or S_b intersected with [0, i] (block), output in q's dtype.
+ * lse may be NULL (then it lives in the workspace).  The N x N mass matrix is never
+ * written to memory.  budget_k in [1, 4096]; block_q in [1, N].
+ */
+int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
+                            const void* k, const void* v, int budget_k, int block_q,
+                            int32_t* sup_idx, int32_t* sup_len, float* sup_mass, float* lse,
+                            void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Pass 1 alone: per-head log-sum-exp of the causal scores, lse [Hq, N] fp32
+ * (technical report §2.1: the dense distribution each head's probabilities come from).
+ */
+size_t tam_attention_lse_workspace(int64_t N, int Hq, int Hkv, int d, int dtype);
+int tam_attention_lse(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
+                      float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Head-collapsed indexer support (technical report §2.2 "Head-Collapsed Indexer":
+ * one token score shared by all heads, top-k of it):
+ *   score[i,j] = q_idx[i] . k_idx[j] for j <= i (no scale: ranking only),
+ *   S_i = top-min(k, i+1) of score_i with the same ranking and output layout as above,
+ *   sup_score holds the scores of the chosen keys.
+ * q_idx, k_idx: [N, d_idx] in `dtype` (bf16 or fp32), d_idx in {16, 32, 64, 128}.
+ * block_q must be 1 (per-query support).
+ */
+size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int block_q);
+int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const void* k_idx,
+                     int budget_k, int block_q, int32_t* sup_idx, int32_t* sup_len,
+                     float* sup_score, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Pass 3 alone: attention recomputed on a given support (technical report §2.1,
+ * "Ausführung": original Q, K, V restricted to the selected tokens).
+ * block_q == 1: row i of sup_idx (first sup_len[i] entries) is query i's support.
+ * block_q  > 1: row b = i / block_q is shared by the block's queries; query i uses the
+ *               entries j <= i.  Entries < 0 or > i are skipped.  kmax = row stride of
+ *               sup_idx (>= every sup_len).  A query whose support is empty gets a zero
+ *               output row and lse = -inf.
+ */
+size_t tam_sparse_attention_workspace(int64_t N, int Hq, int Hkv, int d, int dtype);
+int tam_sparse_support_attention(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
+                                 const void* k, const void* v, const int32_t* sup_idx,
+                                 const int32_t* sup_len, int kmax, int block_q, void* out,
+                                 float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Dense causal GQA prefill (the FlashAttention-2 comparator the abstract measures
+ * against): out[i,h] = softmax_{j<=i}(scale * q[i,h].k[j,g(h)]) v[j,g(h)], lse optional.
+ */
+size_t tam_dense_workspace(int64_t N, int Hq, int Hkv, int d, int dtype);
+int tam_dense_gqa_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
+                          const void* k, const void* v, void* out, float* lse, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/*
+ * Waits for `stream`, then reads the device status block at the start of
+ * `workspace` that the last call using this workspace wrote.  Returns TAM_OK,
+ * TAM_ERR_TIMEOUT, TAM_ERR_OVERFLOW or TAM_ERR_CUDA.  `detail` (may be NULL)
+ * receives 8 int32 words: [0] status, [1] kernel id, [2..7] kernel-specific.
+ */
+int tam_check_status(const void* workspace, void* stream, int32_t* detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TAM_H */

@@ -1,0 +1,115 @@
+"""The C-ABI library loads, exports every symbol tam.h declares, and rejects bad
+arguments on the host before touching the GPU (no compute call runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tam.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tam_[a-z_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(tam_lib):
+    L = tam_lib.lib()
+    names = _declared()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(tam_lib.EXPORTED)
+
+
+def test_version_and_status_strings(tam_lib):
+    assert tam_lib.version() >= 100
+    for code in range(7):
+        assert tam_lib.status_string(code) != "unknown status"
+    assert tam_lib.status_string(99) == "unknown status"
+
+
+def test_workspace_queries(tam_lib):
+    L = tam_lib.lib()
+    ws = L.tam_mass_oracle_workspace(4096, 32, 8, 128, tam_lib.TAM_BF16, 256, 1)
+    assert ws > 0 and ws % 256 == 0
+    assert L.tam_mass_oracle_workspace(4096, 32, 8, 128, tam_lib.TAM_BF16, 256, 64) > 0
+    # rejected arguments give 0
+    assert L.tam_mass_oracle_workspace(4096, 30, 8, 128, 0, 256, 1) == 0      # Hq % Hkv
+    assert L.tam_mass_oracle_workspace(4096, 32, 8, 96, 0, 256, 1) == 0       # d
+    assert L.tam_mass_oracle_workspace(4096, 32, 8, 128, 0, 0, 1) == 0        # k < 1
+    assert L.tam_mass_oracle_workspace(4096, 32, 8, 128, 0, 5000, 1) == 0     # k > 4096
+    assert L.tam_mass_oracle_workspace(4096, 32, 8, 128, 0, 256, 0) == 0      # block_q < 1
+    assert L.tam_mass_oracle_workspace(4096, 32, 8, 128, 7, 256, 1) == 0      # dtype
+    assert L.tam_indexer_workspace(4096, 64, 0, 1024, 1) > 0
+    assert L.tam_indexer_workspace(4096, 48, 0, 1024, 1) == 0
+    for f in ("tam_attention_lse_workspace", "tam_sparse_attention_workspace",
+              "tam_dense_workspace"):
+        assert getattr(L, f)(4096, 32, 8, 128, 0) >= 256
+
+
+def _fake(addr=1 << 20):
+    return ctypes.c_void_p(addr)        # aligned, never dereferenced: calls fail validation first
+
+
+def test_host_side_argument_errors(tam_lib):
+    L = tam_lib.lib()
+    T = tam_lib
+    f = _fake()
+    # null pointers
+    rc = L.tam_mass_oracle_prefill(64, 4, 1, 64, 0, None, f, f, 8, 1, f, f, f, None, None, f,
+                                   1 << 30, None)
+    assert rc == T.TAM_ERR_INVALID_ARG
+    # misaligned pointer
+    rc = L.tam_mass_oracle_prefill(64, 4, 1, 64, 0, ctypes.c_void_p((1 << 20) + 2), f, f, 8, 1,
+                                   f, f, f, None, None, f, 1 << 30, None)
+    assert rc == T.TAM_ERR_INVALID_ARG
+    # bad shapes / budgets
+    assert L.tam_mass_oracle_prefill(64, 6, 4, 64, 0, f, f, f, 8, 1, f, f, f, None, None, f,
+                                     1 << 30, None) == T.TAM_ERR_INVALID_ARG
+    assert L.tam_mass_oracle_prefill(64, 4, 1, 80, 0, f, f, f, 8, 1, f, f, f, None, None, f,
+                                     1 << 30, None) == T.TAM_ERR_UNSUPPORTED
+    assert L.tam_mass_oracle_prefill(64, 4, 1, 64, 0, f, f, f, 0, 1, f, f, f, None, None, f,
+                                     1 << 30, None) == T.TAM_ERR_INVALID_ARG
+    assert L.tam_mass_oracle_prefill(64, 4, 1, 64, 0, f, f, f, 8192, 1, f, f, f, None, None, f,
+                                     1 << 30, None) == T.TAM_ERR_UNSUPPORTED
+    assert L.tam_mass_oracle_prefill(64, 4, 1, 64, 0, f, f, f, 8, 0, f, f, f, None, None, f,
+                                     1 << 30, None) == T.TAM_ERR_INVALID_ARG
+    # N * k >= 2^31
+    assert L.tam_mass_oracle_prefill(1 << 21, 4, 1, 64, 0, f, f, f, 1024, 1, f, f, f, None, None,
+                                     f, 1 << 40, None) == T.TAM_ERR_UNSUPPORTED
+    # workspace too small
+    assert L.tam_mass_oracle_prefill(64, 4, 1, 64, 0, f, f, f, 8, 1, f, f, f, None, None, f, 16,
+                                     None) == T.TAM_ERR_WORKSPACE
+    assert L.tam_indexer_topk(64, 64, 0, f, f, 8, 2, f, f, f, f, 1 << 30,
+                              None) == T.TAM_ERR_UNSUPPORTED          # block-shared indexer
+    assert L.tam_indexer_topk(64, 40, 0, f, f, 8, 1, f, f, f, f, 1 << 30,
+                              None) == T.TAM_ERR_UNSUPPORTED
+    assert L.tam_sparse_support_attention(64, 4, 1, 64, 0, f, f, f, None, f, 8, 1, f, None, f,
+                                          1 << 20, None) == T.TAM_ERR_INVALID_ARG
+    assert L.tam_dense_gqa_prefill(64, 4, 1, 64, 0, f, f, f, f, None, f, 8,
+                                   None) == T.TAM_ERR_WORKSPACE
+    assert L.tam_attention_lse(64, 4, 1, 64, 0, f, f, None, f, 256, None) == T.TAM_ERR_INVALID_ARG
+    assert L.tam_check_status(None, None, None) == T.TAM_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    """With libtam.so absent the binding raises instead of computing anything elsewhere."""
+    import top_attention_mass_b200 as tam
+    monkeypatch.setattr(tam, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(tam, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        tam.lib()
+
+
+def test_product_does_not_import_the_oracle():
+    """Nothing in the package refers to the oracle."""
+    pkg = os.path.join(ROOT, "top_attention_mass_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                txt = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, fn
+                assert "liboracle" not in txt and "orc_" not in txt, fn

@@ -1,0 +1,75 @@
+// Internal launcher interface between the C ABI (tam_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace tam {
+
+struct LseArgs {
+    int64_t N;
+    int Hq, Hkv, d, dtype;
+    const void* q;
+    const void* k;
+    float sl2;            // scale * log2(e)
+    float* lse;           // [Hq, N] natural log
+    int32_t* status;
+};
+
+struct MassArgs {
+    int64_t N;
+    int Hq, Hkv, d, dtype;
+    const void* q;
+    const void* k;
+    const float* lse;     // [Hq, N] from pass 1
+    float sl2;
+    int budget, block_q, n_sel;
+    int n_ctas;           // persistent blocks (CUDA-core path)
+    float* scratch;       // n_ctas * N floats (CUDA-core path)
+    void* cand;           // candidate buffers (tensor-core path)
+    int cand_cap;         // entries per query row in `cand`
+    int32_t* sup_idx;
+    int32_t* sup_len;
+    float* sup_mass;
+    int32_t* status;
+};
+
+struct AttnArgs {
+    int64_t N;
+    int Hq, Hkv, d, dtype;
+    const void* q;
+    const void* k;
+    const void* v;
+    float sl2;
+    const int32_t* sup_idx;   // null = dense causal
+    const int32_t* sup_len;
+    int kmax, block_q;
+    void* out;
+    float* lse;
+    int32_t* status;
+};
+
+struct IndexerArgs {
+    int64_t N;
+    int d_idx, dtype;
+    const void* q_idx;
+    const void* k_idx;
+    int budget;
+    int n_ctas;
+    float* scratch;
+    void* cand;
+    int cand_cap;
+    int32_t* sup_idx;
+    int32_t* sup_len;
+    float* sup_score;
+    int32_t* status;
+};
+
+// CUDA-core kernels (any dtype, any supported shape).
+cudaError_t simt_lse(const LseArgs& a, cudaStream_t st);
+cudaError_t simt_mass_select(const MassArgs& a, cudaStream_t st);
+cudaError_t simt_attention(const AttnArgs& a, cudaStream_t st);
+cudaError_t simt_indexer_select(const IndexerArgs& a, cudaStream_t st);
+
+}  // namespace tam

@@ -1,0 +1,258 @@
+// C ABI of libtam.so: argument checks, workspace layout and kernel dispatch.
+// Declarations and their contracts: include/tam.h.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "launch.h"
+
+using namespace tam;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxBudget = 4096;
+constexpr int kSimtPersistentCtas = 1024;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by every attention-shaped call.
+int check_shape(int64_t N, int Hq, int Hkv, int d, int dtype) {
+    if (N < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TAM_ERR_INVALID_ARG;
+    if (dtype != TAM_BF16 && dtype != TAM_F32) return TAM_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return TAM_ERR_UNSUPPORTED;
+    if (N >= (int64_t(1) << 31) - 1) return TAM_ERR_UNSUPPORTED;
+    // the CUDA-core kernels stage one query row (all heads) in shared memory
+    if ((size_t)(Hq * d + Hq) * sizeof(float) > 200 * 1024) return TAM_ERR_UNSUPPORTED;
+    return TAM_OK;
+}
+
+int check_budget(int64_t N, int budget_k, int block_q) {
+    if (budget_k < 1 || block_q < 1) return TAM_ERR_INVALID_ARG;
+    if (budget_k > kMaxBudget) return TAM_ERR_UNSUPPORTED;
+    if (N * (int64_t)budget_k >= (int64_t(1) << 31)) return TAM_ERR_UNSUPPORTED;
+    return TAM_OK;
+}
+
+inline int64_t n_selection_units(int64_t N, int block_q) {
+    return block_q == 1 ? N : (N + block_q - 1) / block_q;
+}
+
+// Workspace layout of tam_mass_oracle_prefill.
+struct MassPlan {
+    size_t off_lse, off_scratch, total;
+    int n_ctas;
+};
+
+MassPlan plan_mass(int64_t N, int Hq, int block_q) {
+    MassPlan p;
+    const int64_t n_sel = n_selection_units(N, block_q);
+    p.n_ctas = (int)std::min<int64_t>(n_sel, kSimtPersistentCtas);
+    p.off_lse = kStatusBytes;
+    p.off_scratch = p.off_lse + align256((size_t)Hq * N * sizeof(float));
+    p.total = p.off_scratch + align256((size_t)p.n_ctas * N * sizeof(float));
+    return p;
+}
+
+struct IndexerPlan {
+    size_t off_scratch, total;
+    int n_ctas;
+};
+
+IndexerPlan plan_indexer(int64_t N) {
+    IndexerPlan p;
+    p.n_ctas = (int)std::min<int64_t>(N, kSimtPersistentCtas);
+    p.off_scratch = kStatusBytes;
+    p.total = p.off_scratch + align256((size_t)p.n_ctas * N * sizeof(float));
+    return p;
+}
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? TAM_OK : TAM_ERR_CUDA; }
+
+inline float score_log2_scale(int d) { return (float)(1.0 / std::sqrt((double)d)) * kLog2e; }
+
+int start_call(void* workspace, cudaStream_t st) {
+    return cuda_status(cudaMemsetAsync(workspace, 0, kStatusBytes, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int tam_version(void) { return kVersion; }
+
+const char* tam_status_string(int s) {
+    switch (s) {
+        case TAM_OK: return "ok";
+        case TAM_ERR_INVALID_ARG: return "invalid argument";
+        case TAM_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case TAM_ERR_WORKSPACE: return "workspace too small";
+        case TAM_ERR_CUDA: return "CUDA error";
+        case TAM_ERR_TIMEOUT: return "device wait timed out";
+        case TAM_ERR_OVERFLOW: return "candidate buffer overflow";
+        default: return "unknown status";
+    }
+}
+
+size_t tam_mass_oracle_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
+                                 int block_q) {
+    if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK) return 0;
+    if (check_budget(N, budget_k, block_q) != TAM_OK) return 0;
+    return plan_mass(N, Hq, block_q).total;
+}
+
+int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
+                            const void* k, const void* v, int budget_k, int block_q,
+                            int32_t* sup_idx, int32_t* sup_len, float* sup_mass, float* lse,
+                            void* out, void* workspace, size_t ws_bytes, void* stream) {
+    int rc = check_shape(N, Hq, Hkv, d, dtype);
+    if (rc) return rc;
+    rc = check_budget(N, budget_k, block_q);
+    if (rc) return rc;
+    if (!q || !k || !sup_idx || !sup_len || !sup_mass || !workspace) return TAM_ERR_INVALID_ARG;
+    if (out && !v) return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, sup_idx, sup_len, sup_mass, lse, out, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return TAM_ERR_INVALID_ARG;
+    const MassPlan plan = plan_mass(N, Hq, block_q);
+    if (ws_bytes < plan.total) return TAM_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    int32_t* status = (int32_t*)ws;
+    float* lse_buf = lse ? lse : (float*)(ws + plan.off_lse);
+    if ((rc = start_call(workspace, st))) return rc;
+
+    const float sl2 = score_log2_scale(d);
+    LseArgs la{N, Hq, Hkv, d, dtype, q, k, sl2, lse_buf, status};
+    if ((rc = cuda_status(simt_lse(la, st)))) return rc;
+
+    MassArgs ma{};
+    ma.N = N; ma.Hq = Hq; ma.Hkv = Hkv; ma.d = d; ma.dtype = dtype;
+    ma.q = q; ma.k = k; ma.lse = lse_buf; ma.sl2 = sl2;
+    ma.budget = budget_k; ma.block_q = block_q; ma.n_sel = (int)n_selection_units(N, block_q);
+    ma.n_ctas = plan.n_ctas; ma.scratch = (float*)(ws + plan.off_scratch);
+    ma.sup_idx = sup_idx; ma.sup_len = sup_len; ma.sup_mass = sup_mass; ma.status = status;
+    if ((rc = cuda_status(simt_mass_select(ma, st)))) return rc;
+
+    if (out) {
+        AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, sl2, sup_idx, sup_len, budget_k, block_q,
+                    out, nullptr, status};
+        if ((rc = cuda_status(simt_attention(aa, st)))) return rc;
+    }
+    return TAM_OK;
+}
+
+size_t tam_attention_lse_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {
+    if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK) return 0;
+    return kStatusBytes;
+}
+
+int tam_attention_lse(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
+                      float* lse, void* workspace, size_t ws_bytes, void* stream) {
+    int rc = check_shape(N, Hq, Hkv, d, dtype);
+    if (rc) return rc;
+    if (!q || !k || !lse || !workspace) return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, lse, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
+    if (ws_bytes < kStatusBytes) return TAM_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((rc = start_call(workspace, st))) return rc;
+    LseArgs la{N, Hq, Hkv, d, dtype, q, k, score_log2_scale(d), lse, (int32_t*)workspace};
+    return cuda_status(simt_lse(la, st));
+}
+
+size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
+    if (N < 1 || (d_idx != 16 && d_idx != 32 && d_idx != 64 && d_idx != 128)) return 0;
+    if (dtype != TAM_BF16 && dtype != TAM_F32) return 0;
+    if (check_budget(N, budget_k, block_q) != TAM_OK || block_q != 1) return 0;
+    return plan_indexer(N).total;
+}
+
+int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const void* k_idx,
+                     int budget_k, int block_q, int32_t* sup_idx, int32_t* sup_len,
+                     float* sup_score, void* workspace, size_t ws_bytes, void* stream) {
+    if (N < 1 || d_idx < 1 || (dtype != TAM_BF16 && dtype != TAM_F32)) return TAM_ERR_INVALID_ARG;
+    if (d_idx != 16 && d_idx != 32 && d_idx != 64 && d_idx != 128) return TAM_ERR_UNSUPPORTED;
+    if (N >= (int64_t(1) << 31) - 1) return TAM_ERR_UNSUPPORTED;
+    int rc = check_budget(N, budget_k, block_q);
+    if (rc) return rc;
+    if (block_q != 1) return TAM_ERR_UNSUPPORTED;
+    if (!q_idx || !k_idx || !sup_idx || !sup_len || !sup_score || !workspace)
+        return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q_idx, k_idx, sup_idx, sup_len, sup_score, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
+    const IndexerPlan plan = plan_indexer(N);
+    if (ws_bytes < plan.total) return TAM_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    if ((rc = start_call(workspace, st))) return rc;
+    IndexerArgs ia{};
+    ia.N = N; ia.d_idx = d_idx; ia.dtype = dtype; ia.q_idx = q_idx; ia.k_idx = k_idx;
+    ia.budget = budget_k; ia.n_ctas = plan.n_ctas; ia.scratch = (float*)(ws + plan.off_scratch);
+    ia.sup_idx = sup_idx; ia.sup_len = sup_len; ia.sup_score = sup_score;
+    ia.status = (int32_t*)ws;
+    return cuda_status(simt_indexer_select(ia, st));
+}
+
+size_t tam_sparse_attention_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {
+    if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK) return 0;
+    return kStatusBytes;
+}
+
+int tam_sparse_support_attention(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
+                                 const void* k, const void* v, const int32_t* sup_idx,
+                                 const int32_t* sup_len, int kmax, int block_q, void* out,
+                                 float* lse, void* workspace, size_t ws_bytes, void* stream) {
+    int rc = check_shape(N, Hq, Hkv, d, dtype);
+    if (rc) return rc;
+    rc = check_budget(N, kmax, block_q);
+    if (rc) return rc;
+    if (!q || !k || !v || !sup_idx || !sup_len || !out || !workspace) return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, sup_idx, sup_len, out, lse, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return TAM_ERR_INVALID_ARG;
+    if (ws_bytes < kStatusBytes) return TAM_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((rc = start_call(workspace, st))) return rc;
+    AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, score_log2_scale(d), sup_idx, sup_len, kmax,
+                block_q, out, lse, (int32_t*)workspace};
+    return cuda_status(simt_attention(aa, st));
+}
+
+size_t tam_dense_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {
+    if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK) return 0;
+    return kStatusBytes;
+}
+
+int tam_dense_gqa_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
+                          const void* k, const void* v, void* out, float* lse, void* workspace,
+                          size_t ws_bytes, void* stream) {
+    int rc = check_shape(N, Hq, Hkv, d, dtype);
+    if (rc) return rc;
+    if (!q || !k || !v || !out || !workspace) return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, out, lse, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return TAM_ERR_INVALID_ARG;
+    if (ws_bytes < kStatusBytes) return TAM_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((rc = start_call(workspace, st))) return rc;
+    AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, score_log2_scale(d), nullptr, nullptr, 0, 1,
+                out, lse, (int32_t*)workspace};
+    return cuda_status(simt_attention(aa, st));
+}
+
+int tam_check_status(const void* workspace, void* stream, int32_t* detail) {
+    if (!workspace) return TAM_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return TAM_ERR_CUDA;
+    int32_t w[8];
+    if (cudaMemcpy(w, workspace, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return TAM_ERR_CUDA;
+    if (detail) std::memcpy(detail, w, sizeof(w));
+    return w[0];
+}
+
+}  // extern "C"
