@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the attention-mass top-k path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of every step of the hot path over one layer of the 32K
+workload (N=32768, Hq=32, Hkv=8, d=128, bf16; sink at token 0, 64 planted
+needles):
+  pass 1  per-head LSE                            (attention_lse)
+  pass 2  mass + per-query top-k, k=655           (mass_select, block_q=1)
+  pass 3  per-query gathered sparse attention     (sparse_support_attention)
+  pass 2  mass + block-shared top-k, B_q=64       (mass_select, block_q=64)
+  pass 3  block-shared sparse attention           (sparse_support_attention)
+  indexer top-k, d_idx=64, k=1024                 (indexer_topk)
+  pass 3  on the indexer support                  (sparse_support_attention)
+  dense causal GQA prefill (comparator)           (dense_gqa_prefill)
+value = query tokens of all ranks / step time (max over ranks).  With N > 1 GPUs
+every rank runs an independent replica of the workload (weak scaling, no
+collective on the data path).  `--impl reference` times the fp64 CPU oracle on a
+bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import tam_synth  # noqa: E402
+
+METRIC = "query-tokens/s per GQA layer (mass-oracle, sparse pass) at 32K; % of roofline"
+UNIT = "q-tok/s"
+WORKLOAD = "gqa32k_2pct"
+BLOCK_Q = 64
+INDEXER_K = 1024
+D_IDX = 64
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def causal_pairs(N: int) -> int:
+    return N * (N + 1) // 2
+
+
+def support_pairs(N: int, k: int) -> int:
+    i = np.arange(N, dtype=np.int64)
+    return int(np.minimum(k, i + 1).sum())
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.device = device
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            target = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            target = str(self.device)
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", target, f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1].split()[0]))
+                    smax.append(float(parts[2].split()[0]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ the device step
+
+class Step:
+    """All rows of the hot path on device-resident inputs; CUDA events between calls."""
+
+    NAMES = ("pass1_lse", "pass2_mass_topk", "pass3_gather", "pass2_block_mass_topk",
+             "pass3_block", "indexer_topk", "pass3_indexer_support", "dense_prefill")
+
+    def __init__(self, tam, w, q, k, v, qx, kx):
+        self.tam, self.w = tam, w
+        self.q, self.k, self.v, self.qx, self.kx = q, k, v, qx, kx
+        self.ws = tam.Workspace(q.device)
+        self.outputs = {}
+
+    def run(self, events=None):
+        t, w = self.tam, self.w
+        ev = events or [None] * 9
+
+        def mark(n):
+            if ev[n] is not None:
+                ev[n].record()
+        mark(0)
+        lse = t.attention_lse(self.q, self.k, workspace=self.ws, check=False)
+        mark(1)
+        s1 = t.mass_select(self.q, self.k, lse, w.budget_k, 1, workspace=self.ws, check=False)
+        mark(2)
+        o1 = t.sparse_support_attention(self.q, self.k, self.v, s1.idx, s1.length, 1,
+                                        workspace=self.ws, check=False)
+        mark(3)
+        s2 = t.mass_select(self.q, self.k, lse, w.budget_k, BLOCK_Q, workspace=self.ws,
+                           check=False)
+        mark(4)
+        o2 = t.sparse_support_attention(self.q, self.k, self.v, s2.idx, s2.length, BLOCK_Q,
+                                        workspace=self.ws, check=False)
+        mark(5)
+        s3 = t.indexer_topk(self.qx, self.kx, INDEXER_K, workspace=self.ws, check=False)
+        mark(6)
+        o3 = t.sparse_support_attention(self.q, self.k, self.v, s3.idx, s3.length, 1,
+                                        workspace=self.ws, check=False)
+        mark(7)
+        od = t.dense_gqa_prefill(self.q, self.k, self.v, workspace=self.ws, check=False)
+        mark(8)
+        self.outputs = {"lse": lse, "s1_idx": s1.idx, "s1_len": s1.length, "s1_mass": s1.value,
+                        "o1": o1, "s2_idx": s2.idx, "s2_len": s2.length, "s2_mass": s2.value,
+                        "o2": o2, "s3_idx": s3.idx, "s3_len": s3.length, "s3_score": s3.value,
+                        "o3": o3, "od": od}
+        return self.outputs
+
+
+def algorithmic_work(w, N, outs):
+    """Per-row algorithmic flops/bytes (what the method must do, not what it avoids)."""
+    Hq, Hkv, d = w.Hq, w.Hkv, w.d
+    elt = 2
+    cp = causal_pairs(N)
+    qo = 2 * N * Hq * d * elt                         # read Q, write O
+    sp1 = support_pairs(N, w.budget_k)
+    sp3 = support_pairs(N, INDEXER_K)
+    # block-shared: gathered rows per block and attended pairs per query (from the supports)
+    s2_len = outs["s2_len"].cpu().numpy().astype(np.int64)
+    s2_idx = outs["s2_idx"].cpu().numpy()
+    nb = len(s2_len)
+    blk_rows = int(s2_len.sum())
+    attended = 0
+    for b in range(nb):
+        sel = np.sort(s2_idx[b, :s2_len[b]])
+        i0, i1 = b * BLOCK_Q, min(N, (b + 1) * BLOCK_Q)
+        rows = np.arange(i0, i1)
+        attended += int(np.searchsorted(sel, rows, side="right").sum())
+    gather = lambda pairs: pairs * Hkv * 2 * d * elt  # noqa: E731  K and V rows of every group
+    return {
+        "pass1_lse": {"bound": "tensor", "flops": 2.0 * d * Hq * cp},
+        "pass2_mass_topk": {"bound": "tensor", "flops": 2.0 * d * Hq * cp},
+        "pass3_gather": {"bound": "hbm",
+                         "bytes": float(gather(sp1) + qo + N * w.budget_k * 4 + N * 4)},
+        "pass2_block_mass_topk": {"bound": "tensor", "flops": 2.0 * d * Hq * cp},
+        "pass3_block": {"bound": "hbm", "bytes": float(gather(blk_rows) + qo + nb * w.budget_k * 4),
+                        "flops": 4.0 * d * Hq * attended},
+        "indexer_topk": {"bound": "tensor", "flops": 2.0 * D_IDX * cp},
+        "pass3_indexer_support": {"bound": "hbm",
+                                  "bytes": float(gather(sp3) + qo + N * INDEXER_K * 4 + N * 4)},
+        "dense_prefill": {"bound": "tensor", "flops": 4.0 * d * Hq * cp},
+    }
+
+
+def roofline_of(work, ms, pk, pk_kind):
+    tf_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    if work["bound"] == "tensor":
+        ach = work["flops"] / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": tf_peak, "unit": "TFLOP/s",
+                "frac": ach / tf_peak, "traffic": None,
+                "peak_kind": f"bf16 dense, sustained, of {pk_kind}"}
+    ach = work["bytes"] / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_kind": f"HBM copy, of {pk_kind}"}
+
+
+# ------------------------------------------------------------------ oracle (CPU) arm
+
+def oracle_sample_step(inp, w, n_rows: int):
+    """The fp64 oracle on a bounded, stratified sample of the step; returns the time it
+    would take for the whole step, extrapolated by each part's per-row work."""
+    import oracle
+    N = w.N
+    rows = np.array([int((m + 0.5) * N / n_rows) for m in range(n_rows)], dtype=np.int64)
+    wr = (rows + 1).astype(np.float64)
+    w_all = float(causal_pairs(N))
+    kq = np.minimum(w.budget_k, rows + 1).astype(np.float64)
+    kq_all = float(support_pairs(N, w.budget_k))
+    ki = np.minimum(INDEXER_K, rows + 1).astype(np.float64)
+    ki_all = float(support_pairs(N, INDEXER_K))
+    total = 0.0
+    # pass 1 + pass 2 per query (LSE and mass are computed inside the selection)
+    t0 = time.perf_counter()
+    idx, ln, _ = oracle.topk_rows(inp.q, inp.k, w.budget_k, rows)
+    t1 = time.perf_counter()
+    oracle.attn_rows(inp.q, inp.k, inp.v, rows, sup=idx, sup_len=ln)
+    t2 = time.perf_counter()
+    total += (t1 - t0) * w_all / wr.sum() + (t2 - t1) * kq_all / kq.sum()
+    # block-shared: one block in the middle
+    nb = -(-N // BLOCK_Q)
+    b = nb // 2
+    brows = np.arange(b * BLOCK_Q, min(N, (b + 1) * BLOCK_Q))
+    t0 = time.perf_counter()
+    bidx, bln, _ = oracle.block_topk(inp.q, inp.k, BLOCK_Q, w.budget_k, [b])
+    t1 = time.perf_counter()
+    r, s, sl = oracle.block_rows_support(bidx, bln, BLOCK_Q, N, [b])
+    oracle.attn_rows(inp.q, inp.k, inp.v, r, sup=s, sup_len=sl)
+    t2 = time.perf_counter()
+    total += (t1 - t0) * w_all / float((brows + 1).sum()) + (t2 - t1) * nb
+    # indexer
+    t0 = time.perf_counter()
+    xidx, xln, _ = oracle.indexer_topk_rows(inp.q_idx, inp.k_idx, INDEXER_K, rows)
+    t1 = time.perf_counter()
+    oracle.attn_rows(inp.q, inp.k, inp.v, rows, sup=xidx, sup_len=xln)
+    t2 = time.perf_counter()
+    total += (t1 - t0) * w_all / wr.sum() + (t2 - t1) * ki_all / ki.sum()
+    # dense
+    t0 = time.perf_counter()
+    oracle.attn_rows(inp.q, inp.k, inp.v, rows)
+    t1 = time.perf_counter()
+    total += (t1 - t0) * w_all / wr.sum()
+    return total
+
+
+def calibrate_rows(inp, w, target_s: float):
+    t0 = time.perf_counter()
+    oracle_sample_step(inp, w, 4)
+    dt = time.perf_counter() - t0
+    return int(max(4, min(256, round(4 * target_s / max(dt, 1e-3)))))
+
+
+def cpu_sample_desc(n_rows):
+    return (f"{n_rows} stratified query rows (plus one block of {BLOCK_Q}) of the "
+            f"{WORKLOAD} workload through every step; time extrapolated to all rows by "
+            "per-row work ((i+1) for scoring, min(k, i+1) for the sparse recompute)")
+
+
+def run_reference(args, w, inp, rank, world):
+    import oracle
+    if rank != 0:
+        return
+    n_rows = calibrate_rows(inp, w, 6.0)
+    for _ in range(args.warmup):
+        oracle_sample_step(inp, w, n_rows)
+    ext = [oracle_sample_step(inp, w, n_rows) for _ in range(args.steps)]
+    ms = 1e3 * statistics.mean(ext)
+    value = w.N / (ms * 1e-3)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; stands in for the pages' 4K-100K long-context evaluations)",
+        "config": config_dict(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                         "sample": cpu_sample_desc(n_rows)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w, world):
+    return {"workload": WORKLOAD, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            "budget_k": w.budget_k, "block_q": BLOCK_Q, "indexer_k": INDEXER_K, "d_idx": D_IDX,
+            "global_batch": world, "seq_len": w.N,
+            "parallelism": f"replicas x{world} (independent layers, no collective)",
+            "l2": "256 MB buffer written before every step (L2 is 126 MB)"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, w, inp, rank, world, local_rank):
+    import top_attention_mass_b200 as tam
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    qx, kx = inp.q_idx.to(dev), inp.k_idx.to(dev)
+    step = Step(tam, w, q, k, v, qx, kx)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    for _ in range(args.warmup):
+        step.run()
+    tam.check_status(step.ws.get(256))
+    torch.cuda.synchronize()
+    work = algorithmic_work(w, w.N, step.outputs)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    barrier(world, local_rank)
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = tam.kernel_launches()
+    t_start.record()
+    for s in range(args.steps):
+        flush.fill_(s & 0xff)
+        step.run(ev[s])
+    t_stop.record()
+    torch.cuda.synchronize()
+    launches = tam.kernel_launches() - launches0
+    barrier(world, local_rank)
+    clk = clocks.stop()
+    tam.check_status(step.ws.get(256))
+    total_ms = t_start.elapsed_time(t_stop)
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_step = total_ms / args.steps
+    row_ms = {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps))
+              for i, n in enumerate(Step.NAMES)}
+
+    pk, pk_kind = peaks()
+    rows = {}
+    for n in Step.NAMES:
+        r = roofline_of(work[n], row_ms[n], pk, pk_kind)
+        rows[n] = {"ms": row_ms[n], "q_tok_s": w.N / (row_ms[n] * 1e-3), "roofline": r}
+    dominant = max(Step.NAMES, key=lambda n: row_ms[n])
+
+    e2e = measure_e2e(args, tam, w, inp, dev, world, local_rank)
+
+    if rank != 0:
+        return
+    value = world * w.N / (ms_step * 1e-3)
+    oracle_sparsity = 1.0 - support_pairs(w.N, w.budget_k) / causal_pairs(w.N)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; stands in for the pages' 4K-100K long-context evaluations)",
+        "config": config_dict(w, world),
+        "roofline": {**rows[dominant]["roofline"], "kernel": dominant},
+        "rows": rows,
+        "sparse_pass": {
+            "per_query_q_tok_s": w.N / (row_ms["pass3_gather"] * 1e-3),
+            "speedup_vs_dense": row_ms["dense_prefill"] / row_ms["pass3_gather"],
+            "block_shared_speedup_vs_dense": row_ms["dense_prefill"] / row_ms["pass3_block"],
+            "indexer_support_speedup_vs_dense":
+                row_ms["dense_prefill"] / row_ms["pass3_indexer_support"],
+            "oracle_pass12_plus3_q_tok_s": w.N / 1e-3 / (row_ms["pass1_lse"]
+                                                         + row_ms["pass2_mass_topk"]
+                                                         + row_ms["pass3_gather"]),
+        },
+        "sparsity_selfcheck": {
+            "this_workload": oracle_sparsity,
+            "N4096_k256": 1.0 - support_pairs(4096, 256) / causal_pairs(4096),
+            "N102400_k2048": 1.0 - support_pairs(102400, 2048) / causal_pairs(102400),
+        },
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": launches,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        n_rows = calibrate_rows(inp, w, 15.0)
+        t = oracle_sample_step(inp, w, n_rows)
+        line["cpu_baseline"] = {"value": w.N / t, "unit": UNIT, "cores": oracle.threads(),
+                                "kind": "oracle", "sample": cpu_sample_desc(n_rows)}
+    print(json.dumps(line), flush=True)
+
+
+def measure_e2e(args, tam, w, inp, dev, world, local_rank):
+    """Same step through the public API with pinned host inputs and results."""
+    if args.no_e2e:
+        return None
+    host_in = [inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory(),
+               inp.q_idx.pin_memory(), inp.k_idx.pin_memory()]
+    dev_in = [torch.empty_like(t, device=dev) for t in host_in]
+    step = Step(tam, w, *dev_in)
+    for t_d, t_h in zip(dev_in, host_in):
+        t_d.copy_(t_h)
+    outs = step.run()
+    host_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in outs.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    n = max(1, min(args.steps, 3))
+    barrier(world, local_rank)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        for t_d, t_h in zip(dev_in, host_in):
+            t_d.copy_(t_h, non_blocking=True)
+        outs = step.run()
+        for name, t in outs.items():
+            host_out[name].copy_(t, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world, local_rank)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n
+    return {"value": world * w.N / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n}
+
+
+# ------------------------------------------------------------------ process group plumbing
+
+def barrier(world, local_rank):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local_rank])
+
+
+def max_over_ranks(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = tam_synth.WORKLOADS["indexer32k"]          # the 32K layer plus its indexer head
+    w = tam_synth.Workload(**{**w.__dict__, "name": WORKLOAD, "budget_k": 655})
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        inp = tam_synth.make_inputs(w)
+        run_reference(args, w, inp, rank, world)
+        return
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    inp = tam_synth.make_inputs(w)
+    try:
+        run_ours(args, w, inp, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -108,6 +108,18 @@ int tam_attention_lse(int64_t N, int Hq, int Hkv, int d, int dtype, const void* 
                       float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Pass 2 alone: head-averaged mass and its top-k support, given pass 1's lse [Hq, N]
+ * (technical report §2.1, "Selektion" and "Granularität").  Same support semantics,
+ * ranking and output layout as tam_mass_oracle_prefill; lse is read, not written.
+ */
+size_t tam_mass_select_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
+                                 int block_q);
+int tam_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
+                    const float* lse, int budget_k, int block_q, int32_t* sup_idx,
+                    int32_t* sup_len, float* sup_mass, void* workspace, size_t ws_bytes,
+                    void* stream);
+
+/*
  * Head-collapsed indexer support (technical report §2.2 "Head-Collapsed Indexer":
  * one token score shared by all heads, top-k of it):
  *   score[i,j] = q_idx[i] . k_idx[j] for j <= i (no scale: ranking only),
@@ -144,6 +156,12 @@ size_t tam_dense_workspace(int64_t N, int Hq, int Hkv, int d, int dtype);
 int tam_dense_gqa_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
                           const void* k, const void* v, void* out, float* lse, void* workspace,
                           size_t ws_bytes, void* stream);
+
+/*
+ * Number of CUDA kernels this library has launched in this process so far (all
+ * devices, all entry points; status-block clears are not kernels and do not count).
+ */
+uint64_t tam_kernel_launches(void);
 
 /*
  * Waits for `stream`, then reads the device status block at the start of

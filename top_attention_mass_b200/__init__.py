@@ -10,6 +10,7 @@ Functions (same names as the C entry points, without the ``tam_`` prefix):
 
 * ``mass_oracle_prefill``      passes 1-3 of the attention-mass top-k oracle
 * ``attention_lse``            pass 1 alone (per-head log-sum-exp)
+* ``mass_select``              pass 2 alone (mass + top-k support, given pass 1's lse)
 * ``indexer_topk``             head-collapsed indexer support
 * ``sparse_support_attention`` pass 3 alone (attention on a given support)
 * ``dense_gqa_prefill``        dense causal GQA attention (comparator)
@@ -36,9 +37,10 @@ TAM_BF16, TAM_F32 = 0, 1
 
 EXPORTED = (
     "tam_version", "tam_status_string", "tam_mass_oracle_workspace", "tam_mass_oracle_prefill",
-    "tam_attention_lse_workspace", "tam_attention_lse", "tam_indexer_workspace",
+    "tam_attention_lse_workspace", "tam_attention_lse", "tam_mass_select_workspace",
+    "tam_mass_select", "tam_indexer_workspace",
     "tam_indexer_topk", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
-    "tam_dense_workspace", "tam_dense_gqa_prefill", "tam_check_status",
+    "tam_dense_workspace", "tam_dense_gqa_prefill", "tam_kernel_launches", "tam_check_status",
 )
 
 
@@ -79,6 +81,11 @@ def lib() -> ctypes.CDLL:
         L.tam_attention_lse_workspace.argtypes = [i64, i32, i32, i32, i32]
         L.tam_attention_lse.restype = i32
         L.tam_attention_lse.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, sz, p]
+        L.tam_mass_select_workspace.restype = sz
+        L.tam_mass_select_workspace.argtypes = [i64, i32, i32, i32, i32, i32, i32]
+        L.tam_mass_select.restype = i32
+        L.tam_mass_select.argtypes = [i64, i32, i32, i32, i32, p, p, p, i32, i32, p, p, p, p, sz,
+                                      p]
         L.tam_indexer_workspace.restype = sz
         L.tam_indexer_workspace.argtypes = [i64, i32, i32, i32, i32]
         L.tam_indexer_topk.restype = i32
@@ -92,6 +99,7 @@ def lib() -> ctypes.CDLL:
         L.tam_dense_workspace.argtypes = [i64, i32, i32, i32, i32]
         L.tam_dense_gqa_prefill.restype = i32
         L.tam_dense_gqa_prefill.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, sz, p]
+        L.tam_kernel_launches.restype = ctypes.c_uint64
         L.tam_check_status.restype = i32
         L.tam_check_status.argtypes = [p, p, p]
         _lib = L
@@ -107,6 +115,11 @@ def status_string(code: int) -> str:
 
 def version() -> int:
     return int(lib().tam_version())
+
+
+def kernel_launches() -> int:
+    """Kernels this library has launched in this process (all entry points)."""
+    return int(lib().tam_kernel_launches())
 
 
 # ------------------------------------------------------------------ marshalling helpers
@@ -260,6 +273,31 @@ def attention_lse(q, k, *, workspace: Optional[Workspace] = None, stream=None,
     if check:
         check_status(ws, stream)
     return lse
+
+
+def mass_select(q, k, lse, budget_k: int, block_q: int = 1, *,
+                workspace: Optional[Workspace] = None, stream=None, check: bool = True) -> Support:
+    """Pass 2: head-averaged mass and its top-k support, given pass 1's lse [Hq, N]."""
+    dev = q.device
+    N, Hq, Hkv, d = _shape(q, k)
+    dt = _dtype_code(q)
+    if lse.shape != (Hq, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be [Hq, N] fp32")
+    n_sel = N if block_q == 1 else -(-N // block_q)
+    sup_idx = torch.empty(n_sel, budget_k, dtype=torch.int32, device=dev)
+    sup_len = torch.empty(n_sel, dtype=torch.int32, device=dev)
+    sup_mass = torch.empty(n_sel, budget_k, dtype=torch.float32, device=dev)
+    L = lib()
+    nbytes = L.tam_mass_select_workspace(N, Hq, Hkv, d, dt, budget_k, block_q)
+    ws = _workspace(dev, max(nbytes, 256), workspace)
+    rc = L.tam_mass_select(N, Hq, Hkv, d, dt, _ptr(q.contiguous()), _ptr(k.contiguous()),
+                           _ptr(lse.contiguous()), budget_k, block_q, _ptr(sup_idx), _ptr(sup_len),
+                           _ptr(sup_mass), _ptr(ws), ws.numel() if nbytes else 0,
+                           _stream(dev, stream))
+    _raise(rc, "mass_select")
+    if check:
+        check_status(ws, stream)
+    return Support(sup_idx, sup_len, sup_mass)
 
 
 def indexer_topk(q_idx, k_idx, budget_k: int, block_q: int = 1, *,

@@ -66,6 +66,9 @@ struct IndexerArgs {
     int32_t* status;
 };
 
+// Counts one kernel launch (read back by tam_kernel_launches).
+void note_launch(int n = 1);
+
 // CUDA-core kernels (any dtype, any supported shape).
 cudaError_t simt_lse(const LseArgs& a, cudaStream_t st);
 cudaError_t simt_mass_select(const MassArgs& a, cudaStream_t st);

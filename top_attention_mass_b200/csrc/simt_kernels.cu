@@ -196,6 +196,7 @@ static cudaError_t launch_lse(const LseArgs& a, cudaStream_t st) {
     dim3 grid((unsigned)((a.N + 7) / 8), (unsigned)a.Hq);
     k_lse_simt<T><<<grid, 256, 8 * a.d * sizeof(float), st>>>(
         (const T*)a.q, (const T*)a.k, (int)a.N, a.Hq, a.Hkv, a.d, a.sl2, a.lse);
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -214,6 +215,7 @@ static cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     k_mass_select_simt<T><<<a.n_ctas, 256, smem, st>>>(
         (const T*)a.q, (const T*)a.k, a.lse, (int)a.N, a.Hq, a.Hkv, a.d, a.sl2, a.budget, a.block_q,
         a.n_sel, a.scratch, a.sup_idx, a.sup_len, a.sup_mass);
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -232,6 +234,7 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
     k_attn_rows_simt<T, DPL><<<(unsigned)a.N, 256, smem, st>>>(
         (const T*)a.q, (const T*)a.k, (const T*)a.v, (int)a.N, a.Hq, a.Hkv, a.d, a.sl2, a.sup_idx,
         a.sup_len, a.kmax, a.block_q, (T*)a.out, a.lse);
+    note_launch();
     return cudaGetLastError();
 }
 
@@ -246,6 +249,7 @@ static cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t st) {
     k_indexer_select_simt<T><<<a.n_ctas, 256, a.d_idx * sizeof(float), st>>>(
         (const T*)a.q_idx, (const T*)a.k_idx, (int)a.N, a.d_idx, a.budget, a.scratch, a.sup_idx,
         a.sup_len, a.sup_score);
+    note_launch();
     return cudaGetLastError();
 }
 

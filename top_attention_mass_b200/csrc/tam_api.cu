@@ -1,5 +1,6 @@
 // C ABI of libtam.so: argument checks, workspace layout and kernel dispatch.
 // Declarations and their contracts: include/tam.h.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -7,6 +8,12 @@
 #include "launch.h"
 
 using namespace tam;
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void tam::note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 namespace {
 
@@ -77,11 +84,28 @@ int start_call(void* workspace, cudaStream_t st) {
     return cuda_status(cudaMemsetAsync(workspace, 0, kStatusBytes, st));
 }
 
+// Pass 2 on an already computed lse, into the workspace laid out by plan_mass.
+int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
+                       const float* lse, int budget_k, int block_q, int32_t* sup_idx,
+                       int32_t* sup_len, float* sup_mass, char* ws, const MassPlan& plan,
+                       cudaStream_t st) {
+    MassArgs ma{};
+    ma.N = N; ma.Hq = Hq; ma.Hkv = Hkv; ma.d = d; ma.dtype = dtype;
+    ma.q = q; ma.k = k; ma.lse = lse; ma.sl2 = score_log2_scale(d);
+    ma.budget = budget_k; ma.block_q = block_q; ma.n_sel = (int)n_selection_units(N, block_q);
+    ma.n_ctas = plan.n_ctas; ma.scratch = (float*)(ws + plan.off_scratch);
+    ma.sup_idx = sup_idx; ma.sup_len = sup_len; ma.sup_mass = sup_mass;
+    ma.status = (int32_t*)ws;
+    return cuda_status(simt_mass_select(ma, st));
+}
+
 }  // namespace
 
 extern "C" {
 
 int tam_version(void) { return kVersion; }
+
+uint64_t tam_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* tam_status_string(int s) {
     switch (s) {
@@ -128,13 +152,9 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
     LseArgs la{N, Hq, Hkv, d, dtype, q, k, sl2, lse_buf, status};
     if ((rc = cuda_status(simt_lse(la, st)))) return rc;
 
-    MassArgs ma{};
-    ma.N = N; ma.Hq = Hq; ma.Hkv = Hkv; ma.d = d; ma.dtype = dtype;
-    ma.q = q; ma.k = k; ma.lse = lse_buf; ma.sl2 = sl2;
-    ma.budget = budget_k; ma.block_q = block_q; ma.n_sel = (int)n_selection_units(N, block_q);
-    ma.n_ctas = plan.n_ctas; ma.scratch = (float*)(ws + plan.off_scratch);
-    ma.sup_idx = sup_idx; ma.sup_len = sup_len; ma.sup_mass = sup_mass; ma.status = status;
-    if ((rc = cuda_status(simt_mass_select(ma, st)))) return rc;
+    if ((rc = launch_mass_select(N, Hq, Hkv, d, dtype, q, k, lse_buf, budget_k, block_q, sup_idx,
+                                 sup_len, sup_mass, ws, plan, st)))
+        return rc;
 
     if (out) {
         AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, sl2, sup_idx, sup_len, budget_k, block_q,
@@ -162,6 +182,32 @@ int tam_attention_lse(int64_t N, int Hq, int Hkv, int d, int dtype, const void* 
     if ((rc = start_call(workspace, st))) return rc;
     LseArgs la{N, Hq, Hkv, d, dtype, q, k, score_log2_scale(d), lse, (int32_t*)workspace};
     return cuda_status(simt_lse(la, st));
+}
+
+size_t tam_mass_select_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
+                                 int block_q) {
+    return tam_mass_oracle_workspace(N, Hq, Hkv, d, dtype, budget_k, block_q);
+}
+
+int tam_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
+                    const float* lse, int budget_k, int block_q, int32_t* sup_idx,
+                    int32_t* sup_len, float* sup_mass, void* workspace, size_t ws_bytes,
+                    void* stream) {
+    int rc = check_shape(N, Hq, Hkv, d, dtype);
+    if (rc) return rc;
+    rc = check_budget(N, budget_k, block_q);
+    if (rc) return rc;
+    if (!q || !k || !lse || !sup_idx || !sup_len || !sup_mass || !workspace)
+        return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, lse, sup_idx, sup_len, sup_mass, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
+    const MassPlan plan = plan_mass(N, Hq, block_q);
+    if (ws_bytes < plan.total) return TAM_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((rc = start_call(workspace, st))) return rc;
+    return launch_mass_select(N, Hq, Hkv, d, dtype, q, k, lse, budget_k, block_q, sup_idx, sup_len,
+                              sup_mass, (char*)workspace, plan, st);
 }
 
 size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
