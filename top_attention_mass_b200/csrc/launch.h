@@ -27,8 +27,9 @@ struct MassArgs {
     int budget, block_q, n_sel;
     int n_ctas;           // persistent blocks (CUDA-core path)
     float* scratch;       // n_ctas * N floats (CUDA-core path)
-    void* cand;           // candidate buffers (tensor-core path)
+    void* cand;           // candidate buffers (tensor-core path, per query)
     int cand_cap;         // entries per query row in `cand`
+    void* bmass;          // fixed-point block mass (tensor-core path, block-shared)
     int32_t* sup_idx;
     int32_t* sup_len;
     float* sup_mass;
@@ -68,6 +69,14 @@ struct IndexerArgs {
 
 // Counts one kernel launch (read back by tam_kernel_launches).
 void note_launch(int n = 1);
+
+// Tensor-core kernels (bf16, sm_100a).  *_supported says whether a shape is built.
+bool tc_lse_supported(const LseArgs& a);
+cudaError_t tc_lse(const LseArgs& a, cudaStream_t st);
+int tc_mass_columns(const MassArgs& a);
+bool tc_mass_supported(const MassArgs& a);
+size_t tc_mass_block_bytes(int64_t N, int block_q);
+cudaError_t tc_mass_select(const MassArgs& a, cudaStream_t st);
 
 // CUDA-core kernels (any dtype, any supported shape).
 cudaError_t simt_lse(const LseArgs& a, cudaStream_t st);

@@ -1,0 +1,674 @@
+// Pass 2 on the tensor cores: head-averaged token mass and its top-k support.
+//
+//   P_i[j] = (1/Hq) sum_h exp(scale * q[i,h].k[j,g(h)] - lse[h,i]),  j <= i
+//   per query:  S_i = top-min(k, i+1) of P_i          (ranking: value desc, index asc)
+//   per block:  M_b[j] = sum_{i in block b, i >= j} P_i[j]  -> top-k in k_block_select
+//
+// (arXiv 2606.07703, Abstract: "selects head-averaged token support"; gist.science
+// technical report §2.1, "Mechanismus", "Selektion" and "Granularität".)
+//
+// Orientation: one UMMA per KV group computes S^T = K_g Q_g^T with M = 128 keys
+// and N = NQ columns (BQ queries x G heads of that group).  A CTA keeps Q of its
+// BQ queries for *all* heads resident in shared memory, so the thread that owns a
+// key row adds the probabilities of every head of a query in registers - the head
+// average needs no cross-thread reduction and the N x N mass never leaves the SM.
+// Roles (320 threads):
+//   warp 4      TMA producer: Q (once, all groups), then K_g tiles in a 2-stage ring;
+//   warp 5      MMA issuer: for each key tile, one UMMA chain per group into a ring
+//               of 512/NQ TMEM slots;
+//   warps 0-3   mass warps: thread = key row; exp2 against the pass-1 LSE, sum over
+//               heads -> mass of BQ queries; causal mask; then either the mass tile
+//               goes to shared memory for the select warps (per query) or the
+//               block column sum is added in 2^-40 fixed point (block-shared);
+//   warps 6-9   select warps (per query): each owns BQ/4 queries and runs a streaming
+//               exact top-k: strict threshold tau plus a candidate buffer in global
+//               memory, appended in ascending key order, compacted by a warp radix
+//               select when it fills (keeps exactly k; ties keep the smaller index),
+//               and written ascending at the end.
+#include "launch.h"
+#include "tc_ptx.cuh"
+#include "tma_host.h"
+
+namespace tam {
+namespace {
+
+constexpr int kStages = 2;
+constexpr int kThreads = 320;
+
+struct SelWarpSmem {
+    int hist[256];
+};
+
+// Q (all groups) + K ring + lse2 + barriers, plus (per query) 2 mass tiles and the
+// select warps' histograms.
+__host__ __device__ constexpr int mass_smem_bytes(int NQ, int D, int Hkv, int G, bool block) {
+    return 1024 + Hkv * NQ * D * 2 + kStages * 128 * D * 2 + Hkv * NQ * 4 + 512 +
+           (block ? 0 : 2 * (NQ / G) * 128 * 4 + 4 * (int)sizeof(SelWarpSmem));
+}
+constexpr int kMaxDynSmem = 227 * 1024;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// k-th largest key (non-negative float bits) among buf[0..n) by an MSB-first
+// 4 x 8-bit radix select over the warp.  Returns the key T and how many entries
+// equal to T belong to the top k (the earliest ones in buffer order).
+__device__ __forceinline__ void warp_kth(const uint2* buf, int n, int k, int* hist, uint32_t& T,
+                                         int& take_eq) {
+    const int lane = threadIdx.x & 31;
+    uint32_t prefix = 0, mask = 0;
+    int remaining = k;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = lane; b < 256; b += 32) hist[b] = 0;
+        __syncwarp();
+        for (int e = lane; e < n; e += 32) {
+            const uint32_t key = buf[e].x;
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        }
+        __syncwarp();
+        int c8[8], sum = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            c8[t] = hist[255 - 8 * lane - t];
+            sum += c8[t];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const int excl = incl - sum;
+        const uint32_t who = __ballot_sync(0xffffffffu, excl < remaining && remaining <= incl);
+        const int src = __ffs(who) - 1;
+        int digit = -1, rem = 0, cum = excl;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            if (digit < 0 && cum + c8[t] >= remaining) {
+                digit = 255 - 8 * lane - t;
+                rem = remaining - cum;
+            }
+            cum += c8[t];
+        }
+        digit = __shfl_sync(0xffffffffu, digit, src);
+        rem = __shfl_sync(0xffffffffu, rem, src);
+        prefix |= (uint32_t)digit << shift;
+        mask |= 255u << shift;
+        remaining = rem;
+        __syncwarp();
+    }
+    T = prefix;
+    take_eq = remaining;
+}
+
+// Stable in-place compaction of buf[0..n) to the entries with key > T plus the first
+// take_eq entries with key == T.  Returns the kept count.
+__device__ __forceinline__ int warp_compact(uint2* buf, int n, uint32_t T, int take_eq) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = lanemask_lt();
+    int kept = 0, eq_seen = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int e = base + lane;
+        uint2 x = make_uint2(0u, 0u);
+        if (e < n) x = buf[e];
+        const bool gt = e < n && x.x > T;
+        const bool eq = e < n && x.x == T;
+        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+        const bool keep = gt || (eq && eq_seen + __popc(eqb & lt) < take_eq);
+        const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+        __syncwarp();
+        if (keep) buf[kept + __popc(kb & lt)] = x;
+        kept += __popc(kb);
+        eq_seen += __popc(eqb);
+        __syncwarp();
+    }
+    return kept;
+}
+
+// Final write of one query's support: same selection as warp_compact, written to
+// the output rows (ascending key order is the buffer order), padded with -1 / 0.
+__device__ __forceinline__ void warp_emit(const uint2* buf, int n, uint32_t T, int take_eq,
+                                          bool select_all, int budget, int32_t* out_idx,
+                                          float* out_mass, int32_t* out_len) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = lanemask_lt();
+    int kept = 0, eq_seen = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int e = base + lane;
+        uint2 x = make_uint2(0u, 0u);
+        if (e < n) x = buf[e];
+        const bool gt = e < n && (select_all || x.x > T);
+        const bool eq = e < n && !select_all && x.x == T;
+        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+        const bool keep = gt || (eq && eq_seen + __popc(eqb & lt) < take_eq);
+        const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+            const int p = kept + __popc(kb & lt);
+            out_idx[p] = (int32_t)x.y;
+            out_mass[p] = __uint_as_float(x.x);
+        }
+        kept += __popc(kb);
+        eq_seen += __popc(eqb);
+    }
+    for (int t = kept + lane; t < budget; t += 32) {
+        out_idx[t] = -1;
+        out_mass[t] = 0.f;
+    }
+    if (lane == 0) *out_len = kept;
+}
+
+struct MassParams {
+    int N, Hq, Hkv, n_ctiles, budget, block_q, cap;
+    float sl2, inv_hq;
+    const float* lse;
+    int32_t* sup_idx;
+    int32_t* sup_len;
+    float* sup_mass;
+    uint2* cand;                     // [N][cap] (per query)
+    unsigned long long* bmass;       // triangular block mass (block mode)
+    int32_t* status;
+    uint64_t timeout_ns;
+    int dbg;
+};
+
+// Offset of block b's row in the triangular block-mass buffer.
+__host__ __device__ __forceinline__ int64_t bmass_offset(int64_t b, int block_q) {
+    return (int64_t)block_q * b * (b + 1) / 2;
+}
+
+template <int G, int D, int NQ, bool BLOCK>
+__global__ void __launch_bounds__(kThreads, 1)
+k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+          const MassParams p) {
+    constexpr int BQ = NQ / G;            // queries per CTA
+    constexpr int NH = D / 64;
+    constexpr int R = 512 / NQ;           // TMEM accumulator slots
+    constexpr uint32_t kQHalf = NQ * 128; // bytes of one 64-element half of a group's Q
+    constexpr uint32_t kKHalf = 128 * 128;
+    constexpr uint32_t kKTile = NH * kKHalf;
+    constexpr int QPW = BQ / 4;           // queries per select warp
+    const int Hkv = p.Hkv;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* sQ = base;                                   // Hkv * NH * kQHalf
+    uint8_t* sK = sQ + Hkv * NH * kQHalf;                 // kStages * kKTile
+    float* sLse = reinterpret_cast<float*>(sK + kStages * kKTile);   // Hkv * NQ
+    float* sMass = sLse + Hkv * NQ;                                    // 2 x BQ x 128 (per query)
+    SelWarpSmem* sSel = reinterpret_cast<SelWarpSmem*>(sMass + (BLOCK ? 0 : 2 * BQ * 128));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + (BLOCK ? 0 : 4));
+    uint64_t* q_full = bars;
+    uint64_t* k_full = q_full + 1;
+    uint64_t* k_empty = k_full + kStages;
+    uint64_t* s_full = k_empty + kStages;
+    uint64_t* s_empty = s_full + R;
+    uint64_t* m_full = s_empty + R;
+    uint64_t* m_empty = m_full + 2;
+    uint64_t* mma_done = m_empty + 2;
+    uint64_t* never = mma_done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ct = p.n_ctiles - 1 - (int)blockIdx.x;      // heaviest tile first
+    const int q0 = ct * BQ;
+    const int q_last = min(p.N, q0 + BQ) - 1;
+    const int n_kt = q_last / 128 + 1;
+    const int n_units = n_kt * Hkv;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(&k_full[s], 1);
+            tc::mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < R; ++s) {
+            tc::mbar_init(&s_full[s], 1);
+            tc::mbar_init(&s_empty[s], 128);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&m_full[b], 128);
+            tc::mbar_init(&m_empty[b], 128);
+        }
+        tc::mbar_init(mma_done, 1);
+        tc::mbar_init(never, 1);
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    // log2-domain LSE of every column of every group (+inf for padding queries)
+    for (int t = threadIdx.x; t < Hkv * NQ; t += blockDim.x) {
+        const int g = t / NQ, c = t % NQ;
+        const int i = q0 + c / G, h = g * G + c % G;
+        sLse[t] = (i < p.N) ? p.lse[(size_t)h * p.N + i] * kLog2e : INFINITY;
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const tc::Guard gd{abort_flag, p.status, BLOCK ? KID_BLOCK_MASS_TC : KID_MASS_TC,
+                       p.timeout_ns};
+
+    if (warp == 4) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            tc::prefetch_tmap(&tmQ);
+            tc::prefetch_tmap(&tmK);
+            tc::mbar_arrive_expect_tx(q_full, Hkv * NH * kQHalf);
+            for (int g = 0; g < Hkv; ++g)
+                for (int h = 0; h < NH; ++h)
+                    tc::tma_load_3d(sQ + (g * NH + h) * kQHalf, &tmQ, q_full, h * 64, g * G, q0);
+            int issued = 0;
+            for (int u = 0; u < n_units; ++u) {
+                const int s = u % kStages;
+                const uint32_t ph = (u / kStages) & 1;
+                if (!tc::wait(&k_empty[s], ph ^ 1, gd, 1)) break;
+                const int kt = u / Hkv, g = u % Hkv;
+                tc::mbar_arrive_expect_tx(&k_full[s], kKTile);
+                for (int h = 0; h < NH; ++h)
+                    tc::tma_load_3d(sK + s * kKTile + h * kKHalf, &tmK, &k_full[s], h * 64, g,
+                                    kt * 128);
+                ++issued;
+            }
+            int zero = 0;
+            const tc::Guard drain{&zero, nullptr, 0, p.timeout_ns};
+            for (int u = max(0, issued - kStages); u < issued; ++u)
+                tc::wait(&k_full[u % kStages], (u / kStages) & 1, drain, 0);
+            tc::wait(q_full, 0, drain, 0);
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_bf16_f32(128, NQ);
+            bool ok = tc::wait(q_full, 0, gd, 2);
+            for (int u = 0; ok && u < n_units; ++u) {
+                const int s = u % kStages;
+                const uint32_t ph = (u / kStages) & 1;
+                const int slot = u % R;
+                const uint32_t sph = (u / R) & 1;
+                const int g = u % Hkv;
+                if (!tc::wait(&k_full[s], ph, gd, 3)) break;
+                if (!tc::wait(&s_empty[slot], sph ^ 1, gd, 4)) break;
+                tc::fence_after_sync();
+                const uint32_t ak = tc::smem_u32(sK + s * kKTile);
+                const uint32_t bq = tc::smem_u32(sQ + g * NH * kQHalf);
+#pragma unroll
+                for (int kk = 0; kk < NH * 4; ++kk) {
+                    const uint32_t offk = (kk >> 2) * kKHalf + (kk & 3) * 32;
+                    const uint32_t offq = (kk >> 2) * kQHalf + (kk & 3) * 32;
+                    tc::mma_bf16_ss(tmem + slot * NQ, tc::desc_kmajor_sw128(ak + offk),
+                                    tc::desc_kmajor_sw128(bq + offq), idesc, kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&k_empty[s]);
+                tc::mma_commit(&s_full[slot]);
+            }
+            tc::mma_commit(mma_done);
+            int zero = 0;
+            const tc::Guard drain{&zero, nullptr, 0, p.timeout_ns};
+            tc::wait(mma_done, 0, drain, 0);
+        }
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- mass warps
+        const int row = threadIdx.x;                       // key row of the tile
+        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        bool ok = true;
+        if (p.dbg & kDebugForceTimeout) ok = tc::wait(never, 0, gd, 9);
+        for (int kt = 0; ok && kt < n_kt; ++kt) {
+            float acc[BQ];
+#pragma unroll
+            for (int q = 0; q < BQ; ++q) acc[q] = 0.f;
+            for (int g = 0; g < Hkv; ++g) {
+                const int u = kt * Hkv + g;
+                const int slot = u % R;
+                if (!tc::wait(&s_full[slot], (u / R) & 1, gd, 5)) { ok = false; break; }
+                tc::fence_after_sync();
+                // stream the NQ columns in 32-column chunks, loading chunk c+1 while
+                // chunk c is exponentiated
+                const uint32_t col0 = lane_addr + slot * NQ;
+                uint32_t va[32], vb[32];
+                tc::tmem_ld32(col0, va);
+                tc::tmem_wait_ld(va);
+#pragma unroll
+                for (int c = 0; c < NQ / 32; ++c) {
+                    uint32_t (&cur)[32] = (c & 1) ? vb : va;
+                    uint32_t (&nxt)[32] = (c & 1) ? va : vb;
+                    if (c + 1 < NQ / 32) tc::tmem_ld32(col0 + (c + 1) * 32, nxt);
+                    const float4* l4 = reinterpret_cast<const float4*>(sLse + g * NQ + c * 32);
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 L = l4[c4];
+                        const float Ls[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int col = c * 32 + c4 * 4 + e;
+                            const float sc = __uint_as_float(cur[c4 * 4 + e]);
+                            acc[col / G] += tc::ex2(fmaf(sc, p.sl2, -Ls[e]));
+                        }
+                    }
+                    if (c + 1 < NQ / 32) tc::tmem_wait_ld(nxt);
+                }
+                tc::fence_before_sync();
+                tc::mbar_arrive(&s_empty[slot]);
+            }
+            if (!ok) break;
+            const int j = kt * 128 + row;
+            if constexpr (!BLOCK) {
+                const int mb = kt & 1;
+                if (!tc::wait(&m_empty[mb], ((kt >> 1) & 1) ^ 1, gd, 6)) { ok = false; break; }
+                float* mt = sMass + mb * BQ * 128;
+#pragma unroll
+                for (int q = 0; q < BQ; ++q) {
+                    const int i = q0 + q;
+                    mt[q * 128 + row] = (j <= i && i < p.N) ? acc[q] * p.inv_hq : -1.f;
+                }
+                tc::mbar_arrive(&m_full[mb]);
+            } else {
+                // block column sums, 2^-40 fixed point, one add per (block, key)
+                int cur_b = q0 / p.block_q;
+                float part = 0.f;
+#pragma unroll
+                for (int q = 0; q < BQ; ++q) {
+                    const int i = q0 + q;
+                    if (i < p.N) {
+                        const int b = i / p.block_q;
+                        if (b != cur_b) {
+                            if (part > 0.f)
+                                atomicAdd(&p.bmass[bmass_offset(cur_b, p.block_q) + j],
+                                          (unsigned long long)__float2ll_rn(
+                                              part * p.inv_hq * 1099511627776.0f));
+                            part = 0.f;
+                            cur_b = b;
+                        }
+                        if (j <= i) part += acc[q];
+                    }
+                }
+                if (part > 0.f)
+                    atomicAdd(&p.bmass[bmass_offset(cur_b, p.block_q) + j],
+                              (unsigned long long)__float2ll_rn(part * p.inv_hq * 1099511627776.0f));
+            }
+        }
+    } else if (!BLOCK) {
+        // ---------------------------------------------------------------- select warps
+        const int sw = warp - 6;
+        int* hist = sSel[sw].hist;
+        float tau[QPW];
+        int cnt[QPW];
+#pragma unroll
+        for (int a = 0; a < QPW; ++a) {
+            tau[a] = -1.f;
+            cnt[a] = 0;
+        }
+        bool ok = true;
+        bool overflow = false;
+        for (int kt = 0; ok && kt < n_kt; ++kt) {
+            const int mb = kt & 1;
+            if (!tc::wait(&m_full[mb], (kt >> 1) & 1, gd, 7)) { ok = false; break; }
+            const float* mt = sMass + mb * BQ * 128;
+#pragma unroll
+            for (int a = 0; a < QPW; ++a) {
+                const int q = sw * QPW + a;
+                const int i = q0 + q;
+                if (i >= p.N) continue;
+                uint2* buf = p.cand + (size_t)i * p.cap;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const float v = mt[q * 128 + r * 32 + lane];
+                    const bool pass = v > tau[a];
+                    const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+                    const int pos = cnt[a] + __popc(bal & lanemask_lt());
+                    if (pass) {
+                        if (pos < p.cap)
+                            buf[pos] = make_uint2(__float_as_uint(v), (uint32_t)(kt * 128 + r * 32 + lane));
+                        else
+                            overflow = true;
+                    }
+                    cnt[a] += __popc(bal);
+                }
+                if (cnt[a] > p.cap - 128 && cnt[a] > p.budget) {
+                    __syncwarp();
+                    const int n = min(cnt[a], p.cap);
+                    uint32_t T;
+                    int take_eq;
+                    warp_kth(buf, n, p.budget, hist, T, take_eq);
+                    cnt[a] = warp_compact(buf, n, T, take_eq);
+                    tau[a] = __uint_as_float(T);
+                }
+            }
+            __syncwarp();
+            tc::mbar_arrive(&m_empty[mb]);
+        }
+        if (__any_sync(0xffffffffu, overflow) && lane == 0)
+            report_error(p.status, TAM_ERR_OVERFLOW, KID_MASS_TC, q0);
+        if (ok) {
+#pragma unroll
+            for (int a = 0; a < QPW; ++a) {
+                const int i = q0 + sw * QPW + a;
+                if (i >= p.N) continue;
+                uint2* buf = p.cand + (size_t)i * p.cap;
+                const int n = min(cnt[a], p.cap);
+                __syncwarp();
+                uint32_t T = 0;
+                int take_eq = 0;
+                const bool all = n <= p.budget;
+                if (!all) warp_kth(buf, n, p.budget, hist, T, take_eq);
+                warp_emit(buf, n, T, take_eq, all, p.budget, p.sup_idx + (size_t)i * p.budget,
+                          p.sup_mass + (size_t)i * p.budget, p.sup_len + i);
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- block top-k
+// One CTA per block: exact top-min(k, e_b+1) of the fixed-point block mass row
+// (64-bit keys, 8 x 8-bit radix select), written ascending with the mass as fp32.
+__global__ void __launch_bounds__(256) k_block_select(const unsigned long long* __restrict__ bmass,
+                                                      int N, int block_q, int budget,
+                                                      int32_t* __restrict__ sup_idx,
+                                                      int32_t* __restrict__ sup_len,
+                                                      float* __restrict__ sup_mass) {
+    __shared__ int hist[256];
+    __shared__ int warp_tot[33];
+    __shared__ int s_digit, s_rem;
+    const int b = blockIdx.x;
+    const int n = min(N, (b + 1) * block_q);     // keys 0..e_b
+    const unsigned long long* row = bmass + bmass_offset(b, block_q);
+    const int tid = threadIdx.x, nt = blockDim.x;
+    int32_t* oi = sup_idx + (size_t)b * budget;
+    float* om = sup_mass + (size_t)b * budget;
+    const bool all = n <= budget;
+    unsigned long long T = 0;
+    int take_eq = 0;
+    if (!all) {
+        unsigned long long prefix = 0, mask = 0;
+        int remaining = budget;
+        for (int shift = 56; shift >= 0; shift -= 8) {
+            for (int x = tid; x < 256; x += nt) hist[x] = 0;
+            __syncthreads();
+            for (int j = tid; j < n; j += nt) {
+                const unsigned long long key = row[j];
+                if ((key & mask) == prefix) atomicAdd(&hist[(int)((key >> shift) & 255ull)], 1);
+            }
+            __syncthreads();
+            if (tid == 0) {
+                int cum = 0;
+                for (int x = 255; x >= 0; --x) {
+                    if (cum + hist[x] >= remaining) {
+                        s_digit = x;
+                        s_rem = remaining - cum;
+                        break;
+                    }
+                    cum += hist[x];
+                }
+            }
+            __syncthreads();
+            prefix |= (unsigned long long)s_digit << shift;
+            mask |= 255ull << shift;
+            remaining = s_rem;
+            __syncthreads();
+        }
+        T = prefix;
+        take_eq = remaining;
+    }
+    int base_sel = 0, base_eq = 0;
+    for (int j0 = 0; j0 < n; j0 += nt) {
+        const int j = j0 + tid;
+        unsigned long long key = 0;
+        bool gt = false, eq = false;
+        if (j < n) {
+            key = row[j];
+            gt = all || key > T;
+            eq = !all && key == T;
+        }
+        int eq_tot, sel_tot;
+        const int eq_excl = block_exclusive_scan(eq ? 1 : 0, warp_tot, &eq_tot);
+        const bool sel = gt || (eq && base_eq + eq_excl < take_eq);
+        const int sel_excl = block_exclusive_scan(sel ? 1 : 0, warp_tot, &sel_tot);
+        if (sel) {
+            oi[base_sel + sel_excl] = j;
+            om[base_sel + sel_excl] = (float)((double)key * (1.0 / 1099511627776.0));
+        }
+        base_eq += eq_tot;
+        base_sel += sel_tot;
+    }
+    const int m = min(n, budget);
+    for (int t = m + tid; t < budget; t += nt) {
+        oi[t] = -1;
+        om[t] = 0.f;
+    }
+    if (tid == 0) sup_len[b] = m;
+}
+
+template <int G, int D, int NQ, bool BLOCK>
+cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
+    constexpr int BQ = NQ / G;
+    CUtensorMap tq, tk;
+    const uint64_t d = a.d;
+    if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQ) ||
+        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, a.N, d * 2, (uint64_t)a.Hkv * d * 2, 64, 1, 128))
+        return cudaErrorInvalidValue;
+    MassParams p{};
+    p.N = (int)a.N;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.n_ctiles = (int)((a.N + BQ - 1) / BQ);
+    p.budget = a.budget;
+    p.block_q = a.block_q;
+    p.cap = a.cand_cap;
+    p.sl2 = a.sl2;
+    p.inv_hq = 1.f / (float)a.Hq;
+    p.lse = a.lse;
+    p.sup_idx = a.sup_idx;
+    p.sup_len = a.sup_len;
+    p.sup_mass = a.sup_mass;
+    p.cand = reinterpret_cast<uint2*>(a.cand);
+    p.bmass = reinterpret_cast<unsigned long long*>(a.bmass);
+    p.status = a.status;
+    p.timeout_ns = wait_timeout_ns();
+    p.dbg = debug_flags();
+    const int smem = mass_smem_bytes(NQ, D, a.Hkv, G, BLOCK);
+    auto kern = k_mass_tc<G, D, NQ, BLOCK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (BLOCK) {
+        const int64_t nb = (a.N + a.block_q - 1) / a.block_q;
+        e = cudaMemsetAsync(a.bmass, 0, (size_t)bmass_offset(nb, a.block_q) * 8, st);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<(unsigned)p.n_ctiles, kThreads, smem, st>>>(tq, tk, p);
+    note_launch();
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !BLOCK) return e;
+    const int nb = (int)((a.N + a.block_q - 1) / a.block_q);
+    k_block_select<<<nb, 256, 0, st>>>(p.bmass, p.N, a.block_q, a.budget, a.sup_idx, a.sup_len,
+                                       a.sup_mass);
+    note_launch();
+    return cudaGetLastError();
+}
+
+// Only (G, NQ) pairs with 4..32 queries per CTA are instantiated.
+template <int G, int D, int NQ, bool BLOCK>
+cudaError_t launch_if_valid(const MassArgs& a, cudaStream_t st) {
+    if constexpr (NQ / G >= 4 && NQ / G <= 32 && (NQ / G) % 4 == 0)
+        return launch_mass<G, D, NQ, BLOCK>(a, st);
+    else
+        return cudaErrorNotSupported;
+}
+
+template <int D, int NQ, bool BLOCK>
+cudaError_t dispatch_g(const MassArgs& a, cudaStream_t st) {
+    switch (a.Hq / a.Hkv) {
+        case 1: return launch_if_valid<1, D, NQ, BLOCK>(a, st);
+        case 2: return launch_if_valid<2, D, NQ, BLOCK>(a, st);
+        case 4: return launch_if_valid<4, D, NQ, BLOCK>(a, st);
+        case 8: return launch_if_valid<8, D, NQ, BLOCK>(a, st);
+        case 16: return launch_if_valid<16, D, NQ, BLOCK>(a, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+template <int D, bool BLOCK>
+cudaError_t dispatch_nq(const MassArgs& a, cudaStream_t st) {
+    switch (tc_mass_columns(a)) {
+        case 128: return dispatch_g<D, 128, BLOCK>(a, st);
+        case 64: return dispatch_g<D, 64, BLOCK>(a, st);
+        case 32: return dispatch_g<D, 32, BLOCK>(a, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+template <bool BLOCK>
+cudaError_t dispatch(const MassArgs& a, cudaStream_t st) {
+    return a.d == 64 ? dispatch_nq<64, BLOCK>(a, st) : dispatch_nq<128, BLOCK>(a, st);
+}
+
+}  // namespace
+
+int tc_mass_columns(const MassArgs& a) {
+    // NQ columns per group: 128 (twice the queries per CTA, half the K re-reads) when
+    // the Q of all groups plus the rest of the layout fits in shared memory, else 64.
+    const int G = a.Hq / a.Hkv;
+    const bool block = a.block_q > 1;
+    // (queries per CTA NQ/G kept within [4, 32] so the per-thread accumulators stay
+    // in registers and every select warp owns at least one query)
+    if (a.Hkv > 64 || G < 1) return 0;
+    for (int nq = 128; nq >= 32; nq >>= 1) {
+        const int bq = nq / G;
+        if (bq < 4 || bq > 32) continue;
+        if (mass_smem_bytes(nq, a.d, a.Hkv, G, block) <= kMaxDynSmem) return nq;
+    }
+    return 0;
+}
+
+bool tc_mass_supported(const MassArgs& a) {
+    const int G = a.Hq / a.Hkv;
+    const int nq = tc_mass_columns(a);
+    if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128) || nq == 0) return false;
+    if (!(G == 1 || G == 2 || G == 4 || G == 8 || G == 16)) return false;
+    if ((nq / G) % 4 != 0) return false;                      // whole queries per select warp
+    if (a.block_q > 1 && a.block_q > (1 << 20)) return false;
+    return true;
+}
+
+size_t tc_mass_block_bytes(int64_t N, int block_q) {
+    const int64_t nb = (N + block_q - 1) / block_q;
+    return (size_t)bmass_offset(nb, block_q) * 8;
+}
+
+cudaError_t tc_mass_select(const MassArgs& a, cudaStream_t st) {
+    return a.block_q == 1 ? dispatch<false>(a, st) : dispatch<true>(a, st);
+}
+
+}  // namespace tam

@@ -6,6 +6,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "tma_host.h"
 
 using namespace tam;
 
@@ -47,19 +48,39 @@ inline int64_t n_selection_units(int64_t N, int block_q) {
     return block_q == 1 ? N : (N + block_q - 1) / block_q;
 }
 
-// Workspace layout of tam_mass_oracle_prefill.
+// Workspace layout of tam_mass_oracle_prefill / tam_mass_select: status block, lse
+// (when the caller passes none), then the pass-2 scratch of whichever kernel runs:
+// candidate buffers (tensor cores, per query), fixed-point block mass (tensor cores,
+// block-shared) or staged mass rows (CUDA cores).
 struct MassPlan {
-    size_t off_lse, off_scratch, total;
-    int n_ctas;
+    size_t off_lse, off_work, total;
+    bool tc;
+    int n_ctas, cand_cap;
 };
 
-MassPlan plan_mass(int64_t N, int Hq, int block_q) {
-    MassPlan p;
+MassArgs mass_shape(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k, int block_q) {
+    MassArgs a{};
+    a.N = N; a.Hq = Hq; a.Hkv = Hkv; a.d = d; a.dtype = dtype;
+    a.budget = budget_k; a.block_q = block_q;
+    return a;
+}
+
+MassPlan plan_mass(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k, int block_q) {
+    MassPlan p{};
     const int64_t n_sel = n_selection_units(N, block_q);
+    p.tc = tc_mass_supported(mass_shape(N, Hq, Hkv, d, dtype, budget_k, block_q));
     p.n_ctas = (int)std::min<int64_t>(n_sel, kSimtPersistentCtas);
+    p.cand_cap = candidate_capacity(budget_k);
     p.off_lse = kStatusBytes;
-    p.off_scratch = p.off_lse + align256((size_t)Hq * N * sizeof(float));
-    p.total = p.off_scratch + align256((size_t)p.n_ctas * N * sizeof(float));
+    p.off_work = p.off_lse + align256((size_t)Hq * N * sizeof(float));
+    size_t work;
+    if (!p.tc)
+        work = (size_t)p.n_ctas * N * sizeof(float);
+    else if (block_q == 1)
+        work = (size_t)N * p.cand_cap * 8;
+    else
+        work = tc_mass_block_bytes(N, block_q);
+    p.total = p.off_work + align256(work);
     return p;
 }
 
@@ -78,6 +99,11 @@ IndexerPlan plan_indexer(int64_t N) {
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? TAM_OK : TAM_ERR_CUDA; }
 
+// Pass 1 on the tensor cores where the shape is built, else on the CUDA cores.
+cudaError_t run_lse(const LseArgs& a, cudaStream_t st) {
+    return tc_lse_supported(a) ? tc_lse(a, st) : simt_lse(a, st);
+}
+
 inline float score_log2_scale(int d) { return (float)(1.0 / std::sqrt((double)d)) * kLog2e; }
 
 int start_call(void* workspace, cudaStream_t st) {
@@ -89,14 +115,17 @@ int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void*
                        const float* lse, int budget_k, int block_q, int32_t* sup_idx,
                        int32_t* sup_len, float* sup_mass, char* ws, const MassPlan& plan,
                        cudaStream_t st) {
-    MassArgs ma{};
-    ma.N = N; ma.Hq = Hq; ma.Hkv = Hkv; ma.d = d; ma.dtype = dtype;
+    MassArgs ma = mass_shape(N, Hq, Hkv, d, dtype, budget_k, block_q);
     ma.q = q; ma.k = k; ma.lse = lse; ma.sl2 = score_log2_scale(d);
-    ma.budget = budget_k; ma.block_q = block_q; ma.n_sel = (int)n_selection_units(N, block_q);
-    ma.n_ctas = plan.n_ctas; ma.scratch = (float*)(ws + plan.off_scratch);
+    ma.n_sel = (int)n_selection_units(N, block_q);
+    ma.n_ctas = plan.n_ctas;
+    ma.scratch = (float*)(ws + plan.off_work);
+    ma.cand = ws + plan.off_work;
+    ma.cand_cap = plan.cand_cap;
+    ma.bmass = ws + plan.off_work;
     ma.sup_idx = sup_idx; ma.sup_len = sup_len; ma.sup_mass = sup_mass;
     ma.status = (int32_t*)ws;
-    return cuda_status(simt_mass_select(ma, st));
+    return cuda_status(plan.tc ? tc_mass_select(ma, st) : simt_mass_select(ma, st));
 }
 
 }  // namespace
@@ -124,7 +153,7 @@ size_t tam_mass_oracle_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, i
                                  int block_q) {
     if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK) return 0;
     if (check_budget(N, budget_k, block_q) != TAM_OK) return 0;
-    return plan_mass(N, Hq, block_q).total;
+    return plan_mass(N, Hq, Hkv, d, dtype, budget_k, block_q).total;
 }
 
 int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
@@ -140,7 +169,7 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
     const void* ptrs[] = {q, k, v, sup_idx, sup_len, sup_mass, lse, out, workspace};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return TAM_ERR_INVALID_ARG;
-    const MassPlan plan = plan_mass(N, Hq, block_q);
+    const MassPlan plan = plan_mass(N, Hq, Hkv, d, dtype, budget_k, block_q);
     if (ws_bytes < plan.total) return TAM_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     char* ws = (char*)workspace;
@@ -150,7 +179,7 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
 
     const float sl2 = score_log2_scale(d);
     LseArgs la{N, Hq, Hkv, d, dtype, q, k, sl2, lse_buf, status};
-    if ((rc = cuda_status(simt_lse(la, st)))) return rc;
+    if ((rc = cuda_status(run_lse(la, st)))) return rc;
 
     if ((rc = launch_mass_select(N, Hq, Hkv, d, dtype, q, k, lse_buf, budget_k, block_q, sup_idx,
                                  sup_len, sup_mass, ws, plan, st)))
@@ -181,7 +210,7 @@ int tam_attention_lse(int64_t N, int Hq, int Hkv, int d, int dtype, const void* 
     cudaStream_t st = (cudaStream_t)stream;
     if ((rc = start_call(workspace, st))) return rc;
     LseArgs la{N, Hq, Hkv, d, dtype, q, k, score_log2_scale(d), lse, (int32_t*)workspace};
-    return cuda_status(simt_lse(la, st));
+    return cuda_status(run_lse(la, st));
 }
 
 size_t tam_mass_select_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
@@ -202,7 +231,7 @@ int tam_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
     const void* ptrs[] = {q, k, lse, sup_idx, sup_len, sup_mass, workspace};
     for (const void* p : ptrs)
         if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
-    const MassPlan plan = plan_mass(N, Hq, block_q);
+    const MassPlan plan = plan_mass(N, Hq, Hkv, d, dtype, budget_k, block_q);
     if (ws_bytes < plan.total) return TAM_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     if ((rc = start_call(workspace, st))) return rc;

@@ -1,0 +1,31 @@
+// Host helpers: TMA tensor-map encoding (through the runtime's driver entry point,
+// so the library needs no link-time libcuda) and the wait deadline / debug switches.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tam {
+
+// Encodes a 3-D bf16 tensor map with a 128-byte swizzle.  Dimensions innermost
+// first; strides in bytes for dims 1 and 2 (multiples of 16); box sizes in
+// elements (box0 * 2 must be 128).  Returns false if the driver rejects it.
+bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0,
+                       uint32_t box1, uint32_t box2);
+
+// Deadline of every bounded device wait (ns).  2 s normally; with the debug
+// variable TAM_DEBUG_FORCE_TIMEOUT=1 in the environment a short deadline is used
+// and kernels that support it park one role on a barrier nobody arrives on, so the
+// timeout path can be exercised without faulting anything.
+uint64_t wait_timeout_ns();
+int debug_flags();
+
+// Entries per query row of the streaming top-k candidate buffer; the debug
+// variable TAM_DEBUG_CAND_CAP overrides it (to exercise the overflow report).
+int candidate_capacity(int budget_k);
+
+constexpr int kDebugForceTimeout = 1;
+
+}  // namespace tam

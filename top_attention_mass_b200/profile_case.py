@@ -1,0 +1,59 @@
+"""Run one row of the hot path a few times on a seeded input, for ncu captures.
+
+    python -m top_attention_mass_b200.profile_case --row pass1_lse --N 16384 [--reps 3]
+
+Rows: pass1_lse, pass2_mass_topk, pass2_block_mass_topk, pass3_gather, pass3_block,
+indexer_topk, dense_prefill.  Shapes are those of the 32K workload (Hq=32, Hkv=8,
+d=128, bf16, k=655, B_q=64, indexer d_idx=64 / k=1024) at the given N, so that a
+capture fits the profiler's size rules while the kernels are the benchmarked ones.
+Every launch is checked through the library's status block.
+"""
+import argparse
+import os
+import sys
+
+import torch
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+
+import tam_synth  # noqa: E402
+import top_attention_mass_b200 as tam  # noqa: E402
+
+ROWS = ("pass1_lse", "pass2_mass_topk", "pass2_block_mass_topk", "pass3_gather", "pass3_block",
+        "indexer_topk", "dense_prefill")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--row", choices=ROWS, required=True)
+    ap.add_argument("--N", type=int, default=16384)
+    ap.add_argument("--reps", type=int, default=3)
+    a = ap.parse_args()
+    w = tam_synth.WORKLOADS["indexer32k"]
+    inp = tam_synth.make_inputs(w, N=a.N)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    qx, kx = inp.q_idx.cuda(), inp.k_idx.cuda()
+    lse = tam.attention_lse(q, k)
+    s1 = tam.mass_select(q, k, lse, 655, 1)
+    s2 = tam.mass_select(q, k, lse, 655, 64)
+    for _ in range(a.reps):
+        if a.row == "pass1_lse":
+            tam.attention_lse(q, k)
+        elif a.row == "pass2_mass_topk":
+            tam.mass_select(q, k, lse, 655, 1)
+        elif a.row == "pass2_block_mass_topk":
+            tam.mass_select(q, k, lse, 655, 64)
+        elif a.row == "pass3_gather":
+            tam.sparse_support_attention(q, k, v, s1.idx, s1.length, 1)
+        elif a.row == "pass3_block":
+            tam.sparse_support_attention(q, k, v, s2.idx, s2.length, 64)
+        elif a.row == "indexer_topk":
+            tam.indexer_topk(qx, kx, 1024)
+        else:
+            tam.dense_gqa_prefill(q, k, v)
+    torch.cuda.synchronize()
+    print(f"profile_case {a.row} N={a.N} reps={a.reps} ok")
+
+
+if __name__ == "__main__":
+    main()
