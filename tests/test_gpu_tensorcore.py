@@ -106,3 +106,41 @@ def test_forced_candidate_overflow_is_reported(tam_lib, monkeypatch):
     monkeypatch.delenv("TAM_DEBUG_CAND_CAP")
     res = tam_lib.mass_select(q, k, lse, 40, 1)
     assert int(res.length[-1]) == 40
+
+
+@pytest.mark.parametrize("N,Hq,Hkv,d", [(129, 8, 8, 128), (700, 32, 2, 128), (450, 16, 8, 64),
+                                        (1000, 32, 8, 128), (257, 8, 1, 128), (3000, 16, 4, 128)])
+def test_dense_tensorcore_shapes(tam_lib, oracle_mod, N, Hq, Hkv, d):
+    inp = _inputs(N, Hq, Hkv, d, seed=N, sink=True, needles=3)
+    out, lse = tam_lib.dense_gqa_prefill(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), return_lse=True)
+    rows = tam_synth.sample_rows(N, inp.needle_i, n_random=64) if N > 1000 else None
+    ref, rl = oracle_mod.attn_rows(inp.q, inp.k, inp.v, rows)
+    got = out.float().cpu().numpy()
+    gl = lse.cpu().numpy().T
+    if rows is not None:
+        got, gl = got[rows], gl[rows]
+    check_close(got, ref, OUT_ATOL["bf16"], "dense")
+    check_close(gl, rl, LSE_ATOL, "dense lse")
+
+
+@pytest.mark.parametrize("N,Hq,Hkv,d,kb,bq", [
+    (600, 8, 8, 128, 50, 1), (600, 32, 2, 128, 50, 1), (500, 16, 8, 64, 33, 1),
+    (900, 32, 8, 128, 100, 64), (900, 16, 4, 128, 200, 128), (500, 8, 2, 128, 40, 8),
+    (400, 32, 2, 64, 60, 16), (300, 4, 4, 128, 17, 100)])
+def test_sparse_attention_gather_shapes(tam_lib, oracle_mod, N, Hq, Hkv, d, kb, bq):
+    """Pass 3 on a random support for every head-group size, per query and block-shared
+    (large blocks use the shared-chunk kernel, small ones the per-query gather)."""
+    inp = _inputs(N, Hq, Hkv, d, seed=kb)
+    n_sel = N if bq == 1 else -(-N // bq)
+    last = np.arange(n_sel) if bq == 1 else np.minimum(N - 1, (np.arange(n_sel) + 1) * bq - 1)
+    idx, ln = tam_synth.stress_support(N, kb, seed=3, rows=last)
+    out, lse = tam_lib.sparse_support_attention(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(),
+                                                torch.from_numpy(idx).cuda(),
+                                                torch.from_numpy(ln).cuda(), bq, return_lse=True)
+    if bq == 1:
+        rows, s, sl = np.arange(N), idx, ln
+    else:
+        rows, s, sl = oracle_mod.block_rows_support(idx, ln, bq, N)
+    ref, rl = oracle_mod.attn_rows(inp.q, inp.k, inp.v, rows, sup=s, sup_len=sl)
+    check_close(out.float().cpu().numpy()[rows], ref, OUT_ATOL["bf16"], "gather output")
+    check_close(lse.cpu().numpy().T[rows], rl, LSE_ATOL, "gather lse")

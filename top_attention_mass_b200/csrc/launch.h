@@ -77,6 +77,10 @@ int tc_mass_columns(const MassArgs& a);
 bool tc_mass_supported(const MassArgs& a);
 size_t tc_mass_block_bytes(int64_t N, int block_q);
 cudaError_t tc_mass_select(const MassArgs& a, cudaStream_t st);
+bool tc_dense_supported(const AttnArgs& a);
+cudaError_t tc_dense(const AttnArgs& a, cudaStream_t st);
+bool gather_supported(const AttnArgs& a);
+cudaError_t gather_attention(const AttnArgs& a, cudaStream_t st);
 
 // CUDA-core kernels (any dtype, any supported shape).
 cudaError_t simt_lse(const LseArgs& a, cudaStream_t st);

@@ -53,11 +53,17 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     return m;
 }
 
-// k-th largest key (non-negative float bits) among buf[0..n) by an MSB-first
-// 4 x 8-bit radix select over the warp.  Returns the key T and how many entries
-// equal to T belong to the top k (the earliest ones in buffer order).
-__device__ __forceinline__ void warp_kth(const uint2* buf, int n, int k, int* hist, uint32_t& T,
-                                         int& take_eq) {
+// Candidate buffer of one query: keys[cap] (mass as float bits; non-negative, so
+// the unsigned order is the float order) followed by idx[cap], in ascending key
+// index order.  Every pass over it batches kBatch loads per lane so the L2 latency
+// is paid once per batch, not once per entry.
+constexpr int kBatch = 8;
+
+// k-th largest of keys[0..n) by an MSB-first 4 x 8-bit radix select over the warp.
+// Returns the key T and how many entries equal to T belong to the top k (the
+// earliest ones in buffer order).
+__device__ __forceinline__ void warp_kth(const uint32_t* keys, int n, int k, int* hist,
+                                         uint32_t& T, int& take_eq) {
     const int lane = threadIdx.x & 31;
     uint32_t prefix = 0, mask = 0;
     int remaining = k;
@@ -65,9 +71,18 @@ __device__ __forceinline__ void warp_kth(const uint2* buf, int n, int k, int* hi
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int b = lane; b < 256; b += 32) hist[b] = 0;
         __syncwarp();
-        for (int e = lane; e < n; e += 32) {
-            const uint32_t key = buf[e].x;
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        for (int base = 0; base < n; base += 32 * kBatch) {
+            uint32_t kv[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int e = base + u * 32 + lane;
+                kv[u] = e < n ? keys[e] : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int e = base + u * 32 + lane;
+                if (e < n && (kv[u] & mask) == prefix) atomicAdd(&hist[(kv[u] >> shift) & 255u], 1);
+            }
         }
         __syncwarp();
         int c8[8], sum = 0;
@@ -105,60 +120,51 @@ __device__ __forceinline__ void warp_kth(const uint2* buf, int n, int k, int* hi
     take_eq = remaining;
 }
 
-// Stable in-place compaction of buf[0..n) to the entries with key > T plus the first
-// take_eq entries with key == T.  Returns the kept count.
-__device__ __forceinline__ int warp_compact(uint2* buf, int n, uint32_t T, int take_eq) {
+// Stable selection of the entries with key > T plus the first take_eq entries with
+// key == T (select_all: every entry).  Kept entries go, in order, either back into
+// the buffer (out_idx == null; positions never pass the read position, and a whole
+// batch is read before any of it is written) or to the output row, where the mass
+// is written as float.  Returns the kept count.
+__device__ __forceinline__ int warp_select(uint32_t* keys, uint32_t* idx, int n, uint32_t T,
+                                           int take_eq, bool select_all, int32_t* out_idx,
+                                           float* out_mass) {
     const int lane = threadIdx.x & 31;
     const uint32_t lt = lanemask_lt();
     int kept = 0, eq_seen = 0;
-    for (int base = 0; base < n; base += 32) {
-        const int e = base + lane;
-        uint2 x = make_uint2(0u, 0u);
-        if (e < n) x = buf[e];
-        const bool gt = e < n && x.x > T;
-        const bool eq = e < n && x.x == T;
-        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
-        const bool keep = gt || (eq && eq_seen + __popc(eqb & lt) < take_eq);
-        const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+    for (int base = 0; base < n; base += 32 * kBatch) {
+        uint32_t kv[kBatch], iv[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int e = base + u * 32 + lane;
+            kv[u] = e < n ? keys[e] : 0u;
+            iv[u] = e < n ? idx[e] : 0u;
+        }
         __syncwarp();
-        if (keep) buf[kept + __popc(kb & lt)] = x;
-        kept += __popc(kb);
-        eq_seen += __popc(eqb);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int e = base + u * 32 + lane;
+            const bool in = e < n;
+            const bool gt = in && (select_all || kv[u] > T);
+            const bool eq = in && !select_all && kv[u] == T;
+            const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+            const bool keep = gt || (eq && eq_seen + __popc(eqb & lt) < take_eq);
+            const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+            if (keep) {
+                const int pos = kept + __popc(kb & lt);
+                if (out_idx) {
+                    out_idx[pos] = (int32_t)iv[u];
+                    out_mass[pos] = __uint_as_float(kv[u]);
+                } else {
+                    keys[pos] = kv[u];
+                    idx[pos] = iv[u];
+                }
+            }
+            kept += __popc(kb);
+            eq_seen += __popc(eqb);
+        }
         __syncwarp();
     }
     return kept;
-}
-
-// Final write of one query's support: same selection as warp_compact, written to
-// the output rows (ascending key order is the buffer order), padded with -1 / 0.
-__device__ __forceinline__ void warp_emit(const uint2* buf, int n, uint32_t T, int take_eq,
-                                          bool select_all, int budget, int32_t* out_idx,
-                                          float* out_mass, int32_t* out_len) {
-    const int lane = threadIdx.x & 31;
-    const uint32_t lt = lanemask_lt();
-    int kept = 0, eq_seen = 0;
-    for (int base = 0; base < n; base += 32) {
-        const int e = base + lane;
-        uint2 x = make_uint2(0u, 0u);
-        if (e < n) x = buf[e];
-        const bool gt = e < n && (select_all || x.x > T);
-        const bool eq = e < n && !select_all && x.x == T;
-        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
-        const bool keep = gt || (eq && eq_seen + __popc(eqb & lt) < take_eq);
-        const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-        if (keep) {
-            const int p = kept + __popc(kb & lt);
-            out_idx[p] = (int32_t)x.y;
-            out_mass[p] = __uint_as_float(x.x);
-        }
-        kept += __popc(kb);
-        eq_seen += __popc(eqb);
-    }
-    for (int t = kept + lane; t < budget; t += 32) {
-        out_idx[t] = -1;
-        out_mass[t] = 0.f;
-    }
-    if (lane == 0) *out_len = kept;
 }
 
 struct MassParams {
@@ -168,7 +174,7 @@ struct MassParams {
     int32_t* sup_idx;
     int32_t* sup_len;
     float* sup_mass;
-    uint2* cand;                     // [N][cap] (per query)
+    uint32_t* cand;                  // [N][2*cap]: keys then idx (per query)
     unsigned long long* bmass;       // triangular block mass (block mode)
     int32_t* status;
     uint64_t timeout_ns;
@@ -417,7 +423,8 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 const int q = sw * QPW + a;
                 const int i = q0 + q;
                 if (i >= p.N) continue;
-                uint2* buf = p.cand + (size_t)i * p.cap;
+                uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
+                uint32_t* idxs = keys + p.cap;
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
                     const float v = mt[q * 128 + r * 32 + lane];
@@ -425,10 +432,12 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const uint32_t bal = __ballot_sync(0xffffffffu, pass);
                     const int pos = cnt[a] + __popc(bal & lanemask_lt());
                     if (pass) {
-                        if (pos < p.cap)
-                            buf[pos] = make_uint2(__float_as_uint(v), (uint32_t)(kt * 128 + r * 32 + lane));
-                        else
+                        if (pos < p.cap) {
+                            keys[pos] = __float_as_uint(v);
+                            idxs[pos] = (uint32_t)(kt * 128 + r * 32 + lane);
+                        } else {
                             overflow = true;
+                        }
                     }
                     cnt[a] += __popc(bal);
                 }
@@ -437,8 +446,8 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const int n = min(cnt[a], p.cap);
                     uint32_t T;
                     int take_eq;
-                    warp_kth(buf, n, p.budget, hist, T, take_eq);
-                    cnt[a] = warp_compact(buf, n, T, take_eq);
+                    warp_kth(keys, n, p.budget, hist, T, take_eq);
+                    cnt[a] = warp_select(keys, idxs, n, T, take_eq, false, nullptr, nullptr);
                     tau[a] = __uint_as_float(T);
                 }
             }
@@ -452,15 +461,22 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             for (int a = 0; a < QPW; ++a) {
                 const int i = q0 + sw * QPW + a;
                 if (i >= p.N) continue;
-                uint2* buf = p.cand + (size_t)i * p.cap;
+                uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
+                uint32_t* idxs = keys + p.cap;
                 const int n = min(cnt[a], p.cap);
                 __syncwarp();
                 uint32_t T = 0;
                 int take_eq = 0;
                 const bool all = n <= p.budget;
-                if (!all) warp_kth(buf, n, p.budget, hist, T, take_eq);
-                warp_emit(buf, n, T, take_eq, all, p.budget, p.sup_idx + (size_t)i * p.budget,
-                          p.sup_mass + (size_t)i * p.budget, p.sup_len + i);
+                if (!all) warp_kth(keys, n, p.budget, hist, T, take_eq);
+                int32_t* oi = p.sup_idx + (size_t)i * p.budget;
+                float* om = p.sup_mass + (size_t)i * p.budget;
+                const int kept = warp_select(keys, idxs, n, T, take_eq, all, oi, om);
+                for (int t = kept + lane; t < p.budget; t += 32) {
+                    oi[t] = -1;
+                    om[t] = 0.f;
+                }
+                if (lane == 0) p.sup_len[i] = kept;
             }
         }
     }
@@ -573,7 +589,7 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     p.sup_idx = a.sup_idx;
     p.sup_len = a.sup_len;
     p.sup_mass = a.sup_mass;
-    p.cand = reinterpret_cast<uint2*>(a.cand);
+    p.cand = reinterpret_cast<uint32_t*>(a.cand);
     p.bmass = reinterpret_cast<unsigned long long*>(a.bmass);
     p.status = a.status;
     p.timeout_ns = wait_timeout_ns();

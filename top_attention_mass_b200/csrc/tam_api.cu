@@ -99,6 +99,11 @@ IndexerPlan plan_indexer(int64_t N) {
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? TAM_OK : TAM_ERR_CUDA; }
 
+// Pass 3 with the gathered-row MMA kernels where built, else on the CUDA cores.
+cudaError_t run_sparse_attention(const AttnArgs& a, cudaStream_t st) {
+    return gather_supported(a) ? gather_attention(a, st) : simt_attention(a, st);
+}
+
 // Pass 1 on the tensor cores where the shape is built, else on the CUDA cores.
 cudaError_t run_lse(const LseArgs& a, cudaStream_t st) {
     return tc_lse_supported(a) ? tc_lse(a, st) : simt_lse(a, st);
@@ -188,7 +193,7 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
     if (out) {
         AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, sl2, sup_idx, sup_len, budget_k, block_q,
                     out, nullptr, status};
-        if ((rc = cuda_status(simt_attention(aa, st)))) return rc;
+        if ((rc = cuda_status(run_sparse_attention(aa, st)))) return rc;
     }
     return TAM_OK;
 }
@@ -295,7 +300,7 @@ int tam_sparse_support_attention(int64_t N, int Hq, int Hkv, int d, int dtype, c
     if ((rc = start_call(workspace, st))) return rc;
     AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, score_log2_scale(d), sup_idx, sup_len, kmax,
                 block_q, out, lse, (int32_t*)workspace};
-    return cuda_status(simt_attention(aa, st));
+    return cuda_status(run_sparse_attention(aa, st));
 }
 
 size_t tam_dense_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {
@@ -317,7 +322,7 @@ int tam_dense_gqa_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const vo
     if ((rc = start_call(workspace, st))) return rc;
     AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, score_log2_scale(d), nullptr, nullptr, 0, 1,
                 out, lse, (int32_t*)workspace};
-    return cuda_status(simt_attention(aa, st));
+    return cuda_status(tc_dense_supported(aa) ? tc_dense(aa, st) : simt_attention(aa, st));
 }
 
 int tam_check_status(const void* workspace, void* stream, int32_t* detail) {
