@@ -120,6 +120,27 @@ int tam_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
                     void* stream);
 
 /*
+ * Pass 2 without a caller-provided workspace.  The paper has no counterpart: this
+ * is a library service for callers that cannot allocate device memory (a plugin
+ * whose host engine owns all device memory and hands it only its input and output
+ * tensors; a process that must not call cudaMalloc while serving, because it can
+ * synchronise the device and fail under fragmentation).
+ * Same arguments, semantics and outputs as tam_mass_select, minus the workspace:
+ * the scratch is a 64 MiB static device array inside the library.  Problems whose
+ * tam_mass_select_workspace() exceeds 64 MiB are rejected with TAM_ERR_WORKSPACE
+ * before anything is enqueued.  Nothing is allocated.  The first call on a device
+ * looks up the array's device address (with that device current), so make that
+ * first call before any stream capture.  The call waits for `stream` and returns
+ * the device status (TAM_OK, TAM_ERR_TIMEOUT, TAM_ERR_OVERFLOW).  All calls in the
+ * process share the one array per device and it keeps the last call's contents:
+ * calls that can overlap on the GPU (other streams, other threads) race and must
+ * be serialised by the caller.  A GPU keeps the array until the process exits.
+ */
+int tam_mass_select_noalloc(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
+                            const void* k, const float* lse, int budget_k, int block_q,
+                            int32_t* sup_idx, int32_t* sup_len, float* sup_mass, void* stream);
+
+/*
  * Head-collapsed indexer support (technical report §2.2 "Head-Collapsed Indexer":
  * one token score shared by all heads, top-k of it):
  *   score[i,j] = q_idx[i] . k_idx[j] for j <= i (no scale: ranking only),

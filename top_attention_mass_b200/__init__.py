@@ -38,7 +38,7 @@ TAM_BF16, TAM_F32 = 0, 1
 EXPORTED = (
     "tam_version", "tam_status_string", "tam_mass_oracle_workspace", "tam_mass_oracle_prefill",
     "tam_attention_lse_workspace", "tam_attention_lse", "tam_mass_select_workspace",
-    "tam_mass_select", "tam_indexer_workspace",
+    "tam_mass_select", "tam_mass_select_noalloc", "tam_indexer_workspace",
     "tam_indexer_topk", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
     "tam_dense_workspace", "tam_dense_gqa_prefill", "tam_kernel_launches", "tam_check_status",
 )
@@ -86,6 +86,9 @@ def lib() -> ctypes.CDLL:
         L.tam_mass_select.restype = i32
         L.tam_mass_select.argtypes = [i64, i32, i32, i32, i32, p, p, p, i32, i32, p, p, p, p, sz,
                                       p]
+        L.tam_mass_select_noalloc.restype = i32
+        L.tam_mass_select_noalloc.argtypes = [i64, i32, i32, i32, i32, p, p, p, i32, i32, p, p, p,
+                                              p]
         L.tam_indexer_workspace.restype = sz
         L.tam_indexer_workspace.argtypes = [i64, i32, i32, i32, i32]
         L.tam_indexer_topk.restype = i32
