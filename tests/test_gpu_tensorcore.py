@@ -144,3 +144,41 @@ def test_sparse_attention_gather_shapes(tam_lib, oracle_mod, N, Hq, Hkv, d, kb, 
     ref, rl = oracle_mod.attn_rows(inp.q, inp.k, inp.v, rows, sup=s, sup_len=sl)
     check_close(out.float().cpu().numpy()[rows], ref, OUT_ATOL["bf16"], "gather output")
     check_close(lse.cpu().numpy().T[rows], rl, LSE_ATOL, "gather lse")
+
+
+def test_indexer_ties_keep_smallest_indices(tam_lib):
+    """q_idx = 0 makes every score 0: the smallest key indices must be chosen."""
+    N, kb = 900, 40
+    inp = _inputs(N, 8, 2, 128, seed=3)
+    qx, kx = tam_synth.indexer_projections(inp, 64, seed=2)
+    qx = torch.zeros_like(qx)
+    res = tam_lib.indexer_topk(qx.cuda(), kx.cuda(), kb)
+    gi, gl, gs = res.idx.cpu().numpy(), res.length.cpu().numpy(), res.value.cpu().numpy()
+    for i in range(N):
+        n = min(kb, i + 1)
+        assert gl[i] == n and list(gi[i, :n]) == list(range(n)) and np.all(gs[i, :n] == 0)
+
+
+@pytest.mark.parametrize("N,kb", [(3000, 4), (2500, 300)])
+def test_indexer_heavy_compaction(tam_lib, oracle_mod, N, kb):
+    inp = _inputs(N, 8, 2, 128, seed=kb, sink=True, needles=5)
+    qx, kx = tam_synth.indexer_projections(inp, 64, seed=2)
+    res = tam_lib.indexer_topk(qx.cuda(), kx.cuda(), kb)
+    rows = tam_synth.sample_rows(N, inp.needle_i, n_random=80)
+    oi, ol, _ = oracle_mod.indexer_topk_rows(qx, kx, kb, rows)
+    S = qx.double().numpy()[rows] @ kx.double().numpy().T
+    check_support(res.idx.cpu().numpy()[rows], res.length.cpu().numpy()[rows],
+                  res.value.cpu().numpy()[rows], oi, ol, S, 1e-3, "indexer compaction")
+
+
+def test_indexer_forced_timeout_is_reported(tam_lib, monkeypatch):
+    inp = _inputs(400, 8, 2, 128, seed=9)
+    qx, kx = tam_synth.indexer_projections(inp, 64, seed=2)
+    qx, kx = qx.cuda(), kx.cuda()
+    monkeypatch.setenv("TAM_DEBUG_FORCE_TIMEOUT", "1")
+    with pytest.raises(tam_lib.TamError) as e:
+        tam_lib.indexer_topk(qx, kx, 32)
+    assert e.value.code == tam_lib.TAM_ERR_TIMEOUT
+    monkeypatch.delenv("TAM_DEBUG_FORCE_TIMEOUT")
+    res = tam_lib.indexer_topk(qx, kx, 32)
+    assert int(res.length[-1]) == 32

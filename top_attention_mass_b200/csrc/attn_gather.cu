@@ -107,6 +107,32 @@ __device__ __forceinline__ void issue_chunk(uint32_t buf, const __nv_bfloat16* k
     }
 }
 
+// Warp version of issue_chunk: the chunk's kChunk support indices are read once
+// (one lane each) and broadcast; every lane keeps one 16-byte column `pc` of the
+// rows and issues the K and V copies of each of its rows from one row offset.
+template <int D>
+__device__ __forceinline__ void issue_chunk_warp(uint32_t buf, const __nv_bfloat16* k,
+                                                 const __nv_bfloat16* v, int Hkv, int g,
+                                                 const int32_t* srow, int t_base, int n) {
+    constexpr int RB = D * 2;
+    constexpr int PC = RB / 16;          // 16-byte pieces per row
+    constexpr int RPP = 32 / PC;         // rows covered by one pass of the warp
+    const int lane = threadIdx.x & 31;
+    const int pc = lane % PC, r0 = lane / PC;
+    int jl = -1;
+    if (lane < kChunk && t_base + lane < n) jl = srow[t_base + lane];
+#pragma unroll
+    for (int u = 0; u < kChunk / RPP; ++u) {
+        const int r = u * RPP + r0;
+        const int j = __shfl_sync(0xffffffffu, jl, r);
+        const bool valid = j >= 0;
+        const size_t off = valid ? ((size_t)j * Hkv + g) * D + pc * 8 : 0;
+        const uint32_t dst = buf + swz<RB>(r, pc);
+        cp_async16(dst, k + off, valid);
+        cp_async16(dst + kChunk * RB, v + off, valid);
+    }
+}
+
 // One chunk of keys for one 16-row MMA tile: S = Q K^T (2 n-tiles of 8 keys),
 // masked online softmax (base 2), O += P V.  qa: A fragments of Q (a0..a3 per
 // k-step).  valid(key slot r, row half) decides the mask.  ROW8: rows 8..15 live.
@@ -249,7 +275,7 @@ k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     constexpr int STAGE = 2 * kChunk * RB;
     constexpr bool ROW8 = G > 8;
     extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const uint32_t wbuf = smem_addr(smem) + warp * STAGES * STAGE;
     const int64_t total = (int64_t)N * Hkv;
     for (int64_t item = (int64_t)blockIdx.x * 8 + warp; item < total; item += (int64_t)gridDim.x * 8) {
@@ -275,14 +301,13 @@ k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         const int nch = (n + kChunk - 1) / kChunk;
 #pragma unroll
         for (int s = 0; s < STAGES - 1; ++s) {
-            if (s < nch) issue_chunk<D>(wbuf + s * STAGE, k, v, Hkv, g, srow, s * kChunk, n, lane, 32);
+            if (s < nch) issue_chunk_warp<D>(wbuf + s * STAGE, k, v, Hkv, g, srow, s * kChunk, n);
             cp_async_commit();
         }
         for (int ch = 0; ch < nch; ++ch) {
             const int nx = ch + STAGES - 1;
             if (nx < nch)
-                issue_chunk<D>(wbuf + (nx % STAGES) * STAGE, k, v, Hkv, g, srow, nx * kChunk, n,
-                               lane, 32);
+                issue_chunk_warp<D>(wbuf + (nx % STAGES) * STAGE, k, v, Hkv, g, srow, nx * kChunk, n);
             cp_async_commit();
             cp_async_wait<STAGES - 1>();
             __syncwarp();

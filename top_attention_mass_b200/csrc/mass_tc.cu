@@ -20,11 +20,13 @@
 //               heads -> mass of BQ queries; causal mask; then either the mass tile
 //               goes to shared memory for the select warps (per query) or the
 //               block column sum is added in 2^-40 fixed point (block-shared);
-//   warps 6-9   select warps (per query): each owns BQ/4 queries and runs a streaming
-//               exact top-k: strict threshold tau plus a candidate buffer in global
-//               memory, appended in ascending key order, compacted by a warp radix
-//               select when it fills (keeps exactly k; ties keep the smaller index),
-//               and written ascending at the end.
+//   warps 6-11  select warps (per query): each owns every 6th query of the tile and
+//               runs a streaming exact top-k: a threshold tau plus a candidate buffer
+//               in global memory, appended in ascending key order.  When the buffer
+//               fills, a 2-pass warp radix select finds the 16-bit bin of the k-th
+//               value and drops everything below it (an exact 4-pass select keeps
+//               exactly k when the bin is too crowded); the final emit is exact
+//               (equal values keep the smaller index) and comes out ascending.
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
@@ -33,7 +35,22 @@ namespace tam {
 namespace {
 
 constexpr int kStages = 2;
-constexpr int kThreads = 320;
+constexpr int kSelWarps = 6;                 // warps 6..11
+constexpr int kThreads = 32 * (6 + kSelWarps);
+
+// Kernel modes: head-averaged mass with per-query top-k, block-shared mass sums,
+// or the head-collapsed indexer (one score per (query, key), no exponentials).
+constexpr int kModeQuery = 0, kModeBlock = 1, kModeIndexer = 2;
+
+// Order-preserving map float -> uint32 and back (a < b <=> key(a) < key(b)), so
+// candidate keys of any sign sort as unsigned integers.
+__device__ __forceinline__ uint32_t key_of(float v) {
+    const uint32_t b = __float_as_uint(v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float value_of(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
 
 struct SelWarpSmem {
     int hist[256];
@@ -43,7 +60,7 @@ struct SelWarpSmem {
 // select warps' histograms.
 __host__ __device__ constexpr int mass_smem_bytes(int NQ, int D, int Hkv, int G, bool block) {
     return 1024 + Hkv * NQ * D * 2 + kStages * 128 * D * 2 + Hkv * NQ * 4 + 512 +
-           (block ? 0 : 2 * (NQ / G) * 128 * 4 + 4 * (int)sizeof(SelWarpSmem));
+           (block ? 0 : 2 * (NQ / G) * 128 * 4 + kSelWarps * (int)sizeof(SelWarpSmem));
 }
 constexpr int kMaxDynSmem = 227 * 1024;
 
@@ -53,22 +70,23 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     return m;
 }
 
-// Candidate buffer of one query: keys[cap] (mass as float bits; non-negative, so
-// the unsigned order is the float order) followed by idx[cap], in ascending key
-// index order.  Every pass over it batches kBatch loads per lane so the L2 latency
+// Candidate buffer of one query: keys[cap] (key_of(value)) followed by idx[cap],
+// in ascending key index order.  Every pass over it batches kBatch loads per lane so the L2 latency
 // is paid once per batch, not once per entry.
 constexpr int kBatch = 8;
 
 // k-th largest of keys[0..n) by an MSB-first 4 x 8-bit radix select over the warp.
 // Returns the key T and how many entries equal to T belong to the top k (the
 // earliest ones in buffer order).
+// With passes < 4 the result is the k-th key's leading 8*passes bits (low bits zero):
+// every key >= T is then at least the k-th largest's bin, and there are >= k of them.
 __device__ __forceinline__ void warp_kth(const uint32_t* keys, int n, int k, int* hist,
-                                         uint32_t& T, int& take_eq) {
+                                         uint32_t& T, int& take_eq, int passes = 4) {
     const int lane = threadIdx.x & 31;
     uint32_t prefix = 0, mask = 0;
     int remaining = k;
 #pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int shift = 24; shift >= 32 - 8 * passes; shift -= 8) {
         for (int b = lane; b < 256; b += 32) hist[b] = 0;
         __syncwarp();
         for (int base = 0; base < n; base += 32 * kBatch) {
@@ -123,7 +141,7 @@ __device__ __forceinline__ void warp_kth(const uint32_t* keys, int n, int k, int
 // Stable selection of the entries with key > T plus the first take_eq entries with
 // key == T (select_all: every entry).  Kept entries go, in order, either back into
 // the buffer (out_idx == null; positions never pass the read position, and a whole
-// batch is read before any of it is written) or to the output row, where the mass
+// batch is read before any of it is written) or to the output row, where the value
 // is written as float.  Returns the kept count.
 __device__ __forceinline__ int warp_select(uint32_t* keys, uint32_t* idx, int n, uint32_t T,
                                            int take_eq, bool select_all, int32_t* out_idx,
@@ -153,7 +171,7 @@ __device__ __forceinline__ int warp_select(uint32_t* keys, uint32_t* idx, int n,
                 const int pos = kept + __popc(kb & lt);
                 if (out_idx) {
                     out_idx[pos] = (int32_t)iv[u];
-                    out_mass[pos] = __uint_as_float(kv[u]);
+                    out_mass[pos] = value_of(kv[u]);
                 } else {
                     keys[pos] = kv[u];
                     idx[pos] = iv[u];
@@ -186,7 +204,7 @@ __host__ __device__ __forceinline__ int64_t bmass_offset(int64_t b, int block_q)
     return (int64_t)block_q * b * (b + 1) / 2;
 }
 
-template <int G, int D, int NQ, bool BLOCK>
+template <int G, int D, int NQ, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const MassParams p) {
@@ -196,7 +214,9 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     constexpr uint32_t kQHalf = NQ * 128; // bytes of one 64-element half of a group's Q
     constexpr uint32_t kKHalf = 128 * 128;
     constexpr uint32_t kKTile = NH * kKHalf;
-    constexpr int QPW = BQ / 4;           // queries per select warp
+    constexpr int QPW = (BQ + kSelWarps - 1) / kSelWarps;   // queries per select warp (at most)
+    constexpr bool BLOCK = MODE == kModeBlock;
+    constexpr bool INDEXER = MODE == kModeIndexer;
     const int Hkv = p.Hkv;
 
     extern __shared__ uint8_t smem_raw[];
@@ -207,7 +227,7 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     float* sLse = reinterpret_cast<float*>(sK + kStages * kKTile);   // Hkv * NQ
     float* sMass = sLse + Hkv * NQ;                                    // 2 x BQ x 128 (per query)
     SelWarpSmem* sSel = reinterpret_cast<SelWarpSmem*>(sMass + (BLOCK ? 0 : 2 * BQ * 128));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + (BLOCK ? 0 : 4));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + (BLOCK ? 0 : kSelWarps));
     uint64_t* q_full = bars;
     uint64_t* k_full = q_full + 1;
     uint64_t* k_empty = k_full + kStages;
@@ -239,7 +259,7 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&m_full[b], 128);
-            tc::mbar_init(&m_empty[b], 128);
+            tc::mbar_init(&m_empty[b], 32 * kSelWarps);
         }
         tc::mbar_init(mma_done, 1);
         tc::mbar_init(never, 1);
@@ -247,10 +267,12 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         tc::fence_barrier_init();
     }
     // log2-domain LSE of every column of every group (+inf for padding queries)
-    for (int t = threadIdx.x; t < Hkv * NQ; t += blockDim.x) {
-        const int g = t / NQ, c = t % NQ;
-        const int i = q0 + c / G, h = g * G + c % G;
-        sLse[t] = (i < p.N) ? p.lse[(size_t)h * p.N + i] * kLog2e : INFINITY;
+    if constexpr (!INDEXER) {
+        for (int t = threadIdx.x; t < Hkv * NQ; t += blockDim.x) {
+            const int g = t / NQ, c = t % NQ;
+            const int i = q0 + c / G, h = g * G + c % G;
+            sLse[t] = (i < p.N) ? p.lse[(size_t)h * p.N + i] * kLog2e : INFINITY;
+        }
     }
     if (warp == 0) {
         tc::tmem_alloc(tmem_slot, 512);
@@ -260,7 +282,8 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const tc::Guard gd{abort_flag, p.status, BLOCK ? KID_BLOCK_MASS_TC : KID_MASS_TC,
+    const tc::Guard gd{abort_flag, p.status,
+                       BLOCK ? KID_BLOCK_MASS_TC : (INDEXER ? KID_INDEXER_TC : KID_MASS_TC),
                        p.timeout_ns};
 
     if (warp == 4) {
@@ -347,16 +370,22 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     uint32_t (&cur)[32] = (c & 1) ? vb : va;
                     uint32_t (&nxt)[32] = (c & 1) ? va : vb;
                     if (c + 1 < NQ / 32) tc::tmem_ld32(col0 + (c + 1) * 32, nxt);
-                    const float4* l4 = reinterpret_cast<const float4*>(sLse + g * NQ + c * 32);
+                    if constexpr (INDEXER) {
+                        // one column per query: the raw indexer score
 #pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 L = l4[c4];
-                        const float Ls[4] = {L.x, L.y, L.z, L.w};
+                        for (int e = 0; e < 32; ++e) acc[c * 32 + e] = __uint_as_float(cur[e]);
+                    } else {
+                        const float4* l4 = reinterpret_cast<const float4*>(sLse + g * NQ + c * 32);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int col = c * 32 + c4 * 4 + e;
-                            const float sc = __uint_as_float(cur[c4 * 4 + e]);
-                            acc[col / G] += tc::ex2(fmaf(sc, p.sl2, -Ls[e]));
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            const float4 L = l4[c4];
+                            const float Ls[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int col = c * 32 + c4 * 4 + e;
+                                const float sc = __uint_as_float(cur[c4 * 4 + e]);
+                                acc[col / G] += tc::ex2(fmaf(sc, p.sl2, -Ls[e]));
+                            }
                         }
                     }
                     if (c + 1 < NQ / 32) tc::tmem_wait_ld(nxt);
@@ -373,7 +402,8 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
                 for (int q = 0; q < BQ; ++q) {
                     const int i = q0 + q;
-                    mt[q * 128 + row] = (j <= i && i < p.N) ? acc[q] * p.inv_hq : -1.f;
+                    mt[q * 128 + row] = (j <= i && i < p.N) ? (INDEXER ? acc[q] : acc[q] * p.inv_hq)
+                                                            : -INFINITY;
                 }
                 tc::mbar_arrive(&m_full[mb]);
             } else {
@@ -405,11 +435,12 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         // ---------------------------------------------------------------- select warps
         const int sw = warp - 6;
         int* hist = sSel[sw].hist;
+        // select warp sw owns queries sw, sw + kSelWarps, ... of the tile
         float tau[QPW];
         int cnt[QPW];
 #pragma unroll
         for (int a = 0; a < QPW; ++a) {
-            tau[a] = -1.f;
+            tau[a] = -INFINITY;     // masked entries are -inf and never pass
             cnt[a] = 0;
         }
         bool ok = true;
@@ -420,9 +451,9 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             const float* mt = sMass + mb * BQ * 128;
 #pragma unroll
             for (int a = 0; a < QPW; ++a) {
-                const int q = sw * QPW + a;
+                const int q = sw + a * kSelWarps;
                 const int i = q0 + q;
-                if (i >= p.N) continue;
+                if (q >= BQ || i >= p.N) continue;
                 uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
                 uint32_t* idxs = keys + p.cap;
 #pragma unroll
@@ -433,7 +464,7 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const int pos = cnt[a] + __popc(bal & lanemask_lt());
                     if (pass) {
                         if (pos < p.cap) {
-                            keys[pos] = __float_as_uint(v);
+                            keys[pos] = key_of(v);
                             idxs[pos] = (uint32_t)(kt * 128 + r * 32 + lane);
                         } else {
                             overflow = true;
@@ -446,21 +477,32 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     const int n = min(cnt[a], p.cap);
                     uint32_t T;
                     int take_eq;
-                    warp_kth(keys, n, p.budget, hist, T, take_eq);
-                    cnt[a] = warp_select(keys, idxs, n, T, take_eq, false, nullptr, nullptr);
-                    tau[a] = __uint_as_float(T);
+                    // cheap first: keep every key in the k-th key's 16-bit bin or above
+                    warp_kth(keys, n, p.budget, hist, T, take_eq, 2);
+                    int kept = n;
+                    if (T > 0u) kept = warp_select(keys, idxs, n, T - 1u, 0, false, nullptr, nullptr);
+                    if (kept > p.cap - 256) {
+                        // the bin was too crowded to free space: exact, keeps exactly k
+                        warp_kth(keys, kept, p.budget, hist, T, take_eq, 4);
+                        kept = warp_select(keys, idxs, kept, T, take_eq, false, nullptr, nullptr);
+                        tau[a] = fmaxf(tau[a], value_of(T));   // accept key > T
+                    } else if (T > 0u) {
+                        tau[a] = fmaxf(tau[a], value_of(T - 1u));   // accept key >= T
+                    }
+                    cnt[a] = kept;
                 }
             }
             __syncwarp();
             tc::mbar_arrive(&m_empty[mb]);
         }
         if (__any_sync(0xffffffffu, overflow) && lane == 0)
-            report_error(p.status, TAM_ERR_OVERFLOW, KID_MASS_TC, q0);
+            report_error(p.status, TAM_ERR_OVERFLOW, INDEXER ? KID_INDEXER_TC : KID_MASS_TC, q0);
         if (ok) {
 #pragma unroll
             for (int a = 0; a < QPW; ++a) {
-                const int i = q0 + sw * QPW + a;
-                if (i >= p.N) continue;
+                const int q = sw + a * kSelWarps;
+                const int i = q0 + q;
+                if (q >= BQ || i >= p.N) continue;
                 uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
                 uint32_t* idxs = keys + p.cap;
                 const int n = min(cnt[a], p.cap);
@@ -567,9 +609,10 @@ __global__ void __launch_bounds__(256) k_block_select(const unsigned long long* 
     if (tid == 0) sup_len[b] = m;
 }
 
-template <int G, int D, int NQ, bool BLOCK>
+template <int G, int D, int NQ, int MODE>
 cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     constexpr int BQ = NQ / G;
+    constexpr bool BLOCK = MODE == kModeBlock;
     CUtensorMap tq, tk;
     const uint64_t d = a.d;
     if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQ) ||
@@ -595,7 +638,7 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     p.timeout_ns = wait_timeout_ns();
     p.dbg = debug_flags();
     const int smem = mass_smem_bytes(NQ, D, a.Hkv, G, BLOCK);
-    auto kern = k_mass_tc<G, D, NQ, BLOCK>;
+    auto kern = k_mass_tc<G, D, NQ, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     if (BLOCK) {
@@ -615,39 +658,45 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
 }
 
 // Only (G, NQ) pairs with 4..32 queries per CTA are instantiated.
-template <int G, int D, int NQ, bool BLOCK>
+template <int G, int D, int NQ, int MODE>
 cudaError_t launch_if_valid(const MassArgs& a, cudaStream_t st) {
-    if constexpr (NQ / G >= 4 && NQ / G <= 32 && (NQ / G) % 4 == 0)
-        return launch_mass<G, D, NQ, BLOCK>(a, st);
+    if constexpr (NQ / G >= 4 && NQ / G <= 32)
+        return launch_mass<G, D, NQ, MODE>(a, st);
     else
         return cudaErrorNotSupported;
 }
 
-template <int D, int NQ, bool BLOCK>
+template <int D, int NQ, int MODE>
 cudaError_t dispatch_g(const MassArgs& a, cudaStream_t st) {
     switch (a.Hq / a.Hkv) {
-        case 1: return launch_if_valid<1, D, NQ, BLOCK>(a, st);
-        case 2: return launch_if_valid<2, D, NQ, BLOCK>(a, st);
-        case 4: return launch_if_valid<4, D, NQ, BLOCK>(a, st);
-        case 8: return launch_if_valid<8, D, NQ, BLOCK>(a, st);
-        case 16: return launch_if_valid<16, D, NQ, BLOCK>(a, st);
+        case 1: return launch_if_valid<1, D, NQ, MODE>(a, st);
+        case 2: return launch_if_valid<2, D, NQ, MODE>(a, st);
+        case 4: return launch_if_valid<4, D, NQ, MODE>(a, st);
+        case 8: return launch_if_valid<8, D, NQ, MODE>(a, st);
+        case 16: return launch_if_valid<16, D, NQ, MODE>(a, st);
         default: return cudaErrorNotSupported;
     }
 }
 
-template <int D, bool BLOCK>
+template <int D, int MODE>
 cudaError_t dispatch_nq(const MassArgs& a, cudaStream_t st) {
     switch (tc_mass_columns(a)) {
-        case 128: return dispatch_g<D, 128, BLOCK>(a, st);
-        case 64: return dispatch_g<D, 64, BLOCK>(a, st);
-        case 32: return dispatch_g<D, 32, BLOCK>(a, st);
+        case 128: return dispatch_g<D, 128, MODE>(a, st);
+        case 64: return dispatch_g<D, 64, MODE>(a, st);
+        case 32: return dispatch_g<D, 32, MODE>(a, st);
         default: return cudaErrorNotSupported;
     }
 }
 
-template <bool BLOCK>
+template <int MODE>
 cudaError_t dispatch(const MassArgs& a, cudaStream_t st) {
-    return a.d == 64 ? dispatch_nq<64, BLOCK>(a, st) : dispatch_nq<128, BLOCK>(a, st);
+    return a.d == 64 ? dispatch_nq<64, MODE>(a, st) : dispatch_nq<128, MODE>(a, st);
+}
+
+// The indexer runs as a single-head problem: Hq = Hkv = 1, d = d_idx, 32 queries per CTA.
+cudaError_t launch_indexer_tc(const MassArgs& a, cudaStream_t st) {
+    return a.d == 64 ? launch_mass<1, 64, 32, kModeIndexer>(a, st)
+                     : launch_mass<1, 128, 32, kModeIndexer>(a, st);
 }
 
 }  // namespace
@@ -673,7 +722,6 @@ bool tc_mass_supported(const MassArgs& a) {
     const int nq = tc_mass_columns(a);
     if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128) || nq == 0) return false;
     if (!(G == 1 || G == 2 || G == 4 || G == 8 || G == 16)) return false;
-    if ((nq / G) % 4 != 0) return false;                      // whole queries per select warp
     if (a.block_q > 1 && a.block_q > (1 << 20)) return false;
     return true;
 }
@@ -684,7 +732,31 @@ size_t tc_mass_block_bytes(int64_t N, int block_q) {
 }
 
 cudaError_t tc_mass_select(const MassArgs& a, cudaStream_t st) {
-    return a.block_q == 1 ? dispatch<false>(a, st) : dispatch<true>(a, st);
+    return a.block_q == 1 ? dispatch<kModeQuery>(a, st) : dispatch<kModeBlock>(a, st);
+}
+
+bool tc_indexer_supported(int64_t N, int d_idx, int dtype, int block_q) {
+    return dtype == TAM_BF16 && (d_idx == 64 || d_idx == 128) && block_q == 1 && N >= 1;
+}
+
+cudaError_t tc_indexer_select(const IndexerArgs& ia, cudaStream_t st) {
+    MassArgs a{};
+    a.N = ia.N;
+    a.Hq = 1;
+    a.Hkv = 1;
+    a.d = ia.d_idx;
+    a.dtype = ia.dtype;
+    a.q = ia.q_idx;
+    a.k = ia.k_idx;
+    a.budget = ia.budget;
+    a.block_q = 1;
+    a.cand = ia.cand;
+    a.cand_cap = ia.cand_cap;
+    a.sup_idx = ia.sup_idx;
+    a.sup_len = ia.sup_len;
+    a.sup_mass = ia.sup_score;
+    a.status = ia.status;
+    return launch_indexer_tc(a, st);
 }
 
 }  // namespace tam

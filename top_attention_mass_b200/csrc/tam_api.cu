@@ -84,16 +84,22 @@ MassPlan plan_mass(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k, i
     return p;
 }
 
+// Workspace of tam_indexer_topk: status block, then the candidate buffers of the
+// tensor-core path or the staged score rows of the CUDA-core path.
 struct IndexerPlan {
     size_t off_scratch, total;
-    int n_ctas;
+    bool tc;
+    int n_ctas, cand_cap;
 };
 
-IndexerPlan plan_indexer(int64_t N) {
-    IndexerPlan p;
+IndexerPlan plan_indexer(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
+    IndexerPlan p{};
+    p.tc = tc_indexer_supported(N, d_idx, dtype, block_q);
     p.n_ctas = (int)std::min<int64_t>(N, kSimtPersistentCtas);
+    p.cand_cap = candidate_capacity(budget_k);
     p.off_scratch = kStatusBytes;
-    p.total = p.off_scratch + align256((size_t)p.n_ctas * N * sizeof(float));
+    const size_t work = p.tc ? (size_t)N * p.cand_cap * 8 : (size_t)p.n_ctas * N * sizeof(float);
+    p.total = p.off_scratch + align256(work);
     return p;
 }
 
@@ -248,7 +254,7 @@ size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int 
     if (N < 1 || (d_idx != 16 && d_idx != 32 && d_idx != 64 && d_idx != 128)) return 0;
     if (dtype != TAM_BF16 && dtype != TAM_F32) return 0;
     if (check_budget(N, budget_k, block_q) != TAM_OK || block_q != 1) return 0;
-    return plan_indexer(N).total;
+    return plan_indexer(N, d_idx, dtype, budget_k, block_q).total;
 }
 
 int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const void* k_idx,
@@ -265,7 +271,7 @@ int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const v
     const void* ptrs[] = {q_idx, k_idx, sup_idx, sup_len, sup_score, workspace};
     for (const void* p : ptrs)
         if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
-    const IndexerPlan plan = plan_indexer(N);
+    const IndexerPlan plan = plan_indexer(N, d_idx, dtype, budget_k, block_q);
     if (ws_bytes < plan.total) return TAM_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     char* ws = (char*)workspace;
@@ -273,9 +279,10 @@ int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const v
     IndexerArgs ia{};
     ia.N = N; ia.d_idx = d_idx; ia.dtype = dtype; ia.q_idx = q_idx; ia.k_idx = k_idx;
     ia.budget = budget_k; ia.n_ctas = plan.n_ctas; ia.scratch = (float*)(ws + plan.off_scratch);
+    ia.cand = ws + plan.off_scratch; ia.cand_cap = plan.cand_cap;
     ia.sup_idx = sup_idx; ia.sup_len = sup_len; ia.sup_score = sup_score;
     ia.status = (int32_t*)ws;
-    return cuda_status(simt_indexer_select(ia, st));
+    return cuda_status(plan.tc ? tc_indexer_select(ia, st) : simt_indexer_select(ia, st));
 }
 
 size_t tam_sparse_attention_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {
