@@ -210,16 +210,44 @@ def algorithmic_work(w, N, outs):
     }
 
 
-def roofline_of(work, ms, pk, pk_kind):
+# Random 256-byte row gather from a 140 MB table (the 32K layer's K+V is 134 MB), measured
+# on this machine's B200 with CUDA events (profiles/probe_b200_memory_and_mufu.md): the rate
+# an L2-resident gather can reach, given next to the HBM copy peak for the gather rows.
+L2_GATHER_GBS = 11074.1
+
+
+def traffic_table():
+    """DRAM bytes per launch from the committed ncu capture, for rows whose kernel source
+    is unchanged since the capture (sha256 match); other rows get None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_dram_traffic_gqa32k_step.json")
+    try:
+        with open(path) as f:
+            tab = json.load(f)["rows"]
+    except Exception:
+        return {}
+    out = {}
+    for row, ent in tab.items():
+        try:
+            with open(os.path.join(ROOT, ent["source"]), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() == ent["sha256"]:
+                    out[row] = ent["dram_bytes_per_launch"]
+        except Exception:
+            pass
+    return out
+
+
+def roofline_of(work, ms, pk, pk_kind, traffic=None):
     tf_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     if work["bound"] == "tensor":
         ach = work["flops"] / (ms * 1e-3) / 1e12
         return {"bound": "tensor", "achieved": ach, "peak": tf_peak, "unit": "TFLOP/s",
-                "frac": ach / tf_peak, "traffic": None,
+                "frac": ach / tf_peak, "traffic": traffic,
                 "peak_kind": f"bf16 dense, sustained, of {pk_kind}"}
     ach = work["bytes"] / (ms * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_kind": f"HBM copy, of {pk_kind}"}
+            "frac": ach / pk["hbm_gbs"], "traffic": traffic, "peak_kind": f"HBM copy, of {pk_kind}",
+            "l2_gather_peak": L2_GATHER_GBS, "frac_of_l2_gather_peak": ach / L2_GATHER_GBS}
 
 
 # ------------------------------------------------------------------ oracle (CPU) arm
@@ -355,9 +383,10 @@ def run_ours(args, w, inp, rank, world, local_rank):
               for i, n in enumerate(Step.NAMES)}
 
     pk, pk_kind = peaks()
+    traffic = traffic_table()
     rows = {}
     for n in Step.NAMES:
-        r = roofline_of(work[n], row_ms[n], pk, pk_kind)
+        r = roofline_of(work[n], row_ms[n], pk, pk_kind, traffic.get(n))
         rows[n] = {"ms": row_ms[n], "q_tok_s": w.N / (row_ms[n] * 1e-3), "roofline": r}
     dominant = max(Step.NAMES, key=lambda n: row_ms[n])
 
