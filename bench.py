@@ -128,86 +128,115 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the device step
 
+ROWS_ALL = ("pass1_lse", "pass2_mass_topk", "pass3_gather", "pass2_block_mass_topk",
+            "pass3_block", "indexer_topk", "pass3_indexer_support", "dense_prefill")
+
+
+def rows_of(w) -> tuple:
+    """Rows of the hot path a workload exercises (the 32K default runs all of them)."""
+    rows = ["pass1_lse"]
+    if 1 in w.block_q:
+        rows += ["pass2_mass_topk", "pass3_gather"]
+    if any(b > 1 for b in w.block_q):
+        rows += ["pass2_block_mass_topk", "pass3_block"]
+    if w.d_idx:
+        rows += ["indexer_topk", "pass3_indexer_support"]
+    rows.append("dense_prefill")
+    return tuple(rows)
+
+
 class Step:
-    """All rows of the hot path on device-resident inputs; CUDA events between calls."""
+    """The workload's rows of the hot path on device-resident inputs; CUDA events between
+    calls (events[i] .. events[i+1] brackets row i)."""
 
-    NAMES = ("pass1_lse", "pass2_mass_topk", "pass3_gather", "pass2_block_mass_topk",
-             "pass3_block", "indexer_topk", "pass3_indexer_support", "dense_prefill")
-
-    def __init__(self, tam, w, q, k, v, qx, kx):
+    def __init__(self, tam, w, q, k, v, qx=None, kx=None):
         self.tam, self.w = tam, w
         self.q, self.k, self.v, self.qx, self.kx = q, k, v, qx, kx
+        self.rows = rows_of(w)
+        self.block_q = max(w.block_q)
         self.ws = tam.Workspace(q.device)
         self.outputs = {}
 
     def run(self, events=None):
-        t, w = self.tam, self.w
-        ev = events or [None] * 9
-
-        def mark(n):
+        t, w, ws = self.tam, self.w, self.ws
+        ev = events or [None] * (len(self.rows) + 1)
+        out = {}
+        lse = None
+        for n, row in enumerate(self.rows):
             if ev[n] is not None:
                 ev[n].record()
-        mark(0)
-        lse = t.attention_lse(self.q, self.k, workspace=self.ws, check=False)
-        mark(1)
-        s1 = t.mass_select(self.q, self.k, lse, w.budget_k, 1, workspace=self.ws, check=False)
-        mark(2)
-        o1 = t.sparse_support_attention(self.q, self.k, self.v, s1.idx, s1.length, 1,
-                                        workspace=self.ws, check=False)
-        mark(3)
-        s2 = t.mass_select(self.q, self.k, lse, w.budget_k, BLOCK_Q, workspace=self.ws,
-                           check=False)
-        mark(4)
-        o2 = t.sparse_support_attention(self.q, self.k, self.v, s2.idx, s2.length, BLOCK_Q,
-                                        workspace=self.ws, check=False)
-        mark(5)
-        s3 = t.indexer_topk(self.qx, self.kx, INDEXER_K, workspace=self.ws, check=False)
-        mark(6)
-        o3 = t.sparse_support_attention(self.q, self.k, self.v, s3.idx, s3.length, 1,
-                                        workspace=self.ws, check=False)
-        mark(7)
-        od = t.dense_gqa_prefill(self.q, self.k, self.v, workspace=self.ws, check=False)
-        mark(8)
-        self.outputs = {"lse": lse, "s1_idx": s1.idx, "s1_len": s1.length, "s1_mass": s1.value,
-                        "o1": o1, "s2_idx": s2.idx, "s2_len": s2.length, "s2_mass": s2.value,
-                        "o2": o2, "s3_idx": s3.idx, "s3_len": s3.length, "s3_score": s3.value,
-                        "o3": o3, "od": od}
-        return self.outputs
+            if row == "pass1_lse":
+                lse = out["lse"] = t.attention_lse(self.q, self.k, workspace=ws, check=False)
+            elif row == "pass2_mass_topk":
+                s = t.mass_select(self.q, self.k, lse, w.budget_k, 1, workspace=ws, check=False)
+                out.update(s1_idx=s.idx, s1_len=s.length, s1_mass=s.value)
+            elif row == "pass3_gather":
+                out["o1"] = t.sparse_support_attention(self.q, self.k, self.v, out["s1_idx"],
+                                                       out["s1_len"], 1, workspace=ws, check=False)
+            elif row == "pass2_block_mass_topk":
+                s = t.mass_select(self.q, self.k, lse, w.budget_k, self.block_q, workspace=ws,
+                                  check=False)
+                out.update(s2_idx=s.idx, s2_len=s.length, s2_mass=s.value)
+            elif row == "pass3_block":
+                out["o2"] = t.sparse_support_attention(self.q, self.k, self.v, out["s2_idx"],
+                                                       out["s2_len"], self.block_q, workspace=ws,
+                                                       check=False)
+            elif row == "indexer_topk":
+                s = t.indexer_topk(self.qx, self.kx, self.indexer_k, workspace=ws, check=False)
+                out.update(s3_idx=s.idx, s3_len=s.length, s3_score=s.value)
+            elif row == "pass3_indexer_support":
+                out["o3"] = t.sparse_support_attention(self.q, self.k, self.v, out["s3_idx"],
+                                                       out["s3_len"], 1, workspace=ws, check=False)
+            elif row == "dense_prefill":
+                out["od"] = t.dense_gqa_prefill(self.q, self.k, self.v, workspace=ws, check=False)
+        if ev[len(self.rows)] is not None:
+            ev[len(self.rows)].record()
+        self.outputs = out
+        return out
+
+    @property
+    def indexer_k(self):
+        return INDEXER_K if self.w.name == WORKLOAD else self.w.budget_k
 
 
-def algorithmic_work(w, N, outs):
+def algorithmic_work(step, N):
     """Per-row algorithmic flops/bytes (what the method must do, not what it avoids)."""
+    w, outs = step.w, step.outputs
     Hq, Hkv, d = w.Hq, w.Hkv, w.d
     elt = 2
     cp = causal_pairs(N)
     qo = 2 * N * Hq * d * elt                         # read Q, write O
-    sp1 = support_pairs(N, w.budget_k)
-    sp3 = support_pairs(N, INDEXER_K)
-    # block-shared: gathered rows per block and attended pairs per query (from the supports)
-    s2_len = outs["s2_len"].cpu().numpy().astype(np.int64)
-    s2_idx = outs["s2_idx"].cpu().numpy()
-    nb = len(s2_len)
-    blk_rows = int(s2_len.sum())
-    attended = 0
-    for b in range(nb):
-        sel = np.sort(s2_idx[b, :s2_len[b]])
-        i0, i1 = b * BLOCK_Q, min(N, (b + 1) * BLOCK_Q)
-        rows = np.arange(i0, i1)
-        attended += int(np.searchsorted(sel, rows, side="right").sum())
     gather = lambda pairs: pairs * Hkv * 2 * d * elt  # noqa: E731  K and V rows of every group
-    return {
+    work = {
         "pass1_lse": {"bound": "tensor", "flops": 2.0 * d * Hq * cp},
         "pass2_mass_topk": {"bound": "tensor", "flops": 2.0 * d * Hq * cp},
-        "pass3_gather": {"bound": "hbm",
-                         "bytes": float(gather(sp1) + qo + N * w.budget_k * 4 + N * 4)},
         "pass2_block_mass_topk": {"bound": "tensor", "flops": 2.0 * d * Hq * cp},
-        "pass3_block": {"bound": "hbm", "bytes": float(gather(blk_rows) + qo + nb * w.budget_k * 4),
-                        "flops": 4.0 * d * Hq * attended},
-        "indexer_topk": {"bound": "tensor", "flops": 2.0 * D_IDX * cp},
-        "pass3_indexer_support": {"bound": "hbm",
-                                  "bytes": float(gather(sp3) + qo + N * INDEXER_K * 4 + N * 4)},
+        "indexer_topk": {"bound": "tensor", "flops": 2.0 * (w.d_idx or D_IDX) * cp},
         "dense_prefill": {"bound": "tensor", "flops": 4.0 * d * Hq * cp},
     }
+    if "pass3_gather" in step.rows:
+        sp1 = support_pairs(N, w.budget_k)
+        work["pass3_gather"] = {"bound": "hbm",
+                                "bytes": float(gather(sp1) + qo + N * w.budget_k * 4 + N * 4)}
+    if "pass3_indexer_support" in step.rows:
+        kx = step.indexer_k
+        sp3 = support_pairs(N, kx)
+        work["pass3_indexer_support"] = {"bound": "hbm",
+                                         "bytes": float(gather(sp3) + qo + N * kx * 4 + N * 4)}
+    if "pass3_block" in step.rows:
+        bq = step.block_q
+        s2_len = outs["s2_len"].cpu().numpy().astype(np.int64)
+        s2_idx = outs["s2_idx"].cpu().numpy()
+        nb = len(s2_len)
+        attended = 0
+        for b in range(nb):
+            sel = np.sort(s2_idx[b, :s2_len[b]])
+            rows = np.arange(b * bq, min(N, (b + 1) * bq))
+            attended += int(np.searchsorted(sel, rows, side="right").sum())
+        work["pass3_block"] = {"bound": "hbm",
+                               "bytes": float(gather(int(s2_len.sum())) + qo + nb * w.budget_k * 4),
+                               "flops": 4.0 * d * Hq * attended}
+    return work
 
 
 # Random 256-byte row gather from a 140 MB table (the 32K layer's K+V is 134 MB), measured
@@ -335,9 +364,10 @@ def run_reference(args, w, inp, rank, world):
 
 
 def config_dict(w, world):
-    return {"workload": WORKLOAD, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-            "budget_k": w.budget_k, "block_q": BLOCK_Q, "indexer_k": INDEXER_K, "d_idx": D_IDX,
-            "global_batch": world, "seq_len": w.N,
+    idx_k = INDEXER_K if w.name == WORKLOAD else (w.budget_k if w.d_idx else None)
+    return {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            "budget_k": w.budget_k, "block_q": list(w.block_q), "indexer_k": idx_k,
+            "d_idx": w.d_idx or None, "rope": w.rope_base, "global_batch": world, "seq_len": w.N,
             "parallelism": f"replicas x{world} (independent layers, no collective)",
             "l2": "256 MB buffer written before every step (L2 is 126 MB)"}
 
@@ -349,17 +379,20 @@ def run_ours(args, w, inp, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
-    qx, kx = inp.q_idx.to(dev), inp.k_idx.to(dev)
+    qx = inp.q_idx.to(dev) if inp.q_idx is not None else None
+    kx = inp.k_idx.to(dev) if inp.k_idx is not None else None
     step = Step(tam, w, q, k, v, qx, kx)
+    names = step.rows
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     for _ in range(args.warmup):
         step.run()
     tam.check_status(step.ws.get(256))
     torch.cuda.synchronize()
-    work = algorithmic_work(w, w.N, step.outputs)
+    work = algorithmic_work(step, w.N)
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+          for _ in range(args.steps)]
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
     barrier(world, local_rank)
@@ -380,21 +413,21 @@ def run_ours(args, w, inp, rank, world, local_rank):
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_step = total_ms / args.steps
     row_ms = {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps))
-              for i, n in enumerate(Step.NAMES)}
+              for i, n in enumerate(names)}
 
     pk, pk_kind = peaks()
     traffic = traffic_table()
     rows = {}
-    for n in Step.NAMES:
+    for n in names:
         r = roofline_of(work[n], row_ms[n], pk, pk_kind, traffic.get(n))
         rows[n] = {"ms": row_ms[n], "q_tok_s": w.N / (row_ms[n] * 1e-3), "roofline": r}
-    dominant = max(Step.NAMES, key=lambda n: row_ms[n])
+    dominant = max(names, key=lambda n: row_ms[n])
 
     e2e = measure_e2e(args, tam, w, inp, dev, world, local_rank)
 
     if rank != 0:
         return
-    value = world * w.N / (ms_step * 1e-3)
+    value = job_value(world, w.N, ms_step)
     oracle_sparsity = 1.0 - support_pairs(w.N, w.budget_k) / causal_pairs(w.N)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -404,16 +437,8 @@ def run_ours(args, w, inp, rank, world, local_rank):
         "config": config_dict(w, world),
         "roofline": {**rows[dominant]["roofline"], "kernel": dominant},
         "rows": rows,
-        "sparse_pass": {
-            "per_query_q_tok_s": w.N / (row_ms["pass3_gather"] * 1e-3),
-            "speedup_vs_dense": row_ms["dense_prefill"] / row_ms["pass3_gather"],
-            "block_shared_speedup_vs_dense": row_ms["dense_prefill"] / row_ms["pass3_block"],
-            "indexer_support_speedup_vs_dense":
-                row_ms["dense_prefill"] / row_ms["pass3_indexer_support"],
-            "oracle_pass12_plus3_q_tok_s": w.N / 1e-3 / (row_ms["pass1_lse"]
-                                                         + row_ms["pass2_mass_topk"]
-                                                         + row_ms["pass3_gather"]),
-        },
+        "sparse_pass": sparse_pass_summary(w, row_ms),
+        "support_quality": support_quality(step),
         "sparsity_selfcheck": {
             "this_workload": oracle_sparsity,
             "N4096_k256": 1.0 - support_pairs(4096, 256) / causal_pairs(4096),
@@ -423,7 +448,7 @@ def run_ours(args, w, inp, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": launches,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and w.name == WORKLOAD:
         import oracle
         n_rows = calibrate_rows(inp, w, 15.0)
         t = oracle_sample_step(inp, w, n_rows)
@@ -436,8 +461,9 @@ def measure_e2e(args, tam, w, inp, dev, world, local_rank):
     """Same step through the public API with pinned host inputs and results."""
     if args.no_e2e:
         return None
-    host_in = [inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory(),
-               inp.q_idx.pin_memory(), inp.k_idx.pin_memory()]
+    host_in = [inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory()]
+    if inp.q_idx is not None:
+        host_in += [inp.q_idx.pin_memory(), inp.k_idx.pin_memory()]
     dev_in = [torch.empty_like(t, device=dev) for t in host_in]
     step = Step(tam, w, *dev_in)
     for t_d, t_h in zip(dev_in, host_in):
@@ -461,7 +487,7 @@ def measure_e2e(args, tam, w, inp, dev, world, local_rank):
     torch.cuda.synchronize()
     barrier(world, local_rank)
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n
-    return {"value": world * w.N / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    return {"value": job_value(world, w.N, ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n}
 
 
@@ -470,16 +496,75 @@ def measure_e2e(args, tam, w, inp, dev, world, local_rank):
 def barrier(world, local_rank):
     if world > 1:
         import torch.distributed as dist
-        dist.barrier(device_ids=[local_rank])
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[local_rank])
+        else:
+            dist.barrier()
 
 
 def max_over_ranks(x: float, world: int, dev) -> float:
+    """The slowest rank's time: every replica's step is timed on its own device."""
     if world == 1:
         return x
     import torch.distributed as dist
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: query tokens of all replicas per second of the slowest one."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
+def support_quality(step):
+    """Indexer support vs mass-oracle support (recall@k over rows with i+1 > k, when both
+    use the same k) and each sparse output's max-abs distance from dense attention."""
+    out, w = step.outputs, step.w
+    res = {}
+    od = out["od"].float()
+    for key, name in (("o1", "per_query"), ("o2", "block_shared"), ("o3", "indexer")):
+        if key in out:
+            res[f"{name}_output_vs_dense_max_abs"] = float((out[key].float() - od).abs().max())
+    if "s1_idx" in out and "s3_idx" in out and out["s1_idx"].shape == out["s3_idx"].shape:
+        k = out["s1_idx"].shape[1]
+        a, b = out["s1_idx"][k:].long(), out["s3_idx"][k:].long()       # rows i >= k are full
+        if a.numel():
+            pos = torch.searchsorted(a.contiguous(), b.contiguous()).clamp_(max=k - 1)
+            hit = (torch.gather(a, 1, pos) == b).sum(dim=1).double() / k
+            res["indexer_recall_at_k"] = float(hit.mean())
+            res["recall_k"] = k
+    return res
+
+
+def workload_for(name: str):
+    """The default step is the 32K layer with both supports (B_q = 64) and its indexer
+    head (d_idx = 64, k = 1024 on the same tensors); other names are single workloads."""
+    if name == WORKLOAD:
+        base = tam_synth.WORKLOADS[WORKLOAD]
+        return tam_synth.Workload(**{**base.__dict__, "d_idx": D_IDX})
+    return tam_synth.WORKLOADS[name]
+
+
+def sparse_pass_summary(w, row_ms):
+    out = {}
+    dense = row_ms["dense_prefill"]
+    if "pass3_gather" in row_ms:
+        out["per_query_q_tok_s"] = w.N / (row_ms["pass3_gather"] * 1e-3)
+        out["speedup_vs_dense"] = dense / row_ms["pass3_gather"]
+        out["oracle_pass12_plus3_q_tok_s"] = w.N / 1e-3 / (row_ms["pass1_lse"]
+                                                           + row_ms["pass2_mass_topk"]
+                                                           + row_ms["pass3_gather"])
+    if "pass3_block" in row_ms:
+        out["block_shared_q_tok_s"] = w.N / (row_ms["pass3_block"] * 1e-3)
+        out["block_shared_speedup_vs_dense"] = dense / row_ms["pass3_block"]
+        out["oracle_block_pass12_plus3_q_tok_s"] = w.N / 1e-3 / (
+            row_ms["pass1_lse"] + row_ms["pass2_block_mass_topk"] + row_ms["pass3_block"])
+    if "pass3_indexer_support" in row_ms:
+        out["indexer_support_speedup_vs_dense"] = dense / row_ms["pass3_indexer_support"]
+        out["indexer_path_speedup_vs_dense"] = dense / (row_ms["indexer_topk"]
+                                                        + row_ms["pass3_indexer_support"])
+    return out
 
 
 def main():
@@ -490,16 +575,21 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="gqa32k_2pct (default: every row), gqa4k_needles, longctx_<N>, indexer32k")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    w = tam_synth.WORKLOADS["indexer32k"]          # the 32K layer plus its indexer head
-    w = tam_synth.Workload(**{**w.__dict__, "name": WORKLOAD, "budget_k": 655})
+    w = workload_for(args.workload)
     if args.impl == "reference":
         if rank != 0:
+            return
+        if w.name != WORKLOAD:
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the oracle arm is sampled on the default 32K workload only"}))
             return
         inp = tam_synth.make_inputs(w)
         run_reference(args, w, inp, rank, world)
