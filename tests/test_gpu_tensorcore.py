@@ -182,3 +182,27 @@ def test_indexer_forced_timeout_is_reported(tam_lib, monkeypatch):
     monkeypatch.delenv("TAM_DEBUG_FORCE_TIMEOUT")
     res = tam_lib.indexer_topk(qx, kx, 32)
     assert int(res.length[-1]) == 32
+
+
+@pytest.mark.parametrize("N,Hq,Hkv,d,kb,bq", [(1500, 32, 8, 128, 100, 1), (1500, 32, 8, 128, 100, 64),
+                                              (777, 16, 2, 128, 40, 1), (900, 32, 4, 64, 60, 1),
+                                              (2100, 16, 4, 128, 300, 128), (300, 64, 4, 128, 30, 1)])
+def test_pair_kernel_matches_single_cta_kernel(tam_lib, oracle_mod, monkeypatch, N, Hq, Hkv, d, kb, bq):
+    """The 2-SM pass-2 kernel and the single-CTA one give the same supports (and both
+    match the oracle)."""
+    inp = _inputs(N, Hq, Hkv, d, seed=N + kb, sink=True, needles=4)
+    q, k = inp.q.cuda(), inp.k.cuda()
+    lse = tam_lib.attention_lse(q, k)
+    a = tam_lib.mass_select(q, k, lse, kb, bq)
+    monkeypatch.setenv("TAM_DISABLE_PAIR_KERNELS", "1")
+    b = tam_lib.mass_select(q, k, lse, kb, bq)
+    monkeypatch.delenv("TAM_DISABLE_PAIR_KERNELS")
+    assert torch.equal(a.length, b.length)
+    assert torch.equal(a.idx, b.idx)
+    assert (a.value - b.value).abs().max().item() <= 1e-6 * bq
+    if bq == 1:
+        rows = tam_synth.sample_rows(N, inp.needle_i, n_random=48)
+        oi, ol, _ = oracle_mod.topk_rows(inp.q, inp.k, kb, rows)
+        P = oracle_mod.mass_rows(inp.q, inp.k, rows)
+        check_support(a.idx.cpu().numpy()[rows], a.length.cpu().numpy()[rows],
+                      a.value.cpu().numpy()[rows], oi, ol, P, MASS_ATOL, "pair")

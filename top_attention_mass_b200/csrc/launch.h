@@ -77,6 +77,8 @@ int tc_mass_columns(const MassArgs& a);
 bool tc_mass_supported(const MassArgs& a);
 size_t tc_mass_block_bytes(int64_t N, int block_q);
 cudaError_t tc_mass_select(const MassArgs& a, cudaStream_t st);
+bool pair_mass_supported(const MassArgs& a);
+cudaError_t pair_mass_select(const MassArgs& a, cudaStream_t st);
 bool tc_indexer_supported(int64_t N, int d_idx, int dtype, int block_q);
 cudaError_t tc_indexer_select(const IndexerArgs& a, cudaStream_t st);
 bool tc_dense_supported(const AttnArgs& a);

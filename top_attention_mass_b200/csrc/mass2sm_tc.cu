@@ -1,0 +1,497 @@
+// Pass 2 on CTA pairs: head-averaged mass and its top-k with 2-SM UMMA.
+//
+//   P_i[j] = (1/Hq) sum_h exp(scale * q[i,h].k[j,g(h)] - lse[h,i]),  j <= i
+//   per query:  S_i = top-min(k, i+1) of P_i;   per block: M_b[j] sums, as in mass_tc.cu
+//
+// (arXiv 2606.07703, Abstract; gist.science technical report §2.1 "Selektion",
+// "Granularität".)
+//
+// Same orientation as the single-CTA kernel (S^T = K_g Q_g^T, the key-row thread
+// sums every head of a query in registers), but a cluster of two CTAs issues one
+// M = 256, N = 128 UMMA per KV group: each CTA holds 128 of the 256 keys (A) and
+// the Q rows of 16 of the pair's 32 queries for all heads (its half of B), and each
+// CTA's TMEM receives its 128 keys x all 128 (query, head) columns.  Every K row
+// read from L2 then serves 32 queries instead of 16, and each CTA reads half as many
+// operand bytes per unit of work - the two things that bounded the single-CTA pass.
+//
+// Roles in each CTA (512 threads):
+//   warp 8      TMA producer: this CTA's Q half (once) and its 128 keys of each
+//               256-key tile, counted on CTA 0's barriers;
+//   warp 9      CTA 0 only: issues the pair MMAs into a ring of four 128-column TMEM
+//               slots and commits to the barriers of both CTAs;
+//   warps 0-7   mass warps: thread = key row (warp w reads TMEM lanes 32 (w % 4) ..),
+//               column half w / 4, i.e. the (query, head) columns of half the pair's
+//               queries; exp2 against the pass-1 LSE, sum over heads -> mass of those
+//               queries for 128 keys.  Two warps per TMEM lane quarter keep two
+//               exp streams per scheduler.  Per query, the queries of column half h
+//               belong to the select warps of CTA h, so the warps of the other half
+//               write their values into the peer's shared memory (DSMEM) - both
+//               select groups then see their queries over all 256 keys, in ascending
+//               key order.  Block-shared mass goes to the fixed-point block sums;
+//   warps 10-15 select warps: the streaming exact top-k of mass_tc.cu.
+// Every wait is bounded; the pair shakes hands before it frees TMEM and exits so
+// that no DSMEM write, remote arrive or MMA of one CTA can land after the other left.
+#include "launch.h"
+#include "tc_ptx.cuh"
+#include "tma_host.h"
+#include "warp_select.cuh"
+
+namespace tam {
+namespace {
+
+using namespace sel;
+
+constexpr int kStages = 2;
+constexpr int kSelWarps = 6;
+constexpr int kMassWarps = 8;
+constexpr int kProducerWarp = kMassWarps, kMmaWarp = kMassWarps + 1;
+constexpr int kThreads = 32 * (kMassWarps + 2 + kSelWarps);
+constexpr int kNQ = 128;                // MMA N: (query, head) columns of the pair
+constexpr int kHalfRows = 64;           // B rows held by each CTA
+constexpr int kR = 512 / kNQ;           // TMEM accumulator slots
+constexpr int kTileKeys = 256;          // keys per pair tile (128 per CTA)
+
+__host__ __device__ constexpr int pair_smem_bytes(int D, int Hkv, int G, bool block) {
+    // Q half + K ring + lse of all 128 columns + (per query) one 16 x 256 mass tile and
+    // the select histograms + barriers
+    return 1024 + Hkv * kHalfRows * D * 2 + kStages * 128 * D * 2 + Hkv * kNQ * 4 + 512 +
+           (block ? 0 : (kHalfRows / G) * kTileKeys * 4 + kSelWarps * (int)sizeof(SelWarpSmem));
+}
+constexpr int kMaxDynSmem = 227 * 1024;
+
+struct PairParams {
+    int N, Hq, Hkv, n_pairs, budget, block_q, cap;
+    float sl2, inv_hq;
+    const float* lse;
+    int32_t* sup_idx;
+    int32_t* sup_len;
+    float* sup_mass;
+    uint32_t* cand;
+    unsigned long long* bmass;
+    int32_t* status;
+    uint64_t timeout_ns;
+    int dbg;
+};
+
+__host__ __device__ __forceinline__ int64_t bmass_row(int64_t b, int block_q) {
+    return (int64_t)block_q * b * (b + 1) / 2;
+}
+
+template <int G, int D, bool BLOCK>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const PairParams p) {
+    constexpr int BQP = kNQ / G;              // queries of the pair
+    constexpr int BQC = kHalfRows / G;        // queries whose top-k this CTA owns
+    constexpr int NH = D / 64;
+    constexpr uint32_t kQHalf = kHalfRows * 128;   // one 64-element half of a group's B rows
+    constexpr uint32_t kKHalf = 128 * 128;
+    constexpr uint32_t kKTile = NH * kKHalf;
+    constexpr int QPW = (BQC + kSelWarps - 1) / kSelWarps;
+    const int Hkv = p.Hkv;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* sQ = base;
+    uint8_t* sK = sQ + Hkv * NH * kQHalf;
+    float* sLse = reinterpret_cast<float*>(sK + kStages * kKTile);     // Hkv * 128
+    float* sMass = sLse + Hkv * kNQ;                                   // BQC x 256 (per query)
+    SelWarpSmem* sSel = reinterpret_cast<SelWarpSmem*>(sMass + (BLOCK ? 0 : BQC * kTileKeys));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + (BLOCK ? 0 : kSelWarps));
+    uint64_t* q_full = bars;                 // CTA 0's counts both CTAs' Q bytes
+    uint64_t* k_full = q_full + 1;           // CTA 0's counts both CTAs' K bytes
+    uint64_t* k_empty = k_full + kStages;    // both (pair commits)
+    uint64_t* s_full = k_empty + kStages;    // both (pair commits)
+    uint64_t* s_empty = s_full + kR;         // CTA 0's: both CTAs' mass threads
+    uint64_t* m_full = s_empty + kR;         // each: own + peer mass threads
+    uint64_t* m_empty = m_full + 1;          // each: own + peer select warps
+    uint64_t* mma_done = m_empty + 1;        // both (pair commit)
+    uint64_t* exit_bar = mma_done + 1;       // each: the peer's arrival at the end
+    uint64_t* never = exit_bar + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = tc::cluster_rank();
+    const uint32_t peer = rank ^ 1u;
+    const int pt = p.n_pairs - 1 - (int)(blockIdx.x >> 1);   // heaviest pair first
+    const int q0 = pt * BQP;
+    const int q_last = min(p.N, q0 + BQP) - 1;
+    const int n_kt = q_last / kTileKeys + 1;
+    const int n_units = n_kt * Hkv;
+    const int my_q0 = q0 + (int)rank * BQC;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(&k_full[s], 1);
+            tc::mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < kR; ++s) {
+            tc::mbar_init(&s_full[s], 1);
+            tc::mbar_init(&s_empty[s], 2 * kMassWarps);   // every mass warp of both CTAs
+        }
+        tc::mbar_init(m_full, kMassWarps);        // the mass warps (both CTAs) of this half
+        tc::mbar_init(m_empty, 2 * kSelWarps);
+        tc::mbar_init(mma_done, 1);
+        tc::mbar_init(exit_bar, 1);
+        tc::mbar_init(never, 1);
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    for (int t = threadIdx.x; t < Hkv * kNQ; t += blockDim.x) {
+        const int g = t / kNQ, c = t % kNQ;
+        const int i = q0 + c / G, h = g * G + c % G;
+        sLse[t] = (i < p.N) ? p.lse[(size_t)h * p.N + i] * kLog2e : INFINITY;
+    }
+    if (warp == 0) {
+        tc::tmem_alloc_pair(tmem_slot, 512);
+        tc::tmem_relinquish_pair();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    // both CTAs' barriers must be initialised before either CTA signals the other
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    // a timeout in either CTA aborts both (the flag of the peer is raised over DSMEM)
+    const tc::Guard gd{abort_flag, p.status, BLOCK ? KID_BLOCK_MASS_TC : KID_MASS_TC, p.timeout_ns,
+                       tc::map_to_cta(tc::smem_u32(abort_flag), peer)};
+    int zero = 0;
+    const tc::Guard drain{&zero, nullptr, 0, p.timeout_ns};
+    // the exit handshake outlasts any skew between the two CTAs' wind-down
+    const tc::Guard handshake{&zero, nullptr, 0, 16 * p.timeout_ns};
+
+    if (warp == kProducerWarp) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            tc::prefetch_tmap(&tmQ);
+            tc::prefetch_tmap(&tmK);
+            if (rank == 0) tc::mbar_arrive_expect_tx(q_full, 2u * Hkv * NH * kQHalf);
+            for (int g = 0; g < Hkv; ++g)
+                for (int h = 0; h < NH; ++h)
+                    tc::tma_load_3d_pair(sQ + (g * NH + h) * kQHalf, &tmQ, q_full, h * 64, g * G,
+                                         my_q0);
+            int issued = 0;
+            for (int u = 0; u < n_units; ++u) {
+                const int s = u % kStages;
+                if (!tc::wait(&k_empty[s], ((u / kStages) & 1) ^ 1, gd, 1)) break;
+                const int kt = u / Hkv, g = u % Hkv;
+                if (rank == 0) tc::mbar_arrive_expect_tx(&k_full[s], 2u * kKTile);
+                for (int h = 0; h < NH; ++h)
+                    tc::tma_load_3d_pair(sK + s * kKTile + h * kKHalf, &tmK, &k_full[s], h * 64, g,
+                                         kt * kTileKeys + (int)rank * 128);
+                ++issued;
+            }
+            // the last pair commits on k_empty must have landed before this CTA exits
+            // (when aborting, the MMAs behind them may never have been issued; the
+            // completion of every issued MMA is covered by mma_done)
+            for (int u = max(0, issued - kStages); u < issued && !*abort_flag; ++u)
+                tc::wait(&k_empty[u % kStages], (u / kStages) & 1, drain, 0);
+        }
+    } else if (warp == kMmaWarp) {
+        // ---------------------------------------------------------------- MMA issuer (CTA 0)
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = tc::idesc_bf16_f32(256, kNQ);
+            bool ok = tc::wait(q_full, 0, gd, 2);
+            int done = 0;
+            for (int u = 0; ok && u < n_units; ++u) {
+                const int s = u % kStages, slot = u % kR, g = u % Hkv;
+                if (!tc::wait(&k_full[s], (u / kStages) & 1, gd, 3)) break;
+                if (!tc::wait(&s_empty[slot], ((u / kR) & 1) ^ 1, gd, 4)) break;
+                tc::fence_after_sync();
+                const uint32_t ak = tc::smem_u32(sK + s * kKTile);
+                const uint32_t bq = tc::smem_u32(sQ + g * NH * kQHalf);
+#pragma unroll
+                for (int kk = 0; kk < NH * 4; ++kk) {
+                    const uint32_t offk = (kk >> 2) * kKHalf + (kk & 3) * 32;
+                    const uint32_t offq = (kk >> 2) * kQHalf + (kk & 3) * 32;
+                    tc::mma_bf16_ss_pair(tmem + slot * kNQ, tc::desc_kmajor_sw128(ak + offk),
+                                         tc::desc_kmajor_sw128(bq + offq), idesc, kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit_pair(&k_empty[s], 0x3);
+                tc::mma_commit_pair(&s_full[slot], 0x3);
+                done = u + 1;
+            }
+            tc::mma_commit_pair(mma_done, 0x3);
+            // the peer's last slot releases must have landed before CTA 0 exits (when
+            // aborting, the exit handshake stands in for them)
+            for (int u = max(0, done - kR); u < done && !*abort_flag; ++u)
+                tc::wait_cluster(&s_empty[u % kR], (u / kR) & 1, drain, 0);
+        }
+    } else if (warp < kMassWarps) {
+        // ---------------------------------------------------------------- mass warps
+        constexpr int kCols = kNQ / 2;                 // columns of one half
+        const int quarter = warp & 3, half = warp >> 2;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * kCols);
+        const uint32_t s_empty_leader = tc::map_to_cta(tc::smem_u32(s_empty), 0);
+        // the queries of this half belong to CTA `half`: its m_full and mass tile
+        const bool own = half == (int)rank;
+        const uint32_t m_full_owner = own ? tc::smem_u32(m_full)
+                                          : tc::map_to_cta(tc::smem_u32(m_full), peer);
+        const uint32_t mass_peer = tc::map_to_cta(tc::smem_u32(sMass), peer);
+        bool ok = true;
+        if (p.dbg & kDebugForceTimeout) ok = tc::wait(never, 0, gd, 9);
+        for (int kt = 0; ok && kt < n_kt; ++kt) {
+            float acc[BQC];
+#pragma unroll
+            for (int q = 0; q < BQC; ++q) acc[q] = 0.f;
+            for (int g = 0; g < Hkv; ++g) {
+                const int u = kt * Hkv + g;
+                const int slot = u % kR;
+                if (!tc::wait(&s_full[slot], (u / kR) & 1, gd, 5)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint32_t col0 = lane_addr + slot * kNQ;
+                uint32_t va[32], vb[32];
+                tc::tmem_ld32(col0, va);
+                tc::tmem_wait_ld(va);
+#pragma unroll
+                for (int c = 0; c < kCols / 32; ++c) {
+                    uint32_t (&cur)[32] = (c & 1) ? vb : va;
+                    uint32_t (&nxt)[32] = (c & 1) ? va : vb;
+                    if (c + 1 < kCols / 32) tc::tmem_ld32(col0 + (c + 1) * 32, nxt);
+                    const float4* l4 =
+                        reinterpret_cast<const float4*>(sLse + g * kNQ + half * kCols + c * 32);
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 L = l4[c4];
+                        const float Ls[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int col = c * 32 + c4 * 4 + e;
+                            acc[col / G] += tc::ex2(fmaf(__uint_as_float(cur[c4 * 4 + e]), p.sl2, -Ls[e]));
+                        }
+                    }
+                    if (c + 1 < kCols / 32) tc::tmem_wait_ld(nxt);
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    if (rank == 0) tc::mbar_arrive(&s_empty[slot]);
+                    else tc::mbar_arrive_remote_relaxed(s_empty_leader + (uint32_t)slot * 8u);
+                }
+            }
+            if (!ok) break;
+            const int j = kt * kTileKeys + (int)rank * 128 + row;
+            if constexpr (!BLOCK) {
+                if (!tc::wait_cluster(m_empty, (kt & 1) ^ 1, gd, 6)) { ok = false; break; }
+#pragma unroll
+                for (int ql = 0; ql < BQC; ++ql) {
+                    const int i = q0 + half * BQC + ql;
+                    const float val = (j <= i && i < p.N) ? acc[ql] * p.inv_hq : -INFINITY;
+                    const int off = ql * kTileKeys + (int)rank * 128 + row;
+                    if (own) sMass[off] = val;
+                    else tc::st_cluster_f32(mass_peer + (uint32_t)off * 4u, val);
+                }
+                // every lane's (DSMEM) stores are ordered before lane 0's release
+                asm volatile("fence.acq_rel.cluster;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    if (own) tc::mbar_arrive(m_full);
+                    else tc::mbar_arrive_remote(m_full_owner);
+                }
+            } else {
+                const int qh = q0 + half * BQC;
+                int cur_b = qh / p.block_q;
+                float part = 0.f;
+#pragma unroll
+                for (int q = 0; q < BQC; ++q) {
+                    const int i = qh + q;
+                    if (i < p.N) {
+                        const int b = i / p.block_q;
+                        if (b != cur_b) {
+                            if (part > 0.f)
+                                atomicAdd(&p.bmass[bmass_row(cur_b, p.block_q) + j],
+                                          (unsigned long long)__float2ll_rn(part * p.inv_hq * 1099511627776.0f));
+                            part = 0.f;
+                            cur_b = b;
+                        }
+                        if (j <= i) part += acc[q];
+                    }
+                }
+                if (part > 0.f)
+                    atomicAdd(&p.bmass[bmass_row(cur_b, p.block_q) + j],
+                              (unsigned long long)__float2ll_rn(part * p.inv_hq * 1099511627776.0f));
+            }
+        }
+        if constexpr (!BLOCK) {
+            // the peer's select warps release the last tile remotely: wait for it here
+            if (n_kt > 0 && !*abort_flag) tc::wait_cluster(m_empty, (n_kt - 1) & 1, drain, 0);
+        }
+    } else if constexpr (!BLOCK) {
+        // ---------------------------------------------------------------- select warps
+        const int sw = warp - (kMassWarps + 2);
+        int* hist = sSel[sw].hist;
+        const uint32_t m_empty_peer = tc::map_to_cta(tc::smem_u32(m_empty), peer);
+        float tau[QPW];
+        int cnt[QPW];
+#pragma unroll
+        for (int a = 0; a < QPW; ++a) {
+            tau[a] = -INFINITY;
+            cnt[a] = 0;
+        }
+        bool ok = true;
+        bool overflow = false;
+        for (int kt = 0; ok && kt < n_kt; ++kt) {
+            if (!tc::wait_cluster(m_full, kt & 1, gd, 7)) { ok = false; break; }
+#pragma unroll
+            for (int a = 0; a < QPW; ++a) {
+                const int ql = sw + a * kSelWarps;
+                const int i = my_q0 + ql;
+                if (ql >= BQC || i >= p.N) continue;
+                uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
+                uint32_t* idxs = keys + p.cap;
+#pragma unroll
+                for (int r = 0; r < kTileKeys / 32; ++r) {
+                    const float v = sMass[ql * kTileKeys + r * 32 + lane];
+                    const bool pass = v > tau[a];
+                    const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+                    const int pos = cnt[a] + __popc(bal & lanemask_lt());
+                    if (pass) {
+                        if (pos < p.cap) {
+                            keys[pos] = key_of(v);
+                            idxs[pos] = (uint32_t)(kt * kTileKeys + r * 32 + lane);
+                        } else {
+                            overflow = true;
+                        }
+                    }
+                    cnt[a] += __popc(bal);
+                    if (cnt[a] > p.cap - 32 && cnt[a] > p.budget) {
+                        __syncwarp();
+                        const int n = min(cnt[a], p.cap);
+                        uint32_t T;
+                        int take_eq;
+                        warp_kth(keys, n, p.budget, hist, T, take_eq, 2);
+                        int kept = n;
+                        if (T > 0u) kept = warp_select(keys, idxs, n, T - 1u, 0, false, nullptr, nullptr);
+                        if (kept > p.cap - 96) {
+                            warp_kth(keys, kept, p.budget, hist, T, take_eq, 4);
+                            kept = warp_select(keys, idxs, kept, T, take_eq, false, nullptr, nullptr);
+                            tau[a] = fmaxf(tau[a], value_of(T));
+                        } else if (T > 0u) {
+                            tau[a] = fmaxf(tau[a], value_of(T - 1u));
+                        }
+                        cnt[a] = kept;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(m_empty);
+                tc::mbar_arrive_remote(m_empty_peer);
+            }
+        }
+        if (__any_sync(0xffffffffu, overflow) && lane == 0)
+            report_error(p.status, TAM_ERR_OVERFLOW, KID_MASS_TC, my_q0);
+        if (ok) {
+#pragma unroll
+            for (int a = 0; a < QPW; ++a) {
+                const int ql = sw + a * kSelWarps;
+                const int i = my_q0 + ql;
+                if (ql >= BQC || i >= p.N) continue;
+                uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
+                uint32_t* idxs = keys + p.cap;
+                const int n = min(cnt[a], p.cap);
+                __syncwarp();
+                uint32_t T = 0;
+                int take_eq = 0;
+                const bool all = n <= p.budget;
+                if (!all) warp_kth(keys, n, p.budget, hist, T, take_eq);
+                int32_t* oi = p.sup_idx + (size_t)i * p.budget;
+                float* om = p.sup_mass + (size_t)i * p.budget;
+                const int kept = warp_select(keys, idxs, n, T, take_eq, all, oi, om);
+                for (int t = kept + lane; t < p.budget; t += 32) {
+                    oi[t] = -1;
+                    om[t] = 0.f;
+                }
+                if (lane == 0) p.sup_len[i] = kept;
+            }
+        }
+    }
+    // every CTA waits for the pair MMAs (they write into both CTAs' TMEM)
+    if (threadIdx.x == 0) tc::wait(mma_done, 0, drain, 0);
+    __syncthreads();
+    // pair handshake: neither CTA frees TMEM or exits while the other may still touch it
+    if (threadIdx.x == 0) {
+        tc::mbar_arrive_remote(tc::map_to_cta(tc::smem_u32(exit_bar), peer));
+        tc::wait_cluster(exit_bar, 0, handshake, 0);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc_pair(tmem, 512);
+    }
+}
+
+template <int G, int D, bool BLOCK>
+cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
+    constexpr int BQP = kNQ / G, BQC = kHalfRows / G;
+    CUtensorMap tq, tk;
+    const uint64_t d = a.d;
+    if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQC) ||
+        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, a.N, d * 2, (uint64_t)a.Hkv * d * 2, 64, 1, 128))
+        return cudaErrorInvalidValue;
+    PairParams p{};
+    p.N = (int)a.N;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.n_pairs = (int)((a.N + BQP - 1) / BQP);
+    p.budget = a.budget;
+    p.block_q = a.block_q;
+    p.cap = a.cand_cap;
+    p.sl2 = a.sl2;
+    p.inv_hq = 1.f / (float)a.Hq;
+    p.lse = a.lse;
+    p.sup_idx = a.sup_idx;
+    p.sup_len = a.sup_len;
+    p.sup_mass = a.sup_mass;
+    p.cand = reinterpret_cast<uint32_t*>(a.cand);
+    p.bmass = reinterpret_cast<unsigned long long*>(a.bmass);
+    p.status = a.status;
+    p.timeout_ns = wait_timeout_ns();
+    p.dbg = debug_flags();
+    const int smem = pair_smem_bytes(D, a.Hkv, G, BLOCK);
+    auto kern = k_mass_pair<G, D, BLOCK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (BLOCK) {
+        const int64_t nb = (a.N + a.block_q - 1) / a.block_q;
+        e = cudaMemsetAsync(a.bmass, 0, (size_t)bmass_row(nb, a.block_q) * 8, st);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<(unsigned)(2 * p.n_pairs), kThreads, smem, st>>>(tq, tk, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
+template <int D, bool BLOCK>
+cudaError_t dispatch_g(const MassArgs& a, cudaStream_t st) {
+    switch (a.Hq / a.Hkv) {
+        case 4: return launch_pair<4, D, BLOCK>(a, st);
+        case 8: return launch_pair<8, D, BLOCK>(a, st);
+        case 16: return launch_pair<16, D, BLOCK>(a, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+}  // namespace
+
+bool pair_mass_supported(const MassArgs& a) {
+    const int G = a.Hq / a.Hkv;
+    if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128)) return false;
+    if (G != 4 && G != 8 && G != 16) return false;
+    if (a.block_q > 1 && a.block_q > (1 << 20)) return false;
+    if (a.block_q == 1 && a.budget + 96 > a.cand_cap) return false;   // compaction slack
+    return pair_smem_bytes(a.d, a.Hkv, G, a.block_q > 1) <= kMaxDynSmem;
+}
+
+// Launches the pair kernel only; in block mode the caller runs the block top-k after it.
+cudaError_t pair_mass_select(const MassArgs& a, cudaStream_t st) {
+    const bool block = a.block_q > 1;
+    if (a.d == 64) return block ? dispatch_g<64, true>(a, st) : dispatch_g<64, false>(a, st);
+    return block ? dispatch_g<128, true>(a, st) : dispatch_g<128, false>(a, st);
+}
+
+}  // namespace tam

@@ -58,7 +58,14 @@ struct Guard {
     int32_t* status;            // device status block (may be null)
     int32_t kid;                // kernel id for the report
     uint64_t timeout_ns;
+    uint32_t peer_abort = 0;    // shared::cluster address of the other CTA's flag (0 = none)
 };
+
+__device__ __forceinline__ void raise_abort(const Guard& g) {
+    *g.abort_flag = 1;
+    if (g.peer_abort != 0u)
+        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(g.peer_abort), "r"(1u) : "memory");
+}
 
 // Wait until the phase with parity `parity` of `bar` has completed.  Returns false
 // if the kernel is aborting (another role timed out) or this wait timed out.
@@ -71,7 +78,7 @@ __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, const Guard
             spins = 0;
             if (*g.abort_flag) return false;
             if (global_timer_ns() - t0 > g.timeout_ns) {
-                *g.abort_flag = 1;
+                raise_abort(g);
                 report_error(g.status, TAM_ERR_TIMEOUT, g.kid, where, (int32_t)parity);
                 return false;
             }
@@ -230,6 +237,125 @@ __device__ __forceinline__ void tmem_wait_st() {
 // (tensor-core operand reads) before it signals them through an mbarrier.
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ CTA pairs (clusters of 2)
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address in the shared::cluster window of the variable at shared::cta address `a`
+// in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+
+// Arrive on an mbarrier of another CTA of the cluster (address from map_to_cta), with
+// release semantics at cluster scope: this thread's earlier writes (including
+// st.shared::cluster) are visible to whoever observes the phase completion.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// Remote arrive without memory ordering: for barriers that only hand over TMEM slots,
+// whose ordering comes from the tcgen05 fences around the barrier.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_f32(uint32_t cluster_addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
+}
+
+// Waits with acquire semantics at cluster scope (pairs with mbar_arrive_remote).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity, const Guard& g,
+                                             int where) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    uint32_t spins = 0;
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (++spins == 256) {
+            spins = 0;
+            if (*g.abort_flag) return false;
+            if (global_timer_ns() - t0 > g.timeout_ns) {
+                raise_abort(g);
+                report_error(g.status, TAM_ERR_TIMEOUT, g.kid, where, (int32_t)parity);
+                return false;
+            }
+        }
+    }
+    return true;
+}
+
+// 2-CTA (cta_group::2) forms.  TMEM allocation: the same warp of both CTAs executes
+// them; both CTAs receive the same TMEM address.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// Tile load issued by either CTA of a pair into its own shared memory; the completed
+// bytes are counted on the barrier at the same offset in CTA 0 of the pair (the peer
+// bit of the shared::cluster address is cleared).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint64_t* bar,
+                                                 int c0, int c1, int c2) {
+    const uint32_t leader_bar = smem_u32(bar) & 0xFEFFFFFFu;
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(m), "r"(leader_bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A * B^T with M = 256 split over the pair (each CTA holds
+// 128 rows of A and N/2 rows of B at the same shared-memory offsets); issued by one
+// thread of CTA 0.
+__device__ __forceinline__ void mma_bf16_ss_pair(uint32_t d_tmem, uint64_t a_desc,
+                                                 uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive, in every CTA of `cta_mask`, on the barrier at this offset once the pair MMAs
+// issued so far by this thread have completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
 }
 
 // 2^x on the MUFU unit (inputs far below -126 flush to +0).

@@ -57,6 +57,8 @@ uint64_t wait_timeout_ns() {
     return (debug_flags() & kDebugForceTimeout) ? 20000000ull : 2000000000ull;
 }
 
+bool pair_path_disabled() { return env_int("TAM_DISABLE_PAIR_KERNELS", 0) != 0; }
+
 int debug_flags() { return env_int("TAM_DEBUG_FORCE_TIMEOUT", 0) ? kDebugForceTimeout : 0; }
 
 int candidate_capacity(int budget_k) {

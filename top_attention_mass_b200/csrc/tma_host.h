@@ -28,4 +28,7 @@ int candidate_capacity(int budget_k);
 
 constexpr int kDebugForceTimeout = 1;
 
+// TAM_DISABLE_PAIR_KERNELS=1 routes pass 2 to the single-CTA kernel (A/B comparisons).
+bool pair_path_disabled();
+
 }  // namespace tam
