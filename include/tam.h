@@ -38,10 +38,10 @@
  * enqueued and returned directly: TAM_ERR_INVALID_ARG (null pointer, bad
  * shape, pointer not 16-byte aligned, k < 1, block_q < 1), TAM_ERR_UNSUPPORTED
  * (d not 64/128, k > 4096, N*k >= 2^31, combination not built), TAM_ERR_WORKSPACE
- * (ws_bytes below the size query).  A failed launch returns TAM_ERR_CUDA.
- * Errors found on the device (a bounded wait that gave up, a candidate
- * buffer that overflowed) are recorded in a status block at the start of the
- * workspace and are read by tam_check_status.  No call traps and no call prints.
+ * (ws_bytes below the smallest accepted size).  A failed launch returns TAM_ERR_CUDA.
+ * Errors found on the device (a bounded wait that gave up) are recorded in a
+ * status block at the start of the workspace and are read by tam_check_status.
+ * No call traps and no call prints.
  */
 #ifndef TAM_H
 #define TAM_H
@@ -60,7 +60,7 @@ typedef enum {
     TAM_ERR_WORKSPACE = 3,
     TAM_ERR_CUDA = 4,
     TAM_ERR_TIMEOUT = 5,
-    TAM_ERR_OVERFLOW = 6
+    TAM_ERR_OVERFLOW = 6    /* kept for ABI stability; no current kernel reports it */
 } tam_status;
 
 typedef enum { TAM_BF16 = 0, TAM_F32 = 1 } tam_dtype;
@@ -72,11 +72,24 @@ int tam_version(void);
 const char* tam_status_string(int status);
 
 /*
- * Workspace bytes tam_mass_oracle_prefill needs for this problem (always a
+ * Workspace bytes tam_mass_oracle_prefill prefers for this problem (always a
  * multiple of 256).  Returns 0 for arguments that the call would reject.
+ * Per query on the tensor cores, pass 2 writes the mass rows P_i of a chunk of
+ * queries to the workspace and selects from them; the preferred size takes every
+ * row at once (up to 4 GiB of rows), and any size down to tam_mass_workspace_min()
+ * is accepted and only means more chunks.  Otherwise the two sizes are equal.
  */
 size_t tam_mass_oracle_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
                                  int block_q);
+
+/*
+ * Smallest workspace tam_mass_oracle_prefill, tam_mass_select and
+ * tam_mass_select_noalloc accept for this problem (a multiple of 256; 0 for
+ * arguments the calls would reject).  Per query on the tensor cores that is room
+ * for 64 rows of N floats next to the status block and an lse buffer.
+ */
+size_t tam_mass_workspace_min(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
+                              int block_q);
 
 /*
  * The attention-mass top-k oracle for one causal GQA prefill layer
@@ -91,8 +104,11 @@ size_t tam_mass_oracle_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, i
  *   pass 3  (only if out != NULL) for every head h of query i,
  *           out[i,h] = sum_{j in T_i} softmax_{T_i}(scale * q[i,h].k[j,g(h)]) v[j,g(h)],
  *           T_i = S_i (per query) or S_b intersected with [0, i] (block), output in q's dtype.
- * lse may be NULL (then it lives in the workspace).  The N x N mass matrix is never
- * written to memory.  budget_k in [1, 4096]; block_q in [1, N].
+ * lse may be NULL (then it lives in the workspace).  Per query, the mass rows P_i
+ * are materialised in the workspace chunk by chunk (see tam_mass_oracle_workspace);
+ * block-shared, only the block sums M_b are.  budget_k in [1, 4096]; block_q in [1, N].
+ * A workspace smaller than tam_mass_workspace_min() gives TAM_ERR_WORKSPACE before
+ * anything is enqueued.
  */
 int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
                             const void* k, const void* v, int budget_k, int block_q,
@@ -127,11 +143,12 @@ int tam_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
  * synchronise the device and fail under fragmentation).
  * Same arguments, semantics and outputs as tam_mass_select, minus the workspace:
  * the scratch is a 64 MiB static device array inside the library.  Problems whose
- * tam_mass_select_workspace() exceeds 64 MiB are rejected with TAM_ERR_WORKSPACE
- * before anything is enqueued.  Nothing is allocated.  The first call on a device
+ * tam_mass_workspace_min() exceeds 64 MiB are rejected with TAM_ERR_WORKSPACE
+ * before anything is enqueued; per query, 64 MiB below the preferred size only
+ * means that the mass rows go through in more chunks.  Nothing is allocated.  The first call on a device
  * looks up the array's device address (with that device current), so make that
  * first call before any stream capture.  The call waits for `stream` and returns
- * the device status (TAM_OK, TAM_ERR_TIMEOUT, TAM_ERR_OVERFLOW).  All calls in the
+ * the device status (TAM_OK or TAM_ERR_TIMEOUT).  All calls in the
  * process share the one array per device and it keeps the last call's contents:
  * calls that can overlap on the GPU (other streams, other threads) race and must
  * be serialised by the caller.  A GPU keeps the array until the process exits.
@@ -148,8 +165,12 @@ int tam_mass_select_noalloc(int64_t N, int Hq, int Hkv, int d, int dtype, const 
  *   sup_score holds the scores of the chosen keys.
  * q_idx, k_idx: [N, d_idx] in `dtype` (bf16 or fp32), d_idx in {16, 32, 64, 128}.
  * block_q must be 1 (per-query support).
+ * On the tensor cores the score rows of a chunk of queries are written to the
+ * workspace and selected from; tam_indexer_workspace() is the preferred size (every
+ * row at once, up to 4 GiB), tam_indexer_workspace_min() the smallest accepted.
  */
 size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int block_q);
+size_t tam_indexer_workspace_min(int64_t N, int d_idx, int dtype, int budget_k, int block_q);
 int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const void* k_idx,
                      int budget_k, int block_q, int32_t* sup_idx, int32_t* sup_len,
                      float* sup_score, void* workspace, size_t ws_bytes, void* stream);
@@ -187,7 +208,7 @@ uint64_t tam_kernel_launches(void);
 /*
  * Waits for `stream`, then reads the device status block at the start of
  * `workspace` that the last call using this workspace wrote.  Returns TAM_OK,
- * TAM_ERR_TIMEOUT, TAM_ERR_OVERFLOW or TAM_ERR_CUDA.  `detail` (may be NULL)
+ * TAM_ERR_TIMEOUT or TAM_ERR_CUDA.  `detail` (may be NULL)
  * receives 8 int32 words: [0] status, [1] kernel id, [2..7] kernel-specific.
  */
 int tam_check_status(const void* workspace, void* stream, int32_t* detail);

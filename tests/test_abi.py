@@ -43,7 +43,12 @@ def test_workspace_queries(tam_lib):
     assert L.tam_mass_oracle_workspace(4096, 32, 8, 128, 0, 5000, 1) == 0     # k > 4096
     assert L.tam_mass_oracle_workspace(4096, 32, 8, 128, 0, 256, 0) == 0      # block_q < 1
     assert L.tam_mass_oracle_workspace(4096, 32, 8, 128, 7, 256, 1) == 0      # dtype
+    lo = L.tam_mass_workspace_min(4096, 32, 8, 128, tam_lib.TAM_BF16, 256, 1)
+    assert 0 < lo <= ws
+    assert L.tam_mass_workspace_min(4096, 32, 8, 128, 0, 0, 1) == 0          # k < 1
     assert L.tam_indexer_workspace(4096, 64, 0, 1024, 1) > 0
+    assert 0 < L.tam_indexer_workspace_min(4096, 64, 0, 1024, 1) <= L.tam_indexer_workspace(
+        4096, 64, 0, 1024, 1)
     assert L.tam_indexer_workspace(4096, 48, 0, 1024, 1) == 0
     for f in ("tam_attention_lse_workspace", "tam_sparse_attention_workspace",
               "tam_dense_workspace"):

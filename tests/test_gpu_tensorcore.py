@@ -1,10 +1,10 @@
-"""Tensor-core kernels (bf16): pass-1 LSE for every head-group size, the streaming
-top-k under heavy compaction and massive ties, and the device error paths.
+"""Tensor-core kernels (bf16): pass-1 LSE for every head-group size, the row top-k
+on long rows, in workspace-bounded chunks and under massive ties (more tied keys
+than the selection stages in shared memory), and the device error paths.
 
 The error-path tests fault nothing: a debug environment switch parks one role of
 the kernel on a barrier nobody arrives on (its bounded wait gives up after 20 ms
-and the kernel winds down), or shrinks the candidate buffer below k + 128 so the
-overflow report fires.  The next call on the same context must succeed.
+and the kernel winds down).  The next call on the same context must succeed.
 """
 import numpy as np
 import pytest
@@ -32,8 +32,8 @@ def test_attention_lse_shapes(tam_lib, oracle_mod, N, Hq, Hkv, d):
 
 @pytest.mark.parametrize("N,Hq,Hkv,d,kb", [(3000, 8, 2, 128, 8), (2049, 32, 8, 128, 1),
                                            (1500, 4, 1, 64, 300), (700, 16, 4, 128, 64)])
-def test_mass_select_heavy_compaction(tam_lib, oracle_mod, N, Hq, Hkv, d, kb):
-    """Small k on long rows: the candidate buffer is compacted many times per row."""
+def test_mass_select_small_budget_long_rows(tam_lib, oracle_mod, N, Hq, Hkv, d, kb):
+    """Small k on long rows: the row top-k keeps a few keys of thousands."""
     inp = _inputs(N, Hq, Hkv, d, seed=kb, sink=True, needles=4)
     q, k = inp.q.cuda(), inp.k.cuda()
     lse = tam_lib.attention_lse(q, k)
@@ -42,13 +42,15 @@ def test_mass_select_heavy_compaction(tam_lib, oracle_mod, N, Hq, Hkv, d, kb):
     oi, ol, _ = oracle_mod.topk_rows(inp.q, inp.k, kb, rows)
     P = oracle_mod.mass_rows(inp.q, inp.k, rows)
     check_support(res.idx.cpu().numpy()[rows], res.length.cpu().numpy()[rows],
-                  res.value.cpu().numpy()[rows], oi, ol, P, MASS_ATOL, "compaction")
+                  res.value.cpu().numpy()[rows], oi, ol, P, MASS_ATOL, "small budget")
 
 
-@pytest.mark.parametrize("bq", [1, 64])
-def test_massive_ties_keep_smallest_indices(tam_lib, bq):
-    """Identical keys make every mass of a row equal; the smallest indices must win."""
-    N, kb = 1200, 50
+@pytest.mark.parametrize("N,bq", [(1200, 1), (1200, 64), (9000, 1)])
+def test_massive_ties_keep_smallest_indices(tam_lib, N, bq):
+    """Identical keys make every mass of a row equal; the smallest indices must win.
+    At N = 9000 the tie at the k-th value spans more keys than the row top-k can
+    stage in shared memory (8192), which takes its bisection path."""
+    kb = 50
     inp = _inputs(N, 8, 2, 128, seed=2)
     k = inp.k.clone()
     k[:] = k[0:1]
@@ -95,17 +97,39 @@ def test_forced_wait_timeout_is_reported(tam_lib, oracle_mod, monkeypatch):
     tam_lib.mass_select(q, k, lse, 16, 1)
 
 
-def test_forced_candidate_overflow_is_reported(tam_lib, monkeypatch):
-    inp = _inputs(500, 8, 2, 128, seed=8)
+@pytest.mark.parametrize("frac", [0.3, 0.0])
+def test_mass_select_in_workspace_bounded_chunks(tam_lib, frac):
+    """Per query the mass rows go through a slab in the workspace.  A workspace below
+    the preferred size (frac of the way from the minimum to it; 0 = the minimum) means
+    more chunks and must give bit-identical supports; one byte less than the minimum
+    is refused before anything runs."""
+    N, Hq, Hkv, d, kb = 3000, 32, 8, 128, 100
+    inp = _inputs(N, Hq, Hkv, d, seed=5, sink=True, needles=4)
     q, k = inp.q.cuda(), inp.k.cuda()
     lse = tam_lib.attention_lse(q, k)
-    monkeypatch.setenv("TAM_DEBUG_CAND_CAP", "32")
+    ref = tam_lib.mass_select(q, k, lse, kb, 1)
+    L = tam_lib.lib()
+    pref = L.tam_mass_select_workspace(N, Hq, Hkv, d, 0, kb, 1)
+    lo = L.tam_mass_workspace_min(N, Hq, Hkv, d, 0, kb, 1)
+    assert 0 < lo < pref
+    res = tam_lib.mass_select(q, k, lse, kb, 1, workspace_bytes=int(lo + frac * (pref - lo)))
+    assert torch.equal(res.length, ref.length) and torch.equal(res.idx, ref.idx)
+    assert torch.equal(res.value, ref.value)
     with pytest.raises(tam_lib.TamError) as e:
-        tam_lib.mass_select(q, k, lse, 40, 1)
-    assert e.value.code == tam_lib.TAM_ERR_OVERFLOW
-    monkeypatch.delenv("TAM_DEBUG_CAND_CAP")
-    res = tam_lib.mass_select(q, k, lse, 40, 1)
-    assert int(res.length[-1]) == 40
+        tam_lib.mass_select(q, k, lse, kb, 1, workspace_bytes=lo - 1)
+    assert e.value.code == tam_lib.TAM_ERR_WORKSPACE
+
+
+def test_indexer_in_workspace_bounded_chunks(tam_lib):
+    N, kb = 2500, 300
+    inp = _inputs(N, 8, 2, 128, seed=6, sink=True, needles=5)
+    qx, kx = tam_synth.indexer_projections(inp, 64, seed=2)
+    qx, kx = qx.cuda(), kx.cuda()
+    ref = tam_lib.indexer_topk(qx, kx, kb)
+    lo = tam_lib.lib().tam_indexer_workspace_min(N, 64, 0, kb, 1)
+    res = tam_lib.indexer_topk(qx, kx, kb, workspace_bytes=lo)
+    assert torch.equal(res.length, ref.length) and torch.equal(res.idx, ref.idx)
+    assert torch.equal(res.value, ref.value)
 
 
 @pytest.mark.parametrize("N,Hq,Hkv,d", [(129, 8, 8, 128), (700, 32, 2, 128), (450, 16, 8, 64),
@@ -146,9 +170,10 @@ def test_sparse_attention_gather_shapes(tam_lib, oracle_mod, N, Hq, Hkv, d, kb, 
     check_close(lse.cpu().numpy().T[rows], rl, LSE_ATOL, "gather lse")
 
 
-def test_indexer_ties_keep_smallest_indices(tam_lib):
+@pytest.mark.parametrize("N", [900, 9000])
+def test_indexer_ties_keep_smallest_indices(tam_lib, N):
     """q_idx = 0 makes every score 0: the smallest key indices must be chosen."""
-    N, kb = 900, 40
+    kb = 40
     inp = _inputs(N, 8, 2, 128, seed=3)
     qx, kx = tam_synth.indexer_projections(inp, 64, seed=2)
     qx = torch.zeros_like(qx)
@@ -160,7 +185,7 @@ def test_indexer_ties_keep_smallest_indices(tam_lib):
 
 
 @pytest.mark.parametrize("N,kb", [(3000, 4), (2500, 300)])
-def test_indexer_heavy_compaction(tam_lib, oracle_mod, N, kb):
+def test_indexer_small_budget_long_rows(tam_lib, oracle_mod, N, kb):
     inp = _inputs(N, 8, 2, 128, seed=kb, sink=True, needles=5)
     qx, kx = tam_synth.indexer_projections(inp, 64, seed=2)
     res = tam_lib.indexer_topk(qx.cuda(), kx.cuda(), kb)
@@ -168,7 +193,7 @@ def test_indexer_heavy_compaction(tam_lib, oracle_mod, N, kb):
     oi, ol, _ = oracle_mod.indexer_topk_rows(qx, kx, kb, rows)
     S = qx.double().numpy()[rows] @ kx.double().numpy().T
     check_support(res.idx.cpu().numpy()[rows], res.length.cpu().numpy()[rows],
-                  res.value.cpu().numpy()[rows], oi, ol, S, 1e-3, "indexer compaction")
+                  res.value.cpu().numpy()[rows], oi, ol, S, 1e-3, "indexer small budget")
 
 
 def test_indexer_forced_timeout_is_reported(tam_lib, monkeypatch):

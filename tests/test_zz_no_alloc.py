@@ -53,8 +53,8 @@ def test_noalloc_matches_workspace_entry_point(tam_lib, N, kb, bq):
 
 def test_noalloc_rejects_problems_beyond_the_static_scratch(tam_lib):
     L = tam_lib.lib()
-    N, kb = 65536, 4096                    # candidate buffers alone need ~4.3 GB
-    need = L.tam_mass_select_workspace(N, 32, 8, 128, 0, kb, 1)
+    N, kb = 262144, 4096                   # lse + 64 mass rows alone need ~96 MiB
+    need = L.tam_mass_workspace_min(N, 32, 8, 128, 0, kb, 1)
     assert need > (64 << 20)
     dummy = torch.empty(16, dtype=torch.uint8, device="cuda")
     p = dummy.data_ptr()

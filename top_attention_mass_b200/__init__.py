@@ -36,10 +36,10 @@ TAM_ERR_CUDA, TAM_ERR_TIMEOUT, TAM_ERR_OVERFLOW = 4, 5, 6
 TAM_BF16, TAM_F32 = 0, 1
 
 EXPORTED = (
-    "tam_version", "tam_status_string", "tam_mass_oracle_workspace", "tam_mass_oracle_prefill",
-    "tam_attention_lse_workspace", "tam_attention_lse", "tam_mass_select_workspace",
-    "tam_mass_select", "tam_mass_select_noalloc", "tam_indexer_workspace",
-    "tam_indexer_topk", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
+    "tam_version", "tam_status_string", "tam_mass_oracle_workspace", "tam_mass_workspace_min",
+    "tam_mass_oracle_prefill", "tam_attention_lse_workspace", "tam_attention_lse",
+    "tam_mass_select_workspace", "tam_mass_select", "tam_mass_select_noalloc",
+    "tam_indexer_workspace", "tam_indexer_workspace_min", "tam_indexer_topk", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
     "tam_dense_workspace", "tam_dense_gqa_prefill", "tam_kernel_launches", "tam_check_status",
 )
 
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.tam_status_string.argtypes = [i32]
         L.tam_mass_oracle_workspace.restype = sz
         L.tam_mass_oracle_workspace.argtypes = [i64, i32, i32, i32, i32, i32, i32]
+        L.tam_mass_workspace_min.restype = sz
+        L.tam_mass_workspace_min.argtypes = [i64, i32, i32, i32, i32, i32, i32]
         L.tam_mass_oracle_prefill.restype = i32
         L.tam_mass_oracle_prefill.argtypes = [i64, i32, i32, i32, i32, p, p, p, i32, i32, p, p, p,
                                               p, p, p, sz, p]
@@ -91,6 +93,8 @@ def lib() -> ctypes.CDLL:
                                               p]
         L.tam_indexer_workspace.restype = sz
         L.tam_indexer_workspace.argtypes = [i64, i32, i32, i32, i32]
+        L.tam_indexer_workspace_min.restype = sz
+        L.tam_indexer_workspace_min.argtypes = [i64, i32, i32, i32, i32]
         L.tam_indexer_topk.restype = i32
         L.tam_indexer_topk.argtypes = [i64, i32, i32, p, p, i32, i32, p, p, p, p, sz, p]
         L.tam_sparse_attention_workspace.restype = sz
@@ -226,8 +230,11 @@ class Support:
 def mass_oracle_prefill(q, k, v=None, budget_k: int = 1, block_q: int = 1, *,
                         compute_out: bool = True, return_lse: bool = True,
                         workspace: Optional[Workspace] = None, stream=None, check: bool = True,
-                        device=None) -> Support:
-    """Attention-mass top-k oracle (passes 1-3) for one causal GQA prefill layer."""
+                        device=None, workspace_bytes: Optional[int] = None) -> Support:
+    """Attention-mass top-k oracle (passes 1-3) for one causal GQA prefill layer.
+
+    workspace_bytes: pass this many workspace bytes instead of the preferred size
+    (at least tam_mass_workspace_min; a smaller slab only means more chunks)."""
     dev = _dev_of(q, device)
     (q, k, v), host = _to_device([q, k, v], dev)
     N, Hq, Hkv, d = _shape(q, k)
@@ -246,10 +253,13 @@ def mass_oracle_prefill(q, k, v=None, budget_k: int = 1, block_q: int = 1, *,
         _raise(L.tam_mass_oracle_prefill(N, Hq, Hkv, d, dt, None, None, None, budget_k, block_q,
                                          None, None, None, None, None, None, 0, None),
                "mass_oracle_prefill")
+    if workspace_bytes is not None:
+        nbytes = int(workspace_bytes)
     ws = _workspace(dev, nbytes, workspace)
     rc = L.tam_mass_oracle_prefill(N, Hq, Hkv, d, dt, _ptr(q), _ptr(k), _ptr(v), budget_k, block_q,
                                    _ptr(sup_idx), _ptr(sup_len), _ptr(sup_mass), _ptr(lse),
-                                   _ptr(out), _ptr(ws), ws.numel(), _stream(dev, stream))
+                                   _ptr(out), _ptr(ws), min(ws.numel(), nbytes),
+                                   _stream(dev, stream))
     _raise(rc, "mass_oracle_prefill")
     if check:
         check_status(ws, stream)
@@ -279,8 +289,11 @@ def attention_lse(q, k, *, workspace: Optional[Workspace] = None, stream=None,
 
 
 def mass_select(q, k, lse, budget_k: int, block_q: int = 1, *,
-                workspace: Optional[Workspace] = None, stream=None, check: bool = True) -> Support:
-    """Pass 2: head-averaged mass and its top-k support, given pass 1's lse [Hq, N]."""
+                workspace: Optional[Workspace] = None, stream=None, check: bool = True,
+                workspace_bytes: Optional[int] = None) -> Support:
+    """Pass 2: head-averaged mass and its top-k support, given pass 1's lse [Hq, N].
+
+    workspace_bytes: as in mass_oracle_prefill."""
     dev = q.device
     N, Hq, Hkv, d = _shape(q, k)
     dt = _dtype_code(q)
@@ -292,10 +305,12 @@ def mass_select(q, k, lse, budget_k: int, block_q: int = 1, *,
     sup_mass = torch.empty(n_sel, budget_k, dtype=torch.float32, device=dev)
     L = lib()
     nbytes = L.tam_mass_select_workspace(N, Hq, Hkv, d, dt, budget_k, block_q)
+    if workspace_bytes is not None and nbytes:
+        nbytes = int(workspace_bytes)
     ws = _workspace(dev, max(nbytes, 256), workspace)
     rc = L.tam_mass_select(N, Hq, Hkv, d, dt, _ptr(q.contiguous()), _ptr(k.contiguous()),
                            _ptr(lse.contiguous()), budget_k, block_q, _ptr(sup_idx), _ptr(sup_len),
-                           _ptr(sup_mass), _ptr(ws), ws.numel() if nbytes else 0,
+                           _ptr(sup_mass), _ptr(ws), min(ws.numel(), nbytes) if nbytes else 0,
                            _stream(dev, stream))
     _raise(rc, "mass_select")
     if check:
@@ -305,8 +320,11 @@ def mass_select(q, k, lse, budget_k: int, block_q: int = 1, *,
 
 def indexer_topk(q_idx, k_idx, budget_k: int, block_q: int = 1, *,
                  workspace: Optional[Workspace] = None, stream=None, check: bool = True,
-                 device=None) -> Support:
-    """Head-collapsed indexer support: top-k of q_idx . k_idx per query."""
+                 device=None, workspace_bytes: Optional[int] = None) -> Support:
+    """Head-collapsed indexer support: top-k of q_idx . k_idx per query.
+
+    workspace_bytes: at least tam_indexer_workspace_min (more chunks below the
+    preferred size)."""
     dev = _dev_of(q_idx, device)
     (q_idx, k_idx), host = _to_device([q_idx, k_idx], dev)
     N, dx = q_idx.shape
@@ -318,10 +336,12 @@ def indexer_topk(q_idx, k_idx, budget_k: int, block_q: int = 1, *,
     sup_score = torch.empty(N, budget_k, dtype=torch.float32, device=dev)
     L = lib()
     nbytes = L.tam_indexer_workspace(N, dx, dt, budget_k, block_q)
+    if workspace_bytes is not None and nbytes:
+        nbytes = int(workspace_bytes)
     ws = _workspace(dev, max(nbytes, 256), workspace)
     rc = L.tam_indexer_topk(N, dx, dt, _ptr(q_idx), _ptr(k_idx), budget_k, block_q,
                             _ptr(sup_idx), _ptr(sup_len), _ptr(sup_score), _ptr(ws),
-                            ws.numel() if nbytes else 0, _stream(dev, stream))
+                            min(ws.numel(), nbytes) if nbytes else 0, _stream(dev, stream))
     _raise(rc, "indexer_topk")
     if check:
         check_status(ws, stream)

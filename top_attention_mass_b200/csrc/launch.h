@@ -27,8 +27,8 @@ struct MassArgs {
     int budget, block_q, n_sel;
     int n_ctas;           // persistent blocks (CUDA-core path)
     float* scratch;       // n_ctas * N floats (CUDA-core path)
-    void* cand;           // candidate buffers (tensor-core path, per query)
-    int cand_cap;         // entries per query row in `cand`
+    float* rows;          // triangular slab of mass rows (tensor-core path, per query)
+    int64_t row0, row1;   // the queries whose rows this launch writes (per query)
     void* bmass;          // fixed-point block mass (tensor-core path, block-shared)
     int32_t* sup_idx;
     int32_t* sup_len;
@@ -58,9 +58,9 @@ struct IndexerArgs {
     const void* k_idx;
     int budget;
     int n_ctas;
-    float* scratch;
-    void* cand;
-    int cand_cap;
+    float* scratch;       // n_ctas * N floats (CUDA-core path)
+    float* rows;          // triangular slab of score rows (tensor-core path)
+    int64_t row0, row1;   // the queries whose rows this launch writes
     int32_t* sup_idx;
     int32_t* sup_len;
     float* sup_score;
@@ -76,11 +76,21 @@ cudaError_t tc_lse(const LseArgs& a, cudaStream_t st);
 int tc_mass_columns(const MassArgs& a);
 bool tc_mass_supported(const MassArgs& a);
 size_t tc_mass_block_bytes(int64_t N, int block_q);
-cudaError_t tc_mass_select(const MassArgs& a, cudaStream_t st);
+// Per query: writes the mass rows [row0, row1) to the slab (select with row_topk);
+// block-shared: block sums and the block top-k, the whole of pass 2.
+cudaError_t tc_mass_pass(const MassArgs& a, cudaStream_t st);
 bool pair_mass_supported(const MassArgs& a);
-cudaError_t pair_mass_select(const MassArgs& a, cudaStream_t st);
+cudaError_t pair_mass(const MassArgs& a, cudaStream_t st);
 bool tc_indexer_supported(int64_t N, int d_idx, int dtype, int block_q);
-cudaError_t tc_indexer_select(const IndexerArgs& a, cudaStream_t st);
+// Writes the indexer score rows [row0, row1) to the slab (select with row_topk).
+cudaError_t tc_indexer_rows(const IndexerArgs& a, cudaStream_t st);
+
+// Row slabs: row i (i + 1 values) starts tri(i) - tri(row0) floats after the base.
+inline int64_t tri(int64_t i) { return i * (i + 1) / 2; }
+// Exact top-min(k, i+1) of each slab row i in [row0, row1), ascending key index,
+// ties toward the smaller index; sup_* are indexed by the absolute row i.
+cudaError_t row_topk(const float* slab, int64_t row0, int64_t row1, int budget, int32_t* sup_idx,
+                     int32_t* sup_len, float* sup_val, cudaStream_t st);
 bool tc_dense_supported(const AttnArgs& a);
 cudaError_t tc_dense(const AttnArgs& a, cudaStream_t st);
 bool gather_supported(const AttnArgs& a);

@@ -1,7 +1,8 @@
 // Pass 2 on CTA pairs: head-averaged mass and its top-k with 2-SM UMMA.
 //
 //   P_i[j] = (1/Hq) sum_h exp(scale * q[i,h].k[j,g(h)] - lse[h,i]),  j <= i
-//   per query:  S_i = top-min(k, i+1) of P_i;   per block: M_b[j] sums, as in mass_tc.cu
+//   per query:  the rows P_i, written to a triangular slab for the row top-k;
+//   per block:  M_b[j] = sum_{i in b, j <= i} P_i[j], as in mass_tc.cu
 //
 // (arXiv 2606.07703, Abstract; gist.science technical report §2.1 "Selektion",
 // "Granularität".)
@@ -14,7 +15,7 @@
 // read from L2 then serves 32 queries instead of 16, and each CTA reads half as many
 // operand bytes per unit of work - the two things that bounded the single-CTA pass.
 //
-// Roles in each CTA (512 threads):
+// Roles in each CTA (320 threads):
 //   warp 8      TMA producer: this CTA's Q half (once) and its 128 keys of each
 //               256-key tile, counted on CTA 0's barriers;
 //   warp 9      CTA 0 only: issues the pair MMAs into a ring of four 128-column TMEM
@@ -23,50 +24,39 @@
 //               column half w / 4, i.e. the (query, head) columns of half the pair's
 //               queries; exp2 against the pass-1 LSE, sum over heads -> mass of those
 //               queries for 128 keys.  Two warps per TMEM lane quarter keep two
-//               exp streams per scheduler.  Per query, the queries of column half h
-//               belong to the select warps of CTA h, so the warps of the other half
-//               write their values into the peer's shared memory (DSMEM) - both
-//               select groups then see their queries over all 256 keys, in ascending
-//               key order.  Block-shared mass goes to the fixed-point block sums;
-//   warps 10-15 select warps: the streaming exact top-k of mass_tc.cu.
+//               exp streams per scheduler.  Per query the mass goes to the row slab
+//               (one coalesced 128-byte store per warp and query); block-shared mass
+//               goes to the fixed-point block sums.
 // Every wait is bounded; the pair shakes hands before it frees TMEM and exits so
-// that no DSMEM write, remote arrive or MMA of one CTA can land after the other left.
+// that no remote arrive or MMA of one CTA can land after the other left.
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
-#include "warp_select.cuh"
 
 namespace tam {
 namespace {
 
-using namespace sel;
-
 constexpr int kStages = 2;
-constexpr int kSelWarps = 6;
 constexpr int kMassWarps = 8;
 constexpr int kProducerWarp = kMassWarps, kMmaWarp = kMassWarps + 1;
-constexpr int kThreads = 32 * (kMassWarps + 2 + kSelWarps);
+constexpr int kThreads = 32 * (kMassWarps + 2);
 constexpr int kNQ = 128;                // MMA N: (query, head) columns of the pair
 constexpr int kHalfRows = 64;           // B rows held by each CTA
 constexpr int kR = 512 / kNQ;           // TMEM accumulator slots
 constexpr int kTileKeys = 256;          // keys per pair tile (128 per CTA)
 
-__host__ __device__ constexpr int pair_smem_bytes(int D, int Hkv, int G, bool block) {
-    // Q half + K ring + lse of all 128 columns + (per query) one 16 x 256 mass tile and
-    // the select histograms + barriers
-    return 1024 + Hkv * kHalfRows * D * 2 + kStages * 128 * D * 2 + Hkv * kNQ * 4 + 512 +
-           (block ? 0 : (kHalfRows / G) * kTileKeys * 4 + kSelWarps * (int)sizeof(SelWarpSmem));
+__host__ __device__ constexpr int pair_smem_bytes(int D, int Hkv) {
+    // Q half + K ring + lse of all 128 columns + barriers
+    return 1024 + Hkv * kHalfRows * D * 2 + kStages * 128 * D * 2 + Hkv * kNQ * 4 + 512;
 }
 constexpr int kMaxDynSmem = 227 * 1024;
 
 struct PairParams {
-    int N, Hq, Hkv, n_pairs, budget, block_q, cap;
+    int N, Hq, Hkv, pair0, n_pairs, block_q;
+    int64_t row0, row1;       // per query: the slab holds rows [row0, row1)
     float sl2, inv_hq;
     const float* lse;
-    int32_t* sup_idx;
-    int32_t* sup_len;
-    float* sup_mass;
-    uint32_t* cand;
+    float* rows;
     unsigned long long* bmass;
     int32_t* status;
     uint64_t timeout_ns;
@@ -82,12 +72,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const PairParams p) {
     constexpr int BQP = kNQ / G;              // queries of the pair
-    constexpr int BQC = kHalfRows / G;        // queries whose top-k this CTA owns
+    constexpr int BQC = kHalfRows / G;        // queries of one column half
     constexpr int NH = D / 64;
     constexpr uint32_t kQHalf = kHalfRows * 128;   // one 64-element half of a group's B rows
     constexpr uint32_t kKHalf = 128 * 128;
     constexpr uint32_t kKTile = NH * kKHalf;
-    constexpr int QPW = (BQC + kSelWarps - 1) / kSelWarps;
     const int Hkv = p.Hkv;
 
     extern __shared__ uint8_t smem_raw[];
@@ -96,17 +85,13 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     uint8_t* sQ = base;
     uint8_t* sK = sQ + Hkv * NH * kQHalf;
     float* sLse = reinterpret_cast<float*>(sK + kStages * kKTile);     // Hkv * 128
-    float* sMass = sLse + Hkv * kNQ;                                   // BQC x 256 (per query)
-    SelWarpSmem* sSel = reinterpret_cast<SelWarpSmem*>(sMass + (BLOCK ? 0 : BQC * kTileKeys));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + (BLOCK ? 0 : kSelWarps));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sLse + Hkv * kNQ);
     uint64_t* q_full = bars;                 // CTA 0's counts both CTAs' Q bytes
     uint64_t* k_full = q_full + 1;           // CTA 0's counts both CTAs' K bytes
     uint64_t* k_empty = k_full + kStages;    // both (pair commits)
     uint64_t* s_full = k_empty + kStages;    // both (pair commits)
     uint64_t* s_empty = s_full + kR;         // CTA 0's: both CTAs' mass threads
-    uint64_t* m_full = s_empty + kR;         // each: own + peer mass threads
-    uint64_t* m_empty = m_full + 1;          // each: own + peer select warps
-    uint64_t* mma_done = m_empty + 1;        // both (pair commit)
+    uint64_t* mma_done = s_empty + kR;       // both (pair commit)
     uint64_t* exit_bar = mma_done + 1;       // each: the peer's arrival at the end
     uint64_t* never = exit_bar + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
@@ -115,12 +100,13 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = tc::cluster_rank();
     const uint32_t peer = rank ^ 1u;
-    const int pt = p.n_pairs - 1 - (int)(blockIdx.x >> 1);   // heaviest pair first
+    const int pt = p.pair0 + p.n_pairs - 1 - (int)(blockIdx.x >> 1);   // heaviest pair first
     const int q0 = pt * BQP;
     const int q_last = min(p.N, q0 + BQP) - 1;
     const int n_kt = q_last / kTileKeys + 1;
     const int n_units = n_kt * Hkv;
     const int my_q0 = q0 + (int)rank * BQC;
+    const int64_t slab0 = p.row0 * (p.row0 + 1) / 2;
 
     if (threadIdx.x == 0) {
         tc::mbar_init(q_full, 1);
@@ -132,8 +118,6 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             tc::mbar_init(&s_full[s], 1);
             tc::mbar_init(&s_empty[s], 2 * kMassWarps);   // every mass warp of both CTAs
         }
-        tc::mbar_init(m_full, kMassWarps);        // the mass warps (both CTAs) of this half
-        tc::mbar_init(m_empty, 2 * kSelWarps);
         tc::mbar_init(mma_done, 1);
         tc::mbar_init(exit_bar, 1);
         tc::mbar_init(never, 1);
@@ -227,11 +211,6 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * kCols);
         const uint32_t s_empty_leader = tc::map_to_cta(tc::smem_u32(s_empty), 0);
-        // the queries of this half belong to CTA `half`: its m_full and mass tile
-        const bool own = half == (int)rank;
-        const uint32_t m_full_owner = own ? tc::smem_u32(m_full)
-                                          : tc::map_to_cta(tc::smem_u32(m_full), peer);
-        const uint32_t mass_peer = tc::map_to_cta(tc::smem_u32(sMass), peer);
         bool ok = true;
         if (p.dbg & kDebugForceTimeout) ok = tc::wait(never, 0, gd, 9);
         for (int kt = 0; ok && kt < n_kt; ++kt) {
@@ -276,21 +255,13 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             if (!ok) break;
             const int j = kt * kTileKeys + (int)rank * 128 + row;
             if constexpr (!BLOCK) {
-                if (!tc::wait_cluster(m_empty, (kt & 1) ^ 1, gd, 6)) { ok = false; break; }
+                // row i of the slab starts tri(i) - tri(row0) floats in; lanes store
+                // consecutive keys of one query
 #pragma unroll
                 for (int ql = 0; ql < BQC; ++ql) {
-                    const int i = q0 + half * BQC + ql;
-                    const float val = (j <= i && i < p.N) ? acc[ql] * p.inv_hq : -INFINITY;
-                    const int off = ql * kTileKeys + (int)rank * 128 + row;
-                    if (own) sMass[off] = val;
-                    else tc::st_cluster_f32(mass_peer + (uint32_t)off * 4u, val);
-                }
-                // every lane's (DSMEM) stores are ordered before lane 0's release
-                asm volatile("fence.acq_rel.cluster;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) {
-                    if (own) tc::mbar_arrive(m_full);
-                    else tc::mbar_arrive_remote(m_full_owner);
+                    const int64_t i = q0 + half * BQC + ql;
+                    if (j <= i && i >= p.row0 && i < p.row1)
+                        p.rows[i * (i + 1) / 2 - slab0 + j] = acc[ql] * p.inv_hq;
                 }
             } else {
                 const int qh = q0 + half * BQC;
@@ -314,99 +285,6 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 if (part > 0.f)
                     atomicAdd(&p.bmass[bmass_row(cur_b, p.block_q) + j],
                               (unsigned long long)__float2ll_rn(part * p.inv_hq * 1099511627776.0f));
-            }
-        }
-        if constexpr (!BLOCK) {
-            // the peer's select warps release the last tile remotely: wait for it here
-            if (n_kt > 0 && !*abort_flag) tc::wait_cluster(m_empty, (n_kt - 1) & 1, drain, 0);
-        }
-    } else if constexpr (!BLOCK) {
-        // ---------------------------------------------------------------- select warps
-        const int sw = warp - (kMassWarps + 2);
-        int* hist = sSel[sw].hist;
-        const uint32_t m_empty_peer = tc::map_to_cta(tc::smem_u32(m_empty), peer);
-        float tau[QPW];
-        int cnt[QPW];
-#pragma unroll
-        for (int a = 0; a < QPW; ++a) {
-            tau[a] = -INFINITY;
-            cnt[a] = 0;
-        }
-        bool ok = true;
-        bool overflow = false;
-        for (int kt = 0; ok && kt < n_kt; ++kt) {
-            if (!tc::wait_cluster(m_full, kt & 1, gd, 7)) { ok = false; break; }
-#pragma unroll
-            for (int a = 0; a < QPW; ++a) {
-                const int ql = sw + a * kSelWarps;
-                const int i = my_q0 + ql;
-                if (ql >= BQC || i >= p.N) continue;
-                uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
-                uint32_t* idxs = keys + p.cap;
-#pragma unroll
-                for (int r = 0; r < kTileKeys / 32; ++r) {
-                    const float v = sMass[ql * kTileKeys + r * 32 + lane];
-                    const bool pass = v > tau[a];
-                    const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-                    const int pos = cnt[a] + __popc(bal & lanemask_lt());
-                    if (pass) {
-                        if (pos < p.cap) {
-                            keys[pos] = key_of(v);
-                            idxs[pos] = (uint32_t)(kt * kTileKeys + r * 32 + lane);
-                        } else {
-                            overflow = true;
-                        }
-                    }
-                    cnt[a] += __popc(bal);
-                    if (cnt[a] > p.cap - 32 && cnt[a] > p.budget) {
-                        __syncwarp();
-                        const int n = min(cnt[a], p.cap);
-                        uint32_t T;
-                        int take_eq;
-                        warp_kth(keys, n, p.budget, hist, T, take_eq, 2);
-                        int kept = n;
-                        if (T > 0u) kept = warp_select(keys, idxs, n, T - 1u, 0, false, nullptr, nullptr);
-                        if (kept > p.cap - 96) {
-                            warp_kth(keys, kept, p.budget, hist, T, take_eq, 4);
-                            kept = warp_select(keys, idxs, kept, T, take_eq, false, nullptr, nullptr);
-                            tau[a] = fmaxf(tau[a], value_of(T));
-                        } else if (T > 0u) {
-                            tau[a] = fmaxf(tau[a], value_of(T - 1u));
-                        }
-                        cnt[a] = kept;
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(m_empty);
-                tc::mbar_arrive_remote(m_empty_peer);
-            }
-        }
-        if (__any_sync(0xffffffffu, overflow) && lane == 0)
-            report_error(p.status, TAM_ERR_OVERFLOW, KID_MASS_TC, my_q0);
-        if (ok) {
-#pragma unroll
-            for (int a = 0; a < QPW; ++a) {
-                const int ql = sw + a * kSelWarps;
-                const int i = my_q0 + ql;
-                if (ql >= BQC || i >= p.N) continue;
-                uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
-                uint32_t* idxs = keys + p.cap;
-                const int n = min(cnt[a], p.cap);
-                __syncwarp();
-                uint32_t T = 0;
-                int take_eq = 0;
-                const bool all = n <= p.budget;
-                if (!all) warp_kth(keys, n, p.budget, hist, T, take_eq);
-                int32_t* oi = p.sup_idx + (size_t)i * p.budget;
-                float* om = p.sup_mass + (size_t)i * p.budget;
-                const int kept = warp_select(keys, idxs, n, T, take_eq, all, oi, om);
-                for (int t = kept + lane; t < p.budget; t += 32) {
-                    oi[t] = -1;
-                    om[t] = 0.f;
-                }
-                if (lane == 0) p.sup_len[i] = kept;
             }
         }
     }
@@ -437,22 +315,23 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     p.N = (int)a.N;
     p.Hq = a.Hq;
     p.Hkv = a.Hkv;
-    p.n_pairs = (int)((a.N + BQP - 1) / BQP);
-    p.budget = a.budget;
+    // per query the launch covers the queries [row0, row1) (row0 a multiple of BQP)
+    const int64_t r0 = BLOCK ? 0 : a.row0, r1 = BLOCK ? a.N : a.row1;
+    p.pair0 = (int)(r0 / BQP);
+    p.n_pairs = (int)((r1 + BQP - 1) / BQP) - p.pair0;
+    p.row0 = r0;
+    p.row1 = r1;
     p.block_q = a.block_q;
-    p.cap = a.cand_cap;
     p.sl2 = a.sl2;
     p.inv_hq = 1.f / (float)a.Hq;
     p.lse = a.lse;
-    p.sup_idx = a.sup_idx;
-    p.sup_len = a.sup_len;
-    p.sup_mass = a.sup_mass;
-    p.cand = reinterpret_cast<uint32_t*>(a.cand);
+    p.rows = a.rows;
     p.bmass = reinterpret_cast<unsigned long long*>(a.bmass);
     p.status = a.status;
     p.timeout_ns = wait_timeout_ns();
     p.dbg = debug_flags();
-    const int smem = pair_smem_bytes(D, a.Hkv, G, BLOCK);
+    if (p.n_pairs <= 0) return cudaSuccess;
+    const int smem = pair_smem_bytes(D, a.Hkv);
     auto kern = k_mass_pair<G, D, BLOCK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -483,12 +362,12 @@ bool pair_mass_supported(const MassArgs& a) {
     if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128)) return false;
     if (G != 4 && G != 8 && G != 16) return false;
     if (a.block_q > 1 && a.block_q > (1 << 20)) return false;
-    if (a.block_q == 1 && a.budget + 96 > a.cand_cap) return false;   // compaction slack
-    return pair_smem_bytes(a.d, a.Hkv, G, a.block_q > 1) <= kMaxDynSmem;
+    return pair_smem_bytes(a.d, a.Hkv) <= kMaxDynSmem;
 }
 
-// Launches the pair kernel only; in block mode the caller runs the block top-k after it.
-cudaError_t pair_mass_select(const MassArgs& a, cudaStream_t st) {
+// Launches the pair kernel only: per query it fills the slab rows [row0, row1); per
+// block the caller runs the block top-k after it.
+cudaError_t pair_mass(const MassArgs& a, cudaStream_t st) {
     const bool block = a.block_q > 1;
     if (a.d == 64) return block ? dispatch_g<64, true>(a, st) : dispatch_g<64, false>(a, st);
     return block ? dispatch_g<128, true>(a, st) : dispatch_g<128, false>(a, st);

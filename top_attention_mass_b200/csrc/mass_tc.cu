@@ -1,64 +1,55 @@
-// Pass 2 on the tensor cores: head-averaged token mass and its top-k support.
+// Pass 2 on the tensor cores: head-averaged token mass (and the indexer's scores).
 //
 //   P_i[j] = (1/Hq) sum_h exp(scale * q[i,h].k[j,g(h)] - lse[h,i]),  j <= i
-//   per query:  S_i = top-min(k, i+1) of P_i          (ranking: value desc, index asc)
+//   per query:  the rows P_i, written to a triangular slab; row_topk.cu then
+//               selects S_i = top-min(k, i+1) of each row (value desc, index asc)
 //   per block:  M_b[j] = sum_{i in block b, i >= j} P_i[j]  -> top-k in k_block_select
+//   indexer:    the rows s_i[j] = q_idx[i] . k_idx[j] (one head, no exponentials)
 //
 // (arXiv 2606.07703, Abstract: "selects head-averaged token support"; gist.science
-// technical report §2.1, "Mechanismus", "Selektion" and "Granularität".)
+// technical report §2.1, "Mechanismus", "Selektion" and "Granularität", §2.2 for
+// the indexer.)
 //
 // Orientation: one UMMA per KV group computes S^T = K_g Q_g^T with M = 128 keys
 // and N = NQ columns (BQ queries x G heads of that group).  A CTA keeps Q of its
 // BQ queries for *all* heads resident in shared memory, so the thread that owns a
 // key row adds the probabilities of every head of a query in registers - the head
-// average needs no cross-thread reduction and the N x N mass never leaves the SM.
-// Roles (320 threads):
+// average needs no cross-thread reduction.
+// Roles (192 threads):
 //   warp 4      TMA producer: Q (once, all groups), then K_g tiles in a 2-stage ring;
 //   warp 5      MMA issuer: for each key tile, one UMMA chain per group into a ring
 //               of 512/NQ TMEM slots;
 //   warps 0-3   mass warps: thread = key row; exp2 against the pass-1 LSE, sum over
-//               heads -> mass of BQ queries; causal mask; then either the mass tile
-//               goes to shared memory for the select warps (per query) or the
-//               block column sum is added in 2^-40 fixed point (block-shared);
-//   warps 6-11  select warps (per query): each owns every 6th query of the tile and
-//               runs a streaming exact top-k: a threshold tau plus a candidate buffer
-//               in global memory, appended in ascending key order.  When the buffer
-//               fills, a 2-pass warp radix select finds the 16-bit bin of the k-th
-//               value and drops everything below it (an exact 4-pass select keeps
-//               exactly k when the bin is too crowded); the final emit is exact
-//               (equal values keep the smaller index) and comes out ascending.
+//               heads -> mass of BQ queries; causal mask; then either the mass goes
+//               to the row slab (per query, indexer: lanes store consecutive keys of
+//               one query) or the block column sum is added in 2^-40 fixed point
+//               (block-shared).
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
-#include "warp_select.cuh"
 
 namespace tam {
 namespace {
 
 constexpr int kStages = 2;
-constexpr int kSelWarps = 6;                 // warps 6..11
-constexpr int kThreads = 32 * (6 + kSelWarps);
+constexpr int kThreads = 32 * 6;
 
-// Kernel modes: head-averaged mass with per-query top-k, block-shared mass sums,
-// or the head-collapsed indexer (one score per (query, key), no exponentials).
+// Kernel modes: head-averaged mass rows, block-shared mass sums, or the
+// head-collapsed indexer's score rows (one score per (query, key), no exponentials).
 constexpr int kModeQuery = 0, kModeBlock = 1, kModeIndexer = 2;
 
-using namespace sel;
-
-__host__ __device__ constexpr int mass_smem_bytes(int NQ, int D, int Hkv, int G, bool block) {
-    return 1024 + Hkv * NQ * D * 2 + kStages * 128 * D * 2 + Hkv * NQ * 4 + 512 +
-           (block ? 0 : 2 * (NQ / G) * 128 * 4 + kSelWarps * (int)sizeof(SelWarpSmem));
+// alignment slack + Q (all groups) + K ring + lse2 + barriers
+__host__ __device__ constexpr int mass_smem_bytes(int NQ, int D, int Hkv) {
+    return 1024 + Hkv * NQ * D * 2 + kStages * 128 * D * 2 + Hkv * NQ * 4 + 512;
 }
 constexpr int kMaxDynSmem = 227 * 1024;
 
 struct MassParams {
-    int N, Hq, Hkv, n_ctiles, budget, block_q, cap;
+    int N, Hq, Hkv, ct0, n_ctiles, block_q;
+    int64_t row0, row1;              // per query / indexer: the slab holds rows [row0, row1)
     float sl2, inv_hq;
     const float* lse;
-    int32_t* sup_idx;
-    int32_t* sup_len;
-    float* sup_mass;
-    uint32_t* cand;                  // [N][2*cap]: keys then idx (per query)
+    float* rows;                     // triangular row slab (per query / indexer)
     unsigned long long* bmass;       // triangular block mass (block mode)
     int32_t* status;
     uint64_t timeout_ns;
@@ -80,7 +71,6 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     constexpr uint32_t kQHalf = NQ * 128; // bytes of one 64-element half of a group's Q
     constexpr uint32_t kKHalf = 128 * 128;
     constexpr uint32_t kKTile = NH * kKHalf;
-    constexpr int QPW = (BQ + kSelWarps - 1) / kSelWarps;   // queries per select warp (at most)
     constexpr bool BLOCK = MODE == kModeBlock;
     constexpr bool INDEXER = MODE == kModeIndexer;
     const int Hkv = p.Hkv;
@@ -91,27 +81,24 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     uint8_t* sQ = base;                                   // Hkv * NH * kQHalf
     uint8_t* sK = sQ + Hkv * NH * kQHalf;                 // kStages * kKTile
     float* sLse = reinterpret_cast<float*>(sK + kStages * kKTile);   // Hkv * NQ
-    float* sMass = sLse + Hkv * NQ;                                    // 2 x BQ x 128 (per query)
-    SelWarpSmem* sSel = reinterpret_cast<SelWarpSmem*>(sMass + (BLOCK ? 0 : 2 * BQ * 128));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sSel + (BLOCK ? 0 : kSelWarps));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sLse + Hkv * NQ);
     uint64_t* q_full = bars;
     uint64_t* k_full = q_full + 1;
     uint64_t* k_empty = k_full + kStages;
     uint64_t* s_full = k_empty + kStages;
     uint64_t* s_empty = s_full + R;
-    uint64_t* m_full = s_empty + R;
-    uint64_t* m_empty = m_full + 2;
-    uint64_t* mma_done = m_empty + 2;
+    uint64_t* mma_done = s_empty + R;
     uint64_t* never = mma_done + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
     int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ct = p.n_ctiles - 1 - (int)blockIdx.x;      // heaviest tile first
+    const int ct = p.ct0 + p.n_ctiles - 1 - (int)blockIdx.x;   // heaviest tile first
     const int q0 = ct * BQ;
     const int q_last = min(p.N, q0 + BQ) - 1;
     const int n_kt = q_last / 128 + 1;
     const int n_units = n_kt * Hkv;
+    const int64_t slab0 = p.row0 * (p.row0 + 1) / 2;
 
     if (threadIdx.x == 0) {
         tc::mbar_init(q_full, 1);
@@ -122,10 +109,6 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         for (int s = 0; s < R; ++s) {
             tc::mbar_init(&s_full[s], 1);
             tc::mbar_init(&s_empty[s], 128);
-        }
-        for (int b = 0; b < 2; ++b) {
-            tc::mbar_init(&m_full[b], 128);
-            tc::mbar_init(&m_empty[b], 32 * kSelWarps);
         }
         tc::mbar_init(mma_done, 1);
         tc::mbar_init(never, 1);
@@ -262,16 +245,14 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             if (!ok) break;
             const int j = kt * 128 + row;
             if constexpr (!BLOCK) {
-                const int mb = kt & 1;
-                if (!tc::wait(&m_empty[mb], ((kt >> 1) & 1) ^ 1, gd, 6)) { ok = false; break; }
-                float* mt = sMass + mb * BQ * 128;
+                // row i of the slab starts tri(i) - tri(row0) floats in; lanes store
+                // consecutive keys of one query
 #pragma unroll
                 for (int q = 0; q < BQ; ++q) {
-                    const int i = q0 + q;
-                    mt[q * 128 + row] = (j <= i && i < p.N) ? (INDEXER ? acc[q] : acc[q] * p.inv_hq)
-                                                            : -INFINITY;
+                    const int64_t i = q0 + q;
+                    if (j <= i && i >= p.row0 && i < p.row1)
+                        p.rows[i * (i + 1) / 2 - slab0 + j] = INDEXER ? acc[q] : acc[q] * p.inv_hq;
                 }
-                tc::mbar_arrive(&m_full[mb]);
             } else {
                 // block column sums, 2^-40 fixed point, one add per (block, key)
                 int cur_b = q0 / p.block_q;
@@ -295,96 +276,6 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (part > 0.f)
                     atomicAdd(&p.bmass[bmass_offset(cur_b, p.block_q) + j],
                               (unsigned long long)__float2ll_rn(part * p.inv_hq * 1099511627776.0f));
-            }
-        }
-    } else if (!BLOCK) {
-        // ---------------------------------------------------------------- select warps
-        const int sw = warp - 6;
-        int* hist = sSel[sw].hist;
-        // select warp sw owns queries sw, sw + kSelWarps, ... of the tile
-        float tau[QPW];
-        int cnt[QPW];
-#pragma unroll
-        for (int a = 0; a < QPW; ++a) {
-            tau[a] = -INFINITY;     // masked entries are -inf and never pass
-            cnt[a] = 0;
-        }
-        bool ok = true;
-        bool overflow = false;
-        for (int kt = 0; ok && kt < n_kt; ++kt) {
-            const int mb = kt & 1;
-            if (!tc::wait(&m_full[mb], (kt >> 1) & 1, gd, 7)) { ok = false; break; }
-            const float* mt = sMass + mb * BQ * 128;
-#pragma unroll
-            for (int a = 0; a < QPW; ++a) {
-                const int q = sw + a * kSelWarps;
-                const int i = q0 + q;
-                if (q >= BQ || i >= p.N) continue;
-                uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
-                uint32_t* idxs = keys + p.cap;
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const float v = mt[q * 128 + r * 32 + lane];
-                    const bool pass = v > tau[a];
-                    const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-                    const int pos = cnt[a] + __popc(bal & lanemask_lt());
-                    if (pass) {
-                        if (pos < p.cap) {
-                            keys[pos] = key_of(v);
-                            idxs[pos] = (uint32_t)(kt * 128 + r * 32 + lane);
-                        } else {
-                            overflow = true;
-                        }
-                    }
-                    cnt[a] += __popc(bal);
-                }
-                if (cnt[a] > p.cap - 128 && cnt[a] > p.budget) {
-                    __syncwarp();
-                    const int n = min(cnt[a], p.cap);
-                    uint32_t T;
-                    int take_eq;
-                    // cheap first: keep every key in the k-th key's 16-bit bin or above
-                    warp_kth(keys, n, p.budget, hist, T, take_eq, 2);
-                    int kept = n;
-                    if (T > 0u) kept = warp_select(keys, idxs, n, T - 1u, 0, false, nullptr, nullptr);
-                    if (kept > p.cap - 256) {
-                        // the bin was too crowded to free space: exact, keeps exactly k
-                        warp_kth(keys, kept, p.budget, hist, T, take_eq, 4);
-                        kept = warp_select(keys, idxs, kept, T, take_eq, false, nullptr, nullptr);
-                        tau[a] = fmaxf(tau[a], value_of(T));   // accept key > T
-                    } else if (T > 0u) {
-                        tau[a] = fmaxf(tau[a], value_of(T - 1u));   // accept key >= T
-                    }
-                    cnt[a] = kept;
-                }
-            }
-            __syncwarp();
-            tc::mbar_arrive(&m_empty[mb]);
-        }
-        if (__any_sync(0xffffffffu, overflow) && lane == 0)
-            report_error(p.status, TAM_ERR_OVERFLOW, INDEXER ? KID_INDEXER_TC : KID_MASS_TC, q0);
-        if (ok) {
-#pragma unroll
-            for (int a = 0; a < QPW; ++a) {
-                const int q = sw + a * kSelWarps;
-                const int i = q0 + q;
-                if (q >= BQ || i >= p.N) continue;
-                uint32_t* keys = p.cand + (size_t)i * 2 * p.cap;
-                uint32_t* idxs = keys + p.cap;
-                const int n = min(cnt[a], p.cap);
-                __syncwarp();
-                uint32_t T = 0;
-                int take_eq = 0;
-                const bool all = n <= p.budget;
-                if (!all) warp_kth(keys, n, p.budget, hist, T, take_eq);
-                int32_t* oi = p.sup_idx + (size_t)i * p.budget;
-                float* om = p.sup_mass + (size_t)i * p.budget;
-                const int kept = warp_select(keys, idxs, n, T, take_eq, all, oi, om);
-                for (int t = kept + lane; t < p.budget; t += 32) {
-                    oi[t] = -1;
-                    om[t] = 0.f;
-                }
-                if (lane == 0) p.sup_len[i] = kept;
             }
         }
     }
@@ -488,22 +379,24 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     p.N = (int)a.N;
     p.Hq = a.Hq;
     p.Hkv = a.Hkv;
-    p.n_ctiles = (int)((a.N + BQ - 1) / BQ);
-    p.budget = a.budget;
+    // per query / indexer the launch covers the queries [row0, row1) (row0 a
+    // multiple of BQ)
+    const int64_t r0 = BLOCK ? 0 : a.row0, r1 = BLOCK ? a.N : a.row1;
+    p.ct0 = (int)(r0 / BQ);
+    p.n_ctiles = (int)((r1 + BQ - 1) / BQ) - p.ct0;
+    p.row0 = r0;
+    p.row1 = r1;
     p.block_q = a.block_q;
-    p.cap = a.cand_cap;
     p.sl2 = a.sl2;
     p.inv_hq = 1.f / (float)a.Hq;
     p.lse = a.lse;
-    p.sup_idx = a.sup_idx;
-    p.sup_len = a.sup_len;
-    p.sup_mass = a.sup_mass;
-    p.cand = reinterpret_cast<uint32_t*>(a.cand);
+    p.rows = a.rows;
     p.bmass = reinterpret_cast<unsigned long long*>(a.bmass);
     p.status = a.status;
     p.timeout_ns = wait_timeout_ns();
     p.dbg = debug_flags();
-    const int smem = mass_smem_bytes(NQ, D, a.Hkv, G, BLOCK);
+    if (p.n_ctiles <= 0) return cudaSuccess;
+    const int smem = mass_smem_bytes(NQ, D, a.Hkv);
     auto kern = k_mass_tc<G, D, NQ, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -571,14 +464,13 @@ int tc_mass_columns(const MassArgs& a) {
     // NQ columns per group: 128 (twice the queries per CTA, half the K re-reads) when
     // the Q of all groups plus the rest of the layout fits in shared memory, else 64.
     const int G = a.Hq / a.Hkv;
-    const bool block = a.block_q > 1;
     // (queries per CTA NQ/G kept within [4, 32] so the per-thread accumulators stay
-    // in registers and every select warp owns at least one query)
+    // in registers)
     if (a.Hkv > 64 || G < 1) return 0;
     for (int nq = 128; nq >= 32; nq >>= 1) {
         const int bq = nq / G;
         if (bq < 4 || bq > 32) continue;
-        if (mass_smem_bytes(nq, a.d, a.Hkv, G, block) <= kMaxDynSmem) return nq;
+        if (mass_smem_bytes(nq, a.d, a.Hkv) <= kMaxDynSmem) return nq;
     }
     return 0;
 }
@@ -597,9 +489,9 @@ size_t tc_mass_block_bytes(int64_t N, int block_q) {
     return (size_t)bmass_offset(nb, block_q) * 8;
 }
 
-cudaError_t tc_mass_select(const MassArgs& a, cudaStream_t st) {
+cudaError_t tc_mass_pass(const MassArgs& a, cudaStream_t st) {
     if (pair_mass_supported(a) && !pair_path_disabled()) {
-        cudaError_t e = pair_mass_select(a, st);
+        cudaError_t e = pair_mass(a, st);
         if (e != cudaSuccess || a.block_q == 1) return e;
         const int nb = (int)((a.N + a.block_q - 1) / a.block_q);
         k_block_select<<<nb, 256, 0, st>>>(reinterpret_cast<unsigned long long*>(a.bmass), (int)a.N,
@@ -614,7 +506,7 @@ bool tc_indexer_supported(int64_t N, int d_idx, int dtype, int block_q) {
     return dtype == TAM_BF16 && (d_idx == 64 || d_idx == 128) && block_q == 1 && N >= 1;
 }
 
-cudaError_t tc_indexer_select(const IndexerArgs& ia, cudaStream_t st) {
+cudaError_t tc_indexer_rows(const IndexerArgs& ia, cudaStream_t st) {
     MassArgs a{};
     a.N = ia.N;
     a.Hq = 1;
@@ -625,11 +517,9 @@ cudaError_t tc_indexer_select(const IndexerArgs& ia, cudaStream_t st) {
     a.k = ia.k_idx;
     a.budget = ia.budget;
     a.block_q = 1;
-    a.cand = ia.cand;
-    a.cand_cap = ia.cand_cap;
-    a.sup_idx = ia.sup_idx;
-    a.sup_len = ia.sup_len;
-    a.sup_mass = ia.sup_score;
+    a.rows = ia.rows;
+    a.row0 = ia.row0;
+    a.row1 = ia.row1;
     a.status = ia.status;
     return launch_indexer_tc(a, st);
 }

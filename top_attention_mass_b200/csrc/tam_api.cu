@@ -1,5 +1,6 @@
 // C ABI of libtam.so: argument checks, workspace layout and kernel dispatch.
 // Declarations and their contracts: include/tam.h.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -48,14 +49,42 @@ inline int64_t n_selection_units(int64_t N, int block_q) {
     return block_q == 1 ? N : (N + block_q - 1) / block_q;
 }
 
+// Per-query tensor-core pass 2 (and the indexer) materialise score rows in a
+// triangular slab and select from it; the slab holds the rows of a chunk of
+// queries.  Chunks start at multiples of 64 queries (a multiple of every kernel's
+// query tile); the preferred slab takes the whole problem up to 4 GiB, the smallest
+// usable one any 64 rows (64 N floats).
+constexpr size_t kSlabPrefBytes = size_t(4) << 30;
+constexpr int64_t kChunkRows = 64;
+
+size_t slab_pref_bytes(int64_t N) {
+    return std::min(kSlabPrefBytes, (size_t)tri(N) * sizeof(float));
+}
+size_t slab_min_bytes(int64_t N) {
+    return (size_t)std::min(tri(N), kChunkRows * N) * sizeof(float);
+}
+
+// End of the chunk that starts at r0 (a multiple of 64) for a slab of cap floats
+// (cap >= 64 N): the whole rest if it fits, else the most 64-row steps that do.
+int64_t chunk_end(int64_t r0, int64_t N, int64_t cap) {
+    if (tri(N) - tri(r0) <= cap) return N;
+    int64_t lo = 1, hi = (N - r0) / kChunkRows + 1;
+    while (hi - lo > 1) {
+        const int64_t mid = (lo + hi) / 2;
+        if (tri(r0 + mid * kChunkRows) - tri(r0) <= cap) lo = mid; else hi = mid;
+    }
+    return std::min(N, r0 + lo * kChunkRows);
+}
+
 // Workspace layout of tam_mass_oracle_prefill / tam_mass_select: status block, lse
 // (when the caller passes none), then the pass-2 scratch of whichever kernel runs:
-// candidate buffers (tensor cores, per query), fixed-point block mass (tensor cores,
-// block-shared) or staged mass rows (CUDA cores).
+// the row slab (tensor cores, per query), fixed-point block mass (tensor cores,
+// block-shared) or staged mass rows (CUDA cores).  `total` is the preferred size,
+// `min_total` the smallest accepted (a smaller slab only means more chunks).
 struct MassPlan {
-    size_t off_lse, off_work, total;
-    bool tc;
-    int n_ctas, cand_cap;
+    size_t off_lse, off_work, total, min_total;
+    bool tc, slab;
+    int n_ctas;
 };
 
 MassArgs mass_shape(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k, int block_q) {
@@ -70,36 +99,39 @@ MassPlan plan_mass(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k, i
     const int64_t n_sel = n_selection_units(N, block_q);
     p.tc = tc_mass_supported(mass_shape(N, Hq, Hkv, d, dtype, budget_k, block_q));
     p.n_ctas = (int)std::min<int64_t>(n_sel, kSimtPersistentCtas);
-    p.cand_cap = candidate_capacity(budget_k);
+    p.slab = p.tc && block_q == 1;
     p.off_lse = kStatusBytes;
     p.off_work = p.off_lse + align256((size_t)Hq * N * sizeof(float));
-    size_t work;
+    size_t work, min_work;
     if (!p.tc)
-        work = (size_t)p.n_ctas * N * sizeof(float);
-    else if (block_q == 1)
-        work = (size_t)N * p.cand_cap * 8;
-    else
-        work = tc_mass_block_bytes(N, block_q);
+        work = min_work = (size_t)p.n_ctas * N * sizeof(float);
+    else if (p.slab) {
+        work = slab_pref_bytes(N);
+        min_work = slab_min_bytes(N);
+    } else
+        work = min_work = tc_mass_block_bytes(N, block_q);
     p.total = p.off_work + align256(work);
+    p.min_total = p.off_work + align256(min_work);
     return p;
 }
 
-// Workspace of tam_indexer_topk: status block, then the candidate buffers of the
-// tensor-core path or the staged score rows of the CUDA-core path.
+// Workspace of tam_indexer_topk: status block, then the row slab of the tensor-core
+// path or the staged score rows of the CUDA-core path.
 struct IndexerPlan {
-    size_t off_scratch, total;
+    size_t off_scratch, total, min_total;
     bool tc;
-    int n_ctas, cand_cap;
+    int n_ctas;
 };
 
 IndexerPlan plan_indexer(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
+    (void)budget_k;
     IndexerPlan p{};
     p.tc = tc_indexer_supported(N, d_idx, dtype, block_q);
     p.n_ctas = (int)std::min<int64_t>(N, kSimtPersistentCtas);
-    p.cand_cap = candidate_capacity(budget_k);
     p.off_scratch = kStatusBytes;
-    const size_t work = p.tc ? (size_t)N * p.cand_cap * 8 : (size_t)p.n_ctas * N * sizeof(float);
-    p.total = p.off_scratch + align256(work);
+    const size_t simt = (size_t)p.n_ctas * N * sizeof(float);
+    p.total = p.off_scratch + align256(p.tc ? slab_pref_bytes(N) : simt);
+    p.min_total = p.off_scratch + align256(p.tc ? slab_min_bytes(N) : simt);
     return p;
 }
 
@@ -121,22 +153,35 @@ int start_call(void* workspace, cudaStream_t st) {
     return cuda_status(cudaMemsetAsync(workspace, 0, kStatusBytes, st));
 }
 
-// Pass 2 on an already computed lse, into the workspace laid out by plan_mass.
+// Pass 2 on an already computed lse, into the workspace laid out by plan_mass
+// (ws_bytes >= plan.min_total).
 int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
                        const float* lse, int budget_k, int block_q, int32_t* sup_idx,
-                       int32_t* sup_len, float* sup_mass, char* ws, const MassPlan& plan,
-                       cudaStream_t st) {
+                       int32_t* sup_len, float* sup_mass, char* ws, size_t ws_bytes,
+                       const MassPlan& plan, cudaStream_t st) {
     MassArgs ma = mass_shape(N, Hq, Hkv, d, dtype, budget_k, block_q);
     ma.q = q; ma.k = k; ma.lse = lse; ma.sl2 = score_log2_scale(d);
     ma.n_sel = (int)n_selection_units(N, block_q);
     ma.n_ctas = plan.n_ctas;
     ma.scratch = (float*)(ws + plan.off_work);
-    ma.cand = ws + plan.off_work;
-    ma.cand_cap = plan.cand_cap;
+    ma.rows = (float*)(ws + plan.off_work);
     ma.bmass = ws + plan.off_work;
     ma.sup_idx = sup_idx; ma.sup_len = sup_len; ma.sup_mass = sup_mass;
     ma.status = (int32_t*)ws;
-    return cuda_status(plan.tc ? tc_mass_select(ma, st) : simt_mass_select(ma, st));
+    if (!plan.tc) return cuda_status(simt_mass_select(ma, st));
+    if (!plan.slab) return cuda_status(tc_mass_pass(ma, st));
+    // per query: mass rows of a chunk of queries, then their top-k, chunk by chunk
+    const int64_t cap = (int64_t)((ws_bytes - plan.off_work) / sizeof(float));
+    for (int64_t r0 = 0; r0 < N;) {
+        const int64_t r1 = chunk_end(r0, N, cap);
+        ma.row0 = r0;
+        ma.row1 = r1;
+        cudaError_t e = tc_mass_pass(ma, st);
+        if (e == cudaSuccess) e = row_topk(ma.rows, r0, r1, budget_k, sup_idx, sup_len, sup_mass, st);
+        if (e != cudaSuccess) return TAM_ERR_CUDA;
+        r0 = r1;
+    }
+    return TAM_OK;
 }
 
 }  // namespace
@@ -155,7 +200,7 @@ const char* tam_status_string(int s) {
         case TAM_ERR_WORKSPACE: return "workspace too small";
         case TAM_ERR_CUDA: return "CUDA error";
         case TAM_ERR_TIMEOUT: return "device wait timed out";
-        case TAM_ERR_OVERFLOW: return "candidate buffer overflow";
+        case TAM_ERR_OVERFLOW: return "buffer overflow";
         default: return "unknown status";
     }
 }
@@ -181,7 +226,7 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return TAM_ERR_INVALID_ARG;
     const MassPlan plan = plan_mass(N, Hq, Hkv, d, dtype, budget_k, block_q);
-    if (ws_bytes < plan.total) return TAM_ERR_WORKSPACE;
+    if (ws_bytes < plan.min_total) return TAM_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     char* ws = (char*)workspace;
     int32_t* status = (int32_t*)ws;
@@ -193,7 +238,7 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
     if ((rc = cuda_status(run_lse(la, st)))) return rc;
 
     if ((rc = launch_mass_select(N, Hq, Hkv, d, dtype, q, k, lse_buf, budget_k, block_q, sup_idx,
-                                 sup_len, sup_mass, ws, plan, st)))
+                                 sup_len, sup_mass, ws, ws_bytes, plan, st)))
         return rc;
 
     if (out) {
@@ -202,6 +247,13 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
         if ((rc = cuda_status(run_sparse_attention(aa, st)))) return rc;
     }
     return TAM_OK;
+}
+
+size_t tam_mass_workspace_min(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
+                              int block_q) {
+    if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK) return 0;
+    if (check_budget(N, budget_k, block_q) != TAM_OK) return 0;
+    return plan_mass(N, Hq, Hkv, d, dtype, budget_k, block_q).min_total;
 }
 
 size_t tam_attention_lse_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {
@@ -243,11 +295,11 @@ int tam_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
     for (const void* p : ptrs)
         if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
     const MassPlan plan = plan_mass(N, Hq, Hkv, d, dtype, budget_k, block_q);
-    if (ws_bytes < plan.total) return TAM_ERR_WORKSPACE;
+    if (ws_bytes < plan.min_total) return TAM_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     if ((rc = start_call(workspace, st))) return rc;
     return launch_mass_select(N, Hq, Hkv, d, dtype, q, k, lse, budget_k, block_q, sup_idx, sup_len,
-                              sup_mass, (char*)workspace, plan, st);
+                              sup_mass, (char*)workspace, ws_bytes, plan, st);
 }
 
 size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
@@ -255,6 +307,11 @@ size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int 
     if (dtype != TAM_BF16 && dtype != TAM_F32) return 0;
     if (check_budget(N, budget_k, block_q) != TAM_OK || block_q != 1) return 0;
     return plan_indexer(N, d_idx, dtype, budget_k, block_q).total;
+}
+
+size_t tam_indexer_workspace_min(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
+    if (tam_indexer_workspace(N, d_idx, dtype, budget_k, block_q) == 0) return 0;
+    return plan_indexer(N, d_idx, dtype, budget_k, block_q).min_total;
 }
 
 int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const void* k_idx,
@@ -272,17 +329,29 @@ int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const v
     for (const void* p : ptrs)
         if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
     const IndexerPlan plan = plan_indexer(N, d_idx, dtype, budget_k, block_q);
-    if (ws_bytes < plan.total) return TAM_ERR_WORKSPACE;
+    if (ws_bytes < plan.min_total) return TAM_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
     char* ws = (char*)workspace;
     if ((rc = start_call(workspace, st))) return rc;
     IndexerArgs ia{};
     ia.N = N; ia.d_idx = d_idx; ia.dtype = dtype; ia.q_idx = q_idx; ia.k_idx = k_idx;
     ia.budget = budget_k; ia.n_ctas = plan.n_ctas; ia.scratch = (float*)(ws + plan.off_scratch);
-    ia.cand = ws + plan.off_scratch; ia.cand_cap = plan.cand_cap;
+    ia.rows = (float*)(ws + plan.off_scratch);
     ia.sup_idx = sup_idx; ia.sup_len = sup_len; ia.sup_score = sup_score;
     ia.status = (int32_t*)ws;
-    return cuda_status(plan.tc ? tc_indexer_select(ia, st) : simt_indexer_select(ia, st));
+    if (!plan.tc) return cuda_status(simt_indexer_select(ia, st));
+    // score rows of a chunk of queries, then their top-k, chunk by chunk
+    const int64_t cap = (int64_t)((ws_bytes - plan.off_scratch) / sizeof(float));
+    for (int64_t r0 = 0; r0 < N;) {
+        const int64_t r1 = chunk_end(r0, N, cap);
+        ia.row0 = r0;
+        ia.row1 = r1;
+        cudaError_t e = tc_indexer_rows(ia, st);
+        if (e == cudaSuccess) e = row_topk(ia.rows, r0, r1, budget_k, sup_idx, sup_len, sup_score, st);
+        if (e != cudaSuccess) return TAM_ERR_CUDA;
+        r0 = r1;
+    }
+    return TAM_OK;
 }
 
 size_t tam_sparse_attention_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {

@@ -52,7 +52,7 @@ extern "C" int tam_mass_select_noalloc(int64_t N, int Hq, int Hkv, int d, int dt
                                        const void* q, const void* k, const float* lse,
                                        int budget_k, int block_q, int32_t* sup_idx,
                                        int32_t* sup_len, float* sup_mass, void* stream) {
-    const size_t need = tam_mass_select_workspace(N, Hq, Hkv, d, dtype, budget_k, block_q);
+    const size_t need = tam_mass_workspace_min(N, Hq, Hkv, d, dtype, budget_k, block_q);
     if (need == 0) {
         // let the regular entry point name the argument error (it returns before any launch)
         return tam_mass_select(N, Hq, Hkv, d, dtype, q, k, lse, budget_k, block_q, sup_idx,

@@ -61,12 +61,4 @@ bool pair_path_disabled() { return env_int("TAM_DISABLE_PAIR_KERNELS", 0) != 0; 
 
 int debug_flags() { return env_int("TAM_DEBUG_FORCE_TIMEOUT", 0) ? kDebugForceTimeout : 0; }
 
-int candidate_capacity(int budget_k) {
-    const int forced = env_int("TAM_DEBUG_CAND_CAP", 0);
-    if (forced > 0) return forced;
-    // room for the retained top-k plus one 128-key tile of appends, rounded to 32
-    int cap = 2 * budget_k + 128;
-    return (cap + 31) & ~31;
-}
-
 }  // namespace tam

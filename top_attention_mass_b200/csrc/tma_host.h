@@ -22,10 +22,6 @@ bool make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
 uint64_t wait_timeout_ns();
 int debug_flags();
 
-// Entries per query row of the streaming top-k candidate buffer; the debug
-// variable TAM_DEBUG_CAND_CAP overrides it (to exercise the overflow report).
-int candidate_capacity(int budget_k);
-
 constexpr int kDebugForceTimeout = 1;
 
 // TAM_DISABLE_PAIR_KERNELS=1 routes pass 2 to the single-CTA kernel (A/B comparisons).
