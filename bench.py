@@ -246,8 +246,8 @@ L2_GATHER_GBS = 11074.1
 
 
 def traffic_table():
-    """DRAM bytes per launch from the committed ncu capture, for rows whose kernel source
-    is unchanged since the capture (sha256 match); other rows get None."""
+    """DRAM bytes per launch from the committed ncu capture, for rows whose kernel sources
+    are all unchanged since the capture (sha256 match); other rows get None."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "ncu_dram_traffic_gqa32k_step.json")
     try:
@@ -258,9 +258,12 @@ def traffic_table():
     out = {}
     for row, ent in tab.items():
         try:
-            with open(os.path.join(ROOT, ent["source"]), "rb") as f:
-                if hashlib.sha256(f.read()).hexdigest() == ent["sha256"]:
-                    out[row] = ent["dram_bytes_per_launch"]
+            same = True
+            for src, digest in ent["sources"].items():
+                with open(os.path.join(ROOT, src), "rb") as f:
+                    same = same and hashlib.sha256(f.read()).hexdigest() == digest
+            if same:
+                out[row] = ent["dram_bytes_per_launch"]
         except Exception:
             pass
     return out

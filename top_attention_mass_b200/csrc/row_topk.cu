@@ -15,25 +15,34 @@
 //
 // One CTA per row (longest rows first).  Values are compared as order-preserving
 // 32-bit keys, so any float (negative indexer scores included) orders exactly.
-//   1. threshold guess: the r-th largest of 512 evenly spaced samples, r chosen so
-//      that about 1.25 k + 64 keys of the row are expected at or above it;
-//   2. count the keys >= guess (per warp segment); if the count is outside
-//      [k, kCap] bisect the key range with further counting passes;
-//   3. ordered compaction of the keys >= guess into shared memory (at most kCap);
-//   4. exact k-th key T of the candidates by a 4 x 8-bit radix select, and how
-//      many keys equal to T are taken (the earliest ones);
+//   1. threshold guess: the r-th largest of s evenly spaced samples (s = 512, plus
+//      256 per 2^17 keys of the row, at most 4096), r = mu + 3 sqrt(mu) + 4, mu = s k / n
+//      the expected sample count at or above the k-th key, so that the guess lies
+//      below the k-th key unless the samples are three deviations off; rows of at
+//      most 2k + 256 keys take every key instead;
+//   2-3. one pass over the row, chunk by chunk: each thread takes 8 consecutive
+//      keys, a block-wide scan of the per-thread counts places the keys >= guess in
+//      index order in shared memory (at most cap = max(4096, 2k + 2048); beyond
+//      that they are only counted).  If the count is outside [k, cap], counting
+//      passes bisect the key range for a threshold that fits and the pass repeats;
+//   4. exact k-th key T of the candidates by a radix select over the bits below
+//      their common prefix (8 bits per pass), and how many keys equal to T are
+//      taken (the earliest ones);
 //   5. ordered emission of the candidates > T and the first of those == T.
-// If no guess has a count in [k, kCap] (more than kCap keys tie at the k-th value)
-// the bisection ends with the exact k-th key and step 5 runs over the row itself.
+// If no threshold has a count in [k, cap] (more than cap keys tie at the k-th
+// value) the bisection ends with the exact k-th key and step 5 runs over the row.
 #include "common.cuh"
 #include "launch.h"
 
 namespace tam {
 namespace {
 
-constexpr int kRtThreads = 512;
+constexpr int kRtThreads = 256;
 constexpr int kRtWarps = kRtThreads / 32;
-constexpr int kCap = 8192;     // candidates staged in shared memory
+constexpr int kChunkKeys = 8;  // consecutive keys per thread in one chunk of the row
+
+// Candidates staged in shared memory for budget k.
+__host__ __device__ constexpr int cand_cap(int k) { return 2 * k + 2048 > 4096 ? 2 * k + 2048 : 4096; }
 
 __device__ __forceinline__ uint32_t okey(float v) {
     const uint32_t b = __float_as_uint(v);
@@ -43,19 +52,23 @@ __device__ __forceinline__ float oval(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 __device__ __forceinline__ int64_t tri(int64_t i) { return i * (i + 1) / 2; }
+__device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
 }
 
+// Shared memory of one row: this header, then ckey[cap] and cidx[cap].
 struct RowSmem {
-    uint32_t ckey[kCap];
-    int32_t cidx[kCap];
     int hist[256];
     int wa[kRtWarps];       // per warp segment: count of the first predicate
     int wb[kRtWarps];       // per warp segment: count of keys equal to the threshold
+    int wsc[2][kRtWarps];   // per warp totals of a chunk (double-buffered)
     int scal[4];
+    unsigned int cmax;      // largest candidate key
+    uint32_t* ckey;
+    int32_t* cidx;
 };
 
 // Source of a pass: the row in global memory or the staged candidates.
@@ -74,7 +87,7 @@ struct CandSrc {
 __device__ __forceinline__ int seg_len(int n) { return (((n + kRtWarps - 1) / kRtWarps) + 31) & ~31; }
 
 // Per warp segment: wa = #(key >= T) (GE) or #(key > T) (!GE); wb = #(key == T).
-// Returns the block totals through scal[0] / scal[1].  Contains barriers.
+// Returns the block totals in tot_a / tot_b.  Contains barriers.
 template <class Src, bool GE>
 __device__ void seg_count(const Src& src, int n, uint32_t T, RowSmem& s, int& tot_a, int& tot_b) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -115,11 +128,10 @@ __device__ void seg_count(const Src& src, int n, uint32_t T, RowSmem& s, int& to
     }
 }
 
-// Ordered compaction after seg_count over the same (src, n, T).
-//   GE:  keep key >= T                     -> candidates (ckey / cidx)
-//   !GE: keep key > T, or key == T among the first `quota` such keys -> output row
+// Ordered emission after seg_count<Src, false> over the same (src, n, T): keeps
+// key > T, or key == T among the first `quota` such keys, into the output row.
 // Positions follow source order, so the kept keys stay in ascending index order.
-template <class Src, bool GE>
+template <class Src>
 __device__ void seg_emit(const Src& src, int n, uint32_t T, int quota, RowSmem& s,
                          int32_t* out_idx, float* out_val) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,18 +155,13 @@ __device__ void seg_emit(const Src& src, int n, uint32_t T, int quota, RowSmem& 
         for (int u = 0; u < U; ++u) {
             const int e = base + u * 32 + lane;
             const bool in = e < end;
-            const bool gt = in && (GE ? kv[u] >= T : kv[u] > T);
-            const bool eq = in && !GE && kv[u] == T;
+            const bool gt = in && kv[u] > T;
+            const bool eq = in && kv[u] == T;
             const uint32_t gb = __ballot_sync(0xffffffffu, gt);
             const uint32_t eb = __ballot_sync(0xffffffffu, eq);
             const int g_pre = gt_before + __popc(gb & lt);
             const int e_pre = eq_before + __popc(eb & lt);
-            if (GE) {
-                if (gt) {
-                    s.ckey[g_pre] = kv[u];
-                    s.cidx[g_pre] = src.idx(e);
-                }
-            } else if (gt || (eq && e_pre < quota)) {
+            if (gt || (eq && e_pre < quota)) {
                 const int pos = g_pre + min(e_pre, quota);
                 out_idx[pos] = src.idx(e);
                 out_val[pos] = oval(kv[u]);
@@ -165,19 +172,102 @@ __device__ void seg_emit(const Src& src, int n, uint32_t T, int quota, RowSmem& 
     }
 }
 
-// Exact k-th largest key of the c candidates (k <= c): returns T and how many of
-// the keys equal to T belong to the top k.  Contains barriers.
-__device__ void cand_kth(RowSmem& s, int c, int k, uint32_t& T, int& take_eq) {
+// One pass over the row: the keys >= G, in index order, go to ckey / cidx (at most
+// cap of them; beyond that they are only counted).  Thread t takes the 8
+// consecutive keys at chunk + 8t; a warp scan plus the warp totals of the chunk
+// give every thread its output position.  Returns the count; s.cmax receives the
+// largest key >= G.  Contains barriers.
+__device__ int compact_ge(const RowSrc& row, int n, uint32_t G, RowSmem& s, int cap) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t prefix = 0, mask = 0;
+    constexpr int kStep = kRtThreads * kChunkKeys;
+    int base = 0, buf = 0;
+    uint32_t kmax = 0;
+    // the next chunk's loads are issued before this chunk's scan and barrier
+    float nx[kChunkKeys];
+#pragma unroll
+    for (int u = 0; u < kChunkKeys; ++u) {
+        const int e = threadIdx.x * kChunkKeys + u;
+        nx[u] = e < n ? __ldg(row.row + e) : 0.f;
+    }
+    for (int c0 = 0; c0 < n; c0 += kStep, buf ^= 1) {
+        const int e0 = c0 + threadIdx.x * kChunkKeys;
+        uint32_t kv[kChunkKeys];
+        int cnt = 0;
+#pragma unroll
+        for (int u = 0; u < kChunkKeys; ++u) {
+            kv[u] = okey(nx[u]);
+            cnt += (e0 + u < n && kv[u] >= G) ? 1 : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < kChunkKeys; ++u) {
+            const int e = e0 + kStep + u;
+            nx[u] = e < n ? __ldg(row.row + e) : 0.f;
+        }
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) s.wsc[buf][warp] = incl;
+        __syncthreads();
+        // exclusive prefix of the warp totals (lanes 0..15 hold one warp each)
+        const int wt = lane < kRtWarps ? s.wsc[buf][lane] : 0;
+        int wincl = wt;
+#pragma unroll
+        for (int o = 1; o < kRtWarps; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, wincl, o);
+            if (lane >= o) wincl += y;
+        }
+        const int before = __shfl_sync(0xffffffffu, wincl - wt, warp);
+        const int tot = __shfl_sync(0xffffffffu, wincl, kRtWarps - 1);
+        if (cnt) {
+            int pos = base + before + incl - cnt;
+#pragma unroll
+            for (int u = 0; u < kChunkKeys; ++u) {
+                if (e0 + u < n && kv[u] >= G) {
+                    if (pos < cap) {
+                        s.ckey[pos] = kv[u];
+                        s.cidx[pos] = e0 + u;
+                    }
+                    ++pos;
+                    kmax = max(kmax, kv[u]);
+                }
+            }
+        }
+        base += tot;
+    }
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) atomicMax(&s.cmax, kmax);
+    return base;
+}
+
+// Exact k-th largest key of the c candidates (k <= c), all >= G and <= s.cmax:
+// returns T and how many of the keys equal to T belong to the top k.  The bits
+// above the highest bit where G and cmax differ are common to every candidate, so
+// the radix passes start below them.  Contains barriers.
+__device__ void cand_kth(RowSmem& s, int c, int k, uint32_t G, uint32_t& T, int& take_eq) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t diff = G ^ s.cmax;
+    if (diff == 0u) {           // every candidate equals G
+        T = G;
+        take_eq = k;
+        return;
+    }
+    int hi_bit = 31 - __clz(diff);
+    uint32_t mask = ~(uint32_t)((2ull << hi_bit) - 1ull);
+    uint32_t prefix = G & mask;
     int remaining = k;
 #pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    while (hi_bit >= 0) {
+        const int width = min(8, hi_bit + 1);
+        const int shift = hi_bit + 1 - width;
+        const uint32_t dmask = (1u << width) - 1u;
         for (int b = threadIdx.x; b < 256; b += blockDim.x) s.hist[b] = 0;
         __syncthreads();
         for (int e = threadIdx.x; e < c; e += blockDim.x) {
             const uint32_t kv = s.ckey[e];
-            if ((kv & mask) == prefix) atomicAdd(&s.hist[(kv >> shift) & 255u], 1);
+            if ((kv & mask) == prefix) atomicAdd(&s.hist[(kv >> shift) & dmask], 1);
         }
         __syncthreads();
         if (warp == 0) {
@@ -210,8 +300,9 @@ __device__ void cand_kth(RowSmem& s, int c, int k, uint32_t& T, int& take_eq) {
         }
         __syncthreads();
         prefix |= (uint32_t)s.scal[0] << shift;
-        mask |= 255u << shift;
+        mask |= dmask << shift;
         remaining = s.scal[1];
+        hi_bit = shift - 1;
         __syncthreads();
     }
     T = prefix;
@@ -221,18 +312,18 @@ __device__ void cand_kth(RowSmem& s, int c, int k, uint32_t& T, int& take_eq) {
 struct RowTopkParams {
     const float* slab;
     int64_t row0;
-    int n_rows, budget;
+    int n_rows, budget, cap;
     int32_t* sup_idx;
     int32_t* sup_len;
     float* sup_val;
 };
 
-__global__ void __launch_bounds__(kRtThreads) k_row_topk(const RowTopkParams p) {
+__global__ void __launch_bounds__(kRtThreads, 6) k_row_topk(const RowTopkParams p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     RowSmem& s = *reinterpret_cast<RowSmem*>(smem_raw);
     const int64_t i = p.row0 + (p.n_rows - 1 - (int)blockIdx.x);
     const int n = (int)i + 1;
-    const int k = p.budget;
+    const int k = p.budget, cap = p.cap;
     const RowSrc row{p.slab + (tri(i) - tri(p.row0))};
     int32_t* oi = p.sup_idx + i * (int64_t)k;
     float* ov = p.sup_val + i * (int64_t)k;
@@ -245,29 +336,81 @@ __global__ void __launch_bounds__(kRtThreads) k_row_topk(const RowTopkParams p) 
         if (threadIdx.x == 0) p.sup_len[i] = n;
         return;
     }
+    if (threadIdx.x == 0) {
+        s.ckey = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowSmem));
+        s.cidx = reinterpret_cast<int32_t*>(s.ckey + cap);
+        s.cmax = 0u;
+    }
+    __syncthreads();
 
-    // ---- 1-2: a threshold G with k <= #(key >= G) <= kCap
+    // ---- 1: threshold guess G (rows of at most 2k + 256 keys: G = 0, every key)
+    uint32_t G = 0;
+    if (!(n <= 2 * k + 256 && n <= cap)) {
+        // m samples per thread, evenly spaced over the row, staged in the (still
+        // unused) candidate buffer; warp 0 then finds the r-th largest
+        const int m = min(16, 2 + (n >> 17));
+        const int s_tot = kRtThreads * m;
+        const float step = (float)n / (float)s_tot;
+        for (int u = 0; u < m; ++u) {
+            const int t = threadIdx.x + u * kRtThreads;
+            s.ckey[t] = row.key(min(n - 1, (int)((float)t * step)));
+        }
+        __syncthreads();
+        if (warp_id() == 0) {
+            const float mu = (float)s_tot * (float)k / (float)n;
+            const int r = max(1, min(s_tot, (int)ceilf(mu + 3.f * sqrtf(mu) + 4.f)));
+            const int lane = threadIdx.x & 31;
+            // bits above the highest one where the smallest and largest sample differ
+            // are common to all samples
+            // the first 512 samples sit in registers (16 per lane), the rest are re-read
+            uint32_t v[16];
+            uint32_t mn = 0xffffffffu, mx = 0u;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                v[u] = s.ckey[lane + 32 * u];
+                mn = min(mn, v[u]);
+                mx = max(mx, v[u]);
+            }
+            for (int e = 512 + lane; e < s_tot; e += 32) {
+                mn = min(mn, s.ckey[e]);
+                mx = max(mx, s.ckey[e]);
+            }
+            mn = __reduce_min_sync(0xffffffffu, mn);
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            uint32_t t = mn;
+            if (mn != mx) {
+                const int top = 31 - __clz(mn ^ mx);
+                t = mn & ~(uint32_t)((2ull << top) - 1ull);
+                for (int b = top; b >= 0; --b) {
+                    const uint32_t c = t | (1u << b);
+                    int cl = 0;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) cl += v[u] >= c ? 1 : 0;
+                    for (int e = 512 + lane; e < s_tot; e += 32) cl += s.ckey[e] >= c ? 1 : 0;
+                    if (__reduce_add_sync(0xffffffffu, cl) >= r) t = c;
+                }
+            }
+            if (lane == 0) s.scal[2] = (int)t;
+        }
+        __syncthreads();
+        G = (uint32_t)s.scal[2];
+    }
+    // ---- 2-3: ordered candidates (keys >= G)
+    int cnt = compact_ge(row, n, G, s, cap), dummy;
+    bool found = cnt >= k && cnt <= cap;
     uint64_t lo = 0, hi = 1ull << 32;   // #(key >= lo) >= k;  #(key >= hi) < k
     int c_hi = 0;                       // #(key >= hi)
-    uint32_t G = 0;
-    int cnt = n, dummy;
-    bool found = n <= kCap;             // G = 0 takes the whole row
     if (!found) {
-        // r-th largest of the samples, r so that about 1.25 k + 64 keys are expected >= it
-        const int sidx = (int)(((int64_t)threadIdx.x * n) / kRtThreads);
-        const uint32_t sk = row.key(sidx);
-        const double want = 1.25 * k + 64.0;
-        int r = (int)ceil(want * kRtThreads / n);
-        r = max(1, min(kRtThreads, r));
-        uint32_t t = 0;
-        for (int b = 31; b >= 0; --b) {
-            const uint32_t c = t | (1u << b);
-            if (__syncthreads_count(sk >= c) >= r) t = c;
+        if (cnt < k) {
+            hi = G;
+            c_hi = cnt;
+        } else {
+            lo = G;
         }
-        G = t;
-        for (int probe = 0; probe < 40; ++probe) {
+        while (hi - lo > 1) {
+            G = (uint32_t)((lo + hi) >> 1);
             seg_count<RowSrc, true>(row, n, G, s, cnt, dummy);
-            if (cnt >= k && cnt <= kCap) {
+            if (cnt >= k && cnt <= cap) {
                 found = true;
                 break;
             }
@@ -277,41 +420,40 @@ __global__ void __launch_bounds__(kRtThreads) k_row_topk(const RowTopkParams p) 
             } else {
                 lo = G;
             }
-            if (hi - lo <= 1) break;
-            G = (uint32_t)((lo + hi) >> 1);
+        }
+        if (found) {
+            if (threadIdx.x == 0) s.cmax = 0u;
+            __syncthreads();
+            cnt = compact_ge(row, n, G, s, cap);
         }
     }
     if (found) {
-        // ---- 3: ordered candidates (keys >= G); seg_count above left their warp counts
-        if (G == 0u) seg_count<RowSrc, true>(row, n, 0u, s, cnt, dummy);
-        seg_emit<RowSrc, true>(row, n, G, 0, s, nullptr, nullptr);
         __syncthreads();
         // ---- 4: exact k-th key of the candidates
         uint32_t T;
         int take_eq;
-        cand_kth(s, cnt, k, T, take_eq);
+        cand_kth(s, cnt, k, G, T, take_eq);
         // ---- 5: ordered emission of the top k
         const CandSrc cs{&s};
         seg_count<CandSrc, false>(cs, cnt, T, s, dummy, dummy);
-        seg_emit<CandSrc, false>(cs, cnt, T, take_eq, s, oi, ov);
+        seg_emit<CandSrc>(cs, cnt, T, take_eq, s, oi, ov);
     } else {
-        // more than kCap keys tie at the k-th value: lo is that value, exactly
+        // more than cap keys tie at the k-th value: lo is that value, exactly
         const uint32_t T = (uint32_t)lo;
         seg_count<RowSrc, false>(row, n, T, s, dummy, dummy);
-        seg_emit<RowSrc, false>(row, n, T, k - c_hi, s, oi, ov);
+        seg_emit<RowSrc>(row, n, T, k - c_hi, s, oi, ov);
     }
     if (threadIdx.x == 0) p.sup_len[i] = k;
 }
 
 }  // namespace
 
-size_t row_topk_smem_bytes() { return sizeof(RowSmem); }
-
 cudaError_t row_topk(const float* slab, int64_t row0, int64_t row1, int budget, int32_t* sup_idx,
                      int32_t* sup_len, float* sup_val, cudaStream_t st) {
     if (row1 <= row0) return cudaSuccess;
-    RowTopkParams p{slab, row0, (int)(row1 - row0), budget, sup_idx, sup_len, sup_val};
-    const int smem = (int)sizeof(RowSmem);
+    const int cap = cand_cap(budget);
+    RowTopkParams p{slab, row0, (int)(row1 - row0), budget, cap, sup_idx, sup_len, sup_val};
+    const int smem = (int)sizeof(RowSmem) + cap * 8;
     cudaError_t e = cudaFuncSetAttribute(k_row_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     k_row_topk<<<(unsigned)(row1 - row0), kRtThreads, smem, st>>>(p);
