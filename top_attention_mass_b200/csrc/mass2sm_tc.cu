@@ -240,7 +240,9 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int col = c * 32 + c4 * 4 + e;
-                            acc[col / G] += tc::ex2(fmaf(__uint_as_float(cur[c4 * 4 + e]), p.sl2, -Ls[e]));
+                            // one exponential in four on the FMA pipe, the rest on MUFU
+                            const float x = fmaf(__uint_as_float(cur[c4 * 4 + e]), p.sl2, -Ls[e]);
+                            acc[col / G] += e == 3 ? tc::ex2_fma(x) : tc::ex2(x);
                         }
                     }
                     if (c + 1 < kCols / 32) tc::tmem_wait_ld(nxt);

@@ -365,5 +365,24 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// 2^x on the FMA/ALU pipes, for x <= 0, so that part of a kernel's exponentials
+// leave the MUFU unit.  x = n + f with n = rint(x), obtained by adding 1.5 * 2^23
+// (where the float spacing is 1), and f in [-0.5, 0.5]; 2^f is a degree-4
+// polynomial fitted to 2^f in relative error on Chebyshev nodes (Lawson-weighted
+// least squares; max relative error 2.7e-6 evaluated in fp32 Horner form), and n is
+// added to the exponent field.  x is clamped at -125 so that the field stays
+// positive: inputs below that give about 2^-125 instead of ex2's 0.
+__device__ __forceinline__ float ex2_fma(float x) {
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    const int n = __float_as_int(t) - 0x4B400000;
+    float p = fmaf(0.009570101f, f, 0.055917859f);
+    p = fmaf(p, f, 0.24024744f);
+    p = fmaf(p, f, 0.69312179f);
+    p = fmaf(p, f, 0.99999928f);
+    return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
 }  // namespace tc
 }  // namespace tam
