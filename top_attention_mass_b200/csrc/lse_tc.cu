@@ -163,26 +163,42 @@ k_lse_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             tc::mbar_arrive(&s_empty[b]);
             const int j0 = t * 128;
             const bool diag = (j0 + 127 > q0);
-            float tmax = -INFINITY;
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (j0 + c * 32 + e > i) v[c][e] = __float_as_uint(-INFINITY);
+            }
+            // row max: two independent chains of 3-input max
+            float tm[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    tm[c & 1] = tc::max3(tm[c & 1], __uint_as_float(v[c][e]),
+                                         __uint_as_float(v[c][e + 1]));
+            const float m_new = fmaxf(m, fmaxf(tm[0], tm[1]) * sl2);
+            const float neg = -m_new;
+            // exponentials of column pairs: packed scale-and-shift, packed sums in two chains
+            const uint64_t sl2x2 = tc::f2_pack(sl2, sl2), negx2 = tc::f2_pack(neg, neg);
+            uint64_t sum2[2] = {0ull, 0ull};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float s = __uint_as_float(v[c][e]);
-                    if (diag && j0 + c * 32 + e > i) s = -INFINITY;
-                    v[c][e] = __float_as_uint(s);
-                    tmax = fmaxf(tmax, s);
+                for (int e = 0; e < 32; e += 2) {
+                    const uint64_t x2 = tc::f2_fma(tc::f2_pack(__uint_as_float(v[c][e]),
+                                                               __uint_as_float(v[c][e + 1])),
+                                                   sl2x2, negx2);
+                    float x0, x1;
+                    tc::f2_unpack(x2, x0, x1);
+                    sum2[c & 1] = tc::f2_add(sum2[c & 1], tc::f2_pack(tc::ex2(x0), tc::ex2(x1)));
                 }
             }
-            const float m_new = fmaxf(m, tmax * sl2);
-            const float neg = -m_new;
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) sum += tc::ex2(fmaf(__uint_as_float(v[c][e]), sl2, neg));
-            }
-            l = l * tc::ex2(m - m_new) + sum;
+            float s0, s1, s2, s3;
+            tc::f2_unpack(sum2[0], s0, s1);
+            tc::f2_unpack(sum2[1], s2, s3);
+            l = l * tc::ex2(m - m_new) + ((s0 + s1) + (s2 + s3));
             m = m_new;
         }
         if (ok && i < N && !*abort_flag) lse[(size_t)h * N + i] = (m + __log2f(l)) * kLn2;
