@@ -1,4 +1,4 @@
-"""The FMA-pipe exponential of the pass-2 kernels (csrc/tc_ptx.cuh, ex2_fma) against
+"""The FMA-pipe exponential of the kernels (csrc/tc_ptx.cuh, ex2_fma / ex2_fma2) against
 the mathematics: its coefficients are read from the header and the same steps are
 replayed in float32 (round to nearest integer by adding 1.5 * 2^23, degree-4 Horner
 polynomial in f in [-0.5, 0.5], integer added to the exponent field), then compared
@@ -14,13 +14,12 @@ HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 
 def _coeffs():
     src = open(HDR).read()
-    body = src[src.index("float ex2_fma(float x)"):]
-    body = body[:body.index("}")]
-    nums = [float(m) for m in re.findall(r"(\d+\.\d*)f", body)]
-    # fmaxf(x, -125), the magic constant twice, then c4, c3, c2, c1, c0
-    assert nums[0] == 125.0 and nums[1] == nums[2] == 12582912.0
-    c4, c3, c2, c1, c0 = nums[3:8]
-    return np.float32(c0), np.float32(c1), np.float32(c2), np.float32(c3), np.float32(c4)
+    val = {}
+    for name in ("kEx2C0", "kEx2C1", "kEx2C2", "kEx2C3", "kEx2C4", "kRoundMagic"):
+        m = re.search(name + r"\s*=\s*([0-9.]+)f", src)
+        val[name] = float(m.group(1))
+    assert val["kRoundMagic"] == 12582912.0
+    return tuple(np.float32(val[f"kEx2C{i}"]) for i in range(5))
 
 
 def _ex2_fma(x):

@@ -190,9 +190,16 @@ k_lse_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                     const uint64_t x2 = tc::f2_fma(tc::f2_pack(__uint_as_float(v[c][e]),
                                                                __uint_as_float(v[c][e + 1])),
                                                    sl2x2, negx2);
-                    float x0, x1;
+                    float x0, x1, y0, y1;
                     tc::f2_unpack(x2, x0, x1);
-                    sum2[c & 1] = tc::f2_add(sum2[c & 1], tc::f2_pack(tc::ex2(x0), tc::ex2(x1)));
+                    // one pair in four on the FMA pipe (packed polynomial), the rest on MUFU
+                    if ((e & 7) == 6) {
+                        tc::ex2_fma2(x0, x1, y0, y1);
+                    } else {
+                        y0 = tc::ex2(x0);
+                        y1 = tc::ex2(x1);
+                    }
+                    sum2[c & 1] = tc::f2_add(sum2[c & 1], tc::f2_pack(y0, y1));
                 }
             }
             float s0, s1, s2, s3;

@@ -399,16 +399,37 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // least squares; max relative error 2.7e-6 evaluated in fp32 Horner form), and n is
 // added to the exponent field.  x is clamped at -125 so that the field stays
 // positive: inputs below that give about 2^-125 instead of ex2's 0.
+constexpr float kEx2C0 = 0.99999928f, kEx2C1 = 0.69312179f, kEx2C2 = 0.24024744f,
+                kEx2C3 = 0.055917859f, kEx2C4 = 0.009570101f;
+constexpr float kRoundMagic = 12582912.f;      // 1.5 * 2^23, bits 0x4B400000
+
 __device__ __forceinline__ float ex2_fma(float x) {
     x = fmaxf(x, -125.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
+    const float t = x + kRoundMagic;
+    const float f = x - (t - kRoundMagic);
     const int n = __float_as_int(t) - 0x4B400000;
-    float p = fmaf(0.009570101f, f, 0.055917859f);
-    p = fmaf(p, f, 0.24024744f);
-    p = fmaf(p, f, 0.69312179f);
-    p = fmaf(p, f, 0.99999928f);
+    float p = fmaf(kEx2C4, f, kEx2C3);
+    p = fmaf(p, f, kEx2C2);
+    p = fmaf(p, f, kEx2C1);
+    p = fmaf(p, f, kEx2C0);
     return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// ex2_fma on a pair (x0, x1) with packed adds and FMAs.
+__device__ __forceinline__ void ex2_fma2(float x0, float x1, float& y0, float& y1) {
+    const uint64_t x2 = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t2 = f2_add(x2, f2_pack(kRoundMagic, kRoundMagic));
+    const uint64_t n2 = f2_add(t2, f2_pack(-kRoundMagic, -kRoundMagic));   // rint(x), exact
+    const uint64_t f2 = f2_fma(n2, f2_pack(-1.f, -1.f), x2);                // x - rint(x), exact
+    uint64_t p2 = f2_fma(f2_pack(kEx2C4, kEx2C4), f2, f2_pack(kEx2C3, kEx2C3));
+    p2 = f2_fma(p2, f2, f2_pack(kEx2C2, kEx2C2));
+    p2 = f2_fma(p2, f2, f2_pack(kEx2C1, kEx2C1));
+    p2 = f2_fma(p2, f2, f2_pack(kEx2C0, kEx2C0));
+    float t0, t1, p0, p1;
+    f2_unpack(t2, t0, t1);
+    f2_unpack(p2, p0, p1);
+    y0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
 }
 
 }  // namespace tc
