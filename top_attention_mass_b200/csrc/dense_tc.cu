@@ -201,30 +201,48 @@ k_dense_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             tc::mbar_arrive(&s_empty[b]);
             const int j0 = t * 128;
             const bool diag = (j0 + 127 > q0);
-            float tmax = -INFINITY;
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (j0 + c * 32 + e > i) v[c][e] = __float_as_uint(-INFINITY);
+            }
+            // row max of the raw scores: two chains of 3-input max
+            float tm[2] = {-INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float s = __uint_as_float(v[c][e]) * sl2;
-                    if (diag && j0 + c * 32 + e > i) s = -INFINITY;
-                    v[c][e] = __float_as_uint(s);
-                    tmax = fmaxf(tmax, s);
-                }
+                for (int e = 0; e < 32; e += 2)
+                    tm[c & 1] = tc::max3(tm[c & 1], __uint_as_float(v[c][e]),
+                                         __uint_as_float(v[c][e + 1]));
+            const float tmax = fmaxf(tm[0], tm[1]) * sl2;
             const bool raise = tmax > m_used + kRescaleLog2;
             const float m_new = raise ? tmax : m_used;
             const float corr = tc::ex2(m_used - m_new);     // 0 on the first tile
-            float sum = 0.f;
-            // P in bf16, row r of the swizzled tile (16-byte chunks XOR row%8)
+            const uint64_t sl2x2 = tc::f2_pack(sl2, sl2), negm2 = tc::f2_pack(-m_new, -m_new);
+            uint64_t sum2[2] = {0ull, 0ull};
+            // P in bf16, row r of the swizzled tile (16-byte chunks XOR row%8); column
+            // pairs: packed scale-and-shift and sums, one pair in four on the FMA pipe
 #pragma unroll
             for (int c8 = 0; c8 < 16; ++c8) {
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int col = c8 * 8 + 2 * e;
-                    const float p0 = tc::ex2(__uint_as_float(v[col / 32][col % 32]) - m_new);
-                    const float p1 = tc::ex2(__uint_as_float(v[(col + 1) / 32][(col + 1) % 32]) - m_new);
-                    sum += p0 + p1;
+                    const uint64_t x2 = tc::f2_fma(
+                        tc::f2_pack(__uint_as_float(v[col / 32][col % 32]),
+                                    __uint_as_float(v[(col + 1) / 32][(col + 1) % 32])),
+                        sl2x2, negm2);
+                    float x0, x1, p0, p1;
+                    tc::f2_unpack(x2, x0, x1);
+                    if (e == 3) {
+                        tc::ex2_fma2(x0, x1, p0, p1);
+                    } else {
+                        p0 = tc::ex2(x0);
+                        p1 = tc::ex2(x1);
+                    }
+                    sum2[e & 1] = tc::f2_add(sum2[e & 1], tc::f2_pack(p0, p1));
                     __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<uint32_t*>(&pk);
                 }
@@ -238,7 +256,10 @@ k_dense_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 *dst = make_uint4(w[0], w[1], w[2], w[3]);
             }
             if (!ok) break;
-            l = l * corr + sum;
+            float s0, s1, s2, s3;
+            tc::f2_unpack(sum2[0], s0, s1);
+            tc::f2_unpack(sum2[1], s2, s3);
+            l = l * corr + ((s0 + s1) + (s2 + s3));
             // rescale O in TMEM when this warp's rows raised their max (after P V t-1)
             const bool any_raise = __any_sync(0xffffffffu, raise && t > 0);
             if (any_raise) {
