@@ -366,9 +366,10 @@ def run_reference(args, w, inp, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def config_dict(w, world):
+def config_dict(w, world, launch=None):
     idx_k = INDEXER_K if w.name == WORKLOAD else (w.budget_k if w.d_idx else None)
-    return {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+    extra = {"step_launch": launch} if launch else {}
+    return {**extra, "workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
             "budget_k": w.budget_k, "block_q": list(w.block_q), "indexer_k": idx_k,
             "d_idx": w.d_idx or None, "rope": w.rope_base, "global_batch": world, "seq_len": w.N,
             "parallelism": f"replicas x{world} (independent layers, no collective)",
@@ -394,8 +395,38 @@ def run_ours(args, w, inp, rank, world, local_rank):
     torch.cuda.synchronize()
     work = algorithmic_work(step, w.N)
 
+    # per-row breakdown: eager calls with CUDA events between them (same inputs)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
           for _ in range(args.steps)]
+    for s in range(args.steps):
+        flush.fill_(s & 0xff)
+        step.run(ev[s])
+    torch.cuda.synchronize()
+    tam.check_status(step.ws.get(256))
+    row_ms = {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps))
+              for i, n in enumerate(names)}
+
+    # The step is captured once as a CUDA graph (every library launch of the step,
+    # recorded on the capture stream) and replayed in the timed region, so host-side
+    # enqueue time between the rows does not enter the device time.  --no-graph times
+    # the eager calls instead.
+    graph, per_step_launches = None, 0
+    if not args.no_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            step.run()                      # warm-up on the capture's side stream
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        n0 = tam.kernel_launches()
+        with torch.cuda.graph(graph):
+            step.run()
+        per_step_launches = tam.kernel_launches() - n0
+        graph.replay()
+        torch.cuda.synchronize()
+        tam.check_status(step.ws.get(256))
+
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
     barrier(world, local_rank)
@@ -405,18 +436,21 @@ def run_ours(args, w, inp, rank, world, local_rank):
     t_start.record()
     for s in range(args.steps):
         flush.fill_(s & 0xff)
-        step.run(ev[s])
+        if graph is not None:
+            graph.replay()
+        else:
+            step.run()
     t_stop.record()
     torch.cuda.synchronize()
-    launches = tam.kernel_launches() - launches0
+    launches = (per_step_launches * args.steps if graph is not None
+                else tam.kernel_launches() - launches0)
     barrier(world, local_rank)
     clk = clocks.stop()
     tam.check_status(step.ws.get(256))
     total_ms = t_start.elapsed_time(t_stop)
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_step = total_ms / args.steps
-    row_ms = {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps))
-              for i, n in enumerate(names)}
+
 
     pk, pk_kind = peaks()
     traffic = traffic_table()
@@ -437,7 +471,8 @@ def run_ours(args, w, inp, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; stands in for the pages' 4K-100K long-context evaluations)",
-        "config": config_dict(w, world),
+        "config": config_dict(w, world, "CUDA graph replay of the step's library calls"
+                              if graph is not None else "eager library calls"),
         "roofline": {**rows[dominant]["roofline"], "kernel": dominant},
         "rows": rows,
         "sparse_pass": sparse_pass_summary(w, row_ms),
@@ -578,6 +613,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the eager library calls instead of a CUDA-graph replay of the step")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="gqa32k_2pct (default: every row), gqa4k_needles, longctx_<N>, indexer32k")
     args = ap.parse_args()

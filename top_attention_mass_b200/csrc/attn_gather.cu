@@ -27,6 +27,8 @@ namespace tam {
 namespace {
 
 constexpr int kChunk = 16;    // keys per chunk
+// per-query kernel: warps per CTA (one CTA per SM) and cp.async ring depth per warp
+constexpr int kGatherWarps = 12, kGatherStages = 2;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -265,8 +267,8 @@ __device__ __forceinline__ int count_le(const int32_t* row, int n, int limit) {
 }
 
 // ---------------------------------------------------------------- per query
-template <int D, int G, int STAGES>
-__global__ void __launch_bounds__(256, 1)
+template <int D, int G, int STAGES, int W>
+__global__ void __launch_bounds__(32 * W, 1)
 k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
               const __nv_bfloat16* __restrict__ v, int N, int Hq, int Hkv, float sl2,
               const int32_t* __restrict__ sup_idx, const int32_t* __restrict__ sup_len, int kmax,
@@ -278,7 +280,7 @@ k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     const int warp = threadIdx.x >> 5;
     const uint32_t wbuf = smem_addr(smem) + warp * STAGES * STAGE;
     const int64_t total = (int64_t)N * Hkv;
-    for (int64_t item = (int64_t)blockIdx.x * 8 + warp; item < total; item += (int64_t)gridDim.x * 8) {
+    for (int64_t item = (int64_t)blockIdx.x * W + warp; item < total; item += (int64_t)gridDim.x * W) {
         const int i = (int)(item / Hkv), g = (int)(item % Hkv);
         const int32_t* srow;
         int n;
@@ -408,16 +410,16 @@ k_attn_block(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 
 template <int D, int G>
 cudaError_t launch_gather(const AttnArgs& a, cudaStream_t st) {
-    constexpr int STAGES = 3;
-    constexpr int smem = 8 * STAGES * 2 * kChunk * D * 2;
-    auto kern = k_attn_gather<D, G, STAGES>;
+    constexpr int STAGES = kGatherStages, W = kGatherWarps;
+    constexpr int smem = W * STAGES * 2 * kChunk * D * 2;
+    auto kern = k_attn_gather<D, G, STAGES, W>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int sms = 148;
     int dev;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    kern<<<sms, 256, smem, st>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k,
+    kern<<<sms, 32 * W, smem, st>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k,
                                  (const __nv_bfloat16*)a.v, (int)a.N, a.Hq, a.Hkv, a.sl2,
                                  a.sup_idx, a.sup_len, a.kmax, a.block_q,
                                  (__nv_bfloat16*)a.out, a.lse);
