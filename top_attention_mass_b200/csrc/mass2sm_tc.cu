@@ -15,18 +15,18 @@
 // read from L2 then serves 32 queries instead of 16, and each CTA reads half as many
 // operand bytes per unit of work - the two things that bounded the single-CTA pass.
 //
-// Roles in each CTA (320 threads):
-//   warp 8      TMA producer: this CTA's Q half (once) and its 128 keys of each
+// Roles in each CTA (W = 8 mass warps per query, 16 block-shared; W + 2 warps):
+//   warp W      TMA producer: this CTA's Q half (once) and its 128 keys of each
 //               256-key tile, counted on CTA 0's barriers;
-//   warp 9      CTA 0 only: issues the pair MMAs into a ring of four 128-column TMEM
+//   warp W+1    CTA 0 only: issues the pair MMAs into a ring of four 128-column TMEM
 //               slots and commits to the barriers of both CTAs;
-//   warps 0-7   mass warps: thread = key row (warp w reads TMEM lanes 32 (w % 4) ..),
-//               column half w / 4, i.e. the (query, head) columns of half the pair's
-//               queries; exp2 against the pass-1 LSE, sum over heads -> mass of those
-//               queries for 128 keys.  Two warps per TMEM lane quarter keep two
-//               exp streams per scheduler.  Per query the mass goes to the row slab
-//               (one coalesced 128-byte store per warp and query); block-shared mass
-//               goes to the fixed-point block sums.
+//   warps 0..W-1 mass warps: thread = key row (warp w reads TMEM lanes 32 (w % 4) ..),
+//               column part w / 4 of W / 4 parts, i.e. the (query, head) columns of
+//               that share of the pair's queries; exp2 against the pass-1 LSE, sum
+//               over heads -> mass of those queries for 128 keys.  Several warps per
+//               TMEM lane quarter keep several exp streams per scheduler.  Per query
+//               the mass goes to the row slab (one coalesced 128-byte store per warp
+//               and query); block-shared mass goes to the fixed-point block sums.
 // Every wait is bounded; the pair shakes hands before it frees TMEM and exits so
 // that no remote arrive or MMA of one CTA can land after the other left.
 #include "launch.h"
@@ -37,9 +37,11 @@ namespace tam {
 namespace {
 
 constexpr int kStages = 2;
-constexpr int kMassWarps = 8;
-constexpr int kProducerWarp = kMassWarps, kMmaWarp = kMassWarps + 1;
-constexpr int kThreads = 32 * (kMassWarps + 2);
+// Mass warps: 8 per query (two per TMEM lane quarter), 16 block-shared (four per
+// quarter; measured 5 % faster there, no gain per query).  Then the TMA producer and
+// the MMA issuer.
+__host__ __device__ constexpr int mass_warps(bool block) { return block ? 16 : 8; }
+__host__ __device__ constexpr int pair_threads(bool block) { return 32 * (mass_warps(block) + 2); }
 constexpr int kNQ = 128;                // MMA N: (query, head) columns of the pair
 constexpr int kHalfRows = 64;           // B rows held by each CTA
 constexpr int kR = 512 / kNQ;           // TMEM accumulator slots
@@ -68,9 +70,11 @@ __host__ __device__ __forceinline__ int64_t bmass_row(int64_t b, int block_q) {
 }
 
 template <int G, int D, bool BLOCK>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(BLOCK), 1)
 k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const PairParams p) {
+    constexpr int kMassWarps = mass_warps(BLOCK);
+    constexpr int kProducerWarp = kMassWarps, kMmaWarp = kMassWarps + 1;
     constexpr int BQP = kNQ / G;              // queries of the pair
     constexpr int BQC = kHalfRows / G;        // queries of one column half
     constexpr int NH = D / 64;
@@ -206,17 +210,19 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         }
     } else if (warp < kMassWarps) {
         // ---------------------------------------------------------------- mass warps
-        constexpr int kCols = kNQ / 2;                 // columns of one half
-        const int quarter = warp & 3, half = warp >> 2;
+        constexpr int kParts = kMassWarps / 4;         // warps per TMEM lane quarter
+        constexpr int kCols = kNQ / kParts;            // columns of one part
+        constexpr int kQP = kCols / G;                 // queries of one part
+        const int quarter = warp & 3, part = warp >> 2;
         const int row = quarter * 32 + lane;
-        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * kCols);
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(part * kCols);
         const uint32_t s_empty_leader = tc::map_to_cta(tc::smem_u32(s_empty), 0);
         bool ok = true;
         if (p.dbg & kDebugForceTimeout) ok = tc::wait(never, 0, gd, 9);
         for (int kt = 0; ok && kt < n_kt; ++kt) {
-            float acc[BQC];
+            float acc[kQP];
 #pragma unroll
-            for (int q = 0; q < BQC; ++q) acc[q] = 0.f;
+            for (int q = 0; q < kQP; ++q) acc[q] = 0.f;
             for (int g = 0; g < Hkv; ++g) {
                 const int u = kt * Hkv + g;
                 const int slot = u % kR;
@@ -232,7 +238,7 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     uint32_t (&nxt)[32] = (c & 1) ? va : vb;
                     if (c + 1 < kCols / 32) tc::tmem_ld32(col0 + (c + 1) * 32, nxt);
                     const float4* l4 =
-                        reinterpret_cast<const float4*>(sLse + g * kNQ + half * kCols + c * 32);
+                        reinterpret_cast<const float4*>(sLse + g * kNQ + part * kCols + c * 32);
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4) {
                         const float4 L = l4[c4];
@@ -260,33 +266,33 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 // row i of the slab starts tri(i) - tri(row0) floats in; lanes store
                 // consecutive keys of one query
 #pragma unroll
-                for (int ql = 0; ql < BQC; ++ql) {
-                    const int64_t i = q0 + half * BQC + ql;
+                for (int ql = 0; ql < kQP; ++ql) {
+                    const int64_t i = q0 + part * kQP + ql;
                     if (j <= i && i >= p.row0 && i < p.row1)
                         p.rows[i * (i + 1) / 2 - slab0 + j] = acc[ql] * p.inv_hq;
                 }
             } else {
-                const int qh = q0 + half * BQC;
+                const int qh = q0 + part * kQP;
                 int cur_b = qh / p.block_q;
-                float part = 0.f;
+                float sum = 0.f;
 #pragma unroll
-                for (int q = 0; q < BQC; ++q) {
+                for (int q = 0; q < kQP; ++q) {
                     const int i = qh + q;
                     if (i < p.N) {
                         const int b = i / p.block_q;
                         if (b != cur_b) {
-                            if (part > 0.f)
+                            if (sum > 0.f)
                                 atomicAdd(&p.bmass[bmass_row(cur_b, p.block_q) + j],
-                                          (unsigned long long)__float2ll_rn(part * p.inv_hq * 1099511627776.0f));
-                            part = 0.f;
+                                          (unsigned long long)__float2ll_rn(sum * p.inv_hq * 1099511627776.0f));
+                            sum = 0.f;
                             cur_b = b;
                         }
-                        if (j <= i) part += acc[q];
+                        if (j <= i) sum += acc[q];
                     }
                 }
-                if (part > 0.f)
+                if (sum > 0.f)
                     atomicAdd(&p.bmass[bmass_row(cur_b, p.block_q) + j],
-                              (unsigned long long)__float2ll_rn(part * p.inv_hq * 1099511627776.0f));
+                              (unsigned long long)__float2ll_rn(sum * p.inv_hq * 1099511627776.0f));
             }
         }
     }
@@ -342,7 +348,7 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
         e = cudaMemsetAsync(a.bmass, 0, (size_t)bmass_row(nb, a.block_q) * 8, st);
         if (e != cudaSuccess) return e;
     }
-    kern<<<(unsigned)(2 * p.n_pairs), kThreads, smem, st>>>(tq, tk, p);
+    kern<<<(unsigned)(2 * p.n_pairs), pair_threads(BLOCK), smem, st>>>(tq, tk, p);
     note_launch();
     return cudaGetLastError();
 }
