@@ -55,6 +55,8 @@ def lib():
             L.orc_block_topk.argtypes = [i64, i32, i32, i32, p, p, i32, p, i64, i32, p, p, p]
             L.orc_attn_rows.argtypes = [i64, i32, i32, i32, p, p, p, p, i64, p, p, i64, p, p]
             L.orc_indexer_topk_rows.argtypes = [i64, i32, p, p, p, i64, i32, p, p, p]
+            L.orc_indexer_block_mass.argtypes = [i64, i32, p, p, i32, p, i64, p]
+            L.orc_indexer_block_topk.argtypes = [i64, i32, p, p, i32, p, i64, i32, p, p, p]
             _lib = L
     return _lib
 
@@ -200,6 +202,34 @@ def indexer_topk_rows(q_idx, k_idx, budget: int, rows=None):
     _check(lib().orc_indexer_topk_rows(N, dx, _ptr(qx), _ptr(kx), _ptr(r), len(r), budget,
                                        _ptr(idx), _ptr(ln), _ptr(sc)))
     return idx, ln, sc
+
+
+def _blocks(blocks, N, block_q):
+    return _rows(blocks, -(-N // block_q))
+
+
+def indexer_block_mass(q_idx, k_idx, block_q: int, blocks=None) -> np.ndarray:
+    """Block sums of the per-query softmax of indexer scores: M [nblocks, N] fp64."""
+    qx, kx = _f32(q_idx), _f32(k_idx)
+    N, dx = qx.shape
+    b = _blocks(blocks, N, block_q)
+    M = np.zeros((len(b), N), np.float64)
+    _check(lib().orc_indexer_block_mass(N, dx, _ptr(qx), _ptr(kx), block_q, _ptr(b), len(b),
+                                        _ptr(M)))
+    return M
+
+
+def indexer_block_topk(q_idx, k_idx, block_q: int, budget: int, blocks=None):
+    """Block-shared indexer support: (idx [nb,k] ascending, -1 pad; len [nb]; mass [nb,k])."""
+    qx, kx = _f32(q_idx), _f32(k_idx)
+    N, dx = qx.shape
+    b = _blocks(blocks, N, block_q)
+    idx = np.full((len(b), budget), -1, np.int32)
+    ln = np.zeros(len(b), np.int32)
+    ms = np.zeros((len(b), budget), np.float64)
+    _check(lib().orc_indexer_block_topk(N, dx, _ptr(qx), _ptr(kx), block_q, _ptr(b), len(b),
+                                        budget, _ptr(idx), _ptr(ln), _ptr(ms)))
+    return idx, ln, ms
 
 
 def block_rows_support(block_idx, block_len, block_q: int, N: int, blocks=None):

@@ -17,7 +17,8 @@
 //     a selection block of consecutive queries (b_sel = 64); attention is then
 //     recomputed on the selected support with the original Q, K, V.
 //   * same report, section 2.2 "Head-Collapsed Indexer": one shared token
-//     score across heads, top-k of it, sparse GQA recompute on that support.
+//     score across heads, top-k of it, sparse GQA recompute on that support;
+//     Abstract and section 3.2: the fused, selection-block-shared indexer path.
 //
 // Readings where the pages are silent (each listed in the design notes):
 //   * query head h reads KV head g(h) = floor(h / (Hq/Hkv)) (consecutive grouping);
@@ -27,7 +28,9 @@
 //   * a block's mass is the sum of P_i over its causally valid queries; query i of a
 //     block attends over S_b intersected with [0, i];
 //   * the recompute renormalises the softmax over the support;
-//   * the indexer score is the plain dot product q_idx . k_idx.
+//   * the indexer score is the plain dot product q_idx . k_idx;
+//   * block-shared indexer: each query's scores turned into softmax_{j <= i} (no
+//     scale, the indexer being trained toward a distribution), summed over the block.
 //
 // Every input arrives as fp32 (bf16 and fp32 inputs are exactly representable)
 // and is widened to double before any arithmetic.  All arithmetic is double.
@@ -329,6 +332,60 @@ int orc_indexer_topk_rows(int64_t N, int d_idx, const float* qx, const float* kx
             len[r] = n;
             for (int t = 0; t < budget; ++t) score[r * budget + t] = (t < n) ? s[ir[t]] : 0.0;
         }
+    }
+    return 0;
+}
+
+// Block-shared indexer support ("fused selection-block-shared support", Abstract;
+// technical report section 3.2, per-query vs fused path): the indexer's scores define
+// one distribution per query, q_i[j] = softmax_{j <= i}(q_idx_i . k_idx_j) (no scale),
+// and a block of consecutive queries shares the top-k of their sum, exactly as the
+// block-shared oracle does with the head-averaged mass:
+//   M_b[j] = sum_{i in block b, i >= j} q_i[j],  S_b = top-min(k, e_b+1) of M_b.
+// M[r*N + j] for the listed blocks (0 beyond e_b).
+int orc_indexer_block_mass(int64_t N, int d_idx, const float* qx, const float* kx, int block_q,
+                           const int64_t* blocks, int64_t nblocks, double* M) {
+    if (N <= 0 || d_idx <= 0 || block_q < 1) return 1;
+#pragma omp parallel
+    {
+        std::vector<double> s(N);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nblocks; ++r) {
+            const int64_t b0 = blocks[r] * block_q;
+            const int64_t e = std::min<int64_t>(N, b0 + block_q) - 1;
+            double* Mr = M + r * N;
+            std::fill(Mr, Mr + N, 0.0);
+            for (int64_t i = b0; i <= e; ++i) {
+                const float* qi = qx + i * d_idx;
+                for (int64_t j = 0; j <= i; ++j) {
+                    const float* kj = kx + j * d_idx;
+                    double acc = 0.0;
+                    for (int c = 0; c < d_idx; ++c) acc += (double)qi[c] * (double)kj[c];
+                    s[j] = acc;
+                }
+                const double lse = log_sum_exp(s.data(), i + 1);
+                for (int64_t j = 0; j <= i; ++j) Mr[j] += std::exp(s[j] - lse);
+            }
+        }
+    }
+    return 0;
+}
+
+// S_b for the listed blocks; layout as orc_block_topk (mass[r*k + t] = M_b[idx]).
+int orc_indexer_block_topk(int64_t N, int d_idx, const float* qx, const float* kx, int block_q,
+                           const int64_t* blocks, int64_t nblocks, int budget, int32_t* idx,
+                           int32_t* len, double* mass) {
+    if (budget < 1) return 1;
+    std::vector<double> M((size_t)nblocks * N);
+    int rc = orc_indexer_block_mass(N, d_idx, qx, kx, block_q, blocks, nblocks, M.data());
+    if (rc) return rc;
+    for (int64_t r = 0; r < nblocks; ++r) {
+        const int64_t e = std::min<int64_t>(N, (blocks[r] + 1) * block_q) - 1;
+        int32_t* ir = idx + r * budget;
+        std::fill(ir, ir + budget, -1);
+        const int n = select_top(M.data() + r * N, e + 1, budget, ir);
+        len[r] = n;
+        for (int t = 0; t < budget; ++t) mass[r * budget + t] = (t < n) ? M[r * N + ir[t]] : 0.0;
     }
     return 0;
 }

@@ -264,3 +264,55 @@ def test_sparsity_endpoints_printed_in_report(oracle_mod):
     for kb in (1, 17, 256, 400):
         _, ln, _ = oracle_mod.topk_rows(q, k, kb)
         assert np.array_equal(ln, np.minimum(kb, np.arange(300) + 1))
+
+
+# ------------------------------------------------------------------ block-shared indexer
+def test_indexer_block_brute_force(oracle_mod):
+    """Block sums of the per-query softmax of indexer scores, written out directly: exp of
+    each score over the sum of exps (no log-sum-exp helper), summed over the block's
+    queries with j <= i; selection by counting ranks."""
+    N, dx, bq, kb = 37, 5, 8, 6
+    g = torch.Generator().manual_seed(21)
+    qx = torch.randn(N, dx, generator=g)
+    kx = torch.randn(N, dx, generator=g)
+    qd, kd = qx.double().tolist(), kx.double().tolist()
+    nb = -(-N // bq)
+    M = np.zeros((nb, N))
+    for b in range(nb):
+        for i in range(b * bq, min(N, (b + 1) * bq)):
+            e = [math.exp(sum(qd[i][c] * kd[j][c] for c in range(dx))) for j in range(i + 1)]
+            z = sum(e)
+            for j in range(i + 1):
+                M[b, j] += e[j] / z
+    np.testing.assert_allclose(oracle_mod.indexer_block_mass(qx, kx, bq), M, rtol=0, atol=1e-12)
+    idx, ln, ms = oracle_mod.indexer_block_topk(qx, kx, bq, kb)
+    for b in range(nb):
+        last = min(N, (b + 1) * bq) - 1
+        sel = _py_select(list(M[b, :last + 1]), last + 1, kb)
+        assert list(idx[b, :ln[b]]) == sel
+        np.testing.assert_allclose(ms[b, :ln[b]], M[b, sel], rtol=0, atol=1e-12)
+
+
+def test_indexer_block_invariants(oracle_mod):
+    N, dx = 300, 16
+    g = torch.Generator().manual_seed(22)
+    qx = torch.randn(N, dx, generator=g) * 0.5
+    kx = torch.randn(N, dx, generator=g) * 0.5
+    # every query's softmax sums to one: a block's mass sums to its number of queries
+    for bq in (1, 7, 64):
+        M = oracle_mod.indexer_block_mass(qx, kx, bq)
+        sizes = [min(N, (b + 1) * bq) - b * bq for b in range(M.shape[0])]
+        np.testing.assert_allclose(M.sum(axis=1), sizes, rtol=1e-12)
+    # a block of one query: softmax is monotone in the score, so the support is the
+    # per-query indexer support and the values are the softmax probabilities
+    idx1, ln1, _ = oracle_mod.indexer_block_topk(qx, kx, 1, 20)
+    idx0, ln0, sc0 = oracle_mod.indexer_topk_rows(qx, kx, 20)
+    assert np.array_equal(idx1, idx0) and np.array_equal(ln1, ln0)
+    # q_idx = 0: every row is uniform, M_b[j] = sum_{i in b, i >= j} 1/(i+1) falls with j,
+    # so the support is the first min(k, e_b+1) keys
+    idx, ln, ms = oracle_mod.indexer_block_topk(torch.zeros(N, dx), kx, 64, 10)
+    for b in range(len(ln)):
+        last = min(N, (b + 1) * 64) - 1
+        assert list(idx[b, :ln[b]]) == list(range(min(10, last + 1)))
+        want = [sum(1.0 / (i + 1) for i in range(max(j, b * 64), last + 1)) for j in range(ln[b])]
+        np.testing.assert_allclose(ms[b, :ln[b]], want, rtol=1e-12)
