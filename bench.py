@@ -406,6 +406,8 @@ def run_ours(args, w, inp, rank, world, local_rank):
     row_ms = {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps))
               for i, n in enumerate(names)}
 
+    next_rows = measure_next_rows(args, tam, w, step, flush) if w.name == WORKLOAD else None
+
     # The step is captured once as a CUDA graph (every library launch of the step,
     # recorded on the capture stream) and replayed in the timed region, so host-side
     # enqueue time between the rows does not enter the device time.  --no-graph times
@@ -483,6 +485,7 @@ def run_ours(args, w, inp, rank, world, local_rank):
             "N102400_k2048": 1.0 - support_pairs(102400, 2048) / causal_pairs(102400),
         },
         "clocks": clk,
+        "next_rows": next_rows,
         "e2e": e2e,
         "gpu_launches": launches,
     }
@@ -493,6 +496,33 @@ def run_ours(args, w, inp, rank, world, local_rank):
         line["cpu_baseline"] = {"value": w.N / t, "unit": UNIT, "cores": oracle.threads(),
                                 "kind": "oracle", "sample": cpu_sample_desc(n_rows)}
     print(json.dumps(line), flush=True)
+
+
+def measure_next_rows(args, tam, w, step, flush):
+    """Rows beyond the step (reported, not part of `value`): the fused, selection-block-
+    shared indexer (block sums of each query's softmax of its indexer scores, top-k per
+    block of BLOCK_Q queries) and pass 3 on that support."""
+    bq, kx = BLOCK_Q, INDEXER_K
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for s in range(args.steps):
+        flush.fill_(s & 0xff)
+        ev[s][0].record()
+        sup = tam.indexer_topk(step.qx, step.kx, kx, bq, workspace=step.ws, check=False)
+        ev[s][1].record()
+        tam.sparse_support_attention(step.q, step.k, step.v, sup.idx, sup.length, bq,
+                                     workspace=step.ws, check=False)
+        ev[s][2].record()
+    torch.cuda.synchronize()
+    tam.check_status(step.ws.get(256))
+    t_sel = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    t_att = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    n_sel = sup.length.cpu().numpy().astype(np.int64)
+    return {
+        "indexer_block_topk": {"ms": t_sel, "q_tok_s": w.N / (t_sel * 1e-3), "budget_k": kx,
+                               "block_q": bq},
+        "pass3_indexer_block": {"ms": t_att, "q_tok_s": w.N / (t_att * 1e-3),
+                                "gathered_rows": int(n_sel.sum()) * w.Hkv},
+    }
 
 
 def measure_e2e(args, tam, w, inp, dev, world, local_rank):

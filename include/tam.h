@@ -161,12 +161,17 @@ int tam_mass_select_noalloc(int64_t N, int Hq, int Hkv, int d, int dtype, const 
  * Head-collapsed indexer support (technical report §2.2 "Head-Collapsed Indexer":
  * one token score shared by all heads, top-k of it):
  *   score[i,j] = q_idx[i] . k_idx[j] for j <= i (no scale: ranking only),
- *   S_i = top-min(k, i+1) of score_i with the same ranking and output layout as above,
- *   sup_score holds the scores of the chosen keys.
- * q_idx, k_idx: [N, d_idx] in `dtype` (bf16 or fp32), d_idx in {16, 32, 64, 128}.
- * block_q must be 1 (per-query support).
- * On the tensor cores the score rows of a chunk of queries are written to the
- * workspace and selected from; tam_indexer_workspace() is the preferred size (every
+ *   block_q == 1: S_i = top-min(k, i+1) of score_i with the same ranking and output
+ *                 layout as above; sup_score holds the scores of the chosen keys.
+ *   block_q  > 1: the fused, selection-block-shared path (Abstract; technical report
+ *                 §3.2): q_i = softmax_{j <= i}(score_i) per query (scale 1),
+ *                 M_b[j] = sum_{i in block b, i >= j} q_i[j], S_b = top-min(k, e_b+1) of
+ *                 M_b; rows [n_sel = ceil(N / block_q), k], sup_score holds M_b of the
+ *                 chosen keys.  Pass 3 on it: tam_sparse_support_attention(block_q).
+ * q_idx, k_idx: [N, d_idx] in `dtype` (bf16 or fp32), d_idx in {16, 32, 64, 128}
+ * (block_q > 1: d_idx in {64, 128}).
+ * On the tensor cores the per-query score rows of a chunk of queries are written to
+ * the workspace and selected from; tam_indexer_workspace() is the preferred size (every
  * row at once, up to 4 GiB), tam_indexer_workspace_min() the smallest accepted.
  */
 size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int block_q);

@@ -88,8 +88,10 @@ def test_host_side_argument_errors(tam_lib):
     # workspace too small
     assert L.tam_mass_oracle_prefill(64, 4, 1, 64, 0, f, f, f, 8, 1, f, f, f, None, None, f, 16,
                                      None) == T.TAM_ERR_WORKSPACE
-    assert L.tam_indexer_topk(64, 64, 0, f, f, 8, 2, f, f, f, f, 1 << 30,
-                              None) == T.TAM_ERR_UNSUPPORTED          # block-shared indexer
+    assert L.tam_indexer_topk(64, 32, 0, f, f, 8, 2, f, f, f, f, 1 << 30,
+                              None) == T.TAM_ERR_UNSUPPORTED          # block-shared: d_idx 64/128
+    assert L.tam_indexer_topk(64, 64, 0, f, f, 8, 2, f, f, f, f, 16,
+                              None) == T.TAM_ERR_WORKSPACE            # block-shared indexer
     assert L.tam_indexer_topk(64, 40, 0, f, f, 8, 1, f, f, f, f, 1 << 30,
                               None) == T.TAM_ERR_UNSUPPORTED
     assert L.tam_sparse_support_attention(64, 4, 1, 64, 0, f, f, f, None, f, 8, 1, f, None, f,

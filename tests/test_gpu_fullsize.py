@@ -65,3 +65,25 @@ def test_stress_row_32k(tam_lib, oracle_mod):
     ref, rl = oracle_mod.attn_rows(inp.q, inp.k, inp.v, rows, sup=idx[rows], sup_len=ln[rows])
     check_close(out.float().cpu().numpy()[rows], ref, OUT_ATOL["bf16"], "stress output")
     check_close(lse.cpu().numpy().T[rows], rl, LSE_ATOL, "stress lse")
+
+
+def test_indexer32k_block_shared_full(tam_lib, oracle_mod):
+    """The fused, selection-block-shared indexer at the 32K shape (k = 1024, B_q = 64),
+    checked on sampled blocks, with pass 3 on a few of their rows."""
+    w = tam_synth.WORKLOADS["indexer32k"]
+    inp = tam_synth.make_inputs(w)
+    bq = 64
+    res = tam_lib.indexer_topk(inp.q_idx.cuda(), inp.k_idx.cuda(), w.budget_k, bq)
+    out = tam_lib.sparse_support_attention(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), res.idx,
+                                           res.length, bq)
+    torch.cuda.synchronize()
+    nb = -(-w.N // bq)
+    blocks = tam_synth.sample_blocks(nb, 4)
+    gi, gl, gm = res.idx.cpu().numpy(), res.length.cpu().numpy(), res.value.cpu().numpy()
+    oi, ol, _ = oracle_mod.indexer_block_topk(inp.q_idx, inp.k_idx, bq, w.budget_k, blocks)
+    M = oracle_mod.indexer_block_mass(inp.q_idx, inp.k_idx, bq, blocks)
+    check_support(gi[blocks], gl[blocks], gm[blocks], oi, ol, M, MASS_ATOL * bq, "indexer block 32k")
+    r, s, sl = oracle_mod.block_rows_support(gi[blocks], gl[blocks], bq, w.N, blocks)
+    pick = np.linspace(0, len(r) - 1, 32).astype(int)
+    ref, _ = oracle_mod.attn_rows(inp.q, inp.k, inp.v, r[pick], sup=s[pick], sup_len=sl[pick])
+    check_close(out.float().cpu().numpy()[r[pick]], ref, OUT_ATOL["bf16"], "indexer block output")

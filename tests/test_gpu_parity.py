@@ -197,6 +197,42 @@ def test_indexer_workload_rows(tam_lib, oracle_mod):
                   res.value.cpu().numpy()[rows], oi, ol, S, 1e-3, "indexer32k")
 
 
+@pytest.mark.parametrize("N,dx,kb,bq,dtype", [(300, 64, 32, 64, "bf16"), (1000, 64, 128, 64, "bf16"),
+                                               (777, 128, 100, 128, "bf16"), (450, 64, 40, 16, "f32"),
+                                               (129, 64, 200, 64, "bf16")])
+def test_indexer_block_shared(tam_lib, oracle_mod, N, dx, kb, bq, dtype):
+    """The fused, selection-block-shared indexer: block sums of each query's softmax of
+    its indexer scores, top-k per block; then pass 3 on that support."""
+    inp = _inputs(N, 8, 2, 128, dtype, seed=13 + N, sink=True, needles=3)
+    qx, kx = tam_synth.indexer_projections(inp, dx, seed=2)
+    if dtype == "f32":
+        qx, kx = qx.float(), kx.float()
+    # (the projections give scores with a standard deviation of about 4: a peaked but
+    # not one-hot softmax over the prefix)
+    res = tam_lib.indexer_topk(qx.cuda(), kx.cuda(), kb, bq)
+    gi, gl, gm = res.idx.cpu().numpy(), res.length.cpu().numpy(), res.value.cpu().numpy()
+    oi, ol, _ = oracle_mod.indexer_block_topk(qx, kx, bq, kb)
+    M = oracle_mod.indexer_block_mass(qx, kx, bq)
+    check_support(gi, gl, gm, oi, ol, M, MASS_ATOL * bq, "indexer block")
+    out = tam_lib.sparse_support_attention(*_cuda(inp.q, inp.k, inp.v), res.idx, res.length, bq)
+    r, sup, sl = oracle_mod.block_rows_support(gi, gl, bq, N)
+    ref, _ = oracle_mod.attn_rows(inp.q, inp.k, inp.v, r, sup=sup, sup_len=sl)
+    check_close(out.float().cpu().numpy()[r], ref, OUT_ATOL[dtype], "indexer block output")
+
+
+def test_indexer_block_shared_ties(tam_lib):
+    """q_idx = 0: every query's softmax is uniform, so a block's sums fall with the key
+    index and the support is the first keys."""
+    N, kb, bq = 700, 30, 64
+    inp = _inputs(N, 8, 2, 128, "bf16", seed=3)
+    qx, kx = tam_synth.indexer_projections(inp, 64, seed=2)
+    res = tam_lib.indexer_topk(torch.zeros_like(qx).cuda(), kx.cuda(), kb, bq)
+    gi, gl = res.idx.cpu().numpy(), res.length.cpu().numpy()
+    for b in range(len(gl)):
+        n = min(kb, min(N, (b + 1) * bq))
+        assert gl[b] == n and list(gi[b, :n]) == list(range(n)), b
+
+
 def test_run_twice_bitwise_identical(tam_lib):
     inp = _inputs(700, 32, 8, 128, "bf16", seed=13, sink=True)
     q, k, v = _cuda(inp.q, inp.k, inp.v)

@@ -321,7 +321,9 @@ def mass_select(q, k, lse, budget_k: int, block_q: int = 1, *,
 def indexer_topk(q_idx, k_idx, budget_k: int, block_q: int = 1, *,
                  workspace: Optional[Workspace] = None, stream=None, check: bool = True,
                  device=None, workspace_bytes: Optional[int] = None) -> Support:
-    """Head-collapsed indexer support: top-k of q_idx . k_idx per query.
+    """Head-collapsed indexer support: top-k of q_idx . k_idx per query (block_q = 1), or
+    per block of block_q queries the top-k of the block's summed per-query softmax of
+    those scores (block_q > 1; values are the block sums).
 
     workspace_bytes: at least tam_indexer_workspace_min (more chunks below the
     preferred size)."""
@@ -331,9 +333,10 @@ def indexer_topk(q_idx, k_idx, budget_k: int, block_q: int = 1, *,
     if k_idx.shape != q_idx.shape or k_idx.dtype != q_idx.dtype:
         raise ValueError("q_idx and k_idx must both be [N, d_idx] of one dtype")
     dt = _dtype_code(q_idx)
-    sup_idx = torch.empty(N, budget_k, dtype=torch.int32, device=dev)
-    sup_len = torch.empty(N, dtype=torch.int32, device=dev)
-    sup_score = torch.empty(N, budget_k, dtype=torch.float32, device=dev)
+    n_sel = N if block_q == 1 else -(-N // block_q)
+    sup_idx = torch.empty(n_sel, budget_k, dtype=torch.int32, device=dev)
+    sup_len = torch.empty(n_sel, dtype=torch.int32, device=dev)
+    sup_score = torch.empty(n_sel, budget_k, dtype=torch.float32, device=dev)
     L = lib()
     nbytes = L.tam_indexer_workspace(N, dx, dt, budget_k, block_q)
     if workspace_bytes is not None and nbytes:

@@ -158,9 +158,9 @@ int start_call(void* workspace, cudaStream_t st) {
 int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
                        const float* lse, int budget_k, int block_q, int32_t* sup_idx,
                        int32_t* sup_len, float* sup_mass, char* ws, size_t ws_bytes,
-                       const MassPlan& plan, cudaStream_t st) {
+                       const MassPlan& plan, cudaStream_t st, float sl2) {
     MassArgs ma = mass_shape(N, Hq, Hkv, d, dtype, budget_k, block_q);
-    ma.q = q; ma.k = k; ma.lse = lse; ma.sl2 = score_log2_scale(d);
+    ma.q = q; ma.k = k; ma.lse = lse; ma.sl2 = sl2;
     ma.n_sel = (int)n_selection_units(N, block_q);
     ma.n_ctas = plan.n_ctas;
     ma.scratch = (float*)(ws + plan.off_work);
@@ -238,7 +238,7 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
     if ((rc = cuda_status(run_lse(la, st)))) return rc;
 
     if ((rc = launch_mass_select(N, Hq, Hkv, d, dtype, q, k, lse_buf, budget_k, block_q, sup_idx,
-                                 sup_len, sup_mass, ws, ws_bytes, plan, st)))
+                                 sup_len, sup_mass, ws, ws_bytes, plan, st, sl2)))
         return rc;
 
     if (out) {
@@ -299,18 +299,24 @@ int tam_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
     cudaStream_t st = (cudaStream_t)stream;
     if ((rc = start_call(workspace, st))) return rc;
     return launch_mass_select(N, Hq, Hkv, d, dtype, q, k, lse, budget_k, block_q, sup_idx, sup_len,
-                              sup_mass, (char*)workspace, ws_bytes, plan, st);
+                              sup_mass, (char*)workspace, ws_bytes, plan, st, score_log2_scale(d));
 }
 
 size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
     if (N < 1 || (d_idx != 16 && d_idx != 32 && d_idx != 64 && d_idx != 128)) return 0;
     if (dtype != TAM_BF16 && dtype != TAM_F32) return 0;
-    if (check_budget(N, budget_k, block_q) != TAM_OK || block_q != 1) return 0;
+    if (check_budget(N, budget_k, block_q) != TAM_OK) return 0;
+    if (block_q > 1) {
+        // block-shared: the indexer head as a one-head layer (lse, block mass)
+        if (check_shape(N, 1, 1, d_idx, dtype) != TAM_OK) return 0;
+        return plan_mass(N, 1, 1, d_idx, dtype, budget_k, block_q).total;
+    }
     return plan_indexer(N, d_idx, dtype, budget_k, block_q).total;
 }
 
 size_t tam_indexer_workspace_min(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
     if (tam_indexer_workspace(N, d_idx, dtype, budget_k, block_q) == 0) return 0;
+    if (block_q > 1) return plan_mass(N, 1, 1, d_idx, dtype, budget_k, block_q).min_total;
     return plan_indexer(N, d_idx, dtype, budget_k, block_q).min_total;
 }
 
@@ -322,12 +328,27 @@ int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const v
     if (N >= (int64_t(1) << 31) - 1) return TAM_ERR_UNSUPPORTED;
     int rc = check_budget(N, budget_k, block_q);
     if (rc) return rc;
-    if (block_q != 1) return TAM_ERR_UNSUPPORTED;
     if (!q_idx || !k_idx || !sup_idx || !sup_len || !sup_score || !workspace)
         return TAM_ERR_INVALID_ARG;
     const void* ptrs[] = {q_idx, k_idx, sup_idx, sup_len, sup_score, workspace};
     for (const void* p : ptrs)
         if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
+    if (block_q > 1) {
+        // Block-shared: softmax of the indexer scores per query (scale 1), summed over
+        // the block, top-k of the sums: pass 1 and the block-mass pass 2 of a one-head
+        // layer whose query and key are q_idx and k_idx.
+        if ((rc = check_shape(N, 1, 1, d_idx, dtype))) return rc;
+        const MassPlan plan = plan_mass(N, 1, 1, d_idx, dtype, budget_k, block_q);
+        if (ws_bytes < plan.min_total) return TAM_ERR_WORKSPACE;
+        cudaStream_t st = (cudaStream_t)stream;
+        char* ws = (char*)workspace;
+        if ((rc = start_call(workspace, st))) return rc;
+        float* lse_buf = (float*)(ws + plan.off_lse);
+        LseArgs la{N, 1, 1, d_idx, dtype, q_idx, k_idx, kLog2e, lse_buf, (int32_t*)ws};
+        if ((rc = cuda_status(run_lse(la, st)))) return rc;
+        return launch_mass_select(N, 1, 1, d_idx, dtype, q_idx, k_idx, lse_buf, budget_k, block_q,
+                                  sup_idx, sup_len, sup_score, ws, ws_bytes, plan, st, kLog2e);
+    }
     const IndexerPlan plan = plan_indexer(N, d_idx, dtype, budget_k, block_q);
     if (ws_bytes < plan.min_total) return TAM_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
