@@ -57,6 +57,7 @@ def lib():
             L.orc_indexer_topk_rows.argtypes = [i64, i32, p, p, p, i64, i32, p, p, p]
             L.orc_indexer_block_mass.argtypes = [i64, i32, p, p, i32, p, i64, p]
             L.orc_indexer_block_topk.argtypes = [i64, i32, p, p, i32, p, i64, i32, p, p, p]
+            L.orc_distill_kl_rows.argtypes = [i64, i32, i32, i32, p, p, i32, p, p, p, i64, p]
             _lib = L
     return _lib
 
@@ -230,6 +231,19 @@ def indexer_block_topk(q_idx, k_idx, block_q: int, budget: int, blocks=None):
     _check(lib().orc_indexer_block_topk(N, dx, _ptr(qx), _ptr(kx), block_q, _ptr(b), len(b),
                                         budget, _ptr(idx), _ptr(ln), _ptr(ms)))
     return idx, ln, ms
+
+
+def distill_kl_rows(q, k, q_idx, k_idx, rows=None) -> np.ndarray:
+    """KL(P_i || softmax(q_idx_i . k_idx)) per listed row (fp64)."""
+    q, k = _f32(q), _f32(k)
+    N, Hq, d = q.shape
+    Hkv = k.shape[1]
+    qx, kx = _f32(q_idx), _f32(k_idx)
+    r = _rows(rows, N)
+    kl = np.zeros(len(r), np.float64)
+    _check(lib().orc_distill_kl_rows(N, Hq, Hkv, d, _ptr(q), _ptr(k), qx.shape[1], _ptr(qx),
+                                     _ptr(kx), _ptr(r), len(r), _ptr(kl)))
+    return kl
 
 
 def block_rows_support(block_idx, block_len, block_q: int, N: int, blocks=None):

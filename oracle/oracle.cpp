@@ -18,7 +18,8 @@
 //     recomputed on the selected support with the original Q, K, V.
 //   * same report, section 2.2 "Head-Collapsed Indexer": one shared token
 //     score across heads, top-k of it, sparse GQA recompute on that support;
-//     Abstract and section 3.2: the fused, selection-block-shared indexer path.
+//     Abstract and section 3.2: the fused, selection-block-shared indexer path;
+//     section 2.2 "Trainingsziel": the indexer's KL-distillation target.
 //
 // Readings where the pages are silent (each listed in the design notes):
 //   * query head h reads KV head g(h) = floor(h / (Hq/Hkv)) (consecutive grouping);
@@ -386,6 +387,39 @@ int orc_indexer_block_topk(int64_t N, int d_idx, const float* qx, const float* k
         const int n = select_top(M.data() + r * N, e + 1, budget, ir);
         len[r] = n;
         for (int t = 0; t < budget; ++t) mass[r * budget + t] = (t < n) ? M[r * N + ir[t]] : 0.0;
+    }
+    return 0;
+}
+
+// Distillation target of the indexer (technical report section 2.2, "Trainingsziel":
+// the indexer is trained by KL divergence from the dense attention-mass distribution):
+//   KL_i = sum_{j <= i} P_i[j] * log(P_i[j] / q_i[j]),
+//   q_i[j] = softmax_{j <= i}(q_idx_i . k_idx_j)   (scale 1, as for the fused indexer),
+// with 0 * log 0 = 0.  kl[r] for the listed rows.
+int orc_distill_kl_rows(int64_t N, int Hq, int Hkv, int d, const float* q, const float* k,
+                        int d_idx, const float* qx, const float* kx, const int64_t* rows,
+                        int64_t nrows, double* kl) {
+    if (!shape_ok(N, Hq, Hkv, d) || d_idx <= 0) return 1;
+#pragma omp parallel
+    {
+        std::vector<double> s(N), P(N), t(N);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nrows; ++r) {
+            const int64_t i = rows[r];
+            mass_row(q, k, Hq, Hkv, d, i, P.data(), s.data());
+            const float* qi = qx + i * d_idx;
+            for (int64_t j = 0; j <= i; ++j) {
+                const float* kj = kx + j * d_idx;
+                double acc = 0.0;
+                for (int c = 0; c < d_idx; ++c) acc += (double)qi[c] * (double)kj[c];
+                t[j] = acc;
+            }
+            const double lse = log_sum_exp(t.data(), i + 1);
+            double sum = 0.0;
+            for (int64_t j = 0; j <= i; ++j)
+                if (P[j] > 0.0) sum += P[j] * (std::log(P[j]) - (t[j] - lse));
+            kl[r] = sum;
+        }
     }
     return 0;
 }

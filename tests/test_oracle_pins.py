@@ -316,3 +316,29 @@ def test_indexer_block_invariants(oracle_mod):
         assert list(idx[b, :ln[b]]) == list(range(min(10, last + 1)))
         want = [sum(1.0 / (i + 1) for i in range(max(j, b * 64), last + 1)) for j in range(ln[b])]
         np.testing.assert_allclose(ms[b, :ln[b]], want, rtol=1e-12)
+
+
+# ------------------------------------------------------------------ distillation target
+def test_distill_kl_brute_force_and_zero(oracle_mod):
+    """KL(P_i || softmax(indexer scores)) written out directly on a tiny input; it is
+    zero when the indexer reproduces a one-head layer's own distribution, and positive
+    otherwise."""
+    N, Hq, Hkv, d, dx = 21, 4, 2, 8, 5
+    q, k, _ = _rand(N, Hq, Hkv, d, seed=31)
+    g = torch.Generator().manual_seed(32)
+    qx, kx = torch.randn(N, dx, generator=g), torch.randn(N, dx, generator=g)
+    P = _py_mass(q.double().tolist(), k.double().tolist(), N, Hq, Hkv, d)
+    qd, kd = qx.double().tolist(), kx.double().tolist()
+    want = []
+    for i in range(N):
+        e = [math.exp(sum(qd[i][c] * kd[j][c] for c in range(dx))) for j in range(i + 1)]
+        z = sum(e)
+        want.append(sum(P[i][j] * math.log(P[i][j] / (e[j] / z)) for j in range(i + 1)
+                        if P[i][j] > 0))
+    kl = oracle_mod.distill_kl_rows(q, k, qx, kx)
+    np.testing.assert_allclose(kl, want, rtol=1e-10, atol=1e-12)
+    assert np.all(kl[1:] > 0) and abs(kl[0]) < 1e-15          # row 0: both distributions are {0: 1}
+    # one head, indexer = the layer's own scaled scores: identical distributions
+    q1, k1, _ = _rand(N, 1, 1, 16, seed=33)
+    kl0 = oracle_mod.distill_kl_rows(q1, k1, q1[:, 0, :] / 4.0, k1[:, 0, :])
+    np.testing.assert_allclose(kl0, 0.0, atol=1e-12)
