@@ -501,8 +501,17 @@ def run_ours(args, w, inp, rank, world, local_rank):
 def measure_next_rows(args, tam, w, step, flush):
     """Rows beyond the step (reported, not part of `value`): the fused, selection-block-
     shared indexer (block sums of each query's softmax of its indexer scores, top-k per
-    block of BLOCK_Q queries) and pass 3 on that support."""
+    block of BLOCK_Q queries), pass 3 on that support, and the indexer's distillation
+    target (KL of the indexer's distribution from the head-averaged mass)."""
     bq, kx = BLOCK_Q, INDEXER_K
+    lse = tam.attention_lse(step.q, step.k, workspace=step.ws, check=False)
+    # warm-up (first launches load the kernels; the workspace grows to its largest size)
+    for _ in range(2):
+        sup = tam.indexer_topk(step.qx, step.kx, kx, bq, workspace=step.ws, check=False)
+        tam.sparse_support_attention(step.q, step.k, step.v, sup.idx, sup.length, bq,
+                                     workspace=step.ws, check=False)
+        tam.distill_kl(step.q, step.k, lse, step.qx, step.kx, workspace=step.ws, check=False)
+    torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     for s in range(args.steps):
         flush.fill_(s & 0xff)
@@ -517,7 +526,19 @@ def measure_next_rows(args, tam, w, step, flush):
     t_sel = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     t_att = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     n_sel = sup.length.cpu().numpy().astype(np.int64)
+    # the indexer's distillation target (pass 1's lse is an input, as for pass 2)
+    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for s in range(args.steps):
+        flush.fill_(s & 0xff)
+        evk[s][0].record()
+        tam.distill_kl(step.q, step.k, lse, step.qx, step.kx, workspace=step.ws, check=False)
+        evk[s][1].record()
+    torch.cuda.synchronize()
+    tam.check_status(step.ws.get(256))
+    t_kl = statistics.mean(e[0].elapsed_time(e[1]) for e in evk)
     return {
+        "distill_kl": {"ms": t_kl, "q_tok_s": w.N / (t_kl * 1e-3),
+                       "what": "KL(P_i || softmax(q_idx_i . k_idx)) per query, lse given"},
         "indexer_block_topk": {"ms": t_sel, "q_tok_s": w.N / (t_sel * 1e-3), "budget_k": kx,
                                "block_q": bq},
         "pass3_indexer_block": {"ms": t_att, "q_tok_s": w.N / (t_att * 1e-3),

@@ -181,6 +181,25 @@ int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const v
                      float* sup_score, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * The indexer's distillation target (technical report §2.2, "Trainingsziel": the
+ * head-collapsed indexer is trained by KL divergence from the dense attention-mass
+ * distribution), per query, without returning the N x N distributions:
+ *   kl[i] = sum_{j <= i} P_i[j] log(P_i[j] / q_i[j]),  0 log 0 = 0,
+ *   P_i as in pass 2 (needs pass 1's lse [Hq, N]), q_i = softmax_{j <= i}(q_idx[i] . k_idx[j])
+ *   (scale 1, as for the block-shared indexer).
+ * q, k: as for tam_mass_select (bf16, tensor-core shapes); q_idx, k_idx: [N, d_idx] bf16,
+ * d_idx in {64, 128}; kl: [N] fp32.  Other dtypes or shapes: TAM_ERR_UNSUPPORTED.
+ * The mass rows and the indexer score rows of a chunk of queries go through two slabs
+ * in the workspace: tam_distill_kl_workspace() is the preferred size (every row at
+ * once, up to 2 x 4 GiB), tam_distill_kl_workspace_min() the smallest accepted.
+ */
+size_t tam_distill_kl_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, int d_idx);
+size_t tam_distill_kl_workspace_min(int64_t N, int Hq, int Hkv, int d, int dtype, int d_idx);
+int tam_distill_kl(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
+                   const float* lse, int d_idx, const void* q_idx, const void* k_idx, float* kl,
+                   void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Pass 3 alone: attention recomputed on a given support (technical report §2.1,
  * "Ausführung": original Q, K, V restricted to the selected tokens).
  * block_q == 1: row i of sup_idx (first sup_len[i] entries) is query i's support.

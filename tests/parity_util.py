@@ -18,6 +18,10 @@ REL_TIE = 1e-3
 MASS_ATOL = 1e-4
 OUT_ATOL = {"bf16": 2e-2, "f32": 1e-4}
 LSE_ATOL = 1e-3
+# KL per query: fp32 sums over up to 1e5 keys of P log P and P t, plus a log-sum-exp;
+# the probabilities carry ~3e-6 relative error (exp2 approximations), which moves the
+# sums by ~1e-5 per unit of entropy: 2e-3 absolute leaves an order of magnitude.
+KL_ATOL = 2e-3
 
 
 def check_support(gpu_idx, gpu_len, gpu_val, ora_idx, ora_len, ora_rows, val_atol=MASS_ATOL,

@@ -87,3 +87,16 @@ def test_indexer32k_block_shared_full(tam_lib, oracle_mod):
     pick = np.linspace(0, len(r) - 1, 32).astype(int)
     ref, _ = oracle_mod.attn_rows(inp.q, inp.k, inp.v, r[pick], sup=s[pick], sup_len=sl[pick])
     check_close(out.float().cpu().numpy()[r[pick]], ref, OUT_ATOL["bf16"], "indexer block output")
+
+
+def test_distill_kl_32k_sampled_rows(tam_lib, oracle_mod):
+    """The indexer's distillation target at the 32K shape, on sampled rows."""
+    from parity_util import KL_ATOL
+    w = tam_synth.WORKLOADS["indexer32k"]
+    inp = tam_synth.make_inputs(w)
+    q, k = inp.q.cuda(), inp.k.cuda()
+    lse = tam_lib.attention_lse(q, k)
+    kl = tam_lib.distill_kl(q, k, lse, inp.q_idx.cuda(), inp.k_idx.cuda()).cpu().numpy()
+    rows = tam_synth.sample_rows(w.N, inp.needle_i, n_random=24)
+    check_close(kl[rows], oracle_mod.distill_kl_rows(inp.q, inp.k, inp.q_idx, inp.k_idx, rows),
+                KL_ATOL, "distill kl 32k")

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import tam_synth
-from parity_util import LSE_ATOL, MASS_ATOL, OUT_ATOL, check_close, check_support
+from parity_util import KL_ATOL, LSE_ATOL, MASS_ATOL, OUT_ATOL, check_close, check_support
 
 pytestmark = pytest.mark.gpu
 
@@ -231,6 +231,31 @@ def test_indexer_block_shared_ties(tam_lib):
     for b in range(len(gl)):
         n = min(kb, min(N, (b + 1) * bq))
         assert gl[b] == n and list(gi[b, :n]) == list(range(n)), b
+
+
+@pytest.mark.parametrize("N,Hq,Hkv,d,dx", [(300, 32, 8, 128, 64), (1000, 16, 4, 128, 64),
+                                          (777, 8, 2, 64, 128), (129, 16, 1, 128, 64)])
+def test_distill_kl(tam_lib, oracle_mod, N, Hq, Hkv, d, dx):
+    """KL(P_i || softmax of indexer scores) per query against the oracle."""
+    inp = _inputs(N, Hq, Hkv, d, "bf16", seed=17 + N, sink=True, needles=3)
+    qx, kx = tam_synth.indexer_projections(inp, dx, seed=2)
+    q, k = _cuda(inp.q, inp.k)
+    lse = tam_lib.attention_lse(q, k)
+    kl = tam_lib.distill_kl(q, k, lse, qx.cuda(), kx.cuda()).cpu().numpy()
+    check_close(kl, oracle_mod.distill_kl_rows(inp.q, inp.k, qx, kx), KL_ATOL, "distill kl")
+
+
+def test_distill_kl_in_chunks(tam_lib):
+    """The smallest workspace (more chunks) gives the same values."""
+    N = 1500
+    inp = _inputs(N, 32, 8, 128, "bf16", seed=5)
+    qx, kx = tam_synth.indexer_projections(inp, 64, seed=2)
+    q, k = _cuda(inp.q, inp.k)
+    lse = tam_lib.attention_lse(q, k)
+    ref = tam_lib.distill_kl(q, k, lse, qx.cuda(), kx.cuda())
+    lo = tam_lib.lib().tam_distill_kl_workspace_min(N, 32, 8, 128, 0, 64)
+    got = tam_lib.distill_kl(q, k, lse, qx.cuda(), kx.cuda(), workspace_bytes=lo)
+    assert torch.equal(ref, got)
 
 
 def test_run_twice_bitwise_identical(tam_lib):

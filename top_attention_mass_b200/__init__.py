@@ -39,7 +39,8 @@ EXPORTED = (
     "tam_version", "tam_status_string", "tam_mass_oracle_workspace", "tam_mass_workspace_min",
     "tam_mass_oracle_prefill", "tam_attention_lse_workspace", "tam_attention_lse",
     "tam_mass_select_workspace", "tam_mass_select", "tam_mass_select_noalloc",
-    "tam_indexer_workspace", "tam_indexer_workspace_min", "tam_indexer_topk", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
+    "tam_indexer_workspace", "tam_indexer_workspace_min", "tam_indexer_topk",
+    "tam_distill_kl_workspace", "tam_distill_kl_workspace_min", "tam_distill_kl", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
     "tam_dense_workspace", "tam_dense_gqa_prefill", "tam_kernel_launches", "tam_check_status",
 )
 
@@ -97,6 +98,12 @@ def lib() -> ctypes.CDLL:
         L.tam_indexer_workspace_min.argtypes = [i64, i32, i32, i32, i32]
         L.tam_indexer_topk.restype = i32
         L.tam_indexer_topk.argtypes = [i64, i32, i32, p, p, i32, i32, p, p, p, p, sz, p]
+        L.tam_distill_kl_workspace.restype = sz
+        L.tam_distill_kl_workspace.argtypes = [i64, i32, i32, i32, i32, i32]
+        L.tam_distill_kl_workspace_min.restype = sz
+        L.tam_distill_kl_workspace_min.argtypes = [i64, i32, i32, i32, i32, i32]
+        L.tam_distill_kl.restype = i32
+        L.tam_distill_kl.argtypes = [i64, i32, i32, i32, i32, p, p, p, i32, p, p, p, p, sz, p]
         L.tam_sparse_attention_workspace.restype = sz
         L.tam_sparse_attention_workspace.argtypes = [i64, i32, i32, i32, i32]
         L.tam_sparse_support_attention.restype = i32
@@ -352,6 +359,34 @@ def indexer_topk(q_idx, k_idx, budget_k: int, block_q: int = 1, *,
     if host:
         res = Support(res.idx.cpu(), res.length.cpu(), res.value.cpu())
     return res
+
+
+def distill_kl(q, k, lse, q_idx, k_idx, *, workspace: Optional[Workspace] = None, stream=None,
+               check: bool = True, workspace_bytes: Optional[int] = None) -> torch.Tensor:
+    """The indexer's distillation target per query: KL(P_i || softmax(q_idx_i . k_idx)),
+    P_i the head-averaged mass of pass 2 (given pass 1's lse [Hq, N]).  Returns [N] fp32."""
+    dev = q.device
+    N, Hq, Hkv, d = _shape(q, k)
+    dt = _dtype_code(q)
+    if lse.shape != (Hq, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be [Hq, N] fp32")
+    if q_idx.shape != k_idx.shape or q_idx.shape[0] != N or q_idx.dtype != q.dtype:
+        raise ValueError("q_idx and k_idx must be [N, d_idx] in q's dtype")
+    dx = q_idx.shape[1]
+    kl = torch.empty(N, dtype=torch.float32, device=dev)
+    L = lib()
+    nbytes = L.tam_distill_kl_workspace(N, Hq, Hkv, d, dt, dx)
+    if workspace_bytes is not None and nbytes:
+        nbytes = int(workspace_bytes)
+    ws = _workspace(dev, max(nbytes, 256), workspace)
+    rc = L.tam_distill_kl(N, Hq, Hkv, d, dt, _ptr(q.contiguous()), _ptr(k.contiguous()),
+                          _ptr(lse.contiguous()), dx, _ptr(q_idx.contiguous()),
+                          _ptr(k_idx.contiguous()), _ptr(kl), _ptr(ws),
+                          min(ws.numel(), nbytes) if nbytes else 0, _stream(dev, stream))
+    _raise(rc, "distill_kl")
+    if check:
+        check_status(ws, stream)
+    return kl
 
 
 def sparse_support_attention(q, k, v, sup_idx, sup_len, block_q: int = 1, *,

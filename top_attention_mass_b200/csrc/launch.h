@@ -91,6 +91,10 @@ inline int64_t tri(int64_t i) { return i * (i + 1) / 2; }
 // ties toward the smaller index; sup_* are indexed by the absolute row i.
 cudaError_t row_topk(const float* slab, int64_t row0, int64_t row1, int budget, int32_t* sup_idx,
                      int32_t* sup_len, float* sup_val, cudaStream_t st);
+// kl[i] = KL(P_i || softmax(t_i)) for the rows [row0, row1) of a mass slab and a score
+// slab laid out alike.
+cudaError_t row_kl(const float* mass, const float* score, int64_t row0, int64_t row1, float* kl,
+                   cudaStream_t st);
 bool tc_dense_supported(const AttnArgs& a);
 cudaError_t tc_dense(const AttnArgs& a, cudaStream_t st);
 bool gather_supported(const AttnArgs& a);

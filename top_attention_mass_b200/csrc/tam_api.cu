@@ -375,6 +375,77 @@ int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const v
     return TAM_OK;
 }
 
+namespace {
+// Workspace of tam_distill_kl: status block, then two row slabs of equal size (mass
+// rows of the layer, score rows of the indexer) for a chunk of queries.
+struct KlPlan {
+    size_t off_slab, total, min_total;
+    bool ok;
+};
+
+KlPlan plan_kl(int64_t N, int Hq, int Hkv, int d, int dtype, int d_idx) {
+    KlPlan p{};
+    MassArgs a = mass_shape(N, Hq, Hkv, d, dtype, 1, 1);
+    p.ok = tc_mass_supported(a) && tc_indexer_supported(N, d_idx, dtype, 1);
+    p.off_slab = kStatusBytes;
+    p.total = p.off_slab + 2 * align256(slab_pref_bytes(N));
+    p.min_total = p.off_slab + 2 * align256(slab_min_bytes(N));
+    return p;
+}
+}  // namespace
+
+size_t tam_distill_kl_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, int d_idx) {
+    if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK) return 0;
+    const KlPlan p = plan_kl(N, Hq, Hkv, d, dtype, d_idx);
+    return p.ok ? p.total : 0;
+}
+
+size_t tam_distill_kl_workspace_min(int64_t N, int Hq, int Hkv, int d, int dtype, int d_idx) {
+    if (tam_distill_kl_workspace(N, Hq, Hkv, d, dtype, d_idx) == 0) return 0;
+    return plan_kl(N, Hq, Hkv, d, dtype, d_idx).min_total;
+}
+
+int tam_distill_kl(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
+                   const float* lse, int d_idx, const void* q_idx, const void* k_idx, float* kl,
+                   void* workspace, size_t ws_bytes, void* stream) {
+    int rc = check_shape(N, Hq, Hkv, d, dtype);
+    if (rc) return rc;
+    if (!q || !k || !lse || !q_idx || !k_idx || !kl || !workspace) return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, lse, q_idx, k_idx, kl, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
+    const KlPlan plan = plan_kl(N, Hq, Hkv, d, dtype, d_idx);
+    if (!plan.ok) return TAM_ERR_UNSUPPORTED;
+    if (ws_bytes < plan.min_total) return TAM_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    if ((rc = start_call(workspace, st))) return rc;
+    // two slabs of equal size share what follows the status block
+    const size_t half = ((ws_bytes - plan.off_slab) / 2) & ~size_t(255);
+    float* mass_rows = (float*)(ws + plan.off_slab);
+    float* score_rows = (float*)(ws + plan.off_slab + half);
+    MassArgs ma = mass_shape(N, Hq, Hkv, d, dtype, 1, 1);
+    ma.q = q; ma.k = k; ma.lse = lse; ma.sl2 = score_log2_scale(d);
+    ma.n_sel = (int)N;
+    ma.rows = mass_rows;
+    ma.status = (int32_t*)ws;
+    IndexerArgs ia{};
+    ia.N = N; ia.d_idx = d_idx; ia.dtype = dtype; ia.q_idx = q_idx; ia.k_idx = k_idx;
+    ia.budget = 1; ia.rows = score_rows; ia.status = (int32_t*)ws;
+    const int64_t cap = (int64_t)(half / sizeof(float));
+    for (int64_t r0 = 0; r0 < N;) {
+        const int64_t r1 = chunk_end(r0, N, cap);
+        ma.row0 = ia.row0 = r0;
+        ma.row1 = ia.row1 = r1;
+        cudaError_t e = tc_mass_pass(ma, st);
+        if (e == cudaSuccess) e = tc_indexer_rows(ia, st);
+        if (e == cudaSuccess) e = row_kl(mass_rows, score_rows, r0, r1, kl, st);
+        if (e != cudaSuccess) return TAM_ERR_CUDA;
+        r0 = r1;
+    }
+    return TAM_OK;
+}
+
 size_t tam_sparse_attention_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {
     if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK) return 0;
     return kStatusBytes;
