@@ -58,6 +58,7 @@ def lib():
             L.orc_indexer_block_mass.argtypes = [i64, i32, p, p, i32, p, i64, p]
             L.orc_indexer_block_topk.argtypes = [i64, i32, p, p, i32, p, i64, i32, p, p, p]
             L.orc_distill_kl_rows.argtypes = [i64, i32, i32, i32, p, p, i32, p, p, p, i64, p]
+            L.orc_support_mass_curve.argtypes = [i64, i32, i32, i32, p, p, p, i64, p, i32, p]
             _lib = L
     return _lib
 
@@ -244,6 +245,19 @@ def distill_kl_rows(q, k, q_idx, k_idx, rows=None) -> np.ndarray:
     _check(lib().orc_distill_kl_rows(N, Hq, Hkv, d, _ptr(q), _ptr(k), qx.shape[1], _ptr(qx),
                                      _ptr(kx), _ptr(r), len(r), _ptr(kl)))
     return kl
+
+
+def support_mass_curve(q, k, budgets, rows=None) -> np.ndarray:
+    """Support mass of each listed query at each budget: [n, len(budgets)] fp64."""
+    q, k = _f32(q), _f32(k)
+    N, Hq, d = q.shape
+    Hkv = k.shape[1]
+    r = _rows(rows, N)
+    ks = np.ascontiguousarray(budgets, np.int32)
+    out = np.zeros((len(r), len(ks)), np.float64)
+    _check(lib().orc_support_mass_curve(N, Hq, Hkv, d, _ptr(q), _ptr(k), _ptr(r), len(r), _ptr(ks),
+                                        len(ks), _ptr(out)))
+    return out
 
 
 def block_rows_support(block_idx, block_len, block_q: int, N: int, blocks=None):

@@ -19,7 +19,8 @@
 //   * same report, section 2.2 "Head-Collapsed Indexer": one shared token
 //     score across heads, top-k of it, sparse GQA recompute on that support;
 //     Abstract and section 3.2: the fused, selection-block-shared indexer path;
-//     section 2.2 "Trainingsziel": the indexer's KL-distillation target.
+//     section 2.2 "Trainingsziel": the indexer's KL-distillation target;
+//     section 3.1 "Budget-Sensitivitaet": support mass at several budgets.
 //
 // Readings where the pages are silent (each listed in the design notes):
 //   * query head h reads KV head g(h) = floor(h / (Hq/Hkv)) (consecutive grouping);
@@ -39,6 +40,7 @@
 // OpenMP; nothing else is blocked, fused or reordered.
 
 #include <algorithm>
+#include <functional>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -419,6 +421,35 @@ int orc_distill_kl_rows(int64_t N, int Hq, int Hkv, int d, const float* q, const
             for (int64_t j = 0; j <= i; ++j)
                 if (P[j] > 0.0) sum += P[j] * (std::log(P[j]) - (t[j] - lse));
             kl[r] = sum;
+        }
+    }
+    return 0;
+}
+
+// Budget sweep (technical report section 3.1, "Budget-Sensitivitaet": top-k budgets of
+// 256 to 2048 compared on the same oracle): the support mass of query i at budget k is
+// the sum of its k largest mass values, sum over S_i(k) of P_i[j].  out[r*nk + t] for
+// budget ks[t], for the listed rows.
+int orc_support_mass_curve(int64_t N, int Hq, int Hkv, int d, const float* q, const float* k,
+                           const int64_t* rows, int64_t nrows, const int32_t* ks, int nk,
+                           double* out) {
+    if (!shape_ok(N, Hq, Hkv, d) || nk < 1) return 1;
+    for (int t = 0; t < nk; ++t)
+        if (ks[t] < 1) return 1;
+#pragma omp parallel
+    {
+        std::vector<double> s(N), P(N);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nrows; ++r) {
+            const int64_t i = rows[r];
+            mass_row(q, k, Hq, Hkv, d, i, P.data(), s.data());
+            std::sort(P.begin(), P.begin() + i + 1, std::greater<double>());
+            for (int t = 0; t < nk; ++t) {
+                const int64_t n = std::min<int64_t>(ks[t], i + 1);
+                double acc = 0.0;
+                for (int64_t j = 0; j < n; ++j) acc += P[j];
+                out[r * nk + t] = acc;
+            }
         }
     }
     return 0;

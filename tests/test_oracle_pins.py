@@ -342,3 +342,23 @@ def test_distill_kl_brute_force_and_zero(oracle_mod):
     q1, k1, _ = _rand(N, 1, 1, 16, seed=33)
     kl0 = oracle_mod.distill_kl_rows(q1, k1, q1[:, 0, :] / 4.0, k1[:, 0, :])
     np.testing.assert_allclose(kl0, 0.0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ budget sweep
+def test_support_mass_curve(oracle_mod):
+    """The support mass at budget k equals the summed mass of the oracle's own top-k
+    support (selection, a different code path), grows with k, and is 1 once k covers
+    the causal prefix."""
+    N = 200
+    q, k, _ = _rand(N, 4, 2, 16, seed=41)
+    ks = [1, 5, 32, 150, 300]
+    curve = oracle_mod.support_mass_curve(q, k, ks)
+    P = oracle_mod.mass_rows(q, k)
+    for t, kb in enumerate(ks):
+        idx, ln, ms = oracle_mod.topk_rows(q, k, kb)
+        np.testing.assert_allclose(curve[:, t], ms.sum(axis=1), rtol=1e-12, atol=1e-15)
+        direct = [P[i, idx[i, :ln[i]]].sum() for i in range(N)]
+        np.testing.assert_allclose(curve[:, t], direct, rtol=1e-12, atol=1e-15)
+    assert np.all(np.diff(curve, axis=1) >= -1e-15)
+    full = np.arange(N) + 1 <= 300
+    np.testing.assert_allclose(curve[full, -1], 1.0, rtol=1e-12)
