@@ -501,8 +501,9 @@ def run_ours(args, w, inp, rank, world, local_rank):
 def measure_next_rows(args, tam, w, step, flush):
     """Rows beyond the step (reported, not part of `value`): the fused, selection-block-
     shared indexer (block sums of each query's softmax of its indexer scores, top-k per
-    block of BLOCK_Q queries), pass 3 on that support, and the indexer's distillation
-    target (KL of the indexer's distribution from the head-averaged mass)."""
+    block of BLOCK_Q queries), pass 3 on that support, the indexer's distillation
+    target (KL of the indexer's distribution from the head-averaged mass), and a budget
+    sweep (support mass at k = 256..2048 from one pass 2 at k = 2048)."""
     bq, kx = BLOCK_Q, INDEXER_K
     lse = tam.attention_lse(step.q, step.k, workspace=step.ws, check=False)
     # warm-up (first launches load the kernels; the workspace grows to its largest size)
@@ -536,7 +537,29 @@ def measure_next_rows(args, tam, w, step, flush):
     torch.cuda.synchronize()
     tam.check_status(step.ws.get(256))
     t_kl = statistics.mean(e[0].elapsed_time(e[1]) for e in evk)
+    # budget sweep from one pass 2 at k_max = 2048: per-query support mass at 256..2048
+    lse1 = lse
+    budgets = [256, 512, 1024, 2048]
+    sup = tam.mass_select(step.q, step.k, lse1, budgets[-1], 1, workspace=step.ws, check=False)
+    tam.support_mass_curve(sup.value, sup.length, budgets)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for s in range(args.steps):
+        flush.fill_(s & 0xff)
+        evs[s][0].record()
+        sup = tam.mass_select(step.q, step.k, lse1, budgets[-1], 1, workspace=step.ws, check=False)
+        evs[s][1].record()
+        curve = tam.support_mass_curve(sup.value, sup.length, budgets)
+        evs[s][2].record()
+    torch.cuda.synchronize()
+    tam.check_status(step.ws.get(256))
+    t_p2 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    t_cv = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    mean_mass = curve.mean(dim=0).cpu().tolist()
     return {
+        "budget_sweep": {"ms_pass2_kmax": t_p2, "ms_curve": t_cv, "budgets": budgets,
+                         "mean_support_mass": mean_mass,
+                         "sparsity": [1.0 - support_pairs(w.N, b) / causal_pairs(w.N) for b in budgets]},
         "distill_kl": {"ms": t_kl, "q_tok_s": w.N / (t_kl * 1e-3),
                        "what": "KL(P_i || softmax(q_idx_i . k_idx)) per query, lse given"},
         "indexer_block_topk": {"ms": t_sel, "q_tok_s": w.N / (t_sel * 1e-3), "budget_k": kx,

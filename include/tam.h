@@ -200,6 +200,21 @@ int tam_distill_kl(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, 
                    void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Budget sweep from one pass-2 run (technical report §3.1, "Budget-Sensitivitaet":
+ * the oracle compared at top-k budgets of 256 to 2048): for each row r of a top-kmax
+ * support (sup_val [n_rows, kmax] fp32 values >= 0, e.g. sup_mass of tam_mass_select,
+ * sup_len [n_rows]) and each budget budgets[t] (host array, 1 <= n_budgets <= 16),
+ *   out[r, t] = sum of the budgets[t] largest values of row r   (the whole row if
+ *               budgets[t] >= sup_len[r]),
+ * which is the support mass of the top-budgets[t] support whenever budgets[t] <= kmax.
+ * out: [n_rows, n_budgets] fp32, device.  kmax <= 4096.  No workspace; argument errors
+ * return before anything is enqueued.  The sparsity at a budget is a closed form
+ * (1 - sum_i min(k, i+1) / sum_i (i+1)) and needs no call.
+ */
+int tam_support_mass_curve(int64_t n_rows, int kmax, const float* sup_val, const int32_t* sup_len,
+                           const int32_t* budgets, int n_budgets, float* out, void* stream);
+
+/*
  * Pass 3 alone: attention recomputed on a given support (technical report §2.1,
  * "Ausführung": original Q, K, V restricted to the selected tokens).
  * block_q == 1: row i of sup_idx (first sup_len[i] entries) is query i's support.

@@ -258,6 +258,36 @@ def test_distill_kl_in_chunks(tam_lib):
     assert torch.equal(ref, got)
 
 
+@pytest.mark.parametrize("N,Hq,Hkv,d,kmax,bq", [(1000, 32, 8, 128, 256, 1), (600, 16, 4, 128, 700, 1),
+                                               (900, 32, 8, 128, 128, 64)])
+def test_support_mass_curve(tam_lib, oracle_mod, N, Hq, Hkv, d, kmax, bq):
+    """Budget sweep from one top-kmax pass 2: per row, the mass of the top-k for several k."""
+    inp = _inputs(N, Hq, Hkv, d, "bf16", seed=23 + N, sink=True, needles=4)
+    q, k = _cuda(inp.q, inp.k)
+    lse = tam_lib.attention_lse(q, k)
+    sup = tam_lib.mass_select(q, k, lse, kmax, bq)
+    ks = [1, 16, kmax // 2, kmax, kmax + 50]
+    curve = tam_lib.support_mass_curve(sup.value, sup.length, ks).cpu().numpy()
+    if bq == 1:
+        ref = oracle_mod.support_mass_curve(inp.q, inp.k, ks[:-1])
+        check_close(curve[:, :-1], ref, 1e-3, "support mass curve")
+    # a budget above kmax can only sum the whole top-kmax row
+    assert np.array_equal(curve[:, -1], curve[:, -2])
+    # and against the GPU's own top-k supports at each budget
+    for t, kb in enumerate(ks[:-1]):
+        s2 = tam_lib.mass_select(q, k, lse, kb, bq)
+        check_close(curve[:, t], s2.value.sum(dim=1).cpu().numpy(), 1e-3 * bq, f"k={kb}")
+
+
+def test_support_mass_curve_rejects(tam_lib):
+    x = torch.zeros(4, 8, device="cuda")
+    ln = torch.full((4,), 8, dtype=torch.int32, device="cuda")
+    with pytest.raises(tam_lib.TamError):
+        tam_lib.support_mass_curve(x, ln, [0])
+    with pytest.raises(tam_lib.TamError):
+        tam_lib.support_mass_curve(x, ln, list(range(1, 18)))
+
+
 def test_run_twice_bitwise_identical(tam_lib):
     inp = _inputs(700, 32, 8, 128, "bf16", seed=13, sink=True)
     q, k, v = _cuda(inp.q, inp.k, inp.v)

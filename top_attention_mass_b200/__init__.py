@@ -40,7 +40,8 @@ EXPORTED = (
     "tam_mass_oracle_prefill", "tam_attention_lse_workspace", "tam_attention_lse",
     "tam_mass_select_workspace", "tam_mass_select", "tam_mass_select_noalloc",
     "tam_indexer_workspace", "tam_indexer_workspace_min", "tam_indexer_topk",
-    "tam_distill_kl_workspace", "tam_distill_kl_workspace_min", "tam_distill_kl", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
+    "tam_distill_kl_workspace", "tam_distill_kl_workspace_min", "tam_distill_kl",
+    "tam_support_mass_curve", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
     "tam_dense_workspace", "tam_dense_gqa_prefill", "tam_kernel_launches", "tam_check_status",
 )
 
@@ -104,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.tam_distill_kl_workspace_min.argtypes = [i64, i32, i32, i32, i32, i32]
         L.tam_distill_kl.restype = i32
         L.tam_distill_kl.argtypes = [i64, i32, i32, i32, i32, p, p, p, i32, p, p, p, p, sz, p]
+        L.tam_support_mass_curve.restype = i32
+        L.tam_support_mass_curve.argtypes = [i64, i32, p, p, p, i32, p, p]
         L.tam_sparse_attention_workspace.restype = sz
         L.tam_sparse_attention_workspace.argtypes = [i64, i32, i32, i32, i32]
         L.tam_sparse_support_attention.restype = i32
@@ -387,6 +390,22 @@ def distill_kl(q, k, lse, q_idx, k_idx, *, workspace: Optional[Workspace] = None
     if check:
         check_status(ws, stream)
     return kl
+
+
+def support_mass_curve(sup_val, sup_len, budgets, *, stream=None) -> torch.Tensor:
+    """Budget sweep: [rows, len(budgets)] fp32, the sum of the k largest values of each
+    support row for every budget k (rows of a top-kmax support, e.g. Support.value)."""
+    dev = sup_val.device
+    if sup_val.dim() != 2 or sup_val.dtype != torch.float32 or sup_len.dtype != torch.int32:
+        raise TypeError("sup_val [rows, kmax] fp32 and sup_len [rows] int32")
+    rows, kmax = sup_val.shape
+    ks = (ctypes.c_int32 * len(budgets))(*[int(b) for b in budgets])
+    out = torch.empty(rows, len(budgets), dtype=torch.float32, device=dev)
+    rc = lib().tam_support_mass_curve(rows, kmax, _ptr(sup_val.contiguous()),
+                                      _ptr(sup_len.contiguous()), ks, len(budgets), _ptr(out),
+                                      _stream(dev, stream))
+    _raise(rc, "support_mass_curve")
+    return out
 
 
 def sparse_support_attention(q, k, v, sup_idx, sup_len, block_q: int = 1, *,

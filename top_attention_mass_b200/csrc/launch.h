@@ -91,6 +91,12 @@ inline int64_t tri(int64_t i) { return i * (i + 1) / 2; }
 // ties toward the smaller index; sup_* are indexed by the absolute row i.
 cudaError_t row_topk(const float* slab, int64_t row0, int64_t row1, int budget, int32_t* sup_idx,
                      int32_t* sup_len, float* sup_val, cudaStream_t st);
+// out[r, t] = sum of the ks[t] largest values of support row r (rows of a top-kmax
+// support: val [rows, kmax], len [rows]); nk <= kMaxSweepBudgets, kmax <= 4096.
+constexpr int kMaxSweepBudgets = 16;
+cudaError_t support_mass_curve(const float* val, const int32_t* len, int64_t rows, int kmax,
+                               const int32_t* ks, int nk, float* out, cudaStream_t st);
+
 // kl[i] = KL(P_i || softmax(t_i)) for the rows [row0, row1) of a mass slab and a score
 // slab laid out alike.
 cudaError_t row_kl(const float* mass, const float* score, int64_t row0, int64_t row1, float* kl,

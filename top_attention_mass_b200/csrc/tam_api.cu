@@ -446,6 +446,21 @@ int tam_distill_kl(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, 
     return TAM_OK;
 }
 
+int tam_support_mass_curve(int64_t n_rows, int kmax, const float* sup_val, const int32_t* sup_len,
+                           const int32_t* budgets, int n_budgets, float* out, void* stream) {
+    if (n_rows < 0 || kmax < 1 || !budgets || n_budgets < 1) return TAM_ERR_INVALID_ARG;
+    if (kmax > kMaxBudget || n_budgets > kMaxSweepBudgets) return TAM_ERR_UNSUPPORTED;
+    for (int t = 0; t < n_budgets; ++t)
+        if (budgets[t] < 1) return TAM_ERR_INVALID_ARG;
+    if (n_rows == 0) return TAM_OK;
+    if (!sup_val || !sup_len || !out) return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {sup_val, sup_len, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
+    return cuda_status(support_mass_curve(sup_val, sup_len, n_rows, kmax, budgets, n_budgets, out,
+                                          (cudaStream_t)stream));
+}
+
 size_t tam_sparse_attention_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {
     if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK) return 0;
     return kStatusBytes;
