@@ -281,7 +281,13 @@ k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
     const uint32_t wbuf = smem_addr(smem) + warp * STAGES * STAGE;
     const int64_t total = (int64_t)N * Hkv;
     for (int64_t item = (int64_t)blockIdx.x * W + warp; item < total; item += (int64_t)gridDim.x * W) {
-        const int i = (int)(item / Hkv), g = (int)(item % Hkv);
+        // KV groups in two halves when Hkv is even: all queries of the first half of the
+        // groups, then the second, so that each half's K/V (67 MB at the 32K layer) stays
+        // in L2 while it is gathered
+        const int gh = (Hkv % 2 == 0) ? Hkv / 2 : Hkv;
+        const int64_t per_half = (int64_t)N * gh;
+        const int64_t rem = item % per_half;
+        const int i = (int)(rem / gh), g = (int)(item / per_half) * gh + (int)(rem % gh);
         const int32_t* srow;
         int n;
         if (block_q == 1) {
