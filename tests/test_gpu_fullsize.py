@@ -100,3 +100,19 @@ def test_distill_kl_32k_sampled_rows(tam_lib, oracle_mod):
     rows = tam_synth.sample_rows(w.N, inp.needle_i, n_random=24)
     check_close(kl[rows], oracle_mod.distill_kl_rows(inp.q, inp.k, inp.q_idx, inp.k_idx, rows),
                 KL_ATOL, "distill kl 32k")
+
+
+def test_per_query_65k_in_chunks(tam_lib, oracle_mod):
+    """Per-query pass 2 at N = 65536 (16/4 heads, k = 2048): the mass rows (8.6 GB) exceed
+    the 4 GiB preferred slab, so they go through in chunks; sampled rows vs the oracle."""
+    w = tam_synth.WORKLOADS["longctx_65536"]
+    inp = tam_synth.make_inputs(w)
+    q, k = inp.q.cuda(), inp.k.cuda()
+    lse = tam_lib.attention_lse(q, k)
+    res = tam_lib.mass_select(q, k, lse, w.budget_k, 1)
+    torch.cuda.synchronize()
+    rows = np.concatenate([tam_synth.sample_rows(w.N, n_random=10), [w.N - 1, w.N // 2 + 31]])
+    oi, ol, _ = oracle_mod.topk_rows(inp.q, inp.k, w.budget_k, rows)
+    P = oracle_mod.mass_rows(inp.q, inp.k, rows)
+    check_support(res.idx.cpu().numpy()[rows], res.length.cpu().numpy()[rows],
+                  res.value.cpu().numpy()[rows], oi, ol, P, MASS_ATOL, "per query 65k")
