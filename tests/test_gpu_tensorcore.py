@@ -231,3 +231,49 @@ def test_pair_kernel_matches_single_cta_kernel(tam_lib, oracle_mod, monkeypatch,
         P = oracle_mod.mass_rows(inp.q, inp.k, rows)
         check_support(a.idx.cpu().numpy()[rows], a.length.cpu().numpy()[rows],
                       a.value.cpu().numpy()[rows], oi, ol, P, MASS_ATOL, "pair")
+
+
+@pytest.mark.parametrize("N,Hq,Hkv,d,kb,bq", [(1000, 32, 8, 128, 100, 64), (777, 16, 4, 128, 300, 128),
+                                              (600, 8, 1, 64, 80, 64), (513, 16, 2, 128, 50, 32)])
+def test_block_pass3_tensorcore_matches(tam_lib, oracle_mod, monkeypatch, N, Hq, Hkv, d, kb, bq):
+    """Block-shared pass 3 on tcgen05 over gathered chunks agrees with the oracle and with
+    the mma.sync kernel (TAM_DISABLE_BLOCK_TC=1)."""
+    inp = _inputs(N, Hq, Hkv, d, seed=N + bq, sink=True, needles=3)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    lse0 = tam_lib.attention_lse(q, k)
+    sup = tam_lib.mass_select(q, k, lse0, kb, bq)
+    out, lse = tam_lib.sparse_support_attention(q, k, v, sup.idx, sup.length, bq, return_lse=True)
+    monkeypatch.setenv("TAM_DISABLE_BLOCK_TC", "1")
+    out2, lse2 = tam_lib.sparse_support_attention(q, k, v, sup.idx, sup.length, bq, return_lse=True)
+    monkeypatch.delenv("TAM_DISABLE_BLOCK_TC")
+    gi, gl = sup.idx.cpu().numpy(), sup.length.cpu().numpy()
+    rows, s, sl = oracle_mod.block_rows_support(gi, gl, bq, N)
+    ref, rl = oracle_mod.attn_rows(inp.q, inp.k, inp.v, rows, sup=s, sup_len=sl)
+    check_close(out.float().cpu().numpy()[rows], ref, OUT_ATOL["bf16"], "block tc output")
+    check_close(lse.cpu().numpy().T[rows], rl, LSE_ATOL, "block tc lse")
+    assert (out.float() - out2.float()).abs().max().item() <= OUT_ATOL["bf16"]
+
+
+def test_block_pass3_tensorcore_empty_rows(tam_lib, oracle_mod):
+    """Hand-made block supports: queries before their block's first key (and a tile with
+    none at all) get a zero row and lse = -inf; keys past a query are masked."""
+    N, Hq, Hkv, d, bq, kmax = 256, 16, 4, 128, 64, 8
+    inp = _inputs(N, Hq, Hkv, d, seed=9)
+    rows_sup = [[40, 41, 42, 50], [0, 5, 100, 120, 127], [], [255]]
+    idx = np.full((4, kmax), -1, np.int32)
+    ln = np.zeros(4, np.int32)
+    for b, r in enumerate(rows_sup):
+        idx[b, :len(r)] = r
+        ln[b] = len(r)
+    out, lse = tam_lib.sparse_support_attention(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(),
+                                                torch.from_numpy(idx).cuda(),
+                                                torch.from_numpy(ln).cuda(), bq, return_lse=True)
+    rows, s, sl = oracle_mod.block_rows_support(idx, ln, bq, N)
+    ref, rl = oracle_mod.attn_rows(inp.q, inp.k, inp.v, rows, sup=s, sup_len=sl)
+    o = out.float().cpu().numpy()[rows]
+    check_close(o, ref, OUT_ATOL["bf16"], "block tc output (empty rows)")
+    lg = lse.cpu().numpy().T[rows]
+    empty = ~np.isfinite(rl)
+    assert np.array_equal(empty, ~np.isfinite(lg))
+    assert np.all(o[empty.all(axis=1)] == 0)
+    check_close(lg[~empty], rl[~empty], LSE_ATOL, "block tc lse (empty rows)")

@@ -1,0 +1,452 @@
+// Block-shared pass 3 on the tensor cores: attention recomputed on a block's support.
+//
+//   out[i,h] = sum_{j in T_i} softmax_{T_i}(scale * q[i,h].k[j,g(h)]) v[j,g(h)],
+//   T_i = S_b intersected with [0, i], b = i / block_q
+//
+// (arXiv 2606.07703, Abstract: "recomputes attention only on that support";
+// gist.science technical report §2.1 "Ausführung" and "Granularität": the support is
+// selected once for a block of consecutive queries.)
+//
+// The flash-style pipeline of the dense kernel over gathered keys.  One CTA owns one
+// KV group g and a tile of 128/G queries of block b (the G query heads packed as the
+// 128 UMMA rows, row = query*G + head); its keys are the entries of S_b up to the
+// tile's last query, in chunks of 128:
+//   gather warps (6-7)  cp.async the K and V rows of the chunk (two keys per thread,
+//                       zero-filled past the support) into 128-byte-swizzled shared
+//                       tiles laid out as a TMA tile load would leave them, stage the
+//                       key indices for the mask, fence to the async proxy and arrive;
+//   warp 4              TMA of the Q tile (once);
+//   warp 5              S = Q K^T into one of two TMEM buffers, then O += P V, S of
+//                       chunk t+1 issued before P V of chunk t;
+//   softmax warps 0-3   thread = row: mask (key not in [0, i] or past the support),
+//                       lazy online softmax in exp2 as in the dense kernel, P as bf16
+//                       into a swizzled shared tile; rows with no key get a zero output
+//                       row and lse = -inf.
+#include "launch.h"
+#include "tc_ptx.cuh"
+#include "tma_host.h"
+
+namespace tam {
+namespace {
+
+constexpr int kStages = 2;
+constexpr int kKeys = 128;                  // keys per chunk
+constexpr int kHalf = 128 * 64 * 2;         // one 128-row x 64-element swizzled half
+constexpr int kThreads = 256;
+constexpr int kGatherWarp0 = 6;             // warps 6..7 gather
+constexpr int kGatherThreads = kThreads - kGatherWarp0 * 32;
+constexpr float kRescaleLog2 = 8.f;
+
+template <int D>
+constexpr int block_tc_smem_bytes() {
+    // slack + Q + K ring + V ring + P + staged key indices + barriers
+    return 1024 + (D / 64) * kHalf * (1 + 2 * kStages) + 2 * kHalf + kStages * kKeys * 4 + 256;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+    const int n = valid ? 16 : 0;           // n = 0 writes 16 zero bytes
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Entries of an ascending support row (first n) that are <= limit.
+__device__ __forceinline__ int count_le(const int32_t* row, int n, int limit) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (row[mid] <= limit && row[mid] >= 0) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+struct BlockTcParams {
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    int N, Hq, Hkv, tiles_per_block, n_tiles;
+    int block_q, kmax;
+    float sl2;
+    const int32_t* sup_idx;
+    const int32_t* sup_len;
+    __nv_bfloat16* out;
+    float* lse;
+    int32_t* status;
+    uint64_t timeout_ns;
+};
+
+template <int G, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) {
+    constexpr int BQ = 128 / G;
+    constexpr int NH = D / 64;
+    constexpr uint32_t kTile = NH * kHalf;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* sQ = base;
+    uint8_t* sK = sQ + kTile;
+    uint8_t* sV = sK + kStages * kTile;
+    uint8_t* sP = sV + kStages * kTile;                 // 2 halves of 64 keys
+    int32_t* sIdx = reinterpret_cast<int32_t*>(sP + 2 * kHalf);    // kStages x 128
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sIdx + kStages * kKeys);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = q_full + 1;
+    uint64_t* kv_empty = kv_full + kStages;
+    uint64_t* s_full = kv_empty + kStages;
+    uint64_t* s_empty = s_full + 2;
+    uint64_t* p_full = s_empty + 2;
+    uint64_t* o_done = p_full + 1;
+    uint64_t* mma_done = o_done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = (int)(blockIdx.x % p.Hkv);
+    const int tile = p.n_tiles - 1 - (int)(blockIdx.x / p.Hkv);     // later blocks first
+    const int b = tile / p.tiles_per_block;
+    const int q0 = b * p.block_q + (tile % p.tiles_per_block) * BQ;
+    if (q0 >= p.N) return;                                          // uniform for the CTA
+    const int q_last = min(p.N, q0 + BQ) - 1;
+    const int32_t* srow = p.sup_idx + (size_t)b * p.kmax;
+    const int n_t = count_le(srow, min(p.sup_len[b], p.kmax), q_last);
+    const int n_ch = (n_t + kKeys - 1) / kKeys;
+
+    if (n_ch == 0) {
+        // no support key at or before any query of the tile: zero rows, lse = -inf
+        if (threadIdx.x < 128) {
+            const int r = threadIdx.x;
+            const int i = q0 + r / G, h = g * G + r % G;
+            if (i < p.N) {
+                __nv_bfloat16* orow = p.out + ((size_t)i * p.Hq + h) * D;
+                for (int c = 0; c < D; ++c) orow[c] = __float2bfloat16_rn(0.f);
+                if (p.lse) p.lse[(size_t)h * p.N + i] = -INFINITY;
+            }
+        }
+        return;
+    }
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(&kv_full[s], kGatherThreads);   // every gather thread
+            tc::mbar_init(&kv_empty[s], 1);
+        }
+        for (int bb = 0; bb < 2; ++bb) {
+            tc::mbar_init(&s_full[bb], 1);
+            tc::mbar_init(&s_empty[bb], 128);
+        }
+        tc::mbar_init(p_full, 128);
+        tc::mbar_init(o_done, 1);
+        tc::mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_o = tmem + 256;           // O accumulator: columns 256..256+D
+    const tc::Guard gd{abort_flag, p.status, KID_BLOCK_ATTN, p.timeout_ns};
+
+    if (warp >= kGatherWarp0) {
+        // ---------------------------------------------------------------- gather
+        const int r0 = threadIdx.x - kGatherWarp0 * 32;   // key rows r0, r0 + 64 of the chunk
+        const __nv_bfloat16* kbase = p.k + (size_t)g * D;
+        const __nv_bfloat16* vbase = p.v + (size_t)g * D;
+        const size_t row_stride = (size_t)p.Hkv * D;
+        for (int t = 0; t < n_ch; ++t) {
+            const int s = t % kStages;
+            if (!tc::wait(&kv_empty[s], ((t / kStages) & 1) ^ 1, gd, 1)) break;
+            const uint32_t dk = tc::smem_u32(sK + s * kTile), dv = tc::smem_u32(sV + s * kTile);
+#pragma unroll
+            for (int rr = 0; rr < kKeys / kGatherThreads; ++rr) {
+                const int r = r0 + rr * kGatherThreads;
+                const int c = t * kKeys + r;
+                const int j = c < n_t ? srow[c] : -1;
+                sIdx[s * kKeys + r] = j;
+                const bool valid = j >= 0;
+                const size_t off = valid ? (size_t)j * row_stride : 0;
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+#pragma unroll
+                    for (int pc = 0; pc < 8; ++pc) {
+                        const uint32_t o = h * kHalf + r * 128 + ((pc ^ (r & 7)) << 4);
+                        cp_async16(dk + o, kbase + off + h * 64 + pc * 8, valid);
+                        cp_async16(dv + o, vbase + off + h * 64 + pc * 8, valid);
+                    }
+            }
+            cp_async_commit();
+            // signal chunk t as soon as it has landed (made visible to the tensor core):
+            // the MMA issuer waits for it before it frees the stage chunk t+1 needs
+            cp_async_wait<0>();
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&kv_full[s]);
+        }
+        cp_async_wait<0>();
+    } else if (warp == 4) {
+        // ---------------------------------------------------------------- Q (TMA)
+        if (lane == 0) {
+            tc::prefetch_tmap(&tmQ);
+            tc::mbar_arrive_expect_tx(q_full, kTile);
+            for (int h = 0; h < NH; ++h)
+                tc::tma_load_3d(sQ + h * kHalf, &tmQ, q_full, h * 64, g * G, q0);
+            int zero = 0;
+            const tc::Guard drain{&zero, nullptr, 0, p.timeout_ns};
+            tc::wait(q_full, 0, drain, 0);
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128);
+            constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, false, true);
+            const uint32_t aq = tc::smem_u32(sQ);
+            const uint32_t ap = tc::smem_u32(sP);
+            bool ok = tc::wait(q_full, 0, gd, 3);
+            auto issue_s = [&](int t) -> bool {
+                const int s = t % kStages, bb = t & 1;
+                if (!tc::wait(&kv_full[s], (t / kStages) & 1, gd, 4)) return false;
+                if (!tc::wait(&s_empty[bb], ((t >> 1) & 1) ^ 1, gd, 5)) return false;
+                tc::fence_after_sync();
+                const uint32_t ak = tc::smem_u32(sK + s * kTile);
+#pragma unroll
+                for (int kk = 0; kk < NH * 4; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    tc::mma_bf16_ss(tmem + bb * 128, tc::desc_kmajor_sw128(aq + off),
+                                    tc::desc_kmajor_sw128(ak + off), idesc_s, kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&s_full[bb]);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int t = 0; ok && t < n_ch; ++t) {
+                if (t + 1 < n_ch && !issue_s(t + 1)) break;
+                const int s = t % kStages;
+                if (!tc::wait(p_full, t & 1, gd, 7)) break;
+                tc::fence_after_sync();
+                const uint32_t av = tc::smem_u32(sV + s * kTile);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {   // 128 keys in steps of 16
+                    const uint32_t offp = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    tc::mma_bf16_ss(tmem_o, tc::desc_kmajor_sw128(ap + offp),
+                                    tc::desc_mnmajor_sw128(av + kk * 16 * 128, kHalf), idesc_o,
+                                    (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc::mma_commit(&kv_empty[s]);
+                tc::mma_commit(o_done);
+            }
+            tc::mma_commit(mma_done);
+            int zero = 0;
+            const tc::Guard drain{&zero, nullptr, 0, p.timeout_ns};
+            tc::wait(mma_done, 0, drain, 0);
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax
+        const int r = threadIdx.x;
+        const int i = q0 + r / G;
+        const int h = g * G + r % G;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float sl2 = p.sl2;
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        uint8_t* prow0 = sP + r * 128;               // row r of half 0
+        for (int t = 0; ok && t < n_ch; ++t) {
+            const int bb = t & 1, s = t % kStages;
+            if (!tc::wait(&s_full[bb], (t >> 1) & 1, gd, 8)) { ok = false; break; }
+            tc::fence_after_sync();
+            uint32_t v[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tc::tmem_ld32(tmem + lane_off + bb * 128 + c * 32, v[c]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tc::tmem_wait_ld(v[c]);
+            tc::fence_before_sync();
+            tc::mbar_arrive(&s_empty[bb]);
+            // mask: keys past the support (index -1) or after query i
+            const int4* ix4 = reinterpret_cast<const int4*>(sIdx + s * kKeys);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const int4 jj = ix4[c * 8 + e4];
+                    const int js[4] = {jj.x, jj.y, jj.z, jj.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (js[e] < 0 || js[e] > i) v[c][e4 * 4 + e] = __float_as_uint(-INFINITY);
+                }
+            float tm[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    tm[c & 1] = tc::max3(tm[c & 1], __uint_as_float(v[c][e]),
+                                         __uint_as_float(v[c][e + 1]));
+            const float tmax = fmaxf(tm[0], tm[1]) * sl2;
+            const bool raise = tmax > m_used + kRescaleLog2;
+            const float m_new = raise ? tmax : m_used;
+            // a row with no key so far keeps l = 0 and a zero P row
+            const bool none = m_new == -INFINITY;
+            const float corr = none ? 1.f : tc::ex2(m_used - m_new);     // 0 on the first key
+            const uint64_t sl2x2 = tc::f2_pack(sl2, sl2);
+            const uint64_t negm2 = tc::f2_pack(none ? 0.f : -m_new, none ? 0.f : -m_new);
+            uint64_t sum2[2] = {0ull, 0ull};
+#pragma unroll
+            for (int c8 = 0; c8 < 16; ++c8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int col = c8 * 8 + 2 * e;
+                    const float s0 = __uint_as_float(v[col / 32][col % 32]);
+                    const float s1 = __uint_as_float(v[(col + 1) / 32][(col + 1) % 32]);
+                    const uint64_t x2 = tc::f2_fma(tc::f2_pack(s0, s1), sl2x2, negm2);
+                    float x0, x1, p0, p1;
+                    tc::f2_unpack(x2, x0, x1);
+                    if (e == 3) {
+                        tc::ex2_fma2(x0, x1, p0, p1);
+                    } else {
+                        p0 = tc::ex2(x0);
+                        p1 = tc::ex2(x1);
+                    }
+                    // masked keys are exactly 0 (the polynomial path would leave ~2^-125)
+                    p0 = s0 == -INFINITY ? 0.f : p0;
+                    p1 = s1 == -INFINITY ? 0.f : p1;
+                    sum2[e & 1] = tc::f2_add(sum2[e & 1], tc::f2_pack(p0, p1));
+                    __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+                    w[e] = *reinterpret_cast<uint32_t*>(&pk);
+                }
+                const int half = c8 >> 3, chunk = c8 & 7;
+                // P V of chunk t-1 must have finished reading the P tile before it is
+                // overwritten; wait once, before the first store
+                if (c8 == 0 && t > 0) {
+                    if (!tc::wait(o_done, (t - 1) & 1, gd, 9)) { ok = false; break; }
+                }
+                uint4* dst = reinterpret_cast<uint4*>(prow0 + half * kHalf + ((chunk ^ (r & 7)) << 4));
+                *dst = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            if (!ok) break;
+            float a0, a1, a2, a3;
+            tc::f2_unpack(sum2[0], a0, a1);
+            tc::f2_unpack(sum2[1], a2, a3);
+            l = l * corr + ((a0 + a1) + (a2 + a3));
+            const bool any_raise = __any_sync(0xffffffffu, raise && t > 0 && !none);
+            if (any_raise) {
+                tc::fence_after_sync();
+                const float f = (raise && t > 0 && !none) ? corr : 1.f;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tc::tmem_ld32(tmem_o + lane_off + c * 32, o);
+                    tc::tmem_wait_ld(o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                    tc::tmem_st32(tmem_o + lane_off + c * 32, o);
+                }
+                tc::tmem_wait_st();
+            }
+            m_used = m_new;
+            tc::fence_proxy_async_smem();
+            tc::fence_before_sync();
+            tc::mbar_arrive(p_full);
+        }
+        // epilogue: wait for the last P V, normalise, store bf16 rows
+        if (ok && tc::wait(o_done, (n_ch - 1) & 1, gd, 10)) {
+            tc::fence_after_sync();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16* orow = p.out + ((size_t)i * p.Hq + h) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tc::tmem_ld32(tmem_o + lane_off + c * 32, o);
+                tc::tmem_wait_ld(o);
+                if (i < p.N) {
+#pragma unroll
+                    for (int e8 = 0; e8 < 4; ++e8) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            __nv_bfloat162 pk = __floats2bfloat162_rn(
+                                __uint_as_float(o[e8 * 8 + 2 * e]) * inv,
+                                __uint_as_float(o[e8 * 8 + 2 * e + 1]) * inv);
+                            w[e] = *reinterpret_cast<uint32_t*>(&pk);
+                        }
+                        *reinterpret_cast<uint4*>(orow + c * 32 + e8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+            if (p.lse && i < p.N) p.lse[(size_t)h * p.N + i] = (m_used + __log2f(l)) * kLn2;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int G, int D>
+cudaError_t launch_block_tc(const AttnArgs& a, cudaStream_t st) {
+    constexpr int BQ = 128 / G;
+    CUtensorMap tq;
+    const uint64_t d = a.d;
+    if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQ))
+        return cudaErrorInvalidValue;
+    BlockTcParams p{};
+    p.k = (const __nv_bfloat16*)a.k;
+    p.v = (const __nv_bfloat16*)a.v;
+    p.N = (int)a.N;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.block_q = a.block_q;
+    p.kmax = a.kmax;
+    p.tiles_per_block = a.block_q / BQ;
+    const int nb = (int)((a.N + a.block_q - 1) / a.block_q);
+    p.n_tiles = nb * p.tiles_per_block;
+    p.sl2 = a.sl2;
+    p.sup_idx = a.sup_idx;
+    p.sup_len = a.sup_len;
+    p.out = (__nv_bfloat16*)a.out;
+    p.lse = a.lse;
+    p.status = a.status;
+    p.timeout_ns = wait_timeout_ns();
+    constexpr int smem = block_tc_smem_bytes<D>();
+    auto kern = k_attn_block_tc<G, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(p.n_tiles * a.Hkv), kThreads, smem, st>>>(tq, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t dispatch_g(const AttnArgs& a, cudaStream_t st) {
+    switch (a.Hq / a.Hkv) {
+        case 1: return launch_block_tc<1, D>(a, st);
+        case 2: return launch_block_tc<2, D>(a, st);
+        case 4: return launch_block_tc<4, D>(a, st);
+        case 8: return launch_block_tc<8, D>(a, st);
+        case 16: return launch_block_tc<16, D>(a, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+}  // namespace
+
+bool block_tc_supported(const AttnArgs& a) {
+    const int G = a.Hq / a.Hkv;
+    if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128) || a.block_q <= 1) return false;
+    if (!(G == 1 || G == 2 || G == 4 || G == 8 || G == 16)) return false;
+    return a.block_q % (128 / G) == 0 && a.sup_idx != nullptr;
+}
+
+cudaError_t block_attention_tc(const AttnArgs& a, cudaStream_t st) {
+    return a.d == 64 ? dispatch_g<64>(a, st) : dispatch_g<128>(a, st);
+}
+
+}  // namespace tam

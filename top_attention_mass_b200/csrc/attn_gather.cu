@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "tma_host.h"
 
 namespace tam {
 namespace {
@@ -472,7 +473,11 @@ bool gather_supported(const AttnArgs& a) {
 }
 
 cudaError_t gather_attention(const AttnArgs& a, cudaStream_t st) {
-    // block-shared supports go to the shared-chunk kernel when blocks have enough rows
+    // block-shared supports: tcgen05 over gathered chunks where the query tiles fit the
+    // blocks (attn_block_tc.cu), else the shared-chunk kernel when blocks have enough
+    // rows, else one warp per (query, group)
+    if (a.block_q > 1 && block_tc_supported(a) && !block_tc_disabled())
+        return block_attention_tc(a, st);
     const bool block = a.block_q > 1 && (int64_t)a.block_q * (a.Hq / a.Hkv) >= 64;
     return a.d == 64 ? dispatch<64>(a, st, block) : dispatch<128>(a, st, block);
 }

@@ -105,6 +105,8 @@ bool tc_dense_supported(const AttnArgs& a);
 cudaError_t tc_dense(const AttnArgs& a, cudaStream_t st);
 bool gather_supported(const AttnArgs& a);
 cudaError_t gather_attention(const AttnArgs& a, cudaStream_t st);
+bool block_tc_supported(const AttnArgs& a);
+cudaError_t block_attention_tc(const AttnArgs& a, cudaStream_t st);
 
 // CUDA-core kernels (any dtype, any supported shape).
 cudaError_t simt_lse(const LseArgs& a, cudaStream_t st);

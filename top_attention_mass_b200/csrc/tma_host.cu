@@ -59,6 +59,8 @@ uint64_t wait_timeout_ns() {
 
 bool pair_path_disabled() { return env_int("TAM_DISABLE_PAIR_KERNELS", 0) != 0; }
 
+bool block_tc_disabled() { return env_int("TAM_DISABLE_BLOCK_TC", 0) != 0; }
+
 int debug_flags() { return env_int("TAM_DEBUG_FORCE_TIMEOUT", 0) ? kDebugForceTimeout : 0; }
 
 }  // namespace tam

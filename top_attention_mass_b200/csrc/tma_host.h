@@ -26,5 +26,7 @@ constexpr int kDebugForceTimeout = 1;
 
 // TAM_DISABLE_PAIR_KERNELS=1 routes pass 2 to the single-CTA kernel (A/B comparisons).
 bool pair_path_disabled();
+// TAM_DISABLE_BLOCK_TC=1 routes block-shared pass 3 to the mma.sync kernel (A/B comparisons).
+bool block_tc_disabled();
 
 }  // namespace tam
