@@ -46,6 +46,9 @@ WORKLOAD = "gqa32k_2pct"
 BLOCK_Q = 64
 INDEXER_K = 1024
 D_IDX = 64
+# packed batch of mixed lengths (sums to the 32K workload's token count)
+VARLEN_SEQS = (8192, 4096, 2048, 6144, 1024, 3072, 5120, 3072)
+VARLEN_K = 256
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -556,7 +559,38 @@ def measure_next_rows(args, tam, w, step, flush):
     t_p2 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     t_cv = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     mean_mass = curve.mean(dim=0).cpu().tolist()
+    # packed batch: the step's tokens as VARLEN_SEQS independent sequences, per-query
+    # support at VARLEN_K (passes 1-3), and the dense comparator on the same batch
+    cu = [0]
+    for n in VARLEN_SEQS:
+        cu.append(cu[-1] + n)
+    vl = None
+    if cu[-1] == w.N:
+        for _ in range(2):
+            tam.mass_oracle_prefill_varlen(step.q, step.k, step.v, cu, VARLEN_K, 1,
+                                           workspace=step.ws, check=False)
+            tam.dense_gqa_prefill_varlen(step.q, step.k, step.v, cu, workspace=step.ws,
+                                         check=False)
+        torch.cuda.synchronize()
+        evv = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        for s in range(args.steps):
+            flush.fill_(s & 0xff)
+            evv[s][0].record()
+            tam.mass_oracle_prefill_varlen(step.q, step.k, step.v, cu, VARLEN_K, 1,
+                                           workspace=step.ws, check=False)
+            evv[s][1].record()
+            tam.dense_gqa_prefill_varlen(step.q, step.k, step.v, cu, workspace=step.ws,
+                                         check=False)
+            evv[s][2].record()
+        torch.cuda.synchronize()
+        tam.check_status(step.ws.get(256))
+        t_vo = statistics.mean(e[0].elapsed_time(e[1]) for e in evv)
+        t_vd = statistics.mean(e[1].elapsed_time(e[2]) for e in evv)
+        vl = {"seq_lens": list(VARLEN_SEQS), "budget_k": VARLEN_K,
+              "ms_oracle_passes_1_3": t_vo, "q_tok_s_oracle": w.N / (t_vo * 1e-3),
+              "ms_dense": t_vd, "q_tok_s_dense": w.N / (t_vd * 1e-3)}
     return {
+        "varlen_batch": vl,
         "budget_sweep": {"ms_pass2_kmax": t_p2, "ms_curve": t_cv, "budgets": budgets,
                          "mean_support_mass": mean_mass,
                          "sparsity": [1.0 - support_pairs(w.N, b) / causal_pairs(w.N) for b in budgets]},

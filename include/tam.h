@@ -27,7 +27,20 @@
  *   n_sel = N for per-query support (block_q == 1), ceil(N / block_q) otherwise.
  *
  * dtype: TAM_BF16 (bf16 storage, fp32 accumulation; tensor cores) or TAM_F32
- * (fp32 storage and arithmetic on CUDA cores).
+ * (fp32 storage and arithmetic on CUDA cores).  Head dim d: 64 or 128 (tensor
+ * cores for bf16), or 256 (CUDA-core kernels for either dtype: same results,
+ * lower throughput).
+ *
+ * Packed batches ("_varlen" entry points).  n_seq independent causal sequences
+ * are packed along the token axis: sequence s owns tokens [cu[s], cu[s+1]) of
+ * q/k/v/out (T = cu[n_seq] rows in the layouts above, positions restarting at 0
+ * in every sequence).  cu_seqlens is a HOST array of n_seq + 1 int64 with
+ * cu[0] = 0, non-decreasing (empty sequences are allowed), T < 2^31.  Per
+ * sequence the results are exactly those of the single-sequence call on its
+ * slice: key indices in sup_idx are positions within the sequence; selection
+ * rows are packed in sequence order (sequence s starts at row
+ * sum_{s'<s} n_sel(N_s')); lse is packed as one [Hq, N_s] block per sequence,
+ * block s starting at element Hq * cu[s].
  *
  * Ownership.  The caller allocates and frees every buffer, including the
  * workspace; the library never allocates device memory.  Every launch goes to
@@ -36,8 +49,9 @@
  *
  * Errors.  Argument errors are detected on the host before anything is
  * enqueued and returned directly: TAM_ERR_INVALID_ARG (null pointer, bad
- * shape, pointer not 16-byte aligned, k < 1, block_q < 1), TAM_ERR_UNSUPPORTED
- * (d not 64/128, k > 4096, N*k >= 2^31, combination not built), TAM_ERR_WORKSPACE
+ * shape, pointer not 16-byte aligned, k < 1, block_q < 1, bad cu_seqlens),
+ * TAM_ERR_UNSUPPORTED (d not 64/128/256, k > 4096, N*k >= 2^31, combination not
+ * built), TAM_ERR_WORKSPACE
  * (ws_bytes below the smallest accepted size).  A failed launch returns TAM_ERR_CUDA.
  * Errors found on the device (a bounded wait that gave up) are recorded in a
  * status block at the start of the workspace and are read by tam_check_status.
@@ -114,6 +128,28 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
                             const void* k, const void* v, int budget_k, int block_q,
                             int32_t* sup_idx, int32_t* sup_len, float* sup_mass, float* lse,
                             void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Workspace bytes tam_mass_oracle_prefill_varlen prefers: the largest of
+ * tam_mass_oracle_workspace over the batch's sequences (the sequences run one after
+ * another and share it).  0 for arguments the call would reject.
+ */
+size_t tam_mass_oracle_workspace_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv,
+                                        int d, int dtype, int budget_k, int block_q);
+
+/*
+ * tam_mass_oracle_prefill over a packed batch of independent sequences (layout in
+ * the header comment, "Packed batches").  Each sequence runs passes 1-3 on its own
+ * causal prefix, with the same budget_k and block_q; sup_idx/sup_len/sup_mass hold
+ * sum_s n_sel(N_s) rows, lse (or NULL) Hq * T floats, out (or NULL) [T, Hq, d].
+ * ws_bytes must reach the largest sequence's tam_mass_workspace_min, else
+ * TAM_ERR_WORKSPACE before anything is enqueued.
+ */
+int tam_mass_oracle_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv, int d,
+                                   int dtype, const void* q, const void* k, const void* v,
+                                   int budget_k, int block_q, int32_t* sup_idx, int32_t* sup_len,
+                                   float* sup_mass, float* lse, void* out, void* workspace,
+                                   size_t ws_bytes, void* stream);
 
 /*
  * Pass 1 alone: per-head log-sum-exp of the causal scores, lse [Hq, N] fp32
@@ -237,6 +273,16 @@ size_t tam_dense_workspace(int64_t N, int Hq, int Hkv, int d, int dtype);
 int tam_dense_gqa_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
                           const void* k, const void* v, void* out, float* lse, void* workspace,
                           size_t ws_bytes, void* stream);
+
+/*
+ * tam_dense_gqa_prefill over a packed batch of independent causal sequences (layout
+ * in the header comment, "Packed batches"): out [T, Hq, d], lse (or NULL) one
+ * [Hq, N_s] block per sequence.  Workspace: tam_dense_workspace bytes (any N).
+ */
+int tam_dense_gqa_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv, int d,
+                                 int dtype, const void* q, const void* k, const void* v,
+                                 void* out, float* lse, void* workspace, size_t ws_bytes,
+                                 void* stream);
 
 /*
  * Number of CUDA kernels this library has launched in this process so far (all

@@ -281,3 +281,76 @@ def sparsity(sup_sizes_per_query, N: int) -> float:
     """1 - (selected causal pairs) / (all causal pairs)."""
     total = N * (N + 1) // 2
     return 1.0 - float(np.sum(sup_sizes_per_query)) / total
+
+
+# ------------------------------------------------------------------ packed batches
+# A packed batch holds independent causal sequences back to back along the token
+# axis (sequence s owns tokens [cu[s], cu[s+1])); every quantity above is computed
+# per sequence on its own slice, positions restarting at 0.
+
+
+def seq_slices(cu_seqlens):
+    cu = np.asarray(cu_seqlens, np.int64)
+    if cu.ndim != 1 or cu.size < 2 or cu[0] != 0 or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens: [n_seq + 1], starts at 0, non-decreasing")
+    return [(int(cu[s]), int(cu[s + 1])) for s in range(cu.size - 1)]
+
+
+def varlen_mass_packed(q, k, cu_seqlens) -> np.ndarray:
+    """Head-averaged mass of every packed query over the packed keys, [T, T] fp64
+    (zero outside the query's own sequence and causal prefix)."""
+    q, k = _f32(q), _f32(k)
+    T = q.shape[0]
+    P = np.zeros((T, T), np.float64)
+    for t0, t1 in seq_slices(cu_seqlens):
+        if t1 > t0:
+            P[t0:t1, t0:t1] = mass_rows(q[t0:t1], k[t0:t1])
+    return P
+
+
+def varlen_support(q, k, cu_seqlens, budget: int, block_q: int = 1):
+    """Support of every sequence (per query, or per block of block_q queries), rows
+    packed in sequence order, key indices local to the sequence:
+    (idx [n_sel, k] int32 ascending, -1 pad; len [n_sel]; value [n_sel, k] fp64)."""
+    q, k = _f32(q), _f32(k)
+    parts = []
+    for t0, t1 in seq_slices(cu_seqlens):
+        if t1 == t0:
+            continue
+        if block_q == 1:
+            parts.append(topk_rows(q[t0:t1], k[t0:t1], budget))
+        else:
+            parts.append(block_topk(q[t0:t1], k[t0:t1], block_q, budget))
+    if not parts:
+        return (np.zeros((0, budget), np.int32), np.zeros(0, np.int32),
+                np.zeros((0, budget), np.float64))
+    return tuple(np.concatenate([p[c] for p in parts]) for c in range(3))
+
+
+def varlen_attn(q, k, v, cu_seqlens, sup=None, sup_len=None, block_q: int = 1):
+    """Attention of every packed query on its sequence (sup None: dense causal; else
+    the packed support rows as varlen_support lays them out, block rows expanded to
+    their queries): (out [T, Hq, d] fp64, lse [T, Hq] fp64)."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    T, Hq, d = q.shape
+    out = np.zeros((T, Hq, d), np.float64)
+    lse = np.zeros((T, Hq), np.float64)
+    sel0 = 0
+    for t0, t1 in seq_slices(cu_seqlens):
+        n = t1 - t0
+        if n == 0:
+            continue
+        n_sel = n if block_q == 1 else -(-n // block_q)
+        if sup is None:
+            o, l = attn_rows(q[t0:t1], k[t0:t1], v[t0:t1])
+        else:
+            si = np.asarray(sup)[sel0:sel0 + n_sel]
+            sl = np.asarray(sup_len)[sel0:sel0 + n_sel]
+            if block_q == 1:
+                o, l = attn_rows(q[t0:t1], k[t0:t1], v[t0:t1], sup=si, sup_len=sl)
+            else:
+                r, s, ln = block_rows_support(si, sl, block_q, n)
+                o, l = attn_rows(q[t0:t1], k[t0:t1], v[t0:t1], r, sup=s, sup_len=ln)
+        out[t0:t1], lse[t0:t1] = o, l
+        sel0 += n_sel
+    return out, lse

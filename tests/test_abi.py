@@ -120,3 +120,45 @@ def test_product_does_not_import_the_oracle():
                 txt = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, fn
                 assert "liboracle" not in txt and "orc_" not in txt, fn
+
+
+def test_varlen_and_head_dim_host_checks(tam_lib):
+    """Packed-batch offsets and head dims are validated on the host (no launch here)."""
+    import numpy as np
+    L = tam_lib.lib()
+    T = tam_lib
+    f = _fake()
+
+    def cu_ptr(a):
+        arr = np.ascontiguousarray(a, np.int64)
+        return arr, arr.ctypes.data_as(ctypes.c_void_p)
+
+    good, gp = cu_ptr([0, 100, 100, 4096])
+    ws = L.tam_mass_oracle_workspace_varlen(3, gp, 32, 8, 128, T.TAM_BF16, 256, 1)
+    assert ws > 0 and ws % 256 == 0
+    # the largest sequence sets the size: equal to the single-sequence query for it
+    assert ws == L.tam_mass_oracle_workspace(3996, 32, 8, 128, T.TAM_BF16, 256, 1)
+    assert L.tam_mass_oracle_workspace_varlen(3, gp, 32, 8, 256, T.TAM_BF16, 256, 1) > 0
+    assert L.tam_mass_oracle_workspace_varlen(3, gp, 32, 8, 96, T.TAM_BF16, 256, 1) == 0
+    for bad in ([1, 100], [0, 50, 40], [0, 1 << 31]):
+        arr, bp = cu_ptr(bad)
+        n = len(bad) - 1
+        assert L.tam_mass_oracle_workspace_varlen(n, bp, 32, 8, 128, 0, 8, 1) == 0
+        assert L.tam_mass_oracle_prefill_varlen(n, bp, 32, 8, 128, 0, f, f, f, 8, 1, f, f, f, None,
+                                                None, f, 1 << 30, None) != T.TAM_OK
+        assert L.tam_dense_gqa_prefill_varlen(n, bp, 32, 8, 128, 0, f, f, f, f, None, f, 1 << 20,
+                                              None) != T.TAM_OK
+    assert L.tam_mass_oracle_prefill_varlen(0, gp, 32, 8, 128, 0, f, f, f, 8, 1, f, f, f, None,
+                                            None, f, 1 << 30, None) == T.TAM_ERR_INVALID_ARG
+    assert L.tam_mass_oracle_prefill_varlen(3, None, 32, 8, 128, 0, f, f, f, 8, 1, f, f, f, None,
+                                            None, f, 1 << 30, None) == T.TAM_ERR_INVALID_ARG
+    # workspace below the largest sequence's minimum
+    assert L.tam_mass_oracle_prefill_varlen(3, gp, 32, 8, 128, 0, f, f, f, 8, 1, f, f, f, None,
+                                            None, f, 4096, None) == T.TAM_ERR_WORKSPACE
+    assert L.tam_dense_gqa_prefill_varlen(3, gp, 32, 8, 128, 0, f, f, f, f, None, f, 16,
+                                          None) == T.TAM_ERR_WORKSPACE
+    assert L.tam_dense_gqa_prefill_varlen(3, gp, 32, 8, 80, 0, f, f, f, f, None, f, 1 << 20,
+                                          None) == T.TAM_ERR_UNSUPPORTED
+    # head dim 256 is accepted by the single-sequence queries too
+    assert L.tam_mass_oracle_workspace(4096, 32, 8, 256, T.TAM_BF16, 256, 1) > 0
+    assert L.tam_dense_workspace(4096, 32, 8, 256, T.TAM_F32) > 0

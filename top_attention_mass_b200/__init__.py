@@ -14,6 +14,8 @@ Functions (same names as the C entry points, without the ``tam_`` prefix):
 * ``indexer_topk``             head-collapsed indexer support
 * ``sparse_support_attention`` pass 3 alone (attention on a given support)
 * ``dense_gqa_prefill``        dense causal GQA attention (comparator)
+* ``mass_oracle_prefill_varlen``, ``dense_gqa_prefill_varlen``
+                               the same over a packed batch of sequences
 
 Inputs may be CUDA tensors, or CPU tensors (ideally pinned): then they are
 copied to ``device``, the call runs there, and the results come back to the CPU.
@@ -43,6 +45,8 @@ EXPORTED = (
     "tam_distill_kl_workspace", "tam_distill_kl_workspace_min", "tam_distill_kl",
     "tam_support_mass_curve", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
     "tam_dense_workspace", "tam_dense_gqa_prefill", "tam_kernel_launches", "tam_check_status",
+    "tam_mass_oracle_workspace_varlen", "tam_mass_oracle_prefill_varlen",
+    "tam_dense_gqa_prefill_varlen",
 )
 
 
@@ -116,6 +120,14 @@ def lib() -> ctypes.CDLL:
         L.tam_dense_workspace.argtypes = [i64, i32, i32, i32, i32]
         L.tam_dense_gqa_prefill.restype = i32
         L.tam_dense_gqa_prefill.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, sz, p]
+        L.tam_mass_oracle_workspace_varlen.restype = sz
+        L.tam_mass_oracle_workspace_varlen.argtypes = [i32, p, i32, i32, i32, i32, i32, i32]
+        L.tam_mass_oracle_prefill_varlen.restype = i32
+        L.tam_mass_oracle_prefill_varlen.argtypes = [i32, p, i32, i32, i32, i32, p, p, p, i32, i32,
+                                                     p, p, p, p, p, p, sz, p]
+        L.tam_dense_gqa_prefill_varlen.restype = i32
+        L.tam_dense_gqa_prefill_varlen.argtypes = [i32, p, i32, i32, i32, i32, p, p, p, p, p, p,
+                                                   sz, p]
         L.tam_kernel_launches.restype = ctypes.c_uint64
         L.tam_check_status.restype = i32
         L.tam_check_status.argtypes = [p, p, p]
@@ -452,6 +464,102 @@ def dense_gqa_prefill(q, k, v, *, return_lse: bool = False,
     rc = L.tam_dense_gqa_prefill(N, Hq, Hkv, d, dt, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                  _ptr(lse), _ptr(ws), ws.numel(), _stream(dev, stream))
     _raise(rc, "dense_gqa_prefill")
+    if check:
+        check_status(ws, stream)
+    if host:
+        out = out.cpu()
+        lse = None if lse is None else lse.cpu()
+    return (out, lse) if return_lse else out
+
+
+# ------------------------------------------------------------------ packed batches
+
+def _cu_host(cu_seqlens) -> torch.Tensor:
+    """cu_seqlens as a contiguous host int64 tensor (the library reads it on the host)."""
+    cu = torch.as_tensor(cu_seqlens, dtype=torch.int64, device="cpu").contiguous()
+    if cu.dim() != 1 or cu.numel() < 2:
+        raise ValueError("cu_seqlens is [n_seq + 1] int64")
+    return cu
+
+
+def selection_offsets(cu_seqlens, block_q: int = 1) -> torch.Tensor:
+    """First selection row of every sequence of a packed batch ([n_seq + 1] int64)."""
+    cu = _cu_host(cu_seqlens)
+    n = cu[1:] - cu[:-1]
+    n_sel = n if block_q == 1 else (n + block_q - 1) // block_q
+    return torch.cat([torch.zeros(1, dtype=torch.int64), torch.cumsum(n_sel, 0)])
+
+
+def lse_block(lse: torch.Tensor, cu_seqlens, s: int) -> torch.Tensor:
+    """The [Hq, N_s] lse block of sequence s inside a packed varlen lse."""
+    cu = _cu_host(cu_seqlens)
+    t0, t1 = int(cu[s]), int(cu[s + 1])
+    Hq = lse.numel() // int(cu[-1]) if int(cu[-1]) else 0
+    return lse[Hq * t0:Hq * t1].view(Hq, t1 - t0)
+
+
+def mass_oracle_prefill_varlen(q, k, v, cu_seqlens, budget_k: int, block_q: int = 1, *,
+                               compute_out: bool = True, return_lse: bool = True,
+                               workspace: Optional[Workspace] = None, stream=None,
+                               check: bool = True, device=None) -> Support:
+    """mass_oracle_prefill over a packed batch: q [T, Hq, d], k/v [T, Hkv, d], sequence s
+    owning tokens [cu_seqlens[s], cu_seqlens[s+1]).  Support rows are packed in sequence
+    order (see ``selection_offsets``), key indices are positions within the sequence,
+    and ``lse`` is flat (one [Hq, N_s] block per sequence, see ``lse_block``)."""
+    cu = _cu_host(cu_seqlens)
+    n_seq = cu.numel() - 1
+    dev = _dev_of(q, device)
+    (q, k, v), host = _to_device([q, k, v], dev)
+    T, Hq, Hkv, d = _shape(q, k)
+    if int(cu[-1]) != T:
+        raise ValueError("cu_seqlens[-1] must equal the packed token count")
+    if compute_out and v is None:
+        raise ValueError("v is needed for the recomputed output")
+    dt = _dtype_code(q)
+    n_sel = int(selection_offsets(cu, block_q)[-1])
+    sup_idx = torch.empty(n_sel, budget_k, dtype=torch.int32, device=dev)
+    sup_len = torch.empty(n_sel, dtype=torch.int32, device=dev)
+    sup_mass = torch.empty(n_sel, budget_k, dtype=torch.float32, device=dev)
+    lse = torch.empty(Hq * T, dtype=torch.float32, device=dev) if return_lse else None
+    out = torch.empty_like(q) if compute_out else None
+    L = lib()
+    cu_p = ctypes.c_void_p(cu.data_ptr())
+    nbytes = L.tam_mass_oracle_workspace_varlen(n_seq, cu_p, Hq, Hkv, d, dt, budget_k, block_q)
+    ws = _workspace(dev, max(nbytes, 256), workspace)
+    rc = L.tam_mass_oracle_prefill_varlen(n_seq, cu_p, Hq, Hkv, d, dt, _ptr(q), _ptr(k), _ptr(v),
+                                          budget_k, block_q, _ptr(sup_idx), _ptr(sup_len),
+                                          _ptr(sup_mass), _ptr(lse), _ptr(out), _ptr(ws),
+                                          ws.numel() if nbytes else 0, _stream(dev, stream))
+    _raise(rc, "mass_oracle_prefill_varlen")
+    if check:
+        check_status(ws, stream)
+    res = Support(sup_idx, sup_len, sup_mass, lse, out)
+    if host:
+        res = Support(*[None if t is None else t.cpu() for t in
+                        (res.idx, res.length, res.value, res.lse, res.out)])
+    return res
+
+
+def dense_gqa_prefill_varlen(q, k, v, cu_seqlens, *, return_lse: bool = False,
+                             workspace: Optional[Workspace] = None, stream=None,
+                             check: bool = True, device=None):
+    """dense_gqa_prefill over a packed batch (layout as mass_oracle_prefill_varlen)."""
+    cu = _cu_host(cu_seqlens)
+    n_seq = cu.numel() - 1
+    dev = _dev_of(q, device)
+    (q, k, v), host = _to_device([q, k, v], dev)
+    T, Hq, Hkv, d = _shape(q, k)
+    if int(cu[-1]) != T:
+        raise ValueError("cu_seqlens[-1] must equal the packed token count")
+    dt = _dtype_code(q)
+    out = torch.empty_like(q)
+    lse = torch.empty(Hq * T, dtype=torch.float32, device=dev) if return_lse else None
+    L = lib()
+    ws = _workspace(dev, 256, workspace)
+    rc = L.tam_dense_gqa_prefill_varlen(n_seq, ctypes.c_void_p(cu.data_ptr()), Hq, Hkv, d, dt,
+                                        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(ws),
+                                        ws.numel(), _stream(dev, stream))
+    _raise(rc, "dense_gqa_prefill_varlen")
     if check:
         check_status(ws, stream)
     if host:

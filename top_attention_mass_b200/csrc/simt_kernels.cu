@@ -238,10 +238,18 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <typename T>
+static cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st) {
+    switch (a.d) {
+        case 64: return launch_attn_t<T, 2>(a, st);
+        case 128: return launch_attn_t<T, 4>(a, st);
+        case 256: return launch_attn_t<T, 8>(a, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
 cudaError_t simt_attention(const AttnArgs& a, cudaStream_t st) {
-    if (a.dtype == TAM_F32)
-        return a.d == 64 ? launch_attn_t<float, 2>(a, st) : launch_attn_t<float, 4>(a, st);
-    return a.d == 64 ? launch_attn_t<__nv_bfloat16, 2>(a, st) : launch_attn_t<__nv_bfloat16, 4>(a, st);
+    return a.dtype == TAM_F32 ? launch_attn<float>(a, st) : launch_attn<__nv_bfloat16>(a, st);
 }
 
 template <typename T>

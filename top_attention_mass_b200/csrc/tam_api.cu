@@ -31,7 +31,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 int check_shape(int64_t N, int Hq, int Hkv, int d, int dtype) {
     if (N < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TAM_ERR_INVALID_ARG;
     if (dtype != TAM_BF16 && dtype != TAM_F32) return TAM_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return TAM_ERR_UNSUPPORTED;
+    // 64 and 128 run on the tensor cores; 256 on the CUDA-core kernels
+    if (d != 64 && d != 128 && d != 256) return TAM_ERR_UNSUPPORTED;
     if (N >= (int64_t(1) << 31) - 1) return TAM_ERR_UNSUPPORTED;
     // the CUDA-core kernels stage one query row (all heads) in shared memory
     if ((size_t)(Hq * d + Hq) * sizeof(float) > 200 * 1024) return TAM_ERR_UNSUPPORTED;
@@ -184,6 +185,59 @@ int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void*
     return TAM_OK;
 }
 
+// Null and alignment checks of the prefill entry points.
+int check_prefill_ptrs(const void* q, const void* k, const void* v, const void* sup_idx,
+                       const void* sup_len, const void* sup_mass, const void* lse,
+                       const void* out, const void* workspace) {
+    if (!q || !k || !sup_idx || !sup_len || !sup_mass || !workspace) return TAM_ERR_INVALID_ARG;
+    if (out && !v) return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, sup_idx, sup_len, sup_mass, lse, out, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return TAM_ERR_INVALID_ARG;
+    return TAM_OK;
+}
+
+// Passes 1-3 of one causal sequence of N tokens (the status block is already cleared).
+int run_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, const void* k,
+                const void* v, int budget_k, int block_q, int32_t* sup_idx, int32_t* sup_len,
+                float* sup_mass, float* lse, void* out, char* ws, size_t ws_bytes,
+                const MassPlan& plan, cudaStream_t st) {
+    int32_t* status = (int32_t*)ws;
+    float* lse_buf = lse ? lse : (float*)(ws + plan.off_lse);
+    const float sl2 = score_log2_scale(d);
+    int rc;
+    LseArgs la{N, Hq, Hkv, d, dtype, q, k, sl2, lse_buf, status};
+    if ((rc = cuda_status(run_lse(la, st)))) return rc;
+
+    if ((rc = launch_mass_select(N, Hq, Hkv, d, dtype, q, k, lse_buf, budget_k, block_q, sup_idx,
+                                 sup_len, sup_mass, ws, ws_bytes, plan, st, sl2)))
+        return rc;
+
+    if (out) {
+        AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, sl2, sup_idx, sup_len, budget_k, block_q,
+                    out, nullptr, status};
+        if ((rc = cuda_status(run_sparse_attention(aa, st)))) return rc;
+    }
+    return TAM_OK;
+}
+
+// Host-side cumulative lengths of a packed batch: cu[0] = 0, non-decreasing, total
+// below 2^31 tokens.  Empty sequences are allowed.
+int check_cu_seqlens(int n_seq, const int64_t* cu, int64_t* max_len) {
+    if (n_seq < 1 || !cu || cu[0] != 0) return TAM_ERR_INVALID_ARG;
+    int64_t mx = 0;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t n = cu[s + 1] - cu[s];
+        if (n < 0) return TAM_ERR_INVALID_ARG;
+        mx = std::max(mx, n);
+    }
+    if (cu[n_seq] >= (int64_t(1) << 31) - 1) return TAM_ERR_UNSUPPORTED;
+    *max_len = mx;
+    return TAM_OK;
+}
+
+inline size_t elt_bytes(int dtype) { return dtype == TAM_F32 ? 4 : 2; }
+
 }  // namespace
 
 extern "C" {
@@ -220,31 +274,67 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
     if (rc) return rc;
     rc = check_budget(N, budget_k, block_q);
     if (rc) return rc;
-    if (!q || !k || !sup_idx || !sup_len || !sup_mass || !workspace) return TAM_ERR_INVALID_ARG;
-    if (out && !v) return TAM_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, sup_idx, sup_len, sup_mass, lse, out, workspace};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return TAM_ERR_INVALID_ARG;
+    if ((rc = check_prefill_ptrs(q, k, v, sup_idx, sup_len, sup_mass, lse, out, workspace)))
+        return rc;
     const MassPlan plan = plan_mass(N, Hq, Hkv, d, dtype, budget_k, block_q);
     if (ws_bytes < plan.min_total) return TAM_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
-    char* ws = (char*)workspace;
-    int32_t* status = (int32_t*)ws;
-    float* lse_buf = lse ? lse : (float*)(ws + plan.off_lse);
     if ((rc = start_call(workspace, st))) return rc;
+    return run_prefill(N, Hq, Hkv, d, dtype, q, k, v, budget_k, block_q, sup_idx, sup_len,
+                       sup_mass, lse, out, (char*)workspace, ws_bytes, plan, st);
+}
 
-    const float sl2 = score_log2_scale(d);
-    LseArgs la{N, Hq, Hkv, d, dtype, q, k, sl2, lse_buf, status};
-    if ((rc = cuda_status(run_lse(la, st)))) return rc;
+size_t tam_mass_oracle_workspace_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv,
+                                        int d, int dtype, int budget_k, int block_q) {
+    int64_t max_len = 0;
+    if (check_cu_seqlens(n_seq, cu_seqlens, &max_len) != TAM_OK) return 0;
+    if (check_shape(std::max<int64_t>(max_len, 1), Hq, Hkv, d, dtype) != TAM_OK) return 0;
+    if (check_budget(std::max<int64_t>(max_len, 1), budget_k, block_q) != TAM_OK) return 0;
+    size_t total = kStatusBytes;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t n = cu_seqlens[s + 1] - cu_seqlens[s];
+        if (n > 0) total = std::max(total, plan_mass(n, Hq, Hkv, d, dtype, budget_k, block_q).total);
+    }
+    return total;
+}
 
-    if ((rc = launch_mass_select(N, Hq, Hkv, d, dtype, q, k, lse_buf, budget_k, block_q, sup_idx,
-                                 sup_len, sup_mass, ws, ws_bytes, plan, st, sl2)))
+int tam_mass_oracle_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv, int d,
+                                   int dtype, const void* q, const void* k, const void* v,
+                                   int budget_k, int block_q, int32_t* sup_idx, int32_t* sup_len,
+                                   float* sup_mass, float* lse, void* out, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+    int64_t max_len = 0;
+    int rc = check_cu_seqlens(n_seq, cu_seqlens, &max_len);
+    if (rc) return rc;
+    if ((rc = check_shape(std::max<int64_t>(max_len, 1), Hq, Hkv, d, dtype))) return rc;
+    if ((rc = check_budget(std::max<int64_t>(max_len, 1), budget_k, block_q))) return rc;
+    if ((rc = check_prefill_ptrs(q, k, v, sup_idx, sup_len, sup_mass, lse, out, workspace)))
         return rc;
-
-    if (out) {
-        AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, sl2, sup_idx, sup_len, budget_k, block_q,
-                    out, nullptr, status};
-        if ((rc = cuda_status(run_sparse_attention(aa, st)))) return rc;
+    if (ws_bytes < kStatusBytes) return TAM_ERR_WORKSPACE;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t n = cu_seqlens[s + 1] - cu_seqlens[s];
+        if (n > 0 && ws_bytes < plan_mass(n, Hq, Hkv, d, dtype, budget_k, block_q).min_total)
+            return TAM_ERR_WORKSPACE;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((rc = start_call(workspace, st))) return rc;
+    // The sequences are independent problems: each one runs the single-sequence path on
+    // its slice of the packed tensors, one after another on `stream`, reusing the
+    // workspace (stream order separates them).
+    const size_t qrow = (size_t)Hq * d * elt_bytes(dtype), krow = (size_t)Hkv * d * elt_bytes(dtype);
+    int64_t sel0 = 0;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t t0 = cu_seqlens[s], n = cu_seqlens[s + 1] - t0;
+        if (n == 0) continue;
+        const MassPlan plan = plan_mass(n, Hq, Hkv, d, dtype, budget_k, block_q);
+        rc = run_prefill(n, Hq, Hkv, d, dtype, (const char*)q + t0 * qrow,
+                         (const char*)k + t0 * krow, v ? (const char*)v + t0 * krow : nullptr,
+                         budget_k, block_q, sup_idx + sel0 * budget_k, sup_len + sel0,
+                         sup_mass + sel0 * budget_k, lse ? lse + (size_t)Hq * t0 : nullptr,
+                         out ? (char*)out + t0 * qrow : nullptr, (char*)workspace, ws_bytes, plan,
+                         st);
+        if (rc) return rc;
+        sel0 += n_selection_units(n, block_q);
     }
     return TAM_OK;
 }
@@ -506,6 +596,35 @@ int tam_dense_gqa_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const vo
     AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, score_log2_scale(d), nullptr, nullptr, 0, 1,
                 out, lse, (int32_t*)workspace};
     return cuda_status(tc_dense_supported(aa) ? tc_dense(aa, st) : simt_attention(aa, st));
+}
+
+int tam_dense_gqa_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv, int d,
+                                 int dtype, const void* q, const void* k, const void* v,
+                                 void* out, float* lse, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+    int64_t max_len = 0;
+    int rc = check_cu_seqlens(n_seq, cu_seqlens, &max_len);
+    if (rc) return rc;
+    if ((rc = check_shape(std::max<int64_t>(max_len, 1), Hq, Hkv, d, dtype))) return rc;
+    if (!q || !k || !v || !out || !workspace) return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, out, lse, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return TAM_ERR_INVALID_ARG;
+    if (ws_bytes < kStatusBytes) return TAM_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((rc = start_call(workspace, st))) return rc;
+    const size_t qrow = (size_t)Hq * d * elt_bytes(dtype), krow = (size_t)Hkv * d * elt_bytes(dtype);
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t t0 = cu_seqlens[s], n = cu_seqlens[s + 1] - t0;
+        if (n == 0) continue;
+        AttnArgs aa{n, Hq, Hkv, d, dtype, (const char*)q + t0 * qrow, (const char*)k + t0 * krow,
+                    (const char*)v + t0 * krow, score_log2_scale(d), nullptr, nullptr, 0, 1,
+                    (char*)out + t0 * qrow, lse ? lse + (size_t)Hq * t0 : nullptr,
+                    (int32_t*)workspace};
+        if ((rc = cuda_status(tc_dense_supported(aa) ? tc_dense(aa, st) : simt_attention(aa, st))))
+            return rc;
+    }
+    return TAM_OK;
 }
 
 int tam_check_status(const void* workspace, void* stream, int32_t* detail) {
