@@ -11,8 +11,8 @@
 // KV group g and a tile of 128/G queries of block b (the G query heads packed as the
 // 128 UMMA rows, row = query*G + head); its keys are the entries of S_b up to the
 // tile's last query, in chunks of 128:
-//   gather warps (6-7)  cp.async the K and V rows of the chunk (two keys per thread,
-//                       zero-filled past the support) into 128-byte-swizzled shared
+//   gather warps (6-7)  cp.async the K and V rows of the chunk (whole rows per warp
+//                       instruction, zero-filled past the support) into 128-byte-swizzled shared
 //                       tiles laid out as a TMA tile load would leave them, stage the
 //                       key indices for the mask, fence to the async proxy and arrive;
 //   warp 4              TMA of the Q tile (once);
@@ -52,17 +52,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Entries of an ascending support row (first n) that are <= limit.
-__device__ __forceinline__ int count_le(const int32_t* row, int n, int limit) {
-    int lo = 0, hi = n;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (row[mid] <= limit && row[mid] >= 0) lo = mid + 1;
-        else hi = mid;
-    }
-    return lo;
 }
 
 struct BlockTcParams {
@@ -113,7 +102,27 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
     if (q0 >= p.N) return;                                          // uniform for the CTA
     const int q_last = min(p.N, q0 + BQ) - 1;
     const int32_t* srow = p.sup_idx + (size_t)b * p.kmax;
-    const int n_t = count_le(srow, min(p.sup_len[b], p.kmax), q_last);
+    // n_t = 1 + the last position of the (ascending) support row holding a key <= q_last:
+    // one round of independent loads across the CTA and a max-reduction, instead of a
+    // chain of dependent loads; the first chunk's indices are staged on the way.
+    __shared__ int s_last[kThreads / 32];
+    {
+        const int len = min(p.sup_len[b], p.kmax);
+        int last = 0;
+#pragma unroll 4
+        for (int c = threadIdx.x; c < len; c += kThreads) {
+            const int j = srow[c];
+            if (j <= q_last) last = c + 1;
+            if (c < kKeys) sIdx[c] = j;
+        }
+        if (threadIdx.x < kKeys && (int)threadIdx.x >= len) sIdx[threadIdx.x] = -1;
+        last = __reduce_max_sync(0xffffffffu, last);
+        if (lane == 0) s_last[warp] = last;
+    }
+    __syncthreads();
+    int n_t = 0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) n_t = max(n_t, s_last[w]);
     const int n_ch = (n_t + kKeys - 1) / kKeys;
 
     if (n_ch == 0) {
@@ -159,30 +168,52 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
 
     if (warp >= kGatherWarp0) {
         // ---------------------------------------------------------------- gather
-        const int r0 = threadIdx.x - kGatherWarp0 * 32;   // key rows r0, r0 + 64 of the chunk
-        const __nv_bfloat16* kbase = p.k + (size_t)g * D;
-        const __nv_bfloat16* vbase = p.v + (size_t)g * D;
+        // Warp gw copies key rows [64 gw, 64 gw + 64) of each chunk.  Lane l owns the
+        // indices of rows 64 gw + l and 64 gw + 32 + l; the copies go row-contiguous:
+        // PR lanes share one row (lane % PR = its 16-byte piece), so one warp
+        // instruction moves 32 / PR whole rows with every sector fully used.
+        const int gw = warp - kGatherWarp0;
+        constexpr int PR = D / 8;                          // 16-byte pieces per row
+        constexpr int RPI = 32 / PR;                       // rows per warp instruction
+        constexpr int RPW = kKeys / (kGatherThreads / 32); // rows per gather warp
+        constexpr int RR = RPW / 32;                       // index registers per lane
+        static_assert(RR * 32 == RPW && RPI * PR == 32, "gather tiling");
+        const int piece = lane % PR, sub = lane / PR;
+        const uint32_t half_off = (uint32_t)(piece / 8) * kHalf;
+        const int pc = piece % 8;
+        const __nv_bfloat16* kbase = p.k + (size_t)g * D + piece * 8;
+        const __nv_bfloat16* vbase = p.v + (size_t)g * D + piece * 8;
         const size_t row_stride = (size_t)p.Hkv * D;
+        int jn[RR];                                        // indices of the next chunk
+#pragma unroll
+        for (int rr = 0; rr < RR; ++rr) {
+            const int r = gw * RPW + rr * 32 + lane;
+            jn[rr] = r < n_t ? sIdx[r] : -1;              // chunk 0, staged above
+        }
         for (int t = 0; t < n_ch; ++t) {
             const int s = t % kStages;
             if (!tc::wait(&kv_empty[s], ((t / kStages) & 1) ^ 1, gd, 1)) break;
             const uint32_t dk = tc::smem_u32(sK + s * kTile), dv = tc::smem_u32(sV + s * kTile);
+            int js[RR];
 #pragma unroll
-            for (int rr = 0; rr < kKeys / kGatherThreads; ++rr) {
-                const int r = r0 + rr * kGatherThreads;
-                const int c = t * kKeys + r;
-                const int j = c < n_t ? srow[c] : -1;
-                sIdx[s * kKeys + r] = j;
+            for (int rr = 0; rr < RR; ++rr) {
+                const int j = jn[rr];
+                js[rr] = (j >= 0 && j < p.N) ? j : -1;
+                sIdx[s * kKeys + gw * RPW + rr * 32 + lane] = js[rr];
+                // the next chunk's indices load while this chunk's rows are in flight
+                const int c = (t + 1) * kKeys + gw * RPW + rr * 32 + lane;
+                jn[rr] = c < n_t ? srow[c] : -1;
+            }
+#pragma unroll
+            for (int it = 0; it < RPW / RPI; ++it) {
+                const int rl = it * RPI + sub;             // row within the warp's share
+                const int j = __shfl_sync(0xffffffffu, js[(it * RPI) >> 5], rl & 31);
+                const int r = gw * RPW + rl;
                 const bool valid = j >= 0;
                 const size_t off = valid ? (size_t)j * row_stride : 0;
-#pragma unroll
-                for (int h = 0; h < NH; ++h)
-#pragma unroll
-                    for (int pc = 0; pc < 8; ++pc) {
-                        const uint32_t o = h * kHalf + r * 128 + ((pc ^ (r & 7)) << 4);
-                        cp_async16(dk + o, kbase + off + h * 64 + pc * 8, valid);
-                        cp_async16(dv + o, vbase + off + h * 64 + pc * 8, valid);
-                    }
+                const uint32_t o = half_off + r * 128 + ((pc ^ (r & 7)) << 4);
+                cp_async16(dk + o, kbase + off, valid);
+                cp_async16(dv + o, vbase + off, valid);
             }
             cp_async_commit();
             // signal chunk t as soon as it has landed (made visible to the tensor core):
