@@ -217,6 +217,20 @@ int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const v
                      float* sup_score, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * tam_indexer_topk over a packed batch (layout in the header comment, "Packed
+ * batches"): q_idx, k_idx [T, d_idx]; each sequence selects among its own keys;
+ * sup_* hold sum_s n_sel(N_s) rows with positions local to the sequence.  The
+ * workspace query returns the largest single-sequence size (0 for rejected
+ * arguments); ws_bytes must reach the largest sequence's tam_indexer_workspace_min.
+ */
+size_t tam_indexer_workspace_varlen(int n_seq, const int64_t* cu_seqlens, int d_idx, int dtype,
+                                    int budget_k, int block_q);
+int tam_indexer_topk_varlen(int n_seq, const int64_t* cu_seqlens, int d_idx, int dtype,
+                            const void* q_idx, const void* k_idx, int budget_k, int block_q,
+                            int32_t* sup_idx, int32_t* sup_len, float* sup_score, void* workspace,
+                            size_t ws_bytes, void* stream);
+
+/*
  * The indexer's distillation target (technical report §2.2, "Trainingsziel": the
  * head-collapsed indexer is trained by KL divergence from the dense attention-mass
  * distribution), per query, without returning the N x N distributions:
@@ -264,6 +278,19 @@ int tam_sparse_support_attention(int64_t N, int Hq, int Hkv, int d, int dtype, c
                                  const void* k, const void* v, const int32_t* sup_idx,
                                  const int32_t* sup_len, int kmax, int block_q, void* out,
                                  float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * tam_sparse_support_attention over a packed batch (layout in the header comment,
+ * "Packed batches"): the support rows of sequence s (positions local to it) start at
+ * row sum_{s'<s} n_sel(N_s'), as tam_mass_oracle_prefill_varlen and
+ * tam_indexer_topk_varlen write them.  Workspace: tam_sparse_attention_workspace bytes.
+ */
+int tam_sparse_support_attention_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv,
+                                        int d, int dtype, const void* q, const void* k,
+                                        const void* v, const int32_t* sup_idx,
+                                        const int32_t* sup_len, int kmax, int block_q, void* out,
+                                        float* lse, void* workspace, size_t ws_bytes,
+                                        void* stream);
 
 /*
  * Dense causal GQA prefill (the FlashAttention-2 comparator the abstract measures

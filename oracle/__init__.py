@@ -354,3 +354,22 @@ def varlen_attn(q, k, v, cu_seqlens, sup=None, sup_len=None, block_q: int = 1):
         out[t0:t1], lse[t0:t1] = o, l
         sel0 += n_sel
     return out, lse
+
+
+def varlen_indexer_support(q_idx, k_idx, cu_seqlens, budget: int, block_q: int = 1):
+    """Indexer support of every sequence of a packed batch (per query, or block-shared
+    over block_q queries), rows packed in sequence order, key indices local:
+    (idx [n_sel, k] int32 ascending, -1 pad; len [n_sel]; value [n_sel, k] fp64)."""
+    qx, kx = _f32(q_idx), _f32(k_idx)
+    parts = []
+    for t0, t1 in seq_slices(cu_seqlens):
+        if t1 == t0:
+            continue
+        if block_q == 1:
+            parts.append(indexer_topk_rows(qx[t0:t1], kx[t0:t1], budget))
+        else:
+            parts.append(indexer_block_topk(qx[t0:t1], kx[t0:t1], block_q, budget))
+    if not parts:
+        return (np.zeros((0, budget), np.int32), np.zeros(0, np.int32),
+                np.zeros((0, budget), np.float64))
+    return tuple(np.concatenate([p[c] for p in parts]) for c in range(3))

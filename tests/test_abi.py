@@ -162,3 +162,30 @@ def test_varlen_and_head_dim_host_checks(tam_lib):
     # head dim 256 is accepted by the single-sequence queries too
     assert L.tam_mass_oracle_workspace(4096, 32, 8, 256, T.TAM_BF16, 256, 1) > 0
     assert L.tam_dense_workspace(4096, 32, 8, 256, T.TAM_F32) > 0
+
+
+def test_varlen_indexer_and_pass3_host_checks(tam_lib):
+    import numpy as np
+    L = tam_lib.lib()
+    T = tam_lib
+    f = _fake()
+    good = np.array([0, 64, 64, 4096], np.int64)
+    gp = good.ctypes.data_as(ctypes.c_void_p)
+    assert L.tam_indexer_workspace_varlen(3, gp, 64, T.TAM_BF16, 1024, 1) == \
+        L.tam_indexer_workspace(4032, 64, T.TAM_BF16, 1024, 1)
+    assert L.tam_indexer_workspace_varlen(3, gp, 40, T.TAM_BF16, 1024, 1) == 0
+    bad = np.array([0, 50, 40], np.int64)
+    bp = bad.ctypes.data_as(ctypes.c_void_p)
+    assert L.tam_indexer_workspace_varlen(2, bp, 64, T.TAM_BF16, 8, 1) == 0
+    assert L.tam_indexer_topk_varlen(2, bp, 64, 0, f, f, 8, 1, f, f, f, f, 1 << 30,
+                                     None) == T.TAM_ERR_INVALID_ARG
+    assert L.tam_indexer_topk_varlen(3, gp, 32, 0, f, f, 8, 2, f, f, f, f, 1 << 30,
+                                     None) == T.TAM_ERR_UNSUPPORTED       # block-shared: d_idx 64/128
+    assert L.tam_indexer_topk_varlen(3, gp, 64, 0, f, f, 8, 1, f, f, f, f, 64,
+                                     None) == T.TAM_ERR_WORKSPACE
+    assert L.tam_sparse_support_attention_varlen(2, bp, 32, 8, 128, 0, f, f, f, f, f, 8, 1, f, None,
+                                                 f, 1 << 20, None) == T.TAM_ERR_INVALID_ARG
+    assert L.tam_sparse_support_attention_varlen(3, gp, 32, 8, 128, 0, f, f, f, None, f, 8, 1, f,
+                                                 None, f, 1 << 20, None) == T.TAM_ERR_INVALID_ARG
+    assert L.tam_sparse_support_attention_varlen(3, gp, 32, 8, 128, 0, f, f, f, f, f, 8, 1, f, None,
+                                                 f, 16, None) == T.TAM_ERR_WORKSPACE

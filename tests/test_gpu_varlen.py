@@ -112,6 +112,49 @@ def test_varlen_rejects_bad_offsets(tam_lib):
         tam_lib.mass_oracle_prefill_varlen(q, k, v, [0, 63], 8)      # does not cover the tokens
 
 
+@pytest.mark.parametrize("cu,dx,kb,bq", [([0, 1, 130, 130, 393, 457, 1000], 64, 32, 1),
+                                         ([0, 1, 130, 130, 393, 457, 1000], 64, 24, 64),
+                                         ([0, 300, 301, 700], 32, 16, 1)])
+def test_indexer_varlen(tam_lib, oracle_mod, cu, dx, kb, bq):
+    """Indexer support over a packed batch: each sequence against the oracle on its
+    slice and bit for bit against the single-sequence call; then pass 3 on it."""
+    inp = _inputs(cu[-1], 8, 2, 128, "bf16", seed=cu[-1] + bq, sink=True)
+    qx, kx = tam_synth.indexer_projections(inp, dx, seed=2)
+    res = tam_lib.indexer_topk_varlen(qx.cuda(), kx.cuda(), cu, kb, bq)
+    gi, gl, gv = res.idx.cpu().numpy(), res.length.cpu().numpy(), res.value.cpu().numpy()
+    sel = tam_lib.selection_offsets(cu, bq).numpy()
+    assert gi.shape[0] == sel[-1]
+    for s in range(len(cu) - 1):
+        t0, t1 = cu[s], cu[s + 1]
+        if t1 == t0:
+            continue
+        r0, r1 = sel[s], sel[s + 1]
+        one = tam_lib.indexer_topk(qx[t0:t1].cuda(), kx[t0:t1].cuda(), kb, bq)
+        assert torch.equal(one.idx.cpu(), res.idx[r0:r1].cpu())
+        assert torch.equal(one.value.cpu(), res.value[r0:r1].cpu())
+        if bq == 1:
+            oi, ol, _ = oracle_mod.indexer_topk_rows(qx[t0:t1], kx[t0:t1], kb)
+            S = qx[t0:t1].double().numpy() @ kx[t0:t1].double().numpy().T
+            check_support(gi[r0:r1], gl[r0:r1], gv[r0:r1], oi, ol, S, 1e-3, f"indexer seq {s}")
+        else:
+            oi, ol, _ = oracle_mod.indexer_block_topk(qx[t0:t1], kx[t0:t1], bq, kb)
+            M = oracle_mod.indexer_block_mass(qx[t0:t1], kx[t0:t1], bq)
+            check_support(gi[r0:r1], gl[r0:r1], gv[r0:r1], oi, ol, M, MASS_ATOL * bq,
+                          f"indexer block seq {s}")
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    out = tam_lib.sparse_support_attention_varlen(q, k, v, res.idx, res.length, cu, bq)
+    ref, _ = oracle_mod.varlen_attn(inp.q, inp.k, inp.v, cu, sup=gi, sup_len=gl, block_q=bq)
+    check_close(out.float().cpu().numpy(), ref, OUT_ATOL["bf16"], "varlen pass 3 on indexer")
+    for s in range(len(cu) - 1):
+        t0, t1 = cu[s], cu[s + 1]
+        if t1 > t0:
+            # (copies: a slice of the lengths need not start on a 16-byte boundary)
+            one = tam_lib.sparse_support_attention(q[t0:t1], k[t0:t1], v[t0:t1],
+                                                   res.idx[sel[s]:sel[s + 1]].clone(),
+                                                   res.length[sel[s]:sel[s + 1]].clone(), bq)
+            assert torch.equal(one, out[t0:t1])
+
+
 # ---------------------------------------------------------------- head dim 256
 
 @pytest.mark.parametrize("N,Hq,Hkv,dtype,kb,bq", [(200, 4, 1, "f32", 8, 1),

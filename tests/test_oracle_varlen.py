@@ -137,3 +137,50 @@ def test_packed_sparse_attention_on_support(oracle_mod, block_q):
         p = np.exp(sc - sc.max(axis=1, keepdims=True))
         p /= p.sum(axis=1, keepdims=True)
         np.testing.assert_allclose(out[i], np.einsum("hj,jhc->hc", p, vh[keys]), atol=1e-12)
+
+
+def _brute_indexer_scores(qx, kx, cu):
+    s = qx.astype(np.float64) @ kx.astype(np.float64).T
+    _, allowed = _mask(cu)
+    return np.where(allowed, s, -np.inf), allowed
+
+
+@pytest.mark.parametrize("budget", [1, 4, 9])
+def test_packed_indexer_per_query(oracle_mod, budget):
+    rng = np.random.default_rng(21)
+    T = CU[-1]
+    qx = rng.standard_normal((T, 16)).astype(np.float32)
+    kx = rng.standard_normal((T, 16)).astype(np.float32)
+    idx, ln, val = oracle_mod.varlen_indexer_support(qx, kx, CU, budget)
+    s, allowed = _brute_indexer_scores(qx, kx, CU)
+    seq, _ = _mask(CU)
+    cu = np.asarray(CU)
+    for i in range(T):
+        t0 = cu[seq[i]]
+        want = [j - t0 for j in _rank_select(s[i], list(np.nonzero(allowed[i])[0]), budget)]
+        assert ln[i] == min(budget, i - t0 + 1)
+        assert list(idx[i, :ln[i]]) == want, i
+        np.testing.assert_allclose(val[i, :ln[i]], s[i, np.array(want) + t0], atol=1e-9)
+
+
+@pytest.mark.parametrize("budget,block_q", [(3, 4), (5, 8)])
+def test_packed_indexer_block(oracle_mod, budget, block_q):
+    rng = np.random.default_rng(22)
+    T = CU[-1]
+    qx = rng.standard_normal((T, 16)).astype(np.float32)
+    kx = rng.standard_normal((T, 16)).astype(np.float32)
+    idx, ln, val = oracle_mod.varlen_indexer_support(qx, kx, CU, budget, block_q)
+    s, _ = _brute_indexer_scores(qx, kx, CU)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)               # per-query softmax over visible keys
+    row = 0
+    for t0, t1 in zip(CU[:-1], CU[1:]):
+        for b0 in range(t0, t1, block_q):
+            e = min(t1, b0 + block_q) - 1
+            M = p[b0:e + 1].sum(axis=0)
+            want = [j - t0 for j in _rank_select(M, list(range(t0, e + 1)), budget)]
+            assert ln[row] == min(budget, e - t0 + 1)
+            assert list(idx[row, :ln[row]]) == want, (t0, b0)
+            np.testing.assert_allclose(val[row, :ln[row]], M[np.array(want) + t0], atol=1e-12)
+            row += 1
+    assert row == idx.shape[0]

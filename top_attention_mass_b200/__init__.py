@@ -14,7 +14,8 @@ Functions (same names as the C entry points, without the ``tam_`` prefix):
 * ``indexer_topk``             head-collapsed indexer support
 * ``sparse_support_attention`` pass 3 alone (attention on a given support)
 * ``dense_gqa_prefill``        dense causal GQA attention (comparator)
-* ``mass_oracle_prefill_varlen``, ``dense_gqa_prefill_varlen``
+* ``mass_oracle_prefill_varlen``, ``dense_gqa_prefill_varlen``, ``indexer_topk_varlen``,
+  ``sparse_support_attention_varlen``
                                the same over a packed batch of sequences
 
 Inputs may be CUDA tensors, or CPU tensors (ideally pinned): then they are
@@ -46,7 +47,8 @@ EXPORTED = (
     "tam_support_mass_curve", "tam_sparse_attention_workspace", "tam_sparse_support_attention",
     "tam_dense_workspace", "tam_dense_gqa_prefill", "tam_kernel_launches", "tam_check_status",
     "tam_mass_oracle_workspace_varlen", "tam_mass_oracle_prefill_varlen",
-    "tam_dense_gqa_prefill_varlen",
+    "tam_dense_gqa_prefill_varlen", "tam_indexer_workspace_varlen", "tam_indexer_topk_varlen",
+    "tam_sparse_support_attention_varlen",
 )
 
 
@@ -128,6 +130,13 @@ def lib() -> ctypes.CDLL:
         L.tam_dense_gqa_prefill_varlen.restype = i32
         L.tam_dense_gqa_prefill_varlen.argtypes = [i32, p, i32, i32, i32, i32, p, p, p, p, p, p,
                                                    sz, p]
+        L.tam_indexer_workspace_varlen.restype = sz
+        L.tam_indexer_workspace_varlen.argtypes = [i32, p, i32, i32, i32, i32]
+        L.tam_indexer_topk_varlen.restype = i32
+        L.tam_indexer_topk_varlen.argtypes = [i32, p, i32, i32, p, p, i32, i32, p, p, p, p, sz, p]
+        L.tam_sparse_support_attention_varlen.restype = i32
+        L.tam_sparse_support_attention_varlen.argtypes = [i32, p, i32, i32, i32, i32, p, p, p, p, p,
+                                                          i32, i32, p, p, p, sz, p]
         L.tam_kernel_launches.restype = ctypes.c_uint64
         L.tam_check_status.restype = i32
         L.tam_check_status.argtypes = [p, p, p]
@@ -560,6 +569,75 @@ def dense_gqa_prefill_varlen(q, k, v, cu_seqlens, *, return_lse: bool = False,
                                         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(ws),
                                         ws.numel(), _stream(dev, stream))
     _raise(rc, "dense_gqa_prefill_varlen")
+    if check:
+        check_status(ws, stream)
+    if host:
+        out = out.cpu()
+        lse = None if lse is None else lse.cpu()
+    return (out, lse) if return_lse else out
+
+
+def indexer_topk_varlen(q_idx, k_idx, cu_seqlens, budget_k: int, block_q: int = 1, *,
+                        workspace: Optional[Workspace] = None, stream=None, check: bool = True,
+                        device=None) -> Support:
+    """indexer_topk over a packed batch: q_idx, k_idx [T, d_idx]; support rows packed in
+    sequence order (see ``selection_offsets``), positions local to each sequence."""
+    cu = _cu_host(cu_seqlens)
+    n_seq = cu.numel() - 1
+    dev = _dev_of(q_idx, device)
+    (q_idx, k_idx), host = _to_device([q_idx, k_idx], dev)
+    if q_idx.dim() != 2 or k_idx.shape != q_idx.shape or k_idx.dtype != q_idx.dtype:
+        raise ValueError("q_idx and k_idx are [T, d_idx] of one dtype")
+    T, dx = q_idx.shape
+    if int(cu[-1]) != T:
+        raise ValueError("cu_seqlens[-1] must equal the packed token count")
+    dt = _dtype_code(q_idx)
+    n_sel = int(selection_offsets(cu, block_q)[-1])
+    sup_idx = torch.empty(n_sel, budget_k, dtype=torch.int32, device=dev)
+    sup_len = torch.empty(n_sel, dtype=torch.int32, device=dev)
+    sup_score = torch.empty(n_sel, budget_k, dtype=torch.float32, device=dev)
+    L = lib()
+    cu_p = ctypes.c_void_p(cu.data_ptr())
+    nbytes = L.tam_indexer_workspace_varlen(n_seq, cu_p, dx, dt, budget_k, block_q)
+    ws = _workspace(dev, max(nbytes, 256), workspace)
+    rc = L.tam_indexer_topk_varlen(n_seq, cu_p, dx, dt, _ptr(q_idx), _ptr(k_idx), budget_k,
+                                   block_q, _ptr(sup_idx), _ptr(sup_len), _ptr(sup_score),
+                                   _ptr(ws), ws.numel() if nbytes else 0, _stream(dev, stream))
+    _raise(rc, "indexer_topk_varlen")
+    if check:
+        check_status(ws, stream)
+    res = Support(sup_idx, sup_len, sup_score)
+    if host:
+        res = Support(res.idx.cpu(), res.length.cpu(), res.value.cpu())
+    return res
+
+
+def sparse_support_attention_varlen(q, k, v, sup_idx, sup_len, cu_seqlens, block_q: int = 1, *,
+                                    return_lse: bool = False,
+                                    workspace: Optional[Workspace] = None, stream=None,
+                                    check: bool = True, device=None):
+    """sparse_support_attention over a packed batch; support rows as the varlen selection
+    calls lay them out.  Returns out [T, Hq, d] (and the flat per-sequence lse blocks)."""
+    cu = _cu_host(cu_seqlens)
+    n_seq = cu.numel() - 1
+    dev = _dev_of(q, device)
+    (q, k, v, sup_idx, sup_len), host = _to_device([q, k, v, sup_idx, sup_len], dev)
+    T, Hq, Hkv, d = _shape(q, k)
+    if int(cu[-1]) != T:
+        raise ValueError("cu_seqlens[-1] must equal the packed token count")
+    if sup_idx.dtype != torch.int32 or sup_len.dtype != torch.int32:
+        raise TypeError("sup_idx and sup_len are int32")
+    dt = _dtype_code(q)
+    out = torch.empty_like(q)
+    lse = torch.empty(Hq * T, dtype=torch.float32, device=dev) if return_lse else None
+    L = lib()
+    ws = _workspace(dev, 256, workspace)
+    rc = L.tam_sparse_support_attention_varlen(n_seq, ctypes.c_void_p(cu.data_ptr()), Hq, Hkv, d,
+                                               dt, _ptr(q), _ptr(k), _ptr(v), _ptr(sup_idx),
+                                               _ptr(sup_len), sup_idx.shape[1], block_q, _ptr(out),
+                                               _ptr(lse), _ptr(ws), ws.numel(),
+                                               _stream(dev, stream))
+    _raise(rc, "sparse_support_attention_varlen")
     if check:
         check_status(ws, stream)
     if host:

@@ -238,6 +238,70 @@ int check_cu_seqlens(int n_seq, const int64_t* cu, int64_t* max_len) {
 
 inline size_t elt_bytes(int dtype) { return dtype == TAM_F32 ? 4 : 2; }
 
+// Range checks of the indexer entry points (dtype and d_idx >= 1 checked by the caller).
+int check_indexer_args(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
+    if (d_idx != 16 && d_idx != 32 && d_idx != 64 && d_idx != 128) return TAM_ERR_UNSUPPORTED;
+    if (N >= (int64_t(1) << 31) - 1) return TAM_ERR_UNSUPPORTED;
+    int rc = check_budget(N, budget_k, block_q);
+    if (rc) return rc;
+    // block-shared: the indexer head runs as a one-head layer (tensor-core head dims)
+    if (block_q > 1) return check_shape(N, 1, 1, d_idx, dtype);
+    return TAM_OK;
+}
+
+int check_indexer_ptrs(const void* q_idx, const void* k_idx, const void* sup_idx,
+                       const void* sup_len, const void* sup_score, const void* workspace) {
+    if (!q_idx || !k_idx || !sup_idx || !sup_len || !sup_score || !workspace)
+        return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q_idx, k_idx, sup_idx, sup_len, sup_score, workspace};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
+    return TAM_OK;
+}
+
+size_t indexer_min_bytes(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
+    if (block_q > 1) return plan_mass(N, 1, 1, d_idx, dtype, budget_k, block_q).min_total;
+    return plan_indexer(N, d_idx, dtype, budget_k, block_q).min_total;
+}
+
+// Indexer support of one sequence of N tokens (arguments checked, status cleared).
+int run_indexer(int64_t N, int d_idx, int dtype, const void* q_idx, const void* k_idx,
+                int budget_k, int block_q, int32_t* sup_idx, int32_t* sup_len, float* sup_score,
+                char* ws, size_t ws_bytes, cudaStream_t st) {
+    int rc;
+    if (block_q > 1) {
+        // Block-shared: softmax of the indexer scores per query (scale 1), summed over
+        // the block, top-k of the sums: pass 1 and the block-mass pass 2 of a one-head
+        // layer whose query and key are q_idx and k_idx.
+        const MassPlan plan = plan_mass(N, 1, 1, d_idx, dtype, budget_k, block_q);
+        float* lse_buf = (float*)(ws + plan.off_lse);
+        LseArgs la{N, 1, 1, d_idx, dtype, q_idx, k_idx, kLog2e, lse_buf, (int32_t*)ws};
+        if ((rc = cuda_status(run_lse(la, st)))) return rc;
+        return launch_mass_select(N, 1, 1, d_idx, dtype, q_idx, k_idx, lse_buf, budget_k, block_q,
+                                  sup_idx, sup_len, sup_score, ws, ws_bytes, plan, st, kLog2e);
+    }
+    const IndexerPlan plan = plan_indexer(N, d_idx, dtype, budget_k, block_q);
+    IndexerArgs ia{};
+    ia.N = N; ia.d_idx = d_idx; ia.dtype = dtype; ia.q_idx = q_idx; ia.k_idx = k_idx;
+    ia.budget = budget_k; ia.n_ctas = plan.n_ctas; ia.scratch = (float*)(ws + plan.off_scratch);
+    ia.rows = (float*)(ws + plan.off_scratch);
+    ia.sup_idx = sup_idx; ia.sup_len = sup_len; ia.sup_score = sup_score;
+    ia.status = (int32_t*)ws;
+    if (!plan.tc) return cuda_status(simt_indexer_select(ia, st));
+    // score rows of a chunk of queries, then their top-k, chunk by chunk
+    const int64_t cap = (int64_t)((ws_bytes - plan.off_scratch) / sizeof(float));
+    for (int64_t r0 = 0; r0 < N;) {
+        const int64_t r1 = chunk_end(r0, N, cap);
+        ia.row0 = r0;
+        ia.row1 = r1;
+        cudaError_t e = tc_indexer_rows(ia, st);
+        if (e == cudaSuccess) e = row_topk(ia.rows, r0, r1, budget_k, sup_idx, sup_len, sup_score, st);
+        if (e != cudaSuccess) return TAM_ERR_CUDA;
+        r0 = r1;
+    }
+    return TAM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -414,53 +478,60 @@ int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const v
                      int budget_k, int block_q, int32_t* sup_idx, int32_t* sup_len,
                      float* sup_score, void* workspace, size_t ws_bytes, void* stream) {
     if (N < 1 || d_idx < 1 || (dtype != TAM_BF16 && dtype != TAM_F32)) return TAM_ERR_INVALID_ARG;
-    if (d_idx != 16 && d_idx != 32 && d_idx != 64 && d_idx != 128) return TAM_ERR_UNSUPPORTED;
-    if (N >= (int64_t(1) << 31) - 1) return TAM_ERR_UNSUPPORTED;
-    int rc = check_budget(N, budget_k, block_q);
+    int rc = check_indexer_args(N, d_idx, dtype, budget_k, block_q);
     if (rc) return rc;
-    if (!q_idx || !k_idx || !sup_idx || !sup_len || !sup_score || !workspace)
-        return TAM_ERR_INVALID_ARG;
-    const void* ptrs[] = {q_idx, k_idx, sup_idx, sup_len, sup_score, workspace};
-    for (const void* p : ptrs)
-        if (!aligned16(p)) return TAM_ERR_INVALID_ARG;
-    if (block_q > 1) {
-        // Block-shared: softmax of the indexer scores per query (scale 1), summed over
-        // the block, top-k of the sums: pass 1 and the block-mass pass 2 of a one-head
-        // layer whose query and key are q_idx and k_idx.
-        if ((rc = check_shape(N, 1, 1, d_idx, dtype))) return rc;
-        const MassPlan plan = plan_mass(N, 1, 1, d_idx, dtype, budget_k, block_q);
-        if (ws_bytes < plan.min_total) return TAM_ERR_WORKSPACE;
-        cudaStream_t st = (cudaStream_t)stream;
-        char* ws = (char*)workspace;
-        if ((rc = start_call(workspace, st))) return rc;
-        float* lse_buf = (float*)(ws + plan.off_lse);
-        LseArgs la{N, 1, 1, d_idx, dtype, q_idx, k_idx, kLog2e, lse_buf, (int32_t*)ws};
-        if ((rc = cuda_status(run_lse(la, st)))) return rc;
-        return launch_mass_select(N, 1, 1, d_idx, dtype, q_idx, k_idx, lse_buf, budget_k, block_q,
-                                  sup_idx, sup_len, sup_score, ws, ws_bytes, plan, st, kLog2e);
-    }
-    const IndexerPlan plan = plan_indexer(N, d_idx, dtype, budget_k, block_q);
-    if (ws_bytes < plan.min_total) return TAM_ERR_WORKSPACE;
+    if ((rc = check_indexer_ptrs(q_idx, k_idx, sup_idx, sup_len, sup_score, workspace))) return rc;
+    if (ws_bytes < indexer_min_bytes(N, d_idx, dtype, budget_k, block_q)) return TAM_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
-    char* ws = (char*)workspace;
     if ((rc = start_call(workspace, st))) return rc;
-    IndexerArgs ia{};
-    ia.N = N; ia.d_idx = d_idx; ia.dtype = dtype; ia.q_idx = q_idx; ia.k_idx = k_idx;
-    ia.budget = budget_k; ia.n_ctas = plan.n_ctas; ia.scratch = (float*)(ws + plan.off_scratch);
-    ia.rows = (float*)(ws + plan.off_scratch);
-    ia.sup_idx = sup_idx; ia.sup_len = sup_len; ia.sup_score = sup_score;
-    ia.status = (int32_t*)ws;
-    if (!plan.tc) return cuda_status(simt_indexer_select(ia, st));
-    // score rows of a chunk of queries, then their top-k, chunk by chunk
-    const int64_t cap = (int64_t)((ws_bytes - plan.off_scratch) / sizeof(float));
-    for (int64_t r0 = 0; r0 < N;) {
-        const int64_t r1 = chunk_end(r0, N, cap);
-        ia.row0 = r0;
-        ia.row1 = r1;
-        cudaError_t e = tc_indexer_rows(ia, st);
-        if (e == cudaSuccess) e = row_topk(ia.rows, r0, r1, budget_k, sup_idx, sup_len, sup_score, st);
-        if (e != cudaSuccess) return TAM_ERR_CUDA;
-        r0 = r1;
+    return run_indexer(N, d_idx, dtype, q_idx, k_idx, budget_k, block_q, sup_idx, sup_len,
+                       sup_score, (char*)workspace, ws_bytes, st);
+}
+
+size_t tam_indexer_workspace_varlen(int n_seq, const int64_t* cu_seqlens, int d_idx, int dtype,
+                                    int budget_k, int block_q) {
+    int64_t max_len = 0;
+    if (check_cu_seqlens(n_seq, cu_seqlens, &max_len) != TAM_OK) return 0;
+    if (d_idx < 1 || (dtype != TAM_BF16 && dtype != TAM_F32)) return 0;
+    if (check_indexer_args(std::max<int64_t>(max_len, 1), d_idx, dtype, budget_k, block_q)) return 0;
+    size_t total = kStatusBytes;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t n = cu_seqlens[s + 1] - cu_seqlens[s];
+        if (n > 0) total = std::max(total, tam_indexer_workspace(n, d_idx, dtype, budget_k, block_q));
+    }
+    return total;
+}
+
+int tam_indexer_topk_varlen(int n_seq, const int64_t* cu_seqlens, int d_idx, int dtype,
+                            const void* q_idx, const void* k_idx, int budget_k, int block_q,
+                            int32_t* sup_idx, int32_t* sup_len, float* sup_score, void* workspace,
+                            size_t ws_bytes, void* stream) {
+    int64_t max_len = 0;
+    int rc = check_cu_seqlens(n_seq, cu_seqlens, &max_len);
+    if (rc) return rc;
+    if (d_idx < 1 || (dtype != TAM_BF16 && dtype != TAM_F32)) return TAM_ERR_INVALID_ARG;
+    if ((rc = check_indexer_args(std::max<int64_t>(max_len, 1), d_idx, dtype, budget_k, block_q)))
+        return rc;
+    if ((rc = check_indexer_ptrs(q_idx, k_idx, sup_idx, sup_len, sup_score, workspace))) return rc;
+    if (ws_bytes < kStatusBytes) return TAM_ERR_WORKSPACE;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t n = cu_seqlens[s + 1] - cu_seqlens[s];
+        if (n > 0 && ws_bytes < indexer_min_bytes(n, d_idx, dtype, budget_k, block_q))
+            return TAM_ERR_WORKSPACE;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((rc = start_call(workspace, st))) return rc;
+    const size_t row = (size_t)d_idx * elt_bytes(dtype);
+    int64_t sel0 = 0;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t t0 = cu_seqlens[s], n = cu_seqlens[s + 1] - t0;
+        if (n == 0) continue;
+        rc = run_indexer(n, d_idx, dtype, (const char*)q_idx + t0 * row,
+                         (const char*)k_idx + t0 * row, budget_k, block_q,
+                         sup_idx + sel0 * budget_k, sup_len + sel0, sup_score + sel0 * budget_k,
+                         (char*)workspace, ws_bytes, st);
+        if (rc) return rc;
+        sel0 += n_selection_units(n, block_q);
     }
     return TAM_OK;
 }
@@ -574,6 +645,39 @@ int tam_sparse_support_attention(int64_t N, int Hq, int Hkv, int d, int dtype, c
     AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, score_log2_scale(d), sup_idx, sup_len, kmax,
                 block_q, out, lse, (int32_t*)workspace};
     return cuda_status(run_sparse_attention(aa, st));
+}
+
+int tam_sparse_support_attention_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv,
+                                        int d, int dtype, const void* q, const void* k,
+                                        const void* v, const int32_t* sup_idx,
+                                        const int32_t* sup_len, int kmax, int block_q, void* out,
+                                        float* lse, void* workspace, size_t ws_bytes,
+                                        void* stream) {
+    int64_t max_len = 0;
+    int rc = check_cu_seqlens(n_seq, cu_seqlens, &max_len);
+    if (rc) return rc;
+    if ((rc = check_shape(std::max<int64_t>(max_len, 1), Hq, Hkv, d, dtype))) return rc;
+    if ((rc = check_budget(std::max<int64_t>(max_len, 1), kmax, block_q))) return rc;
+    if (!q || !k || !v || !sup_idx || !sup_len || !out || !workspace) return TAM_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, sup_idx, sup_len, out, lse, workspace};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return TAM_ERR_INVALID_ARG;
+    if (ws_bytes < kStatusBytes) return TAM_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((rc = start_call(workspace, st))) return rc;
+    const size_t qrow = (size_t)Hq * d * elt_bytes(dtype), krow = (size_t)Hkv * d * elt_bytes(dtype);
+    int64_t sel0 = 0;
+    for (int s = 0; s < n_seq; ++s) {
+        const int64_t t0 = cu_seqlens[s], n = cu_seqlens[s + 1] - t0;
+        if (n == 0) continue;
+        AttnArgs aa{n, Hq, Hkv, d, dtype, (const char*)q + t0 * qrow, (const char*)k + t0 * krow,
+                    (const char*)v + t0 * krow, score_log2_scale(d), sup_idx + sel0 * kmax,
+                    sup_len + sel0, kmax, block_q, (char*)out + t0 * qrow,
+                    lse ? lse + (size_t)Hq * t0 : nullptr, (int32_t*)workspace};
+        if ((rc = cuda_status(run_sparse_attention(aa, st)))) return rc;
+        sel0 += n_selection_units(n, block_q);
+    }
+    return TAM_OK;
 }
 
 size_t tam_dense_workspace(int64_t N, int Hq, int Hkv, int d, int dtype) {
