@@ -189,3 +189,21 @@ def test_varlen_indexer_and_pass3_host_checks(tam_lib):
                                                  None, f, 1 << 20, None) == T.TAM_ERR_INVALID_ARG
     assert L.tam_sparse_support_attention_varlen(3, gp, 32, 8, 128, 0, f, f, f, f, f, 8, 1, f, None,
                                                  f, 16, None) == T.TAM_ERR_WORKSPACE
+
+
+def test_packed_batch_helpers():
+    """Host-side helpers of the varlen binding (no device involved)."""
+    import torch
+    import top_attention_mass_b200 as tam
+    cu = [0, 1, 130, 130, 393]
+    assert tam.selection_offsets(cu, 1).tolist() == [0, 1, 130, 130, 393]
+    # blocks of 64: 1 -> 1, 129 -> 3, 0 -> 0, 263 -> 5
+    assert tam.selection_offsets(cu, 64).tolist() == [0, 1, 4, 4, 9]
+    Hq = 3
+    flat = torch.arange(Hq * 393, dtype=torch.float32)
+    blk = tam.lse_block(flat, cu, 3)
+    assert blk.shape == (Hq, 263)
+    assert blk[0, 0].item() == Hq * 130 and blk[2, 262].item() == Hq * 393 - 1
+    assert tam.lse_block(flat, cu, 2).shape == (Hq, 0)
+    with pytest.raises(ValueError):
+        tam.selection_offsets([0], 1)
