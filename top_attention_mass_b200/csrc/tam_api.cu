@@ -457,21 +457,16 @@ int tam_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
 }
 
 size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
-    if (N < 1 || (d_idx != 16 && d_idx != 32 && d_idx != 64 && d_idx != 128)) return 0;
-    if (dtype != TAM_BF16 && dtype != TAM_F32) return 0;
-    if (check_budget(N, budget_k, block_q) != TAM_OK) return 0;
-    if (block_q > 1) {
-        // block-shared: the indexer head as a one-head layer (lse, block mass)
-        if (check_shape(N, 1, 1, d_idx, dtype) != TAM_OK) return 0;
-        return plan_mass(N, 1, 1, d_idx, dtype, budget_k, block_q).total;
-    }
+    if (N < 1 || d_idx < 1 || (dtype != TAM_BF16 && dtype != TAM_F32)) return 0;
+    if (check_indexer_args(N, d_idx, dtype, budget_k, block_q) != TAM_OK) return 0;
+    // block-shared: the indexer head as a one-head layer (lse, block mass)
+    if (block_q > 1) return plan_mass(N, 1, 1, d_idx, dtype, budget_k, block_q).total;
     return plan_indexer(N, d_idx, dtype, budget_k, block_q).total;
 }
 
 size_t tam_indexer_workspace_min(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
     if (tam_indexer_workspace(N, d_idx, dtype, budget_k, block_q) == 0) return 0;
-    if (block_q > 1) return plan_mass(N, 1, 1, d_idx, dtype, budget_k, block_q).min_total;
-    return plan_indexer(N, d_idx, dtype, budget_k, block_q).min_total;
+    return indexer_min_bytes(N, d_idx, dtype, budget_k, block_q);
 }
 
 int tam_indexer_topk(int64_t N, int d_idx, int dtype, const void* q_idx, const void* k_idx,
