@@ -38,6 +38,16 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def build_selftest(out_dir: str) -> str:
+    """Compile the stand-alone C++ self-test (selftest.cpp + oracle.cpp) into out_dir."""
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "oracle_selftest")
+    cmd = ["g++", "-O2", "-std=c++17", "-fopenmp", os.path.join(_HERE, "selftest.cpp"), _SRC,
+           "-o", exe]
+    subprocess.run(cmd, check=True)
+    return exe
+
+
 def lib():
     global _lib
     with _lock:

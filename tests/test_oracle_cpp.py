@@ -2,16 +2,12 @@
 against oracle.cpp and run as a binary: direct evaluation of the mass, the
 support rule, nesting and monotonicity in k, block of one, k >= i+1 = dense, and
 the Q = 0 closed form."""
-import os
 import subprocess
-
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_oracle_selftest_binary(tmp_path):
-    exe = str(tmp_path / "oracle_selftest")
-    src = [os.path.join(ROOT, "oracle", "selftest.cpp"), os.path.join(ROOT, "oracle", "oracle.cpp")]
-    subprocess.run(["g++", "-O2", "-std=c++17", "-fopenmp", *src, "-o", exe], check=True)
+    import oracle
+    exe = oracle.build_selftest(str(tmp_path))
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "all passed" in r.stdout
