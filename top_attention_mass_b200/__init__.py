@@ -180,7 +180,12 @@ def _stream(device: torch.device, stream=None):
 
 
 class Workspace:
-    """A reusable device workspace (uint8 tensor) that grows on demand."""
+    """A reusable device workspace (uint8 tensor) that grows on demand.
+
+    A call that gets no workspace uses one default workspace per device.  Calls are
+    ordered on their stream, so that is safe for one stream at a time; calls that run
+    concurrently on several streams need one Workspace each (the status block and the
+    scratch would otherwise be shared)."""
 
     def __init__(self, device=None):
         self.device = torch.device(device or "cuda")
