@@ -207,3 +207,21 @@ def test_packed_batch_helpers():
     assert tam.lse_block(flat, cu, 2).shape == (Hq, 0)
     with pytest.raises(ValueError):
         tam.selection_offsets([0], 1)
+
+
+@pytest.mark.parametrize("N", [1, 64, 65, 1000, 4096, 32768, 65536])
+def test_workspace_sizes_follow_the_documented_layout(tam_lib, N):
+    """Per query on the tensor cores: status block (256 B), lse (Hq*N floats), then the
+    row slab -- every row i (i+1 floats) up to 4 GiB preferred, 64 rows of N floats at
+    least (both capped by the whole triangle)."""
+    L = tam_lib.lib()
+    Hq, Hkv, d, k = 32, 8, 128, 16
+    a256 = lambda x: (x + 255) // 256 * 256              # noqa: E731
+    tri = N * (N + 1) // 2
+    head = 256 + a256(Hq * N * 4)
+    pref = L.tam_mass_oracle_workspace(N, Hq, Hkv, d, tam_lib.TAM_BF16, k, 1)
+    lo = L.tam_mass_workspace_min(N, Hq, Hkv, d, tam_lib.TAM_BF16, k, 1)
+    assert pref == head + a256(min(4 << 30, tri * 4))
+    assert lo == head + a256(min(tri, 64 * N) * 4)
+    # the mass-select and no-lse variants share the layout
+    assert L.tam_mass_select_workspace(N, Hq, Hkv, d, tam_lib.TAM_BF16, k, 1) == pref
