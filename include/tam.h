@@ -180,14 +180,17 @@ int tam_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
  * Same arguments, semantics and outputs as tam_mass_select, minus the workspace:
  * the scratch is a 64 MiB static device array inside the library.  Problems whose
  * tam_mass_workspace_min() exceeds 64 MiB are rejected with TAM_ERR_WORKSPACE
- * before anything is enqueued; per query, 64 MiB below the preferred size only
- * means that the mass rows go through in more chunks.  Nothing is allocated.  The first call on a device
- * looks up the array's device address (with that device current), so make that
- * first call before any stream capture.  The call waits for `stream` and returns
- * the device status (TAM_OK or TAM_ERR_TIMEOUT).  All calls in the
- * process share the one array per device and it keeps the last call's contents:
- * calls that can overlap on the GPU (other streams, other threads) race and must
- * be serialised by the caller.  A GPU keeps the array until the process exits.
+ * before anything is enqueued; a problem whose preferred workspace is larger than
+ * 64 MiB but whose minimum fits runs in more chunks.  Nothing is allocated.  Every
+ * call looks up the array's device address on the current device (a host-side
+ * query), so the call works again after the context is torn down and re-created.
+ * The call blocks: it waits for `stream` and returns the device status (TAM_OK or
+ * TAM_ERR_TIMEOUT), so it cannot be used inside a stream capture.  All calls in
+ * the process share the one array per device and it keeps the last call's
+ * contents: calls that can overlap on the GPU (other streams, other threads) race
+ * and must be serialised by the caller.  The 64 MiB are reserved on every device
+ * where the library's module is loaded, whether or not this call is used, and are
+ * held until the process exits.
  */
 int tam_mass_select_noalloc(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q,
                             const void* k, const float* lse, int budget_k, int block_q,

@@ -10,40 +10,30 @@
 // and output buffer; nothing here calls cudaMalloc, cudaFree or any allocating
 // library routine.
 //
-// The array is ordinary module memory: a GPU on which it has been used keeps it
-// until the process exits.  In host code its name is only a host-side stand-in,
-// so its device address is looked up once per device with cudaGetSymbolAddress
-// (on the first call on that device, with that device current) and that address
-// is what the kernels receive.
+// The array is ordinary module memory: it is reserved on a device whenever the
+// library's module is loaded there (at the first launch of any of its kernels
+// under lazy loading, at context creation under eager loading), whether or not
+// this entry point is ever called, and the device keeps it until the process
+// exits.  In host code its name is only a host-side stand-in, so every call looks
+// up its device address with cudaGetSymbolAddress, with the caller's device
+// current, and that address is what the kernels receive.  Nothing is cached: a
+// torn-down and re-created context (cudaDeviceReset) may load the module at
+// another address, and a cached pointer would then point at unmapped memory.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "../../include/tam.h"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(64) << 20;   // 64 MiB per device
-constexpr int kMaxDevices = 64;
-
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the static scratch on the current device; looked up once per
-// device.  Returns null if the device index is out of range or the lookup fails.
+// Device address of the static scratch on the current device, or null if the
+// lookup fails.  The lookup is a host-side query (no stream work).
 void* scratch_for_current_device() {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
-            return nullptr;
-        g_scratch_addr[dev] = p;
-    }
-    return g_scratch_addr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+    return p;
 }
 
 }  // namespace
