@@ -2,22 +2,33 @@
 """Benchmark of the attention-mass top-k path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
 
-One step = one pass of every step of the hot path over one layer of the 32K
-workload (N=32768, Hq=32, Hkv=8, d=128, bf16; sink at token 0, 64 planted
-needles):
-  pass 1  per-head LSE                            (attention_lse)
-  pass 2  mass + per-query top-k, k=655           (mass_select, block_q=1)
-  pass 3  per-query gathered sparse attention     (sparse_support_attention)
-  pass 2  mass + block-shared top-k, B_q=64       (mass_select, block_q=64)
-  pass 3  block-shared sparse attention           (sparse_support_attention)
-  indexer top-k, d_idx=64, k=1024                 (indexer_topk)
-  pass 3  on the indexer support                  (sparse_support_attention)
-  dense causal GQA prefill (comparator)           (dense_gqa_prefill)
-value = query tokens of all ranks / step time (max over ranks).  With N > 1 GPUs
-every rank runs an independent replica of the workload (weak scaling, no
-collective on the data path).  `--impl reference` times the fp64 CPU oracle on a
-bounded sample of the same workload instead (rank 0 only).
+The step (what `value` measures) is one call of the attention-mass oracle,
+tam_mass_oracle_prefill, on one causal GQA prefill layer of the 32K workload
+(N=32768, Hq=32, Hkv=8, d=128, bf16; sink at token 0, 64 planted needles) with
+per-query support k=655: pass 1 (per-head LSE), pass 2 (head-averaged mass and its
+top-k, streamed) and pass 3 (the sparse recompute on the support: the gathered
+sparse attention).  value = query tokens of all ranks / step time (max over
+ranks), i.e. the metric "query-tokens/s per GQA layer (mass oracle, sparse pass)".
+
+Reported beside it (not part of value):
+  rows            each pass of the step timed on its own entry point, with its roofline
+                  (roofline = the longest of them);
+  block_shared    the same call with block-shared support (B_q = 64), and its passes;
+  all_rows_step   every row of the hot path in one CUDA graph: both oracles, the
+                  indexer top-k (d_idx = 64, k = 1024) and pass 3 on its support, the
+                  dense comparator;
+  gather_out_of_l2  per-query pass 3 on a 262144-token layer whose K/V halves are four
+                  times the L2 (random support, k = 2048), against HBM;
+  support_quality the indexer's support against the mass oracle's at k = 1024
+                  (recall@k, output difference), outputs against dense;
+  next_rows       the fused block-shared indexer, the distillation target, the budget
+                  sweep and a packed batch of eight sequences.
+With N > 1 GPUs every rank runs an independent replica of the workload (weak
+scaling, no collective on the data path).  `--impl reference` times the fp64 CPU
+oracle on a bounded sample of the step instead (rank 0 only).  `--workload` runs
+another configuration (gqa4k_needles, longctx_<N>, indexer32k) as the step.
 """
 from __future__ import annotations
 
@@ -49,6 +60,13 @@ D_IDX = 64
 # packed batch of mixed lengths (sums to the 32K workload's token count)
 VARLEN_SEQS = (8192, 4096, 2048, 6144, 1024, 3072, 5120, 3072)
 VARLEN_K = 256
+# per-query pass 3 with K/V far beyond the L2: 256K tokens (the longest context of the
+# pages' TTFT figures), Hq 32 / Hkv 8, so that each half of the KV groups the gather walks
+# (2 KB of K and V per key) is 537 MB against 126 MB of L2
+GATHER_BIG = dict(N=262144, Hq=32, Hkv=8, d=128, k=2048)
+# L2 ceiling of this GPU as ncu states it (peak L2 sector rate x 32 B), read from the
+# committed capture summarised in profiles/l2_sector_peak_b200.md
+L2_PEAK_GBS = 34580.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -129,14 +147,84 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-# ------------------------------------------------------------------ the device step
+# ------------------------------------------------------------------ the calls
 
-ROWS_ALL = ("pass1_lse", "pass2_mass_topk", "pass3_gather", "pass2_block_mass_topk",
-            "pass3_block", "indexer_topk", "pass3_indexer_support", "dense_prefill")
+class Calls:
+    """Device-resident inputs of one workload and the library calls of every row."""
+
+    def __init__(self, tam, w, q, k, v, qx=None, kx=None):
+        self.tam, self.w = tam, w
+        self.q, self.k, self.v, self.qx, self.kx = q, k, v, qx, kx
+        self.ws = tam.Workspace(q.device)
+        self.out = {}
+
+    @property
+    def per_query(self):
+        return 1 in self.w.block_q
+
+    @property
+    def block_q(self):
+        return max(self.w.block_q)
+
+    @property
+    def indexer_k(self):
+        return INDEXER_K if self.w.name == WORKLOAD else self.w.budget_k
+
+    # the step: one oracle call (per query if the workload has it, else block-shared)
+    def prefill(self, block_q=None):
+        bq = block_q or (1 if self.per_query else self.block_q)
+        r = self.tam.mass_oracle_prefill(self.q, self.k, self.v, self.w.budget_k, bq,
+                                         workspace=self.ws, check=False)
+        tag = "p1" if bq == 1 else "pb"
+        self.out.update({f"{tag}_idx": r.idx, f"{tag}_len": r.length, f"{tag}_mass": r.value,
+                         f"{tag}_lse": r.lse, f"{tag}_out": r.out})
+        return r
+
+    def row(self, name):
+        t, w, ws, o = self.tam, self.w, self.ws, self.out
+        if name == "pass1_lse":
+            o["lse"] = t.attention_lse(self.q, self.k, workspace=ws, check=False)
+        elif name == "pass2_mass_topk":
+            s = t.mass_select(self.q, self.k, o["lse"], w.budget_k, 1, workspace=ws, check=False)
+            o.update(s1_idx=s.idx, s1_len=s.length, s1_mass=s.value)
+        elif name == "pass3_gather":
+            o["o1"] = t.sparse_support_attention(self.q, self.k, self.v, o["s1_idx"], o["s1_len"],
+                                                 1, workspace=ws, check=False)
+        elif name == "pass2_block_mass_topk":
+            s = t.mass_select(self.q, self.k, o["lse"], w.budget_k, self.block_q, workspace=ws,
+                              check=False)
+            o.update(s2_idx=s.idx, s2_len=s.length, s2_mass=s.value)
+        elif name == "pass3_block":
+            o["o2"] = t.sparse_support_attention(self.q, self.k, self.v, o["s2_idx"], o["s2_len"],
+                                                 self.block_q, workspace=ws, check=False)
+        elif name == "indexer_topk":
+            s = t.indexer_topk(self.qx, self.kx, self.indexer_k, workspace=ws, check=False)
+            o.update(s3_idx=s.idx, s3_len=s.length, s3_score=s.value)
+        elif name == "pass3_indexer_support":
+            o["o3"] = t.sparse_support_attention(self.q, self.k, self.v, o["s3_idx"], o["s3_len"],
+                                                 1, workspace=ws, check=False)
+        elif name == "dense_prefill":
+            o["od"] = t.dense_gqa_prefill(self.q, self.k, self.v, workspace=ws, check=False)
+        else:
+            raise KeyError(name)
+
+    def rows(self, names, events=None):
+        for n, name in enumerate(names):
+            if events is not None:
+                events[n].record()
+            self.row(name)
+        if events is not None:
+            events[len(names)].record()
 
 
-def rows_of(w) -> tuple:
-    """Rows of the hot path a workload exercises (the 32K default runs all of them)."""
+def step_rows(w):
+    """The passes of the step, each on its own entry point (per query, else block)."""
+    if 1 in w.block_q:
+        return ("pass1_lse", "pass2_mass_topk", "pass3_gather")
+    return ("pass1_lse", "pass2_block_mass_topk", "pass3_block")
+
+
+def all_rows(w):
     rows = ["pass1_lse"]
     if 1 in w.block_q:
         rows += ["pass2_mass_topk", "pass3_gather"]
@@ -148,63 +236,57 @@ def rows_of(w) -> tuple:
     return tuple(rows)
 
 
-class Step:
-    """The workload's rows of the hot path on device-resident inputs; CUDA events between
-    calls (events[i] .. events[i+1] brackets row i)."""
-
-    def __init__(self, tam, w, q, k, v, qx=None, kx=None):
-        self.tam, self.w = tam, w
-        self.q, self.k, self.v, self.qx, self.kx = q, k, v, qx, kx
-        self.rows = rows_of(w)
-        self.block_q = max(w.block_q)
-        self.ws = tam.Workspace(q.device)
-        self.outputs = {}
-
-    def run(self, events=None):
-        t, w, ws = self.tam, self.w, self.ws
-        ev = events or [None] * (len(self.rows) + 1)
-        out = {}
-        lse = None
-        for n, row in enumerate(self.rows):
-            if ev[n] is not None:
-                ev[n].record()
-            if row == "pass1_lse":
-                lse = out["lse"] = t.attention_lse(self.q, self.k, workspace=ws, check=False)
-            elif row == "pass2_mass_topk":
-                s = t.mass_select(self.q, self.k, lse, w.budget_k, 1, workspace=ws, check=False)
-                out.update(s1_idx=s.idx, s1_len=s.length, s1_mass=s.value)
-            elif row == "pass3_gather":
-                out["o1"] = t.sparse_support_attention(self.q, self.k, self.v, out["s1_idx"],
-                                                       out["s1_len"], 1, workspace=ws, check=False)
-            elif row == "pass2_block_mass_topk":
-                s = t.mass_select(self.q, self.k, lse, w.budget_k, self.block_q, workspace=ws,
-                                  check=False)
-                out.update(s2_idx=s.idx, s2_len=s.length, s2_mass=s.value)
-            elif row == "pass3_block":
-                out["o2"] = t.sparse_support_attention(self.q, self.k, self.v, out["s2_idx"],
-                                                       out["s2_len"], self.block_q, workspace=ws,
-                                                       check=False)
-            elif row == "indexer_topk":
-                s = t.indexer_topk(self.qx, self.kx, self.indexer_k, workspace=ws, check=False)
-                out.update(s3_idx=s.idx, s3_len=s.length, s3_score=s.value)
-            elif row == "pass3_indexer_support":
-                out["o3"] = t.sparse_support_attention(self.q, self.k, self.v, out["s3_idx"],
-                                                       out["s3_len"], 1, workspace=ws, check=False)
-            elif row == "dense_prefill":
-                out["od"] = t.dense_gqa_prefill(self.q, self.k, self.v, workspace=ws, check=False)
-        if ev[len(self.rows)] is not None:
-            ev[len(self.rows)].record()
-        self.outputs = out
-        return out
-
-    @property
-    def indexer_k(self):
-        return INDEXER_K if self.w.name == WORKLOAD else self.w.budget_k
+def capture(tam, dev, fn):
+    """fn's library launches captured once as a CUDA graph (after a warm-up on the
+    capture's side stream); returns (graph, kernels launched per replay)."""
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    n0 = tam.kernel_launches()
+    with torch.cuda.graph(g):
+        fn()
+    n = tam.kernel_launches() - n0
+    g.replay()
+    torch.cuda.synchronize()
+    return g, n
 
 
-def algorithmic_work(step, N):
+def time_replays(graph, flush, steps, warm=False):
+    """Per-replay device times (ms) of `graph`; the L2 is flushed before every replay
+    (outside the timed events) unless warm."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for s in range(steps):
+        if not warm:
+            flush.fill_(s & 0xff)
+        ev[s][0].record()
+        graph.replay()
+        ev[s][1].record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def row_times(calls, names, flush, steps):
+    """Eager per-row device times: CUDA events between the calls, L2 flushed first."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+          for _ in range(steps)]
+    for s in range(steps):
+        flush.fill_(s & 0xff)
+        calls.rows(names, ev[s])
+    torch.cuda.synchronize()
+    return {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps))
+            for i, n in enumerate(names)}
+
+
+# ------------------------------------------------------------------ rooflines
+
+def algorithmic_work(calls, N):
     """Per-row algorithmic flops/bytes (what the method must do, not what it avoids)."""
-    w, outs = step.w, step.outputs
+    w, outs = calls.w, calls.out
     Hq, Hkv, d = w.Hq, w.Hkv, w.d
     elt = 2
     cp = causal_pairs(N)
@@ -217,17 +299,14 @@ def algorithmic_work(step, N):
         "indexer_topk": {"bound": "tensor", "flops": 2.0 * (w.d_idx or D_IDX) * cp},
         "dense_prefill": {"bound": "tensor", "flops": 4.0 * d * Hq * cp},
     }
-    if "pass3_gather" in step.rows:
-        sp1 = support_pairs(N, w.budget_k)
-        work["pass3_gather"] = {"bound": "hbm",
-                                "bytes": float(gather(sp1) + qo + N * w.budget_k * 4 + N * 4)}
-    if "pass3_indexer_support" in step.rows:
-        kx = step.indexer_k
-        sp3 = support_pairs(N, kx)
-        work["pass3_indexer_support"] = {"bound": "hbm",
-                                         "bytes": float(gather(sp3) + qo + N * kx * 4 + N * 4)}
-    if "pass3_block" in step.rows:
-        bq = step.block_q
+    sp1 = support_pairs(N, w.budget_k)
+    work["pass3_gather"] = {"bound": "l2", "bytes": float(gather(sp1) + qo + N * w.budget_k * 4 + N * 4)}
+    kx = calls.indexer_k
+    sp3 = support_pairs(N, kx)
+    work["pass3_indexer_support"] = {"bound": "l2",
+                                     "bytes": float(gather(sp3) + qo + N * kx * 4 + N * 4)}
+    if "s2_len" in outs:
+        bq = calls.block_q
         s2_len = outs["s2_len"].cpu().numpy().astype(np.int64)
         s2_idx = outs["s2_idx"].cpu().numpy()
         nb = len(s2_len)
@@ -242,10 +321,26 @@ def algorithmic_work(step, N):
     return work
 
 
-# Random 256-byte row gather from a 140 MB table (the 32K layer's K+V is 134 MB), measured
-# on this machine's B200 with CUDA events (profiles/probe_b200_memory_and_mufu.md): the rate
-# an L2-resident gather can reach, given next to the HBM copy peak for the gather rows.
-L2_GATHER_GBS = 11074.1
+def roofline_of(work, ms, pk, pk_kind, traffic=None):
+    tf_peak = pk.get("bf16_tflops", pk.get("bf16_tflops_sustained"))
+    if work["bound"] == "tensor":
+        ach = work["flops"] / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": tf_peak, "unit": "TFLOP/s",
+                "frac": ach / tf_peak, "traffic": traffic,
+                "peak_kind": f"bf16 dense, burst, of {pk_kind}"}
+    ach = work["bytes"] / (ms * 1e-3) / 1e9
+    r = {"bound": work["bound"], "achieved": ach, "unit": "GB/s", "traffic": traffic,
+         "frac_of_hbm": ach / pk["hbm_gbs"]}
+    if work["bound"] == "l2":
+        r.update(peak=L2_PEAK_GBS, frac=ach / L2_PEAK_GBS,
+                 peak_kind="L2 sector ceiling per ncu (profiles/l2_sector_peak_b200.md); the "
+                           "K/V gathered (134 MB, walked in two 67 MB halves) stays in L2")
+    else:
+        r.update(bound="hbm", peak=pk["hbm_gbs"], frac=ach / pk["hbm_gbs"],
+                 peak_kind=f"HBM copy, of {pk_kind}")
+    if "flops" in work:
+        r["tflops"] = work["flops"] / (ms * 1e-3) / 1e12
+    return r
 
 
 def traffic_table():
@@ -272,85 +367,59 @@ def traffic_table():
     return out
 
 
-def roofline_of(work, ms, pk, pk_kind, traffic=None):
-    tf_peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
-    if work["bound"] == "tensor":
-        ach = work["flops"] / (ms * 1e-3) / 1e12
-        return {"bound": "tensor", "achieved": ach, "peak": tf_peak, "unit": "TFLOP/s",
-                "frac": ach / tf_peak, "traffic": traffic,
-                "peak_kind": f"bf16 dense, sustained, of {pk_kind}"}
-    ach = work["bytes"] / (ms * 1e-3) / 1e9
-    return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": ach / pk["hbm_gbs"], "traffic": traffic, "peak_kind": f"HBM copy, of {pk_kind}",
-            "l2_gather_peak": L2_GATHER_GBS, "frac_of_l2_gather_peak": ach / L2_GATHER_GBS}
-
-
 # ------------------------------------------------------------------ oracle (CPU) arm
 
 def oracle_sample_step(inp, w, n_rows: int):
-    """The fp64 oracle on a bounded, stratified sample of the step; returns the time it
-    would take for the whole step, extrapolated by each part's per-row work."""
+    """The fp64 oracle on a bounded, stratified sample of the step (passes 1-3 for the
+    step's support); returns the time it would take for the whole step, extrapolated
+    by each part's per-row work ((i+1) for scoring, min(k, i+1) for the recompute)."""
     import oracle
     N = w.N
     rows = np.array([int((m + 0.5) * N / n_rows) for m in range(n_rows)], dtype=np.int64)
     wr = (rows + 1).astype(np.float64)
     w_all = float(causal_pairs(N))
-    kq = np.minimum(w.budget_k, rows + 1).astype(np.float64)
-    kq_all = float(support_pairs(N, w.budget_k))
-    ki = np.minimum(INDEXER_K, rows + 1).astype(np.float64)
-    ki_all = float(support_pairs(N, INDEXER_K))
-    total = 0.0
-    # pass 1 + pass 2 per query (LSE and mass are computed inside the selection)
+    if 1 in w.block_q:
+        kq = np.minimum(w.budget_k, rows + 1).astype(np.float64)
+        kq_all = float(support_pairs(N, w.budget_k))
+        t0 = time.perf_counter()
+        idx, ln, _ = oracle.topk_rows(inp.q, inp.k, w.budget_k, rows)
+        t1 = time.perf_counter()
+        oracle.attn_rows(inp.q, inp.k, inp.v, rows, sup=idx, sup_len=ln)
+        t2 = time.perf_counter()
+        return (t1 - t0) * w_all / wr.sum() + (t2 - t1) * kq_all / kq.sum()
+    bq = max(w.block_q)
+    nb = -(-N // bq)
+    blocks = np.unique(np.minimum(nb - 1, (rows // bq)))[: max(1, n_rows // 8)]
+    brows = np.concatenate([np.arange(b * bq, min(N, (b + 1) * bq)) for b in blocks])
     t0 = time.perf_counter()
-    idx, ln, _ = oracle.topk_rows(inp.q, inp.k, w.budget_k, rows)
+    bidx, bln, _ = oracle.block_topk(inp.q, inp.k, bq, w.budget_k, blocks)
     t1 = time.perf_counter()
-    oracle.attn_rows(inp.q, inp.k, inp.v, rows, sup=idx, sup_len=ln)
-    t2 = time.perf_counter()
-    total += (t1 - t0) * w_all / wr.sum() + (t2 - t1) * kq_all / kq.sum()
-    # block-shared: one block in the middle
-    nb = -(-N // BLOCK_Q)
-    b = nb // 2
-    brows = np.arange(b * BLOCK_Q, min(N, (b + 1) * BLOCK_Q))
-    t0 = time.perf_counter()
-    bidx, bln, _ = oracle.block_topk(inp.q, inp.k, BLOCK_Q, w.budget_k, [b])
-    t1 = time.perf_counter()
-    r, s, sl = oracle.block_rows_support(bidx, bln, BLOCK_Q, N, [b])
+    r, s, sl = oracle.block_rows_support(bidx, bln, bq, N, blocks)
     oracle.attn_rows(inp.q, inp.k, inp.v, r, sup=s, sup_len=sl)
     t2 = time.perf_counter()
-    total += (t1 - t0) * w_all / float((brows + 1).sum()) + (t2 - t1) * nb
-    # indexer
-    t0 = time.perf_counter()
-    xidx, xln, _ = oracle.indexer_topk_rows(inp.q_idx, inp.k_idx, INDEXER_K, rows)
-    t1 = time.perf_counter()
-    oracle.attn_rows(inp.q, inp.k, inp.v, rows, sup=xidx, sup_len=xln)
-    t2 = time.perf_counter()
-    total += (t1 - t0) * w_all / wr.sum() + (t2 - t1) * ki_all / ki.sum()
-    # dense
-    t0 = time.perf_counter()
-    oracle.attn_rows(inp.q, inp.k, inp.v, rows)
-    t1 = time.perf_counter()
-    total += (t1 - t0) * w_all / wr.sum()
-    return total
+    return (t1 - t0) * w_all / float((brows + 1).sum()) + (t2 - t1) * nb / len(blocks)
 
 
 def calibrate_rows(inp, w, target_s: float):
     t0 = time.perf_counter()
     oracle_sample_step(inp, w, 4)
     dt = time.perf_counter() - t0
-    return int(max(4, min(256, round(4 * target_s / max(dt, 1e-3)))))
+    return int(max(4, min(512, round(4 * target_s / max(dt, 1e-3)))))
 
 
-def cpu_sample_desc(n_rows):
-    return (f"{n_rows} stratified query rows (plus one block of {BLOCK_Q}) of the "
-            f"{WORKLOAD} workload through every step; time extrapolated to all rows by "
-            "per-row work ((i+1) for scoring, min(k, i+1) for the sparse recompute)")
+def cpu_sample_desc(w, n_rows):
+    what = ("query rows" if 1 in w.block_q else f"blocks of {max(w.block_q)} queries (about "
+            f"{max(1, n_rows // 8)})")
+    return (f"{n_rows} stratified {what} of the {w.name} workload through passes 1-3 of the "
+            "step; time extrapolated to all rows by per-row work ((i+1) for scoring, "
+            "min(k, i+1) for the sparse recompute)")
 
 
 def run_reference(args, w, inp, rank, world):
     import oracle
     if rank != 0:
         return
-    n_rows = calibrate_rows(inp, w, 6.0)
+    n_rows = calibrate_rows(inp, w, 3.0)
     for _ in range(args.warmup):
         oracle_sample_step(inp, w, n_rows)
     ext = [oracle_sample_step(inp, w, n_rows) for _ in range(args.steps)]
@@ -363,20 +432,21 @@ def run_reference(args, w, inp, rank, world):
         "data": "synthetic (seeded; stands in for the pages' 4K-100K long-context evaluations)",
         "config": config_dict(w, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-                         "sample": cpu_sample_desc(n_rows)},
+                         "sample": cpu_sample_desc(w, n_rows)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def config_dict(w, world, launch=None):
-    idx_k = INDEXER_K if w.name == WORKLOAD else (w.budget_k if w.d_idx else None)
-    extra = {"step_launch": launch} if launch else {}
-    return {**extra, "workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-            "budget_k": w.budget_k, "block_q": list(w.block_q), "indexer_k": idx_k,
-            "d_idx": w.d_idx or None, "rope": w.rope_base, "global_batch": world, "seq_len": w.N,
+def config_dict(w, world):
+    bq = 1 if 1 in w.block_q else max(w.block_q)
+    return {"workload": w.name, "N": w.N, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            "budget_k": w.budget_k, "block_q": bq,
+            "step": (f"one tam_mass_oracle_prefill call: pass 1, pass 2 and its "
+                     f"{'per-query' if bq == 1 else f'block-shared (B_q {bq})'} top-k, pass 3"),
+            "rope": w.rope_base, "global_batch": world, "seq_len": w.N,
             "parallelism": f"replicas x{world} (independent layers, no collective)",
-            "l2": "256 MB buffer written before every step (L2 is 126 MB)"}
+            "l2": "256 MB buffer written before every timed step (L2 is 126 MB)"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -388,204 +458,274 @@ def run_ours(args, w, inp, rank, world, local_rank):
     q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
     qx = inp.q_idx.to(dev) if inp.q_idx is not None else None
     kx = inp.k_idx.to(dev) if inp.k_idx is not None else None
-    step = Step(tam, w, q, k, v, qx, kx)
-    names = step.rows
+    calls = Calls(tam, w, q, k, v, qx, kx)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    names = step_rows(w)
+    block_q = 1 if calls.per_query else calls.block_q
 
+    # warm-up: the step and its passes (the first launches load the kernels)
     for _ in range(args.warmup):
-        step.run()
-    tam.check_status(step.ws.get(256))
+        calls.prefill()
+        calls.rows(names)
     torch.cuda.synchronize()
-    work = algorithmic_work(step, w.N)
+    tam.check_status(calls.ws.get(256))
+    fb_rows = (tam.mass_fallback_rows(q, k, w.budget_k, calls.ws) if calls.per_query else None)
 
-    # per-row breakdown: eager calls with CUDA events between them (same inputs)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
-          for _ in range(args.steps)]
-    for s in range(args.steps):
-        flush.fill_(s & 0xff)
-        step.run(ev[s])
-    torch.cuda.synchronize()
-    tam.check_status(step.ws.get(256))
-    row_ms = {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps))
-              for i, n in enumerate(names)}
-
-    next_rows = measure_next_rows(args, tam, w, step, flush) if w.name == WORKLOAD else None
-
-    # The step is captured once as a CUDA graph (every library launch of the step,
-    # recorded on the capture stream) and replayed in the timed region, so host-side
-    # enqueue time between the rows does not enter the device time.  --no-graph times
-    # the eager calls instead.
-    graph, per_step_launches = None, 0
-    if not args.no_graph:
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(torch.cuda.current_stream(dev))
-        with torch.cuda.stream(side):
-            step.run()                      # warm-up on the capture's side stream
-        torch.cuda.current_stream(dev).wait_stream(side)
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        n0 = tam.kernel_launches()
-        with torch.cuda.graph(graph):
-            step.run()
-        per_step_launches = tam.kernel_launches() - n0
-        graph.replay()
-        torch.cuda.synchronize()
-        tam.check_status(step.ws.get(256))
-
-    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # the step as one CUDA graph (every launch of the call), replayed in the timed region
+    graph, per_step_launches = capture(tam, dev, lambda: calls.prefill(block_q))
+    tam.check_status(calls.ws.get(256))
     clocks = ClockSampler(local_rank)
     barrier(world, local_rank)
     torch.cuda.synchronize()
     clocks.start()
-    launches0 = tam.kernel_launches()
-    t_start.record()
-    for s in range(args.steps):
-        flush.fill_(s & 0xff)
-        if graph is not None:
-            graph.replay()
-        else:
-            step.run()
-    t_stop.record()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    times = time_replays(graph, flush, args.steps)
+    t1.record()
     torch.cuda.synchronize()
-    launches = (per_step_launches * args.steps if graph is not None
-                else tam.kernel_launches() - launches0)
     barrier(world, local_rank)
     clk = clocks.stop()
-    tam.check_status(step.ws.get(256))
-    total_ms = t_start.elapsed_time(t_stop)
-    total_ms = max_over_ranks(total_ms, world, dev)
-    ms_step = total_ms / args.steps
+    tam.check_status(calls.ws.get(256))
+    ms_step = max_over_ranks(statistics.mean(times), world, dev)
+    region_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    warm_ms = statistics.mean(time_replays(graph, flush, args.steps, warm=True))
+    launches = per_step_launches * args.steps
+    del graph
 
-
+    # the passes of the step, each on its own entry point
     pk, pk_kind = peaks()
     traffic = traffic_table()
+    row_ms = row_times(calls, names, flush, args.steps)
+    tam.check_status(calls.ws.get(256))
+
+    extra = {}
+    if w.name == WORKLOAD:
+        extra = measure_extras(args, tam, w, calls, flush, dev)
+    work = algorithmic_work(calls, w.N)
     rows = {}
     for n in names:
-        r = roofline_of(work[n], row_ms[n], pk, pk_kind, traffic.get(n))
-        rows[n] = {"ms": row_ms[n], "q_tok_s": w.N / (row_ms[n] * 1e-3), "roofline": r}
+        rows[n] = {"ms": row_ms[n], "q_tok_s": w.N / (row_ms[n] * 1e-3),
+                   "roofline": roofline_of(work[n], row_ms[n], pk, pk_kind, traffic.get(n))}
     dominant = max(names, key=lambda n: row_ms[n])
+    for key in ("block_shared", "all_rows_step"):
+        for n, r in extra.get(key, {}).get("rows", {}).items():
+            r["roofline"] = roofline_of(work[n], r["ms"], pk, pk_kind, traffic.get(n))
 
-    e2e = measure_e2e(args, tam, w, inp, dev, world, local_rank)
+    e2e = measure_e2e(args, tam, w, inp, dev, world, local_rank, block_q)
 
     if rank != 0:
         return
     value = job_value(world, w.N, ms_step)
-    oracle_sparsity = 1.0 - support_pairs(w.N, w.budget_k) / causal_pairs(w.N)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; stands in for the pages' 4K-100K long-context evaluations)",
-        "config": config_dict(w, world, "CUDA graph replay of the step's library calls"
-                              if graph is not None else "eager library calls"),
+        "config": config_dict(w, world),
         "roofline": {**rows[dominant]["roofline"], "kernel": dominant},
         "rows": rows,
-        "sparse_pass": sparse_pass_summary(w, row_ms),
-        "support_quality": support_quality(step),
+        "timed_region_ms": region_ms,
+        "warm_l2_ms_per_step": warm_ms,
+        "fallback_rows": fb_rows,
+        **extra,
         "sparsity_selfcheck": {
-            "this_workload": oracle_sparsity,
+            "this_workload": 1.0 - support_pairs(w.N, w.budget_k) / causal_pairs(w.N),
             "N4096_k256": 1.0 - support_pairs(4096, 256) / causal_pairs(4096),
             "N102400_k2048": 1.0 - support_pairs(102400, 2048) / causal_pairs(102400),
         },
         "clocks": clk,
-        "next_rows": next_rows,
         "e2e": e2e,
         "gpu_launches": launches,
     }
-    if world == 1 and not args.no_cpu_baseline and w.name == WORKLOAD:
+    if world == 1 and not args.no_cpu_baseline:
         import oracle
         n_rows = calibrate_rows(inp, w, 15.0)
         t = oracle_sample_step(inp, w, n_rows)
         line["cpu_baseline"] = {"value": w.N / t, "unit": UNIT, "cores": oracle.threads(),
-                                "kind": "oracle", "sample": cpu_sample_desc(n_rows)}
+                                "kind": "oracle", "sample": cpu_sample_desc(w, n_rows)}
     print(json.dumps(line), flush=True)
 
 
-def measure_next_rows(args, tam, w, step, flush):
+def measure_extras(args, tam, w, calls, flush, dev):
+    """Everything reported beside the step on the 32K workload (see the module doc)."""
+    out = {}
+    # block-shared oracle call (B_q = 64) and its passes
+    g, _ = capture(tam, dev, lambda: calls.prefill(BLOCK_Q))
+    ms_b = statistics.mean(time_replays(g, flush, args.steps))
+    del g
+    brows = ("pass1_lse", "pass2_block_mass_topk", "pass3_block")
+    calls.rows(brows)
+    bt = row_times(calls, brows, flush, args.steps)
+    out["block_shared"] = {"block_q": BLOCK_Q, "ms": ms_b, "q_tok_s": w.N / (ms_b * 1e-3),
+                           "rows": {n: {"ms": bt[n], "q_tok_s": w.N / (bt[n] * 1e-3)} for n in brows}}
+    # every row of the hot path in one graph
+    names = all_rows(w)
+    g, _ = capture(tam, dev, lambda: calls.rows(names))
+    ms_all = statistics.mean(time_replays(g, flush, args.steps))
+    del g
+    at = row_times(calls, names, flush, args.steps)
+    tam.check_status(calls.ws.get(256))
+    out["all_rows_step"] = {"rows_in_order": list(names), "ms": ms_all,
+                            "q_tok_s": w.N / (ms_all * 1e-3),
+                            "rows": {n: {"ms": at[n], "q_tok_s": w.N / (at[n] * 1e-3)} for n in names}}
+    dense = at["dense_prefill"]
+    out["sparse_pass"] = {
+        "per_query_pass3_speedup_vs_dense": dense / at["pass3_gather"],
+        "block_shared_pass3_speedup_vs_dense": dense / at["pass3_block"],
+        "indexer_support_pass3_speedup_vs_dense": dense / at["pass3_indexer_support"],
+        "indexer_path_speedup_vs_dense": dense / (at["indexer_topk"] + at["pass3_indexer_support"]),
+        "per_query_oracle_passes_1_3_vs_dense": dense / (at["pass1_lse"] + at["pass2_mass_topk"]
+                                                         + at["pass3_gather"]),
+    }
+    out["support_quality"] = support_quality(tam, w, calls, flush, args.steps)
+    out["gather_out_of_l2"] = measure_gather_big(tam, dev, flush, args.steps)
+    out["next_rows"] = measure_next_rows(args, tam, w, calls, flush)
+    return out
+
+
+def support_quality(tam, w, calls, flush, steps):
+    """C5: the indexer's support (k = 1024) against the mass oracle's per-query support
+    at the same k on the same tensors: recall@k over the rows with i+1 > k, and the
+    max-abs difference of the two pass-3 outputs; each sparse output against dense;
+    and the random-support stress row's pass-3 time at this k."""
+    o = calls.out
+    kx = calls.indexer_k
+    m = tam.mass_select(calls.q, calls.k, o["lse"], kx, 1, workspace=calls.ws, check=False)
+    om = tam.sparse_support_attention(calls.q, calls.k, calls.v, m.idx, m.length, 1,
+                                      workspace=calls.ws, check=False)
+    a, b = m.idx[kx:].long(), o["s3_idx"][kx:].long()          # rows i >= k hold k keys
+    res = {"recall_k": kx}
+    if a.numel():
+        pos = torch.searchsorted(a.contiguous(), b.contiguous()).clamp_(max=kx - 1)
+        hit = (torch.gather(a, 1, pos) == b).sum(dim=1).double() / kx
+        res["indexer_recall_at_k"] = float(hit.mean())
+    res["indexer_output_vs_mass_oracle_max_abs"] = float((o["o3"].float() - om.float()).abs().max())
+    res["indexer_output_vs_mass_oracle_mean_abs"] = float((o["o3"].float() - om.float()).abs().mean())
+    od = o["od"].float()
+    for key, name in (("o1", "per_query"), ("o2", "block_shared"), ("o3", "indexer")):
+        res[f"{name}_output_vs_dense_max_abs"] = float((o[key].float() - od).abs().max())
+    # stress row: uniform-random support of the indexer's budget
+    sidx, slen = tam_synth.stratified_support(w.N, kx, seed=7, device=calls.q.device)
+    f = lambda: tam.sparse_support_attention(calls.q, calls.k, calls.v, sidx, slen, 1,  # noqa: E731
+                                             workspace=calls.ws, check=False)
+    f()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for s in range(steps):
+        flush.fill_(s & 0xff)
+        ev[s][0].record()
+        f()
+        ev[s][1].record()
+    torch.cuda.synchronize()
+    res["stress_row_pass3_ms"] = statistics.mean(x.elapsed_time(y) for x, y in ev)
+    res["stress_row_support"] = f"one uniform key per stratum of [0, i], k = {kx}"
+    del m, om, sidx, slen
+    return res
+
+
+def measure_gather_big(tam, dev, flush, steps):
+    """Per-query pass 3 with K/V far beyond the L2: 262144 tokens, Hq 32 / Hkv 8, d 128,
+    random support of k = 2048 per query (one uniform key per stratum of [0, i]);
+    inputs drawn on the device (the values do not matter to a gather's time)."""
+    c = GATHER_BIG
+    N, Hq, Hkv, d, kb = c["N"], c["Hq"], c["Hkv"], c["d"], c["k"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    q = torch.randn(N, Hq, d, generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn(N, Hkv, d, generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn(N, Hkv, d, generator=g, device=dev).to(torch.bfloat16)
+    idx, ln = tam_synth.stratified_support(N, kb, seed=9, device=dev)
+    ws = tam.Workspace(dev)
+    f = lambda: tam.sparse_support_attention(q, k, v, idx, ln, 1, workspace=ws, check=False)  # noqa: E731
+    f()
+    torch.cuda.synchronize()
+    n = max(2, min(steps, 3))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    for s in range(n):
+        flush.fill_(s & 0xff)
+        ev[s][0].record()
+        f()
+        ev[s][1].record()
+    torch.cuda.synchronize()
+    tam.check_status(ws.get(256))
+    ms = statistics.mean(x.elapsed_time(y) for x, y in ev)
+    gathered = support_pairs(N, kb) * Hkv * 2 * d * 2
+    nbytes = gathered + 2 * N * Hq * d * 2 + N * kb * 4 + N * 4
+    pk, pk_kind = peaks()
+    ach = nbytes / (ms * 1e-3) / 1e9
+    del q, k, v, idx, ln, ws
+    torch.cuda.empty_cache()
+    return {"N": N, "Hq": Hq, "Hkv": Hkv, "d": d, "budget_k": kb,
+            "kv_bytes_per_half_of_the_groups": N * (Hkv // 2) * 2 * d * 2,
+            "ms": ms, "q_tok_s": N / (ms * 1e-3), "bytes": nbytes,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / pk["hbm_gbs"], "peak_kind": f"HBM copy, of {pk_kind}",
+                         "frac_of_8tbs_nominal": ach / 8000.0}}
+
+
+def measure_next_rows(args, tam, w, calls, flush):
     """Rows beyond the step (reported, not part of `value`): the fused, selection-block-
     shared indexer (block sums of each query's softmax of its indexer scores, top-k per
     block of BLOCK_Q queries), pass 3 on that support, the indexer's distillation
-    target (KL of the indexer's distribution from the head-averaged mass), and a budget
-    sweep (support mass at k = 256..2048 from one pass 2 at k = 2048)."""
+    target (KL of the indexer's distribution from the head-averaged mass), a budget
+    sweep (support mass at k = 256..2048 from one pass 2 at k = 2048) and a packed
+    batch of eight sequences."""
     bq, kx = BLOCK_Q, INDEXER_K
-    lse = tam.attention_lse(step.q, step.k, workspace=step.ws, check=False)
-    # warm-up (first launches load the kernels; the workspace grows to its largest size)
-    for _ in range(2):
-        sup = tam.indexer_topk(step.qx, step.kx, kx, bq, workspace=step.ws, check=False)
-        tam.sparse_support_attention(step.q, step.k, step.v, sup.idx, sup.length, bq,
-                                     workspace=step.ws, check=False)
-        tam.distill_kl(step.q, step.k, lse, step.qx, step.kx, workspace=step.ws, check=False)
-    torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    for s in range(args.steps):
-        flush.fill_(s & 0xff)
-        ev[s][0].record()
-        sup = tam.indexer_topk(step.qx, step.kx, kx, bq, workspace=step.ws, check=False)
-        ev[s][1].record()
-        tam.sparse_support_attention(step.q, step.k, step.v, sup.idx, sup.length, bq,
-                                     workspace=step.ws, check=False)
-        ev[s][2].record()
-    torch.cuda.synchronize()
-    tam.check_status(step.ws.get(256))
-    t_sel = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    t_att = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    n_sel = sup.length.cpu().numpy().astype(np.int64)
-    # the indexer's distillation target (pass 1's lse is an input, as for pass 2)
-    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for s in range(args.steps):
-        flush.fill_(s & 0xff)
-        evk[s][0].record()
-        tam.distill_kl(step.q, step.k, lse, step.qx, step.kx, workspace=step.ws, check=False)
-        evk[s][1].record()
-    torch.cuda.synchronize()
-    tam.check_status(step.ws.get(256))
-    t_kl = statistics.mean(e[0].elapsed_time(e[1]) for e in evk)
-    # budget sweep from one pass 2 at k_max = 2048: per-query support mass at 256..2048
-    lse1 = lse
+    ws = calls.ws
+    lse = tam.attention_lse(calls.q, calls.k, workspace=ws, check=False)
+
+    def timed(fns):
+        for _ in range(2):
+            for fn in fns:
+                fn()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+              for _ in range(args.steps)]
+        for s in range(args.steps):
+            flush.fill_(s & 0xff)
+            for i, fn in enumerate(fns):
+                ev[s][i].record()
+                fn()
+            ev[s][-1].record()
+        torch.cuda.synchronize()
+        tam.check_status(ws.get(256))
+        return [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(len(fns))]
+
+    box = {}
+
+    def sel():
+        box["sup"] = tam.indexer_topk(calls.qx, calls.kx, kx, bq, workspace=ws, check=False)
+
+    def att():
+        tam.sparse_support_attention(calls.q, calls.k, calls.v, box["sup"].idx,
+                                     box["sup"].length, bq, workspace=ws, check=False)
+
+    t_sel, t_att = timed([sel, att])
+    n_sel = box["sup"].length.cpu().numpy().astype(np.int64)
+    (t_kl,) = timed([lambda: tam.distill_kl(calls.q, calls.k, lse, calls.qx, calls.kx,
+                                            workspace=ws, check=False)])
     budgets = [256, 512, 1024, 2048]
-    sup = tam.mass_select(step.q, step.k, lse1, budgets[-1], 1, workspace=step.ws, check=False)
-    tam.support_mass_curve(sup.value, sup.length, budgets)
-    torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    for s in range(args.steps):
-        flush.fill_(s & 0xff)
-        evs[s][0].record()
-        sup = tam.mass_select(step.q, step.k, lse1, budgets[-1], 1, workspace=step.ws, check=False)
-        evs[s][1].record()
-        curve = tam.support_mass_curve(sup.value, sup.length, budgets)
-        evs[s][2].record()
-    torch.cuda.synchronize()
-    tam.check_status(step.ws.get(256))
-    t_p2 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    t_cv = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    mean_mass = curve.mean(dim=0).cpu().tolist()
-    # packed batch: the step's tokens as VARLEN_SEQS independent sequences, per-query
-    # support at VARLEN_K (passes 1-3), and the dense comparator on the same batch
+
+    def p2():
+        box["s"] = tam.mass_select(calls.q, calls.k, lse, budgets[-1], 1, workspace=ws, check=False)
+
+    def curve():
+        box["c"] = tam.support_mass_curve(box["s"].value, box["s"].length, budgets)
+
+    t_p2, t_cv = timed([p2, curve])
+    mean_mass = box["c"].mean(dim=0).cpu().tolist()
     cu = [0]
     for n in VARLEN_SEQS:
         cu.append(cu[-1] + n)
     vl = None
     if cu[-1] == w.N:
-        for _ in range(2):
-            tam.mass_oracle_prefill_varlen(step.q, step.k, step.v, cu, VARLEN_K, 1,
-                                           workspace=step.ws, check=False)
-            tam.dense_gqa_prefill_varlen(step.q, step.k, step.v, cu, workspace=step.ws,
-                                         check=False)
-        torch.cuda.synchronize()
-        evv = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-        for s in range(args.steps):
-            flush.fill_(s & 0xff)
-            evv[s][0].record()
-            tam.mass_oracle_prefill_varlen(step.q, step.k, step.v, cu, VARLEN_K, 1,
-                                           workspace=step.ws, check=False)
-            evv[s][1].record()
-            tam.dense_gqa_prefill_varlen(step.q, step.k, step.v, cu, workspace=step.ws,
-                                         check=False)
-            evv[s][2].record()
-        torch.cuda.synchronize()
-        tam.check_status(step.ws.get(256))
-        t_vo = statistics.mean(e[0].elapsed_time(e[1]) for e in evv)
-        t_vd = statistics.mean(e[1].elapsed_time(e[2]) for e in evv)
+        t_vo, t_vd = timed([
+            lambda: tam.mass_oracle_prefill_varlen(calls.q, calls.k, calls.v, cu, VARLEN_K, 1,
+                                                   workspace=ws, check=False),
+            lambda: tam.dense_gqa_prefill_varlen(calls.q, calls.k, calls.v, cu, workspace=ws,
+                                                 check=False)])
         vl = {"seq_lens": list(VARLEN_SEQS), "budget_k": VARLEN_K,
               "ms_oracle_passes_1_3": t_vo, "q_tok_s_oracle": w.N / (t_vo * 1e-3),
               "ms_dense": t_vd, "q_tok_s_dense": w.N / (t_vd * 1e-3)}
@@ -603,36 +743,33 @@ def measure_next_rows(args, tam, w, step, flush):
     }
 
 
-def measure_e2e(args, tam, w, inp, dev, world, local_rank):
-    """Same step through the public API with pinned host inputs and results.
+def measure_e2e(args, tam, w, inp, dev, world, local_rank, block_q):
+    """The step through the public API with pinned host inputs and results.
 
-    Every step copies its inputs in from pinned host memory and every output back,
-    on two copy streams next to the compute stream: inputs go to one of two device
-    sets (the copy for step s+1 overlaps step s), and each row's outputs start back
-    to the host as soon as that row is done.  The timed region runs from the first
-    input copy to the last output copy."""
+    Every step copies its inputs (Q, K, V) in from pinned host memory and every output
+    (support indices, lengths, masses, lse, sparse output) back, on two copy streams
+    next to the compute stream: inputs go to one of two device sets (the copy for step
+    s+1 overlaps step s), and the outputs of step s go back once it is done.  The timed
+    region runs from the first input copy to the last output copy."""
     if args.no_e2e:
         return None
     host_in = [inp.q.pin_memory(), inp.k.pin_memory(), inp.v.pin_memory()]
-    if inp.q_idx is not None:
-        host_in += [inp.q_idx.pin_memory(), inp.k_idx.pin_memory()]
     sets = [[torch.empty_like(t, device=dev) for t in host_in] for _ in range(2)]
-    steps = [Step(tam, w, *d) for d in sets]
-    for t_d, t_h in zip(sets[0], host_in):
-        t_d.copy_(t_h)
-    outs = steps[0].run()
-    host_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in outs.items()}
-    steps[1].ws = steps[0].ws                    # one workspace: the steps run in order
-    for t_d, t_h in zip(sets[1], host_in):
-        t_d.copy_(t_h)
-    steps[1].run()
+    ws = tam.Workspace(dev)
+
+    def call(b):
+        q, k, v = sets[b]
+        r = tam.mass_oracle_prefill(q, k, v, w.budget_k, block_q, workspace=ws, check=False)
+        return [r.idx, r.length, r.value, r.lse, r.out]
+
+    for b in range(2):
+        for t_d, t_h in zip(sets[b], host_in):
+            t_d.copy_(t_h)
+    outs = call(0)
+    host_out = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+    torch.cuda.synchronize()
     h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    # which outputs each row produces (copied back once that row is done)
-    row_outs = {"pass1_lse": ["lse"], "pass2_mass_topk": ["s1_idx", "s1_len", "s1_mass"],
-                "pass3_gather": ["o1"], "pass2_block_mass_topk": ["s2_idx", "s2_len", "s2_mass"],
-                "pass3_block": ["o2"], "indexer_topk": ["s3_idx", "s3_len", "s3_score"],
-                "pass3_indexer_support": ["o3"], "dense_prefill": ["od"]}
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
     comp = torch.cuda.current_stream(dev)
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     n = max(2, min(args.steps, 4))
@@ -640,8 +777,7 @@ def measure_e2e(args, tam, w, inp, dev, world, local_rank):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(comp)
-    in_ready = [torch.cuda.Event() for _ in range(n)]
-    done = [None] * n                            # compute of step s finished reading its set
+    done = [None] * n
     for s in range(n):
         b = s % 2
         if s == 0:
@@ -651,28 +787,27 @@ def measure_e2e(args, tam, w, inp, dev, world, local_rank):
         with torch.cuda.stream(s_in):
             for t_d, t_h in zip(sets[b], host_in):
                 t_d.copy_(t_h, non_blocking=True)
-        in_ready[s].record(s_in)
-        comp.wait_event(in_ready[s])
-        step = steps[b]
-        ev = [torch.cuda.Event() for _ in range(len(step.rows) + 1)]
-        outs = step.run(ev)
+        ready = torch.cuda.Event()
+        ready.record(s_in)
+        comp.wait_event(ready)
+        outs = call(b)
         done[s] = torch.cuda.Event()
         done[s].record(comp)
-        for r, row in enumerate(step.rows):
-            s_out.wait_event(ev[r + 1])
-            with torch.cuda.stream(s_out):
-                for name in row_outs[row]:
-                    t = outs[name]
-                    t.record_stream(s_out)
-                    host_out[name].copy_(t, non_blocking=True)
+        s_out.wait_event(done[s])
+        with torch.cuda.stream(s_out):
+            for t, h in zip(outs, host_out):
+                t.record_stream(s_out)
+                h.copy_(t, non_blocking=True)
     comp.wait_stream(s_out)
     e1.record(comp)
     torch.cuda.synchronize()
+    tam.check_status(ws.get(256))
     barrier(world, local_rank)
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n
     return {"value": job_value(world, w.N, ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n,
-            "overlap": "inputs double-buffered on a copy stream; outputs copied per row on a second one"}
+            "call": "top_attention_mass_b200.mass_oracle_prefill (C ABI tam_mass_oracle_prefill)",
+            "overlap": "inputs double-buffered on a copy stream; outputs copied back on a second one"}
 
 
 # ------------------------------------------------------------------ process group plumbing
@@ -701,26 +836,6 @@ def job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
     return world * tokens_per_rank / (ms_per_step * 1e-3)
 
 
-def support_quality(step):
-    """Indexer support vs mass-oracle support (recall@k over rows with i+1 > k, when both
-    use the same k) and each sparse output's max-abs distance from dense attention."""
-    out, w = step.outputs, step.w
-    res = {}
-    od = out["od"].float()
-    for key, name in (("o1", "per_query"), ("o2", "block_shared"), ("o3", "indexer")):
-        if key in out:
-            res[f"{name}_output_vs_dense_max_abs"] = float((out[key].float() - od).abs().max())
-    if "s1_idx" in out and "s3_idx" in out and out["s1_idx"].shape == out["s3_idx"].shape:
-        k = out["s1_idx"].shape[1]
-        a, b = out["s1_idx"][k:].long(), out["s3_idx"][k:].long()       # rows i >= k are full
-        if a.numel():
-            pos = torch.searchsorted(a.contiguous(), b.contiguous()).clamp_(max=k - 1)
-            hit = (torch.gather(a, 1, pos) == b).sum(dim=1).double() / k
-            res["indexer_recall_at_k"] = float(hit.mean())
-            res["recall_k"] = k
-    return res
-
-
 def workload_for(name: str):
     """The default step is the 32K layer with both supports (B_q = 64) and its indexer
     head (d_idx = 64, k = 1024 on the same tensors); other names are single workloads."""
@@ -728,27 +843,6 @@ def workload_for(name: str):
         base = tam_synth.WORKLOADS[WORKLOAD]
         return tam_synth.Workload(**{**base.__dict__, "d_idx": D_IDX})
     return tam_synth.WORKLOADS[name]
-
-
-def sparse_pass_summary(w, row_ms):
-    out = {}
-    dense = row_ms["dense_prefill"]
-    if "pass3_gather" in row_ms:
-        out["per_query_q_tok_s"] = w.N / (row_ms["pass3_gather"] * 1e-3)
-        out["speedup_vs_dense"] = dense / row_ms["pass3_gather"]
-        out["oracle_pass12_plus3_q_tok_s"] = w.N / 1e-3 / (row_ms["pass1_lse"]
-                                                           + row_ms["pass2_mass_topk"]
-                                                           + row_ms["pass3_gather"])
-    if "pass3_block" in row_ms:
-        out["block_shared_q_tok_s"] = w.N / (row_ms["pass3_block"] * 1e-3)
-        out["block_shared_speedup_vs_dense"] = dense / row_ms["pass3_block"]
-        out["oracle_block_pass12_plus3_q_tok_s"] = w.N / 1e-3 / (
-            row_ms["pass1_lse"] + row_ms["pass2_block_mass_topk"] + row_ms["pass3_block"])
-    if "pass3_indexer_support" in row_ms:
-        out["indexer_support_speedup_vs_dense"] = dense / row_ms["pass3_indexer_support"]
-        out["indexer_path_speedup_vs_dense"] = dense / (row_ms["indexer_topk"]
-                                                        + row_ms["pass3_indexer_support"])
-    return out
 
 
 def main():
@@ -759,10 +853,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-graph", action="store_true",
-                    help="time the eager library calls instead of a CUDA-graph replay of the step")
     ap.add_argument("--workload", default=WORKLOAD,
-                    help="gqa32k_2pct (default: every row), gqa4k_needles, longctx_<N>, indexer32k")
+                    help="gqa32k_2pct (default), gqa4k_needles, longctx_<N>, indexer32k")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -772,10 +864,6 @@ def main():
     w = workload_for(args.workload)
     if args.impl == "reference":
         if rank != 0:
-            return
-        if w.name != WORKLOAD:
-            print(json.dumps({"impl": "reference", "unavailable":
-                              "the oracle arm is sampled on the default 32K workload only"}))
             return
         inp = tam_synth.make_inputs(w)
         run_reference(args, w, inp, rank, world)

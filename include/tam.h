@@ -88,9 +88,26 @@ const char* tam_status_string(int status);
 /*
  * Workspace bytes tam_mass_oracle_prefill prefers for this problem (always a
  * multiple of 256).  Returns 0 for arguments that the call would reject.
- * Per query on the tensor cores, pass 2 writes the mass rows P_i of a chunk of
- * queries to the workspace and selects from them; the preferred size takes every
- * row at once (up to 4 GiB of rows), and any size down to tam_mass_workspace_min()
+ * Per query on the tensor cores, pass 2 selects without writing the mass rows:
+ *   1. a sample pass scores every 2^L-th key of each row (L >= 4, the smallest
+ *      leaving at most 4096 sampled keys per row) and sets the row's threshold
+ *      tau_i = the r-th largest sampled mass, r = ceil(mu + 5 sqrt(mu) + 4) with
+ *      mu = s min(k, i+1) / (i+1) the expected number of sampled keys at or above
+ *      the k-th value among the row's s = (i >> L) + 1 samples (rows of at most
+ *      `cap` keys keep every key: tau_i = -inf);
+ *   2. the scoring pass keeps only the keys with P_i[j] >= tau_i, in nseg
+ *      candidate segments per row (8 on CTA pairs, 4 otherwise) of seg_cap
+ *      entries each, seg_cap = 32 * ceil((ceil(1.5 * 2^L * (r0 + 1) / nseg) + 32)
+ *      / 32), r0 the threshold rank for mu = k / 2^L, cap = nseg * seg_cap;
+ *   3. an exact select runs over each row's candidates; a row whose candidates
+ *      fell short of min(k, i+1) or overflowed a segment is recomputed whole on
+ *      the CUDA cores and selected exactly (the results are the same).
+ * Layout after the status block (256 B) and lse (Hq*N floats, 256-aligned):
+ * tau [N] f32, fallback list [1 + N] i32, counts [N * nseg] i32 (each
+ * 256-aligned), then a region that holds in turn the sample rows of a chunk of
+ * queries, the candidates of a chunk (cap entries of 8 bytes per row) and the
+ * fallback rows' scratch.  The preferred region takes every row at once (and at
+ * least min(N, 148) rows of N floats); any size down to tam_mass_workspace_min()
  * is accepted and only means more chunks.  Otherwise the two sizes are equal.
  */
 size_t tam_mass_oracle_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
@@ -99,8 +116,9 @@ size_t tam_mass_oracle_workspace(int64_t N, int Hq, int Hkv, int d, int dtype, i
 /*
  * Smallest workspace tam_mass_oracle_prefill, tam_mass_select and
  * tam_mass_select_noalloc accept for this problem (a multiple of 256; 0 for
- * arguments the calls would reject).  Per query on the tensor cores that is room
- * for 64 rows of N floats next to the status block and an lse buffer.
+ * arguments the calls would reject).  Per query on the tensor cores the region
+ * then holds the largest of 64 rows of samples, 64 rows of candidates and 64 rows
+ * of N floats (enough for the materialised rows below, and for one fallback row).
  */
 size_t tam_mass_workspace_min(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
                               int block_q);
@@ -118,9 +136,12 @@ size_t tam_mass_workspace_min(int64_t N, int Hq, int Hkv, int d, int dtype, int 
  *   pass 3  (only if out != NULL) for every head h of query i,
  *           out[i,h] = sum_{j in T_i} softmax_{T_i}(scale * q[i,h].k[j,g(h)]) v[j,g(h)],
  *           T_i = S_i (per query) or S_b intersected with [0, i] (block), output in q's dtype.
- * lse may be NULL (then it lives in the workspace).  Per query, the mass rows P_i
- * are materialised in the workspace chunk by chunk (see tam_mass_oracle_workspace);
- * block-shared, only the block sums M_b are.  budget_k in [1, 4096]; block_q in [1, N].
+ * lse may be NULL (then it lives in the workspace).  Per query, no mass row P_i
+ * is written: only the keys at or above a sampled threshold are kept and selected
+ * from (see tam_mass_oracle_workspace); block-shared, only the block sums M_b are
+ * written.  With TAM_MATERIALISE_ROWS=1 in the environment the per-query rows are
+ * written to the workspace region chunk by chunk and selected from there instead
+ * (same results; for A/B comparisons).  budget_k in [1, 4096]; block_q in [1, N].
  * A workspace smaller than tam_mass_workspace_min() gives TAM_ERR_WORKSPACE before
  * anything is enqueued.
  */
@@ -209,9 +230,11 @@ int tam_mass_select_noalloc(int64_t N, int Hq, int Hkv, int d, int dtype, const 
  *                 chosen keys.  Pass 3 on it: tam_sparse_support_attention(block_q).
  * q_idx, k_idx: [N, d_idx] in `dtype` (bf16 or fp32), d_idx in {16, 32, 64, 128}
  * (block_q > 1: d_idx in {64, 128}).
- * On the tensor cores the per-query score rows of a chunk of queries are written to
- * the workspace and selected from; tam_indexer_workspace() is the preferred size (every
- * row at once, up to 4 GiB), tam_indexer_workspace_min() the smallest accepted.
+ * On the tensor cores the per-query selection streams as in tam_mass_oracle_prefill
+ * (sampled thresholds, 4 candidate segments per row, fallback rows on the CUDA cores;
+ * same workspace layout after the status block, with no lse);
+ * tam_indexer_workspace() is the preferred size (every row at once),
+ * tam_indexer_workspace_min() the smallest accepted.
  */
 size_t tam_indexer_workspace(int64_t N, int d_idx, int dtype, int budget_k, int block_q);
 size_t tam_indexer_workspace_min(int64_t N, int d_idx, int dtype, int budget_k, int block_q);
@@ -313,6 +336,19 @@ int tam_dense_gqa_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, i
                                  int dtype, const void* q, const void* k, const void* v,
                                  void* out, float* lse, void* workspace, size_t ws_bytes,
                                  void* stream);
+
+/*
+ * Diagnostics of the streamed per-query selection: how many rows of the last
+ * per-query tam_mass_oracle_prefill / tam_mass_select (or tam_indexer_topk) call
+ * that used `workspace` for this problem went to the fallback path (their sampled
+ * threshold was above the k-th value, or a candidate segment overflowed).  Waits
+ * for `stream`.  Returns -1 for arguments those calls would reject, for problems
+ * that do not stream (CUDA-core path, block_q > 1) and with TAM_MATERIALISE_ROWS=1.
+ */
+int64_t tam_mass_fallback_rows(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
+                               const void* workspace, void* stream);
+int64_t tam_indexer_fallback_rows(int64_t N, int d_idx, int dtype, int budget_k,
+                                  const void* workspace, void* stream);
 
 /*
  * Number of CUDA kernels this library has launched in this process so far (all

@@ -193,6 +193,31 @@ def stress_support(N: int, budget_k: int, seed: int = 7, rows=None):
     return idx, ln
 
 
+def stratified_support(N: int, budget_k: int, seed: int = 7, device="cpu"):
+    """A random support for timing runs at large N, drawn in bulk with torch: row i keeps
+    every key when i + 1 <= k, else one uniform key from each of the k strata
+    [floor(t (i+1) / k), floor((t+1) (i+1) / k)), t = 0..k-1 (distinct, ascending).
+    Returns (idx [N,k] int32, -1 padded; len [N] int32) on `device`."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    idx = torch.empty(N, budget_k, dtype=torch.int32, device=device)
+    ln = torch.clamp(torch.arange(1, N + 1, device=device), max=budget_k).to(torch.int32)
+    t = torch.arange(budget_k, device=device, dtype=torch.int64)
+    chunk = max(1, (1 << 24) // budget_k)
+    for r0 in range(0, N, chunk):
+        i = torch.arange(r0, min(N, r0 + chunk), device=device, dtype=torch.int64)[:, None]
+        n = i + 1
+        lo = (t[None, :] * n) // budget_k
+        hi = ((t[None, :] + 1) * n) // budget_k
+        u = torch.rand(lo.shape, generator=g, device=device, dtype=torch.float64)
+        sel = lo + torch.floor(u * (hi - lo)).to(torch.int64)
+        full = n <= budget_k
+        sel = torch.where(full, t[None, :].expand_as(sel), sel)
+        sel = torch.where(t[None, :] < n, sel, torch.full_like(sel, -1))
+        idx[r0:r0 + len(i)] = sel.to(torch.int32)
+    return idx, ln
+
+
 def sample_rows(N: int, needle_i=(), n_random: int = 256, seed: int = 11) -> np.ndarray:
     """Rows checked at large N: first and last 64, every needle's query, seeded random rows."""
     rng = np.random.default_rng(seed)

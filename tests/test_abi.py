@@ -209,19 +209,48 @@ def test_packed_batch_helpers():
         tam.selection_offsets([0], 1)
 
 
+def _stream_layout(N, k, nseg, head):
+    """The streamed per-query selection's workspace after `head` bytes, as include/tam.h
+    documents it: sample stride 2^L (the smallest L >= 4 leaving at most 4096 sampled
+    keys per row), segment capacity from the threshold rank, then tau, the fallback
+    list, the counts and a region that holds the sample rows, the candidates or the
+    fallback scratch; returns (preferred, minimum) sizes."""
+    import math
+    a256 = lambda x: (x + 255) // 256 * 256              # noqa: E731
+    L = 4
+    while ((N - 1) >> L) + 1 > 4096:
+        L += 1
+    mu = k / (1 << L)
+    r = math.ceil(mu + 5.0 * math.sqrt(mu) + 4.0)
+    per = math.ceil(1.5 * (1 << L) * (r + 1.0) / nseg) + 32
+    seg_cap = (per + 31) // 32 * 32
+    cap = nseg * seg_cap
+    off_region = head + a256(N * 4) + a256((N + 1) * 4) + a256(N * nseg * 4)
+
+    def sample_offset(i):
+        a, b = i >> L, i & ((1 << L) - 1)
+        return i + ((a * (a - 1) // 2) << L) + a * b
+
+    tri = N * (N + 1) // 2
+    pref = max(sample_offset(N) * 4, N * cap * 8, min(N, 148) * N * 4)
+    s_max = ((N - 1) >> L) + 1
+    lo = max(min(N, 64) * s_max * 4, min(N, 64) * cap * 8, min(tri, 64 * N) * 4)
+    return off_region + a256(pref), off_region + a256(lo)
+
+
 @pytest.mark.parametrize("N", [1, 64, 65, 1000, 4096, 32768, 65536])
 def test_workspace_sizes_follow_the_documented_layout(tam_lib, N):
     """Per query on the tensor cores: status block (256 B), lse (Hq*N floats), then the
-    row slab -- every row i (i+1 floats) up to 4 GiB preferred, 64 rows of N floats at
-    least (both capped by the whole triangle)."""
+    streamed selection (thresholds, fallback list, candidate counts and a region sized
+    for every row's candidates at once, at least 64 rows of them)."""
     L = tam_lib.lib()
     Hq, Hkv, d, k = 32, 8, 128, 16
     a256 = lambda x: (x + 255) // 256 * 256              # noqa: E731
-    tri = N * (N + 1) // 2
     head = 256 + a256(Hq * N * 4)
     pref = L.tam_mass_oracle_workspace(N, Hq, Hkv, d, tam_lib.TAM_BF16, k, 1)
     lo = L.tam_mass_workspace_min(N, Hq, Hkv, d, tam_lib.TAM_BF16, k, 1)
-    assert pref == head + a256(min(4 << 30, tri * 4))
-    assert lo == head + a256(min(tri, 64 * N) * 4)
+    want_pref, want_lo = _stream_layout(N, k, 8, head)     # CTA pairs: 8 segments per row
+    assert pref == want_pref
+    assert lo == want_lo
     # the mass-select and no-lse variants share the layout
     assert L.tam_mass_select_workspace(N, Hq, Hkv, d, tam_lib.TAM_BF16, k, 1) == pref

@@ -39,8 +39,13 @@ def run_mass_case(tam, oracle, inp, budget, block_q, rows=None, blocks=None, dty
         oi, ol, _ = oracle.topk_rows(inp.q, inp.k, budget, rows)
         P = oracle.mass_rows(inp.q, inp.k, rows)
         ndiff = check_support(gi[rows], gl[rows], gm[rows], oi, ol, P, MASS_ATOL, "per-query")
+        # pass 3 alone: the oracle on the GPU's own support
         ref, _ = oracle.attn_rows(inp.q, inp.k, inp.v, rows, sup=gi[rows], sup_len=gl[rows])
         check_close(out[rows], ref, OUT_ATOL[dtype], "sparse output")
+        # end to end: the oracle's output on its own support (differs from the line above
+        # only on rows whose supports differ at near-ties)
+        ref_e2e, _ = oracle.attn_rows(inp.q, inp.k, inp.v, rows, sup=oi, sup_len=ol)
+        check_close(out[rows], ref_e2e, OUT_ATOL[dtype], "end-to-end sparse output")
     else:
         nb = -(-N // block_q)
         if blocks is None:
@@ -53,6 +58,9 @@ def run_mass_case(tam, oracle, inp, budget, block_q, rows=None, blocks=None, dty
         r, s, sl = oracle.block_rows_support(gi[blocks], gl[blocks], block_q, N, blocks)
         ref, _ = oracle.attn_rows(inp.q, inp.k, inp.v, r, sup=s, sup_len=sl)
         check_close(out[r], ref, OUT_ATOL[dtype], "block sparse output")
+        r2, s2, sl2 = oracle.block_rows_support(oi, ol, block_q, N, blocks)
+        ref_e2e, _ = oracle.attn_rows(inp.q, inp.k, inp.v, r2, sup=s2, sup_len=sl2)
+        check_close(out[r2], ref_e2e, OUT_ATOL[dtype], "end-to-end block sparse output")
     return ndiff
 
 
@@ -98,7 +106,7 @@ def test_gqa4k_needles_workload(tam_lib, oracle_mod):
 def test_gqa32k_workload_per_query(tam_lib, oracle_mod):
     w = tam_synth.WORKLOADS["gqa32k_2pct"]
     inp = tam_synth.make_inputs(w)
-    rows = tam_synth.sample_rows(w.N, inp.needle_i, n_random=128)
+    rows = tam_synth.sample_rows(w.N, inp.needle_i, n_random=256)
     run_mass_case(tam_lib, oracle_mod, inp, w.budget_k, 1, rows=rows)
 
 
@@ -107,7 +115,7 @@ def test_gqa32k_workload_block_shared(tam_lib, oracle_mod):
     w = tam_synth.WORKLOADS["gqa32k_2pct"]
     inp = tam_synth.make_inputs(w)
     nb = -(-w.N // 64)
-    blocks = tam_synth.sample_blocks(nb, 8)
+    blocks = tam_synth.sample_blocks(nb, 16)
     run_mass_case(tam_lib, oracle_mod, inp, w.budget_k, 64, blocks=blocks)
 
 

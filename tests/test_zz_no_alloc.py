@@ -4,8 +4,11 @@ Such callers (a plugin whose host engine owns all device memory, a process that
 must not cudaMalloc while serving) get the scratch from a static device array in
 the library.  The test calls the entry point through the C ABI twice in a row and
 compares each result with the regular workspace-based entry point, within the
-support/mass tolerance the other parity tests use; it also checks that a problem
-larger than the static scratch is refused before anything runs.  The file sorts
+support/mass tolerance the other parity tests use.  One case per query fits the
+static scratch whole, one is block-shared, and one (N = 8192, k = 1024) prefers
+about 200 MB of workspace, so that inside the 64 MiB it runs in several chunks.  It
+also checks that a problem larger than the static scratch is refused before anything
+runs.  The file sorts
 last so that a run stopping at the first failure has run every other test first.
 """
 import ctypes
@@ -29,15 +32,21 @@ def _noalloc(L, q, k, lse, kb, bq, out):
                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("N,kb,bq", [(2048, 128, 1), (3000, 200, 64)])
-def test_noalloc_matches_workspace_entry_point(tam_lib, N, kb, bq):
-    w = tam_synth.custom("noalloc", N, 32, 8, 128, dtype="bf16", seed=21, sink=True, needles=8)
+@pytest.mark.parametrize("N,Hq,Hkv,kb,bq", [(2048, 32, 8, 128, 1), (3000, 32, 8, 200, 64),
+                                             (8192, 8, 2, 1024, 1)])
+def test_noalloc_matches_workspace_entry_point(tam_lib, N, Hq, Hkv, kb, bq):
+    w = tam_synth.custom("noalloc", N, Hq, Hkv, 128, dtype="bf16", seed=21, sink=True, needles=8)
     inp = tam_synth.make_inputs(w)
     q, k = inp.q.cuda(), inp.k.cuda()
     lse = tam_lib.attention_lse(q, k)
     ref = tam_lib.mass_select(q, k, lse, kb, bq)
     n_sel = N if bq == 1 else -(-N // bq)
     L = tam_lib.lib()
+    if N == 8192:
+        # the regular call's preferred workspace is well above the static scratch, the
+        # smallest one well below it: the no-alloc call runs in chunks
+        assert L.tam_mass_oracle_workspace(N, Hq, Hkv, 128, 0, kb, bq) > 2 * (64 << 20)
+        assert L.tam_mass_workspace_min(N, Hq, Hkv, 128, 0, kb, bq) < (16 << 20)
     for _ in range(2):
         out = (torch.full((n_sel, kb), 7, dtype=torch.int32, device="cuda"),
                torch.full((n_sel,), 7, dtype=torch.int32, device="cuda"),

@@ -48,7 +48,7 @@ EXPORTED = (
     "tam_dense_workspace", "tam_dense_gqa_prefill", "tam_kernel_launches", "tam_check_status",
     "tam_mass_oracle_workspace_varlen", "tam_mass_oracle_prefill_varlen",
     "tam_dense_gqa_prefill_varlen", "tam_indexer_workspace_varlen", "tam_indexer_topk_varlen",
-    "tam_sparse_support_attention_varlen",
+    "tam_sparse_support_attention_varlen", "tam_mass_fallback_rows", "tam_indexer_fallback_rows",
 )
 
 
@@ -137,6 +137,10 @@ def lib() -> ctypes.CDLL:
         L.tam_sparse_support_attention_varlen.restype = i32
         L.tam_sparse_support_attention_varlen.argtypes = [i32, p, i32, i32, i32, i32, p, p, p, p, p,
                                                           i32, i32, p, p, p, sz, p]
+        L.tam_mass_fallback_rows.restype = i64
+        L.tam_mass_fallback_rows.argtypes = [i64, i32, i32, i32, i32, i32, p, p]
+        L.tam_indexer_fallback_rows.restype = i64
+        L.tam_indexer_fallback_rows.argtypes = [i64, i32, i32, i32, p, p]
         L.tam_kernel_launches.restype = ctypes.c_uint64
         L.tam_check_status.restype = i32
         L.tam_check_status.argtypes = [p, p, p]
@@ -158,6 +162,23 @@ def version() -> int:
 def kernel_launches() -> int:
     """Kernels this library has launched in this process (all entry points)."""
     return int(lib().tam_kernel_launches())
+
+
+def mass_fallback_rows(q, k, budget_k: int, workspace, stream=None) -> int:
+    """Rows of the last per-query mass selection in `workspace` (a Workspace or the
+    uint8 tensor a call used) that went to the fallback path; -1 if it does not stream."""
+    N, Hq, Hkv, d = _shape(q, k)
+    t = workspace.get(256) if isinstance(workspace, Workspace) else workspace
+    return int(lib().tam_mass_fallback_rows(N, Hq, Hkv, d, _dtype_code(q), budget_k, _ptr(t),
+                                            _stream(t.device, stream)))
+
+
+def indexer_fallback_rows(q_idx, budget_k: int, workspace, stream=None) -> int:
+    """As mass_fallback_rows, for the last per-query indexer selection."""
+    N, dx = q_idx.shape
+    t = workspace.get(256) if isinstance(workspace, Workspace) else workspace
+    return int(lib().tam_indexer_fallback_rows(N, dx, _dtype_code(q_idx), budget_k, _ptr(t),
+                                               _stream(t.device, stream)))
 
 
 # ------------------------------------------------------------------ marshalling helpers
@@ -270,7 +291,7 @@ def mass_oracle_prefill(q, k, v=None, budget_k: int = 1, block_q: int = 1, *,
     """Attention-mass top-k oracle (passes 1-3) for one causal GQA prefill layer.
 
     workspace_bytes: pass this many workspace bytes instead of the preferred size
-    (at least tam_mass_workspace_min; a smaller slab only means more chunks)."""
+    (at least tam_mass_workspace_min; a smaller workspace only means more chunks)."""
     dev = _dev_of(q, device)
     (q, k, v), host = _to_device([q, k, v], dev)
     N, Hq, Hkv, d = _shape(q, k)

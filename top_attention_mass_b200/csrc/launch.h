@@ -29,6 +29,12 @@ struct MassArgs {
     float* scratch;       // n_ctas * N floats (CUDA-core path)
     float* rows;          // triangular slab of mass rows (tensor-core path, per query)
     int64_t row0, row1;   // the queries whose rows this launch writes (per query)
+    int kst_log2;         // rows mode: only the keys j = m << kst_log2 (sample rows)
+    bool stream;          // per query: threshold-filtered candidates instead of rows
+    const float* tau;     // stream: threshold of every query [N]
+    void* cand;           // stream: candidate segments of the rows [row0, row1)
+    int32_t* cnt;         // stream: appended count per (row, segment)
+    int seg_cap;          // stream: entries per segment
     void* bmass;          // fixed-point block mass (tensor-core path, block-shared)
     int32_t* sup_idx;
     int32_t* sup_len;
@@ -61,6 +67,12 @@ struct IndexerArgs {
     float* scratch;       // n_ctas * N floats (CUDA-core path)
     float* rows;          // triangular slab of score rows (tensor-core path)
     int64_t row0, row1;   // the queries whose rows this launch writes
+    int kst_log2;         // rows mode: only the keys j = m << kst_log2 (sample rows)
+    bool stream;          // threshold-filtered candidates instead of rows
+    const float* tau;
+    void* cand;
+    int32_t* cnt;
+    int seg_cap;
     int32_t* sup_idx;
     int32_t* sup_len;
     float* sup_score;
@@ -82,8 +94,13 @@ cudaError_t tc_mass_pass(const MassArgs& a, cudaStream_t st);
 bool pair_mass_supported(const MassArgs& a);
 cudaError_t pair_mass(const MassArgs& a, cudaStream_t st);
 bool tc_indexer_supported(int64_t N, int d_idx, int dtype, int block_q);
-// Writes the indexer score rows [row0, row1) to the slab (select with row_topk).
+// Writes the indexer score rows [row0, row1) to the slab (select with row_topk), or
+// with a.stream their threshold-filtered candidate segments (select with cand_select).
 cudaError_t tc_indexer_rows(const IndexerArgs& a, cudaStream_t st);
+// Candidate segments per row written by the per-query kernel tc_mass_pass would run
+// for this shape (8 on CTA pairs, 4 on single CTAs; the indexer always 4).
+int tc_mass_segments(const MassArgs& a);
+constexpr int kIndexerSegments = 4;
 
 // Row slabs: row i (i + 1 values) starts tri(i) - tri(row0) floats after the base.
 inline int64_t tri(int64_t i) { return i * (i + 1) / 2; }
@@ -91,6 +108,33 @@ inline int64_t tri(int64_t i) { return i * (i + 1) / 2; }
 // ties toward the smaller index; sup_* are indexed by the absolute row i.
 cudaError_t row_topk(const float* slab, int64_t row0, int64_t row1, int budget, int32_t* sup_idx,
                      int32_t* sup_len, float* sup_val, cudaStream_t st);
+// Rows sampled every 2^L keys: row i' holds (i' >> L) + 1 values; row i starts
+// sample_offset(i, L) - sample_offset(row0, L) floats after the slab base.
+__host__ __device__ inline int64_t sample_offset(int64_t i, int L) {
+    const int64_t a = i >> L, b = i & ((int64_t(1) << L) - 1);
+    return i + ((a * (a - 1) / 2) << L) + a * b;
+}
+// Per-row thresholds from a sample slab: for rows of at most `take_all` keys
+// tau = -inf (every key is a candidate); otherwise the r-th largest of the row's
+// s = (i >> L) + 1 samples, r = ceil(mu + z sqrt(mu) + 4), mu = s min(k, i+1) / (i+1),
+// clamped to [1, s].  `force` (debug): 1 sets tau = +inf, 2 tau = -inf on the
+// sampled rows, so that every such row falls back.
+cudaError_t sample_tau(const float* slab, int64_t row0, int64_t row1, int L, int budget,
+                       int take_all, float z, int force, float* tau, cudaStream_t st);
+// Exact top-min(k, i+1) of each row i in [row0, row1) from its candidate segments
+// (nseg per row, seg_cap entries each, (value bits, key) in key order, counts in cnt),
+// written like row_topk.  A row whose segments overflowed or hold fewer than
+// min(k, i+1) keys is appended to the fallback list fb (fb[0] = count, fb[1 + t] = row)
+// and its outputs are left to the fallback.
+cudaError_t cand_select(const void* cand, const int32_t* cnt, int64_t row0, int64_t row1,
+                        int nseg, int seg_cap, int budget, int32_t* sup_idx, int32_t* sup_len,
+                        float* sup_val, int32_t* fb, cudaStream_t st);
+// The rows on a fallback list, computed whole on the CUDA cores and selected exactly
+// (n_ctas persistent blocks, each with an N-float row of scratch).
+cudaError_t fallback_mass_rows(const MassArgs& a, const int32_t* fb, float* scratch, int n_ctas,
+                               cudaStream_t st);
+cudaError_t fallback_indexer_rows(const IndexerArgs& a, const int32_t* fb, float* scratch,
+                                  int n_ctas, cudaStream_t st);
 // out[r, t] = sum of the ks[t] largest values of support row r (rows of a top-kmax
 // support: val [rows, kmax], len [rows]); nk <= kMaxSweepBudgets, kmax <= 4096.
 constexpr int kMaxSweepBudgets = 16;

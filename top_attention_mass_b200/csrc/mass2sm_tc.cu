@@ -1,8 +1,13 @@
 // Pass 2 on CTA pairs: head-averaged mass and its top-k with 2-SM UMMA.
 //
 //   P_i[j] = (1/Hq) sum_h exp(scale * q[i,h].k[j,g(h)] - lse[h,i]),  j <= i
-//   per query:  the rows P_i, written to a triangular slab for the row top-k;
-//   per block:  M_b[j] = sum_{i in b, j <= i} P_i[j], as in mass_tc.cu
+//   rows:    the rows P_i (or, with a key stride 2^L, their values at the sampled
+//            keys j = m 2^L only), written to a triangular slab;
+//   stream:  per query, only the keys with P_i[j] >= tau_i are kept: each mass warp
+//            appends them to its own segment of the row's candidate buffer, so the
+//            N x N mass never reaches memory (the exact top-k over the candidates
+//            is row_topk.cu's cand_select);
+//   block:   M_b[j] = sum_{i in b, j <= i} P_i[j], as in mass_tc.cu
 //
 // (arXiv 2606.07703, Abstract; gist.science technical report §2.1 "Selektion",
 // "Granularität".)
@@ -24,9 +29,12 @@
 //               column part w / 4 of W / 4 parts, i.e. the (query, head) columns of
 //               that share of the pair's queries; exp2 against the pass-1 LSE, sum
 //               over heads -> mass of those queries for 128 keys.  Several warps per
-//               TMEM lane quarter keep several exp streams per scheduler.  Per query
-//               the mass goes to the row slab (one coalesced 128-byte store per warp
-//               and query); block-shared mass goes to the fixed-point block sums.
+//               TMEM lane quarter keep several exp streams per scheduler.  Rows mode
+//               stores the mass to the row slab (one coalesced 128-byte store per warp
+//               and query); stream mode ballots the keys at or above the query's
+//               threshold and appends them (value, key) to the warp's segment of the
+//               row (a warp-uniform running count, no atomics; segments stay in key
+//               order); block-shared mass goes to the fixed-point block sums.
 // Every wait is bounded; the pair shakes hands before it frees TMEM and exits so
 // that no remote arrive or MMA of one CTA can land after the other left.
 #include "launch.h"
@@ -37,6 +45,7 @@ namespace tam {
 namespace {
 
 constexpr int kStages = 2;
+constexpr int kModeRows = 0, kModeBlock = 1, kModeStream = 2;
 // Mass warps: 8 per query (two per TMEM lane quarter), 16 block-shared (four per
 // quarter; measured 5 % faster there, no gain per query).  Then the TMA producer and
 // the MMA issuer.
@@ -48,17 +57,22 @@ constexpr int kR = 512 / kNQ;           // TMEM accumulator slots
 constexpr int kTileKeys = 256;          // keys per pair tile (128 per CTA)
 
 __host__ __device__ constexpr int pair_smem_bytes(int D, int Hkv) {
-    // Q half + K ring + lse of all 128 columns + barriers
-    return 1024 + Hkv * kHalfRows * D * 2 + kStages * 128 * D * 2 + Hkv * kNQ * 4 + 512;
+    // Q half + K ring + lse of all 128 columns + thresholds + barriers
+    return 1024 + Hkv * kHalfRows * D * 2 + kStages * 128 * D * 2 + Hkv * kNQ * 4 + 128 + 512;
 }
 constexpr int kMaxDynSmem = 227 * 1024;
 
 struct PairParams {
     int N, Hq, Hkv, pair0, n_pairs, block_q;
-    int64_t row0, row1;       // per query: the slab holds rows [row0, row1)
+    int64_t row0, row1;       // per query: the rows [row0, row1) of this launch
+    int kst_log2;             // rows mode: key m of the K map sits at position m << kst_log2
+    int seg_cap;              // stream mode: entries per candidate segment
     float sl2, inv_hq;
     const float* lse;
     float* rows;
+    const float* tau;         // stream mode: threshold of every query [N]
+    uint2* cand;              // stream mode: (value bits, key) of rows [row0, row1)
+    int32_t* cnt;             // stream mode: appended count per (row, segment)
     unsigned long long* bmass;
     int32_t* status;
     uint64_t timeout_ns;
@@ -69,10 +83,18 @@ __host__ __device__ __forceinline__ int64_t bmass_row(int64_t b, int block_q) {
     return (int64_t)block_q * b * (b + 1) / 2;
 }
 
-template <int G, int D, bool BLOCK>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(BLOCK), 1)
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+template <int G, int D, int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads(MODE == kModeBlock), 1)
 k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const PairParams p) {
+    constexpr bool BLOCK = MODE == kModeBlock;
+    constexpr bool STREAM = MODE == kModeStream;
     constexpr int kMassWarps = mass_warps(BLOCK);
     constexpr int kProducerWarp = kMassWarps, kMmaWarp = kMassWarps + 1;
     constexpr int BQP = kNQ / G;              // queries of the pair
@@ -89,7 +111,8 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     uint8_t* sQ = base;
     uint8_t* sK = sQ + Hkv * NH * kQHalf;
     float* sLse = reinterpret_cast<float*>(sK + kStages * kKTile);     // Hkv * 128
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sLse + Hkv * kNQ);
+    float* sTau = sLse + Hkv * kNQ;                                      // 32 (stream)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sTau + 32);
     uint64_t* q_full = bars;                 // CTA 0's counts both CTAs' Q bytes
     uint64_t* k_full = q_full + 1;           // CTA 0's counts both CTAs' K bytes
     uint64_t* k_empty = k_full + kStages;    // both (pair commits)
@@ -107,10 +130,10 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int pt = p.pair0 + p.n_pairs - 1 - (int)(blockIdx.x >> 1);   // heaviest pair first
     const int q0 = pt * BQP;
     const int q_last = min(p.N, q0 + BQP) - 1;
-    const int n_kt = q_last / kTileKeys + 1;
+    const int n_kt = (q_last >> p.kst_log2) / kTileKeys + 1;
     const int n_units = n_kt * Hkv;
     const int my_q0 = q0 + (int)rank * BQC;
-    const int64_t slab0 = p.row0 * (p.row0 + 1) / 2;
+    const int64_t slab0 = sample_offset(p.row0, p.kst_log2);
 
     if (threadIdx.x == 0) {
         tc::mbar_init(q_full, 1);
@@ -132,6 +155,12 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int g = t / kNQ, c = t % kNQ;
         const int i = q0 + c / G, h = g * G + c % G;
         sLse[t] = (i < p.N) ? p.lse[(size_t)h * p.N + i] * kLog2e : INFINITY;
+    }
+    if constexpr (STREAM) {
+        for (int c = threadIdx.x; c < BQP; c += blockDim.x) {
+            const int64_t i = q0 + c;
+            sTau[c] = (i < p.row1) ? p.tau[i] : INFINITY;
+        }
     }
     if (warp == 0) {
         tc::tmem_alloc_pair(tmem_slot, 512);
@@ -217,6 +246,11 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(part * kCols);
         const uint32_t s_empty_leader = tc::map_to_cta(tc::smem_u32(s_empty), 0);
+        // stream mode: this warp's segment of every row and its running counts
+        const int seg = (int)rank * 4 + quarter;
+        int cnt[STREAM ? kQP : 1];
+#pragma unroll
+        for (int q = 0; q < (STREAM ? kQP : 1); ++q) cnt[q] = 0;
         bool ok = true;
         if (p.dbg & kDebugForceTimeout) ok = tc::wait(never, 0, gd, 9);
         for (int kt = 0; ok && kt < n_kt; ++kt) {
@@ -261,17 +295,38 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 }
             }
             if (!ok) break;
-            const int j = kt * kTileKeys + (int)rank * 128 + row;
-            if constexpr (!BLOCK) {
-                // row i of the slab starts tri(i) - tri(row0) floats in; lanes store
+            const int m = kt * kTileKeys + (int)rank * 128 + row;   // key (or sample) index
+            if constexpr (MODE == kModeRows) {
+                // row i of the slab starts off(i) - off(row0) floats in; lanes store
                 // consecutive keys of one query
+                const int64_t j = (int64_t)m << p.kst_log2;
 #pragma unroll
                 for (int ql = 0; ql < kQP; ++ql) {
                     const int64_t i = q0 + part * kQP + ql;
                     if (j <= i && i >= p.row0 && i < p.row1)
-                        p.rows[i * (i + 1) / 2 - slab0 + j] = acc[ql] * p.inv_hq;
+                        p.rows[sample_offset(i, p.kst_log2) - slab0 + m] = acc[ql] * p.inv_hq;
+                }
+            } else if constexpr (STREAM) {
+                // keys at or above the query's threshold, appended in key order to this
+                // warp's segment (positions past the capacity are only counted)
+                const uint32_t lt = lanemask_lt();
+#pragma unroll
+                for (int ql = 0; ql < kQP; ++ql) {
+                    const int qi = part * kQP + ql;
+                    const int64_t i = q0 + qi;
+                    const float v = acc[ql] * p.inv_hq;
+                    const bool pass = m <= i && i < p.row1 && v >= sTau[qi];
+                    const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+                    if (bal != 0u) {
+                        const int pos = cnt[ql] + __popc(bal & lt);
+                        if (pass && pos < p.seg_cap)
+                            p.cand[((i - p.row0) * 8 + seg) * (int64_t)p.seg_cap + pos] =
+                                make_uint2(__float_as_uint(v), (uint32_t)m);
+                        cnt[ql] += __popc(bal);
+                    }
                 }
             } else {
+                const int j = m;
                 const int qh = q0 + part * kQP;
                 int cur_b = qh / p.block_q;
                 float sum = 0.f;
@@ -295,6 +350,15 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                               (unsigned long long)__float2ll_rn(sum * p.inv_hq * 1099511627776.0f));
             }
         }
+        if constexpr (STREAM) {
+            if (ok && lane == 0) {
+#pragma unroll
+                for (int ql = 0; ql < kQP; ++ql) {
+                    const int64_t i = q0 + part * kQP + ql;
+                    if (i < p.row1) p.cnt[(i - p.row0) * 8 + seg] = cnt[ql];
+                }
+            }
+        }
     }
     // every CTA waits for the pair MMAs (they write into both CTAs' TMEM)
     if (threadIdx.x == 0) tc::wait(mma_done, 0, drain, 0);
@@ -311,13 +375,19 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     }
 }
 
-template <int G, int D, bool BLOCK>
+template <int G, int D, int MODE>
 cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
+    constexpr bool BLOCK = MODE == kModeBlock;
     constexpr int BQP = kNQ / G, BQC = kHalfRows / G;
     CUtensorMap tq, tk;
     const uint64_t d = a.d;
+    // rows mode with a key stride reads every 2^L-th key row: the same K with an L-fold
+    // longer row pitch and (N - 1) >> L + 1 rows
+    const int L = MODE == kModeRows ? a.kst_log2 : 0;
+    const uint64_t n_keys = (uint64_t)((a.N - 1) >> L) + 1;
     if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQC) ||
-        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, a.N, d * 2, (uint64_t)a.Hkv * d * 2, 64, 1, 128))
+        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, n_keys, d * 2, ((uint64_t)a.Hkv * d * 2) << L, 64,
+                           1, 128))
         return cudaErrorInvalidValue;
     PairParams p{};
     p.N = (int)a.N;
@@ -329,18 +399,23 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     p.n_pairs = (int)((r1 + BQP - 1) / BQP) - p.pair0;
     p.row0 = r0;
     p.row1 = r1;
+    p.kst_log2 = L;
+    p.seg_cap = a.seg_cap;
     p.block_q = a.block_q;
     p.sl2 = a.sl2;
     p.inv_hq = 1.f / (float)a.Hq;
     p.lse = a.lse;
     p.rows = a.rows;
+    p.tau = a.tau;
+    p.cand = reinterpret_cast<uint2*>(a.cand);
+    p.cnt = a.cnt;
     p.bmass = reinterpret_cast<unsigned long long*>(a.bmass);
     p.status = a.status;
     p.timeout_ns = wait_timeout_ns();
     p.dbg = debug_flags();
     if (p.n_pairs <= 0) return cudaSuccess;
     const int smem = pair_smem_bytes(D, a.Hkv);
-    auto kern = k_mass_pair<G, D, BLOCK>;
+    auto kern = k_mass_pair<G, D, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     if (BLOCK) {
@@ -353,14 +428,20 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-template <int D, bool BLOCK>
+template <int D, int MODE>
 cudaError_t dispatch_g(const MassArgs& a, cudaStream_t st) {
     switch (a.Hq / a.Hkv) {
-        case 4: return launch_pair<4, D, BLOCK>(a, st);
-        case 8: return launch_pair<8, D, BLOCK>(a, st);
-        case 16: return launch_pair<16, D, BLOCK>(a, st);
+        case 4: return launch_pair<4, D, MODE>(a, st);
+        case 8: return launch_pair<8, D, MODE>(a, st);
+        case 16: return launch_pair<16, D, MODE>(a, st);
         default: return cudaErrorNotSupported;
     }
+}
+
+template <int D>
+cudaError_t dispatch_mode(const MassArgs& a, cudaStream_t st) {
+    if (a.block_q > 1) return dispatch_g<D, kModeBlock>(a, st);
+    return a.stream ? dispatch_g<D, kModeStream>(a, st) : dispatch_g<D, kModeRows>(a, st);
 }
 
 }  // namespace
@@ -373,12 +454,11 @@ bool pair_mass_supported(const MassArgs& a) {
     return pair_smem_bytes(a.d, a.Hkv) <= kMaxDynSmem;
 }
 
-// Launches the pair kernel only: per query it fills the slab rows [row0, row1); per
-// block the caller runs the block top-k after it.
+// Launches the pair kernel only: per query it fills the slab rows [row0, row1) (rows
+// mode) or their candidate segments (stream mode); per block the caller runs the
+// block top-k after it.
 cudaError_t pair_mass(const MassArgs& a, cudaStream_t st) {
-    const bool block = a.block_q > 1;
-    if (a.d == 64) return block ? dispatch_g<64, true>(a, st) : dispatch_g<64, false>(a, st);
-    return block ? dispatch_g<128, true>(a, st) : dispatch_g<128, false>(a, st);
+    return a.d == 64 ? dispatch_mode<64>(a, st) : dispatch_mode<128>(a, st);
 }
 
 }  // namespace tam

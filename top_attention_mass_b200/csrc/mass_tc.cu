@@ -1,10 +1,14 @@
 // Pass 2 on the tensor cores: head-averaged token mass (and the indexer's scores).
 //
 //   P_i[j] = (1/Hq) sum_h exp(scale * q[i,h].k[j,g(h)] - lse[h,i]),  j <= i
-//   per query:  the rows P_i, written to a triangular slab; row_topk.cu then
-//               selects S_i = top-min(k, i+1) of each row (value desc, index asc)
+//   per query:  the rows P_i, written to a triangular slab (with a key stride 2^L
+//               only the sampled keys j = m 2^L); row_topk.cu then selects
+//               S_i = top-min(k, i+1) of each row (value desc, index asc);
+//               or, streamed, only the keys with P_i[j] >= tau_i, appended to the
+//               row's candidate segments (one per mass warp) for cand_select
 //   per block:  M_b[j] = sum_{i in block b, i >= j} P_i[j]  -> top-k in k_block_select
-//   indexer:    the rows s_i[j] = q_idx[i] . k_idx[j] (one head, no exponentials)
+//   indexer:    the rows s_i[j] = q_idx[i] . k_idx[j] (one head, no exponentials),
+//               as rows, sample rows or streamed candidates like the mass
 //
 // (arXiv 2606.07703, Abstract: "selects head-averaged token support"; gist.science
 // technical report §2.1, "Mechanismus", "Selektion" and "Granularität", §2.2 for
@@ -22,8 +26,10 @@
 //   warps 0-3   mass warps: thread = key row; exp2 against the pass-1 LSE, sum over
 //               heads -> mass of BQ queries; causal mask; then either the mass goes
 //               to the row slab (per query, indexer: lanes store consecutive keys of
-//               one query) or the block column sum is added in 2^-40 fixed point
-//               (block-shared).
+//               one query), or the keys at or above the query's threshold are
+//               appended to warp w's segment of the row (streamed: a warp ballot and
+//               a warp-uniform running count, no atomics), or the block column sum
+//               is added in 2^-40 fixed point (block-shared).
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
@@ -34,22 +40,29 @@ namespace {
 constexpr int kStages = 2;
 constexpr int kThreads = 32 * 6;
 
-// Kernel modes: head-averaged mass rows, block-shared mass sums, or the
-// head-collapsed indexer's score rows (one score per (query, key), no exponentials).
-constexpr int kModeQuery = 0, kModeBlock = 1, kModeIndexer = 2;
+// Kernel modes: head-averaged mass rows, block-shared mass sums, the
+// head-collapsed indexer's score rows (one score per (query, key), no exponentials),
+// and the streamed (threshold-filtered) forms of the mass and indexer rows.
+constexpr int kModeQuery = 0, kModeBlock = 1, kModeIndexer = 2, kModeQueryStream = 3,
+              kModeIndexerStream = 4;
 
-// alignment slack + Q (all groups) + K ring + lse2 + barriers
+// alignment slack + Q (all groups) + K ring + lse2 + thresholds + barriers
 __host__ __device__ constexpr int mass_smem_bytes(int NQ, int D, int Hkv) {
-    return 1024 + Hkv * NQ * D * 2 + kStages * 128 * D * 2 + Hkv * NQ * 4 + 512;
+    return 1024 + Hkv * NQ * D * 2 + kStages * 128 * D * 2 + Hkv * NQ * 4 + 128 + 512;
 }
 constexpr int kMaxDynSmem = 227 * 1024;
 
 struct MassParams {
     int N, Hq, Hkv, ct0, n_ctiles, block_q;
-    int64_t row0, row1;              // per query / indexer: the slab holds rows [row0, row1)
+    int64_t row0, row1;              // per query / indexer: the rows [row0, row1)
+    int kst_log2;                    // rows modes: key m of the K map is at m << kst_log2
+    int seg_cap;                     // stream modes: entries per candidate segment
     float sl2, inv_hq;
     const float* lse;
     float* rows;                     // triangular row slab (per query / indexer)
+    const float* tau;                // stream modes: threshold of every query [N]
+    uint2* cand;                     // stream modes: (value bits, key) of rows [row0, row1)
+    int32_t* cnt;                    // stream modes: appended count per (row, segment)
     unsigned long long* bmass;       // triangular block mass (block mode)
     int32_t* status;
     uint64_t timeout_ns;
@@ -72,7 +85,8 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     constexpr uint32_t kKHalf = 128 * 128;
     constexpr uint32_t kKTile = NH * kKHalf;
     constexpr bool BLOCK = MODE == kModeBlock;
-    constexpr bool INDEXER = MODE == kModeIndexer;
+    constexpr bool INDEXER = MODE == kModeIndexer || MODE == kModeIndexerStream;
+    constexpr bool STREAM = MODE == kModeQueryStream || MODE == kModeIndexerStream;
     const int Hkv = p.Hkv;
 
     extern __shared__ uint8_t smem_raw[];
@@ -81,7 +95,8 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     uint8_t* sQ = base;                                   // Hkv * NH * kQHalf
     uint8_t* sK = sQ + Hkv * NH * kQHalf;                 // kStages * kKTile
     float* sLse = reinterpret_cast<float*>(sK + kStages * kKTile);   // Hkv * NQ
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sLse + Hkv * NQ);
+    float* sTau = sLse + Hkv * NQ;                                   // 32 (stream)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sTau + 32);
     uint64_t* q_full = bars;
     uint64_t* k_full = q_full + 1;
     uint64_t* k_empty = k_full + kStages;
@@ -96,9 +111,9 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int ct = p.ct0 + p.n_ctiles - 1 - (int)blockIdx.x;   // heaviest tile first
     const int q0 = ct * BQ;
     const int q_last = min(p.N, q0 + BQ) - 1;
-    const int n_kt = q_last / 128 + 1;
+    const int n_kt = (q_last >> p.kst_log2) / 128 + 1;
     const int n_units = n_kt * Hkv;
-    const int64_t slab0 = p.row0 * (p.row0 + 1) / 2;
+    const int64_t slab0 = sample_offset(p.row0, p.kst_log2);
 
     if (threadIdx.x == 0) {
         tc::mbar_init(q_full, 1);
@@ -121,6 +136,12 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             const int g = t / NQ, c = t % NQ;
             const int i = q0 + c / G, h = g * G + c % G;
             sLse[t] = (i < p.N) ? p.lse[(size_t)h * p.N + i] * kLog2e : INFINITY;
+        }
+    }
+    if constexpr (STREAM) {
+        for (int c = threadIdx.x; c < BQ; c += blockDim.x) {
+            const int64_t i = q0 + c;
+            sTau[c] = (i < p.row1) ? p.tau[i] : INFINITY;
         }
     }
     if (warp == 0) {
@@ -197,6 +218,10 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         // ---------------------------------------------------------------- mass warps
         const int row = threadIdx.x;                       // key row of the tile
         const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        // stream modes: warp w writes segment w of every row, with running counts
+        int cnt[STREAM ? BQ : 1];
+#pragma unroll
+        for (int q = 0; q < (STREAM ? BQ : 1); ++q) cnt[q] = 0;
         bool ok = true;
         if (p.dbg & kDebugForceTimeout) ok = tc::wait(never, 0, gd, 9);
         for (int kt = 0; ok && kt < n_kt; ++kt) {
@@ -245,15 +270,36 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 tc::mbar_arrive(&s_empty[slot]);
             }
             if (!ok) break;
-            const int j = kt * 128 + row;
-            if constexpr (!BLOCK) {
-                // row i of the slab starts tri(i) - tri(row0) floats in; lanes store
-                // consecutive keys of one query
+            const int j = kt * 128 + row;                     // key (or sample) index
+            if constexpr (STREAM) {
+                // keys at or above the query's threshold, appended in key order to this
+                // warp's segment (positions past the capacity are only counted)
+                uint32_t lt;
+                asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt));
 #pragma unroll
                 for (int q = 0; q < BQ; ++q) {
                     const int64_t i = q0 + q;
-                    if (j <= i && i >= p.row0 && i < p.row1)
-                        p.rows[i * (i + 1) / 2 - slab0 + j] = INDEXER ? acc[q] : acc[q] * p.inv_hq;
+                    const float v = INDEXER ? acc[q] : acc[q] * p.inv_hq;
+                    const bool pass = j <= i && i < p.row1 && v >= sTau[q];
+                    const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+                    if (bal != 0u) {
+                        const int pos = cnt[q] + __popc(bal & lt);
+                        if (pass && pos < p.seg_cap)
+                            p.cand[((i - p.row0) * 4 + warp) * (int64_t)p.seg_cap + pos] =
+                                make_uint2(__float_as_uint(v), (uint32_t)j);
+                        cnt[q] += __popc(bal);
+                    }
+                }
+            } else if constexpr (!BLOCK) {
+                // row i of the slab starts off(i) - off(row0) floats in; lanes store
+                // consecutive keys of one query
+                const int64_t jp = (int64_t)j << p.kst_log2;  // key position
+#pragma unroll
+                for (int q = 0; q < BQ; ++q) {
+                    const int64_t i = q0 + q;
+                    if (jp <= i && i >= p.row0 && i < p.row1)
+                        p.rows[sample_offset(i, p.kst_log2) - slab0 + j] =
+                            INDEXER ? acc[q] : acc[q] * p.inv_hq;
                 }
             } else {
                 // block column sums, 2^-40 fixed point, one add per (block, key)
@@ -278,6 +324,15 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (part > 0.f)
                     atomicAdd(&p.bmass[bmass_offset(cur_b, p.block_q) + j],
                               (unsigned long long)__float2ll_rn(part * p.inv_hq * 1099511627776.0f));
+            }
+        }
+        if constexpr (STREAM) {
+            if (ok && lane == 0) {
+#pragma unroll
+                for (int q = 0; q < BQ; ++q) {
+                    const int64_t i = q0 + q;
+                    if (i < p.row1) p.cnt[(i - p.row0) * 4 + warp] = cnt[q];
+                }
             }
         }
     }
@@ -372,10 +427,16 @@ template <int G, int D, int NQ, int MODE>
 cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     constexpr int BQ = NQ / G;
     constexpr bool BLOCK = MODE == kModeBlock;
+    constexpr bool ROWS = MODE == kModeQuery || MODE == kModeIndexer;
     CUtensorMap tq, tk;
     const uint64_t d = a.d;
+    // rows modes with a key stride read every 2^L-th key row: the same K with an
+    // L-fold longer row pitch and (N - 1) >> L + 1 rows
+    const int L = ROWS ? a.kst_log2 : 0;
+    const uint64_t n_keys = (uint64_t)((a.N - 1) >> L) + 1;
     if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQ) ||
-        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, a.N, d * 2, (uint64_t)a.Hkv * d * 2, 64, 1, 128))
+        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, n_keys, d * 2, ((uint64_t)a.Hkv * d * 2) << L, 64,
+                           1, 128))
         return cudaErrorInvalidValue;
     MassParams p{};
     p.N = (int)a.N;
@@ -388,11 +449,16 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     p.n_ctiles = (int)((r1 + BQ - 1) / BQ) - p.ct0;
     p.row0 = r0;
     p.row1 = r1;
+    p.kst_log2 = L;
+    p.seg_cap = a.seg_cap;
     p.block_q = a.block_q;
     p.sl2 = a.sl2;
     p.inv_hq = 1.f / (float)a.Hq;
     p.lse = a.lse;
     p.rows = a.rows;
+    p.tau = a.tau;
+    p.cand = reinterpret_cast<uint2*>(a.cand);
+    p.cnt = a.cnt;
     p.bmass = reinterpret_cast<unsigned long long*>(a.bmass);
     p.status = a.status;
     p.timeout_ns = wait_timeout_ns();
@@ -456,6 +522,9 @@ cudaError_t dispatch(const MassArgs& a, cudaStream_t st) {
 
 // The indexer runs as a single-head problem: Hq = Hkv = 1, d = d_idx, 32 queries per CTA.
 cudaError_t launch_indexer_tc(const MassArgs& a, cudaStream_t st) {
+    if (a.stream)
+        return a.d == 64 ? launch_mass<1, 64, 32, kModeIndexerStream>(a, st)
+                         : launch_mass<1, 128, 32, kModeIndexerStream>(a, st);
     return a.d == 64 ? launch_mass<1, 64, 32, kModeIndexer>(a, st)
                      : launch_mass<1, 128, 32, kModeIndexer>(a, st);
 }
@@ -501,7 +570,12 @@ cudaError_t tc_mass_pass(const MassArgs& a, cudaStream_t st) {
         note_launch();
         return cudaGetLastError();
     }
-    return a.block_q == 1 ? dispatch<kModeQuery>(a, st) : dispatch<kModeBlock>(a, st);
+    if (a.block_q > 1) return dispatch<kModeBlock>(a, st);
+    return a.stream ? dispatch<kModeQueryStream>(a, st) : dispatch<kModeQuery>(a, st);
+}
+
+int tc_mass_segments(const MassArgs& a) {
+    return (pair_mass_supported(a) && !pair_path_disabled()) ? 8 : 4;
 }
 
 bool tc_indexer_supported(int64_t N, int d_idx, int dtype, int block_q) {
@@ -522,6 +596,12 @@ cudaError_t tc_indexer_rows(const IndexerArgs& ia, cudaStream_t st) {
     a.rows = ia.rows;
     a.row0 = ia.row0;
     a.row1 = ia.row1;
+    a.kst_log2 = ia.kst_log2;
+    a.stream = ia.stream;
+    a.tau = ia.tau;
+    a.cand = ia.cand;
+    a.cnt = ia.cnt;
+    a.seg_cap = ia.seg_cap;
     a.status = ia.status;
     return launch_indexer_tc(a, st);
 }

@@ -446,7 +446,201 @@ __global__ void __launch_bounds__(kRtThreads, 6) k_row_topk(const RowTopkParams 
     if (threadIdx.x == 0) p.sup_len[i] = k;
 }
 
+// ---------------------------------------------------------------- streamed selection
+// Threshold of each row from its sampled keys (a lower bound of the row's k-th
+// value unless the samples are z deviations off; cand_select checks it).
+struct SampleTauParams {
+    const float* slab;
+    int64_t row0;
+    int n_rows, L, budget, take_all, force;
+    float z;
+    float* tau;
+};
+
+__global__ void __launch_bounds__(kRtThreads) k_sample_tau(const SampleTauParams p) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    RowSmem& s = *reinterpret_cast<RowSmem*>(smem_raw);
+    const int64_t i = p.row0 + (p.n_rows - 1 - (int)blockIdx.x);
+    const int n = (int)i + 1;
+    if (n <= p.take_all) {
+        if (threadIdx.x == 0) p.tau[i] = -INFINITY;
+        return;
+    }
+    if (p.force) {
+        if (threadIdx.x == 0) p.tau[i] = p.force == 1 ? INFINITY : -INFINITY;
+        return;
+    }
+    const int ns = (int)(i >> p.L) + 1;
+    const float* row = p.slab + (sample_offset(i, p.L) - sample_offset(p.row0, p.L));
+    if (threadIdx.x == 0) {
+        s.ckey = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowSmem));
+        s.cmax = 0u;
+        s.scal[3] = -1;                       // smallest key, as ~x to use atomicMax
+    }
+    __syncthreads();
+    uint32_t mx = 0u, mn = 0xffffffffu;
+    for (int t = threadIdx.x; t < ns; t += blockDim.x) {
+        const uint32_t kv = okey(__ldg(row + t));
+        s.ckey[t] = kv;
+        mx = max(mx, kv);
+        mn = min(mn, kv);
+    }
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    mn = __reduce_min_sync(0xffffffffu, mn);
+    if ((threadIdx.x & 31) == 0) {
+        atomicMax(&s.cmax, mx);
+        atomicMin(reinterpret_cast<unsigned int*>(&s.scal[3]), mn);
+    }
+    __syncthreads();
+    const int k = min(p.budget, n);
+    const float mu = (float)ns * (float)k / (float)n;
+    const int r = max(1, min(ns, (int)ceilf(mu + p.z * sqrtf(mu) + 4.f)));
+    uint32_t T;
+    int take_eq;
+    cand_kth(s, ns, r, (uint32_t)s.scal[3], T, take_eq);
+    if (threadIdx.x == 0) p.tau[i] = oval(T);
+}
+
+// Exact top-k of a row from its candidate segments.  Each segment was written by
+// one warp in key order, so a key's rank in the merged row is its position in its
+// own segment plus, in every other segment, the number of keys below it (binary
+// search); the merged candidates then go through the same k-th key search and
+// ordered emission as the materialised rows.
+struct CandSelParams {
+    const uint2* cand;
+    const int32_t* cnt;
+    int64_t row0;
+    int n_rows, nseg, seg_cap, budget;
+    int32_t* sup_idx;
+    int32_t* sup_len;
+    float* sup_val;
+    int32_t* fb;
+};
+
+constexpr int kMaxSegments = 8;
+
+__global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams p) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    RowSmem& s = *reinterpret_cast<RowSmem*>(smem_raw);
+    __shared__ int soff[kMaxSegments + 1];
+    __shared__ int sflag;
+    const int64_t i = p.row0 + (p.n_rows - 1 - (int)blockIdx.x);
+    const int n = (int)i + 1;
+    const int k = min(p.budget, n);
+    const int cap = p.nseg * p.seg_cap;
+    uint32_t* akey = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowSmem)) + 2 * cap;
+    int32_t* aidx = reinterpret_cast<int32_t*>(akey + cap);
+    if (threadIdx.x == 0) {
+        s.ckey = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowSmem));
+        s.cidx = reinterpret_cast<int32_t*>(s.ckey + cap);
+        s.cmax = 0u;
+        s.scal[3] = -1;
+        const int32_t* c = p.cnt + (i - p.row0) * p.nseg;
+        int tot = 0;
+        bool bad = false;
+        for (int g = 0; g < p.nseg; ++g) {
+            const int cg = c[g];
+            bad = bad || cg < 0 || cg > p.seg_cap;
+            soff[g] = tot;
+            tot += max(0, min(cg, p.seg_cap));
+        }
+        soff[p.nseg] = tot;
+        // overflowed segments lost keys; fewer than k keys means the threshold was
+        // above the k-th value: either way the row goes to the fallback
+        sflag = bad || tot < k;
+        if (sflag) {
+            const int t = atomicAdd(p.fb, 1);
+            p.fb[1 + t] = (int32_t)i;
+        }
+    }
+    __syncthreads();
+    if (sflag) return;
+    const int tot = soff[p.nseg];
+    // load the segments back to back
+    const uint2* base = p.cand + (i - p.row0) * (int64_t)cap;
+    uint32_t mx = 0u, mn = 0xffffffffu;
+    for (int t = threadIdx.x; t < tot; t += blockDim.x) {
+        int g = 0;
+        while (g + 1 < p.nseg && soff[g + 1] <= t) ++g;
+        const uint2 e = base[g * p.seg_cap + (t - soff[g])];
+        const uint32_t kv = okey(__uint_as_float(e.x));
+        akey[t] = kv;
+        aidx[t] = (int32_t)e.y;
+        mx = max(mx, kv);
+        mn = min(mn, kv);
+    }
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    mn = __reduce_min_sync(0xffffffffu, mn);
+    if ((threadIdx.x & 31) == 0) {
+        atomicMax(&s.cmax, mx);
+        atomicMin(reinterpret_cast<unsigned int*>(&s.scal[3]), mn);
+    }
+    __syncthreads();
+    // merge: rank = own position + keys below it in every other segment
+    for (int t = threadIdx.x; t < tot; t += blockDim.x) {
+        int g = 0;
+        while (g + 1 < p.nseg && soff[g + 1] <= t) ++g;
+        const int32_t x = aidx[t];
+        int rank = t - soff[g];
+        for (int h = 0; h < p.nseg; ++h) {
+            if (h == g) continue;
+            int lo = soff[h], hi = soff[h + 1];
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (aidx[mid] < x) lo = mid + 1; else hi = mid;
+            }
+            rank += lo - soff[h];
+        }
+        s.ckey[rank] = akey[t];
+        s.cidx[rank] = x;
+    }
+    const uint32_t G = (uint32_t)s.scal[3];
+    __syncthreads();
+    int32_t* oi = p.sup_idx + i * (int64_t)p.budget;
+    float* ov = p.sup_val + i * (int64_t)p.budget;
+    uint32_t T = 0u;
+    int take_eq = 0;
+    if (tot > k) cand_kth(s, tot, k, G, T, take_eq);   // else every candidate is kept
+    const CandSrc cs{&s};
+    int dummy;
+    seg_count<CandSrc, false>(cs, tot, T, s, dummy, dummy);
+    seg_emit<CandSrc>(cs, tot, T, take_eq, s, oi, ov);
+    for (int t = k + threadIdx.x; t < p.budget; t += blockDim.x) {
+        oi[t] = -1;
+        ov[t] = 0.f;
+    }
+    if (threadIdx.x == 0) p.sup_len[i] = k;
+}
+
 }  // namespace
+
+cudaError_t sample_tau(const float* slab, int64_t row0, int64_t row1, int L, int budget,
+                       int take_all, float z, int force, float* tau, cudaStream_t st) {
+    if (row1 <= row0) return cudaSuccess;
+    SampleTauParams p{slab, row0, (int)(row1 - row0), L, budget, take_all, force, z, tau};
+    const int max_samples = (int)((row1 - 1) >> L) + 1;
+    const int smem = (int)sizeof(RowSmem) + max_samples * 4;
+    cudaError_t e = cudaFuncSetAttribute(k_sample_tau, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k_sample_tau<<<(unsigned)(row1 - row0), kRtThreads, smem, st>>>(p);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t cand_select(const void* cand, const int32_t* cnt, int64_t row0, int64_t row1,
+                        int nseg, int seg_cap, int budget, int32_t* sup_idx, int32_t* sup_len,
+                        float* sup_val, int32_t* fb, cudaStream_t st) {
+    if (row1 <= row0) return cudaSuccess;
+    if (nseg < 1 || nseg > kMaxSegments) return cudaErrorInvalidValue;
+    CandSelParams p{reinterpret_cast<const uint2*>(cand), cnt, row0, (int)(row1 - row0), nseg,
+                    seg_cap, budget, sup_idx, sup_len, sup_val, fb};
+    const int smem = (int)sizeof(RowSmem) + nseg * seg_cap * 16;
+    cudaError_t e = cudaFuncSetAttribute(k_cand_select, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k_cand_select<<<(unsigned)(row1 - row0), kRtThreads, smem, st>>>(p);
+    note_launch();
+    return cudaGetLastError();
+}
 
 cudaError_t row_topk(const float* slab, int64_t row0, int64_t row1, int budget, int32_t* sup_idx,
                      int32_t* sup_len, float* sup_val, cudaStream_t st) {

@@ -190,6 +190,74 @@ __global__ void __launch_bounds__(256) k_indexer_select_simt(
     }
 }
 
+// ---------------------------------------------------------------- fallback rows
+// Rows whose streamed candidates could not be used (a threshold above the k-th value,
+// or a full candidate segment): each persistent block takes rows off the list
+// fb (fb[0] = count, fb[1 + t] = row), computes the whole row into its scratch row
+// and selects from it exactly.
+template <typename T>
+__global__ void __launch_bounds__(256) k_mass_rows_fallback(
+    const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ lse, int N, int Hq,
+    int Hkv, int d, float sl2, int budget, const int32_t* __restrict__ fb,
+    float* __restrict__ scratch, int32_t* __restrict__ sup_idx, int32_t* __restrict__ sup_len,
+    float* __restrict__ sup_mass) {
+    extern __shared__ float smem[];
+    __shared__ SelectSmem sel;
+    float* qs = smem;              // Hq * d
+    float* lse2 = smem + Hq * d;   // Hq
+    float* row = scratch + (size_t)blockIdx.x * N;
+    const int G = Hq / Hkv;
+    const float inv_hq = 1.f / (float)Hq;
+    const int n_fb = fb[0];
+    for (int t = blockIdx.x; t < n_fb; t += gridDim.x) {
+        const int i = fb[1 + t];
+        __syncthreads();
+        for (int x = threadIdx.x; x < Hq * d; x += blockDim.x) qs[x] = to_f(q[(size_t)i * Hq * d + x]);
+        for (int h = threadIdx.x; h < Hq; h += blockDim.x) lse2[h] = lse[(size_t)h * N + i] * kLog2e;
+        __syncthreads();
+        for (int j = threadIdx.x; j <= i; j += blockDim.x) {
+            float p = 0.f;
+            for (int h = 0; h < Hq; ++h) {
+                const T* kj = k + ((size_t)j * Hkv + h / G) * d;
+                const float* qh = qs + h * d;
+                float sc = 0.f;
+                for (int c = 0; c < d; ++c) sc = fmaf(qh[c], to_f(kj[c]), sc);
+                p += exp2f(sc * sl2 - lse2[h]);
+            }
+            row[j] = p * inv_hq;
+        }
+        __syncthreads();
+        block_select_topk(row, i + 1, budget, sup_idx + (size_t)i * budget,
+                          sup_mass + (size_t)i * budget, sup_len + i, sel);
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_indexer_rows_fallback(
+    const T* __restrict__ qx, const T* __restrict__ kx, int dx, int budget,
+    const int32_t* __restrict__ fb, int N, float* __restrict__ scratch,
+    int32_t* __restrict__ sup_idx, int32_t* __restrict__ sup_len, float* __restrict__ sup_score) {
+    extern __shared__ float qs[];   // dx
+    __shared__ SelectSmem sel;
+    float* row = scratch + (size_t)blockIdx.x * N;
+    const int n_fb = fb[0];
+    for (int t = blockIdx.x; t < n_fb; t += gridDim.x) {
+        const int i = fb[1 + t];
+        __syncthreads();
+        for (int c = threadIdx.x; c < dx; c += blockDim.x) qs[c] = to_f(qx[(size_t)i * dx + c]);
+        __syncthreads();
+        for (int j = threadIdx.x; j <= i; j += blockDim.x) {
+            const T* kj = kx + (size_t)j * dx;
+            float sc = 0.f;
+            for (int c = 0; c < dx; ++c) sc = fmaf(qs[c], to_f(kj[c]), sc);
+            row[j] = sc;
+        }
+        __syncthreads();
+        block_select_topk(row, i + 1, budget, sup_idx + (size_t)i * budget,
+                          sup_score + (size_t)i * budget, sup_len + i, sel);
+    }
+}
+
 // ---------------------------------------------------------------- launchers
 template <typename T>
 static cudaError_t launch_lse(const LseArgs& a, cudaStream_t st) {
@@ -263,6 +331,46 @@ static cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t st) {
 
 cudaError_t simt_indexer_select(const IndexerArgs& a, cudaStream_t st) {
     return a.dtype == TAM_F32 ? launch_indexer<float>(a, st) : launch_indexer<__nv_bfloat16>(a, st);
+}
+
+template <typename T>
+static cudaError_t launch_mass_fallback(const MassArgs& a, const int32_t* fb, float* scratch,
+                                        int n_ctas, cudaStream_t st) {
+    const size_t smem = (size_t)(a.Hq * a.d + a.Hq) * sizeof(float);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_mass_rows_fallback<T>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    k_mass_rows_fallback<T><<<n_ctas, 256, smem, st>>>(
+        (const T*)a.q, (const T*)a.k, a.lse, (int)a.N, a.Hq, a.Hkv, a.d, a.sl2, a.budget, fb,
+        scratch, a.sup_idx, a.sup_len, a.sup_mass);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t fallback_mass_rows(const MassArgs& a, const int32_t* fb, float* scratch, int n_ctas,
+                               cudaStream_t st) {
+    if (n_ctas < 1) return cudaErrorInvalidValue;
+    return a.dtype == TAM_F32 ? launch_mass_fallback<float>(a, fb, scratch, n_ctas, st)
+                              : launch_mass_fallback<__nv_bfloat16>(a, fb, scratch, n_ctas, st);
+}
+
+template <typename T>
+static cudaError_t launch_indexer_fallback(const IndexerArgs& a, const int32_t* fb,
+                                           float* scratch, int n_ctas, cudaStream_t st) {
+    k_indexer_rows_fallback<T><<<n_ctas, 256, a.d_idx * sizeof(float), st>>>(
+        (const T*)a.q_idx, (const T*)a.k_idx, a.d_idx, a.budget, fb, (int)a.N, scratch, a.sup_idx,
+        a.sup_len, a.sup_score);
+    note_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t fallback_indexer_rows(const IndexerArgs& a, const int32_t* fb, float* scratch,
+                                  int n_ctas, cudaStream_t st) {
+    if (n_ctas < 1) return cudaErrorInvalidValue;
+    return a.dtype == TAM_F32 ? launch_indexer_fallback<float>(a, fb, scratch, n_ctas, st)
+                              : launch_indexer_fallback<__nv_bfloat16>(a, fb, scratch, n_ctas, st);
 }
 
 }  // namespace tam

@@ -50,13 +50,20 @@ inline int64_t n_selection_units(int64_t N, int block_q) {
     return block_q == 1 ? N : (N + block_q - 1) / block_q;
 }
 
-// Per-query tensor-core pass 2 (and the indexer) materialise score rows in a
-// triangular slab and select from it; the slab holds the rows of a chunk of
-// queries.  Chunks start at multiples of 64 queries (a multiple of every kernel's
-// query tile); the preferred slab takes the whole problem up to 4 GiB, the smallest
-// usable one any 64 rows (64 N floats).
+// Per-query selection on the tensor cores (pass 2 and the indexer) streams: a sample
+// pass scores every 2^L-th key of each row and sets the row's threshold tau_i, then
+// the scoring kernel keeps only the keys at or above tau_i, in fixed candidate
+// segments, and an exact select runs over those; rows whose candidates fall short
+// or overflow are recomputed whole on the CUDA cores.  Nothing of size N x N is
+// written.  With TAM_MATERIALISE_ROWS=1 the rows are written instead, to a
+// triangular slab, and selected from there (A/B comparisons).  Both forms run in
+// chunks of queries sized by the workspace; chunks start at multiples of 64 queries
+// (a multiple of every kernel's query tile).
 constexpr size_t kSlabPrefBytes = size_t(4) << 30;
 constexpr int64_t kChunkRows = 64;
+constexpr int kMaxSamplesPerRow = 4096;   // sets the sample stride
+constexpr float kTauSigmas = 5.f;         // margin of the sampled threshold
+constexpr int kFallbackCtas = 148;
 
 size_t slab_pref_bytes(int64_t N) {
     return std::min(kSlabPrefBytes, (size_t)tri(N) * sizeof(float));
@@ -65,27 +72,129 @@ size_t slab_min_bytes(int64_t N) {
     return (size_t)std::min(tri(N), kChunkRows * N) * sizeof(float);
 }
 
-// End of the chunk that starts at r0 (a multiple of 64) for a slab of cap floats
-// (cap >= 64 N): the whole rest if it fits, else the most 64-row steps that do.
-int64_t chunk_end(int64_t r0, int64_t N, int64_t cap) {
-    if (tri(N) - tri(r0) <= cap) return N;
+// End of the chunk that starts at r0 (a multiple of 64) for a buffer of cap floats,
+// where rows [r0, r1) take off(r1) - off(r0) floats (off non-decreasing, and 64 rows
+// always fit): the whole rest if it fits, else the most 64-row steps that do.
+template <class Off>
+int64_t chunk_end_by(int64_t r0, int64_t N, int64_t cap, Off off) {
+    if (off(N) - off(r0) <= cap) return N;
     int64_t lo = 1, hi = (N - r0) / kChunkRows + 1;
     while (hi - lo > 1) {
         const int64_t mid = (lo + hi) / 2;
-        if (tri(r0 + mid * kChunkRows) - tri(r0) <= cap) lo = mid; else hi = mid;
+        if (off(std::min(N, r0 + mid * kChunkRows)) - off(r0) <= cap) lo = mid; else hi = mid;
     }
     return std::min(N, r0 + lo * kChunkRows);
 }
 
+int64_t chunk_end(int64_t r0, int64_t N, int64_t cap) {
+    return chunk_end_by(r0, N, cap, [](int64_t i) { return tri(i); });
+}
+
+// Layout and sizes of the streamed selection, after the caller's other regions:
+//   tau [N] f32 | fallback list [1 + N] i32 | counts [N * nseg] i32 | region
+// The region holds, one after the other, the sample rows of a chunk, the candidate
+// segments of a chunk, and finally the fallback rows' scratch (or, materialised,
+// the row slab of a chunk).
+struct StreamPlan {
+    int L = 0;                    // sample stride 2^L
+    int nseg = 0, seg_cap = 0;    // candidate segments per row and entries per segment
+    int cap = 0;                  // nseg * seg_cap: rows of at most cap keys keep every key
+    size_t off_tau = 0, off_fb = 0, off_cnt = 0, off_region = 0;
+    size_t region_pref = 0, region_min = 0;
+};
+
+int sample_log2(int64_t N) {
+    int L = 4;
+    while (((N - 1) >> L) + 1 > kMaxSamplesPerRow) ++L;
+    return L;
+}
+
+// Threshold rank r = ceil(mu + z sqrt(mu) + 4) of mu = k / 2^L expected sampled keys
+// at or above the k-th value; about 2^L (r + 1) keys of a row then pass, and the
+// segments hold half as many again (plus 32 each) before they overflow.
+int segment_capacity(int budget, int L, int nseg) {
+    const double mu = (double)budget / (double)(1 << L);
+    const double r = std::ceil(mu + kTauSigmas * std::sqrt(mu) + 4.0);
+    const double expect = (double)(1 << L) * (r + 1.0);
+    const int per = (int)std::ceil(1.5 * expect / nseg) + 32;
+    return (per + 31) & ~31;
+}
+
+StreamPlan plan_stream(int64_t N, int budget, int nseg, size_t off) {
+    StreamPlan sp;
+    sp.L = sample_log2(N);
+    sp.nseg = nseg;
+    sp.seg_cap = segment_capacity(budget, sp.L, nseg);
+    sp.cap = nseg * sp.seg_cap;
+    sp.off_tau = off;
+    sp.off_fb = sp.off_tau + align256((size_t)N * 4);
+    sp.off_cnt = sp.off_fb + align256((size_t)(N + 1) * 4);
+    sp.off_region = sp.off_cnt + align256((size_t)N * nseg * 4);
+    const size_t samples_all = (size_t)sample_offset(N, sp.L) * 4;
+    const size_t cand_all = (size_t)N * sp.cap * 8;
+    const size_t fb_pref = (size_t)std::min<int64_t>(N, kFallbackCtas) * N * 4;
+    sp.region_pref = std::max({samples_all, cand_all, fb_pref});
+    if (materialise_rows()) sp.region_pref = std::max(sp.region_pref, slab_pref_bytes(N));
+    const int64_t s_max = ((N - 1) >> sp.L) + 1;
+    sp.region_min = std::max({(size_t)std::min<int64_t>(N, kChunkRows) * s_max * 4,
+                              (size_t)std::min<int64_t>(N, kChunkRows) * sp.cap * 8,
+                              slab_min_bytes(N)});
+    return sp;
+}
+
+// The streamed per-query selection over a region of `region_bytes` (>= region_min).
+// sample(r0, r1, L, slab) scores the sampled keys of rows [r0, r1) into slab;
+// scan(c0, c1) writes the candidate segments and counts of rows [c0, c1) to the
+// region; fallback(fb, scratch, n_ctas) redoes the listed rows.
+template <class Sample, class Scan, class Fallback>
+cudaError_t run_stream_select(const StreamPlan& sp, char* ws, size_t region_bytes, int64_t N,
+                              int budget, int32_t* sup_idx, int32_t* sup_len, float* sup_val,
+                              cudaStream_t st, Sample sample, Scan scan, Fallback fallback) {
+    float* tau = (float*)(ws + sp.off_tau);
+    int32_t* fb = (int32_t*)(ws + sp.off_fb);
+    int32_t* cnt = (int32_t*)(ws + sp.off_cnt);
+    char* region = ws + sp.off_region;
+    cudaError_t e = cudaMemsetAsync(fb, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return e;
+    // rows of at most cap keys keep every key: no samples needed below r_start
+    const int64_t r_start = std::min<int64_t>(N, (sp.cap / kChunkRows) * kChunkRows);
+    const int force = debug_force_fallback();
+    if ((e = sample_tau(nullptr, 0, r_start, sp.L, budget, sp.cap, kTauSigmas, force, tau, st)))
+        return e;
+    const int L = sp.L;
+    const int64_t slab_cap = (int64_t)(region_bytes / 4);
+    for (int64_t r0 = r_start; r0 < N;) {
+        const int64_t r1 = chunk_end_by(r0, N, slab_cap, [L](int64_t i) { return sample_offset(i, L); });
+        if ((e = sample(r0, r1, L, (float*)region))) return e;
+        if ((e = sample_tau((const float*)region, r0, r1, L, budget, sp.cap, kTauSigmas, force, tau,
+                            st)))
+            return e;
+        r0 = r1;
+    }
+    const int64_t rows_per_chunk =
+        std::max<int64_t>(kChunkRows, (int64_t)(region_bytes / ((size_t)sp.cap * 8)) / kChunkRows * kChunkRows);
+    for (int64_t c0 = 0; c0 < N; c0 += rows_per_chunk) {
+        const int64_t c1 = std::min(N, c0 + rows_per_chunk);
+        if ((e = scan(c0, c1, tau, (void*)region, cnt))) return e;
+        if ((e = cand_select(region, cnt, c0, c1, sp.nseg, sp.seg_cap, budget, sup_idx, sup_len,
+                             sup_val, fb, st)))
+            return e;
+    }
+    const int n_ctas = (int)std::min<int64_t>(
+        {(int64_t)kFallbackCtas, N, (int64_t)(region_bytes / ((size_t)N * 4))});
+    return fallback(fb, (float*)region, std::max(1, n_ctas));
+}
+
 // Workspace layout of tam_mass_oracle_prefill / tam_mass_select: status block, lse
 // (when the caller passes none), then the pass-2 scratch of whichever kernel runs:
-// the row slab (tensor cores, per query), fixed-point block mass (tensor cores,
-// block-shared) or staged mass rows (CUDA cores).  `total` is the preferred size,
-// `min_total` the smallest accepted (a smaller slab only means more chunks).
+// the streamed selection (tensor cores, per query), fixed-point block mass (tensor
+// cores, block-shared) or staged mass rows (CUDA cores).  `total` is the preferred
+// size, `min_total` the smallest accepted (a smaller region only means more chunks).
 struct MassPlan {
     size_t off_lse, off_work, total, min_total;
-    bool tc, slab;
+    bool tc, stream;
     int n_ctas;
+    StreamPlan sp;
 };
 
 MassArgs mass_shape(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k, int block_q) {
@@ -98,41 +207,50 @@ MassArgs mass_shape(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k, 
 MassPlan plan_mass(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k, int block_q) {
     MassPlan p{};
     const int64_t n_sel = n_selection_units(N, block_q);
-    p.tc = tc_mass_supported(mass_shape(N, Hq, Hkv, d, dtype, budget_k, block_q));
+    const MassArgs shape = mass_shape(N, Hq, Hkv, d, dtype, budget_k, block_q);
+    p.tc = tc_mass_supported(shape);
     p.n_ctas = (int)std::min<int64_t>(n_sel, kSimtPersistentCtas);
-    p.slab = p.tc && block_q == 1;
+    p.stream = p.tc && block_q == 1;
     p.off_lse = kStatusBytes;
     p.off_work = p.off_lse + align256((size_t)Hq * N * sizeof(float));
     size_t work, min_work;
-    if (!p.tc)
+    if (!p.tc) {
         work = min_work = (size_t)p.n_ctas * N * sizeof(float);
-    else if (p.slab) {
-        work = slab_pref_bytes(N);
-        min_work = slab_min_bytes(N);
-    } else
+    } else if (p.stream) {
+        p.sp = plan_stream(N, budget_k, tc_mass_segments(shape), p.off_work);
+        p.total = p.sp.off_region + align256(p.sp.region_pref);
+        p.min_total = p.sp.off_region + align256(p.sp.region_min);
+        return p;
+    } else {
         work = min_work = tc_mass_block_bytes(N, block_q);
+    }
     p.total = p.off_work + align256(work);
     p.min_total = p.off_work + align256(min_work);
     return p;
 }
 
-// Workspace of tam_indexer_topk: status block, then the row slab of the tensor-core
-// path or the staged score rows of the CUDA-core path.
+// Workspace of tam_indexer_topk: status block, then the streamed selection of the
+// tensor-core path or the staged score rows of the CUDA-core path.
 struct IndexerPlan {
     size_t off_scratch, total, min_total;
     bool tc;
     int n_ctas;
+    StreamPlan sp;
 };
 
 IndexerPlan plan_indexer(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
-    (void)budget_k;
     IndexerPlan p{};
     p.tc = tc_indexer_supported(N, d_idx, dtype, block_q);
     p.n_ctas = (int)std::min<int64_t>(N, kSimtPersistentCtas);
     p.off_scratch = kStatusBytes;
-    const size_t simt = (size_t)p.n_ctas * N * sizeof(float);
-    p.total = p.off_scratch + align256(p.tc ? slab_pref_bytes(N) : simt);
-    p.min_total = p.off_scratch + align256(p.tc ? slab_min_bytes(N) : simt);
+    if (p.tc) {
+        p.sp = plan_stream(N, budget_k, kIndexerSegments, p.off_scratch);
+        p.total = p.sp.off_region + align256(p.sp.region_pref);
+        p.min_total = p.sp.off_region + align256(p.sp.region_min);
+    } else {
+        const size_t simt = (size_t)p.n_ctas * N * sizeof(float);
+        p.total = p.min_total = p.off_scratch + align256(simt);
+    }
     return p;
 }
 
@@ -170,19 +288,42 @@ int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void*
     ma.sup_idx = sup_idx; ma.sup_len = sup_len; ma.sup_mass = sup_mass;
     ma.status = (int32_t*)ws;
     if (!plan.tc) return cuda_status(simt_mass_select(ma, st));
-    if (!plan.slab) return cuda_status(tc_mass_pass(ma, st));
-    // per query: mass rows of a chunk of queries, then their top-k, chunk by chunk
-    const int64_t cap = (int64_t)((ws_bytes - plan.off_work) / sizeof(float));
-    for (int64_t r0 = 0; r0 < N;) {
-        const int64_t r1 = chunk_end(r0, N, cap);
-        ma.row0 = r0;
-        ma.row1 = r1;
-        cudaError_t e = tc_mass_pass(ma, st);
-        if (e == cudaSuccess) e = row_topk(ma.rows, r0, r1, budget_k, sup_idx, sup_len, sup_mass, st);
-        if (e != cudaSuccess) return TAM_ERR_CUDA;
-        r0 = r1;
+    if (!plan.stream) return cuda_status(tc_mass_pass(ma, st));
+    const StreamPlan& sp = plan.sp;
+    char* region = ws + sp.off_region;
+    const size_t region_bytes = ws_bytes - sp.off_region;
+    if (materialise_rows()) {
+        // mass rows of a chunk of queries, then their top-k, chunk by chunk
+        const int64_t cap = (int64_t)(region_bytes / sizeof(float));
+        ma.rows = (float*)region;
+        for (int64_t r0 = 0; r0 < N;) {
+            const int64_t r1 = chunk_end(r0, N, cap);
+            ma.row0 = r0;
+            ma.row1 = r1;
+            cudaError_t e = tc_mass_pass(ma, st);
+            if (e == cudaSuccess)
+                e = row_topk(ma.rows, r0, r1, budget_k, sup_idx, sup_len, sup_mass, st);
+            if (e != cudaSuccess) return TAM_ERR_CUDA;
+            r0 = r1;
+        }
+        return TAM_OK;
     }
-    return TAM_OK;
+    auto sample = [&](int64_t r0, int64_t r1, int L, float* slab) {
+        MassArgs a = ma;
+        a.row0 = r0; a.row1 = r1; a.kst_log2 = L; a.rows = slab;
+        return tc_mass_pass(a, st);
+    };
+    auto scan = [&](int64_t c0, int64_t c1, const float* tau, void* cand, int32_t* cnt) {
+        MassArgs a = ma;
+        a.row0 = c0; a.row1 = c1; a.stream = true; a.tau = tau; a.cand = cand; a.cnt = cnt;
+        a.seg_cap = sp.seg_cap;
+        return tc_mass_pass(a, st);
+    };
+    auto fallback = [&](const int32_t* fb, float* scratch, int n_ctas) {
+        return fallback_mass_rows(ma, fb, scratch, n_ctas, st);
+    };
+    return cuda_status(run_stream_select(sp, ws, region_bytes, N, budget_k, sup_idx, sup_len,
+                                         sup_mass, st, sample, scan, fallback));
 }
 
 // Null and alignment checks of the prefill entry points.
@@ -288,18 +429,41 @@ int run_indexer(int64_t N, int d_idx, int dtype, const void* q_idx, const void* 
     ia.sup_idx = sup_idx; ia.sup_len = sup_len; ia.sup_score = sup_score;
     ia.status = (int32_t*)ws;
     if (!plan.tc) return cuda_status(simt_indexer_select(ia, st));
-    // score rows of a chunk of queries, then their top-k, chunk by chunk
-    const int64_t cap = (int64_t)((ws_bytes - plan.off_scratch) / sizeof(float));
-    for (int64_t r0 = 0; r0 < N;) {
-        const int64_t r1 = chunk_end(r0, N, cap);
-        ia.row0 = r0;
-        ia.row1 = r1;
-        cudaError_t e = tc_indexer_rows(ia, st);
-        if (e == cudaSuccess) e = row_topk(ia.rows, r0, r1, budget_k, sup_idx, sup_len, sup_score, st);
-        if (e != cudaSuccess) return TAM_ERR_CUDA;
-        r0 = r1;
+    const StreamPlan& sp = plan.sp;
+    char* region = ws + sp.off_region;
+    const size_t region_bytes = ws_bytes - sp.off_region;
+    if (materialise_rows()) {
+        // score rows of a chunk of queries, then their top-k, chunk by chunk
+        const int64_t cap = (int64_t)(region_bytes / sizeof(float));
+        ia.rows = (float*)region;
+        for (int64_t r0 = 0; r0 < N;) {
+            const int64_t r1 = chunk_end(r0, N, cap);
+            ia.row0 = r0;
+            ia.row1 = r1;
+            cudaError_t e = tc_indexer_rows(ia, st);
+            if (e == cudaSuccess)
+                e = row_topk(ia.rows, r0, r1, budget_k, sup_idx, sup_len, sup_score, st);
+            if (e != cudaSuccess) return TAM_ERR_CUDA;
+            r0 = r1;
+        }
+        return TAM_OK;
     }
-    return TAM_OK;
+    auto sample = [&](int64_t r0, int64_t r1, int L, float* slab) {
+        IndexerArgs a = ia;
+        a.row0 = r0; a.row1 = r1; a.kst_log2 = L; a.rows = slab;
+        return tc_indexer_rows(a, st);
+    };
+    auto scan = [&](int64_t c0, int64_t c1, const float* tau, void* cand, int32_t* cnt) {
+        IndexerArgs a = ia;
+        a.row0 = c0; a.row1 = c1; a.stream = true; a.tau = tau; a.cand = cand; a.cnt = cnt;
+        a.seg_cap = sp.seg_cap;
+        return tc_indexer_rows(a, st);
+    };
+    auto fallback = [&](const int32_t* fb, float* scratch, int n_ctas) {
+        return fallback_indexer_rows(ia, fb, scratch, n_ctas, st);
+    };
+    return cuda_status(run_stream_select(sp, ws, region_bytes, N, budget_k, sup_idx, sup_len,
+                                         sup_score, st, sample, scan, fallback));
 }
 
 }  // namespace
@@ -724,6 +888,36 @@ int tam_dense_gqa_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, i
             return rc;
     }
     return TAM_OK;
+}
+
+namespace {
+int64_t read_fallback_count(const void* workspace, size_t off_fb, void* stream) {
+    if (!workspace) return -1;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return -1;
+    int32_t c = 0;
+    if (cudaMemcpy(&c, (const char*)workspace + off_fb, sizeof(c), cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+        return -1;
+    return c;
+}
+}  // namespace
+
+int64_t tam_mass_fallback_rows(int64_t N, int Hq, int Hkv, int d, int dtype, int budget_k,
+                               const void* workspace, void* stream) {
+    if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK || check_budget(N, budget_k, 1) != TAM_OK)
+        return -1;
+    const MassPlan plan = plan_mass(N, Hq, Hkv, d, dtype, budget_k, 1);
+    if (!plan.stream || materialise_rows()) return -1;
+    return read_fallback_count(workspace, plan.sp.off_fb, stream);
+}
+
+int64_t tam_indexer_fallback_rows(int64_t N, int d_idx, int dtype, int budget_k,
+                                  const void* workspace, void* stream) {
+    if (N < 1 || d_idx < 1 || (dtype != TAM_BF16 && dtype != TAM_F32)) return -1;
+    if (check_indexer_args(N, d_idx, dtype, budget_k, 1) != TAM_OK) return -1;
+    const IndexerPlan plan = plan_indexer(N, d_idx, dtype, budget_k, 1);
+    if (!plan.tc || materialise_rows()) return -1;
+    return read_fallback_count(workspace, plan.sp.off_fb, stream);
 }
 
 int tam_check_status(const void* workspace, void* stream, int32_t* detail) {

@@ -61,6 +61,13 @@ bool pair_path_disabled() { return env_int("TAM_DISABLE_PAIR_KERNELS", 0) != 0; 
 
 bool block_tc_disabled() { return env_int("TAM_DISABLE_BLOCK_TC", 0) != 0; }
 
+bool materialise_rows() { return env_int("TAM_MATERIALISE_ROWS", 0) != 0; }
+
+int debug_force_fallback() {
+    const int v = env_int("TAM_DEBUG_FORCE_FALLBACK", 0);
+    return (v == 1 || v == 2) ? v : 0;
+}
+
 int debug_flags() { return env_int("TAM_DEBUG_FORCE_TIMEOUT", 0) ? kDebugForceTimeout : 0; }
 
 }  // namespace tam

@@ -28,5 +28,13 @@ constexpr int kDebugForceTimeout = 1;
 bool pair_path_disabled();
 // TAM_DISABLE_BLOCK_TC=1 routes block-shared pass 3 to the mma.sync kernel (A/B comparisons).
 bool block_tc_disabled();
+// TAM_MATERIALISE_ROWS=1 routes the per-query selection (mass and indexer) through
+// materialised score rows and the row top-k instead of the streamed candidates
+// (A/B comparisons).
+bool materialise_rows();
+// TAM_DEBUG_FORCE_FALLBACK=1 (threshold above every key) or =2 (threshold below every
+// key) sends every row the streamed selection would sample to the fallback path, so
+// that path can be tested on ordinary inputs.
+int debug_force_fallback();
 
 }  // namespace tam
