@@ -10,11 +10,13 @@
 // The flash-style pipeline of the dense kernel over gathered keys.  One CTA owns one
 // KV group g and a tile of 128/G queries of block b (the G query heads packed as the
 // 128 UMMA rows, row = query*G + head); its keys are the entries of S_b up to the
-// tile's last query, in chunks of 128:
+// tile's last query, in chunks of 64 in a four-stage ring:
 //   gather warps (6-7)  cp.async the K and V rows of the chunk (whole rows per warp
 //                       instruction, zero-filled past the support) into 128-byte-swizzled shared
 //                       tiles laid out as a TMA tile load would leave them, stage the
-//                       key indices for the mask, fence to the async proxy and arrive;
+//                       key indices for the mask; a chunk is signalled (fence to the async
+//                       proxy, arrive) once the copies of the two chunks after it are in
+//                       flight, so three chunks of rows travel at once;
 //   warp 4              TMA of the Q tile (once);
 //   warp 5              S = Q K^T into one of two TMEM buffers, then O += P V, S of
 //                       chunk t+1 issued before P V of chunk t;
@@ -29,9 +31,12 @@
 namespace tam {
 namespace {
 
-constexpr int kStages = 2;
-constexpr int kKeys = 128;                  // keys per chunk
-constexpr int kHalf = 128 * 64 * 2;         // one 128-row x 64-element swizzled half
+constexpr int kStages = 4;
+constexpr int kLag = 2;                     // chunks in flight behind the one being signalled
+constexpr int kKeys = 64;                   // keys per chunk
+constexpr int kHalf = 128 * 64 * 2;         // one 128-row x 64-element swizzled half (Q, P)
+constexpr int kHalfKV = kKeys * 64 * 2;     // one 64-key x 64-element swizzled half (K, V)
+static_assert(kLag < kStages - 1, "the gather may run at most kStages - 2 chunks ahead");
 constexpr int kThreads = 256;
 constexpr int kGatherWarp0 = 6;             // warps 6..7 gather
 constexpr int kGatherThreads = kThreads - kGatherWarp0 * 32;
@@ -40,7 +45,7 @@ constexpr float kRescaleLog2 = 8.f;
 template <int D>
 constexpr int block_tc_smem_bytes() {
     // slack + Q + K ring + V ring + P + staged key indices + barriers
-    return 1024 + (D / 64) * kHalf * (1 + 2 * kStages) + 2 * kHalf + kStages * kKeys * 4 + 256;
+    return 1024 + (D / 64) * (kHalf + 2 * kStages * kHalfKV) + kHalf + kStages * kKeys * 4 + 256;
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -73,15 +78,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) {
     constexpr int BQ = 128 / G;
     constexpr int NH = D / 64;
-    constexpr uint32_t kTile = NH * kHalf;
+    constexpr uint32_t kTile = NH * kHalf;        // Q
+    constexpr uint32_t kTileKV = NH * kHalfKV;    // one chunk of K (or V)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* sQ = base;
     uint8_t* sK = sQ + kTile;
-    uint8_t* sV = sK + kStages * kTile;
-    uint8_t* sP = sV + kStages * kTile;                 // 2 halves of 64 keys
-    int32_t* sIdx = reinterpret_cast<int32_t*>(sP + 2 * kHalf);    // kStages x 128
+    uint8_t* sV = sK + kStages * kTileKV;
+    uint8_t* sP = sV + kStages * kTileKV;               // 128 rows x 64 keys
+    int32_t* sIdx = reinterpret_cast<int32_t*>(sP + kHalf);        // kStages x kKeys
     uint64_t* bars = reinterpret_cast<uint64_t*>(sIdx + kStages * kKeys);
     uint64_t* q_full = bars;
     uint64_t* kv_full = q_full + 1;
@@ -179,7 +185,7 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
         constexpr int RR = RPW / 32;                       // index registers per lane
         static_assert(RR * 32 == RPW && RPI * PR == 32, "gather tiling");
         const int piece = lane % PR, sub = lane / PR;
-        const uint32_t half_off = (uint32_t)(piece / 8) * kHalf;
+        const uint32_t half_off = (uint32_t)(piece / 8) * kHalfKV;
         const int pc = piece % 8;
         const __nv_bfloat16* kbase = p.k + (size_t)g * D + piece * 8;
         const __nv_bfloat16* vbase = p.v + (size_t)g * D + piece * 8;
@@ -190,10 +196,11 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
             const int r = gw * RPW + rr * 32 + lane;
             jn[rr] = r < n_t ? sIdx[r] : -1;              // chunk 0, staged above
         }
+        int signalled = 0;                                  // chunks announced so far
         for (int t = 0; t < n_ch; ++t) {
             const int s = t % kStages;
             if (!tc::wait(&kv_empty[s], ((t / kStages) & 1) ^ 1, gd, 1)) break;
-            const uint32_t dk = tc::smem_u32(sK + s * kTile), dv = tc::smem_u32(sV + s * kTile);
+            const uint32_t dk = tc::smem_u32(sK + s * kTileKV), dv = tc::smem_u32(sV + s * kTileKV);
             int js[RR];
 #pragma unroll
             for (int rr = 0; rr < RR; ++rr) {
@@ -216,13 +223,22 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
                 cp_async16(dv + o, vbase + off, valid);
             }
             cp_async_commit();
-            // signal chunk t as soon as it has landed (made visible to the tensor core):
-            // the MMA issuer waits for it before it frees the stage chunk t+1 needs
-            cp_async_wait<0>();
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&kv_full[s]);
+            // chunk t - kLag has landed once at most kLag newer groups are pending:
+            // make it visible to the tensor core and signal it
+            if (t >= kLag) {
+                cp_async_wait<kLag>();
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(&kv_full[(t - kLag) % kStages]);
+                signalled = t - kLag + 1;
+            }
         }
         cp_async_wait<0>();
+        tc::fence_proxy_async_smem();
+        // the last chunks (every chunk issued, or stopped early: whatever was issued)
+        for (int t = signalled; t < n_ch; ++t) {
+            if (*abort_flag) break;
+            tc::mbar_arrive(&kv_full[t % kStages]);
+        }
     } else if (warp == 4) {
         // ---------------------------------------------------------------- Q (TMA)
         if (lane == 0) {
@@ -237,7 +253,7 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
     } else if (warp == 5) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, 128);
+            constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kKeys);
             constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, D, false, true);
             const uint32_t aq = tc::smem_u32(sQ);
             const uint32_t ap = tc::smem_u32(sP);
@@ -247,12 +263,13 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
                 if (!tc::wait(&kv_full[s], (t / kStages) & 1, gd, 4)) return false;
                 if (!tc::wait(&s_empty[bb], ((t >> 1) & 1) ^ 1, gd, 5)) return false;
                 tc::fence_after_sync();
-                const uint32_t ak = tc::smem_u32(sK + s * kTile);
+                const uint32_t ak = tc::smem_u32(sK + s * kTileKV);
 #pragma unroll
                 for (int kk = 0; kk < NH * 4; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    tc::mma_bf16_ss(tmem + bb * 128, tc::desc_kmajor_sw128(aq + off),
-                                    tc::desc_kmajor_sw128(ak + off), idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t offq = (kk >> 2) * kHalf + (kk & 3) * 32;
+                    const uint32_t offk = (kk >> 2) * kHalfKV + (kk & 3) * 32;
+                    tc::mma_bf16_ss(tmem + bb * kKeys, tc::desc_kmajor_sw128(aq + offq),
+                                    tc::desc_kmajor_sw128(ak + offk), idesc_s, kk > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(&s_full[bb]);
                 return true;
@@ -263,12 +280,11 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
                 const int s = t % kStages;
                 if (!tc::wait(p_full, t & 1, gd, 7)) break;
                 tc::fence_after_sync();
-                const uint32_t av = tc::smem_u32(sV + s * kTile);
+                const uint32_t av = tc::smem_u32(sV + s * kTileKV);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {   // 128 keys in steps of 16
-                    const uint32_t offp = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    tc::mma_bf16_ss(tmem_o, tc::desc_kmajor_sw128(ap + offp),
-                                    tc::desc_mnmajor_sw128(av + kk * 16 * 128, kHalf), idesc_o,
+                for (int kk = 0; kk < kKeys / 16; ++kk) {   // the chunk's keys in steps of 16
+                    tc::mma_bf16_ss(tmem_o, tc::desc_kmajor_sw128(ap + kk * 32),
+                                    tc::desc_mnmajor_sw128(av + kk * 16 * 128, kHalfKV), idesc_o,
                                     (t > 0 || kk > 0) ? 1u : 0u);
                 }
                 tc::mma_commit(&kv_empty[s]);
@@ -288,22 +304,23 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
         const float sl2 = p.sl2;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        uint8_t* prow0 = sP + r * 128;               // row r of half 0
+        uint8_t* prow0 = sP + r * 128;               // row r of the P tile
         for (int t = 0; ok && t < n_ch; ++t) {
             const int bb = t & 1, s = t % kStages;
             if (!tc::wait(&s_full[bb], (t >> 1) & 1, gd, 8)) { ok = false; break; }
             tc::fence_after_sync();
-            uint32_t v[4][32];
+            constexpr int NC = kKeys / 32;            // 32-column loads of a chunk
+            uint32_t v[NC][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tc::tmem_ld32(tmem + lane_off + bb * 128 + c * 32, v[c]);
+            for (int c = 0; c < NC; ++c) tc::tmem_ld32(tmem + lane_off + bb * kKeys + c * 32, v[c]);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tc::tmem_wait_ld(v[c]);
+            for (int c = 0; c < NC; ++c) tc::tmem_wait_ld(v[c]);
             tc::fence_before_sync();
             tc::mbar_arrive(&s_empty[bb]);
             // mask: keys past the support (index -1) or after query i
             const int4* ix4 = reinterpret_cast<const int4*>(sIdx + s * kKeys);
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < NC; ++c)
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
                     const int4 jj = ix4[c * 8 + e4];
@@ -314,7 +331,7 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
                 }
             float tm[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < NC; ++c)
 #pragma unroll
                 for (int e = 0; e < 32; e += 2)
                     tm[c & 1] = tc::max3(tm[c & 1], __uint_as_float(v[c][e]),
@@ -329,7 +346,7 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
             const uint64_t negm2 = tc::f2_pack(none ? 0.f : -m_new, none ? 0.f : -m_new);
             uint64_t sum2[2] = {0ull, 0ull};
 #pragma unroll
-            for (int c8 = 0; c8 < 16; ++c8) {
+            for (int c8 = 0; c8 < kKeys / 8; ++c8) {
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -352,13 +369,12 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
                     __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<uint32_t*>(&pk);
                 }
-                const int half = c8 >> 3, chunk = c8 & 7;
                 // P V of chunk t-1 must have finished reading the P tile before it is
                 // overwritten; wait once, before the first store
                 if (c8 == 0 && t > 0) {
                     if (!tc::wait(o_done, (t - 1) & 1, gd, 9)) { ok = false; break; }
                 }
-                uint4* dst = reinterpret_cast<uint4*>(prow0 + half * kHalf + ((chunk ^ (r & 7)) << 4));
+                uint4* dst = reinterpret_cast<uint4*>(prow0 + ((c8 ^ (r & 7)) << 4));
                 *dst = make_uint4(w[0], w[1], w[2], w[3]);
             }
             if (!ok) break;

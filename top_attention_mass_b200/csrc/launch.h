@@ -126,6 +126,10 @@ cudaError_t sample_tau(const float* slab, int64_t row0, int64_t row1, int L, int
 // written like row_topk.  A row whose segments overflowed or hold fewer than
 // min(k, i+1) keys is appended to the fallback list fb (fb[0] = count, fb[1 + t] = row)
 // and its outputs are left to the fallback.
+// Shared memory cand_select needs for rows of up to max_row_keys keys and cap
+// candidates each; it runs only when that is at most kCandSelectMaxSmem.
+int cand_select_smem(int64_t max_row_keys, int cap);
+constexpr int kCandSelectMaxSmem = 227 * 1024;
 cudaError_t cand_select(const void* cand, const int32_t* cnt, int64_t row0, int64_t row1,
                         int nseg, int seg_cap, int budget, int32_t* sup_idx, int32_t* sup_len,
                         float* sup_val, int32_t* fb, cudaStream_t st);

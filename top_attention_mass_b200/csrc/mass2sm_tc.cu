@@ -37,6 +37,8 @@
 //               order); block-shared mass goes to the fixed-point block sums.
 // Every wait is bounded; the pair shakes hands before it frees TMEM and exits so
 // that no remote arrive or MMA of one CTA can land after the other left.
+#include <cstdlib>
+
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
@@ -44,8 +46,8 @@
 namespace tam {
 namespace {
 
-constexpr int kStages = 2;
 constexpr int kModeRows = 0, kModeBlock = 1, kModeStream = 2;
+constexpr int kMaxStages = 6;           // K ring: as many full key tiles as fit, 2..6
 // Mass warps: 8 per query (two per TMEM lane quarter), 16 block-shared (four per
 // quarter; measured 5 % faster there, no gain per query).  Then the TMA producer and
 // the MMA issuer.
@@ -56,17 +58,27 @@ constexpr int kHalfRows = 64;           // B rows held by each CTA
 constexpr int kR = 512 / kNQ;           // TMEM accumulator slots
 constexpr int kTileKeys = 256;          // keys per pair tile (128 per CTA)
 
-__host__ __device__ constexpr int pair_smem_bytes(int D, int Hkv) {
-    // Q half + K ring + lse of all 128 columns + thresholds + barriers
-    return 1024 + Hkv * kHalfRows * D * 2 + kStages * 128 * D * 2 + Hkv * kNQ * 4 + 128 + 512;
-}
 constexpr int kMaxDynSmem = 227 * 1024;
+// alignment slack + Q half + lse of all 128 columns + thresholds + barriers
+__host__ __device__ constexpr int pair_fixed_bytes(int D, int Hkv) {
+    return 1024 + Hkv * kHalfRows * D * 2 + Hkv * kNQ * 4 + 128 + 512;
+}
+// Key tiles (128 keys x D per CTA) in the K ring: what fits next to Q, at most kMaxStages
+// (0 if fewer than two fit).
+__host__ __device__ constexpr int pair_stages(int D, int Hkv) {
+    return (kMaxDynSmem - pair_fixed_bytes(D, Hkv)) / (128 * D * 2) >= kMaxStages
+               ? kMaxStages
+               : ((kMaxDynSmem - pair_fixed_bytes(D, Hkv)) / (128 * D * 2) >= 2
+                      ? (kMaxDynSmem - pair_fixed_bytes(D, Hkv)) / (128 * D * 2)
+                      : 0);
+}
 
 struct PairParams {
     int N, Hq, Hkv, pair0, n_pairs, block_q;
     int64_t row0, row1;       // per query: the rows [row0, row1) of this launch
     int kst_log2;             // rows mode: key m of the K map sits at position m << kst_log2
     int seg_cap;              // stream mode: entries per candidate segment
+    int stages;               // key tiles in the K ring
     float sl2, inv_hq;
     const float* lse;
     float* rows;
@@ -104,6 +116,7 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     constexpr uint32_t kKHalf = 128 * 128;
     constexpr uint32_t kKTile = NH * kKHalf;
     const int Hkv = p.Hkv;
+    const int kStages = p.stages;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -115,8 +128,8 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     uint64_t* bars = reinterpret_cast<uint64_t*>(sTau + 32);
     uint64_t* q_full = bars;                 // CTA 0's counts both CTAs' Q bytes
     uint64_t* k_full = q_full + 1;           // CTA 0's counts both CTAs' K bytes
-    uint64_t* k_empty = k_full + kStages;    // both (pair commits)
-    uint64_t* s_full = k_empty + kStages;    // both (pair commits)
+    uint64_t* k_empty = k_full + kMaxStages; // both (pair commits)
+    uint64_t* s_full = k_empty + kMaxStages; // both (pair commits)
     uint64_t* s_empty = s_full + kR;         // CTA 0's: both CTAs' mass threads
     uint64_t* mma_done = s_empty + kR;       // both (pair commit)
     uint64_t* exit_bar = mma_done + 1;       // each: the peer's arrival at the end
@@ -316,14 +329,13 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     const int64_t i = q0 + qi;
                     const float v = acc[ql] * p.inv_hq;
                     const bool pass = m <= i && i < p.row1 && v >= sTau[qi];
+                    // no warp-uniform branch: the queries' ballot chains interleave
                     const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-                    if (bal != 0u) {
-                        const int pos = cnt[ql] + __popc(bal & lt);
-                        if (pass && pos < p.seg_cap)
-                            p.cand[((i - p.row0) * 8 + seg) * (int64_t)p.seg_cap + pos] =
-                                make_uint2(__float_as_uint(v), (uint32_t)m);
-                        cnt[ql] += __popc(bal);
-                    }
+                    const int pos = cnt[ql] + __popc(bal & lt);
+                    if (pass && pos < p.seg_cap)
+                        p.cand[((i - p.row0) * 8 + seg) * (int64_t)p.seg_cap + pos] =
+                            make_uint2(__float_as_uint(v), (uint32_t)m);
+                    cnt[ql] += __popc(bal);
                 }
             } else {
                 const int j = m;
@@ -401,6 +413,12 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     p.row1 = r1;
     p.kst_log2 = L;
     p.seg_cap = a.seg_cap;
+    p.stages = pair_stages(D, a.Hkv);
+    {   // TAM_PAIR_STAGES=n caps the ring (A/B comparisons)
+        const char* env = std::getenv("TAM_PAIR_STAGES");
+        const int cap = env ? std::atoi(env) : 0;
+        if (cap >= 2 && cap < p.stages) p.stages = cap;
+    }
     p.block_q = a.block_q;
     p.sl2 = a.sl2;
     p.inv_hq = 1.f / (float)a.Hq;
@@ -414,7 +432,7 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     p.timeout_ns = wait_timeout_ns();
     p.dbg = debug_flags();
     if (p.n_pairs <= 0) return cudaSuccess;
-    const int smem = pair_smem_bytes(D, a.Hkv);
+    const int smem = pair_fixed_bytes(D, a.Hkv) + p.stages * 128 * D * 2;
     auto kern = k_mass_pair<G, D, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -451,7 +469,7 @@ bool pair_mass_supported(const MassArgs& a) {
     if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128)) return false;
     if (G != 4 && G != 8 && G != 16) return false;
     if (a.block_q > 1 && a.block_q > (1 << 20)) return false;
-    return pair_smem_bytes(a.d, a.Hkv) <= kMaxDynSmem;
+    return pair_stages(a.d, a.Hkv) > 0;
 }
 
 // Launches the pair kernel only: per query it fills the slab rows [row0, row1) (rows

@@ -19,17 +19,19 @@
 // BQ queries for *all* heads resident in shared memory, so the thread that owns a
 // key row adds the probabilities of every head of a query in registers - the head
 // average needs no cross-thread reduction.
-// Roles (192 threads):
-//   warp 4      TMA producer: Q (once, all groups), then K_g tiles in a 2-stage ring;
-//   warp 5      MMA issuer: for each key tile, one UMMA chain per group into a ring
+// Roles (320 threads):
+//   warp 8      TMA producer: Q (once, all groups), then K_g tiles in a 2-stage ring;
+//   warp 9      MMA issuer: for each key tile, one UMMA chain per group into a ring
 //               of 512/NQ TMEM slots;
-//   warps 0-3   mass warps: thread = key row; exp2 against the pass-1 LSE, sum over
-//               heads -> mass of BQ queries; causal mask; then either the mass goes
-//               to the row slab (per query, indexer: lanes store consecutive keys of
-//               one query), or the keys at or above the query's threshold are
-//               appended to warp w's segment of the row (streamed: a warp ballot and
-//               a warp-uniform running count, no atomics), or the block column sum
-//               is added in 2^-40 fixed point (block-shared).
+//   warps 0-7   mass warps: thread = key row (warp w reads TMEM lanes 32 (w % 4) ..),
+//               half w / 4 of the columns; exp2 against the pass-1 LSE, sum over
+//               heads -> mass of BQ / 2 queries; causal mask; then either the mass
+//               goes to the row slab (per query, indexer: lanes store consecutive keys
+//               of one query), or the keys at or above the query's threshold are
+//               appended to segment w % 4 of the query's row (streamed: a warp ballot
+//               and a warp-uniform running count, no atomics; each segment has one
+//               writer, so it stays in key order), or the block column sum is added
+//               in 2^-40 fixed point (block-shared).
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
@@ -38,7 +40,10 @@ namespace tam {
 namespace {
 
 constexpr int kStages = 2;
-constexpr int kThreads = 32 * 6;
+// Eight mass warps (two per TMEM lane quarter, each on half of the columns), then the
+// TMA producer and the MMA issuer.
+constexpr int kMassWarps = 8;
+constexpr int kThreads = 32 * (kMassWarps + 2);
 
 // Kernel modes: head-averaged mass rows, block-shared mass sums, the
 // head-collapsed indexer's score rows (one score per (query, key), no exponentials),
@@ -123,7 +128,7 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
         for (int s = 0; s < R; ++s) {
             tc::mbar_init(&s_full[s], 1);
-            tc::mbar_init(&s_empty[s], 128);
+            tc::mbar_init(&s_empty[s], 32 * kMassWarps);
         }
         tc::mbar_init(mma_done, 1);
         tc::mbar_init(never, 1);
@@ -156,7 +161,7 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                        BLOCK ? KID_BLOCK_MASS_TC : (INDEXER ? KID_INDEXER_TC : KID_MASS_TC),
                        p.timeout_ns};
 
-    if (warp == 4) {
+    if (warp == kMassWarps) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
             tc::prefetch_tmap(&tmQ);
@@ -183,7 +188,7 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 tc::wait(&k_full[u % kStages], (u / kStages) & 1, drain, 0);
             tc::wait(q_full, 0, drain, 0);
         }
-    } else if (warp == 5) {
+    } else if (warp == kMassWarps + 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_bf16_f32(128, NQ);
@@ -214,49 +219,60 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             const tc::Guard drain{&zero, nullptr, 0, p.timeout_ns};
             tc::wait(mma_done, 0, drain, 0);
         }
-    } else if (warp < 4) {
+    } else if (warp < kMassWarps) {
         // ---------------------------------------------------------------- mass warps
-        const int row = threadIdx.x;                       // key row of the tile
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-        // stream modes: warp w writes segment w of every row, with running counts
-        int cnt[STREAM ? BQ : 1];
+        constexpr int kParts = kMassWarps / 4;         // warps per TMEM lane quarter
+        constexpr int kCols = NQ / kParts;             // columns of one part
+        constexpr int kQP = kCols / G;                 // queries of one part
+        constexpr int CW = kCols < 32 ? kCols : 32;    // columns per TMEM load
+        const int quarter = warp & 3, part = warp >> 2;
+        const int row = quarter * 32 + lane;           // key row of the tile
+        const uint32_t lane_addr =
+            tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(part * kCols);
+        // stream modes: the quarter-q warps write segment q of their queries' rows, with
+        // running counts
+        int cnt[STREAM ? kQP : 1];
 #pragma unroll
-        for (int q = 0; q < (STREAM ? BQ : 1); ++q) cnt[q] = 0;
+        for (int q = 0; q < (STREAM ? kQP : 1); ++q) cnt[q] = 0;
         bool ok = true;
         if (p.dbg & kDebugForceTimeout) ok = tc::wait(never, 0, gd, 9);
         for (int kt = 0; ok && kt < n_kt; ++kt) {
-            float acc[BQ];
+            float acc[kQP];
 #pragma unroll
-            for (int q = 0; q < BQ; ++q) acc[q] = 0.f;
+            for (int q = 0; q < kQP; ++q) acc[q] = 0.f;
             for (int g = 0; g < Hkv; ++g) {
                 const int u = kt * Hkv + g;
                 const int slot = u % R;
                 if (!tc::wait(&s_full[slot], (u / R) & 1, gd, 5)) { ok = false; break; }
                 tc::fence_after_sync();
-                // stream the NQ columns in 32-column chunks, loading chunk c+1 while
-                // chunk c is exponentiated
+                // stream this part's columns in CW-column chunks, loading chunk c+1
+                // while chunk c is exponentiated
                 const uint32_t col0 = lane_addr + slot * NQ;
-                uint32_t va[32], vb[32];
-                tc::tmem_ld32(col0, va);
+                uint32_t va[CW], vb[CW];
+                if constexpr (CW == 32) tc::tmem_ld32(col0, va); else tc::tmem_ld16(col0, va);
                 tc::tmem_wait_ld(va);
 #pragma unroll
-                for (int c = 0; c < NQ / 32; ++c) {
-                    uint32_t (&cur)[32] = (c & 1) ? vb : va;
-                    uint32_t (&nxt)[32] = (c & 1) ? va : vb;
-                    if (c + 1 < NQ / 32) tc::tmem_ld32(col0 + (c + 1) * 32, nxt);
+                for (int c = 0; c < kCols / CW; ++c) {
+                    uint32_t (&cur)[CW] = (c & 1) ? vb : va;
+                    uint32_t (&nxt)[CW] = (c & 1) ? va : vb;
+                    if (c + 1 < kCols / CW) {
+                        if constexpr (CW == 32) tc::tmem_ld32(col0 + (c + 1) * CW, nxt);
+                        else tc::tmem_ld16(col0 + (c + 1) * CW, nxt);
+                    }
                     if constexpr (INDEXER) {
                         // one column per query: the raw indexer score
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) acc[c * 32 + e] = __uint_as_float(cur[e]);
+                        for (int e = 0; e < CW; ++e) acc[c * CW + e] = __uint_as_float(cur[e]);
                     } else {
-                        const float4* l4 = reinterpret_cast<const float4*>(sLse + g * NQ + c * 32);
+                        const float4* l4 = reinterpret_cast<const float4*>(
+                            sLse + g * NQ + part * kCols + c * CW);
 #pragma unroll
-                        for (int c4 = 0; c4 < 8; ++c4) {
+                        for (int c4 = 0; c4 < CW / 4; ++c4) {
                             const float4 L = l4[c4];
                             const float Ls[4] = {L.x, L.y, L.z, L.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const int col = c * 32 + c4 * 4 + e;
+                                const int col = c * CW + c4 * 4 + e;
                                 const float sc = __uint_as_float(cur[c4 * 4 + e]);
                                 // one exponential in four on the FMA pipe, the rest on MUFU
                                 const float x = fmaf(sc, p.sl2, -Ls[e]);
@@ -264,74 +280,75 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                             }
                         }
                     }
-                    if (c + 1 < NQ / 32) tc::tmem_wait_ld(nxt);
+                    if (c + 1 < kCols / CW) tc::tmem_wait_ld(nxt);
                 }
                 tc::fence_before_sync();
                 tc::mbar_arrive(&s_empty[slot]);
             }
             if (!ok) break;
             const int j = kt * 128 + row;                     // key (or sample) index
+            const int qp0 = q0 + part * kQP;                  // first query of this part
             if constexpr (STREAM) {
                 // keys at or above the query's threshold, appended in key order to this
                 // warp's segment (positions past the capacity are only counted)
                 uint32_t lt;
                 asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt));
 #pragma unroll
-                for (int q = 0; q < BQ; ++q) {
-                    const int64_t i = q0 + q;
+                for (int q = 0; q < kQP; ++q) {
+                    const int64_t i = qp0 + q;
                     const float v = INDEXER ? acc[q] : acc[q] * p.inv_hq;
-                    const bool pass = j <= i && i < p.row1 && v >= sTau[q];
+                    const bool pass = j <= i && i < p.row1 && v >= sTau[part * kQP + q];
+                    // no warp-uniform branch: the queries' ballot chains interleave
                     const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-                    if (bal != 0u) {
-                        const int pos = cnt[q] + __popc(bal & lt);
-                        if (pass && pos < p.seg_cap)
-                            p.cand[((i - p.row0) * 4 + warp) * (int64_t)p.seg_cap + pos] =
-                                make_uint2(__float_as_uint(v), (uint32_t)j);
-                        cnt[q] += __popc(bal);
-                    }
+                    const int pos = cnt[q] + __popc(bal & lt);
+                    if (pass && pos < p.seg_cap)
+                        p.cand[((i - p.row0) * 4 + quarter) * (int64_t)p.seg_cap + pos] =
+                            make_uint2(__float_as_uint(v), (uint32_t)j);
+                    cnt[q] += __popc(bal);
                 }
             } else if constexpr (!BLOCK) {
                 // row i of the slab starts off(i) - off(row0) floats in; lanes store
                 // consecutive keys of one query
                 const int64_t jp = (int64_t)j << p.kst_log2;  // key position
 #pragma unroll
-                for (int q = 0; q < BQ; ++q) {
-                    const int64_t i = q0 + q;
+                for (int q = 0; q < kQP; ++q) {
+                    const int64_t i = qp0 + q;
                     if (jp <= i && i >= p.row0 && i < p.row1)
                         p.rows[sample_offset(i, p.kst_log2) - slab0 + j] =
                             INDEXER ? acc[q] : acc[q] * p.inv_hq;
                 }
             } else {
-                // block column sums, 2^-40 fixed point, one add per (block, key)
-                int cur_b = q0 / p.block_q;
-                float part = 0.f;
+                // block column sums of this part's queries, 2^-40 fixed point, one add
+                // per (block, key, part)
+                int cur_b = qp0 / p.block_q;
+                float sum = 0.f;
 #pragma unroll
-                for (int q = 0; q < BQ; ++q) {
-                    const int i = q0 + q;
+                for (int q = 0; q < kQP; ++q) {
+                    const int i = qp0 + q;
                     if (i < p.N) {
                         const int b = i / p.block_q;
                         if (b != cur_b) {
-                            if (part > 0.f)
+                            if (sum > 0.f)
                                 atomicAdd(&p.bmass[bmass_offset(cur_b, p.block_q) + j],
                                           (unsigned long long)__float2ll_rn(
-                                              part * p.inv_hq * 1099511627776.0f));
-                            part = 0.f;
+                                              sum * p.inv_hq * 1099511627776.0f));
+                            sum = 0.f;
                             cur_b = b;
                         }
-                        if (j <= i) part += acc[q];
+                        if (j <= i) sum += acc[q];
                     }
                 }
-                if (part > 0.f)
+                if (sum > 0.f)
                     atomicAdd(&p.bmass[bmass_offset(cur_b, p.block_q) + j],
-                              (unsigned long long)__float2ll_rn(part * p.inv_hq * 1099511627776.0f));
+                              (unsigned long long)__float2ll_rn(sum * p.inv_hq * 1099511627776.0f));
             }
         }
         if constexpr (STREAM) {
             if (ok && lane == 0) {
 #pragma unroll
-                for (int q = 0; q < BQ; ++q) {
-                    const int64_t i = q0 + q;
-                    if (i < p.row1) p.cnt[(i - p.row0) * 4 + warp] = cnt[q];
+                for (int q = 0; q < kQP; ++q) {
+                    const int64_t i = q0 + part * kQP + q;
+                    if (i < p.row1) p.cnt[(i - p.row0) * 4 + quarter] = cnt[q];
                 }
             }
         }

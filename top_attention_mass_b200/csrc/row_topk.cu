@@ -31,6 +31,9 @@
 //   5. ordered emission of the candidates > T and the first of those == T.
 // If no threshold has a count in [k, cap] (more than cap keys tie at the k-th
 // value) the bisection ends with the exact k-th key and step 5 runs over the row.
+#include <algorithm>
+#include <climits>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -501,16 +504,17 @@ __global__ void __launch_bounds__(kRtThreads) k_sample_tau(const SampleTauParams
     if (threadIdx.x == 0) p.tau[i] = oval(T);
 }
 
-// Exact top-k of a row from its candidate segments.  Each segment was written by
-// one warp in key order, so a key's rank in the merged row is its position in its
-// own segment plus, in every other segment, the number of keys below it (binary
-// search); the merged candidates then go through the same k-th key search and
-// ordered emission as the materialised rows.
+// Exact top-k of a row from its candidate segments.  The k-th key T is found by the
+// same radix select as for materialised rows; the kept keys are then marked in a
+// bitmap over the row's key indices (one bit per key 0..i), whose word-wise prefix
+// popcount gives every kept key its place in ascending index order.  Equal values at T
+// keep the smallest indices: when more keys equal T than are taken, the equal keys
+// are marked in a second bitmap and the cut-off index is the take-th set bit.
 struct CandSelParams {
     const uint2* cand;
     const int32_t* cnt;
     int64_t row0;
-    int n_rows, nseg, seg_cap, budget;
+    int n_rows, nseg, seg_cap, budget, max_words;
     int32_t* sup_idx;
     int32_t* sup_len;
     float* sup_val;
@@ -519,22 +523,43 @@ struct CandSelParams {
 
 constexpr int kMaxSegments = 8;
 
+// Exclusive prefix of the popcounts of words [0, nw) into pre[]: thread t sums a
+// contiguous range, one block scan (s.hist as its scratch, so not during a radix
+// pass), then each thread writes its range.  Contains barriers.  Returns the total.
+__device__ int word_prefix(const uint32_t* bits, int* pre, int nw, RowSmem& s) {
+    const int per = (nw + kRtThreads - 1) / kRtThreads;
+    const int w0 = min(nw, (int)threadIdx.x * per), w1 = min(nw, w0 + per);
+    int c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(bits[w]);
+    int tot;
+    int run = block_exclusive_scan(c, s.hist, &tot);        // hist: free scratch here
+    for (int w = w0; w < w1; ++w) {
+        pre[w] = run;
+        run += __popc(bits[w]);
+    }
+    __syncthreads();
+    return tot;
+}
+
 __global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams p) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     RowSmem& s = *reinterpret_cast<RowSmem*>(smem_raw);
     __shared__ int soff[kMaxSegments + 1];
-    __shared__ int sflag;
+    __shared__ int sflag, s_ceq, s_cut;
     const int64_t i = p.row0 + (p.n_rows - 1 - (int)blockIdx.x);
     const int n = (int)i + 1;
     const int k = min(p.budget, n);
     const int cap = p.nseg * p.seg_cap;
-    uint32_t* akey = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowSmem)) + 2 * cap;
-    int32_t* aidx = reinterpret_cast<int32_t*>(akey + cap);
+    const int nw = (n + 31) >> 5;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowSmem)) + 2 * cap;
+    int* pre = reinterpret_cast<int*>(bits + p.max_words);
     if (threadIdx.x == 0) {
         s.ckey = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowSmem));
         s.cidx = reinterpret_cast<int32_t*>(s.ckey + cap);
         s.cmax = 0u;
         s.scal[3] = -1;
+        s_ceq = 0;
+        s_cut = 0x7fffffff;
         const int32_t* c = p.cnt + (i - p.row0) * p.nseg;
         int tot = 0;
         bool bad = false;
@@ -556,7 +581,7 @@ __global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams 
     __syncthreads();
     if (sflag) return;
     const int tot = soff[p.nseg];
-    // load the segments back to back
+    // the segments back to back, and a clear bitmap
     const uint2* base = p.cand + (i - p.row0) * (int64_t)cap;
     uint32_t mx = 0u, mn = 0xffffffffu;
     for (int t = threadIdx.x; t < tot; t += blockDim.x) {
@@ -564,11 +589,12 @@ __global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams 
         while (g + 1 < p.nseg && soff[g + 1] <= t) ++g;
         const uint2 e = base[g * p.seg_cap + (t - soff[g])];
         const uint32_t kv = okey(__uint_as_float(e.x));
-        akey[t] = kv;
-        aidx[t] = (int32_t)e.y;
+        s.ckey[t] = kv;
+        s.cidx[t] = (int32_t)e.y;
         mx = max(mx, kv);
         mn = min(mn, kv);
     }
+    for (int w = threadIdx.x; w < nw; w += blockDim.x) bits[w] = 0u;
     mx = __reduce_max_sync(0xffffffffu, mx);
     mn = __reduce_min_sync(0xffffffffu, mn);
     if ((threadIdx.x & 31) == 0) {
@@ -576,35 +602,69 @@ __global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams 
         atomicMin(reinterpret_cast<unsigned int*>(&s.scal[3]), mn);
     }
     __syncthreads();
-    // merge: rank = own position + keys below it in every other segment
-    for (int t = threadIdx.x; t < tot; t += blockDim.x) {
-        int g = 0;
-        while (g + 1 < p.nseg && soff[g + 1] <= t) ++g;
-        const int32_t x = aidx[t];
-        int rank = t - soff[g];
-        for (int h = 0; h < p.nseg; ++h) {
-            if (h == g) continue;
-            int lo = soff[h], hi = soff[h + 1];
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (aidx[mid] < x) lo = mid + 1; else hi = mid;
-            }
-            rank += lo - soff[h];
-        }
-        s.ckey[rank] = akey[t];
-        s.cidx[rank] = x;
-    }
-    const uint32_t G = (uint32_t)s.scal[3];
-    __syncthreads();
-    int32_t* oi = p.sup_idx + i * (int64_t)p.budget;
-    float* ov = p.sup_val + i * (int64_t)p.budget;
     uint32_t T = 0u;
     int take_eq = 0;
-    if (tot > k) cand_kth(s, tot, k, G, T, take_eq);   // else every candidate is kept
-    const CandSrc cs{&s};
-    int dummy;
-    seg_count<CandSrc, false>(cs, tot, T, s, dummy, dummy);
-    seg_emit<CandSrc>(cs, tot, T, take_eq, s, oi, ov);
+    if (tot > k) cand_kth(s, tot, k, (uint32_t)s.scal[3], T, take_eq);  // else keep them all
+    // keys above T; count the keys equal to T
+    int ceq = 0;
+    for (int t = threadIdx.x; t < tot; t += blockDim.x) {
+        const uint32_t kv = s.ckey[t];
+        if (kv > T) {
+            const int x = s.cidx[t];
+            atomicOr(&bits[x >> 5], 1u << (x & 31));
+        }
+        ceq += kv == T && tot > k;
+    }
+    ceq = __reduce_add_sync(0xffffffffu, ceq);
+    if ((threadIdx.x & 31) == 0 && ceq) atomicAdd(&s_ceq, ceq);
+    __syncthreads();
+    if (take_eq > 0 && s_ceq > take_eq) {
+        // more keys tie at T than are taken: the cut-off is the take_eq-th smallest index
+        uint32_t* eqb = reinterpret_cast<uint32_t*>(pre);
+        for (int w = threadIdx.x; w < nw; w += blockDim.x) eqb[w] = 0u;
+        __syncthreads();
+        for (int t = threadIdx.x; t < tot; t += blockDim.x)
+            if (s.ckey[t] == T) atomicOr(&eqb[s.cidx[t] >> 5], 1u << (s.cidx[t] & 31));
+        __syncthreads();
+        const int per = (nw + kRtThreads - 1) / kRtThreads;
+        const int w0 = min(nw, (int)threadIdx.x * per), w1 = min(nw, w0 + per);
+        int c = 0;
+        for (int w = w0; w < w1; ++w) c += __popc(eqb[w]);
+        int tot_eq;
+        int run = block_exclusive_scan(c, s.hist, &tot_eq);
+        for (int w = w0; w < w1; ++w) {
+            const uint32_t word = eqb[w];
+            const int pc = __popc(word);
+            if (run < take_eq && take_eq <= run + pc) {
+                uint32_t m = word;
+                for (int r = take_eq - run; r > 1; --r) m &= m - 1;   // drop the lower bits
+                s_cut = w * 32 + (__ffs(m) - 1);
+            }
+            run += pc;
+        }
+        __syncthreads();
+    }
+    if (take_eq > 0) {
+        const int cut = s_cut;
+        for (int t = threadIdx.x; t < tot; t += blockDim.x) {
+            const int x = s.cidx[t];
+            if (s.ckey[t] == T && x <= cut) atomicOr(&bits[x >> 5], 1u << (x & 31));
+        }
+    }
+    __syncthreads();
+    word_prefix(bits, pre, nw, s);
+    int32_t* oi = p.sup_idx + i * (int64_t)p.budget;
+    float* ov = p.sup_val + i * (int64_t)p.budget;
+    for (int t = threadIdx.x; t < tot; t += blockDim.x) {
+        const int x = s.cidx[t];
+        const uint32_t word = bits[x >> 5];
+        const uint32_t bit = 1u << (x & 31);
+        if (word & bit) {
+            const int pos = pre[x >> 5] + __popc(word & (bit - 1u));
+            oi[pos] = x;
+            ov[pos] = oval(s.ckey[t]);
+        }
+    }
     for (int t = k + threadIdx.x; t < p.budget; t += blockDim.x) {
         oi[t] = -1;
         ov[t] = 0.f;
@@ -627,14 +687,21 @@ cudaError_t sample_tau(const float* slab, int64_t row0, int64_t row1, int L, int
     return cudaGetLastError();
 }
 
+int cand_select_smem(int64_t max_row_keys, int cap) {
+    const int64_t words = (max_row_keys + 31) / 32;
+    return (int)std::min<int64_t>(INT32_MAX, (int64_t)sizeof(RowSmem) + (int64_t)cap * 8 + words * 8);
+}
+
 cudaError_t cand_select(const void* cand, const int32_t* cnt, int64_t row0, int64_t row1,
                         int nseg, int seg_cap, int budget, int32_t* sup_idx, int32_t* sup_len,
                         float* sup_val, int32_t* fb, cudaStream_t st) {
     if (row1 <= row0) return cudaSuccess;
     if (nseg < 1 || nseg > kMaxSegments) return cudaErrorInvalidValue;
+    const int max_words = (int)((row1 + 31) / 32);
     CandSelParams p{reinterpret_cast<const uint2*>(cand), cnt, row0, (int)(row1 - row0), nseg,
-                    seg_cap, budget, sup_idx, sup_len, sup_val, fb};
-    const int smem = (int)sizeof(RowSmem) + nseg * seg_cap * 16;
+                    seg_cap, budget, max_words, sup_idx, sup_len, sup_val, fb};
+    const int smem = cand_select_smem(row1, nseg * seg_cap);
+    if (smem > kCandSelectMaxSmem) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(k_cand_select, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     k_cand_select<<<(unsigned)(row1 - row0), kRtThreads, smem, st>>>(p);

@@ -96,6 +96,7 @@ int64_t chunk_end(int64_t r0, int64_t N, int64_t cap) {
 // segments of a chunk, and finally the fallback rows' scratch (or, materialised,
 // the row slab of a chunk).
 struct StreamPlan {
+    bool materialise = false;     // rows written and selected instead (see below)
     int L = 0;                    // sample stride 2^L
     int nseg = 0, seg_cap = 0;    // candidate segments per row and entries per segment
     int cap = 0;                  // nseg * seg_cap: rows of at most cap keys keep every key
@@ -134,7 +135,10 @@ StreamPlan plan_stream(int64_t N, int budget, int nseg, size_t off) {
     const size_t cand_all = (size_t)N * sp.cap * 8;
     const size_t fb_pref = (size_t)std::min<int64_t>(N, kFallbackCtas) * N * 4;
     sp.region_pref = std::max({samples_all, cand_all, fb_pref});
-    if (materialise_rows()) sp.region_pref = std::max(sp.region_pref, slab_pref_bytes(N));
+    // the select keeps a bitmap of the row's keys in shared memory: rows too long for it
+    // (N beyond about 800K keys) are materialised and selected from the slab instead
+    sp.materialise = materialise_rows() || cand_select_smem(N, sp.cap) > kCandSelectMaxSmem;
+    if (sp.materialise) sp.region_pref = std::max(sp.region_pref, slab_pref_bytes(N));
     const int64_t s_max = ((N - 1) >> sp.L) + 1;
     sp.region_min = std::max({(size_t)std::min<int64_t>(N, kChunkRows) * s_max * 4,
                               (size_t)std::min<int64_t>(N, kChunkRows) * sp.cap * 8,
@@ -292,7 +296,7 @@ int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void*
     const StreamPlan& sp = plan.sp;
     char* region = ws + sp.off_region;
     const size_t region_bytes = ws_bytes - sp.off_region;
-    if (materialise_rows()) {
+    if (sp.materialise) {
         // mass rows of a chunk of queries, then their top-k, chunk by chunk
         const int64_t cap = (int64_t)(region_bytes / sizeof(float));
         ma.rows = (float*)region;
@@ -432,7 +436,7 @@ int run_indexer(int64_t N, int d_idx, int dtype, const void* q_idx, const void* 
     const StreamPlan& sp = plan.sp;
     char* region = ws + sp.off_region;
     const size_t region_bytes = ws_bytes - sp.off_region;
-    if (materialise_rows()) {
+    if (sp.materialise) {
         // score rows of a chunk of queries, then their top-k, chunk by chunk
         const int64_t cap = (int64_t)(region_bytes / sizeof(float));
         ia.rows = (float*)region;
@@ -907,7 +911,7 @@ int64_t tam_mass_fallback_rows(int64_t N, int Hq, int Hkv, int d, int dtype, int
     if (check_shape(N, Hq, Hkv, d, dtype) != TAM_OK || check_budget(N, budget_k, 1) != TAM_OK)
         return -1;
     const MassPlan plan = plan_mass(N, Hq, Hkv, d, dtype, budget_k, 1);
-    if (!plan.stream || materialise_rows()) return -1;
+    if (!plan.stream || plan.sp.materialise) return -1;
     return read_fallback_count(workspace, plan.sp.off_fb, stream);
 }
 
@@ -916,7 +920,7 @@ int64_t tam_indexer_fallback_rows(int64_t N, int d_idx, int dtype, int budget_k,
     if (N < 1 || d_idx < 1 || (dtype != TAM_BF16 && dtype != TAM_F32)) return -1;
     if (check_indexer_args(N, d_idx, dtype, budget_k, 1) != TAM_OK) return -1;
     const IndexerPlan plan = plan_indexer(N, d_idx, dtype, budget_k, 1);
-    if (!plan.tc || materialise_rows()) return -1;
+    if (!plan.tc || plan.sp.materialise) return -1;
     return read_fallback_count(workspace, plan.sp.off_fb, stream);
 }
 

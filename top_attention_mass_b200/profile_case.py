@@ -6,6 +6,9 @@ Rows: pass1_lse, pass2_mass_topk, pass2_block_mass_topk, pass3_gather, pass3_blo
 indexer_topk, dense_prefill.  Shapes are those of the 32K workload (Hq=32, Hkv=8,
 d=128, bf16, k=655, B_q=64, indexer d_idx=64 / k=1024) at the given N, so that a
 capture fits the profiler's size rules while the kernels are the benchmarked ones.
+pass3_gather_stress is the benchmark's out-of-L2 gather: per-query pass 3 on
+device-drawn inputs of the same head shape with a random support of k = 2048 (one
+uniform key per stratum of [0, i]); at N = 262144 its K/V halves are 537 MB each.
 Every launch is checked through the library's status block.
 """
 import argparse
@@ -20,7 +23,19 @@ import tam_synth  # noqa: E402
 import top_attention_mass_b200 as tam  # noqa: E402
 
 ROWS = ("pass1_lse", "pass2_mass_topk", "pass2_block_mass_topk", "pass3_gather", "pass3_block",
-        "indexer_topk", "dense_prefill")
+        "indexer_topk", "dense_prefill", "pass3_gather_stress")
+
+
+def gather_stress(N, reps):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    q = torch.randn(N, 32, 128, generator=g, device="cuda").to(torch.bfloat16)
+    k = torch.randn(N, 8, 128, generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn(N, 8, 128, generator=g, device="cuda").to(torch.bfloat16)
+    idx, ln = tam_synth.stratified_support(N, 2048, seed=9, device="cuda")
+    for _ in range(reps):
+        tam.sparse_support_attention(q, k, v, idx, ln, 1)
+    torch.cuda.synchronize()
 
 
 def main():
@@ -29,6 +44,10 @@ def main():
     ap.add_argument("--N", type=int, default=16384)
     ap.add_argument("--reps", type=int, default=3)
     a = ap.parse_args()
+    if a.row == "pass3_gather_stress":
+        gather_stress(a.N, a.reps)
+        print(f"profile_case {a.row} N={a.N} reps={a.reps} ok")
+        return
     w = tam_synth.WORKLOADS["indexer32k"]
     inp = tam_synth.make_inputs(w, N=a.N)
     q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
