@@ -498,9 +498,12 @@ def run_ours(args, w, inp, rank, world, local_rank):
     traffic = traffic_table()
     row_ms = row_times(calls, names, flush, args.steps)
     tam.check_status(calls.ws.get(256))
+    # the dense comparator on the same layer (every workload), for the sparse-pass speedup
+    dense_ms = row_times(calls, ("dense_prefill",), flush, args.steps)["dense_prefill"]
+    tam.check_status(calls.ws.get(256))
 
     extra = {}
-    if w.name == WORKLOAD:
+    if w.name == WORKLOAD and not args.no_extras:
         extra = measure_extras(args, tam, w, calls, flush, dev)
     work = algorithmic_work(calls, w.N)
     rows = {}
@@ -525,6 +528,12 @@ def run_ours(args, w, inp, rank, world, local_rank):
         "config": config_dict(w, world),
         "roofline": {**rows[dominant]["roofline"], "kernel": dominant},
         "rows": rows,
+        "dense_comparator": {
+            "ms": dense_ms, "q_tok_s": w.N / (dense_ms * 1e-3),
+            "roofline": roofline_of({"bound": "tensor", "flops": 4.0 * w.d * w.Hq * causal_pairs(w.N)},
+                                    dense_ms, pk, pk_kind),
+            "step_vs_dense": dense_ms / ms_step,
+            "sparse_pass3_speedup_vs_dense": dense_ms / row_ms[names[-1]]},
         "timed_region_ms": region_ms,
         "warm_l2_ms_per_step": warm_ms,
         "fallback_rows": fb_rows,
@@ -853,6 +862,9 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the step and its passes only (no block-shared call, all-rows "
+                         "step, out-of-L2 gather, support quality or next rows)")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="gqa32k_2pct (default), gqa4k_needles, longctx_<N>, indexer32k")
     args = ap.parse_args()

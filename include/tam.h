@@ -89,16 +89,18 @@ const char* tam_status_string(int status);
  * Workspace bytes tam_mass_oracle_prefill prefers for this problem (always a
  * multiple of 256).  Returns 0 for arguments that the call would reject.
  * Per query on the tensor cores, pass 2 selects without writing the mass rows:
- *   1. a sample pass scores every 2^L-th key of each row (L >= 4, the smallest
- *      leaving at most 4096 sampled keys per row) and sets the row's threshold
- *      tau_i = the r-th largest sampled mass, r = ceil(mu + 5 sqrt(mu) + 4) with
- *      mu = s min(k, i+1) / (i+1) the expected number of sampled keys at or above
- *      the k-th value among the row's s = (i >> L) + 1 samples (rows of at most
- *      `cap` keys keep every key: tau_i = -inf);
+ *   1. a sample pass scores every S-th key of each row (S the smallest prime of
+ *      at least 17 that leaves at most 4096 sampled keys per row; a prime stride
+ *      does not line up with power-of-two structure in the key positions) and sets
+ *      the row's threshold tau_i = the r-th largest sampled mass,
+ *      r = ceil(mu + 5 sqrt(mu) + 4) with mu = s min(k, i+1) / (i+1) the expected
+ *      number of sampled keys at or above the k-th value among the row's
+ *      s = i / S + 1 samples (rows of at most `cap` keys keep every key:
+ *      tau_i = -inf);
  *   2. the scoring pass keeps only the keys with P_i[j] >= tau_i, in nseg
  *      candidate segments per row (8 on CTA pairs, 4 otherwise) of seg_cap
- *      entries each, seg_cap = 32 * ceil((ceil(1.5 * 2^L * (r0 + 1) / nseg) + 32)
- *      / 32), r0 the threshold rank for mu = k / 2^L, cap = nseg * seg_cap;
+ *      entries each, seg_cap = 32 * ceil((ceil(1.5 * S * (r0 + 1) / nseg) + 32)
+ *      / 32), r0 the threshold rank for mu = k / S, cap = nseg * seg_cap;
  *   3. an exact select runs over each row's candidates; a row whose candidates
  *      fell short of min(k, i+1) or overflowed a segment is recomputed whole on
  *      the CUDA cores and selected exactly (the results are the same).

@@ -211,29 +211,29 @@ def test_packed_batch_helpers():
 
 def _stream_layout(N, k, nseg, head):
     """The streamed per-query selection's workspace after `head` bytes, as include/tam.h
-    documents it: sample stride 2^L (the smallest L >= 4 leaving at most 4096 sampled
-    keys per row), segment capacity from the threshold rank, then tau, the fallback
-    list, the counts and a region that holds the sample rows, the candidates or the
-    fallback scratch; returns (preferred, minimum) sizes."""
+    documents it: sample stride S (the smallest prime of at least 17 leaving at most
+    4096 sampled keys per row), segment capacity from the threshold rank, then tau, the
+    fallback list, the counts and a region that holds the sample rows, the candidates
+    or the fallback scratch; returns (preferred, minimum) sizes."""
     import math
     a256 = lambda x: (x + 255) // 256 * 256              # noqa: E731
-    L = 4
-    while ((N - 1) >> L) + 1 > 4096:
-        L += 1
-    mu = k / (1 << L)
+    S = max(17, -(-N // 4096))
+    while any(S % f == 0 for f in range(2, int(math.isqrt(S)) + 1)) or (N - 1) // S + 1 > 4096:
+        S += 1
+    mu = k / S
     r = math.ceil(mu + 5.0 * math.sqrt(mu) + 4.0)
-    per = math.ceil(1.5 * (1 << L) * (r + 1.0) / nseg) + 32
+    per = math.ceil(1.5 * S * (r + 1.0) / nseg) + 32
     seg_cap = (per + 31) // 32 * 32
     cap = nseg * seg_cap
     off_region = head + a256(N * 4) + a256((N + 1) * 4) + a256(N * nseg * 4)
 
     def sample_offset(i):
-        a, b = i >> L, i & ((1 << L) - 1)
-        return i + ((a * (a - 1) // 2) << L) + a * b
+        a, b = i // S, i % S
+        return i + S * (a * (a - 1) // 2) + a * b
 
     tri = N * (N + 1) // 2
     pref = max(sample_offset(N) * 4, N * cap * 8, min(N, 148) * N * 4)
-    s_max = ((N - 1) >> L) + 1
+    s_max = (N - 1) // S + 1
     lo = max(min(N, 64) * s_max * 4, min(N, 64) * cap * 8, min(tri, 64 * N) * 4)
     return off_region + a256(pref), off_region + a256(lo)
 

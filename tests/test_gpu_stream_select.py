@@ -143,3 +143,22 @@ def test_gqa32k_needs_no_fallback(tam_lib):
     ws = tam_lib.Workspace()
     _select(tam_lib, q, k, lse, w.budget_k, ws)
     assert tam_lib.mass_fallback_rows(q, k, w.budget_k, ws) == 0
+
+
+def test_rope_grid_needles_need_almost_no_fallback(tam_lib, oracle_mod):
+    """The long-context tensors (RoPE, sink, needles on a grid of N/32 positions) per
+    query: the sampled thresholds hold (at most one row in a thousand falls back), and
+    sampled rows match the oracle."""
+    w = tam_synth.WORKLOADS["longctx_16384"]
+    inp = tam_synth.make_inputs(w)
+    q, k = inp.q.cuda(), inp.k.cuda()
+    lse = tam_lib.attention_lse(q, k)
+    ws = tam_lib.Workspace()
+    kb = 655
+    res = _select(tam_lib, q, k, lse, kb, ws)
+    assert tam_lib.mass_fallback_rows(q, k, kb, ws) <= w.N // 1000
+    rows = tam_synth.sample_rows(w.N, inp.needle_i, n_random=64)
+    oi, ol, _ = oracle_mod.topk_rows(inp.q, inp.k, kb, rows)
+    P = oracle_mod.mass_rows(inp.q, inp.k, rows)
+    check_support(res.idx.cpu().numpy()[rows], res.length.cpu().numpy()[rows],
+                  res.value.cpu().numpy()[rows], oi, ol, P, MASS_ATOL, "rope grid needles")

@@ -29,7 +29,7 @@ struct MassArgs {
     float* scratch;       // n_ctas * N floats (CUDA-core path)
     float* rows;          // triangular slab of mass rows (tensor-core path, per query)
     int64_t row0, row1;   // the queries whose rows this launch writes (per query)
-    int kst_log2;         // rows mode: only the keys j = m << kst_log2 (sample rows)
+    int kst;              // rows mode: only the keys j = m * kst (sample rows); 1 = every key
     bool stream;          // per query: threshold-filtered candidates instead of rows
     const float* tau;     // stream: threshold of every query [N]
     void* cand;           // stream: candidate segments of the rows [row0, row1)
@@ -67,7 +67,7 @@ struct IndexerArgs {
     float* scratch;       // n_ctas * N floats (CUDA-core path)
     float* rows;          // triangular slab of score rows (tensor-core path)
     int64_t row0, row1;   // the queries whose rows this launch writes
-    int kst_log2;         // rows mode: only the keys j = m << kst_log2 (sample rows)
+    int kst;              // rows mode: only the keys j = m * kst (sample rows); 1 = every key
     bool stream;          // threshold-filtered candidates instead of rows
     const float* tau;
     void* cand;
@@ -108,18 +108,19 @@ inline int64_t tri(int64_t i) { return i * (i + 1) / 2; }
 // ties toward the smaller index; sup_* are indexed by the absolute row i.
 cudaError_t row_topk(const float* slab, int64_t row0, int64_t row1, int budget, int32_t* sup_idx,
                      int32_t* sup_len, float* sup_val, cudaStream_t st);
-// Rows sampled every 2^L keys: row i' holds (i' >> L) + 1 values; row i starts
-// sample_offset(i, L) - sample_offset(row0, L) floats after the slab base.
-__host__ __device__ inline int64_t sample_offset(int64_t i, int L) {
-    const int64_t a = i >> L, b = i & ((int64_t(1) << L) - 1);
-    return i + ((a * (a - 1) / 2) << L) + a * b;
+// Rows sampled every S keys: row i' holds i' / S + 1 values, so the rows before
+// i = a S + b hold i + S a (a - 1) / 2 + a b (tri(i) for S = 1); row i starts
+// sample_offset(i, S) - sample_offset(row0, S) floats after the slab base.
+__host__ __device__ inline int64_t sample_offset(int64_t i, int S) {
+    const int64_t a = i / S, b = i - a * S;
+    return i + S * (a * (a - 1) / 2) + a * b;
 }
 // Per-row thresholds from a sample slab: for rows of at most `take_all` keys
 // tau = -inf (every key is a candidate); otherwise the r-th largest of the row's
-// s = (i >> L) + 1 samples, r = ceil(mu + z sqrt(mu) + 4), mu = s min(k, i+1) / (i+1),
+// s = i / S + 1 samples, r = ceil(mu + z sqrt(mu) + 4), mu = s min(k, i+1) / (i+1),
 // clamped to [1, s].  `force` (debug): 1 sets tau = +inf, 2 tau = -inf on the
 // sampled rows, so that every such row falls back.
-cudaError_t sample_tau(const float* slab, int64_t row0, int64_t row1, int L, int budget,
+cudaError_t sample_tau(const float* slab, int64_t row0, int64_t row1, int S, int budget,
                        int take_all, float z, int force, float* tau, cudaStream_t st);
 // Exact top-min(k, i+1) of each row i in [row0, row1) from its candidate segments
 // (nseg per row, seg_cap entries each, (value bits, key) in key order, counts in cnt),

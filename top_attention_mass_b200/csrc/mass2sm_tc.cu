@@ -76,7 +76,7 @@ __host__ __device__ constexpr int pair_stages(int D, int Hkv) {
 struct PairParams {
     int N, Hq, Hkv, pair0, n_pairs, block_q;
     int64_t row0, row1;       // per query: the rows [row0, row1) of this launch
-    int kst_log2;             // rows mode: key m of the K map sits at position m << kst_log2
+    int kst;                  // rows mode: key m of the K map sits at position m * kst
     int seg_cap;              // stream mode: entries per candidate segment
     int stages;               // key tiles in the K ring
     float sl2, inv_hq;
@@ -143,10 +143,10 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int pt = p.pair0 + p.n_pairs - 1 - (int)(blockIdx.x >> 1);   // heaviest pair first
     const int q0 = pt * BQP;
     const int q_last = min(p.N, q0 + BQP) - 1;
-    const int n_kt = (q_last >> p.kst_log2) / kTileKeys + 1;
+    const int n_kt = (q_last / p.kst) / kTileKeys + 1;
     const int n_units = n_kt * Hkv;
     const int my_q0 = q0 + (int)rank * BQC;
-    const int64_t slab0 = sample_offset(p.row0, p.kst_log2);
+    const int64_t slab0 = sample_offset(p.row0, p.kst);
 
     if (threadIdx.x == 0) {
         tc::mbar_init(q_full, 1);
@@ -312,12 +312,12 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             if constexpr (MODE == kModeRows) {
                 // row i of the slab starts off(i) - off(row0) floats in; lanes store
                 // consecutive keys of one query
-                const int64_t j = (int64_t)m << p.kst_log2;
+                const int64_t j = (int64_t)m * p.kst;
 #pragma unroll
                 for (int ql = 0; ql < kQP; ++ql) {
                     const int64_t i = q0 + part * kQP + ql;
                     if (j <= i && i >= p.row0 && i < p.row1)
-                        p.rows[sample_offset(i, p.kst_log2) - slab0 + m] = acc[ql] * p.inv_hq;
+                        p.rows[sample_offset(i, p.kst) - slab0 + m] = acc[ql] * p.inv_hq;
                 }
             } else if constexpr (STREAM) {
                 // keys at or above the query's threshold, appended in key order to this
@@ -393,12 +393,12 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     constexpr int BQP = kNQ / G, BQC = kHalfRows / G;
     CUtensorMap tq, tk;
     const uint64_t d = a.d;
-    // rows mode with a key stride reads every 2^L-th key row: the same K with an L-fold
-    // longer row pitch and (N - 1) >> L + 1 rows
-    const int L = MODE == kModeRows ? a.kst_log2 : 0;
-    const uint64_t n_keys = (uint64_t)((a.N - 1) >> L) + 1;
+    // rows mode with a key stride reads every S-th key row: the same K with an S-fold
+    // longer row pitch and (N - 1) / S + 1 rows
+    const int S = (MODE == kModeRows && a.kst > 1) ? a.kst : 1;
+    const uint64_t n_keys = (uint64_t)((a.N - 1) / S) + 1;
     if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQC) ||
-        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, n_keys, d * 2, ((uint64_t)a.Hkv * d * 2) << L, 64,
+        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, n_keys, d * 2, (uint64_t)a.Hkv * d * 2 * S, 64,
                            1, 128))
         return cudaErrorInvalidValue;
     PairParams p{};
@@ -411,7 +411,7 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     p.n_pairs = (int)((r1 + BQP - 1) / BQP) - p.pair0;
     p.row0 = r0;
     p.row1 = r1;
-    p.kst_log2 = L;
+    p.kst = S;
     p.seg_cap = a.seg_cap;
     p.stages = pair_stages(D, a.Hkv);
     {   // TAM_PAIR_STAGES=n caps the ring (A/B comparisons)

@@ -1,8 +1,8 @@
 // Pass 2 on the tensor cores: head-averaged token mass (and the indexer's scores).
 //
 //   P_i[j] = (1/Hq) sum_h exp(scale * q[i,h].k[j,g(h)] - lse[h,i]),  j <= i
-//   per query:  the rows P_i, written to a triangular slab (with a key stride 2^L
-//               only the sampled keys j = m 2^L); row_topk.cu then selects
+//   per query:  the rows P_i, written to a triangular slab (with a key stride S
+//               only the sampled keys j = m S); row_topk.cu then selects
 //               S_i = top-min(k, i+1) of each row (value desc, index asc);
 //               or, streamed, only the keys with P_i[j] >= tau_i, appended to the
 //               row's candidate segments (one per mass warp) for cand_select
@@ -60,7 +60,7 @@ constexpr int kMaxDynSmem = 227 * 1024;
 struct MassParams {
     int N, Hq, Hkv, ct0, n_ctiles, block_q;
     int64_t row0, row1;              // per query / indexer: the rows [row0, row1)
-    int kst_log2;                    // rows modes: key m of the K map is at m << kst_log2
+    int kst;                         // rows modes: key m of the K map is at m * kst
     int seg_cap;                     // stream modes: entries per candidate segment
     float sl2, inv_hq;
     const float* lse;
@@ -116,9 +116,9 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int ct = p.ct0 + p.n_ctiles - 1 - (int)blockIdx.x;   // heaviest tile first
     const int q0 = ct * BQ;
     const int q_last = min(p.N, q0 + BQ) - 1;
-    const int n_kt = (q_last >> p.kst_log2) / 128 + 1;
+    const int n_kt = (q_last / p.kst) / 128 + 1;
     const int n_units = n_kt * Hkv;
-    const int64_t slab0 = sample_offset(p.row0, p.kst_log2);
+    const int64_t slab0 = sample_offset(p.row0, p.kst);
 
     if (threadIdx.x == 0) {
         tc::mbar_init(q_full, 1);
@@ -309,12 +309,12 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             } else if constexpr (!BLOCK) {
                 // row i of the slab starts off(i) - off(row0) floats in; lanes store
                 // consecutive keys of one query
-                const int64_t jp = (int64_t)j << p.kst_log2;  // key position
+                const int64_t jp = (int64_t)j * p.kst;        // key position
 #pragma unroll
                 for (int q = 0; q < kQP; ++q) {
                     const int64_t i = qp0 + q;
                     if (jp <= i && i >= p.row0 && i < p.row1)
-                        p.rows[sample_offset(i, p.kst_log2) - slab0 + j] =
+                        p.rows[sample_offset(i, p.kst) - slab0 + j] =
                             INDEXER ? acc[q] : acc[q] * p.inv_hq;
                 }
             } else {
@@ -447,12 +447,12 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     constexpr bool ROWS = MODE == kModeQuery || MODE == kModeIndexer;
     CUtensorMap tq, tk;
     const uint64_t d = a.d;
-    // rows modes with a key stride read every 2^L-th key row: the same K with an
-    // L-fold longer row pitch and (N - 1) >> L + 1 rows
-    const int L = ROWS ? a.kst_log2 : 0;
-    const uint64_t n_keys = (uint64_t)((a.N - 1) >> L) + 1;
+    // rows modes with a key stride read every S-th key row: the same K with an
+    // S-fold longer row pitch and (N - 1) / S + 1 rows
+    const int S = (ROWS && a.kst > 1) ? a.kst : 1;
+    const uint64_t n_keys = (uint64_t)((a.N - 1) / S) + 1;
     if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQ) ||
-        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, n_keys, d * 2, ((uint64_t)a.Hkv * d * 2) << L, 64,
+        !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, n_keys, d * 2, (uint64_t)a.Hkv * d * 2 * S, 64,
                            1, 128))
         return cudaErrorInvalidValue;
     MassParams p{};
@@ -466,7 +466,7 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     p.n_ctiles = (int)((r1 + BQ - 1) / BQ) - p.ct0;
     p.row0 = r0;
     p.row1 = r1;
-    p.kst_log2 = L;
+    p.kst = S;
     p.seg_cap = a.seg_cap;
     p.block_q = a.block_q;
     p.sl2 = a.sl2;
@@ -613,7 +613,7 @@ cudaError_t tc_indexer_rows(const IndexerArgs& ia, cudaStream_t st) {
     a.rows = ia.rows;
     a.row0 = ia.row0;
     a.row1 = ia.row1;
-    a.kst_log2 = ia.kst_log2;
+    a.kst = ia.kst;
     a.stream = ia.stream;
     a.tau = ia.tau;
     a.cand = ia.cand;

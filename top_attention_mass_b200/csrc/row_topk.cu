@@ -455,7 +455,7 @@ __global__ void __launch_bounds__(kRtThreads, 6) k_row_topk(const RowTopkParams 
 struct SampleTauParams {
     const float* slab;
     int64_t row0;
-    int n_rows, L, budget, take_all, force;
+    int n_rows, S, budget, take_all, force;
     float z;
     float* tau;
 };
@@ -473,8 +473,8 @@ __global__ void __launch_bounds__(kRtThreads) k_sample_tau(const SampleTauParams
         if (threadIdx.x == 0) p.tau[i] = p.force == 1 ? INFINITY : -INFINITY;
         return;
     }
-    const int ns = (int)(i >> p.L) + 1;
-    const float* row = p.slab + (sample_offset(i, p.L) - sample_offset(p.row0, p.L));
+    const int ns = (int)(i / p.S) + 1;
+    const float* row = p.slab + (sample_offset(i, p.S) - sample_offset(p.row0, p.S));
     if (threadIdx.x == 0) {
         s.ckey = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowSmem));
         s.cmax = 0u;
@@ -674,11 +674,11 @@ __global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams 
 
 }  // namespace
 
-cudaError_t sample_tau(const float* slab, int64_t row0, int64_t row1, int L, int budget,
+cudaError_t sample_tau(const float* slab, int64_t row0, int64_t row1, int S, int budget,
                        int take_all, float z, int force, float* tau, cudaStream_t st) {
     if (row1 <= row0) return cudaSuccess;
-    SampleTauParams p{slab, row0, (int)(row1 - row0), L, budget, take_all, force, z, tau};
-    const int max_samples = (int)((row1 - 1) >> L) + 1;
+    SampleTauParams p{slab, row0, (int)(row1 - row0), S, budget, take_all, force, z, tau};
+    const int max_samples = (int)((row1 - 1) / S) + 1;
     const int smem = (int)sizeof(RowSmem) + max_samples * 4;
     cudaError_t e = cudaFuncSetAttribute(k_sample_tau, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

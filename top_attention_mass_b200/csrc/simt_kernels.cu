@@ -195,6 +195,29 @@ __global__ void __launch_bounds__(256) k_indexer_select_simt(
 // or a full candidate segment): each persistent block takes rows off the list
 // fb (fb[0] = count, fb[1 + t] = row), computes the whole row into its scratch row
 // and selects from it exactly.
+// Eight consecutive elements of a row as floats (one 16-byte load for bf16, two for fp32).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&x)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        x[2 * e] = f.x;
+        x[2 * e + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void load8(const float* p, float (&x)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+// Thread = key: for each KV group it reads the key row in 16-byte pieces and adds the
+// dot products of all G query heads of the group (at most kMaxG) at once, the query
+// row staged in shared memory as fp32 (read as broadcasts).
+constexpr int kMaxG = 16;
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_mass_rows_fallback(
     const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ lse, int N, int Hq,
@@ -217,12 +240,27 @@ __global__ void __launch_bounds__(256) k_mass_rows_fallback(
         __syncthreads();
         for (int j = threadIdx.x; j <= i; j += blockDim.x) {
             float p = 0.f;
-            for (int h = 0; h < Hq; ++h) {
-                const T* kj = k + ((size_t)j * Hkv + h / G) * d;
-                const float* qh = qs + h * d;
-                float sc = 0.f;
-                for (int c = 0; c < d; ++c) sc = fmaf(qh[c], to_f(kj[c]), sc);
-                p += exp2f(sc * sl2 - lse2[h]);
+            for (int g = 0; g < Hkv; ++g) {
+                const T* kj = k + ((size_t)j * Hkv + g) * d;
+                const float* qg = qs + (size_t)g * G * d;
+                float dot[kMaxG];
+#pragma unroll
+                for (int hh = 0; hh < kMaxG; ++hh) dot[hh] = 0.f;
+                for (int c = 0; c < d; c += 8) {
+                    float kv[8];
+                    load8(kj + c, kv);
+#pragma unroll
+                    for (int hh = 0; hh < kMaxG; ++hh) {
+                        if (hh < G) {
+                            const float* qh = qg + hh * d + c;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) dot[hh] = fmaf(qh[e], kv[e], dot[hh]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int hh = 0; hh < kMaxG; ++hh)
+                    if (hh < G) p += exp2f(dot[hh] * sl2 - lse2[g * G + hh]);
             }
             row[j] = p * inv_hq;
         }
@@ -249,7 +287,12 @@ __global__ void __launch_bounds__(256) k_indexer_rows_fallback(
         for (int j = threadIdx.x; j <= i; j += blockDim.x) {
             const T* kj = kx + (size_t)j * dx;
             float sc = 0.f;
-            for (int c = 0; c < dx; ++c) sc = fmaf(qs[c], to_f(kj[c]), sc);
+            for (int c = 0; c < dx; c += 8) {
+                float kv[8];
+                load8(kj + c, kv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sc = fmaf(qs[c + e], kv[e], sc);
+            }
             row[j] = sc;
         }
         __syncthreads();
@@ -351,7 +394,8 @@ static cudaError_t launch_mass_fallback(const MassArgs& a, const int32_t* fb, fl
 
 cudaError_t fallback_mass_rows(const MassArgs& a, const int32_t* fb, float* scratch, int n_ctas,
                                cudaStream_t st) {
-    if (n_ctas < 1) return cudaErrorInvalidValue;
+    // the fallback reads rows in 8-element pieces and holds one dot product per head of a group
+    if (n_ctas < 1 || a.d % 8 != 0 || a.Hq / a.Hkv > kMaxG) return cudaErrorInvalidValue;
     return a.dtype == TAM_F32 ? launch_mass_fallback<float>(a, fb, scratch, n_ctas, st)
                               : launch_mass_fallback<__nv_bfloat16>(a, fb, scratch, n_ctas, st);
 }
@@ -368,7 +412,7 @@ static cudaError_t launch_indexer_fallback(const IndexerArgs& a, const int32_t* 
 
 cudaError_t fallback_indexer_rows(const IndexerArgs& a, const int32_t* fb, float* scratch,
                                   int n_ctas, cudaStream_t st) {
-    if (n_ctas < 1) return cudaErrorInvalidValue;
+    if (n_ctas < 1 || a.d_idx % 8 != 0) return cudaErrorInvalidValue;
     return a.dtype == TAM_F32 ? launch_indexer_fallback<float>(a, fb, scratch, n_ctas, st)
                               : launch_indexer_fallback<__nv_bfloat16>(a, fb, scratch, n_ctas, st);
 }

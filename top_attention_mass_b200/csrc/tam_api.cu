@@ -51,7 +51,7 @@ inline int64_t n_selection_units(int64_t N, int block_q) {
 }
 
 // Per-query selection on the tensor cores (pass 2 and the indexer) streams: a sample
-// pass scores every 2^L-th key of each row and sets the row's threshold tau_i, then
+// pass scores every S-th key of each row and sets the row's threshold tau_i, then
 // the scoring kernel keeps only the keys at or above tau_i, in fixed candidate
 // segments, and an exact select runs over those; rows whose candidates fall short
 // or overflow are recomputed whole on the CUDA cores.  Nothing of size N x N is
@@ -97,41 +97,50 @@ int64_t chunk_end(int64_t r0, int64_t N, int64_t cap) {
 // the row slab of a chunk).
 struct StreamPlan {
     bool materialise = false;     // rows written and selected instead (see below)
-    int L = 0;                    // sample stride 2^L
+    int S = 1;                    // sample stride: every S-th key is scored
     int nseg = 0, seg_cap = 0;    // candidate segments per row and entries per segment
     int cap = 0;                  // nseg * seg_cap: rows of at most cap keys keep every key
     size_t off_tau = 0, off_fb = 0, off_cnt = 0, off_region = 0;
     size_t region_pref = 0, region_min = 0;
 };
 
-int sample_log2(int64_t N) {
-    int L = 4;
-    while (((N - 1) >> L) + 1 > kMaxSamplesPerRow) ++L;
-    return L;
+// Sample stride: the smallest prime of at least 17 that leaves at most
+// kMaxSamplesPerRow sampled keys per row.  A prime stride does not line up with
+// power-of-two structure in the key positions (a document or chunk grid, tokens
+// planted every N/32 positions), which would put such keys in every row's sample.
+int sample_stride(int64_t N) {
+    int64_t S = std::max<int64_t>(17, (N + kMaxSamplesPerRow - 1) / kMaxSamplesPerRow);
+    auto prime = [](int64_t x) {
+        for (int64_t f = 2; f * f <= x; ++f)
+            if (x % f == 0) return false;
+        return true;
+    };
+    while (!prime(S) || ((N - 1) / S) + 1 > kMaxSamplesPerRow) ++S;
+    return (int)S;
 }
 
-// Threshold rank r = ceil(mu + z sqrt(mu) + 4) of mu = k / 2^L expected sampled keys
-// at or above the k-th value; about 2^L (r + 1) keys of a row then pass, and the
+// Threshold rank r = ceil(mu + z sqrt(mu) + 4) of mu = k / S expected sampled keys
+// at or above the k-th value; about S (r + 1) keys of a row then pass, and the
 // segments hold half as many again (plus 32 each) before they overflow.
-int segment_capacity(int budget, int L, int nseg) {
-    const double mu = (double)budget / (double)(1 << L);
+int segment_capacity(int budget, int S, int nseg) {
+    const double mu = (double)budget / (double)S;
     const double r = std::ceil(mu + kTauSigmas * std::sqrt(mu) + 4.0);
-    const double expect = (double)(1 << L) * (r + 1.0);
+    const double expect = (double)S * (r + 1.0);
     const int per = (int)std::ceil(1.5 * expect / nseg) + 32;
     return (per + 31) & ~31;
 }
 
 StreamPlan plan_stream(int64_t N, int budget, int nseg, size_t off) {
     StreamPlan sp;
-    sp.L = sample_log2(N);
+    sp.S = sample_stride(N);
     sp.nseg = nseg;
-    sp.seg_cap = segment_capacity(budget, sp.L, nseg);
+    sp.seg_cap = segment_capacity(budget, sp.S, nseg);
     sp.cap = nseg * sp.seg_cap;
     sp.off_tau = off;
     sp.off_fb = sp.off_tau + align256((size_t)N * 4);
     sp.off_cnt = sp.off_fb + align256((size_t)(N + 1) * 4);
     sp.off_region = sp.off_cnt + align256((size_t)N * nseg * 4);
-    const size_t samples_all = (size_t)sample_offset(N, sp.L) * 4;
+    const size_t samples_all = (size_t)sample_offset(N, sp.S) * 4;
     const size_t cand_all = (size_t)N * sp.cap * 8;
     const size_t fb_pref = (size_t)std::min<int64_t>(N, kFallbackCtas) * N * 4;
     sp.region_pref = std::max({samples_all, cand_all, fb_pref});
@@ -139,7 +148,7 @@ StreamPlan plan_stream(int64_t N, int budget, int nseg, size_t off) {
     // (N beyond about 800K keys) are materialised and selected from the slab instead
     sp.materialise = materialise_rows() || cand_select_smem(N, sp.cap) > kCandSelectMaxSmem;
     if (sp.materialise) sp.region_pref = std::max(sp.region_pref, slab_pref_bytes(N));
-    const int64_t s_max = ((N - 1) >> sp.L) + 1;
+    const int64_t s_max = (N - 1) / sp.S + 1;
     sp.region_min = std::max({(size_t)std::min<int64_t>(N, kChunkRows) * s_max * 4,
                               (size_t)std::min<int64_t>(N, kChunkRows) * sp.cap * 8,
                               slab_min_bytes(N)});
@@ -147,7 +156,7 @@ StreamPlan plan_stream(int64_t N, int budget, int nseg, size_t off) {
 }
 
 // The streamed per-query selection over a region of `region_bytes` (>= region_min).
-// sample(r0, r1, L, slab) scores the sampled keys of rows [r0, r1) into slab;
+// sample(r0, r1, S, slab) scores the sampled keys of rows [r0, r1) into slab;
 // scan(c0, c1) writes the candidate segments and counts of rows [c0, c1) to the
 // region; fallback(fb, scratch, n_ctas) redoes the listed rows.
 template <class Sample, class Scan, class Fallback>
@@ -163,14 +172,14 @@ cudaError_t run_stream_select(const StreamPlan& sp, char* ws, size_t region_byte
     // rows of at most cap keys keep every key: no samples needed below r_start
     const int64_t r_start = std::min<int64_t>(N, (sp.cap / kChunkRows) * kChunkRows);
     const int force = debug_force_fallback();
-    if ((e = sample_tau(nullptr, 0, r_start, sp.L, budget, sp.cap, kTauSigmas, force, tau, st)))
+    if ((e = sample_tau(nullptr, 0, r_start, sp.S, budget, sp.cap, kTauSigmas, force, tau, st)))
         return e;
-    const int L = sp.L;
+    const int S = sp.S;
     const int64_t slab_cap = (int64_t)(region_bytes / 4);
     for (int64_t r0 = r_start; r0 < N;) {
-        const int64_t r1 = chunk_end_by(r0, N, slab_cap, [L](int64_t i) { return sample_offset(i, L); });
-        if ((e = sample(r0, r1, L, (float*)region))) return e;
-        if ((e = sample_tau((const float*)region, r0, r1, L, budget, sp.cap, kTauSigmas, force, tau,
+        const int64_t r1 = chunk_end_by(r0, N, slab_cap, [S](int64_t i) { return sample_offset(i, S); });
+        if ((e = sample(r0, r1, S, (float*)region))) return e;
+        if ((e = sample_tau((const float*)region, r0, r1, S, budget, sp.cap, kTauSigmas, force, tau,
                             st)))
             return e;
         r0 = r1;
@@ -312,9 +321,9 @@ int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void*
         }
         return TAM_OK;
     }
-    auto sample = [&](int64_t r0, int64_t r1, int L, float* slab) {
+    auto sample = [&](int64_t r0, int64_t r1, int S, float* slab) {
         MassArgs a = ma;
-        a.row0 = r0; a.row1 = r1; a.kst_log2 = L; a.rows = slab;
+        a.row0 = r0; a.row1 = r1; a.kst = S; a.rows = slab;
         return tc_mass_pass(a, st);
     };
     auto scan = [&](int64_t c0, int64_t c1, const float* tau, void* cand, int32_t* cnt) {
@@ -452,9 +461,9 @@ int run_indexer(int64_t N, int d_idx, int dtype, const void* q_idx, const void* 
         }
         return TAM_OK;
     }
-    auto sample = [&](int64_t r0, int64_t r1, int L, float* slab) {
+    auto sample = [&](int64_t r0, int64_t r1, int S, float* slab) {
         IndexerArgs a = ia;
-        a.row0 = r0; a.row1 = r1; a.kst_log2 = L; a.rows = slab;
+        a.row0 = r0; a.row1 = r1; a.kst = S; a.rows = slab;
         return tc_indexer_rows(a, st);
     };
     auto scan = [&](int64_t c0, int64_t c1, const float* tau, void* cand, int32_t* cnt) {
