@@ -271,14 +271,17 @@ def time_replays(graph, flush, steps, warm=False):
 
 
 def row_times(calls, names, flush, steps):
-    """Eager per-row device times: CUDA events between the calls, L2 flushed first."""
+    """Eager per-row device times: CUDA events between the calls, L2 flushed first; one
+    untimed round first, then the median over `steps` rounds (an eager call's events also
+    see host-side gaps, which the median keeps out)."""
+    calls.rows(names)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
           for _ in range(steps)]
     for s in range(steps):
         flush.fill_(s & 0xff)
         calls.rows(names, ev[s])
     torch.cuda.synchronize()
-    return {n: statistics.mean(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps))
+    return {n: statistics.median(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps))
             for i, n in enumerate(names)}
 
 
@@ -700,7 +703,7 @@ def measure_next_rows(args, tam, w, calls, flush):
             ev[s][-1].record()
         torch.cuda.synchronize()
         tam.check_status(ws.get(256))
-        return [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(len(fns))]
+        return [statistics.median(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(len(fns))]
 
     box = {}
 

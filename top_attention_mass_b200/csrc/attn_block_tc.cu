@@ -8,22 +8,26 @@
 // selected once for a block of consecutive queries.)
 //
 // The flash-style pipeline of the dense kernel over gathered keys.  One CTA owns one
-// KV group g and a tile of 128/G queries of block b (the G query heads packed as the
-// 128 UMMA rows, row = query*G + head); its keys are the entries of S_b up to the
-// tile's last query, in chunks of 64 in a four-stage ring:
-//   gather warps (6-7)  cp.async the K and V rows of the chunk (whole rows per warp
+// KV group g and TT tiles of 128/G queries of block b (TT = 2 when the block has an
+// even number of tiles; the G query heads packed as the 128 UMMA rows of a tile,
+// row = query*G + head); its keys are the entries of S_b up to its last query, in
+// chunks of 64 in a four-stage ring, gathered once for all of its tiles:
+//   gather warps        cp.async the K and V rows of the chunk (whole rows per warp
 //                       instruction, zero-filled past the support) into 128-byte-swizzled shared
 //                       tiles laid out as a TMA tile load would leave them, stage the
 //                       key indices for the mask; a chunk is signalled (fence to the async
 //                       proxy, arrive) once the copies of the two chunks after it are in
 //                       flight, so three chunks of rows travel at once;
-//   warp 4              TMA of the Q tile (once);
-//   warp 5              S = Q K^T into one of two TMEM buffers, then O += P V, S of
-//                       chunk t+1 issued before P V of chunk t;
-//   softmax warps 0-3   thread = row: mask (key not in [0, i] or past the support),
-//                       lazy online softmax in exp2 as in the dense kernel, P as bf16
-//                       into a swizzled shared tile; rows with no key get a zero output
-//                       row and lse = -inf.
+//   TMA warp            the Q tiles (once);
+//   MMA warp            per chunk, S = Q K^T of every tile into one of its two TMEM
+//                       buffers, then O += P V per tile, S of chunk t+1 issued before
+//                       P V of chunk t;
+//   softmax warpgroups  one per tile (warps 4tt..4tt+3), thread = row: mask (key not in
+//                       [0, i] or past the support), lazy online softmax in exp2 as in
+//                       the dense kernel, P as bf16 into the tile's swizzled shared
+//                       tile; rows with no key get a zero output row and lse = -inf.
+// With two tiles the softmax of one overlaps the MMAs of the other, and every gathered
+// key row serves twice the queries.
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
@@ -37,15 +41,17 @@ constexpr int kKeys = 64;                   // keys per chunk
 constexpr int kHalf = 128 * 64 * 2;         // one 128-row x 64-element swizzled half (Q, P)
 constexpr int kHalfKV = kKeys * 64 * 2;     // one 64-key x 64-element swizzled half (K, V)
 static_assert(kLag < kStages - 1, "the gather may run at most kStages - 2 chunks ahead");
-constexpr int kThreads = 256;
-constexpr int kGatherWarp0 = 6;             // warps 6..7 gather
-constexpr int kGatherThreads = kThreads - kGatherWarp0 * 32;
+constexpr int kGatherThreads = 64;          // two gather warps
 constexpr float kRescaleLog2 = 8.f;
 
-template <int D>
+// TT softmax warpgroups, then the TMA warp, the MMA warp and the two gather warps.
+__host__ __device__ constexpr int block_threads(int TT) { return 32 * (4 * TT + 4); }
+
+template <int D, int TT>
 constexpr int block_tc_smem_bytes() {
-    // slack + Q + K ring + V ring + P + staged key indices + barriers
-    return 1024 + (D / 64) * (kHalf + 2 * kStages * kHalfKV) + kHalf + kStages * kKeys * 4 + 256;
+    // slack + Q tiles + K ring + V ring + P tiles + staged key indices + barriers
+    return 1024 + (D / 64) * (TT * kHalf + 2 * kStages * kHalfKV) + TT * kHalf +
+           kStages * kKeys * 4 + 256;
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -62,7 +68,7 @@ __device__ __forceinline__ void cp_async_wait() {
 struct BlockTcParams {
     const __nv_bfloat16* k;
     const __nv_bfloat16* v;
-    int N, Hq, Hkv, tiles_per_block, n_tiles;
+    int N, Hq, Hkv, tiles_per_block, n_ctas_per_group;
     int block_q, kmax;
     float sl2;
     const int32_t* sup_idx;
@@ -73,46 +79,55 @@ struct BlockTcParams {
     uint64_t timeout_ns;
 };
 
-template <int G, int D>
-__global__ void __launch_bounds__(kThreads, 1)
-k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) {
+// DENSE: the same pipeline over every key 0..q_last (the dense comparator): the TMA
+// warp also streams the K and V chunks (tmK, tmV with 64-row boxes) and the mask is the
+// causal one; the gather warps stay idle.
+template <int G, int D, int TT, bool DENSE>
+__global__ void __launch_bounds__(block_threads(TT), 1)
+k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const BlockTcParams p) {
+    constexpr int kThreads = block_threads(TT);
+    constexpr int kTmaWarp = 4 * TT, kMmaWarp = 4 * TT + 1, kGatherWarp0 = 4 * TT + 2;
     constexpr int BQ = 128 / G;
     constexpr int NH = D / 64;
-    constexpr uint32_t kTile = NH * kHalf;        // Q
+    constexpr uint32_t kTile = NH * kHalf;        // Q of one tile
     constexpr uint32_t kTileKV = NH * kHalfKV;    // one chunk of K (or V)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint8_t* sQ = base;
-    uint8_t* sK = sQ + kTile;
+    uint8_t* sQ = base;                                 // TT tiles
+    uint8_t* sK = sQ + TT * kTile;
     uint8_t* sV = sK + kStages * kTileKV;
-    uint8_t* sP = sV + kStages * kTileKV;               // 128 rows x 64 keys
-    int32_t* sIdx = reinterpret_cast<int32_t*>(sP + kHalf);        // kStages x kKeys
+    uint8_t* sP = sV + kStages * kTileKV;               // TT tiles of 128 rows x 64 keys
+    int32_t* sIdx = reinterpret_cast<int32_t*>(sP + TT * kHalf);   // kStages x kKeys
     uint64_t* bars = reinterpret_cast<uint64_t*>(sIdx + kStages * kKeys);
     uint64_t* q_full = bars;
     uint64_t* kv_full = q_full + 1;
     uint64_t* kv_empty = kv_full + kStages;
-    uint64_t* s_full = kv_empty + kStages;
-    uint64_t* s_empty = s_full + 2;
-    uint64_t* p_full = s_empty + 2;
-    uint64_t* o_done = p_full + 1;
-    uint64_t* mma_done = o_done + 1;
+    uint64_t* s_full = kv_empty + kStages;              // [tile][buffer]
+    uint64_t* s_empty = s_full + 2 * TT;                // [tile][buffer]
+    uint64_t* p_full = s_empty + 2 * TT;                // [tile]
+    uint64_t* o_done = p_full + TT;                     // [tile]
+    uint64_t* mma_done = o_done + TT;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = (int)(blockIdx.x % p.Hkv);
-    const int tile = p.n_tiles - 1 - (int)(blockIdx.x / p.Hkv);     // later blocks first
-    const int b = tile / p.tiles_per_block;
-    const int q0 = b * p.block_q + (tile % p.tiles_per_block) * BQ;
+    // the CTA's TT consecutive tiles (within one block: tiles_per_block % TT == 0)
+    const int tile0 = (p.n_ctas_per_group - 1 - (int)(blockIdx.x / p.Hkv)) * TT;  // later first
+    const int b = tile0 / p.tiles_per_block;
+    const int q0 = b * p.block_q + (tile0 % p.tiles_per_block) * BQ;
     if (q0 >= p.N) return;                                          // uniform for the CTA
-    const int q_last = min(p.N, q0 + BQ) - 1;
+    const int q_last = min(p.N, q0 + TT * BQ) - 1;
     const int32_t* srow = p.sup_idx + (size_t)b * p.kmax;
     // n_t = 1 + the last position of the (ascending) support row holding a key <= q_last:
     // one round of independent loads across the CTA and a max-reduction, instead of a
     // chain of dependent loads; the first chunk's indices are staged on the way.
     __shared__ int s_last[kThreads / 32];
-    {
+    if (DENSE) {
+        if (threadIdx.x < kThreads / 32) s_last[threadIdx.x] = q_last + 1;
+    } else {
         const int len = min(p.sup_len[b], p.kmax);
         int last = 0;
 #pragma unroll 4
@@ -132,10 +147,10 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
     const int n_ch = (n_t + kKeys - 1) / kKeys;
 
     if (n_ch == 0) {
-        // no support key at or before any query of the tile: zero rows, lse = -inf
-        if (threadIdx.x < 128) {
-            const int r = threadIdx.x;
-            const int i = q0 + r / G, h = g * G + r % G;
+        // no support key at or before any query of the tiles: zero rows, lse = -inf
+        if (threadIdx.x < 128 * TT) {
+            const int r = threadIdx.x % 128, tt = threadIdx.x / 128;
+            const int i = q0 + tt * BQ + r / G, h = g * G + r % G;
             if (i < p.N) {
                 __nv_bfloat16* orow = p.out + ((size_t)i * p.Hq + h) * D;
                 for (int c = 0; c < D; ++c) orow[c] = __float2bfloat16_rn(0.f);
@@ -148,15 +163,17 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
     if (threadIdx.x == 0) {
         tc::mbar_init(q_full, 1);
         for (int s = 0; s < kStages; ++s) {
-            tc::mbar_init(&kv_full[s], kGatherThreads);   // every gather thread
+            tc::mbar_init(&kv_full[s], DENSE ? 1 : kGatherThreads);   // TMA, or every gather thread
             tc::mbar_init(&kv_empty[s], 1);
         }
-        for (int bb = 0; bb < 2; ++bb) {
-            tc::mbar_init(&s_full[bb], 1);
-            tc::mbar_init(&s_empty[bb], 128);
+        for (int x = 0; x < 2 * TT; ++x) {
+            tc::mbar_init(&s_full[x], 1);
+            tc::mbar_init(&s_empty[x], 128);
         }
-        tc::mbar_init(p_full, 128);
-        tc::mbar_init(o_done, 1);
+        for (int tt = 0; tt < TT; ++tt) {
+            tc::mbar_init(&p_full[tt], 128);
+            tc::mbar_init(&o_done[tt], 1);
+        }
         tc::mbar_init(mma_done, 1);
         *abort_flag = 0;
         tc::fence_barrier_init();
@@ -169,10 +186,11 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_o = tmem + 256;           // O accumulator: columns 256..256+D
-    const tc::Guard gd{abort_flag, p.status, KID_BLOCK_ATTN, p.timeout_ns};
+    // tile tt: S buffers at columns 128 tt + {0, 64}, O accumulator at 256 + 128 tt
+    const tc::Guard gd{abort_flag, p.status, DENSE ? KID_DENSE_TC : KID_BLOCK_ATTN, p.timeout_ns};
 
     if (warp >= kGatherWarp0) {
+      if constexpr (!DENSE) {
         // ---------------------------------------------------------------- gather
         // Warp gw copies key rows [64 gw, 64 gw + 64) of each chunk.  Lane l owns the
         // indices of rows 64 gw + l and 64 gw + 32 + l; the copies go row-contiguous:
@@ -239,18 +257,44 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
             if (*abort_flag) break;
             tc::mbar_arrive(&kv_full[t % kStages]);
         }
-    } else if (warp == 4) {
+      }
+    } else if (warp == kTmaWarp) {
         // ---------------------------------------------------------------- Q (TMA)
         if (lane == 0) {
             tc::prefetch_tmap(&tmQ);
-            tc::mbar_arrive_expect_tx(q_full, kTile);
-            for (int h = 0; h < NH; ++h)
-                tc::tma_load_3d(sQ + h * kHalf, &tmQ, q_full, h * 64, g * G, q0);
+            tc::mbar_arrive_expect_tx(q_full, TT * kTile);
+            for (int tt = 0; tt < TT; ++tt)
+                for (int h = 0; h < NH; ++h)
+                    tc::tma_load_3d(sQ + tt * kTile + h * kHalf, &tmQ, q_full, h * 64, g * G,
+                                    q0 + tt * BQ);
+            if (DENSE) {
+                // K and V chunks of keys 64 t .. 64 t + 63 (past N the box reads zeros,
+                // and the causal mask drops those keys)
+                tc::prefetch_tmap(&tmK);
+                tc::prefetch_tmap(&tmV);
+                int issued = 0;
+                for (int t = 0; t < n_ch; ++t) {
+                    const int s = t % kStages;
+                    if (!tc::wait(&kv_empty[s], ((t / kStages) & 1) ^ 1, gd, 1)) break;
+                    tc::mbar_arrive_expect_tx(&kv_full[s], 2 * kTileKV);
+                    for (int h = 0; h < NH; ++h) {
+                        tc::tma_load_3d(sK + s * kTileKV + h * kHalfKV, &tmK, &kv_full[s], h * 64, g,
+                                        t * kKeys);
+                        tc::tma_load_3d(sV + s * kTileKV + h * kHalfKV, &tmV, &kv_full[s], h * 64, g,
+                                        t * kKeys);
+                    }
+                    issued = t + 1;
+                }
+                int zero0 = 0;
+                const tc::Guard drain0{&zero0, nullptr, 0, p.timeout_ns};
+                for (int t = max(0, issued - kStages); t < issued; ++t)
+                    tc::wait(&kv_full[t % kStages], (t / kStages) & 1, drain0, 0);
+            }
             int zero = 0;
             const tc::Guard drain{&zero, nullptr, 0, p.timeout_ns};
             tc::wait(q_full, 0, drain, 0);
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kKeys);
@@ -261,34 +305,42 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
             auto issue_s = [&](int t) -> bool {
                 const int s = t % kStages, bb = t & 1;
                 if (!tc::wait(&kv_full[s], (t / kStages) & 1, gd, 4)) return false;
-                if (!tc::wait(&s_empty[bb], ((t >> 1) & 1) ^ 1, gd, 5)) return false;
+                for (int tt = 0; tt < TT; ++tt)
+                    if (!tc::wait(&s_empty[tt * 2 + bb], ((t >> 1) & 1) ^ 1, gd, 5)) return false;
                 tc::fence_after_sync();
                 const uint32_t ak = tc::smem_u32(sK + s * kTileKV);
 #pragma unroll
-                for (int kk = 0; kk < NH * 4; ++kk) {
-                    const uint32_t offq = (kk >> 2) * kHalf + (kk & 3) * 32;
-                    const uint32_t offk = (kk >> 2) * kHalfKV + (kk & 3) * 32;
-                    tc::mma_bf16_ss(tmem + bb * kKeys, tc::desc_kmajor_sw128(aq + offq),
-                                    tc::desc_kmajor_sw128(ak + offk), idesc_s, kk > 0 ? 1u : 0u);
+                for (int tt = 0; tt < TT; ++tt) {
+#pragma unroll
+                    for (int kk = 0; kk < NH * 4; ++kk) {
+                        const uint32_t offq = tt * kTile + (kk >> 2) * kHalf + (kk & 3) * 32;
+                        const uint32_t offk = (kk >> 2) * kHalfKV + (kk & 3) * 32;
+                        tc::mma_bf16_ss(tmem + tt * 128 + bb * kKeys, tc::desc_kmajor_sw128(aq + offq),
+                                        tc::desc_kmajor_sw128(ak + offk), idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    tc::mma_commit(&s_full[tt * 2 + bb]);
                 }
-                tc::mma_commit(&s_full[bb]);
                 return true;
             };
             if (ok) ok = issue_s(0);
             for (int t = 0; ok && t < n_ch; ++t) {
                 if (t + 1 < n_ch && !issue_s(t + 1)) break;
                 const int s = t % kStages;
-                if (!tc::wait(p_full, t & 1, gd, 7)) break;
-                tc::fence_after_sync();
                 const uint32_t av = tc::smem_u32(sV + s * kTileKV);
+                for (int tt = 0; ok && tt < TT; ++tt) {
+                    if (!tc::wait(&p_full[tt], t & 1, gd, 7)) { ok = false; break; }
+                    tc::fence_after_sync();
 #pragma unroll
-                for (int kk = 0; kk < kKeys / 16; ++kk) {   // the chunk's keys in steps of 16
-                    tc::mma_bf16_ss(tmem_o, tc::desc_kmajor_sw128(ap + kk * 32),
-                                    tc::desc_mnmajor_sw128(av + kk * 16 * 128, kHalfKV), idesc_o,
-                                    (t > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kKeys / 16; ++kk) {   // the chunk's keys in steps of 16
+                        tc::mma_bf16_ss(tmem + 256 + tt * 128,
+                                        tc::desc_kmajor_sw128(ap + tt * kHalf + kk * 32),
+                                        tc::desc_mnmajor_sw128(av + kk * 16 * 128, kHalfKV), idesc_o,
+                                        (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(&o_done[tt]);
                 }
+                if (!ok) break;
                 tc::mma_commit(&kv_empty[s]);
-                tc::mma_commit(o_done);
             }
             tc::mma_commit(mma_done);
             int zero = 0;
@@ -297,38 +349,55 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
         }
     } else {
         // ---------------------------------------------------------------- softmax
-        const int r = threadIdx.x;
-        const int i = q0 + r / G;
+        const int tt = warp >> 2;                    // this warpgroup's tile
+        const int r = threadIdx.x & 127;
+        const int i = q0 + tt * BQ + r / G;
         const int h = g * G + r % G;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tmem_s = tmem + tt * 128;     // the tile's two S buffers
+        const uint32_t tmem_o = tmem + 256 + tt * 128;
+        uint64_t* my_s_full = s_full + tt * 2;
+        uint64_t* my_s_empty = s_empty + tt * 2;
+        uint64_t* my_p_full = p_full + tt;
+        uint64_t* my_o_done = o_done + tt;
         const float sl2 = p.sl2;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        uint8_t* prow0 = sP + r * 128;               // row r of the P tile
+        uint8_t* prow0 = sP + tt * kHalf + r * 128;  // row r of the tile's P
         for (int t = 0; ok && t < n_ch; ++t) {
             const int bb = t & 1, s = t % kStages;
-            if (!tc::wait(&s_full[bb], (t >> 1) & 1, gd, 8)) { ok = false; break; }
+            if (!tc::wait(&my_s_full[bb], (t >> 1) & 1, gd, 8)) { ok = false; break; }
             tc::fence_after_sync();
             constexpr int NC = kKeys / 32;            // 32-column loads of a chunk
             uint32_t v[NC][32];
 #pragma unroll
-            for (int c = 0; c < NC; ++c) tc::tmem_ld32(tmem + lane_off + bb * kKeys + c * 32, v[c]);
+            for (int c = 0; c < NC; ++c) tc::tmem_ld32(tmem_s + lane_off + bb * kKeys + c * 32, v[c]);
 #pragma unroll
             for (int c = 0; c < NC; ++c) tc::tmem_wait_ld(v[c]);
             tc::fence_before_sync();
-            tc::mbar_arrive(&s_empty[bb]);
+            tc::mbar_arrive(&my_s_empty[bb]);
             // mask: keys past the support (index -1) or after query i
-            const int4* ix4 = reinterpret_cast<const int4*>(sIdx + s * kKeys);
+            if (DENSE) {
+                if ((t + 1) * kKeys - 1 > i) {           // only the chunks that reach past i
 #pragma unroll
-            for (int c = 0; c < NC; ++c)
+                    for (int c = 0; c < NC; ++c)
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const int4 jj = ix4[c * 8 + e4];
-                    const int js[4] = {jj.x, jj.y, jj.z, jj.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        if (js[e] < 0 || js[e] > i) v[c][e4 * 4 + e] = __float_as_uint(-INFINITY);
+                        for (int e = 0; e < 32; ++e)
+                            if (t * kKeys + c * 32 + e > i) v[c][e] = __float_as_uint(-INFINITY);
                 }
+            } else {
+                const int4* ix4 = reinterpret_cast<const int4*>(sIdx + s * kKeys);
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const int4 jj = ix4[c * 8 + e4];
+                        const int js[4] = {jj.x, jj.y, jj.z, jj.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (js[e] < 0 || js[e] > i) v[c][e4 * 4 + e] = __float_as_uint(-INFINITY);
+                    }
+            }
             float tm[2] = {-INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < NC; ++c)
@@ -372,7 +441,7 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
                 // P V of chunk t-1 must have finished reading the P tile before it is
                 // overwritten; wait once, before the first store
                 if (c8 == 0 && t > 0) {
-                    if (!tc::wait(o_done, (t - 1) & 1, gd, 9)) { ok = false; break; }
+                    if (!tc::wait(my_o_done, (t - 1) & 1, gd, 9)) { ok = false; break; }
                 }
                 uint4* dst = reinterpret_cast<uint4*>(prow0 + ((c8 ^ (r & 7)) << 4));
                 *dst = make_uint4(w[0], w[1], w[2], w[3]);
@@ -400,10 +469,10 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
             m_used = m_new;
             tc::fence_proxy_async_smem();
             tc::fence_before_sync();
-            tc::mbar_arrive(p_full);
+            tc::mbar_arrive(my_p_full);
         }
         // epilogue: wait for the last P V, normalise, store bf16 rows
-        if (ok && tc::wait(o_done, (n_ch - 1) & 1, gd, 10)) {
+        if (ok && tc::wait(my_o_done, (n_ch - 1) & 1, gd, 10)) {
             tc::fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16* orow = p.out + ((size_t)i * p.Hq + h) * D;
@@ -437,24 +506,40 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const BlockTcParams p) 
     }
 }
 
-template <int G, int D>
+template <int G, int D, int TT, bool DENSE>
 cudaError_t launch_block_tc(const AttnArgs& a, cudaStream_t st) {
     constexpr int BQ = 128 / G;
-    CUtensorMap tq;
+    CUtensorMap tq, tk, tv;
     const uint64_t d = a.d;
     if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQ))
         return cudaErrorInvalidValue;
+    if (DENSE) {
+        if (!make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, a.N, d * 2, (uint64_t)a.Hkv * d * 2, 64, 1, kKeys) ||
+            !make_tmap_3d_bf16(&tv, a.v, d, a.Hkv, a.N, d * 2, (uint64_t)a.Hkv * d * 2, 64, 1, kKeys))
+            return cudaErrorInvalidValue;
+    } else {
+        tk = tq;                                // unused by the gathering form
+        tv = tq;
+    }
     BlockTcParams p{};
     p.k = (const __nv_bfloat16*)a.k;
     p.v = (const __nv_bfloat16*)a.v;
     p.N = (int)a.N;
     p.Hq = a.Hq;
     p.Hkv = a.Hkv;
-    p.block_q = a.block_q;
-    p.kmax = a.kmax;
-    p.tiles_per_block = a.block_q / BQ;
-    const int nb = (int)((a.N + a.block_q - 1) / a.block_q);
-    p.n_tiles = nb * p.tiles_per_block;
+    if (DENSE) {
+        // one "block" per CTA: TT query tiles, keys 0 .. the last of their queries
+        p.block_q = TT * BQ;
+        p.kmax = 0;
+        p.tiles_per_block = TT;
+        p.n_ctas_per_group = (int)((a.N + TT * BQ - 1) / (TT * BQ));
+    } else {
+        p.block_q = a.block_q;
+        p.kmax = a.kmax;
+        p.tiles_per_block = a.block_q / BQ;
+        const int nb = (int)((a.N + a.block_q - 1) / a.block_q);
+        p.n_ctas_per_group = nb * p.tiles_per_block / TT;
+    }
     p.sl2 = a.sl2;
     p.sup_idx = a.sup_idx;
     p.sup_len = a.sup_len;
@@ -462,23 +547,32 @@ cudaError_t launch_block_tc(const AttnArgs& a, cudaStream_t st) {
     p.lse = a.lse;
     p.status = a.status;
     p.timeout_ns = wait_timeout_ns();
-    constexpr int smem = block_tc_smem_bytes<D>();
-    auto kern = k_attn_block_tc<G, D>;
+    constexpr int smem = block_tc_smem_bytes<D, TT>();
+    static_assert(smem <= 227 * 1024, "block pass 3 shared memory");
+    auto kern = k_attn_block_tc<G, D, TT, DENSE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(p.n_tiles * a.Hkv), kThreads, smem, st>>>(tq, p);
+    kern<<<(unsigned)(p.n_ctas_per_group * a.Hkv), block_threads(TT), smem, st>>>(tq, tk, tv, p);
     note_launch();
     return cudaGetLastError();
 }
 
-template <int D>
+// Two tiles per CTA when the block has an even number of tiles, else one (dense: two).
+template <int G, int D, bool DENSE>
+cudaError_t launch_tt(const AttnArgs& a, cudaStream_t st) {
+    if (DENSE) return launch_block_tc<G, D, 2, true>(a, st);
+    return (a.block_q / (128 / G)) % 2 == 0 ? launch_block_tc<G, D, 2, false>(a, st)
+                                             : launch_block_tc<G, D, 1, false>(a, st);
+}
+
+template <int D, bool DENSE>
 cudaError_t dispatch_g(const AttnArgs& a, cudaStream_t st) {
     switch (a.Hq / a.Hkv) {
-        case 1: return launch_block_tc<1, D>(a, st);
-        case 2: return launch_block_tc<2, D>(a, st);
-        case 4: return launch_block_tc<4, D>(a, st);
-        case 8: return launch_block_tc<8, D>(a, st);
-        case 16: return launch_block_tc<16, D>(a, st);
+        case 1: return launch_tt<1, D, DENSE>(a, st);
+        case 2: return launch_tt<2, D, DENSE>(a, st);
+        case 4: return launch_tt<4, D, DENSE>(a, st);
+        case 8: return launch_tt<8, D, DENSE>(a, st);
+        case 16: return launch_tt<16, D, DENSE>(a, st);
         default: return cudaErrorNotSupported;
     }
 }
@@ -493,7 +587,17 @@ bool block_tc_supported(const AttnArgs& a) {
 }
 
 cudaError_t block_attention_tc(const AttnArgs& a, cudaStream_t st) {
-    return a.d == 64 ? dispatch_g<64>(a, st) : dispatch_g<128>(a, st);
+    return a.d == 64 ? dispatch_g<64, false>(a, st) : dispatch_g<128, false>(a, st);
+}
+
+bool dense_pair_tiles_supported(const AttnArgs& a) {
+    const int G = a.Hq / a.Hkv;
+    if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128)) return false;
+    return G == 1 || G == 2 || G == 4 || G == 8 || G == 16;
+}
+
+cudaError_t dense_pair_tiles(const AttnArgs& a, cudaStream_t st) {
+    return a.d == 64 ? dispatch_g<64, true>(a, st) : dispatch_g<128, true>(a, st);
 }
 
 }  // namespace tam

@@ -156,6 +156,10 @@ bool gather_supported(const AttnArgs& a);
 cudaError_t gather_attention(const AttnArgs& a, cudaStream_t st);
 bool block_tc_supported(const AttnArgs& a);
 cudaError_t block_attention_tc(const AttnArgs& a, cudaStream_t st);
+// Dense causal attention on the block kernel's two-tile pipeline (TMA K/V chunks of 64
+// keys, two query tiles per CTA); used with TAM_DENSE_PAIR_TILES=1.
+bool dense_pair_tiles_supported(const AttnArgs& a);
+cudaError_t dense_pair_tiles(const AttnArgs& a, cudaStream_t st);
 
 // CUDA-core kernels (any dtype, any supported shape).
 cudaError_t simt_lse(const LseArgs& a, cudaStream_t st);

@@ -37,8 +37,6 @@
 //               order); block-shared mass goes to the fixed-point block sums.
 // Every wait is bounded; the pair shakes hands before it frees TMEM and exits so
 // that no remote arrive or MMA of one CTA can land after the other left.
-#include <cstdlib>
-
 #include "launch.h"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
@@ -47,7 +45,9 @@ namespace tam {
 namespace {
 
 constexpr int kModeRows = 0, kModeBlock = 1, kModeStream = 2;
-constexpr int kMaxStages = 6;           // K ring: as many full key tiles as fit, 2..6
+// K ring of two key tiles (deeper rings, up to four tiles where Q leaves room, measured
+// no faster: the pipeline is not waiting on K)
+constexpr int kStages = 2;
 // Mass warps: 8 per query (two per TMEM lane quarter), 16 block-shared (four per
 // quarter; measured 5 % faster there, no gain per query).  Then the TMA producer and
 // the MMA issuer.
@@ -59,18 +59,9 @@ constexpr int kR = 512 / kNQ;           // TMEM accumulator slots
 constexpr int kTileKeys = 256;          // keys per pair tile (128 per CTA)
 
 constexpr int kMaxDynSmem = 227 * 1024;
-// alignment slack + Q half + lse of all 128 columns + thresholds + barriers
-__host__ __device__ constexpr int pair_fixed_bytes(int D, int Hkv) {
-    return 1024 + Hkv * kHalfRows * D * 2 + Hkv * kNQ * 4 + 128 + 512;
-}
-// Key tiles (128 keys x D per CTA) in the K ring: what fits next to Q, at most kMaxStages
-// (0 if fewer than two fit).
-__host__ __device__ constexpr int pair_stages(int D, int Hkv) {
-    return (kMaxDynSmem - pair_fixed_bytes(D, Hkv)) / (128 * D * 2) >= kMaxStages
-               ? kMaxStages
-               : ((kMaxDynSmem - pair_fixed_bytes(D, Hkv)) / (128 * D * 2) >= 2
-                      ? (kMaxDynSmem - pair_fixed_bytes(D, Hkv)) / (128 * D * 2)
-                      : 0);
+__host__ __device__ constexpr int pair_smem_bytes(int D, int Hkv) {
+    // alignment slack + Q half + K ring + lse of all 128 columns + thresholds + barriers
+    return 1024 + Hkv * kHalfRows * D * 2 + kStages * 128 * D * 2 + Hkv * kNQ * 4 + 128 + 512;
 }
 
 struct PairParams {
@@ -78,7 +69,6 @@ struct PairParams {
     int64_t row0, row1;       // per query: the rows [row0, row1) of this launch
     int kst;                  // rows mode: key m of the K map sits at position m * kst
     int seg_cap;              // stream mode: entries per candidate segment
-    int stages;               // key tiles in the K ring
     float sl2, inv_hq;
     const float* lse;
     float* rows;
@@ -116,7 +106,6 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     constexpr uint32_t kKHalf = 128 * 128;
     constexpr uint32_t kKTile = NH * kKHalf;
     const int Hkv = p.Hkv;
-    const int kStages = p.stages;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -128,8 +117,8 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     uint64_t* bars = reinterpret_cast<uint64_t*>(sTau + 32);
     uint64_t* q_full = bars;                 // CTA 0's counts both CTAs' Q bytes
     uint64_t* k_full = q_full + 1;           // CTA 0's counts both CTAs' K bytes
-    uint64_t* k_empty = k_full + kMaxStages; // both (pair commits)
-    uint64_t* s_full = k_empty + kMaxStages; // both (pair commits)
+    uint64_t* k_empty = k_full + kStages;    // both (pair commits)
+    uint64_t* s_full = k_empty + kStages;    // both (pair commits)
     uint64_t* s_empty = s_full + kR;         // CTA 0's: both CTAs' mass threads
     uint64_t* mma_done = s_empty + kR;       // both (pair commit)
     uint64_t* exit_bar = mma_done + 1;       // each: the peer's arrival at the end
@@ -259,8 +248,14 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(part * kCols);
         const uint32_t s_empty_leader = tc::map_to_cta(tc::smem_u32(s_empty), 0);
-        // stream mode: this warp's segment of every row and its running counts
+        // stream mode: this warp's segment of every row and its running counts; the
+        // candidates of (query qbase + ql, this segment) start at entry off0 + ql * qstride
+        // (32-bit: the host keeps a chunk's candidate buffer below 2^32 entries)
         const int seg = (int)rank * 4 + quarter;
+        const int qbase = q0 + part * kQP;
+        const uint32_t qstride = 8u * (uint32_t)p.seg_cap;
+        const uint32_t off0 = (uint32_t)(qbase - (int)p.row0) * qstride + (uint32_t)(seg * p.seg_cap);
+        const int qend = STREAM ? min(kQP, (int)(p.row1 - qbase)) : 0;   // queries in the launch
         int cnt[STREAM ? kQP : 1];
 #pragma unroll
         for (int q = 0; q < (STREAM ? kQP : 1); ++q) cnt[q] = 0;
@@ -310,30 +305,35 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             if (!ok) break;
             const int m = kt * kTileKeys + (int)rank * 128 + row;   // key (or sample) index
             if constexpr (MODE == kModeRows) {
-                // row i of the slab starts off(i) - off(row0) floats in; lanes store
-                // consecutive keys of one query
-                const int64_t j = (int64_t)m * p.kst;
+                // row i of the slab starts off(i) - off(row0) floats in (32-bit: the host
+                // keeps a chunk's slab below 2^32 floats) and holds i / S + 1 values; the
+                // offsets of this part's rows follow from the first one by adding
+                // i / S + 1, so no division runs per key tile.  Lanes store consecutive
+                // keys of one query; key m sits at position m S <= i iff m <= i / S.
+                int a = qbase / p.kst, b = qbase - a * p.kst;   // first row's i / S, i % S
+                uint32_t off = (uint32_t)(qbase + (int64_t)p.kst * ((int64_t)a * (a - 1) / 2) +
+                                          (int64_t)a * b - slab0);
 #pragma unroll
                 for (int ql = 0; ql < kQP; ++ql) {
-                    const int64_t i = q0 + part * kQP + ql;
-                    if (j <= i && i >= p.row0 && i < p.row1)
-                        p.rows[sample_offset(i, p.kst) - slab0 + m] = acc[ql] * p.inv_hq;
+                    if (m <= a && qbase + ql < p.row1) p.rows[off + (uint32_t)m] = acc[ql] * p.inv_hq;
+                    off += (uint32_t)a + 1u;
+                    if (++b == p.kst) { b = 0; ++a; }
                 }
             } else if constexpr (STREAM) {
                 // keys at or above the query's threshold, appended in key order to this
-                // warp's segment (positions past the capacity are only counted)
+                // warp's segment (positions past the capacity are only counted); no
+                // warp-uniform branch, so the queries' ballot chains interleave
                 const uint32_t lt = lanemask_lt();
+                const bool below = m <= qbase;        // key at or before every query here
 #pragma unroll
                 for (int ql = 0; ql < kQP; ++ql) {
-                    const int qi = part * kQP + ql;
-                    const int64_t i = q0 + qi;
                     const float v = acc[ql] * p.inv_hq;
-                    const bool pass = m <= i && i < p.row1 && v >= sTau[qi];
-                    // no warp-uniform branch: the queries' ballot chains interleave
+                    const bool pass = ql < qend && (below || m <= qbase + ql) &&
+                                      v >= sTau[part * kQP + ql];
                     const uint32_t bal = __ballot_sync(0xffffffffu, pass);
                     const int pos = cnt[ql] + __popc(bal & lt);
                     if (pass && pos < p.seg_cap)
-                        p.cand[((i - p.row0) * 8 + seg) * (int64_t)p.seg_cap + pos] =
+                        p.cand[off0 + (uint32_t)ql * qstride + (uint32_t)pos] =
                             make_uint2(__float_as_uint(v), (uint32_t)m);
                     cnt[ql] += __popc(bal);
                 }
@@ -413,12 +413,6 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     p.row1 = r1;
     p.kst = S;
     p.seg_cap = a.seg_cap;
-    p.stages = pair_stages(D, a.Hkv);
-    {   // TAM_PAIR_STAGES=n caps the ring (A/B comparisons)
-        const char* env = std::getenv("TAM_PAIR_STAGES");
-        const int cap = env ? std::atoi(env) : 0;
-        if (cap >= 2 && cap < p.stages) p.stages = cap;
-    }
     p.block_q = a.block_q;
     p.sl2 = a.sl2;
     p.inv_hq = 1.f / (float)a.Hq;
@@ -432,7 +426,7 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     p.timeout_ns = wait_timeout_ns();
     p.dbg = debug_flags();
     if (p.n_pairs <= 0) return cudaSuccess;
-    const int smem = pair_fixed_bytes(D, a.Hkv) + p.stages * 128 * D * 2;
+    const int smem = pair_smem_bytes(D, a.Hkv);
     auto kern = k_mass_pair<G, D, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -469,7 +463,7 @@ bool pair_mass_supported(const MassArgs& a) {
     if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128)) return false;
     if (G != 4 && G != 8 && G != 16) return false;
     if (a.block_q > 1 && a.block_q > (1 << 20)) return false;
-    return pair_stages(a.d, a.Hkv) > 0;
+    return pair_smem_bytes(a.d, a.Hkv) <= kMaxDynSmem;
 }
 
 // Launches the pair kernel only: per query it fills the slab rows [row0, row1) (rows

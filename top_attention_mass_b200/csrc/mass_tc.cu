@@ -230,7 +230,13 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         const uint32_t lane_addr =
             tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(part * kCols);
         // stream modes: the quarter-q warps write segment q of their queries' rows, with
-        // running counts
+        // running counts; the candidates of (query qbase + q, segment) start at entry
+        // off0 + q * qstride (32-bit: the host keeps a chunk below 2^32 entries)
+        const int qbase = q0 + part * kQP;
+        const uint32_t qstride = 4u * (uint32_t)p.seg_cap;
+        const uint32_t off0 =
+            (uint32_t)(qbase - (int)p.row0) * qstride + (uint32_t)(quarter * p.seg_cap);
+        const int qend = STREAM ? min(kQP, (int)(p.row1 - qbase)) : 0;
         int cnt[STREAM ? kQP : 1];
 #pragma unroll
         for (int q = 0; q < (STREAM ? kQP : 1); ++q) cnt[q] = 0;
@@ -290,32 +296,38 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             const int qp0 = q0 + part * kQP;                  // first query of this part
             if constexpr (STREAM) {
                 // keys at or above the query's threshold, appended in key order to this
-                // warp's segment (positions past the capacity are only counted)
+                // warp's segment (positions past the capacity are only counted); no
+                // warp-uniform branch, so the queries' ballot chains interleave
                 uint32_t lt;
                 asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt));
+                const bool below = j <= qbase;        // key at or before every query here
 #pragma unroll
                 for (int q = 0; q < kQP; ++q) {
-                    const int64_t i = qp0 + q;
                     const float v = INDEXER ? acc[q] : acc[q] * p.inv_hq;
-                    const bool pass = j <= i && i < p.row1 && v >= sTau[part * kQP + q];
-                    // no warp-uniform branch: the queries' ballot chains interleave
+                    const bool pass = q < qend && (below || j <= qbase + q) &&
+                                      v >= sTau[part * kQP + q];
                     const uint32_t bal = __ballot_sync(0xffffffffu, pass);
                     const int pos = cnt[q] + __popc(bal & lt);
                     if (pass && pos < p.seg_cap)
-                        p.cand[((i - p.row0) * 4 + quarter) * (int64_t)p.seg_cap + pos] =
+                        p.cand[off0 + (uint32_t)q * qstride + (uint32_t)pos] =
                             make_uint2(__float_as_uint(v), (uint32_t)j);
                     cnt[q] += __popc(bal);
                 }
             } else if constexpr (!BLOCK) {
-                // row i of the slab starts off(i) - off(row0) floats in; lanes store
-                // consecutive keys of one query
-                const int64_t jp = (int64_t)j * p.kst;        // key position
+                // row i of the slab starts off(i) - off(row0) floats in (32-bit: the host
+                // keeps a chunk's slab below 2^32 floats) and holds i / S + 1 values; the
+                // offsets of this part's rows follow from the first one by adding
+                // i / S + 1, so no division runs per key tile.  Lanes store consecutive
+                // keys of one query; key j sits at position j S <= i iff j <= i / S.
+                int a = qbase / p.kst, b = qbase - a * p.kst;   // first row's i / S, i % S
+                uint32_t off = (uint32_t)(qbase + (int64_t)p.kst * ((int64_t)a * (a - 1) / 2) +
+                                          (int64_t)a * b - slab0);
 #pragma unroll
                 for (int q = 0; q < kQP; ++q) {
-                    const int64_t i = qp0 + q;
-                    if (jp <= i && i >= p.row0 && i < p.row1)
-                        p.rows[sample_offset(i, p.kst) - slab0 + j] =
-                            INDEXER ? acc[q] : acc[q] * p.inv_hq;
+                    if (j <= a && qbase + q < p.row1)
+                        p.rows[off + (uint32_t)j] = INDEXER ? acc[q] : acc[q] * p.inv_hq;
+                    off += (uint32_t)a + 1u;
+                    if (++b == p.kst) { b = 0; ++a; }
                 }
             } else {
                 // block column sums of this part's queries, 2^-40 fixed point, one add

@@ -545,7 +545,7 @@ __global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams 
     extern __shared__ __align__(16) uint8_t smem_raw[];
     RowSmem& s = *reinterpret_cast<RowSmem*>(smem_raw);
     __shared__ int soff[kMaxSegments + 1];
-    __shared__ int sflag, s_ceq, s_cut;
+    __shared__ int sflag, s_ceq, s_cut, s_badidx;
     const int64_t i = p.row0 + (p.n_rows - 1 - (int)blockIdx.x);
     const int n = (int)i + 1;
     const int k = min(p.budget, n);
@@ -560,6 +560,7 @@ __global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams 
         s.scal[3] = -1;
         s_ceq = 0;
         s_cut = 0x7fffffff;
+        s_badidx = 0;
         const int32_t* c = p.cnt + (i - p.row0) * p.nseg;
         int tot = 0;
         bool bad = false;
@@ -589,6 +590,9 @@ __global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams 
         while (g + 1 < p.nseg && soff[g + 1] <= t) ++g;
         const uint2 e = base[g * p.seg_cap + (t - soff[g])];
         const uint32_t kv = okey(__uint_as_float(e.x));
+        // a key outside [0, i] can only come from a scan that did not finish (a wait
+        // that gave up): the row is left to the fallback and never indexes the bitmap
+        if (e.y > (uint32_t)i) s_badidx = 1;
         s.ckey[t] = kv;
         s.cidx[t] = (int32_t)e.y;
         mx = max(mx, kv);
@@ -602,6 +606,13 @@ __global__ void __launch_bounds__(kRtThreads) k_cand_select(const CandSelParams 
         atomicMin(reinterpret_cast<unsigned int*>(&s.scal[3]), mn);
     }
     __syncthreads();
+    if (s_badidx) {
+        if (threadIdx.x == 0) {
+            const int t = atomicAdd(p.fb, 1);
+            p.fb[1 + t] = (int32_t)i;
+        }
+        return;
+    }
     uint32_t T = 0u;
     int take_eq = 0;
     if (tot > k) cand_kth(s, tot, k, (uint32_t)s.scal[3], T, take_eq);  // else keep them all

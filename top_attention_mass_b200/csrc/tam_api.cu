@@ -175,7 +175,8 @@ cudaError_t run_stream_select(const StreamPlan& sp, char* ws, size_t region_byte
     if ((e = sample_tau(nullptr, 0, r_start, sp.S, budget, sp.cap, kTauSigmas, force, tau, st)))
         return e;
     const int S = sp.S;
-    const int64_t slab_cap = (int64_t)(region_bytes / 4);
+    // slab offsets within a chunk are 32-bit in the scoring kernels
+    const int64_t slab_cap = std::min<int64_t>((int64_t)(region_bytes / 4), (int64_t(1) << 32) - 1);
     for (int64_t r0 = r_start; r0 < N;) {
         const int64_t r1 = chunk_end_by(r0, N, slab_cap, [S](int64_t i) { return sample_offset(i, S); });
         if ((e = sample(r0, r1, S, (float*)region))) return e;
@@ -184,8 +185,10 @@ cudaError_t run_stream_select(const StreamPlan& sp, char* ws, size_t region_byte
             return e;
         r0 = r1;
     }
-    const int64_t rows_per_chunk =
-        std::max<int64_t>(kChunkRows, (int64_t)(region_bytes / ((size_t)sp.cap * 8)) / kChunkRows * kChunkRows);
+    // candidate offsets within a chunk are 32-bit in the scan kernels
+    const int64_t fit = std::min<int64_t>((int64_t)(region_bytes / ((size_t)sp.cap * 8)),
+                                          (int64_t(1) << 32) / sp.cap - kChunkRows);
+    const int64_t rows_per_chunk = std::max<int64_t>(kChunkRows, fit / kChunkRows * kChunkRows);
     for (int64_t c0 = 0; c0 < N; c0 += rows_per_chunk) {
         const int64_t c1 = std::min(N, c0 + rows_per_chunk);
         if ((e = scan(c0, c1, tau, (void*)region, cnt))) return e;
@@ -274,6 +277,15 @@ cudaError_t run_sparse_attention(const AttnArgs& a, cudaStream_t st) {
     return gather_supported(a) ? gather_attention(a, st) : simt_attention(a, st);
 }
 
+// Dense causal attention: the single-tile tensor-core kernel (128-key tiles), or with
+// TAM_DENSE_PAIR_TILES=1 the block-shared pass-3 pipeline over all keys (two query
+// tiles per CTA, 64-key chunks; measured 10 % slower at 32K, kept for A/B comparisons),
+// or the CUDA cores for other shapes.
+cudaError_t run_dense(const AttnArgs& a, cudaStream_t st) {
+    if (dense_pair_tiles_supported(a) && dense_pair_tiles_selected()) return dense_pair_tiles(a, st);
+    return tc_dense_supported(a) ? tc_dense(a, st) : simt_attention(a, st);
+}
+
 // Pass 1 on the tensor cores where the shape is built, else on the CUDA cores.
 cudaError_t run_lse(const LseArgs& a, cudaStream_t st) {
     return tc_lse_supported(a) ? tc_lse(a, st) : simt_lse(a, st);
@@ -307,7 +319,8 @@ int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void*
     const size_t region_bytes = ws_bytes - sp.off_region;
     if (sp.materialise) {
         // mass rows of a chunk of queries, then their top-k, chunk by chunk
-        const int64_t cap = (int64_t)(region_bytes / sizeof(float));
+        const int64_t cap = std::min<int64_t>((int64_t)(region_bytes / sizeof(float)),
+                                              (int64_t(1) << 32) - 1);   // 32-bit row offsets
         ma.rows = (float*)region;
         for (int64_t r0 = 0; r0 < N;) {
             const int64_t r1 = chunk_end(r0, N, cap);
@@ -447,7 +460,8 @@ int run_indexer(int64_t N, int d_idx, int dtype, const void* q_idx, const void* 
     const size_t region_bytes = ws_bytes - sp.off_region;
     if (sp.materialise) {
         // score rows of a chunk of queries, then their top-k, chunk by chunk
-        const int64_t cap = (int64_t)(region_bytes / sizeof(float));
+        const int64_t cap = std::min<int64_t>((int64_t)(region_bytes / sizeof(float)),
+                                              (int64_t(1) << 32) - 1);   // 32-bit row offsets
         ia.rows = (float*)region;
         for (int64_t r0 = 0; r0 < N;) {
             const int64_t r1 = chunk_end(r0, N, cap);
@@ -765,7 +779,8 @@ int tam_distill_kl(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, 
     IndexerArgs ia{};
     ia.N = N; ia.d_idx = d_idx; ia.dtype = dtype; ia.q_idx = q_idx; ia.k_idx = k_idx;
     ia.budget = 1; ia.rows = score_rows; ia.status = (int32_t*)ws;
-    const int64_t cap = (int64_t)(half / sizeof(float));
+    const int64_t cap = std::min<int64_t>((int64_t)(half / sizeof(float)),
+                                          (int64_t(1) << 32) - 1);       // 32-bit row offsets
     for (int64_t r0 = 0; r0 < N;) {
         const int64_t r1 = chunk_end(r0, N, cap);
         ma.row0 = ia.row0 = r0;
@@ -871,7 +886,7 @@ int tam_dense_gqa_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const vo
     if ((rc = start_call(workspace, st))) return rc;
     AttnArgs aa{N, Hq, Hkv, d, dtype, q, k, v, score_log2_scale(d), nullptr, nullptr, 0, 1,
                 out, lse, (int32_t*)workspace};
-    return cuda_status(tc_dense_supported(aa) ? tc_dense(aa, st) : simt_attention(aa, st));
+    return cuda_status(run_dense(aa, st));
 }
 
 int tam_dense_gqa_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv, int d,
@@ -897,7 +912,7 @@ int tam_dense_gqa_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, i
                     (const char*)v + t0 * krow, score_log2_scale(d), nullptr, nullptr, 0, 1,
                     (char*)out + t0 * qrow, lse ? lse + (size_t)Hq * t0 : nullptr,
                     (int32_t*)workspace};
-        if ((rc = cuda_status(tc_dense_supported(aa) ? tc_dense(aa, st) : simt_attention(aa, st))))
+        if ((rc = cuda_status(run_dense(aa, st))))
             return rc;
     }
     return TAM_OK;

@@ -63,6 +63,8 @@ bool block_tc_disabled() { return env_int("TAM_DISABLE_BLOCK_TC", 0) != 0; }
 
 bool materialise_rows() { return env_int("TAM_MATERIALISE_ROWS", 0) != 0; }
 
+bool dense_pair_tiles_selected() { return env_int("TAM_DENSE_PAIR_TILES", 0) != 0; }
+
 int debug_force_fallback() {
     const int v = env_int("TAM_DEBUG_FORCE_FALLBACK", 0);
     return (v == 1 || v == 2) ? v : 0;

@@ -32,6 +32,9 @@ bool block_tc_disabled();
 // materialised score rows and the row top-k instead of the streamed candidates
 // (A/B comparisons).
 bool materialise_rows();
+// TAM_DENSE_PAIR_TILES=1 runs dense attention on the block-shared pass-3 pipeline (two
+// query tiles per CTA) instead of the single-tile kernel (A/B comparisons).
+bool dense_pair_tiles_selected();
 // TAM_DEBUG_FORCE_FALLBACK=1 (threshold above every key) or =2 (threshold below every
 // key) sends every row the streamed selection would sample to the fallback path, so
 // that path can be tested on ordinary inputs.
