@@ -147,6 +147,25 @@ def test_dense_tensorcore_shapes(tam_lib, oracle_mod, N, Hq, Hkv, d):
     check_close(gl, rl, LSE_ATOL, "dense lse")
 
 
+@pytest.mark.parametrize("N,Hq,Hkv,d", [(1, 4, 1, 64), (333, 32, 8, 128), (1000, 16, 4, 64),
+                                         (2100, 8, 8, 128), (777, 16, 1, 128)])
+def test_dense_on_the_two_tile_pipeline(tam_lib, oracle_mod, monkeypatch, N, Hq, Hkv, d):
+    """The A/B form of the dense comparator (TAM_DENSE_PAIR_TILES=1: the block-shared
+    pass-3 pipeline over every key, two query tiles per CTA, odd tile counts included)."""
+    inp = _inputs(N, Hq, Hkv, d, seed=N + 1, sink=True)
+    monkeypatch.setenv("TAM_DENSE_PAIR_TILES", "1")
+    out, lse = tam_lib.dense_gqa_prefill(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), return_lse=True)
+    torch.cuda.synchronize()
+    monkeypatch.delenv("TAM_DENSE_PAIR_TILES")
+    rows = tam_synth.sample_rows(N, n_random=64) if N > 1000 else None
+    ref, rl = oracle_mod.attn_rows(inp.q, inp.k, inp.v, rows)
+    got, gl = out.float().cpu().numpy(), lse.cpu().numpy().T
+    if rows is not None:
+        got, gl = got[rows], gl[rows]
+    check_close(got, ref, OUT_ATOL["bf16"], "dense, two-tile pipeline")
+    check_close(gl, rl, LSE_ATOL, "dense lse, two-tile pipeline")
+
+
 @pytest.mark.parametrize("N,Hq,Hkv,d,kb,bq", [
     (600, 8, 8, 128, 50, 1), (600, 32, 2, 128, 50, 1), (500, 16, 8, 64, 33, 1),
     (900, 32, 8, 128, 100, 64), (900, 16, 4, 128, 200, 128), (500, 8, 2, 128, 40, 8),

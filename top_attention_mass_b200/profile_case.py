@@ -9,9 +9,13 @@ capture fits the profiler's size rules while the kernels are the benchmarked one
 pass3_gather_stress is the benchmark's out-of-L2 gather: per-query pass 3 on
 device-drawn inputs of the same head shape with a random support of k = 2048 (one
 uniform key per stratum of [0, i]); at N = 262144 its K/V halves are 537 MB each.
+`--row all` runs every row once, in the benchmark's order, after one untimed round, and
+prints the library's kernel-launch count of each row in the last round as JSON, so that
+a one-pass capture of the whole sequence can be split by row.
 Every launch is checked through the library's status block.
 """
 import argparse
+import json
 import os
 import sys
 
@@ -23,7 +27,10 @@ import tam_synth  # noqa: E402
 import top_attention_mass_b200 as tam  # noqa: E402
 
 ROWS = ("pass1_lse", "pass2_mass_topk", "pass2_block_mass_topk", "pass3_gather", "pass3_block",
-        "indexer_topk", "dense_prefill", "pass3_gather_stress")
+        "indexer_topk", "dense_prefill", "pass3_gather_stress", "all")
+# the benchmark's order of the rows of the hot path
+ALL_ORDER = ("pass1_lse", "pass2_mass_topk", "pass3_gather", "pass2_block_mass_topk", "pass3_block",
+             "indexer_topk", "pass3_indexer_support", "dense_prefill")
 
 
 def gather_stress(N, reps):
@@ -52,26 +59,47 @@ def main():
     inp = tam_synth.make_inputs(w, N=a.N)
     q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
     qx, kx = inp.q_idx.cuda(), inp.k_idx.cuda()
-    lse = tam.attention_lse(q, k)
-    # supports only for the pass-3 rows, so the first launches of a pass-2 kernel are the
-    # row's own
-    s1 = tam.mass_select(q, k, lse, 655, 1) if a.row == "pass3_gather" else None
-    s2 = tam.mass_select(q, k, lse, 655, 64) if a.row == "pass3_block" else None
-    for _ in range(a.reps):
-        if a.row == "pass1_lse":
-            tam.attention_lse(q, k)
-        elif a.row == "pass2_mass_topk":
-            tam.mass_select(q, k, lse, 655, 1)
-        elif a.row == "pass2_block_mass_topk":
-            tam.mass_select(q, k, lse, 655, 64)
-        elif a.row == "pass3_gather":
-            tam.sparse_support_attention(q, k, v, s1.idx, s1.length, 1)
-        elif a.row == "pass3_block":
-            tam.sparse_support_attention(q, k, v, s2.idx, s2.length, 64)
-        elif a.row == "indexer_topk":
-            tam.indexer_topk(qx, kx, 1024)
+    ws = tam.Workspace(q.device)
+    box = {"lse": tam.attention_lse(q, k, workspace=ws)}
+
+    def run(row):
+        if row == "pass1_lse":
+            box["lse"] = tam.attention_lse(q, k, workspace=ws)
+        elif row == "pass2_mass_topk":
+            box["s1"] = tam.mass_select(q, k, box["lse"], 655, 1, workspace=ws)
+        elif row == "pass2_block_mass_topk":
+            box["s2"] = tam.mass_select(q, k, box["lse"], 655, 64, workspace=ws)
+        elif row == "pass3_gather":
+            tam.sparse_support_attention(q, k, v, box["s1"].idx, box["s1"].length, 1, workspace=ws)
+        elif row == "pass3_block":
+            tam.sparse_support_attention(q, k, v, box["s2"].idx, box["s2"].length, 64, workspace=ws)
+        elif row == "indexer_topk":
+            box["s3"] = tam.indexer_topk(qx, kx, 1024, workspace=ws)
+        elif row == "pass3_indexer_support":
+            tam.sparse_support_attention(q, k, v, box["s3"].idx, box["s3"].length, 1, workspace=ws)
         else:
-            tam.dense_gqa_prefill(q, k, v)
+            tam.dense_gqa_prefill(q, k, v, workspace=ws)
+
+    if a.row == "all":
+        for row in ALL_ORDER:
+            run(row)
+        counts = {}
+        for _ in range(a.reps):
+            for row in ALL_ORDER:
+                n0 = tam.kernel_launches()
+                run(row)
+                counts[row] = tam.kernel_launches() - n0
+        torch.cuda.synchronize()
+        print(json.dumps({"launches_per_row": counts}))
+    else:
+        # supports only for the pass-3 rows, so the first launches of a pass-2 kernel are
+        # the row's own
+        if a.row == "pass3_gather":
+            run("pass2_mass_topk")
+        if a.row == "pass3_block":
+            run("pass2_block_mass_topk")
+        for _ in range(a.reps):
+            run(a.row)
     torch.cuda.synchronize()
     print(f"profile_case {a.row} N={a.N} reps={a.reps} ok")
 
