@@ -24,7 +24,7 @@ Reported beside it (not part of value):
   support_quality the indexer's support against the mass oracle's at k = 1024
                   (recall@k, output difference), outputs against dense;
   next_rows       the fused block-shared indexer, the distillation target, the budget
-                  sweep and a packed batch of eight sequences.
+                  sweep, a packed batch of eight sequences and a head-dim-256 layer.
 With N > 1 GPUs every rank runs an independent replica of the workload (weak
 scaling, no collective on the data path).  `--impl reference` times the fp64 CPU
 oracle on a bounded sample of the step instead (rank 0 only).  `--workload` runs
@@ -64,6 +64,8 @@ VARLEN_K = 256
 # pages' TTFT figures), Hq 32 / Hkv 8, so that each half of the KV groups the gather walks
 # (2 KB of K and V per key) is 537 MB against 126 MB of L2
 GATHER_BIG = dict(N=262144, Hq=32, Hkv=8, d=128, k=2048)
+# a head-dim-256 layer with the same bytes per token (q 16 x 256, k/v 8 x 256)
+HEAD_DIM_256 = dict(N=32768, Hq=16, Hkv=8, d=256, k=655)
 # L2 ceiling of this GPU as ncu states it (peak L2 sector rate x 32 B), read from the
 # committed capture summarised in profiles/l2_sector_peak_b200.md
 L2_PEAK_GBS = 34580.0
@@ -741,7 +743,9 @@ def measure_next_rows(args, tam, w, calls, flush):
         vl = {"seq_lens": list(VARLEN_SEQS), "budget_k": VARLEN_K,
               "ms_oracle_passes_1_3": t_vo, "q_tok_s_oracle": w.N / (t_vo * 1e-3),
               "ms_dense": t_vd, "q_tok_s_dense": w.N / (t_vd * 1e-3)}
+    hd = measure_head_dim_256(tam, calls.q.device, timed)
     return {
+        "head_dim_256": hd,
         "varlen_batch": vl,
         "budget_sweep": {"ms_pass2_kmax": t_p2, "ms_curve": t_cv, "budgets": budgets,
                          "mean_support_mass": mean_mass,
@@ -753,6 +757,32 @@ def measure_next_rows(args, tam, w, calls, flush):
         "pass3_indexer_block": {"ms": t_att, "q_tok_s": w.N / (t_att * 1e-3),
                                 "gathered_rows": int(n_sel.sum()) * w.Hkv},
     }
+
+
+def measure_head_dim_256(tam, dev, timed):
+    """A d = 256 layer with the 32K layer's bytes per token (N 32768, Hq 16 / Hkv 8):
+    the per-query oracle call (k = 655) and the dense comparator, inputs drawn on the
+    device."""
+    c = HEAD_DIM_256
+    N, Hq, Hkv, d, kb = c["N"], c["Hq"], c["Hkv"], c["d"], c["k"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(3)
+    q = torch.randn(N, Hq, d, generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn(N, Hkv, d, generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn(N, Hkv, d, generator=g, device=dev).to(torch.bfloat16)
+    ws = tam.Workspace(dev)
+    t_or, t_de = timed([
+        lambda: tam.mass_oracle_prefill(q, k, v, kb, 1, workspace=ws, check=False),
+        lambda: tam.dense_gqa_prefill(q, k, v, workspace=ws, check=False)])
+    fb = tam.mass_fallback_rows(q, k, kb, ws)
+    pk, _ = peaks()
+    dense_tf = 4.0 * d * Hq * causal_pairs(N) / (t_de * 1e-3) / 1e12
+    del q, k, v, ws
+    torch.cuda.empty_cache()
+    return {**c, "ms_oracle_passes_1_3": t_or, "q_tok_s_oracle": N / (t_or * 1e-3),
+            "fallback_rows": fb, "ms_dense": t_de, "q_tok_s_dense": N / (t_de * 1e-3),
+            "dense_tflops": dense_tf,
+            "dense_frac_of_burst": dense_tf / pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])}
 
 
 def measure_e2e(args, tam, w, inp, dev, world, local_rank, block_q):

@@ -27,9 +27,11 @@
  *   n_sel = N for per-query support (block_q == 1), ceil(N / block_q) otherwise.
  *
  * dtype: TAM_BF16 (bf16 storage, fp32 accumulation; tensor cores) or TAM_F32
- * (fp32 storage and arithmetic on CUDA cores).  Head dim d: 64 or 128 (tensor
- * cores for bf16), or 256 (CUDA-core kernels for either dtype: same results,
- * lower throughput).
+ * (fp32 storage and arithmetic on CUDA cores).  Head dim d: 64, 128 or 256.  bf16
+ * runs on the tensor cores at every d, except pass 2 at d = 256 when the Q tile of
+ * every KV group does not fit in shared memory (more than 8 KV groups, or more than 4
+ * with 16 query heads per group: CUDA cores, same results), and the indexer, whose
+ * head is 16..128 wide.
  *
  * Packed batches ("_varlen" entry points).  n_seq independent causal sequences
  * are packed along the token axis: sequence s owns tokens [cu[s], cu[s+1]) of
@@ -154,8 +156,10 @@ int tam_mass_oracle_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const 
 
 /*
  * Workspace bytes tam_mass_oracle_prefill_varlen prefers: the largest of
- * tam_mass_oracle_workspace over the batch's sequences (the sequences run one after
- * another and share it).  0 for arguments the call would reject.
+ * tam_mass_oracle_workspace over the batch's sequences (their pass 2 runs one after
+ * another and shares it), plus Hq * T * 4 bytes rounded up to 256, plus 256, for the
+ * packed LSE of the whole batch when the caller passes lse = NULL.  0 for arguments
+ * the call would reject.
  */
 size_t tam_mass_oracle_workspace_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv,
                                         int d, int dtype, int budget_k, int block_q);
@@ -165,8 +169,12 @@ size_t tam_mass_oracle_workspace_varlen(int n_seq, const int64_t* cu_seqlens, in
  * the header comment, "Packed batches").  Each sequence runs passes 1-3 on its own
  * causal prefix, with the same budget_k and block_q; sup_idx/sup_len/sup_mass hold
  * sum_s n_sel(N_s) rows, lse (or NULL) Hq * T floats, out (or NULL) [T, Hq, d].
- * ws_bytes must reach the largest sequence's tam_mass_workspace_min, else
- * TAM_ERR_WORKSPACE before anything is enqueued.
+ * Launches (bf16 tensor-core shapes): pass 1 of every sequence in one launch per
+ * table of up to 128 sequences (query tiles ordered heaviest first over the whole
+ * table), pass 2 sequence by sequence, and pass 3 for per-query supports again one
+ * launch per table (block-shared: sequence by sequence).  ws_bytes must reach the
+ * largest sequence's tam_mass_workspace_min (plus the packed-LSE bytes above when
+ * lse is NULL), else TAM_ERR_WORKSPACE before anything is enqueued.
  */
 int tam_mass_oracle_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv, int d,
                                    int dtype, const void* q, const void* k, const void* v,
@@ -311,7 +319,9 @@ int tam_sparse_support_attention(int64_t N, int Hq, int Hkv, int d, int dtype, c
  * tam_sparse_support_attention over a packed batch (layout in the header comment,
  * "Packed batches"): the support rows of sequence s (positions local to it) start at
  * row sum_{s'<s} n_sel(N_s'), as tam_mass_oracle_prefill_varlen and
- * tam_indexer_topk_varlen write them.  Workspace: tam_sparse_attention_workspace bytes.
+ * tam_indexer_topk_varlen write them.  Per-query supports (block_q = 1) run as one
+ * launch per table of up to 128 sequences.  Workspace: tam_sparse_attention_workspace
+ * bytes.
  */
 int tam_sparse_support_attention_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv,
                                         int d, int dtype, const void* q, const void* k,
@@ -332,7 +342,9 @@ int tam_dense_gqa_prefill(int64_t N, int Hq, int Hkv, int d, int dtype, const vo
 /*
  * tam_dense_gqa_prefill over a packed batch of independent causal sequences (layout
  * in the header comment, "Packed batches"): out [T, Hq, d], lse (or NULL) one
- * [Hq, N_s] block per sequence.  Workspace: tam_dense_workspace bytes (any N).
+ * [Hq, N_s] block per sequence.  bf16 runs as one launch per table of up to 128
+ * sequences, query tiles ordered heaviest first over the table.  Workspace:
+ * tam_dense_workspace bytes (any N).
  */
 int tam_dense_gqa_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv, int d,
                                  int dtype, const void* q, const void* k, const void* v,

@@ -136,8 +136,10 @@ def test_varlen_and_head_dim_host_checks(tam_lib):
     good, gp = cu_ptr([0, 100, 100, 4096])
     ws = L.tam_mass_oracle_workspace_varlen(3, gp, 32, 8, 128, T.TAM_BF16, 256, 1)
     assert ws > 0 and ws % 256 == 0
-    # the largest sequence sets the size: equal to the single-sequence query for it
-    assert ws == L.tam_mass_oracle_workspace(3996, 32, 8, 128, T.TAM_BF16, 256, 1)
+    # the largest sequence sets the size (the single-sequence query for it), plus the packed
+    # LSE of the whole batch (Hq x T floats, rounded up to 256 bytes, and 256 bytes of slack)
+    lse_bytes = (32 * 4096 * 4 + 255) // 256 * 256 + 256
+    assert ws == L.tam_mass_oracle_workspace(3996, 32, 8, 128, T.TAM_BF16, 256, 1) + lse_bytes
     assert L.tam_mass_oracle_workspace_varlen(3, gp, 32, 8, 256, T.TAM_BF16, 256, 1) > 0
     assert L.tam_mass_oracle_workspace_varlen(3, gp, 32, 8, 96, T.TAM_BF16, 256, 1) == 0
     for bad in ([1, 100], [0, 50, 40], [0, 1 << 31]):

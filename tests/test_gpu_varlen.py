@@ -174,6 +174,84 @@ def test_head_dim_256(tam_lib, oracle_mod, N, Hq, Hkv, dtype, kb, bq):
     check_close(dense.float().cpu().numpy(), dref, OUT_ATOL[dtype], "d=256 dense")
 
 
+@pytest.mark.parametrize("N,Hq,Hkv,kb,bq", [(700, 8, 2, 40, 1), (300, 4, 4, 17, 1),
+                                             (1000, 16, 1, 64, 1), (520, 16, 4, 33, 64),
+                                             (1000, 16, 1, 64, 128), (389, 8, 8, 20, 16)])
+def test_head_dim_256_tensor_cores(tam_lib, oracle_mod, N, Hq, Hkv, kb, bq):
+    """bf16 at d = 256 on the tensor-core kernels (pass 1, the single-CTA pass 2 with
+    the streamed selection or the block sums, the 256-wide gather or the block-shared
+    tcgen05 pass 3): several tiles with a ragged tail, every head ratio shape."""
+    inp = _inputs(N, Hq, Hkv, 256, "bf16", seed=N + Hq + bq, sink=True, needles=2)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    res = tam_lib.mass_oracle_prefill(q, k, v, kb, bq)
+    torch.cuda.synchronize()
+    cu = [0, N]
+    gi, gl = _per_sequence_checks(tam_lib, oracle_mod, inp, cu, _flat_lse(res), kb, bq, Hq)
+    ref, _ = oracle_mod.varlen_attn(inp.q, inp.k, inp.v, cu, sup=gi, sup_len=gl, block_q=bq)
+    check_close(res.out.float().cpu().numpy(), ref, OUT_ATOL["bf16"], "d=256 sparse output")
+
+
+@pytest.mark.parametrize("N,Hq,Hkv", [(1, 4, 1), (777, 16, 2), (300, 32, 2), (129, 8, 8)])
+def test_dense_head_dim_256_tensor_cores(tam_lib, oracle_mod, N, Hq, Hkv):
+    inp = _inputs(N, Hq, Hkv, 256, "bf16", seed=N + 5, sink=True)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    out, lse = tam_lib.dense_gqa_prefill(q, k, v, return_lse=True)
+    ref, rl = oracle_mod.attn_rows(inp.q, inp.k, inp.v)
+    check_close(out.float().cpu().numpy(), ref, OUT_ATOL["bf16"], "d=256 dense")
+    check_close(lse.cpu().numpy().T, rl, LSE_ATOL, "d=256 dense lse")
+
+
+# ---------------------------------------------------------------- one launch per batch
+
+def _ragged_cu(n_seq, max_len, seed):
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, max_len + 1, size=n_seq)
+    lens[rng.integers(0, n_seq)] = max_len            # one full-length sequence
+    return [0] + np.cumsum(lens).tolist()
+
+
+@pytest.mark.parametrize("n_seq,max_len,d", [(8, 700, 128), (300, 40, 128), (140, 90, 64)])
+def test_dense_varlen_one_launch_per_table(tam_lib, n_seq, max_len, d):
+    """The packed dense call is one launch per table of up to 128 sequences, and every
+    sequence's rows equal the single-sequence call on its slice bit for bit."""
+    cu = _ragged_cu(n_seq, max_len, seed=n_seq)
+    inp = _inputs(cu[-1], 16, 4, d, "bf16", seed=n_seq + 1)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    n0 = tam_lib.kernel_launches()
+    out, lse = tam_lib.dense_gqa_prefill_varlen(q, k, v, cu, return_lse=True)
+    torch.cuda.synchronize()
+    assert tam_lib.kernel_launches() - n0 == (n_seq + 127) // 128
+    for s in range(n_seq):
+        t0, t1 = cu[s], cu[s + 1]
+        if t1 == t0:
+            continue
+        one, ol = tam_lib.dense_gqa_prefill(q[t0:t1], k[t0:t1], v[t0:t1], return_lse=True)
+        assert torch.equal(one, out[t0:t1]), s
+        assert torch.equal(ol, tam_lib.lse_block(lse, cu, s)), s
+
+
+def test_mass_oracle_varlen_many_sequences(tam_lib, oracle_mod):
+    """A batch of 300 short sequences (three tables): pass 1 and pass 3 as one launch per
+    table, and every sequence bit for bit equal to the single-sequence call."""
+    cu = _ragged_cu(300, 48, seed=7)
+    inp = _inputs(cu[-1], 8, 2, 128, "bf16", seed=11, sink=True)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    res = tam_lib.mass_oracle_prefill_varlen(q, k, v, cu, 12, 1)
+    torch.cuda.synchronize()
+    for s in range(0, 300, 7):
+        t0, t1 = cu[s], cu[s + 1]
+        if t1 == t0:
+            continue
+        one = tam_lib.mass_oracle_prefill(q[t0:t1], k[t0:t1], v[t0:t1], 12, 1)
+        assert torch.equal(one.idx, res.idx[t0:t1]) and torch.equal(one.length, res.length[t0:t1])
+        assert torch.equal(one.value, res.value[t0:t1])
+        assert torch.equal(one.out, res.out[t0:t1])
+        assert torch.equal(one.lse, tam_lib.lse_block(res.lse, cu, s))
+    gi, gl = res.idx.cpu().numpy(), res.length.cpu().numpy()
+    ref, _ = oracle_mod.varlen_attn(inp.q, inp.k, inp.v, cu, sup=gi, sup_len=gl, block_q=1)
+    check_close(res.out.float().cpu().numpy(), ref, OUT_ATOL["bf16"], "varlen 300 sequences")
+
+
 def _flat_lse(res):
     """A single sequence's [Hq, N] lse is its own packed block."""
     return type(res)(res.idx, res.length, res.value, res.lse.reshape(-1), res.out)

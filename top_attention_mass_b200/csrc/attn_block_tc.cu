@@ -35,12 +35,15 @@
 namespace tam {
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kLag = 2;                     // chunks in flight behind the one being signalled
 constexpr int kKeys = 64;                   // keys per chunk
 constexpr int kHalf = 128 * 64 * 2;         // one 128-row x 64-element swizzled half (Q, P)
 constexpr int kHalfKV = kKeys * 64 * 2;     // one 64-key x 64-element swizzled half (K, V)
-static_assert(kLag < kStages - 1, "the gather may run at most kStages - 2 chunks ahead");
+// K/V ring depth and gather lag (chunks in flight behind the one being signalled): four
+// and two; at d = 256, where one chunk of K and V is 64 KB, two and none.
+template <int D>
+__host__ __device__ constexpr int kv_stages() { return D == 256 ? 2 : 4; }
+template <int D>
+__host__ __device__ constexpr int gather_lag() { return D == 256 ? 0 : 2; }
 constexpr int kGatherThreads = 64;          // two gather warps
 constexpr float kRescaleLog2 = 8.f;
 
@@ -50,8 +53,8 @@ __host__ __device__ constexpr int block_threads(int TT) { return 32 * (4 * TT + 
 template <int D, int TT>
 constexpr int block_tc_smem_bytes() {
     // slack + Q tiles + K ring + V ring + P tiles + staged key indices + barriers
-    return 1024 + (D / 64) * (TT * kHalf + 2 * kStages * kHalfKV) + TT * kHalf +
-           kStages * kKeys * 4 + 256;
+    return 1024 + (D / 64) * (TT * kHalf + 2 * kv_stages<D>() * kHalfKV) + TT * kHalf +
+           kv_stages<D>() * kKeys * 4 + 256;
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -87,6 +90,9 @@ __global__ void __launch_bounds__(block_threads(TT), 1)
 k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const BlockTcParams p) {
     constexpr int kThreads = block_threads(TT);
+    constexpr int kStages = kv_stages<D>(), kLag = gather_lag<D>();
+    static_assert(kLag < kStages - 1, "the gather may run at most kStages - 2 chunks ahead");
+    static_assert(256 + 128 * (TT - 1) + D <= 512, "TMEM columns: O of tile tt at 256 + 128 tt");
     constexpr int kTmaWarp = 4 * TT, kMmaWarp = 4 * TT + 1, kGatherWarp0 = 4 * TT + 2;
     constexpr int BQ = 128 / G;
     constexpr int NH = D / 64;
@@ -560,9 +566,14 @@ cudaError_t launch_block_tc(const AttnArgs& a, cudaStream_t st) {
 // Two tiles per CTA when the block has an even number of tiles, else one (dense: two).
 template <int G, int D, bool DENSE>
 cudaError_t launch_tt(const AttnArgs& a, cudaStream_t st) {
-    if (DENSE) return launch_block_tc<G, D, 2, true>(a, st);
-    return (a.block_q / (128 / G)) % 2 == 0 ? launch_block_tc<G, D, 2, false>(a, st)
-                                             : launch_block_tc<G, D, 1, false>(a, st);
+    if constexpr (D == 256) {
+        // one tile (its O takes TMEM columns 256..511); no dense form
+        return DENSE ? cudaErrorNotSupported : launch_block_tc<G, D, 1, false>(a, st);
+    } else {
+        if (DENSE) return launch_block_tc<G, D, 2, true>(a, st);
+        return (a.block_q / (128 / G)) % 2 == 0 ? launch_block_tc<G, D, 2, false>(a, st)
+                                                 : launch_block_tc<G, D, 1, false>(a, st);
+    }
 }
 
 template <int D, bool DENSE>
@@ -581,13 +592,18 @@ cudaError_t dispatch_g(const AttnArgs& a, cudaStream_t st) {
 
 bool block_tc_supported(const AttnArgs& a) {
     const int G = a.Hq / a.Hkv;
-    if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128) || a.block_q <= 1) return false;
+    if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128 && a.d != 256) || a.block_q <= 1)
+        return false;
     if (!(G == 1 || G == 2 || G == 4 || G == 8 || G == 16)) return false;
     return a.block_q % (128 / G) == 0 && a.sup_idx != nullptr;
 }
 
 cudaError_t block_attention_tc(const AttnArgs& a, cudaStream_t st) {
-    return a.d == 64 ? dispatch_g<64, false>(a, st) : dispatch_g<128, false>(a, st);
+    switch (a.d) {
+        case 64: return dispatch_g<64, false>(a, st);
+        case 128: return dispatch_g<128, false>(a, st);
+        default: return dispatch_g<256, false>(a, st);
+    }
 }
 
 bool dense_pair_tiles_supported(const AttnArgs& a) {

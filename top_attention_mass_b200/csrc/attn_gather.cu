@@ -271,33 +271,50 @@ __device__ __forceinline__ int count_le(const int32_t* row, int n, int limit) {
 template <int D, int G, int STAGES, int W>
 __global__ void __launch_bounds__(32 * W, 1)
 k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-              const __nv_bfloat16* __restrict__ v, int N, int Hq, int Hkv, float sl2,
-              const int32_t* __restrict__ sup_idx, const int32_t* __restrict__ sup_len, int kmax,
-              int block_q, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+              const __nv_bfloat16* __restrict__ v, const __grid_constant__ SeqTable seqs, int Hq,
+              int Hkv, float sl2, const int32_t* __restrict__ sup_idx,
+              const int32_t* __restrict__ sup_len, int kmax, int block_q,
+              __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     constexpr int RB = D * 2;
     constexpr int STAGE = 2 * kChunk * RB;
     constexpr bool ROW8 = G > 8;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5;
     const uint32_t wbuf = smem_addr(smem) + warp * STAGES * STAGE;
-    const int64_t total = (int64_t)N * Hkv;
+    // the table's rows (packed tokens); per query, selection row = token row
+    const int rows = seqs.cu[seqs.n_seq] - seqs.cu[0];
+    const int64_t total = (int64_t)rows * Hkv;
     for (int64_t item = (int64_t)blockIdx.x * W + warp; item < total; item += (int64_t)gridDim.x * W) {
         // KV groups in two halves when Hkv is even: all queries of the first half of the
         // groups, then the second, so that each half's K/V (67 MB at the 32K layer) stays
         // in L2 while it is gathered
         const int gh = (Hkv % 2 == 0) ? Hkv / 2 : Hkv;
-        const int64_t per_half = (int64_t)N * gh;
+        const int64_t per_half = (int64_t)rows * gh;
         const int64_t rem = item % per_half;
-        const int i = (int)(rem / gh), g = (int)(item / per_half) * gh + (int)(rem % gh);
+        const int i = seqs.cu[0] + (int)(rem / gh), g = (int)(item / per_half) * gh + (int)(rem % gh);
+        // the query's sequence: its first token and length (keys are positions within it)
+        int tok0 = seqs.cu[0], N = rows;
+        if (seqs.n_seq > 1) {
+            int lo = 0, hi = seqs.n_seq - 1;          // the last s with cu[s] <= i
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (seqs.cu[mid] <= i) lo = mid;
+                else hi = mid - 1;
+            }
+            tok0 = seqs.cu[lo];
+            N = seqs.cu[lo + 1] - tok0;
+        }
+        const __nv_bfloat16* ks = k + (size_t)tok0 * Hkv * D;
+        const __nv_bfloat16* vs = v + (size_t)tok0 * Hkv * D;
         const int32_t* srow;
         int n;
         if (block_q == 1) {
             srow = sup_idx + (size_t)i * kmax;
             n = min(sup_len[i], kmax);
         } else {
-            const int b = i / block_q;
+            const int b = (i - tok0) / block_q;
             srow = sup_idx + (size_t)b * kmax;
-            n = count_le(srow, min(sup_len[b], kmax), i);
+            n = count_le(srow, min(sup_len[b], kmax), i - tok0);
         }
         uint32_t qa[D / 16][4];
         load_q_frags<D>(qa, [&](int r) -> const __nv_bfloat16* {
@@ -310,13 +327,13 @@ k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         const int nch = (n + kChunk - 1) / kChunk;
 #pragma unroll
         for (int s = 0; s < STAGES - 1; ++s) {
-            if (s < nch) issue_chunk_warp<D>(wbuf + s * STAGE, k, v, Hkv, g, srow, s * kChunk, n);
+            if (s < nch) issue_chunk_warp<D>(wbuf + s * STAGE, ks, vs, Hkv, g, srow, s * kChunk, n);
             cp_async_commit();
         }
         for (int ch = 0; ch < nch; ++ch) {
             const int nx = ch + STAGES - 1;
             if (nx < nch)
-                issue_chunk_warp<D>(wbuf + (nx % STAGES) * STAGE, k, v, Hkv, g, srow, nx * kChunk, n);
+                issue_chunk_warp<D>(wbuf + (nx % STAGES) * STAGE, ks, vs, Hkv, g, srow, nx * kChunk, n);
             cp_async_commit();
             cp_async_wait<STAGES - 1>();
             __syncwarp();
@@ -330,7 +347,7 @@ k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
             if (row >= G) return false;
             const int h = g * G + row;
             dst = out + ((size_t)i * Hq + h) * D;
-            ld = lse ? lse + (size_t)h * N + i : nullptr;
+            ld = lse ? lse + (size_t)Hq * tok0 + (size_t)h * N + (i - tok0) : nullptr;
             return true;
         });
     }
@@ -417,7 +434,8 @@ k_attn_block(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 
 template <int D, int G>
 cudaError_t launch_gather(const AttnArgs& a, cudaStream_t st) {
-    constexpr int STAGES = kGatherStages, W = kGatherWarps;
+    // d = 256: six warps (a 32 KB ring each, and twice the registers per warp)
+    constexpr int STAGES = kGatherStages, W = D == 256 ? 6 : kGatherWarps;
     constexpr int smem = W * STAGES * 2 * kChunk * D * 2;
     auto kern = k_attn_gather<D, G, STAGES, W>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -426,12 +444,14 @@ cudaError_t launch_gather(const AttnArgs& a, cudaStream_t st) {
     int dev;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    kern<<<sms, 32 * W, smem, st>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k,
-                                 (const __nv_bfloat16*)a.v, (int)a.N, a.Hq, a.Hkv, a.sl2,
-                                 a.sup_idx, a.sup_len, a.kmax, a.block_q,
-                                 (__nv_bfloat16*)a.out, a.lse);
-    note_launch();
-    return cudaGetLastError();
+    return with_table(a.N, a.seqs, [&](const SeqTable& t) {
+        if (t.cu[t.n_seq] == t.cu[0]) return cudaSuccess;
+        kern<<<sms, 32 * W, smem, st>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k,
+                                     (const __nv_bfloat16*)a.v, t, a.Hq, a.Hkv, a.sl2, a.sup_idx,
+                                     a.sup_len, a.kmax, a.block_q, (__nv_bfloat16*)a.out, a.lse);
+        note_launch();
+        return cudaGetLastError();
+    });
 }
 
 template <int D, int G>
@@ -454,13 +474,25 @@ cudaError_t launch_block(const AttnArgs& a, cudaStream_t st) {
 
 template <int D>
 cudaError_t dispatch(const AttnArgs& a, cudaStream_t st, bool block) {
-    switch (a.Hq / a.Hkv) {
-        case 1: return block ? launch_block<D, 1>(a, st) : launch_gather<D, 1>(a, st);
-        case 2: return block ? launch_block<D, 2>(a, st) : launch_gather<D, 2>(a, st);
-        case 4: return block ? launch_block<D, 4>(a, st) : launch_gather<D, 4>(a, st);
-        case 8: return block ? launch_block<D, 8>(a, st) : launch_gather<D, 8>(a, st);
-        case 16: return block ? launch_block<D, 16>(a, st) : launch_gather<D, 16>(a, st);
-        default: return cudaErrorNotSupported;
+    if constexpr (D == 256) {
+        // one warp per (query, group) only: 16 warps of 256-wide accumulators do not fit
+        switch (a.Hq / a.Hkv) {
+            case 1: return launch_gather<D, 1>(a, st);
+            case 2: return launch_gather<D, 2>(a, st);
+            case 4: return launch_gather<D, 4>(a, st);
+            case 8: return launch_gather<D, 8>(a, st);
+            case 16: return launch_gather<D, 16>(a, st);
+            default: return cudaErrorNotSupported;
+        }
+    } else {
+        switch (a.Hq / a.Hkv) {
+            case 1: return block ? launch_block<D, 1>(a, st) : launch_gather<D, 1>(a, st);
+            case 2: return block ? launch_block<D, 2>(a, st) : launch_gather<D, 2>(a, st);
+            case 4: return block ? launch_block<D, 4>(a, st) : launch_gather<D, 4>(a, st);
+            case 8: return block ? launch_block<D, 8>(a, st) : launch_gather<D, 8>(a, st);
+            case 16: return block ? launch_block<D, 16>(a, st) : launch_gather<D, 16>(a, st);
+            default: return cudaErrorNotSupported;
+        }
     }
 }
 
@@ -468,7 +500,7 @@ cudaError_t dispatch(const AttnArgs& a, cudaStream_t st, bool block) {
 
 bool gather_supported(const AttnArgs& a) {
     const int G = a.Hq / a.Hkv;
-    return a.dtype == TAM_BF16 && a.sup_idx != nullptr && (a.d == 64 || a.d == 128) &&
+    return a.dtype == TAM_BF16 && a.sup_idx != nullptr && (a.d == 64 || a.d == 128 || a.d == 256) &&
            (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
 }
 
@@ -479,7 +511,11 @@ cudaError_t gather_attention(const AttnArgs& a, cudaStream_t st) {
     if (a.block_q > 1 && block_tc_supported(a) && !block_tc_disabled())
         return block_attention_tc(a, st);
     const bool block = a.block_q > 1 && (int64_t)a.block_q * (a.Hq / a.Hkv) >= 64;
-    return a.d == 64 ? dispatch<64>(a, st, block) : dispatch<128>(a, st, block);
+    switch (a.d) {
+        case 64: return dispatch<64>(a, st, block);
+        case 128: return dispatch<128>(a, st, block);
+        default: return dispatch<256>(a, st, false);
+    }
 }
 
 }  // namespace tam

@@ -23,24 +23,28 @@
 namespace tam {
 namespace {
 
-constexpr int kStages = 2;
 constexpr int kHalf = 128 * 64 * 2;     // one 128-row x 64-element swizzled half
 constexpr int kThreads = 192;
 constexpr float kRescaleLog2 = 8.f;     // lazy rescale threshold (factor 256)
 
+// K and V ring depth: two tiles each, one at d = 256 (a 256-wide tile is 64 KB)
+template <int D>
+constexpr int dense_stages() { return D == 256 ? 1 : 2; }
+
 template <int D>
 constexpr int dense_smem_bytes() {
     // Q + K ring + V ring + P + barriers
-    return 1024 + (D / 64) * kHalf * (1 + 2 * kStages) + 2 * kHalf + 512;
+    return 1024 + (D / 64) * kHalf * (1 + 2 * dense_stages<D>()) + 2 * kHalf + 512;
 }
 
 template <int G, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_dense_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, int N, int Hq, int Hkv, int n_qtiles,
-           float sl2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int32_t* status,
-           uint64_t timeout_ns) {
+           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ SeqTable seqs, int Hq,
+           int Hkv, float sl2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+           int32_t* status, uint64_t timeout_ns) {
     constexpr int BQ = 128 / G;
+    constexpr int kStages = dense_stages<D>();
     constexpr int NH = D / 64;
     constexpr uint32_t kTile = NH * kHalf;
     extern __shared__ uint8_t smem_raw[];
@@ -65,9 +69,11 @@ k_dense_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = n_qtiles - 1 - (int)(blockIdx.x / Hkv);
+    int sq, qt;
+    seq_tile<BQ>(seqs, (int)(blockIdx.x / Hkv), sq, qt);
     const int g = (int)(blockIdx.x % Hkv);
-    const int q0 = qt * BQ;
+    const int tok0 = seqs.cu[sq], N = seqs.cu[sq + 1] - tok0;   // this tile's sequence
+    const int q0 = qt * BQ;                                     // positions within it
     const int q_last = min(N, q0 + BQ) - 1;
     const int n_kt = q_last / 128 + 1;
 
@@ -106,7 +112,7 @@ k_dense_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             tc::prefetch_tmap(&tmK);
             tc::prefetch_tmap(&tmV);
             tc::mbar_arrive_expect_tx(q_full, kTile);
-            for (int h = 0; h < NH; ++h) tc::tma_load_3d(sQ + h * kHalf, &tmQ, q_full, h * 64, g * G, q0);
+            for (int h = 0; h < NH; ++h) tc::tma_load_3d(sQ + h * kHalf, &tmQ, q_full, h * 64, g * G, tok0 + q0);
             // K runs up to kStages tiles ahead of S; V up to kStages tiles ahead of P V.
             int nk = 0, nv = 0;
             bool ok = true;
@@ -116,14 +122,14 @@ k_dense_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     if (!tc::wait(&k_empty[s], ((nk / kStages) & 1) ^ 1, gd, 1)) { ok = false; break; }
                     tc::mbar_arrive_expect_tx(&k_full[s], kTile);
                     for (int h = 0; h < NH; ++h)
-                        tc::tma_load_3d(sK + s * kTile + h * kHalf, &tmK, &k_full[s], h * 64, g, nk * 128);
+                        tc::tma_load_3d(sK + s * kTile + h * kHalf, &tmK, &k_full[s], h * 64, g, tok0 + nk * 128);
                     ++nk;
                 } else {
                     const int s = nv % kStages;
                     if (!tc::wait(&v_empty[s], ((nv / kStages) & 1) ^ 1, gd, 2)) { ok = false; break; }
                     tc::mbar_arrive_expect_tx(&v_full[s], kTile);
                     for (int h = 0; h < NH; ++h)
-                        tc::tma_load_3d(sV + s * kTile + h * kHalf, &tmV, &v_full[s], h * 64, g, nv * 128);
+                        tc::tma_load_3d(sV + s * kTile + h * kHalf, &tmV, &v_full[s], h * 64, g, tok0 + nv * 128);
                     ++nv;
                 }
             }
@@ -285,7 +291,7 @@ k_dense_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (ok && tc::wait(o_done, (n_kt - 1) & 1, gd, 10)) {
             tc::fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = out + ((size_t)i * Hq + h) * D;
+            __nv_bfloat16* orow = out + ((size_t)(tok0 + i) * Hq + h) * D;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -306,7 +312,7 @@ k_dense_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     }
                 }
             }
-            if (lse && i < N) lse[(size_t)h * N + i] = (m_used + __log2f(l)) * kLn2;
+            if (lse && i < N) lse[(size_t)Hq * tok0 + (size_t)h * N + i] = (m_used + __log2f(l)) * kLn2;
         }
     }
     __syncthreads();
@@ -325,16 +331,20 @@ cudaError_t launch_dense(const AttnArgs& a, cudaStream_t st) {
         !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, a.N, d * 2, (uint64_t)a.Hkv * d * 2, 64, 1, 128) ||
         !make_tmap_3d_bf16(&tv, a.v, d, a.Hkv, a.N, d * 2, (uint64_t)a.Hkv * d * 2, 64, 1, 128))
         return cudaErrorInvalidValue;
-    const int n_qtiles = (int)((a.N + BQ - 1) / BQ);
     constexpr int smem = dense_smem_bytes<D>();
+    static_assert(smem <= 227 * 1024, "dense tile layout exceeds shared memory");
     auto kern = k_dense_tc<G, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(n_qtiles * a.Hkv), kThreads, smem, st>>>(
-        tq, tk, tv, (int)a.N, a.Hq, a.Hkv, n_qtiles, a.sl2, (__nv_bfloat16*)a.out, a.lse,
-        a.status, wait_timeout_ns());
-    note_launch();
-    return cudaGetLastError();
+    return with_table(a.N, a.seqs, [&](const SeqTable& t) {
+        const int n_tiles = seq_table_tiles(t, BQ);
+        if (n_tiles == 0) return cudaSuccess;
+        kern<<<(unsigned)(n_tiles * a.Hkv), kThreads, smem, st>>>(
+            tq, tk, tv, t, a.Hq, a.Hkv, a.sl2, (__nv_bfloat16*)a.out, a.lse, a.status,
+            wait_timeout_ns());
+        note_launch();
+        return cudaGetLastError();
+    });
 }
 
 template <int D>
@@ -353,12 +363,16 @@ cudaError_t dispatch_g(const AttnArgs& a, cudaStream_t st) {
 
 bool tc_dense_supported(const AttnArgs& a) {
     const int G = a.Hq / a.Hkv;
-    return a.dtype == TAM_BF16 && (a.d == 64 || a.d == 128) &&
+    return a.dtype == TAM_BF16 && (a.d == 64 || a.d == 128 || a.d == 256) &&
            (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
 }
 
 cudaError_t tc_dense(const AttnArgs& a, cudaStream_t st) {
-    return a.d == 64 ? dispatch_g<64>(a, st) : dispatch_g<128>(a, st);
+    switch (a.d) {
+        case 64: return dispatch_g<64>(a, st);
+        case 128: return dispatch_g<128>(a, st);
+        default: return dispatch_g<256>(a, st);
+    }
 }
 
 }  // namespace tam

@@ -7,14 +7,93 @@
 
 namespace tam {
 
+// Packed batches in one launch: sequence s of the table owns the tokens
+// [cu[s], cu[s+1]) of the packed q/k/v rows (a single-sequence call is the table
+// {1, N, {0, N}}).  The kernels that take a table number their query tiles of BQ rows
+// over all of its sequences, heaviest first: every tile with local index L (rows
+// [L BQ, (L+1) BQ) of its sequence) comes before every tile with a smaller L, and
+// within one L the sequences go in order.  Larger batches run as several tables.
+constexpr int kMaxSeqPerLaunch = 128;
+struct SeqTable {
+    int n_seq;
+    int max_len;                      // longest sequence of the table
+    int cu[kMaxSeqPerLaunch + 1];     // absolute token offsets, non-decreasing
+};
+
+inline int seq_table_tiles(const SeqTable& t, int BQ) {
+    int n = 0;
+    for (int s = 0; s < t.n_seq; ++s) n += (t.cu[s + 1] - t.cu[s] + BQ - 1) / BQ;
+    return n;
+}
+
+// Runs fn on the launch's table: *seqs, or the single sequence [0, N) when seqs is null.
+template <class F>
+cudaError_t with_table(int64_t N, const SeqTable* seqs, F&& fn) {
+    if (seqs) return fn(*seqs);
+    SeqTable t{};
+    t.n_seq = 1;
+    t.max_len = (int)N;
+    t.cu[0] = 0;
+    t.cu[1] = (int)N;
+    return fn(t);
+}
+
+#ifdef __CUDACC__
+// (sequence, local tile) of the b-th tile of the table in the order above.  Every lane
+// of the calling warp must take part; all of them get the same answer.
+template <int BQ>
+__device__ __forceinline__ void seq_tile(const SeqTable& t, int b, int& s_out, int& L_out) {
+    if (t.n_seq == 1) {
+        s_out = 0;
+        L_out = (t.cu[1] - t.cu[0] + BQ - 1) / BQ - 1 - b;
+        return;
+    }
+    const int lane = threadIdx.x & 31;
+    // tiles whose local index is at least L
+    auto at_least = [&](int L) {
+        int c = 0;
+        for (int s = lane; s < t.n_seq; s += 32)
+            c += max(0, (t.cu[s + 1] - t.cu[s] + BQ - 1) / BQ - L);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        return c;
+    };
+    // the largest L with at_least(L) > b
+    int lo = 0, hi = (t.max_len + BQ - 1) / BQ - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (at_least(mid) > b) lo = mid;
+        else hi = mid - 1;
+    }
+    // the p-th sequence (in order) that has a tile at index lo
+    int p = b - at_least(lo + 1);
+    s_out = 0;
+    for (int s0 = 0; s0 < t.n_seq; s0 += 32) {
+        const int s = s0 + lane;
+        const bool has = s < t.n_seq && (t.cu[s + 1] - t.cu[s] + BQ - 1) / BQ > lo;
+        unsigned m = __ballot_sync(0xffffffffu, has);
+        const int c = __popc(m);
+        if (p < c) {
+            for (int q = 0; q < p; ++q) m &= m - 1;
+            s_out = s0 + __ffs(m) - 1;
+            break;
+        }
+        p -= c;
+    }
+    L_out = lo;
+}
+#endif
+
 struct LseArgs {
     int64_t N;
     int Hq, Hkv, d, dtype;
     const void* q;
     const void* k;
     float sl2;            // scale * log2(e)
-    float* lse;           // [Hq, N] natural log
+    float* lse;           // [Hq, N] natural log (packed batch: [Hq, N_s] per sequence s,
+                          // starting at element Hq * cu[s])
     int32_t* status;
+    const SeqTable* seqs = nullptr;   // packed batch on the N = T packed rows (tensor cores)
 };
 
 struct MassArgs {
@@ -55,6 +134,7 @@ struct AttnArgs {
     void* out;
     float* lse;
     int32_t* status;
+    const SeqTable* seqs = nullptr;   // packed batch on the N = T packed rows (see LseArgs)
 };
 
 struct IndexerArgs {

@@ -34,9 +34,9 @@ constexpr int lse_smem_bytes() {
 
 template <int G, int D>
 __global__ void __launch_bounds__(kThreads, 2)
-k_lse_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK, int N,
-         int Hkv, int n_qtiles, float sl2, float* __restrict__ lse, int32_t* status,
-         uint64_t timeout_ns, int dbg) {
+k_lse_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+         const __grid_constant__ SeqTable seqs, int Hq, int Hkv, float sl2,
+         float* __restrict__ lse, int32_t* status, uint64_t timeout_ns, int dbg) {
     constexpr int BQ = 128 / G;
     constexpr int NH = D / 64;
     constexpr uint32_t kTileBytes = NH * kHalfBytes;
@@ -57,9 +57,11 @@ k_lse_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
     int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = n_qtiles - 1 - (int)(blockIdx.x / Hkv);
+    int sq, qt;
+    seq_tile<BQ>(seqs, (int)(blockIdx.x / Hkv), sq, qt);
     const int g = (int)(blockIdx.x % Hkv);
-    const int q0 = qt * BQ;
+    const int tok0 = seqs.cu[sq], N = seqs.cu[sq + 1] - tok0;   // this tile's sequence
+    const int q0 = qt * BQ;                                     // positions within it
     const int q_last = min(N, q0 + BQ) - 1;
     const int n_kt = q_last / 128 + 1;
 
@@ -93,7 +95,7 @@ k_lse_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             tc::prefetch_tmap(&tmQ);
             tc::prefetch_tmap(&tmK);
             tc::mbar_arrive_expect_tx(q_full, kTileBytes);
-            for (int h = 0; h < NH; ++h) tc::tma_load_3d(sQ + h * kHalfBytes, &tmQ, q_full, h * 64, g * G, q0);
+            for (int h = 0; h < NH; ++h) tc::tma_load_3d(sQ + h * kHalfBytes, &tmQ, q_full, h * 64, g * G, tok0 + q0);
             int issued = 0;
             for (int t = 0; t < n_kt; ++t) {
                 const int s = t % kStages;
@@ -102,7 +104,7 @@ k_lse_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
                 tc::mbar_arrive_expect_tx(&k_full[s], kTileBytes);
                 for (int h = 0; h < NH; ++h)
                     tc::tma_load_3d(sK + (s * NH + h) * kHalfBytes, &tmK, &k_full[s], h * 64, g,
-                                    t * 128);
+                                    tok0 + t * 128);
                 ++issued;
             }
             // let the last loads of every stage land before the CTA may exit
@@ -208,7 +210,8 @@ k_lse_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtens
             l = l * tc::ex2(m - m_new) + ((s0 + s1) + (s2 + s3));
             m = m_new;
         }
-        if (ok && i < N && !*abort_flag) lse[(size_t)h * N + i] = (m + __log2f(l)) * kLn2;
+        if (ok && i < N && !*abort_flag)
+            lse[(size_t)Hq * tok0 + (size_t)h * N + i] = (m + __log2f(l)) * kLn2;
     }
     __syncthreads();
     if (warp == 0) {
@@ -225,16 +228,18 @@ cudaError_t launch_lse_tc(const LseArgs& a, cudaStream_t st) {
     if (!make_tmap_3d_bf16(&tq, a.q, d, a.Hq, a.N, d * 2, (uint64_t)a.Hq * d * 2, 64, G, BQ) ||
         !make_tmap_3d_bf16(&tk, a.k, d, a.Hkv, a.N, d * 2, (uint64_t)a.Hkv * d * 2, 64, 1, 128))
         return cudaErrorInvalidValue;
-    const int n_qtiles = (int)((a.N + BQ - 1) / BQ);
     constexpr int smem = lse_smem_bytes<D>();
     auto kern = k_lse_tc<G, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const float sl2 = a.sl2;
-    kern<<<(unsigned)(n_qtiles * a.Hkv), kThreads, smem, st>>>(
-        tq, tk, (int)a.N, a.Hkv, n_qtiles, sl2, a.lse, a.status, wait_timeout_ns(), debug_flags());
-    note_launch();
-    return cudaGetLastError();
+    return with_table(a.N, a.seqs, [&](const SeqTable& t) {
+        const int n_tiles = seq_table_tiles(t, BQ);
+        if (n_tiles == 0) return cudaSuccess;
+        kern<<<(unsigned)(n_tiles * a.Hkv), kThreads, smem, st>>>(
+            tq, tk, t, a.Hq, a.Hkv, a.sl2, a.lse, a.status, wait_timeout_ns(), debug_flags());
+        note_launch();
+        return cudaGetLastError();
+    });
 }
 
 template <int D>
@@ -253,12 +258,16 @@ cudaError_t dispatch_g(const LseArgs& a, cudaStream_t st) {
 
 bool tc_lse_supported(const LseArgs& a) {
     const int G = a.Hq / a.Hkv;
-    return a.dtype == TAM_BF16 && (a.d == 64 || a.d == 128) &&
+    return a.dtype == TAM_BF16 && (a.d == 64 || a.d == 128 || a.d == 256) &&
            (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
 }
 
 cudaError_t tc_lse(const LseArgs& a, cudaStream_t st) {
-    return a.d == 64 ? dispatch_g<64>(a, st) : dispatch_g<128>(a, st);
+    switch (a.d) {
+        case 64: return dispatch_g<64>(a, st);
+        case 128: return dispatch_g<128>(a, st);
+        default: return dispatch_g<256>(a, st);
+    }
 }
 
 }  // namespace tam

@@ -39,7 +39,8 @@
 namespace tam {
 namespace {
 
-constexpr int kStages = 2;
+// K ring depth: two tiles; one where the Q of every group at d = 256 leaves no room
+// for a second 64 KB tile.
 // Eight mass warps (two per TMEM lane quarter, each on half of the columns), then the
 // TMA producer and the MMA issuer.
 constexpr int kMassWarps = 8;
@@ -52,8 +53,8 @@ constexpr int kModeQuery = 0, kModeBlock = 1, kModeIndexer = 2, kModeQueryStream
               kModeIndexerStream = 4;
 
 // alignment slack + Q (all groups) + K ring + lse2 + thresholds + barriers
-__host__ __device__ constexpr int mass_smem_bytes(int NQ, int D, int Hkv) {
-    return 1024 + Hkv * NQ * D * 2 + kStages * 128 * D * 2 + Hkv * NQ * 4 + 128 + 512;
+__host__ __device__ constexpr int mass_smem_bytes(int NQ, int D, int Hkv, int stages = 2) {
+    return 1024 + Hkv * NQ * D * 2 + stages * 128 * D * 2 + Hkv * NQ * 4 + 128 + 512;
 }
 constexpr int kMaxDynSmem = 227 * 1024;
 
@@ -79,7 +80,7 @@ __host__ __device__ __forceinline__ int64_t bmass_offset(int64_t b, int block_q)
     return (int64_t)block_q * b * (b + 1) / 2;
 }
 
-template <int G, int D, int NQ, int MODE>
+template <int G, int D, int NQ, int MODE, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
 k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const MassParams p) {
@@ -452,7 +453,7 @@ __global__ void __launch_bounds__(256) k_block_select(const unsigned long long* 
     if (tid == 0) sup_len[b] = m;
 }
 
-template <int G, int D, int NQ, int MODE>
+template <int G, int D, int NQ, int MODE, int KS>
 cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     constexpr int BQ = NQ / G;
     constexpr bool BLOCK = MODE == kModeBlock;
@@ -493,8 +494,8 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     p.timeout_ns = wait_timeout_ns();
     p.dbg = debug_flags();
     if (p.n_ctiles <= 0) return cudaSuccess;
-    const int smem = mass_smem_bytes(NQ, D, a.Hkv);
-    auto kern = k_mass_tc<G, D, NQ, MODE>;
+    const int smem = mass_smem_bytes(NQ, D, a.Hkv, KS);
+    auto kern = k_mass_tc<G, D, NQ, MODE, KS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     if (BLOCK) {
@@ -513,11 +514,17 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-// Only (G, NQ) pairs with 4..32 queries per CTA are instantiated.
+// Only (G, NQ) pairs with 4..32 queries per CTA are instantiated (at d = 256, NQ <= 64:
+// the wider Q of every group does not fit in shared memory beside the K ring).
 template <int G, int D, int NQ, int MODE>
 cudaError_t launch_if_valid(const MassArgs& a, cudaStream_t st) {
-    if constexpr (NQ / G >= 4 && NQ / G <= 32)
-        return launch_mass<G, D, NQ, MODE>(a, st);
+    if constexpr (NQ / G >= 4 && NQ / G <= 32 && (D < 256 || NQ <= 64)) {
+        if constexpr (D == 256) {
+            if (mass_smem_bytes(NQ, D, a.Hkv, 2) > kMaxDynSmem)
+                return launch_mass<G, D, NQ, MODE, 1>(a, st);
+        }
+        return launch_mass<G, D, NQ, MODE, 2>(a, st);
+    }
     else
         return cudaErrorNotSupported;
 }
@@ -546,16 +553,20 @@ cudaError_t dispatch_nq(const MassArgs& a, cudaStream_t st) {
 
 template <int MODE>
 cudaError_t dispatch(const MassArgs& a, cudaStream_t st) {
-    return a.d == 64 ? dispatch_nq<64, MODE>(a, st) : dispatch_nq<128, MODE>(a, st);
+    switch (a.d) {
+        case 64: return dispatch_nq<64, MODE>(a, st);
+        case 128: return dispatch_nq<128, MODE>(a, st);
+        default: return dispatch_nq<256, MODE>(a, st);
+    }
 }
 
 // The indexer runs as a single-head problem: Hq = Hkv = 1, d = d_idx, 32 queries per CTA.
 cudaError_t launch_indexer_tc(const MassArgs& a, cudaStream_t st) {
     if (a.stream)
-        return a.d == 64 ? launch_mass<1, 64, 32, kModeIndexerStream>(a, st)
-                         : launch_mass<1, 128, 32, kModeIndexerStream>(a, st);
-    return a.d == 64 ? launch_mass<1, 64, 32, kModeIndexer>(a, st)
-                     : launch_mass<1, 128, 32, kModeIndexer>(a, st);
+        return a.d == 64 ? launch_mass<1, 64, 32, kModeIndexerStream, 2>(a, st)
+                         : launch_mass<1, 128, 32, kModeIndexerStream, 2>(a, st);
+    return a.d == 64 ? launch_mass<1, 64, 32, kModeIndexer, 2>(a, st)
+                     : launch_mass<1, 128, 32, kModeIndexer, 2>(a, st);
 }
 
 }  // namespace
@@ -567,10 +578,10 @@ int tc_mass_columns(const MassArgs& a) {
     // (queries per CTA NQ/G kept within [4, 32] so the per-thread accumulators stay
     // in registers)
     if (a.Hkv > 64 || G < 1) return 0;
-    for (int nq = 128; nq >= 32; nq >>= 1) {
+    for (int nq = a.d == 256 ? 64 : 128; nq >= 32; nq >>= 1) {
         const int bq = nq / G;
         if (bq < 4 || bq > 32) continue;
-        if (mass_smem_bytes(nq, a.d, a.Hkv) <= kMaxDynSmem) return nq;
+        if (mass_smem_bytes(nq, a.d, a.Hkv, a.d == 256 ? 1 : 2) <= kMaxDynSmem) return nq;
     }
     return 0;
 }
@@ -578,7 +589,7 @@ int tc_mass_columns(const MassArgs& a) {
 bool tc_mass_supported(const MassArgs& a) {
     const int G = a.Hq / a.Hkv;
     const int nq = tc_mass_columns(a);
-    if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128) || nq == 0) return false;
+    if (a.dtype != TAM_BF16 || (a.d != 64 && a.d != 128 && a.d != 256) || nq == 0) return false;
     if (!(G == 1 || G == 2 || G == 4 || G == 8 || G == 16)) return false;
     if (a.block_q > 1 && a.block_q > (1 << 20)) return false;
     return true;

@@ -24,6 +24,9 @@ constexpr int kMaxBudget = 4096;
 constexpr int kSimtPersistentCtas = 1024;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+// Packed LSE of a whole batch ([Hq, N_s] per sequence) kept at the end of the workspace,
+// with slack to start it on a 256-byte boundary.
+inline size_t packed_lse_bytes(int64_t T, int Hq) { return align256((size_t)Hq * T * 4) + 256; }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -31,7 +34,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 int check_shape(int64_t N, int Hq, int Hkv, int d, int dtype) {
     if (N < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TAM_ERR_INVALID_ARG;
     if (dtype != TAM_BF16 && dtype != TAM_F32) return TAM_ERR_INVALID_ARG;
-    // 64 and 128 run on the tensor cores; 256 on the CUDA-core kernels
+    // bf16 runs on the tensor cores (d = 256 where its tiles fit), fp32 on the CUDA cores
     if (d != 64 && d != 128 && d != 256) return TAM_ERR_UNSUPPORTED;
     if (N >= (int64_t(1) << 31) - 1) return TAM_ERR_UNSUPPORTED;
     // the CUDA-core kernels stage one query row (all heads) in shared memory
@@ -405,6 +408,22 @@ int check_cu_seqlens(int n_seq, const int64_t* cu, int64_t* max_len) {
 
 inline size_t elt_bytes(int dtype) { return dtype == TAM_F32 ? 4 : 2; }
 
+// A packed batch as tables of up to kMaxSeqPerLaunch sequences (one launch per kernel
+// each); tables of empty sequences only are skipped.
+template <class F>
+int for_seq_tables(int n_seq, const int64_t* cu, F&& fn) {
+    for (int s0 = 0; s0 < n_seq; s0 += kMaxSeqPerLaunch) {
+        SeqTable t{};
+        t.n_seq = std::min(kMaxSeqPerLaunch, n_seq - s0);
+        for (int s = 0; s <= t.n_seq; ++s) t.cu[s] = (int)cu[s0 + s];
+        for (int s = 0; s < t.n_seq; ++s) t.max_len = std::max(t.max_len, t.cu[s + 1] - t.cu[s]);
+        if (t.max_len == 0) continue;
+        const int rc = fn(t);
+        if (rc) return rc;
+    }
+    return TAM_OK;
+}
+
 // Range checks of the indexer entry points (dtype and d_idx >= 1 checked by the caller).
 int check_indexer_args(int64_t N, int d_idx, int dtype, int budget_k, int block_q) {
     if (d_idx != 16 && d_idx != 32 && d_idx != 64 && d_idx != 128) return TAM_ERR_UNSUPPORTED;
@@ -550,7 +569,8 @@ size_t tam_mass_oracle_workspace_varlen(int n_seq, const int64_t* cu_seqlens, in
         const int64_t n = cu_seqlens[s + 1] - cu_seqlens[s];
         if (n > 0) total = std::max(total, plan_mass(n, Hq, Hkv, d, dtype, budget_k, block_q).total);
     }
-    return total;
+    // room for the packed LSE of the whole batch (used when the caller passes no lse)
+    return total + packed_lse_bytes(cu_seqlens[n_seq], Hq);
 }
 
 int tam_mass_oracle_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, int Hkv, int d,
@@ -566,17 +586,79 @@ int tam_mass_oracle_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq,
     if ((rc = check_prefill_ptrs(q, k, v, sup_idx, sup_len, sup_mass, lse, out, workspace)))
         return rc;
     if (ws_bytes < kStatusBytes) return TAM_ERR_WORKSPACE;
+    const int64_t T = cu_seqlens[n_seq];
+    const float sl2 = score_log2_scale(d);
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t qrow = (size_t)Hq * d * elt_bytes(dtype), krow = (size_t)Hkv * d * elt_bytes(dtype);
+    LseArgs lall{T, Hq, Hkv, d, dtype, q, k, sl2, lse, (int32_t*)workspace};
+    if (T > 0 && tc_lse_supported(lall)) {
+        // Pass 1 of every sequence in one launch per table, into lse or (when the caller
+        // passes none) the packed-LSE area at the end of the workspace; then pass 2 of each
+        // sequence on its slice; then, for per-query supports, pass 3 of every sequence in
+        // one launch per table.
+        size_t ws2 = ws_bytes;
+        if (!lse) {
+            const size_t lb = packed_lse_bytes(T, Hq);
+            if (ws_bytes < lb + kStatusBytes) return TAM_ERR_WORKSPACE;
+            ws2 = (ws_bytes - lb) & ~size_t(255);
+            lall.lse = (float*)((char*)workspace + ws2);
+        }
+        for (int s = 0; s < n_seq; ++s) {
+            const int64_t n = cu_seqlens[s + 1] - cu_seqlens[s];
+            if (n > 0 && ws2 < plan_mass(n, Hq, Hkv, d, dtype, budget_k, block_q).min_total)
+                return TAM_ERR_WORKSPACE;
+        }
+        if ((rc = start_call(workspace, st))) return rc;
+        rc = for_seq_tables(n_seq, cu_seqlens, [&](const SeqTable& t) {
+            LseArgs la = lall;
+            la.seqs = &t;
+            return cuda_status(tc_lse(la, st));
+        });
+        if (rc) return rc;
+        int64_t sel0 = 0;
+        for (int s = 0; s < n_seq; ++s) {
+            const int64_t t0 = cu_seqlens[s], n = cu_seqlens[s + 1] - t0;
+            if (n == 0) continue;
+            const MassPlan plan = plan_mass(n, Hq, Hkv, d, dtype, budget_k, block_q);
+            rc = launch_mass_select(n, Hq, Hkv, d, dtype, (const char*)q + t0 * qrow,
+                                    (const char*)k + t0 * krow, lall.lse + (size_t)Hq * t0,
+                                    budget_k, block_q, sup_idx + sel0 * budget_k, sup_len + sel0,
+                                    sup_mass + sel0 * budget_k, (char*)workspace, ws2, plan, st,
+                                    sl2);
+            if (rc) return rc;
+            sel0 += n_selection_units(n, block_q);
+        }
+        if (!out) return TAM_OK;
+        AttnArgs aall{T, Hq, Hkv, d, dtype, q, k, v, sl2, sup_idx, sup_len, budget_k, block_q,
+                      out, nullptr, (int32_t*)workspace};
+        if (block_q == 1 && gather_supported(aall))
+            return for_seq_tables(n_seq, cu_seqlens, [&](const SeqTable& t) {
+                AttnArgs aa = aall;
+                aa.seqs = &t;
+                return cuda_status(gather_attention(aa, st));
+            });
+        sel0 = 0;
+        for (int s = 0; s < n_seq; ++s) {
+            const int64_t t0 = cu_seqlens[s], n = cu_seqlens[s + 1] - t0;
+            if (n == 0) continue;
+            AttnArgs aa{n, Hq, Hkv, d, dtype, (const char*)q + t0 * qrow,
+                        (const char*)k + t0 * krow, (const char*)v + t0 * krow, sl2,
+                        sup_idx + sel0 * budget_k, sup_len + sel0, budget_k, block_q,
+                        (char*)out + t0 * qrow, nullptr, (int32_t*)workspace};
+            if ((rc = cuda_status(run_sparse_attention(aa, st)))) return rc;
+            sel0 += n_selection_units(n, block_q);
+        }
+        return TAM_OK;
+    }
     for (int s = 0; s < n_seq; ++s) {
         const int64_t n = cu_seqlens[s + 1] - cu_seqlens[s];
         if (n > 0 && ws_bytes < plan_mass(n, Hq, Hkv, d, dtype, budget_k, block_q).min_total)
             return TAM_ERR_WORKSPACE;
     }
-    cudaStream_t st = (cudaStream_t)stream;
     if ((rc = start_call(workspace, st))) return rc;
-    // The sequences are independent problems: each one runs the single-sequence path on
-    // its slice of the packed tensors, one after another on `stream`, reusing the
-    // workspace (stream order separates them).
-    const size_t qrow = (size_t)Hq * d * elt_bytes(dtype), krow = (size_t)Hkv * d * elt_bytes(dtype);
+    // CUDA-core shapes: each sequence runs the single-sequence path on its slice of the
+    // packed tensors, one after another on `stream`, reusing the workspace (stream order
+    // separates them).
     int64_t sel0 = 0;
     for (int s = 0; s < n_seq; ++s) {
         const int64_t t0 = cu_seqlens[s], n = cu_seqlens[s + 1] - t0;
@@ -853,6 +935,15 @@ int tam_sparse_support_attention_varlen(int n_seq, const int64_t* cu_seqlens, in
     cudaStream_t st = (cudaStream_t)stream;
     if ((rc = start_call(workspace, st))) return rc;
     const size_t qrow = (size_t)Hq * d * elt_bytes(dtype), krow = (size_t)Hkv * d * elt_bytes(dtype);
+    // per-query supports: every sequence in one launch per table
+    AttnArgs aall{cu_seqlens[n_seq], Hq, Hkv, d, dtype, q, k, v, score_log2_scale(d), sup_idx,
+                  sup_len, kmax, block_q, out, lse, (int32_t*)workspace};
+    if (block_q == 1 && gather_supported(aall))
+        return for_seq_tables(n_seq, cu_seqlens, [&](const SeqTable& t) {
+            AttnArgs aa = aall;
+            aa.seqs = &t;
+            return cuda_status(gather_attention(aa, st));
+        });
     int64_t sel0 = 0;
     for (int s = 0; s < n_seq; ++s) {
         const int64_t t0 = cu_seqlens[s], n = cu_seqlens[s + 1] - t0;
@@ -905,6 +996,15 @@ int tam_dense_gqa_prefill_varlen(int n_seq, const int64_t* cu_seqlens, int Hq, i
     cudaStream_t st = (cudaStream_t)stream;
     if ((rc = start_call(workspace, st))) return rc;
     const size_t qrow = (size_t)Hq * d * elt_bytes(dtype), krow = (size_t)Hkv * d * elt_bytes(dtype);
+    // tensor-core shapes: every sequence in one launch per table
+    AttnArgs aall{cu_seqlens[n_seq], Hq, Hkv, d, dtype, q, k, v, score_log2_scale(d), nullptr,
+                  nullptr, 0, 1, out, lse, (int32_t*)workspace};
+    if (tc_dense_supported(aall))
+        return for_seq_tables(n_seq, cu_seqlens, [&](const SeqTable& t) {
+            AttnArgs aa = aall;
+            aa.seqs = &t;
+            return cuda_status(tc_dense(aa, st));
+        });
     for (int s = 0; s < n_seq; ++s) {
         const int64_t t0 = cu_seqlens[s], n = cu_seqlens[s + 1] - t0;
         if (n == 0) continue;

@@ -418,13 +418,14 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // polynomial fitted to 2^f in relative error on Chebyshev nodes (Lawson-weighted
 // least squares; max relative error 2.7e-6 evaluated in fp32 Horner form), and n is
 // added to the exponent field.  x is clamped at -125 so that the field stays
-// positive: inputs below that give about 2^-125 instead of ex2's 0.
+// positive, and inputs below -125 (a masked score's -inf among them) give exactly 0,
+// as ex2 does: a masked key then adds nothing to a P V product, whatever its V row.
 constexpr float kEx2C0 = 0.99999928f, kEx2C1 = 0.69312179f, kEx2C2 = 0.24024744f,
                 kEx2C3 = 0.055917859f, kEx2C4 = 0.009570101f;
 constexpr float kRoundMagic = 12582912.f;      // 1.5 * 2^23, bits 0x4B400000
 
-__device__ __forceinline__ float ex2_fma(float x) {
-    x = fmaxf(x, -125.f);
+__device__ __forceinline__ float ex2_fma(float x0) {
+    const float x = fmaxf(x0, -125.f);
     const float t = x + kRoundMagic;
     const float f = x - (t - kRoundMagic);
     const int n = __float_as_int(t) - 0x4B400000;
@@ -432,7 +433,8 @@ __device__ __forceinline__ float ex2_fma(float x) {
     p = fmaf(p, f, kEx2C2);
     p = fmaf(p, f, kEx2C1);
     p = fmaf(p, f, kEx2C0);
-    return __int_as_float(__float_as_int(p) + (n << 23));
+    const float y = __int_as_float(__float_as_int(p) + (n << 23));
+    return x0 < -125.f ? 0.f : y;
 }
 
 // ex2_fma on a pair (x0, x1) with packed adds and FMAs.
@@ -450,6 +452,8 @@ __device__ __forceinline__ void ex2_fma2(float x0, float x1, float& y0, float& y
     f2_unpack(p2, p0, p1);
     y0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
     y1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
+    y0 = x0 < -125.f ? 0.f : y0;
+    y1 = x1 < -125.f ? 0.f : y1;
 }
 
 }  // namespace tc

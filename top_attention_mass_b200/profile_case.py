@@ -5,7 +5,8 @@
 Rows: pass1_lse, pass2_mass_topk, pass2_block_mass_topk, pass3_gather, pass3_block,
 indexer_topk, dense_prefill.  Shapes are those of the 32K workload (Hq=32, Hkv=8,
 d=128, bf16, k=655, B_q=64, indexer d_idx=64 / k=1024) at the given N, so that a
-capture fits the profiler's size rules while the kernels are the benchmarked ones.
+capture fits the profiler's size rules while the kernels are the benchmarked ones;
+`--head-dim 256` takes a Hq 16 / Hkv 8, d 256 layer instead.
 pass3_gather_stress is the benchmark's out-of-L2 gather: per-query pass 3 on
 device-drawn inputs of the same head shape with a random support of k = 2048 (one
 uniform key per stratum of [0, i]); at N = 262144 its K/V halves are 537 MB each.
@@ -50,12 +51,17 @@ def main():
     ap.add_argument("--row", choices=ROWS, required=True)
     ap.add_argument("--N", type=int, default=16384)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--head-dim", type=int, default=128, choices=(128, 256),
+                    help="256: a Hq 16 / Hkv 8, d 256 layer (same bytes per token)")
     a = ap.parse_args()
     if a.row == "pass3_gather_stress":
         gather_stress(a.N, a.reps)
         print(f"profile_case {a.row} N={a.N} reps={a.reps} ok")
         return
     w = tam_synth.WORKLOADS["indexer32k"]
+    if a.head_dim == 256:
+        w = tam_synth.custom("hd256", a.N, 16, 8, 256, "bf16", 655, (1, 64), sink=True,
+                             needles=64, d_idx=64)
     inp = tam_synth.make_inputs(w, N=a.N)
     q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
     qx, kx = inp.q_idx.cuda(), inp.k_idx.cuda()
