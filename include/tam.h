@@ -76,7 +76,7 @@ typedef enum {
     TAM_ERR_WORKSPACE = 3,
     TAM_ERR_CUDA = 4,
     TAM_ERR_TIMEOUT = 5,
-    TAM_ERR_OVERFLOW = 6    /* kept for ABI stability; no current kernel reports it */
+    TAM_ERR_OVERFLOW = 6    /* debug-checks build only: a store outside its buffer, skipped */
 } tam_status;
 
 typedef enum { TAM_BF16 = 0, TAM_F32 = 1 } tam_dtype;
@@ -373,8 +373,17 @@ uint64_t tam_kernel_launches(void);
 /*
  * Waits for `stream`, then reads the device status block at the start of
  * `workspace` that the last call using this workspace wrote.  Returns TAM_OK,
- * TAM_ERR_TIMEOUT or TAM_ERR_CUDA.  `detail` (may be NULL)
- * receives 8 int32 words: [0] status, [1] kernel id, [2..7] kernel-specific.
+ * TAM_ERR_TIMEOUT or TAM_ERR_CUDA (and, from the debug-checks build libtam_debug.so,
+ * TAM_ERR_OVERFLOW).  `detail` (may be NULL) receives 8 int32 words: [0] status,
+ * [1] kernel id, [2..7] kernel-specific (overflow: [2] site 1 slab row / 2 candidate /
+ * 3 block mass, [3] index, [4] extent, truncated to 32 bits).
+ *
+ * Debug-checks build: compiled with -DTAM_DEBUG_CHECKS (same symbols), the pass-2
+ * kernels check every slab-row, candidate and block-mass store against the extent the
+ * host planned for the launch; instead of an out-of-range store they record
+ * TAM_ERR_OVERFLOW here and skip it.  With the environment variable
+ * TAM_DEBUG_SHRINK_EXTENTS set, the host plans extents of at most 64 entries, so that
+ * the checks fire on stores that still land inside the real buffers.
  */
 int tam_check_status(const void* workspace, void* stream, int32_t* detail);
 

@@ -24,6 +24,16 @@ def test_every_declared_symbol_is_exported(tam_lib):
     assert set(names) == set(tam_lib.EXPORTED)
 
 
+def test_debug_checks_build_exports_the_same_symbols(tam_lib):
+    """libtam_debug.so (the pass-2 stores checked against their extents) is built beside
+    libtam.so and exports every declared symbol too."""
+    path = os.path.join(ROOT, "top_attention_mass_b200", "libtam_debug.so")
+    assert os.path.exists(path), "build() builds the debug-checks library"
+    D = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(D, n), n
+
+
 def test_version_and_status_strings(tam_lib):
     assert tam_lib.version() >= 100
     for code in range(7):

@@ -166,6 +166,31 @@ def test_dense_on_the_two_tile_pipeline(tam_lib, oracle_mod, monkeypatch, N, Hq,
     check_close(gl, rl, LSE_ATOL, "dense lse, two-tile pipeline")
 
 
+@pytest.mark.parametrize("N,Hq,Hkv,d", [(700, 32, 8, 128), (300, 8, 2, 64), (260, 8, 2, 256),
+                                         (150, 16, 1, 128)])
+def test_gather_skips_invalid_support_entries(tam_lib, oracle_mod, N, Hq, Hkv, d):
+    """Per-query pass 3 on supports mixing valid keys with negative ones, keys after the
+    query and keys past the sequence (never read): the result is the oracle's on the
+    valid entries, and a row with no valid entry gives a zero row and lse = -inf."""
+    inp = _inputs(N, Hq, Hkv, d, seed=N + d, sink=True)
+    rng = np.random.default_rng(N + d)
+    kmax = 48
+    sup = rng.integers(0, N, size=(N, kmax)).astype(np.int32)      # about half after i
+    sup[:, ::5] = -7
+    sup[:, 1::7] = N + 1000000
+    sup[:, 2::9] = np.iinfo(np.int32).max
+    ln = rng.integers(0, kmax + 1, size=N).astype(np.int32)
+    ln[N // 2] = kmax
+    sup[N // 2, :] = -1
+    out, lse = tam_lib.sparse_support_attention(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(),
+                                                torch.from_numpy(sup).cuda(),
+                                                torch.from_numpy(ln).cuda(), 1, return_lse=True)
+    ref, rl = oracle_mod.attn_rows(inp.q, inp.k, inp.v, None, sup=sup, sup_len=ln)
+    check_close(out.float().cpu().numpy(), ref, OUT_ATOL["bf16"], "pass 3, invalid entries")
+    check_close(lse.cpu().numpy().T, rl, LSE_ATOL, "pass 3 lse, invalid entries")
+    assert not out[N // 2].float().abs().any()
+
+
 @pytest.mark.parametrize("N,Hq,Hkv,d,kb,bq", [
     (600, 8, 8, 128, 50, 1), (600, 32, 2, 128, 50, 1), (500, 16, 8, 64, 33, 1),
     (900, 32, 8, 128, 100, 64), (900, 16, 4, 128, 200, 128), (500, 8, 2, 128, 40, 8),

@@ -32,7 +32,10 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtam.so")
+# TAM_LIBRARY=debug loads the debug-checks build (pass-2 stores checked against their
+# extents; see tam.h, TAM_ERR_OVERFLOW) instead of the release library
+LIB_PATH = os.path.join(_HERE, "libtam_debug.so" if os.environ.get("TAM_LIBRARY") == "debug"
+                        else "libtam.so")
 
 TAM_OK, TAM_ERR_INVALID_ARG, TAM_ERR_UNSUPPORTED, TAM_ERR_WORKSPACE = 0, 1, 2, 3
 TAM_ERR_CUDA, TAM_ERR_TIMEOUT, TAM_ERR_OVERFLOW = 4, 5, 6

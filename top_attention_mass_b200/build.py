@@ -21,6 +21,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libtam.so")
+# the debug-checks build: pass-2 stores checked against their extents (TAM_DEBUG_CHECKS)
+DEBUG_LIB = os.path.join(PKG, "libtam_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
@@ -54,13 +56,18 @@ def _compile(src: str, obj: str, extra) -> str:
     return r.stderr
 
 
-def build_library(force: bool = False, jobs: int = 0, verbose: bool = False, extra=()) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build_library(force: bool = False, jobs: int = 0, verbose: bool = False, extra=(),
+                  debug_checks: bool = False) -> str:
+    """Compile every csrc/*.cu and link libtam.so (libtam_debug.so with debug_checks)."""
+    build_dir = os.path.join(BUILD, "debug") if debug_checks else BUILD
+    lib_path = DEBUG_LIB if debug_checks else LIB
+    extra = [*extra, "-DTAM_DEBUG_CHECKS"] if debug_checks else list(extra)
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdrs = _headers()
     objs, todo = [], []
     for s in srcs:
-        o = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")
+        o = os.path.join(build_dir, os.path.basename(s)[:-3] + ".o")
         objs.append(o)
         if force or _stale(o, [s, *hdrs, __file__]):
             todo.append((s, o))
@@ -72,14 +79,14 @@ def build_library(force: bool = False, jobs: int = 0, verbose: bool = False, ext
                 msg = f.result()
                 if verbose and msg:
                     print(os.path.basename(futs[f]), msg)
-    if force or todo or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or todo or _stale(lib_path, objs):
+        tmp = lib_path + f".tmp{os.getpid()}"
         cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 def main():
@@ -87,9 +94,11 @@ def main():
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--jobs", type=int, default=0)
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--debug-checks", action="store_true")
     a = ap.parse_args()
     extra = ["-Xptxas", "-v"] if a.ptxas_verbose else []
-    print(build_library(force=a.force or a.ptxas_verbose, jobs=a.jobs, verbose=True, extra=extra))
+    print(build_library(force=a.force or a.ptxas_verbose, jobs=a.jobs, verbose=True, extra=extra,
+                        debug_checks=a.debug_checks))
 
 
 if __name__ == "__main__":

@@ -90,10 +90,10 @@ __device__ __forceinline__ uint32_t swz(int r, int pc) {
 
 // Issue the cp.async copies of one chunk (kChunk K rows then kChunk V rows of KV
 // group g) into `buf`; `nthr` threads starting at `t0` cooperate.  Rows whose slot
-// is past `n` are zero-filled.
+// is past `n`, or whose key is outside [0, N), are zero-filled.
 template <int D>
 __device__ __forceinline__ void issue_chunk(uint32_t buf, const __nv_bfloat16* k,
-                                            const __nv_bfloat16* v, int Hkv, int g,
+                                            const __nv_bfloat16* v, int N, int Hkv, int g,
                                             const int32_t* srow, int t_base, int n, int tid,
                                             int nthr) {
     constexpr int RB = D * 2;
@@ -103,8 +103,9 @@ __device__ __forceinline__ void issue_chunk(uint32_t buf, const __nv_bfloat16* k
         const int mat = p / PIECES;          // 0 = K, 1 = V
         const int r = (p % PIECES) / PC, pc = p % PC;
         const int t = t_base + r;
-        const bool valid = t < n;
-        const int j = valid ? srow[t] : 0;
+        const int jr = t < n ? srow[t] : -1;
+        const bool valid = (unsigned)jr < (unsigned)N;    // keys outside [0, N) are never read
+        const int j = valid ? jr : 0;
         const __nv_bfloat16* src = (mat == 0 ? k : v) + ((size_t)j * Hkv + g) * D + pc * 8;
         cp_async16(buf + mat * kChunk * RB + swz<RB>(r, pc), src, valid);
     }
@@ -112,28 +113,36 @@ __device__ __forceinline__ void issue_chunk(uint32_t buf, const __nv_bfloat16* k
 
 // Warp version of issue_chunk: the chunk's kChunk support indices are read once
 // (one lane each) and broadcast; every lane keeps one 16-byte column `pc` of the
-// rows and issues the K and V copies of each of its rows from one row offset.
+// rows and issues the K and V copies of each of its rows from one row offset.  Keys
+// outside [0, jmax] (jmax = the query's position: negative, later or past the sequence)
+// are not read; their rows are zero-filled.  Returns the chunk's valid slots as bits.
 template <int D>
-__device__ __forceinline__ void issue_chunk_warp(uint32_t buf, const __nv_bfloat16* k,
-                                                 const __nv_bfloat16* v, int Hkv, int g,
-                                                 const int32_t* srow, int t_base, int n) {
+__device__ __forceinline__ uint32_t issue_chunk_warp(uint32_t buf, const __nv_bfloat16* k,
+                                                     const __nv_bfloat16* v, int Hkv, int g,
+                                                     const int32_t* srow, int t_base, int n,
+                                                     int jmax, int tok0) {
     constexpr int RB = D * 2;
     constexpr int PC = RB / 16;          // 16-byte pieces per row
     constexpr int RPP = 32 / PC;         // rows covered by one pass of the warp
     const int lane = threadIdx.x & 31;
     const int pc = lane % PC, r0 = lane / PC;
     int jl = -1;
-    if (lane < kChunk && t_base + lane < n) jl = srow[t_base + lane];
+    if (lane < kChunk && t_base + lane < n) {
+        const int j = srow[t_base + lane];
+        jl = (unsigned)j <= (unsigned)jmax ? j : -1;
+    }
+    const uint32_t bits = __ballot_sync(0xffffffffu, jl >= 0);
 #pragma unroll
     for (int u = 0; u < kChunk / RPP; ++u) {
         const int r = u * RPP + r0;
         const int j = __shfl_sync(0xffffffffu, jl, r);
         const bool valid = j >= 0;
-        const size_t off = valid ? ((size_t)j * Hkv + g) * D + pc * 8 : 0;
+        const size_t off = valid ? ((size_t)(tok0 + j) * Hkv + g) * D + pc * 8 : 0;
         const uint32_t dst = buf + swz<RB>(r, pc);
         cp_async16(dst, k + off, valid);
         cp_async16(dst + kChunk * RB, v + off, valid);
     }
+    return bits;
 }
 
 // One chunk of keys for one 16-row MMA tile: S = Q K^T (2 n-tiles of 8 keys),
@@ -173,14 +182,17 @@ __device__ __forceinline__ void chunk_step(uint32_t kbuf, const uint32_t (&qa)[D
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
         const float m_new = fmaxf(m[hf], mx);
         const float base = (m_new == -INFINITY) ? 0.f : m_new;
-        const float corr = ex2f(m[hf] - base);
-        m[hf] = m_new;
-        l[hf] *= corr;
+        // rescale only when some row of the warp raised its max (else every factor is 1)
+        if (__any_sync(0xffffffffu, m_new != m[hf])) {
+            const float corr = ex2f(m[hf] - base);
+            l[hf] *= corr;
 #pragma unroll
-        for (int nd = 0; nd < D / 8; ++nd) {
-            o[nd][2 * hf] *= corr;
-            o[nd][2 * hf + 1] *= corr;
+            for (int nd = 0; nd < D / 8; ++nd) {
+                o[nd][2 * hf] *= corr;
+                o[nd][2 * hf + 1] *= corr;
+            }
         }
+        m[hf] = m_new;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -256,6 +268,13 @@ __device__ __forceinline__ void write_rows(const float (&m)[2], float (&l)[2],
     }
 }
 
+// Key of slot t of a support row for the causal mask: the index when it is a key of the
+// sequence, else INT32_MAX (never <= a query: the slot is skipped).
+__device__ __forceinline__ int slot_key(const int32_t* row, int t, int n, int N) {
+    const int j = t < n ? row[t] : -1;
+    return (unsigned)j < (unsigned)N ? j : INT32_MAX;
+}
+
 // Number of leading entries of an ascending support row that are <= limit.
 __device__ __forceinline__ int count_le(const int32_t* row, int n, int limit) {
     int lo = 0, hi = n;
@@ -292,20 +311,17 @@ k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         const int64_t per_half = (int64_t)rows * gh;
         const int64_t rem = item % per_half;
         const int i = seqs.cu[0] + (int)(rem / gh), g = (int)(item / per_half) * gh + (int)(rem % gh);
-        // the query's sequence: its first token and length (keys are positions within it)
-        int tok0 = seqs.cu[0], N = rows;
+        // the query's sequence sq: keys are positions within it, from token tok0 on
+        int sq = 0;
         if (seqs.n_seq > 1) {
-            int lo = 0, hi = seqs.n_seq - 1;          // the last s with cu[s] <= i
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (seqs.cu[mid] <= i) lo = mid;
+            int hi = seqs.n_seq - 1;                  // the last s with cu[s] <= i
+            while (sq < hi) {
+                const int mid = (sq + hi + 1) >> 1;
+                if (seqs.cu[mid] <= i) sq = mid;
                 else hi = mid - 1;
             }
-            tok0 = seqs.cu[lo];
-            N = seqs.cu[lo + 1] - tok0;
         }
-        const __nv_bfloat16* ks = k + (size_t)tok0 * Hkv * D;
-        const __nv_bfloat16* vs = v + (size_t)tok0 * Hkv * D;
+        const int tok0 = seqs.cu[sq];
         const int32_t* srow;
         int n;
         if (block_q == 1) {
@@ -324,30 +340,32 @@ k_attn_gather(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         float o[D / 8][4];
 #pragma unroll
         for (int nd = 0; nd < D / 8; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+        static_assert(STAGES == 2, "one chunk in flight beside the one computed");
         const int nch = (n + kChunk - 1) / kChunk;
-#pragma unroll
-        for (int s = 0; s < STAGES - 1; ++s) {
-            if (s < nch) issue_chunk_warp<D>(wbuf + s * STAGE, ks, vs, Hkv, g, srow, s * kChunk, n);
-            cp_async_commit();
-        }
+        const int jmax = i - tok0;                    // keys after the query are skipped
+        uint32_t bits = 0;                            // valid slots of the chunk computed next
+        if (nch > 0) bits = issue_chunk_warp<D>(wbuf, k, v, Hkv, g, srow, 0, n, jmax, tok0);
+        cp_async_commit();
         for (int ch = 0; ch < nch; ++ch) {
-            const int nx = ch + STAGES - 1;
-            if (nx < nch)
-                issue_chunk_warp<D>(wbuf + (nx % STAGES) * STAGE, ks, vs, Hkv, g, srow, nx * kChunk, n);
+            uint32_t next = 0;
+            if (ch + 1 < nch)
+                next = issue_chunk_warp<D>(wbuf + ((ch + 1) & 1) * STAGE, k, v, Hkv, g, srow,
+                                           (ch + 1) * kChunk, n, jmax, tok0);
             cp_async_commit();
-            cp_async_wait<STAGES - 1>();
+            cp_async_wait<1>();
             __syncwarp();
-            const int tb = ch * kChunk;
-            chunk_step<D, ROW8>(wbuf + (ch % STAGES) * STAGE, qa, sl2, m, l, o,
-                                [&](int r, int) { return tb + r < n; });
+            chunk_step<D, ROW8>(wbuf + (ch & 1) * STAGE, qa, sl2, m, l, o,
+                                [&](int r, int) { return (bits >> r) & 1u; });
             __syncwarp();
+            bits = next;
         }
         cp_async_wait<0>();
         write_rows<D>(m, l, o, [&](int row, __nv_bfloat16*& dst, float*& ld) {
             if (row >= G) return false;
             const int h = g * G + row;
             dst = out + ((size_t)i * Hq + h) * D;
-            ld = lse ? lse + (size_t)Hq * tok0 + (size_t)h * N + (i - tok0) : nullptr;
+            const int len = seqs.cu[sq + 1] - tok0;
+            ld = lse ? lse + (size_t)Hq * tok0 + (size_t)h * len + (i - tok0) : nullptr;
             return true;
         });
     }
@@ -396,20 +414,18 @@ k_attn_block(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restric
 #pragma unroll
     for (int s = 0; s < STAGES - 1; ++s) {
         if (s < nch) {
-            issue_chunk<D>(buf0 + s * STAGE, k, v, Hkv, g, srow, s * kChunk, n, threadIdx.x, 512);
-            if (threadIdx.x < kChunk)
-                s_idx[s][threadIdx.x] = (s * kChunk + (int)threadIdx.x < n) ? srow[s * kChunk + threadIdx.x] : INT32_MAX;
+            issue_chunk<D>(buf0 + s * STAGE, k, v, N, Hkv, g, srow, s * kChunk, n, threadIdx.x, 512);
+            if (threadIdx.x < kChunk) s_idx[s][threadIdx.x] = slot_key(srow, s * kChunk + (int)threadIdx.x, n, N);
         }
         cp_async_commit();
     }
     for (int ch = 0; ch < nch; ++ch) {
         const int nx = ch + STAGES - 1;
         if (nx < nch) {
-            issue_chunk<D>(buf0 + (nx % STAGES) * STAGE, k, v, Hkv, g, srow, nx * kChunk, n,
+            issue_chunk<D>(buf0 + (nx % STAGES) * STAGE, k, v, N, Hkv, g, srow, nx * kChunk, n,
                            threadIdx.x, 512);
             if (threadIdx.x < kChunk)
-                s_idx[nx % STAGES][threadIdx.x] =
-                    (nx * kChunk + (int)threadIdx.x < n) ? srow[nx * kChunk + threadIdx.x] : INT32_MAX;
+                s_idx[nx % STAGES][threadIdx.x] = slot_key(srow, nx * kChunk + (int)threadIdx.x, n, N);
         }
         cp_async_commit();
         cp_async_wait<STAGES - 1>();

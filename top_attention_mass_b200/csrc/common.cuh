@@ -34,6 +34,27 @@ __device__ __forceinline__ void report_error(int32_t* status, int32_t code, int3
     }
 }
 
+// ---------------------------------------------------------------- debug-checks build
+// Built with -DTAM_DEBUG_CHECKS (libtam_debug.so), the pass-2 kernels check the index
+// of every slab row, candidate and block-mass store against the extent the host gave
+// the launch (MassArgs::out_cap) and, instead of an out-of-range store, record
+// TAM_ERR_OVERFLOW (detail: the site, the index and the extent, truncated to 32 bits)
+// and skip it.  The release build compiles the checks away.
+#ifdef TAM_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+enum DebugSite : int32_t { kSiteRows = 1, kSiteCand = 2, kSiteBlockMass = 3 };
+
+__device__ __forceinline__ bool in_bounds(int32_t* status, int32_t kid, int32_t site, uint64_t idx,
+                                          uint64_t extent) {
+    if constexpr (!kDebugChecks) return true;
+    if (idx < extent) return true;
+    report_error(status, TAM_ERR_OVERFLOW, kid, site, (int32_t)idx, (int32_t)extent);
+    return false;
+}
+
 // ---------------------------------------------------------------- element loads
 template <typename T> __device__ __forceinline__ float to_f(T x);
 template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }

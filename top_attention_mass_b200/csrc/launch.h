@@ -119,6 +119,9 @@ struct MassArgs {
     int32_t* sup_len;
     float* sup_mass;
     int32_t* status;
+    // entries of rows (floats), cand (pairs) or bmass (u64) the launch may write: checked
+    // by the debug-checks build only
+    uint64_t out_cap = ~uint64_t(0);
 };
 
 struct AttnArgs {
@@ -157,6 +160,7 @@ struct IndexerArgs {
     int32_t* sup_len;
     float* sup_score;
     int32_t* status;
+    uint64_t out_cap = ~uint64_t(0);   // as MassArgs::out_cap
 };
 
 // Counts one kernel launch (read back by tam_kernel_launches).

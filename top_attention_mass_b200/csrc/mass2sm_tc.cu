@@ -38,6 +38,7 @@
 // Every wait is bounded; the pair shakes hands before it frees TMEM and exits so
 // that no remote arrive or MMA of one CTA can land after the other left.
 #include "launch.h"
+#include "mass_exp.cuh"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
 
@@ -68,6 +69,7 @@ struct PairParams {
     int N, Hq, Hkv, pair0, n_pairs, block_q;
     int64_t row0, row1;       // per query: the rows [row0, row1) of this launch
     int kst;                  // rows mode: key m of the K map sits at position m * kst
+    uint64_t out_cap;         // entries of rows / cand / bmass (debug-checks build)
     int seg_cap;              // stream mode: entries per candidate segment
     float sl2, inv_hq;
     const float* lse;
@@ -80,6 +82,13 @@ struct PairParams {
     uint64_t timeout_ns;
     int dbg;
 };
+
+// Adds a block-mass column sum in 2^-40 fixed point (one 64-bit atomic per (block, key)
+// and warp part).
+__device__ __forceinline__ void block_mass_add(const PairParams& p, int64_t at, float sum) {
+    if (in_bounds(p.status, KID_BLOCK_MASS_TC, kSiteBlockMass, (uint64_t)at, p.out_cap))
+        atomicAdd(&p.bmass[at], (unsigned long long)__float2ll_rn(sum * p.inv_hq * 1099511627776.0f));
+}
 
 __host__ __device__ __forceinline__ int64_t bmass_row(int64_t b, int block_q) {
     return (int64_t)block_q * b * (b + 1) / 2;
@@ -156,7 +165,7 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     for (int t = threadIdx.x; t < Hkv * kNQ; t += blockDim.x) {
         const int g = t / kNQ, c = t % kNQ;
         const int i = q0 + c / G, h = g * G + c % G;
-        sLse[t] = (i < p.N) ? p.lse[(size_t)h * p.N + i] * kLog2e : INFINITY;
+        sLse[t] = (i < p.N) ? -p.lse[(size_t)h * p.N + i] * kLog2e : -INFINITY;   // negated
     }
     if constexpr (STREAM) {
         for (int c = threadIdx.x; c < BQP; c += blockDim.x) {
@@ -261,10 +270,10 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         for (int q = 0; q < (STREAM ? kQP : 1); ++q) cnt[q] = 0;
         bool ok = true;
         if (p.dbg & kDebugForceTimeout) ok = tc::wait(never, 0, gd, 9);
+        const uint64_t sl2x2 = tc::f2_pack(p.sl2, p.sl2);
         for (int kt = 0; ok && kt < n_kt; ++kt) {
-            float acc[kQP];
-#pragma unroll
-            for (int q = 0; q < kQP; ++q) acc[q] = 0.f;
+            MassAcc<G, kQP> acc2;
+            acc2.clear();
             for (int g = 0; g < Hkv; ++g) {
                 const int u = kt * Hkv + g;
                 const int slot = u % kR;
@@ -279,19 +288,14 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     uint32_t (&cur)[32] = (c & 1) ? vb : va;
                     uint32_t (&nxt)[32] = (c & 1) ? va : vb;
                     if (c + 1 < kCols / 32) tc::tmem_ld32(col0 + (c + 1) * 32, nxt);
-                    const float4* l4 =
-                        reinterpret_cast<const float4*>(sLse + g * kNQ + part * kCols + c * 32);
+                    const ulonglong2* nl =
+                        reinterpret_cast<const ulonglong2*>(sLse + g * kNQ + part * kCols + c * 32);
 #pragma unroll
                     for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 L = l4[c4];
-                        const float Ls[4] = {L.x, L.y, L.z, L.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int col = c * 32 + c4 * 4 + e;
-                            // one exponential in four on the FMA pipe, the rest on MUFU
-                            const float x = fmaf(__uint_as_float(cur[c4 * 4 + e]), p.sl2, -Ls[e]);
-                            acc[col / G] += e == 3 ? tc::ex2_fma(x) : tc::ex2(x);
-                        }
+                        const ulonglong2 L = nl[c4];
+                        mass_columns4<G, kQP>(acc2, c * 32 + c4 * 4, cur[c4 * 4], cur[c4 * 4 + 1],
+                                              cur[c4 * 4 + 2], cur[c4 * 4 + 3], L.x, L.y, sl2x2,
+                                              (c4 & 1) != 0);
                     }
                     if (c + 1 < kCols / 32) tc::tmem_wait_ld(nxt);
                 }
@@ -303,6 +307,9 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 }
             }
             if (!ok) break;
+            float acc[kQP];
+#pragma unroll
+            for (int q = 0; q < kQP; ++q) acc[q] = acc2.get(q);
             const int m = kt * kTileKeys + (int)rank * 128 + row;   // key (or sample) index
             if constexpr (MODE == kModeRows) {
                 // row i of the slab starts off(i) - off(row0) floats in (32-bit: the host
@@ -315,7 +322,9 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                                           (int64_t)a * b - slab0);
 #pragma unroll
                 for (int ql = 0; ql < kQP; ++ql) {
-                    if (m <= a && qbase + ql < p.row1) p.rows[off + (uint32_t)m] = acc[ql] * p.inv_hq;
+                    if (m <= a && qbase + ql < p.row1 &&
+                        in_bounds(p.status, KID_MASS_TC, kSiteRows, off + (uint32_t)m, p.out_cap))
+                        p.rows[off + (uint32_t)m] = acc[ql] * p.inv_hq;
                     off += (uint32_t)a + 1u;
                     if (++b == p.kst) { b = 0; ++a; }
                 }
@@ -332,9 +341,9 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                                       v >= sTau[part * kQP + ql];
                     const uint32_t bal = __ballot_sync(0xffffffffu, pass);
                     const int pos = cnt[ql] + __popc(bal & lt);
-                    if (pass && pos < p.seg_cap)
-                        p.cand[off0 + (uint32_t)ql * qstride + (uint32_t)pos] =
-                            make_uint2(__float_as_uint(v), (uint32_t)m);
+                    const uint32_t at = off0 + (uint32_t)ql * qstride + (uint32_t)pos;
+                    if (pass && pos < p.seg_cap && in_bounds(p.status, KID_MASS_TC, kSiteCand, at, p.out_cap))
+                        p.cand[at] = make_uint2(__float_as_uint(v), (uint32_t)m);
                     cnt[ql] += __popc(bal);
                 }
             } else {
@@ -349,17 +358,14 @@ k_mass_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                         const int b = i / p.block_q;
                         if (b != cur_b) {
                             if (sum > 0.f)
-                                atomicAdd(&p.bmass[bmass_row(cur_b, p.block_q) + j],
-                                          (unsigned long long)__float2ll_rn(sum * p.inv_hq * 1099511627776.0f));
+                                block_mass_add(p, bmass_row(cur_b, p.block_q) + j, sum);
                             sum = 0.f;
                             cur_b = b;
                         }
                         if (j <= i) sum += acc[q];
                     }
                 }
-                if (sum > 0.f)
-                    atomicAdd(&p.bmass[bmass_row(cur_b, p.block_q) + j],
-                              (unsigned long long)__float2ll_rn(sum * p.inv_hq * 1099511627776.0f));
+                if (sum > 0.f) block_mass_add(p, bmass_row(cur_b, p.block_q) + j, sum);
             }
         }
         if constexpr (STREAM) {
@@ -423,6 +429,7 @@ cudaError_t launch_pair(const MassArgs& a, cudaStream_t st) {
     p.cnt = a.cnt;
     p.bmass = reinterpret_cast<unsigned long long*>(a.bmass);
     p.status = a.status;
+    p.out_cap = a.out_cap;
     p.timeout_ns = wait_timeout_ns();
     p.dbg = debug_flags();
     if (p.n_pairs <= 0) return cudaSuccess;

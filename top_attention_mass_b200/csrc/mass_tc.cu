@@ -33,6 +33,7 @@
 //               writer, so it stays in key order), or the block column sum is added
 //               in 2^-40 fixed point (block-shared).
 #include "launch.h"
+#include "mass_exp.cuh"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
 
@@ -62,6 +63,7 @@ struct MassParams {
     int N, Hq, Hkv, ct0, n_ctiles, block_q;
     int64_t row0, row1;              // per query / indexer: the rows [row0, row1)
     int kst;                         // rows modes: key m of the K map is at m * kst
+    uint64_t out_cap;                // entries of rows / cand / bmass (debug-checks build)
     int seg_cap;                     // stream modes: entries per candidate segment
     float sl2, inv_hq;
     const float* lse;
@@ -78,6 +80,12 @@ struct MassParams {
 // Offset of block b's row in the triangular block-mass buffer.
 __host__ __device__ __forceinline__ int64_t bmass_offset(int64_t b, int block_q) {
     return (int64_t)block_q * b * (b + 1) / 2;
+}
+
+// Adds a block-mass column sum in 2^-40 fixed point.
+__device__ __forceinline__ void block_mass_add(const MassParams& p, int64_t at, float sum) {
+    if (in_bounds(p.status, KID_BLOCK_MASS_TC, kSiteBlockMass, (uint64_t)at, p.out_cap))
+        atomicAdd(&p.bmass[at], (unsigned long long)__float2ll_rn(sum * p.inv_hq * 1099511627776.0f));
 }
 
 template <int G, int D, int NQ, int MODE, int kStages>
@@ -141,7 +149,7 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         for (int t = threadIdx.x; t < Hkv * NQ; t += blockDim.x) {
             const int g = t / NQ, c = t % NQ;
             const int i = q0 + c / G, h = g * G + c % G;
-            sLse[t] = (i < p.N) ? p.lse[(size_t)h * p.N + i] * kLog2e : INFINITY;
+            sLse[t] = (i < p.N) ? -p.lse[(size_t)h * p.N + i] * kLog2e : -INFINITY;   // negated
         }
     }
     if constexpr (STREAM) {
@@ -243,10 +251,11 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         for (int q = 0; q < (STREAM ? kQP : 1); ++q) cnt[q] = 0;
         bool ok = true;
         if (p.dbg & kDebugForceTimeout) ok = tc::wait(never, 0, gd, 9);
+        const uint64_t sl2x2 = tc::f2_pack(p.sl2, p.sl2);
         for (int kt = 0; ok && kt < n_kt; ++kt) {
             float acc[kQP];
-#pragma unroll
-            for (int q = 0; q < kQP; ++q) acc[q] = 0.f;
+            MassAcc<G, kQP> acc2;
+            acc2.clear();
             for (int g = 0; g < Hkv; ++g) {
                 const int u = kt * Hkv + g;
                 const int slot = u % R;
@@ -271,20 +280,15 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
                         for (int e = 0; e < CW; ++e) acc[c * CW + e] = __uint_as_float(cur[e]);
                     } else {
-                        const float4* l4 = reinterpret_cast<const float4*>(
+                        const ulonglong2* nl = reinterpret_cast<const ulonglong2*>(
                             sLse + g * NQ + part * kCols + c * CW);
 #pragma unroll
                         for (int c4 = 0; c4 < CW / 4; ++c4) {
-                            const float4 L = l4[c4];
-                            const float Ls[4] = {L.x, L.y, L.z, L.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int col = c * CW + c4 * 4 + e;
-                                const float sc = __uint_as_float(cur[c4 * 4 + e]);
-                                // one exponential in four on the FMA pipe, the rest on MUFU
-                                const float x = fmaf(sc, p.sl2, -Ls[e]);
-                                acc[col / G] += e == 3 ? tc::ex2_fma(x) : tc::ex2(x);
-                            }
+                            const ulonglong2 L = nl[c4];
+                            mass_columns4<G, kQP>(acc2, c * CW + c4 * 4, cur[c4 * 4],
+                                                  cur[c4 * 4 + 1], cur[c4 * 4 + 2],
+                                                  cur[c4 * 4 + 3], L.x, L.y, sl2x2,
+                                                  (c4 & 1) != 0);
                         }
                     }
                     if (c + 1 < kCols / CW) tc::tmem_wait_ld(nxt);
@@ -293,6 +297,10 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 tc::mbar_arrive(&s_empty[slot]);
             }
             if (!ok) break;
+            if constexpr (!INDEXER) {
+#pragma unroll
+                for (int q = 0; q < kQP; ++q) acc[q] = acc2.get(q);
+            }
             const int j = kt * 128 + row;                     // key (or sample) index
             const int qp0 = q0 + part * kQP;                  // first query of this part
             if constexpr (STREAM) {
@@ -309,9 +317,11 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                                       v >= sTau[part * kQP + q];
                     const uint32_t bal = __ballot_sync(0xffffffffu, pass);
                     const int pos = cnt[q] + __popc(bal & lt);
-                    if (pass && pos < p.seg_cap)
-                        p.cand[off0 + (uint32_t)q * qstride + (uint32_t)pos] =
-                            make_uint2(__float_as_uint(v), (uint32_t)j);
+                    const uint32_t at = off0 + (uint32_t)q * qstride + (uint32_t)pos;
+                    if (pass && pos < p.seg_cap &&
+                        in_bounds(p.status, INDEXER ? KID_INDEXER_TC : KID_MASS_TC, kSiteCand, at,
+                                  p.out_cap))
+                        p.cand[at] = make_uint2(__float_as_uint(v), (uint32_t)j);
                     cnt[q] += __popc(bal);
                 }
             } else if constexpr (!BLOCK) {
@@ -325,7 +335,8 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                                           (int64_t)a * b - slab0);
 #pragma unroll
                 for (int q = 0; q < kQP; ++q) {
-                    if (j <= a && qbase + q < p.row1)
+                    if (j <= a && qbase + q < p.row1 &&
+                        in_bounds(p.status, KID_MASS_TC, kSiteRows, off + (uint32_t)j, p.out_cap))
                         p.rows[off + (uint32_t)j] = INDEXER ? acc[q] : acc[q] * p.inv_hq;
                     off += (uint32_t)a + 1u;
                     if (++b == p.kst) { b = 0; ++a; }
@@ -342,18 +353,14 @@ k_mass_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                         const int b = i / p.block_q;
                         if (b != cur_b) {
                             if (sum > 0.f)
-                                atomicAdd(&p.bmass[bmass_offset(cur_b, p.block_q) + j],
-                                          (unsigned long long)__float2ll_rn(
-                                              sum * p.inv_hq * 1099511627776.0f));
+                                block_mass_add(p, bmass_offset(cur_b, p.block_q) + j, sum);
                             sum = 0.f;
                             cur_b = b;
                         }
                         if (j <= i) sum += acc[q];
                     }
                 }
-                if (sum > 0.f)
-                    atomicAdd(&p.bmass[bmass_offset(cur_b, p.block_q) + j],
-                              (unsigned long long)__float2ll_rn(sum * p.inv_hq * 1099511627776.0f));
+                if (sum > 0.f) block_mass_add(p, bmass_offset(cur_b, p.block_q) + j, sum);
             }
         }
         if constexpr (STREAM) {
@@ -491,6 +498,7 @@ cudaError_t launch_mass(const MassArgs& a, cudaStream_t st) {
     p.cnt = a.cnt;
     p.bmass = reinterpret_cast<unsigned long long*>(a.bmass);
     p.status = a.status;
+    p.out_cap = a.out_cap;
     p.timeout_ns = wait_timeout_ns();
     p.dbg = debug_flags();
     if (p.n_ctiles <= 0) return cudaSuccess;
@@ -642,6 +650,7 @@ cudaError_t tc_indexer_rows(const IndexerArgs& ia, cudaStream_t st) {
     a.cand = ia.cand;
     a.cnt = ia.cnt;
     a.seg_cap = ia.seg_cap;
+    a.out_cap = ia.out_cap;
     a.status = ia.status;
     return launch_indexer_tc(a, st);
 }

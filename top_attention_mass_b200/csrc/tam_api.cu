@@ -316,6 +316,7 @@ int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void*
     ma.sup_idx = sup_idx; ma.sup_len = sup_len; ma.sup_mass = sup_mass;
     ma.status = (int32_t*)ws;
     if (!plan.tc) return cuda_status(simt_mass_select(ma, st));
+    ma.out_cap = debug_extent((ws_bytes - plan.off_work) / 8);   // block mass (u64)
     if (!plan.stream) return cuda_status(tc_mass_pass(ma, st));
     const StreamPlan& sp = plan.sp;
     char* region = ws + sp.off_region;
@@ -325,6 +326,7 @@ int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void*
         const int64_t cap = std::min<int64_t>((int64_t)(region_bytes / sizeof(float)),
                                               (int64_t(1) << 32) - 1);   // 32-bit row offsets
         ma.rows = (float*)region;
+        ma.out_cap = debug_extent((uint64_t)cap);
         for (int64_t r0 = 0; r0 < N;) {
             const int64_t r1 = chunk_end(r0, N, cap);
             ma.row0 = r0;
@@ -340,11 +342,13 @@ int launch_mass_select(int64_t N, int Hq, int Hkv, int d, int dtype, const void*
     auto sample = [&](int64_t r0, int64_t r1, int S, float* slab) {
         MassArgs a = ma;
         a.row0 = r0; a.row1 = r1; a.kst = S; a.rows = slab;
+        a.out_cap = debug_extent(region_bytes / 4);
         return tc_mass_pass(a, st);
     };
     auto scan = [&](int64_t c0, int64_t c1, const float* tau, void* cand, int32_t* cnt) {
         MassArgs a = ma;
         a.row0 = c0; a.row1 = c1; a.stream = true; a.tau = tau; a.cand = cand; a.cnt = cnt;
+        a.out_cap = debug_extent(region_bytes / 8);
         a.seg_cap = sp.seg_cap;
         return tc_mass_pass(a, st);
     };
@@ -482,6 +486,7 @@ int run_indexer(int64_t N, int d_idx, int dtype, const void* q_idx, const void* 
         const int64_t cap = std::min<int64_t>((int64_t)(region_bytes / sizeof(float)),
                                               (int64_t(1) << 32) - 1);   // 32-bit row offsets
         ia.rows = (float*)region;
+        ia.out_cap = debug_extent((uint64_t)cap);
         for (int64_t r0 = 0; r0 < N;) {
             const int64_t r1 = chunk_end(r0, N, cap);
             ia.row0 = r0;
@@ -497,11 +502,13 @@ int run_indexer(int64_t N, int d_idx, int dtype, const void* q_idx, const void* 
     auto sample = [&](int64_t r0, int64_t r1, int S, float* slab) {
         IndexerArgs a = ia;
         a.row0 = r0; a.row1 = r1; a.kst = S; a.rows = slab;
+        a.out_cap = debug_extent(region_bytes / 4);
         return tc_indexer_rows(a, st);
     };
     auto scan = [&](int64_t c0, int64_t c1, const float* tau, void* cand, int32_t* cnt) {
         IndexerArgs a = ia;
         a.row0 = c0; a.row1 = c1; a.stream = true; a.tau = tau; a.cand = cand; a.cnt = cnt;
+        a.out_cap = debug_extent(region_bytes / 8);
         a.seg_cap = sp.seg_cap;
         return tc_indexer_rows(a, st);
     };

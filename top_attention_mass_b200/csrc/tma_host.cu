@@ -70,6 +70,10 @@ int debug_force_fallback() {
     return (v == 1 || v == 2) ? v : 0;
 }
 
+uint64_t debug_extent(uint64_t cap) {
+    return env_int("TAM_DEBUG_SHRINK_EXTENTS", 0) ? (cap < 64 ? cap : 64) : cap;
+}
+
 int debug_flags() { return env_int("TAM_DEBUG_FORCE_TIMEOUT", 0) ? kDebugForceTimeout : 0; }
 
 }  // namespace tam

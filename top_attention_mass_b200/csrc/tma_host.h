@@ -39,5 +39,9 @@ bool dense_pair_tiles_selected();
 // key) sends every row the streamed selection would sample to the fallback path, so
 // that path can be tested on ordinary inputs.
 int debug_force_fallback();
+// Extent handed to a launch for its debug-checks: `cap`, or at most 64 entries when
+// TAM_DEBUG_SHRINK_EXTENTS is set (so that the checks of the debug-checks build fire
+// while every store still lands inside the real buffer, which they then skip).
+uint64_t debug_extent(uint64_t cap);
 
 }  // namespace tam
