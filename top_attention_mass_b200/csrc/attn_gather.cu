@@ -460,7 +460,7 @@ cudaError_t launch_gather(const AttnArgs& a, cudaStream_t st) {
     int dev;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return with_table(a.N, a.seqs, [&](const SeqTable& t) {
+    return with_table(a.N, a.seqs, [&](SeqTable& t) {
         if (t.cu[t.n_seq] == t.cu[0]) return cudaSuccess;
         kern<<<sms, 32 * W, smem, st>>>((const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k,
                                      (const __nv_bfloat16*)a.v, t, a.Hq, a.Hkv, a.sl2, a.sup_idx,

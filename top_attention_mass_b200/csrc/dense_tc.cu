@@ -336,7 +336,7 @@ cudaError_t launch_dense(const AttnArgs& a, cudaStream_t st) {
     auto kern = k_dense_tc<G, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    return with_table(a.N, a.seqs, [&](const SeqTable& t) {
+    return with_table(a.N, a.seqs, [&](SeqTable& t) {
         const int n_tiles = seq_table_tiles(t, BQ);
         if (n_tiles == 0) return cudaSuccess;
         kern<<<(unsigned)(n_tiles * a.Hkv), kThreads, smem, st>>>(

@@ -10,77 +10,72 @@ namespace tam {
 // Packed batches in one launch: sequence s of the table owns the tokens
 // [cu[s], cu[s+1]) of the packed q/k/v rows (a single-sequence call is the table
 // {1, N, {0, N}}).  The kernels that take a table number their query tiles of BQ rows
-// over all of its sequences, heaviest first: every tile with local index L (rows
-// [L BQ, (L+1) BQ) of its sequence) comes before every tile with a smaller L, and
-// within one L the sequences go in order.  Larger batches run as several tables.
+// sequence by sequence, longest sequence first (`order`), each sequence's tiles
+// heaviest (last) first, so that the machine works through the long sequences while
+// the short ones fill the tail, and the CTAs in flight share one or two sequences' K/V
+// in L2.  Larger batches run as several tables.
 constexpr int kMaxSeqPerLaunch = 128;
 struct SeqTable {
     int n_seq;
-    int max_len;                      // longest sequence of the table
-    int cu[kMaxSeqPerLaunch + 1];     // absolute token offsets, non-decreasing
+    int max_len;                        // longest sequence of the table
+    int cu[kMaxSeqPerLaunch + 1];       // absolute token offsets, non-decreasing
+    int order[kMaxSeqPerLaunch];        // sequences by length, longest first
+    int tile0[kMaxSeqPerLaunch + 1];    // first tile of order[r] (set per launch for its BQ)
 };
 
-inline int seq_table_tiles(const SeqTable& t, int BQ) {
-    int n = 0;
-    for (int s = 0; s < t.n_seq; ++s) n += (t.cu[s + 1] - t.cu[s] + BQ - 1) / BQ;
-    return n;
+// Sorts the table's sequences by length (longest first, ties in order).
+inline void seq_table_order(SeqTable& t) {
+    for (int s = 0; s < t.n_seq; ++s) t.order[s] = s;
+    for (int a = 1; a < t.n_seq; ++a) {            // insertion sort: at most 128 entries
+        const int s = t.order[a], n = t.cu[s + 1] - t.cu[s];
+        int b = a;
+        for (; b > 0 && t.cu[t.order[b - 1] + 1] - t.cu[t.order[b - 1]] < n; --b)
+            t.order[b] = t.order[b - 1];
+        t.order[b] = s;
+    }
 }
 
-// Runs fn on the launch's table: *seqs, or the single sequence [0, N) when seqs is null.
+// Fills tile0 for tiles of BQ rows; returns the table's tile count.
+inline int seq_table_tiles(SeqTable& t, int BQ) {
+    t.tile0[0] = 0;
+    for (int r = 0; r < t.n_seq; ++r) {
+        const int s = t.order[r];
+        t.tile0[r + 1] = t.tile0[r] + (t.cu[s + 1] - t.cu[s] + BQ - 1) / BQ;
+    }
+    return t.tile0[t.n_seq];
+}
+
+// Runs fn on a copy of the launch's table: *seqs, or the single sequence [0, N) when
+// seqs is null (the copy is the launch's own, so it may fill tile0).
 template <class F>
 cudaError_t with_table(int64_t N, const SeqTable* seqs, F&& fn) {
-    if (seqs) return fn(*seqs);
     SeqTable t{};
-    t.n_seq = 1;
-    t.max_len = (int)N;
-    t.cu[0] = 0;
-    t.cu[1] = (int)N;
+    if (seqs) {
+        t = *seqs;
+    } else {
+        t.n_seq = 1;
+        t.max_len = (int)N;
+        t.cu[0] = 0;
+        t.cu[1] = (int)N;
+        t.order[0] = 0;
+    }
     return fn(t);
 }
 
 #ifdef __CUDACC__
-// (sequence, local tile) of the b-th tile of the table in the order above.  Every lane
-// of the calling warp must take part; all of them get the same answer.
+// (sequence, local tile) of the b-th tile of the table in the order above; any thread
+// may call it.
 template <int BQ>
 __device__ __forceinline__ void seq_tile(const SeqTable& t, int b, int& s_out, int& L_out) {
-    if (t.n_seq == 1) {
-        s_out = 0;
-        L_out = (t.cu[1] - t.cu[0] + BQ - 1) / BQ - 1 - b;
-        return;
-    }
-    const int lane = threadIdx.x & 31;
-    // tiles whose local index is at least L
-    auto at_least = [&](int L) {
-        int c = 0;
-        for (int s = lane; s < t.n_seq; s += 32)
-            c += max(0, (t.cu[s + 1] - t.cu[s] + BQ - 1) / BQ - L);
-#pragma unroll
-        for (int o = 16; o; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-        return c;
-    };
-    // the largest L with at_least(L) > b
-    int lo = 0, hi = (t.max_len + BQ - 1) / BQ - 1;
+    int lo = 0, hi = t.n_seq - 1;                  // the last r with tile0[r] <= b
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (at_least(mid) > b) lo = mid;
+        if (t.tile0[mid] <= b) lo = mid;
         else hi = mid - 1;
     }
-    // the p-th sequence (in order) that has a tile at index lo
-    int p = b - at_least(lo + 1);
-    s_out = 0;
-    for (int s0 = 0; s0 < t.n_seq; s0 += 32) {
-        const int s = s0 + lane;
-        const bool has = s < t.n_seq && (t.cu[s + 1] - t.cu[s] + BQ - 1) / BQ > lo;
-        unsigned m = __ballot_sync(0xffffffffu, has);
-        const int c = __popc(m);
-        if (p < c) {
-            for (int q = 0; q < p; ++q) m &= m - 1;
-            s_out = s0 + __ffs(m) - 1;
-            break;
-        }
-        p -= c;
-    }
-    L_out = lo;
+    const int s = t.order[lo];
+    s_out = s;
+    L_out = (t.cu[s + 1] - t.cu[s] + BQ - 1) / BQ - 1 - (b - t.tile0[lo]);
 }
 #endif
 

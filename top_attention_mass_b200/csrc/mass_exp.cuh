@@ -8,29 +8,34 @@
 // exponentiated on the FMA pipe and the rest on MUFU.  Both kernels use it so that they
 // give the same mass bit for bit.
 //
-// Columns are (query, head) with the head fastest.  For G >= 2 heads per KV group a
-// pair holds two heads of one query and the query's packed accumulator keeps two
-// partial sums (lo, hi), added at the end (mass_acc_get); for G = 1 a pair holds two
-// queries and its accumulator their two sums.
+// Columns are (query, head) with the head fastest.  For G >= 4 heads per KV group the
+// four columns are heads of one query: the two pairs are added packed and the pair's
+// halves into the query's fp32 sum.  For G = 2 a pair holds two heads of one query and
+// the query's packed accumulator keeps two partial sums (lo, hi), added at the end; for
+// G = 1 a pair holds two queries and its accumulator their two sums.
 #pragma once
 
 #include "tc_ptx.cuh"
 
 namespace tam {
 
-// packed accumulators of kQP queries
+// head sums of kQP queries (fp32 for G >= 4, packed pairs below)
 template <int G, int kQP>
 struct MassAcc {
-    static constexpr int N = G >= 2 ? kQP : kQP / 2;
+    static constexpr int N = G >= 4 ? 1 : (G >= 2 ? kQP : kQP / 2);
     uint64_t v[N];
+    float s[G >= 4 ? kQP : 1];
     __device__ __forceinline__ void clear() {
 #pragma unroll
         for (int a = 0; a < N; ++a) v[a] = 0ull;
+#pragma unroll
+        for (int a = 0; a < (G >= 4 ? kQP : 1); ++a) s[a] = 0.f;
     }
-    // the head sum of query q
     __device__ __forceinline__ float get(int q) const {
         float lo, hi;
-        if constexpr (G >= 2) {
+        if constexpr (G >= 4) {
+            return s[q];
+        } else if constexpr (G >= 2) {
             tc::f2_unpack(v[q], lo, hi);
             return lo + hi;
         } else {
@@ -67,7 +72,9 @@ __device__ __forceinline__ void mass_columns4(MassAcc<G, kQP>& acc, int col, uin
     if constexpr (G >= 4) {
         // all four columns belong to query col / G
         const int q = col / G;
-        acc.v[q] = tc::f2_add(tc::f2_add(acc.v[q], p01), p23);
+        float lo, hi;
+        tc::f2_unpack(tc::f2_add(p01, p23), lo, hi);
+        acc.s[q] += lo + hi;
     } else {
         // G = 2: one query per pair; G = 1: two queries per pair (accumulator col / 2
         // holds columns col, col + 1 either way)

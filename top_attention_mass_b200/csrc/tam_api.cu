@@ -422,6 +422,7 @@ int for_seq_tables(int n_seq, const int64_t* cu, F&& fn) {
         for (int s = 0; s <= t.n_seq; ++s) t.cu[s] = (int)cu[s0 + s];
         for (int s = 0; s < t.n_seq; ++s) t.max_len = std::max(t.max_len, t.cu[s + 1] - t.cu[s]);
         if (t.max_len == 0) continue;
+        seq_table_order(t);
         const int rc = fn(t);
         if (rc) return rc;
     }
