@@ -30,24 +30,26 @@ assert tam.LIB_PATH.endswith("libtam_debug.so"), tam.LIB_PATH
 w = tam_synth.custom("dbg", 3000, 16, 4, 128, dtype="bf16", seed=5, sink=True, needles=3)
 inp = tam_synth.make_inputs(w)
 q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+qx, kx = q[:, 0, :64].contiguous(), k[:, 0, :64].contiguous()
+lse = tam.attention_lse(q, k)
 res = {{}}
-for name, fn in (("perquery", lambda: tam.mass_oracle_prefill(q, k, v, 40, 1, check=False)),
-                 ("block", lambda: tam.mass_oracle_prefill(q, k, v, 40, 64, check=False)),
-                 ("indexer", lambda: tam.indexer_topk(q[:, 0, :64].contiguous(),
-                                                      k[:, 0, :64].contiguous(), 50, check=False))):
+for name in ("perquery", "block", "indexer", "distill"):
     ws = tam.Workspace(q.device)
     if name == "indexer":
-        out = tam.indexer_topk(q[:, 0, :64].contiguous(), k[:, 0, :64].contiguous(), 50,
-                               workspace=ws, check=False)
+        out = tam.indexer_topk(qx, kx, 50, workspace=ws, check=False)
+        saved = {{"idx": out.idx.cpu(), "value": out.value.cpu()}}
+    elif name == "distill":
+        saved = {{"kl": tam.distill_kl(q, k, lse, qx, kx, workspace=ws, check=False).cpu()}}
     else:
         out = tam.mass_oracle_prefill(q, k, v, 40, 1 if name == "perquery" else 64,
                                       workspace=ws, check=False)
+        saved = {{"idx": out.idx.cpu(), "value": out.value.cpu()}}
     try:
         tam.check_status(ws.get(256))
         res[name] = {{"code": 0}}
     except tam.TamError as e:
         res[name] = {{"code": e.code, "detail": list(e.detail)}}
-    torch.save({{"idx": out.idx.cpu(), "value": out.value.cpu()}}, {out!r} + "_" + name + ".pt")
+    torch.save(saved, {out!r} + "_" + name + ".pt")
 print(json.dumps(res))
 """
 
@@ -71,18 +73,21 @@ def test_debug_build_planned_extents_match_release(tam_lib, tmp_path):
     w = tam_synth.custom("dbg", 3000, 16, 4, 128, dtype="bf16", seed=5, sink=True, needles=3)
     inp = tam_synth.make_inputs(w)
     q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    qx, kx = q[:, 0, :64].contiguous(), k[:, 0, :64].contiguous()
     ref = {"perquery": tam_lib.mass_oracle_prefill(q, k, v, 40, 1),
            "block": tam_lib.mass_oracle_prefill(q, k, v, 40, 64),
-           "indexer": tam_lib.indexer_topk(q[:, 0, :64].contiguous(), k[:, 0, :64].contiguous(), 50)}
+           "indexer": tam_lib.indexer_topk(qx, kx, 50)}
     for name, r in ref.items():
         got = torch.load(out + "_" + name + ".pt")
         assert torch.equal(got["idx"], r.idx.cpu()), name
         assert torch.equal(got["value"], r.value.cpu()), name
+    kl = tam_lib.distill_kl(q, k, tam_lib.attention_lse(q, k), qx, kx)
+    assert torch.equal(torch.load(out + "_distill.pt")["kl"], kl.cpu())
 
 
 def test_debug_build_flags_out_of_extent_stores(tam_lib, tmp_path):
     res, _ = _child(tmp_path, shrink=True)
-    sites = {"perquery": (1, 2), "block": (3,), "indexer": (1, 2)}
+    sites = {"perquery": (1, 2), "block": (3,), "indexer": (1, 2), "distill": (1,)}
     for name, r in res.items():
         assert r["code"] == tam_lib.TAM_ERR_OVERFLOW, (name, r)
         assert r["detail"][2] in sites[name], (name, r)       # the store site

@@ -392,17 +392,24 @@ k_attn_block_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                             if (t * kKeys + c * 32 + e > i) v[c][e] = __float_as_uint(-INFINITY);
                 }
             } else {
-                const int4* ix4 = reinterpret_cast<const int4*>(sIdx + s * kKeys);
+                // support rows are ascending: a chunk whose first and last keys lie in
+                // [0, the tile's first query] needs no mask (most chunks: the keys before
+                // the block); otherwise one unsigned compare drops both -1 and keys > i
+                const int jf = sIdx[s * kKeys], jl = sIdx[s * kKeys + kKeys - 1];
+                if (!(jf >= 0 && jl >= 0 && jl <= q0 + tt * BQ)) {
+                    const int4* ix4 = reinterpret_cast<const int4*>(sIdx + s * kKeys);
 #pragma unroll
-                for (int c = 0; c < NC; ++c)
+                    for (int c = 0; c < NC; ++c)
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const int4 jj = ix4[c * 8 + e4];
-                        const int js[4] = {jj.x, jj.y, jj.z, jj.w};
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const int4 jj = ix4[c * 8 + e4];
+                            const int js[4] = {jj.x, jj.y, jj.z, jj.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            if (js[e] < 0 || js[e] > i) v[c][e4 * 4 + e] = __float_as_uint(-INFINITY);
-                    }
+                            for (int e = 0; e < 4; ++e)
+                                if ((unsigned)js[e] > (unsigned)i)
+                                    v[c][e4 * 4 + e] = __float_as_uint(-INFINITY);
+                        }
+                }
             }
             float tm[2] = {-INFINITY, -INFINITY};
 #pragma unroll

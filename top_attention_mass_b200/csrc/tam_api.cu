@@ -871,6 +871,7 @@ int tam_distill_kl(int64_t N, int Hq, int Hkv, int d, int dtype, const void* q, 
     ia.budget = 1; ia.rows = score_rows; ia.status = (int32_t*)ws;
     const int64_t cap = std::min<int64_t>((int64_t)(half / sizeof(float)),
                                           (int64_t(1) << 32) - 1);       // 32-bit row offsets
+    ma.out_cap = ia.out_cap = debug_extent((uint64_t)cap);
     for (int64_t r0 = 0; r0 < N;) {
         const int64_t r1 = chunk_end(r0, N, cap);
         ma.row0 = ia.row0 = r0;
