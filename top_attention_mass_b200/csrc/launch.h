@@ -62,11 +62,10 @@ cudaError_t with_table(int64_t N, const SeqTable* seqs, F&& fn) {
     return fn(t);
 }
 
-#ifdef __CUDACC__
-// (sequence, local tile) of the b-th tile of the table in the order above; any thread
-// may call it.
-template <int BQ>
-__device__ __forceinline__ void seq_tile(const SeqTable& t, int b, int& s_out, int& L_out) {
+// (sequence, local tile) of the b-th tile of the table in the order above, for tiles of
+// BQ rows; any thread may call it (and the host, to check the order).
+__host__ __device__ inline void seq_tile_of(const SeqTable& t, int BQ, int b, int& s_out,
+                                            int& L_out) {
     int lo = 0, hi = t.n_seq - 1;                  // the last r with tile0[r] <= b
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -76,6 +75,12 @@ __device__ __forceinline__ void seq_tile(const SeqTable& t, int b, int& s_out, i
     const int s = t.order[lo];
     s_out = s;
     L_out = (t.cu[s + 1] - t.cu[s] + BQ - 1) / BQ - 1 - (b - t.tile0[lo]);
+}
+
+#ifdef __CUDACC__
+template <int BQ>
+__device__ __forceinline__ void seq_tile(const SeqTable& t, int b, int& s_out, int& L_out) {
+    seq_tile_of(t, BQ, b, s_out, L_out);
 }
 #endif
 
